@@ -1,0 +1,33 @@
+"""Build the CPU oracle (test infrastructure only).
+
+Compiles hgd_oracle.c twice with gcc: libhgd_oracle.so (double arithmetic) and
+libhgd_oracle_f32.so (float arithmetic).  -O2 -ffp-contract=off and no
+fast-math keep every sum in the order the source writes it.
+"""
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "hgd_oracle.c")
+TARGETS = {
+    "libhgd_oracle.so": [],
+    "libhgd_oracle_f32.so": ["-DHGDO_FP32", "-DHGDO_REAL=float"],
+}
+
+
+def build(force: bool = False) -> None:
+    for name, defs in TARGETS.items():
+        out = os.path.join(HERE, name)
+        deps = [SRC, os.path.join(HERE, "hgd_oracle.h"), __file__]
+        if not force and os.path.exists(out) and all(
+                os.path.getmtime(out) >= os.path.getmtime(d) for d in deps):
+            continue
+        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+               "-shared", "-Wall", "-Wextra", "-Wno-unused-parameter", *defs, SRC,
+               "-o", out + ".tmp", "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(out + ".tmp", out)
+
+
+if __name__ == "__main__":
+    build(force=True)
