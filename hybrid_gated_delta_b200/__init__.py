@@ -1,0 +1,329 @@
+"""Python binding of libhgd, the sm_100a hybrid gated-delta decode library.
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of libhgd.so; PyTorch supplies device memory and streams.  The entry
+points have the names of the C ABI in include/hgd.h.  If the library is not
+built, importing this package raises instead of falling back to anything.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhgd.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libhgd.so is not built ({LIB_PATH}); run "
+                      "`python -c 'import __graft_entry__ as g; g.build()'`")
+
+_lib = C.CDLL(LIB_PATH)
+
+HGD_OK = 0
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned",
+          4: "CUDA error", 5: "timeout", 6: "not co-resident", 7: "NaN logit",
+          8: "unsupported device", 9: "buffer too small"}
+
+MAX_LAYERS = 64
+W_IN_NORM, W_IN, W_CONV, W_A_LOG, W_DT_BIAS, W_GNORM, W_OUT, W_POST_NORM, W_GATE, W_UP, W_DOWN = range(11)
+W_LAYER_COUNT = 11
+W_EMBED, W_FINAL_NORM = 100, 101
+LAYER_TENSORS = {"in_norm": W_IN_NORM, "w_in": W_IN, "conv_w": W_CONV, "A_log": W_A_LOG,
+                 "dt_bias": W_DT_BIAS, "gnorm_w": W_GNORM, "w_out": W_OUT, "post_norm": W_POST_NORM,
+                 "w_gate": W_GATE, "w_up": W_UP, "w_down": W_DOWN}
+S_GDN, S_CONV, S_KV, S_POS = range(4)
+
+
+class HgdError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({STATUS.get(code, 'unknown')})")
+        self.code = code
+
+
+class Config(C.Structure):
+    _fields_ = [("n_layers", C.c_int32), ("hidden", C.c_int32), ("vocab", C.c_int32),
+                ("gdn_heads", C.c_int32), ("gdn_dk", C.c_int32), ("gdn_dv", C.c_int32),
+                ("conv_k", C.c_int32), ("attn_q_heads", C.c_int32), ("attn_kv_heads", C.c_int32),
+                ("attn_head_dim", C.c_int32), ("mlp_inter", C.c_int32), ("attn_every", C.c_int32),
+                ("norm_eps", C.c_float), ("rope_base", C.c_float)]
+
+
+class _Model(C.Structure):
+    _fields_ = [("cfg", Config), ("embed", C.c_void_p), ("final_norm", C.c_void_p),
+                ("w", (C.c_void_p * W_LAYER_COUNT) * MAX_LAYERS), ("arena_bytes", C.c_size_t)]
+
+
+class _State(C.Structure):
+    _fields_ = [("B", C.c_int32), ("Tmax", C.c_int32), ("Lmax", C.c_int32),
+                ("arena", C.c_void_p), ("arena_bytes", C.c_size_t), ("off", C.c_size_t * 32)]
+
+
+_p, _i, _i64, _sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
+_SIGS = {
+    "hgd_status_string": ([_i], C.c_char_p),
+    "hgd_version": ([], _i),
+    "hgd_gemv_bf16": ([_p, _p, _p, _i, _i, _i, _i, _p], _i),
+    "hgd_gemv_swiglu_bf16": ([_p, _p, _p, _p, _i, _i, _i, _p], _i),
+    "hgd_conv1d_tail_update": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
+    "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
+    "hgd_model_arena_bytes": ([C.POINTER(Config), C.POINTER(_sz)], _i),
+    "hgd_model_tensor": ([C.POINTER(Config), _i, _i, C.POINTER(_sz), C.POINTER(_sz)], _i),
+    "hgd_model_init": ([C.POINTER(_Model), C.POINTER(Config), _p, _sz], _i),
+    "hgd_state_arena_bytes": ([C.POINTER(Config), _i, _i, _i, C.POINTER(_sz)], _i),
+    "hgd_state_tensor": ([C.POINTER(Config), _i, _i, _i, _i, C.POINTER(_sz), C.POINTER(_sz)], _i),
+    "hgd_state_init": ([C.POINTER(_State), C.POINTER(_Model), _i, _i, _i, _p, _sz], _i),
+    "hgd_decode_layer_stack": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _p, _p, _p, _p, _p], _i),
+    "hgd_decode_layer_stack_launches": ([C.POINTER(_Model), _i, _i], _i),
+}
+for _name, (_args, _ret) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _ret
+
+EXPORTED = tuple(_SIGS)
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != HGD_OK:
+        raise HgdError(fn, rc)
+
+
+def version() -> int:
+    return _lib.hgd_version()
+
+
+def status_string(code: int) -> str:
+    return _lib.hgd_status_string(code).decode()
+
+
+# --------------------------------------------------------------- helpers ----
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libhgd must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need(t, dtype, name):
+    torch = _torch()
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+
+
+# -------------------------------------------------------------- entry points
+
+def gemv_bf16(W, x, y=None, y_is_fp32=True, stream=None):
+    """y[M,N] = x[M,K] . W[N,K]^T (bf16 in, fp32 accumulate)."""
+    torch = _torch()
+    _need(W, torch.bfloat16, "W")
+    _need(x, torch.bfloat16, "x")
+    N, K = W.shape
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32 if y_is_fp32 else torch.bfloat16, device=x.device)
+    _check("hgd_gemv_bf16", _lib.hgd_gemv_bf16(_ptr(W), _ptr(x), _ptr(y), int(y.dtype == torch.float32),
+                                                M, N, K, _stream(stream)))
+    return y
+
+
+def gemv_swiglu_bf16(W_gate, W_up, x, h=None, stream=None):
+    """h[M,I] = bf16(silu(x W_gate^T) * (x W_up^T))."""
+    torch = _torch()
+    for t, n in ((W_gate, "W_gate"), (W_up, "W_up"), (x, "x")):
+        _need(t, torch.bfloat16, n)
+    I, K = W_gate.shape
+    M = x.shape[0]
+    if h is None:
+        h = torch.empty((M, I), dtype=torch.bfloat16, device=x.device)
+    _check("hgd_gemv_swiglu_bf16", _lib.hgd_gemv_swiglu_bf16(_ptr(W_gate), _ptr(W_up), _ptr(x), _ptr(h),
+                                                              M, I, K, _stream(stream)))
+    return h
+
+
+def conv1d_tail_update(x, tail, w, y=None, tail_rec=None, apply_silu=True, stream=None):
+    """x [B,T,C] fp32, tail [B,kc-1,C] fp32 (in place), w [C,kc] bf16."""
+    torch = _torch()
+    _need(x, torch.float32, "x")
+    _need(tail, torch.float32, "tail")
+    _need(w, torch.bfloat16, "w")
+    B, T, Cc = x.shape
+    kc = w.shape[1]
+    if y is None:
+        y = torch.empty_like(x)
+    _check("hgd_conv1d_tail_update", _lib.hgd_conv1d_tail_update(
+        _ptr(x), _ptr(tail), _ptr(w), _ptr(y), _ptr(tail_rec), B, T, Cc, kc, int(apply_silu),
+        _stream(stream)))
+    return y
+
+
+def gdn_decode_step(q, k, v, g, b, S, o=None, o_bf16=None, S_rec=None, l2norm_qk=True,
+                    row_stride=None, B=None, T=None, stream=None):
+    """Gated delta rule rows.  q,k [B,T,H,dk], v [B,T,H,dv] fp32 (or views into one
+    packed [B*T, row_stride] buffer with row_stride given), g,b [B,T,H] fp32,
+    S [B,H,dv,dk] fp32 in place.  Returns o [B,T,H,dv] fp32."""
+    torch = _torch()
+    _need(S, torch.float32, "S")
+    Bs, H, dv, dk = S.shape
+    Tn = g.shape[1] if T is None else T
+    Bn = Bs if B is None else B
+    if row_stride is None:
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _need(t, torch.float32, n)
+            if not t.is_contiguous():
+                raise ValueError(f"{n} must be contiguous")
+        row_stride = H * dk
+        qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    else:
+        qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    if o is None:
+        o = torch.empty((Bn, Tn, H, dv), dtype=torch.float32, device=S.device)
+    _check("hgd_gdn_decode_step", _lib.hgd_gdn_decode_step(
+        qp, kp, vp, int(row_stride), _ptr(g), _ptr(b), _ptr(S), _ptr(o), _ptr(o_bf16), _ptr(S_rec),
+        Bn, Tn, H, dk, dv, int(l2norm_qk), _stream(stream)))
+    return o
+
+
+# ------------------------------------------------------------------ stack
+
+def make_config(cfg: dict) -> Config:
+    c = Config()
+    for name, _ in Config._fields_:
+        setattr(c, name, cfg[name])
+    return c
+
+
+class Model:
+    """Weights in one device arena laid out by libhgd (hgd_model_tensor offsets)."""
+
+    def __init__(self, cfg: dict, weights: dict, device="cuda"):
+        torch = _torch()
+        self.cfg_dict = dict(cfg)
+        self.cfg = make_config(cfg)
+        nbytes = C.c_size_t()
+        _check("hgd_model_arena_bytes", _lib.hgd_model_arena_bytes(C.byref(self.cfg), C.byref(nbytes)))
+        self.arena = torch.zeros(nbytes.value // 2 + 128, dtype=torch.int16, device=device)
+        base = self.arena.data_ptr()
+        pad = (-base) % 256
+        self.arena_u8 = self.arena.view(torch.uint8)[pad:pad + nbytes.value]
+        for name, tid, layer in self._tensors(weights):
+            off, n = self.tensor_offset(layer, tid)
+            arr = weights[name] if layer < 0 else weights["layers"][layer][name]
+            arr = np.ascontiguousarray(arr, dtype=np.uint16).reshape(-1)
+            if arr.size != n:
+                raise ValueError(f"layer {layer} {name}: {arr.size} elements, layout expects {n}")
+            src = torch.from_numpy(arr.view(np.int16))
+            self.arena_u8[off:off + 2 * n].view(torch.int16).copy_(src, non_blocking=False)
+        self.m = _Model()
+        _check("hgd_model_init", _lib.hgd_model_init(C.byref(self.m), C.byref(self.cfg),
+                                                     self.arena_u8.data_ptr(), nbytes.value))
+
+    def _tensors(self, weights):
+        yield "embed", W_EMBED, -1
+        yield "final_norm", W_FINAL_NORM, -1
+        for l, lw in enumerate(weights["layers"]):
+            for name in lw:
+                yield name, LAYER_TENSORS[name], l
+
+    def tensor_offset(self, layer: int, tid: int):
+        off, n = C.c_size_t(), C.c_size_t()
+        _check("hgd_model_tensor", _lib.hgd_model_tensor(C.byref(self.cfg), layer, tid, C.byref(off),
+                                                         C.byref(n)))
+        return off.value, n.value
+
+    def launches(self, B: int, T: int) -> int:
+        return _lib.hgd_decode_layer_stack_launches(C.byref(self.m), B, T)
+
+
+class State:
+    """Per-stream decode state (GDN S, conv tails, KV cache, positions) plus the
+    call scratch, in one device arena laid out by libhgd."""
+
+    def __init__(self, model: Model, B: int, Tmax: int, Lmax: int, init: dict | None = None,
+                 device="cuda"):
+        torch = _torch()
+        self.model, self.B, self.Tmax, self.Lmax = model, B, Tmax, Lmax
+        nbytes = C.c_size_t()
+        _check("hgd_state_arena_bytes", _lib.hgd_state_arena_bytes(C.byref(model.cfg), B, Tmax, Lmax,
+                                                                   C.byref(nbytes)))
+        self.arena = torch.zeros(nbytes.value // 4 + 64, dtype=torch.int32, device=device)
+        pad = (-self.arena.data_ptr()) % 256
+        self.arena_u8 = self.arena.view(torch.uint8)[pad:pad + nbytes.value]
+        self.st = _State()
+        _check("hgd_state_init", _lib.hgd_state_init(C.byref(self.st), C.byref(model.m), B, Tmax, Lmax,
+                                                     self.arena_u8.data_ptr(), nbytes.value))
+        cfg = model.cfg_dict
+        H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+        nkv, hd = cfg["attn_kv_heads"], cfg["attn_head_dim"]
+        n_attn = sum(1 for l in range(cfg["n_layers"]) if l % cfg["attn_every"] == cfg["attn_every"] - 1)
+        n_gdn = cfg["n_layers"] - n_attn
+        Cc = 2 * H * dk + H * dv
+        self.S = self._view(S_GDN, torch.float32, (n_gdn, B, H, dv, dk))
+        self.conv = self._view(S_CONV, torch.float32, (n_gdn, B, kc - 1, Cc))
+        self.kv = self._view(S_KV, torch.bfloat16, (n_attn, 2, B, nkv, Lmax, hd))
+        self.pos = self._view(S_POS, torch.int32, (B,))
+        if init is not None:
+            self.load(init)
+
+    def _view(self, tid, dtype, shape):
+        torch = _torch()
+        off, n = C.c_size_t(), C.c_size_t()
+        _check("hgd_state_tensor", _lib.hgd_state_tensor(C.byref(self.model.cfg), self.B, self.Tmax,
+                                                         self.Lmax, tid, C.byref(off), C.byref(n)))
+        es = torch.empty((), dtype=dtype).element_size()
+        assert int(np.prod(shape)) == n.value
+        return self.arena_u8[off.value:off.value + n.value * es].view(dtype).view(shape)
+
+    def load(self, init: dict) -> None:
+        """Copy host arrays (from hgd_synth.stack_state) into the state tensors."""
+        torch = _torch()
+        self.S.copy_(torch.from_numpy(np.ascontiguousarray(init["S"], np.float32)))
+        self.conv.copy_(torch.from_numpy(np.ascontiguousarray(init["tail"], np.float32)))
+        kv = np.ascontiguousarray(init["kv"], np.uint16)
+        if kv.shape[-2] != self.Lmax:
+            full = np.zeros(kv.shape[:-2] + (self.Lmax, kv.shape[-1]), np.uint16)
+            n = min(self.Lmax, kv.shape[-2])
+            full[..., :n, :] = kv[..., :n, :]
+            kv = full
+        self.kv.view(torch.int16).copy_(torch.from_numpy(kv.view(np.int16)))
+        self.pos.copy_(torch.from_numpy(np.ascontiguousarray(init["pos"], np.int32)))
+
+    def snapshot(self) -> dict:
+        return {"S": self.S.clone(), "conv": self.conv.clone(), "kv": self.kv.clone(), "pos": self.pos.clone()}
+
+    def restore(self, snap: dict) -> None:
+        self.S.copy_(snap["S"]); self.conv.copy_(snap["conv"]); self.kv.copy_(snap["kv"])
+        self.pos.copy_(snap["pos"])
+
+
+def decode_layer_stack(model: Model, state: State, tokens, T: int, logits=None, argmax=None, S_rec=None,
+                       tail_rec=None, status=None, stream=None):
+    """One decode call over T rows of each stream.  tokens [B,T] int32 (device).
+    Returns argmax [B*T] int32 (device)."""
+    torch = _torch()
+    _need(tokens, torch.int32, "tokens")
+    if argmax is None:
+        argmax = torch.empty((state.B * T,), dtype=torch.int32, device=tokens.device)
+    _check("hgd_decode_layer_stack", _lib.hgd_decode_layer_stack(
+        C.byref(model.m), C.byref(state.st), _ptr(tokens), T, _ptr(logits), _ptr(argmax), _ptr(S_rec),
+        _ptr(tail_rec), _ptr(status), _stream(stream)))
+    return argmax

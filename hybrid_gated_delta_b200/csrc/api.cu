@@ -1,0 +1,619 @@
+// api.cu -- extern "C" entry points of libhgd (declared in include/hgd.h):
+// argument validation, launch planning and the per-layer launch sequence of the
+// decode stack.  The library allocates no device memory; every buffer is the
+// caller's.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <utility>
+#include <cstdio>
+#include <cstring>
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "gdn.cuh"
+#include "gemv.cuh"
+
+using namespace hgd;
+
+namespace {
+
+// ------------------------------------------------------------ device info
+struct DevInfo {
+    int ok;    // 1 = sm_100, 0 = unsupported, -1 = cuda error
+    int sms;
+};
+
+int device_info(DevInfo* di) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HGD_ERR_CUDA; }
+    static DevInfo cache[64];
+    static int have[64];
+    if (dev >= 0 && dev < 64 && have[dev]) { *di = cache[dev]; return di->ok == 1 ? HGD_OK : HGD_ERR_UNSUPPORTED_DEVICE; }
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
+    }
+    DevInfo d{major == 10 ? 1 : 0, sms};
+    if (dev >= 0 && dev < 64) { cache[dev] = d; have[dev] = 1; }
+    *di = d;
+    return d.ok == 1 ? HGD_OK : HGD_ERR_UNSUPPORTED_DEVICE;
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status(cudaError_t e) {
+    if (e == cudaSuccess) return HGD_OK;
+    cudaGetLastError();
+    return HGD_ERR_CUDA;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// ------------------------------------------------------------- GEMV plans
+struct GemvPlan {
+    int nt, mchunk, nstage, stage_bytes, x_bytes, kb, nkb;
+    size_t smem;
+};
+
+size_t gv_fixed_bytes(int mp) {
+    return (size_t)(GV_WARPS + 1) * mp * GV_PITCH * 4 + 8 + 2 * 8 * GV_MAX_STAGES + 16;
+}
+
+bool plan_gemv(int M, int K, GemvPlan* pl) {
+    gv_kblocks(K, &pl->kb, &pl->nkb);
+    pl->stage_bytes = GV_ROWS * (pl->kb + GV_PAD) * 2;
+    const int want = (M + 7) / 8;
+    int nt = want <= 1 ? 1 : (want <= 2 ? 2 : 4);
+    for (; nt >= 1; nt >>= 1) {
+        const int mp = 8 * nt;
+        const int xb = gv_align16(mp * (K + GV_PAD) * 2);
+        const long avail = (long)GV_SMEM_LIMIT - xb - (long)gv_fixed_bytes(mp);
+        const long ns = avail / pl->stage_bytes;
+        if (ns >= 2) {
+            pl->nt = nt;
+            pl->mchunk = mp;
+            pl->nstage = (int)std::min<long>(ns, GV_MAX_STAGES);
+            pl->x_bytes = xb;
+            pl->smem = (size_t)pl->nstage * pl->stage_bytes + xb + gv_fixed_bytes(mp);
+            return true;
+        }
+    }
+    return false;
+}
+
+template <int NT, int PRO, int EPI>
+cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cudaStream_t s) {
+    auto kern = k_gemv<NT, PRO, EPI>;
+    static int attr_done[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    }
+    return launch_pdl(kern, dim3(grid), dim3(GV_THREADS), smem, s, p);
+}
+
+template <int PRO, int EPI>
+cudaError_t launch_gemv_nt(int nt, const GemvParams& p, int grid, size_t smem, cudaStream_t s) {
+    switch (nt) {
+        case 1: return launch_gemv_t<1, PRO, EPI>(p, grid, smem, s);
+        case 2: return launch_gemv_t<2, PRO, EPI>(p, grid, smem, s);
+        default: return launch_gemv_t<4, PRO, EPI>(p, grid, smem, s);
+    }
+}
+
+// Launch a GEMV over all M rows, in chunks of the plan's M tile.  `adv` moves
+// the row-indexed pointers of the params to a chunk's first row.
+template <int PRO, int EPI>
+int run_gemv(GemvParams p, int M, int sms, cudaStream_t s, int* launches) {
+    GemvPlan pl;
+    if (!plan_gemv(M, p.K, &pl)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    p.kb = pl.kb;
+    p.nkb = pl.nkb;
+    p.nstage = pl.nstage;
+    p.stage_bytes = pl.stage_bytes;
+    p.x_bytes = pl.x_bytes;
+    p.n_rowblk = (EPI == EPI_SWIGLU) ? (p.N + 7) / 8 : (p.N + GV_ROWS - 1) / GV_ROWS;
+    const int grid = std::min(p.n_rowblk, sms);
+    for (int m0 = 0; m0 < M; m0 += pl.mchunk) {
+        GemvParams q = p;
+        q.M = std::min(pl.mchunk, M - m0);
+        if (q.x) q.x += m0 * q.x_ld;
+        if (q.tokens) q.tokens += m0;
+        if (q.resid_out) q.resid_out += m0 * q.resid_out_ld;
+        if (q.o) q.o += m0 * q.o_ld;
+        if (q.z) q.z += m0 * q.z_ld;
+        if (q.resid) q.resid += m0 * q.resid_ld;
+        if (q.y) {
+            const int es = (EPI == EPI_F32) ? 4 : 2;
+            q.y = reinterpret_cast<uint8_t*>(q.y) + (size_t)m0 * q.y_ld * es;
+        }
+        if (q.logits) q.logits += m0 * q.logits_ld;
+        if (q.best_v) { q.best_v += (size_t)m0 * grid; q.best_i += (size_t)m0 * grid; }
+        cudaError_t e = launch_gemv_nt<PRO, EPI>(pl.nt, q, grid, pl.smem, s);
+        if (e != cudaSuccess) return launch_status(e);
+        if (launches) ++*launches;
+    }
+    return HGD_OK;
+}
+
+int gemv_grid(int N, int rows_per_blk, int sms) { return std::min((N + rows_per_blk - 1) / rows_per_blk, sms); }
+
+int gemv_chunks(int M, int K) {
+    GemvPlan pl;
+    if (!plan_gemv(M, K, &pl)) return -1;
+    return (M + pl.mchunk - 1) / pl.mchunk;
+}
+
+// ------------------------------------------------------------ stack layout
+struct Dims {
+    int L, D, V, H, dk, dv, kc, nq, nkv, hd, I, every;
+    int n_gdn, n_attn;
+    int64_t C, gdn_out, attn_out;
+};
+
+bool is_attn_layer(const hgd_config* c, int l) { return (l % c->attn_every) == c->attn_every - 1; }
+
+int dims_of(const hgd_config* c, Dims* d) {
+    if (!c) return HGD_ERR_INVALID_ARG;
+    if (c->n_layers < 1 || c->n_layers > HGD_MAX_LAYERS || c->attn_every < 1) return HGD_ERR_INVALID_ARG;
+    if (c->hidden < 32 || c->vocab < 1 || c->gdn_heads < 1 || c->mlp_inter < 1 || c->attn_q_heads < 1 ||
+        c->attn_kv_heads < 1)
+        return HGD_ERR_INVALID_ARG;
+    d->L = c->n_layers; d->D = c->hidden; d->V = c->vocab; d->H = c->gdn_heads;
+    d->dk = c->gdn_dk; d->dv = c->gdn_dv; d->kc = c->conv_k; d->nq = c->attn_q_heads;
+    d->nkv = c->attn_kv_heads; d->hd = c->attn_head_dim; d->I = c->mlp_inter; d->every = c->attn_every;
+    d->n_gdn = d->n_attn = 0;
+    for (int l = 0; l < d->L; ++l) (is_attn_layer(c, l) ? d->n_attn : d->n_gdn)++;
+    d->C = 2 * (int64_t)d->H * d->dk + (int64_t)d->H * d->dv;
+    d->gdn_out = d->C + (int64_t)d->H * d->dv + 2 * d->H;
+    d->attn_out = 2 * (int64_t)d->nq * d->hd + 2 * (int64_t)d->nkv * d->hd;
+    return HGD_OK;
+}
+
+int check_supported(const Dims& d) {
+    const bool ok =
+        d.D % 32 == 0 && d.D <= 65536 && (d.H * d.dv) % 32 == 0 && (d.nq * d.hd) % 32 == 0 &&
+        d.I % 32 == 0 && (d.dk == 32 || d.dk == 64 || d.dk == 128 || d.dk == 256) && d.dv % 16 == 0 &&
+        d.dv <= 1024 && d.kc == 4 && d.hd % 32 == 0 && d.hd <= ATTN_MAX_HD && d.nq % d.nkv == 0 &&
+        d.nq / d.nkv <= ATTN_MAX_GROUP;
+    return ok ? HGD_OK : HGD_ERR_UNSUPPORTED_SHAPE;
+}
+
+size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// numel of one weight tensor (0 if absent)
+size_t weight_numel(const Dims& d, const hgd_config* c, int layer, int t) {
+    if (layer < 0) {
+        if (t == HGD_W_EMBED) return (size_t)d.V * d.D;
+        if (t == HGD_W_FINAL_NORM) return (size_t)d.D;
+        return 0;
+    }
+    const bool att = is_attn_layer(c, layer);
+    switch (t) {
+        case HGD_W_IN_NORM: case HGD_W_POST_NORM: return (size_t)d.D;
+        case HGD_W_IN: return (size_t)(att ? d.attn_out : d.gdn_out) * d.D;
+        case HGD_W_CONV: return att ? 0 : (size_t)d.C * d.kc;
+        case HGD_W_A_LOG: case HGD_W_DT_BIAS: return att ? 0 : (size_t)d.H;
+        case HGD_W_GNORM: return att ? 0 : (size_t)d.dv;
+        case HGD_W_OUT: return (size_t)d.D * (att ? (size_t)d.nq * d.hd : (size_t)d.H * d.dv);
+        case HGD_W_GATE: case HGD_W_UP: return (size_t)d.I * d.D;
+        case HGD_W_DOWN: return (size_t)d.D * d.I;
+        default: return 0;
+    }
+}
+
+// Walk the arena in order; returns the total and, if (layer, t) matches, its offset.
+size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_t, size_t* off) {
+    size_t pos = 0;
+    const int glob[2] = {HGD_W_EMBED, HGD_W_FINAL_NORM};
+    for (int g = 0; g < 2; ++g) {
+        if (want_layer == -1 && want_t == glob[g] && off) *off = pos;
+        pos += al256(weight_numel(d, c, -1, glob[g]) * 2);
+    }
+    for (int l = 0; l < d.L; ++l)
+        for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) {
+            const size_t n = weight_numel(d, c, l, t);
+            if (l == want_layer && t == want_t && off) *off = pos;
+            pos += al256(n * 2);
+        }
+    return pos;
+}
+
+enum ScratchIdx {
+    SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
+    SC_BESTV, SC_BESTI, SC_END, SC_COUNT
+};
+constexpr int kBestG = 1024;  // max CTAs of the LM-head launch
+
+int max_chunks_of(int Lmax) { return (Lmax + ATTN_CHUNK - 1) / ATTN_CHUNK; }
+
+void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
+    const int64_t M = (int64_t)B * Tmax;
+    size_t sz[SC_COUNT] = {};
+    sz[SC_S] = (size_t)d.n_gdn * B * d.H * d.dv * d.dk * 4;
+    sz[SC_CONV] = (size_t)d.n_gdn * B * (d.kc - 1) * d.C * 4;
+    sz[SC_KV] = (size_t)d.n_attn * 2 * B * d.nkv * (size_t)Lmax * d.hd * 2;
+    sz[SC_POS] = (size_t)B * 4;
+    sz[SC_RESID] = (size_t)M * d.D * 2;
+    sz[SC_PROJ] = (size_t)M * std::max(d.gdn_out, d.attn_out) * 4;
+    sz[SC_O] = (size_t)M * d.H * d.dv * 4;
+    sz[SC_QROT] = (size_t)M * d.nq * d.hd * 4;
+    sz[SC_ATTN] = (size_t)M * d.nq * d.hd * 2;
+    sz[SC_PART] = (size_t)M * d.nq * max_chunks_of(Lmax) * (d.hd + 2) * 4;
+    sz[SC_MLP] = (size_t)M * d.I * 2;
+    sz[SC_BESTV] = (size_t)M * kBestG * 4;
+    sz[SC_BESTI] = (size_t)M * kBestG * 4;
+    size_t pos = 0;
+    for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
+    off[SC_END] = pos;
+}
+
+int check_state_dims(int B, int Tmax, int Lmax) {
+    if (B < 1 || Tmax < 1 || Lmax < 1) return HGD_ERR_INVALID_ARG;
+    if ((int64_t)B * Tmax > 256 || Lmax > 16384) return HGD_ERR_UNSUPPORTED_SHAPE;
+    return HGD_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* hgd_status_string(int s) {
+    switch (s) {
+        case HGD_OK: return "ok";
+        case HGD_ERR_INVALID_ARG: return "invalid argument";
+        case HGD_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case HGD_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case HGD_ERR_CUDA: return "CUDA runtime error";
+        case HGD_ERR_TIMEOUT: return "in-kernel wait timed out";
+        case HGD_ERR_NOT_CORESIDENT: return "persistent launch cannot be co-resident";
+        case HGD_ERR_NAN: return "NaN logit";
+        case HGD_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+        case HGD_ERR_BUFFER_TOO_SMALL: return "arena smaller than required";
+        default: return "unknown status";
+    }
+}
+
+int hgd_version(void) { return 100; }
+
+int hgd_gemv_bf16(const uint16_t* W, const uint16_t* x, void* y, int y_is_fp32, int M, int N, int K,
+                  hgd_stream_t stream) {
+    if (!W || !x || !y || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (K % 32 != 0 || K > 65536) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(W) || !al16(x) || !al16(y)) return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    GemvParams p = {};
+    p.W = W; p.N = N; p.K = K; p.x = x; p.x_ld = K; p.y = y; p.y_ld = N;
+    if (y_is_fp32) return run_gemv<PRO_COPY, EPI_F32>(p, M, di.sms, (cudaStream_t)stream, nullptr);
+    return run_gemv<PRO_COPY, EPI_BF16>(p, M, di.sms, (cudaStream_t)stream, nullptr);
+}
+
+int hgd_gemv_swiglu_bf16(const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* x, uint16_t* h,
+                         int M, int I, int K, hgd_stream_t stream) {
+    if (!W_gate || !W_up || !x || !h || M < 1 || I < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (K % 32 != 0 || K > 65536) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(W_gate) || !al16(W_up) || !al16(x) || !al16(h)) return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    GemvParams p = {};
+    p.W = W_gate; p.W2 = W_up; p.N = I; p.K = K; p.x = x; p.x_ld = K; p.y = h; p.y_ld = I;
+    return run_gemv<PRO_COPY, EPI_SWIGLU>(p, M, di.sms, (cudaStream_t)stream, nullptr);
+}
+
+int hgd_conv1d_tail_update(const float* x, float* tail, const uint16_t* w, float* y, float* tail_rec,
+                           int B, int T, int C, int kc, int apply_silu, hgd_stream_t stream) {
+    if (!x || !tail || !w || !y || B < 1 || T < 1 || C < 1) return HGD_ERR_INVALID_ARG;
+    if (kc < 2 || kc > 8) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(x) || !al16(tail) || !al16(w) || !al16(y) || (tail_rec && !al16(tail_rec)))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    ConvParams p{x, tail, w, y, tail_rec, B, T, C, kc, apply_silu ? 1 : 0};
+    const int64_t n = (int64_t)B * C;
+    const int blocks = (int)((n + 255) / 256);
+    return launch_status(launch_pdl(k_conv_tail, dim3(blocks), dim3(256), 0, (cudaStream_t)stream, p));
+}
+
+int hgd_gdn_decode_step(const float* q, const float* k, const float* v, int64_t row_stride, const float* g,
+                        const float* b, float* S, float* o, uint16_t* o_bf16, float* S_rec, int B, int T,
+                        int H, int dk, int dv, int l2norm_qk, hgd_stream_t stream) {
+    if (!q || !k || !v || !g || !b || !S || !o || B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1)
+        return HGD_ERR_INVALID_ARG;
+    if (!(dk == 32 || dk == 64 || dk == 128 || dk == 256) || dv % GDN_ROWS != 0 || dv > 1024)
+        return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (row_stride < (int64_t)H * dk || row_stride < (int64_t)H * dv) return HGD_ERR_INVALID_ARG;
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(g) || !al16(b) || !al16(S) || !al16(o) ||
+        (o_bf16 && !al16(o_bf16)) || (S_rec && !al16(S_rec)))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    GdnParams p{q, k, v, row_stride, g, b, S, o, o_bf16, S_rec, B, T, H, dk, dv, l2norm_qk ? 1 : 0};
+    const dim3 grid(B * H, dv / GDN_ROWS), block(GDN_WARPS * 32);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    switch (dk) {
+        case 32: e = launch_pdl(k_gdn_step<1>, grid, block, 0, s, p); break;
+        case 64: e = launch_pdl(k_gdn_step<2>, grid, block, 0, s, p); break;
+        case 128: e = launch_pdl(k_gdn_step<4>, grid, block, 0, s, p); break;
+        default: e = launch_pdl(k_gdn_step<8>, grid, block, 0, s, p); break;
+    }
+    return launch_status(e);
+}
+
+// ---------------------------------------------------------------- stack
+
+int hgd_model_arena_bytes(const hgd_config* cfg, size_t* bytes) {
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if (!bytes) return HGD_ERR_INVALID_ARG;
+    *bytes = weight_walk(d, cfg, -2, -2, nullptr);
+    return HGD_OK;
+}
+
+int hgd_model_tensor(const hgd_config* cfg, int layer, int tensor, size_t* offset, size_t* numel) {
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if (!offset || !numel) return HGD_ERR_INVALID_ARG;
+    if (layer < -1 || layer >= d.L) return HGD_ERR_INVALID_ARG;
+    if (layer == -1 && tensor != HGD_W_EMBED && tensor != HGD_W_FINAL_NORM) return HGD_ERR_INVALID_ARG;
+    if (layer >= 0 && (tensor < 0 || tensor >= HGD_W_LAYER_COUNT)) return HGD_ERR_INVALID_ARG;
+    size_t off = 0;
+    weight_walk(d, cfg, layer, tensor, &off);
+    *offset = off;
+    *numel = weight_numel(d, cfg, layer, tensor);
+    return HGD_OK;
+}
+
+int hgd_model_init(hgd_model* m, const hgd_config* cfg, const void* arena, size_t bytes) {
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if (!m || !arena) return HGD_ERR_INVALID_ARG;
+    if (!al16(arena) || (reinterpret_cast<uintptr_t>(arena) & 255u)) return HGD_ERR_MISALIGNED;
+    const size_t need = weight_walk(d, cfg, -2, -2, nullptr);
+    if (bytes < need) return HGD_ERR_BUFFER_TOO_SMALL;
+    std::memset(m, 0, sizeof(*m));
+    m->cfg = *cfg;
+    const uint8_t* base = static_cast<const uint8_t*>(arena);
+    size_t off = 0;
+    weight_walk(d, cfg, -1, HGD_W_EMBED, &off);
+    m->embed = reinterpret_cast<const uint16_t*>(base + off);
+    weight_walk(d, cfg, -1, HGD_W_FINAL_NORM, &off);
+    m->final_norm = reinterpret_cast<const uint16_t*>(base + off);
+    for (int l = 0; l < d.L; ++l)
+        for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) {
+            if (!weight_numel(d, cfg, l, t)) continue;
+            weight_walk(d, cfg, l, t, &off);
+            m->w[l][t] = reinterpret_cast<const uint16_t*>(base + off);
+        }
+    m->arena_bytes = need;
+    return HGD_OK;
+}
+
+int hgd_state_arena_bytes(const hgd_config* cfg, int B, int Tmax, int Lmax, size_t* bytes) {
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_state_dims(B, Tmax, Lmax))) return rc;
+    if (!bytes) return HGD_ERR_INVALID_ARG;
+    size_t off[SC_COUNT];
+    state_layout(d, B, Tmax, Lmax, off);
+    *bytes = off[SC_END];
+    return HGD_OK;
+}
+
+int hgd_state_tensor(const hgd_config* cfg, int B, int Tmax, int Lmax, int tensor, size_t* offset,
+                     size_t* numel) {
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_state_dims(B, Tmax, Lmax))) return rc;
+    if (!offset || !numel || tensor < 0 || tensor >= HGD_S_COUNT) return HGD_ERR_INVALID_ARG;
+    size_t off[SC_COUNT];
+    state_layout(d, B, Tmax, Lmax, off);
+    *offset = off[tensor];
+    switch (tensor) {
+        case HGD_S_GDN: *numel = (size_t)d.n_gdn * B * d.H * d.dv * d.dk; break;
+        case HGD_S_CONV: *numel = (size_t)d.n_gdn * B * (d.kc - 1) * d.C; break;
+        case HGD_S_KV: *numel = (size_t)d.n_attn * 2 * B * d.nkv * (size_t)Lmax * d.hd; break;
+        default: *numel = (size_t)B; break;
+    }
+    return HGD_OK;
+}
+
+int hgd_state_init(hgd_state* st, const hgd_model* m, int B, int Tmax, int Lmax, void* arena, size_t bytes) {
+    if (!st || !m || !arena) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_state_dims(B, Tmax, Lmax))) return rc;
+    if (reinterpret_cast<uintptr_t>(arena) & 255u) return HGD_ERR_MISALIGNED;
+    size_t off[SC_COUNT];
+    state_layout(d, B, Tmax, Lmax, off);
+    if (bytes < off[SC_END]) return HGD_ERR_BUFFER_TOO_SMALL;
+    std::memset(st, 0, sizeof(*st));
+    st->B = B; st->Tmax = Tmax; st->Lmax = Lmax;
+    st->arena = arena;
+    st->arena_bytes = off[SC_END];
+    for (int i = 0; i < SC_COUNT && i < 32; ++i) st->off[i] = off[i];
+    return HGD_OK;
+}
+
+int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T) {
+    if (!m || B < 1 || T < 1) return -1;
+    Dims d;
+    if (dims_of(&m->cfg, &d)) return -1;
+    const int M = B * T;
+    int n = 0;
+    for (int l = 0; l < d.L; ++l) {
+        const bool att = is_attn_layer(&m->cfg, l);
+        n += gemv_chunks(M, d.D);                                   // in-projection
+        n += att ? 3 : 1;                                           // rope/partial/merge or GDN mixer
+        n += gemv_chunks(M, att ? d.nq * d.hd : d.H * d.dv);        // out-projection
+        n += gemv_chunks(M, d.D) + gemv_chunks(M, d.I);             // SwiGLU, down
+    }
+    n += gemv_chunks(M, d.D) + 1;                                   // LM head, argmax
+    return n;
+}
+
+int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T, float* logits,
+                           int32_t* argmax, float* S_rec, float* tail_rec, int32_t* status_dev,
+                           hgd_stream_t stream) {
+    if (!m || !st || !tokens || !argmax || !st->arena) return HGD_ERR_INVALID_ARG;
+    if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if ((logits && !al16(logits)) || !al16(argmax) || !al16(tokens) || (S_rec && !al16(S_rec)) ||
+        (tail_rec && !al16(tail_rec)))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int B = st->B, M = B * T, Lmax = st->Lmax;
+    uint8_t* A = static_cast<uint8_t*>(st->arena);
+    float* Sall = reinterpret_cast<float*>(A + st->off[SC_S]);
+    float* conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
+    bf16_t* kv = reinterpret_cast<bf16_t*>(A + st->off[SC_KV]);
+    int32_t* pos = reinterpret_cast<int32_t*>(A + st->off[SC_POS]);
+    bf16_t* resid = reinterpret_cast<bf16_t*>(A + st->off[SC_RESID]);
+    float* proj = reinterpret_cast<float*>(A + st->off[SC_PROJ]);
+    float* obuf = reinterpret_cast<float*>(A + st->off[SC_O]);
+    float* qrot = reinterpret_cast<float*>(A + st->off[SC_QROT]);
+    bf16_t* attn = reinterpret_cast<bf16_t*>(A + st->off[SC_ATTN]);
+    float* part = reinterpret_cast<float*>(A + st->off[SC_PART]);
+    bf16_t* mlp = reinterpret_cast<bf16_t*>(A + st->off[SC_MLP]);
+    float* bestv = reinterpret_cast<float*>(A + st->off[SC_BESTV]);
+    int32_t* besti = reinterpret_cast<int32_t*>(A + st->off[SC_BESTI]);
+    const int64_t proj_ld = std::max(d.gdn_out, d.attn_out);
+    const float eps = m->cfg.norm_eps;
+    const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
+    const size_t c_layer = (size_t)B * (d.kc - 1) * d.C;
+    const size_t kv_half = (size_t)B * d.nkv * Lmax * d.hd;
+    const size_t srec_layer = (size_t)B * T * d.H * d.dv * d.dk;
+    const size_t trec_layer = (size_t)B * T * (d.kc - 1) * d.C;
+    int ig = 0, ia = 0;
+    for (int l = 0; l < d.L; ++l) {
+        const uint16_t* const* w = m->w[l];
+        const bool att = is_attn_layer(&m->cfg, l);
+        // input RMSNorm + in-projection (layer 0 gathers the embedding rows)
+        {
+            GemvParams p = {};
+            p.W = w[HGD_W_IN]; p.N = (int)(att ? d.attn_out : d.gdn_out); p.K = d.D;
+            p.x = resid; p.x_ld = d.D; p.norm_w = w[HGD_W_IN_NORM]; p.eps = eps;
+            p.y = proj; p.y_ld = proj_ld; p.status = status_dev;
+            if (l == 0) {
+                p.tokens = tokens; p.embed = m->embed; p.vocab = d.V; p.resid_out = resid; p.resid_out_ld = d.D;
+                rc = run_gemv<PRO_EMBED_RMSNORM, EPI_F32>(p, M, di.sms, s, nullptr);
+            } else {
+                rc = run_gemv<PRO_RMSNORM, EPI_F32>(p, M, di.sms, s, nullptr);
+            }
+            if (rc) return rc;
+        }
+        if (!att) {
+            GdnLayerParams g{};
+            g.proj = proj; g.proj_ld = proj_ld; g.conv_w = w[HGD_W_CONV];
+            g.A_log = w[HGD_W_A_LOG]; g.dt_bias = w[HGD_W_DT_BIAS];
+            g.S = Sall + ig * s_layer; g.tail = conv + ig * c_layer;
+            g.o = obuf; g.o_ld = (int64_t)d.H * d.dv;
+            g.S_rec = S_rec ? S_rec + ig * srec_layer : nullptr;
+            g.tail_rec = tail_rec ? tail_rec + ig * trec_layer : nullptr;
+            g.B = B; g.T = T; g.H = d.H; g.dv = d.dv;
+            const dim3 grid(B * d.H, d.dv / GDN_ROWS), block(GDN_WARPS * 32);
+            cudaError_t e;
+            switch (d.dk) {
+                case 32: e = launch_pdl(k_gdn_layer<1, 4>, grid, block, 0, s, g); break;
+                case 64: e = launch_pdl(k_gdn_layer<2, 4>, grid, block, 0, s, g); break;
+                case 128: e = launch_pdl(k_gdn_layer<4, 4>, grid, block, 0, s, g); break;
+                default: e = launch_pdl(k_gdn_layer<8, 4>, grid, block, 0, s, g); break;
+            }
+            if ((rc = launch_status(e))) return rc;
+            GemvParams p = {};
+            p.W = w[HGD_W_OUT]; p.N = d.D; p.K = d.H * d.dv;
+            p.o = obuf; p.o_ld = (int64_t)d.H * d.dv;
+            p.z = proj + d.C; p.z_ld = proj_ld; p.gnorm_w = w[HGD_W_GNORM]; p.gn_d = d.dv; p.eps = eps;
+            p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
+            if ((rc = run_gemv<PRO_GATED_NORM, EPI_RESID>(p, M, di.sms, s, nullptr))) return rc;
+            ++ig;
+        } else {
+            AttnParams a{};
+            a.proj = proj; a.proj_ld = proj_ld; a.qrot = qrot;
+            a.kcache = kv + (size_t)ia * 2 * kv_half; a.vcache = a.kcache + kv_half;
+            a.pos = pos; a.part = part; a.out = attn; a.status = status_dev;
+            a.B = B; a.T = T; a.nq = d.nq; a.nkv = d.nkv; a.hd = d.hd; a.Lmax = Lmax;
+            a.max_chunks = max_chunks_of(Lmax); a.rope_base = m->cfg.rope_base;
+            cudaError_t e = launch_pdl(k_rope_append, dim3(M), dim3(256), 0, s, a);
+            if ((rc = launch_status(e))) return rc;
+            e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(128), 0, s, a);
+            if ((rc = launch_status(e))) return rc;
+            e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
+            if ((rc = launch_status(e))) return rc;
+            GemvParams p = {};
+            p.W = w[HGD_W_OUT]; p.N = d.D; p.K = d.nq * d.hd;
+            p.x = attn; p.x_ld = (int64_t)d.nq * d.hd;
+            p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
+            if ((rc = run_gemv<PRO_COPY, EPI_RESID>(p, M, di.sms, s, nullptr))) return rc;
+            ++ia;
+        }
+        // MLP: RMSNorm + fused up/gate SwiGLU, then down + residual
+        {
+            GemvParams p = {};
+            p.W = w[HGD_W_GATE]; p.W2 = w[HGD_W_UP]; p.N = d.I; p.K = d.D;
+            p.x = resid; p.x_ld = d.D; p.norm_w = w[HGD_W_POST_NORM]; p.eps = eps;
+            p.y = mlp; p.y_ld = d.I; p.status = status_dev;
+            if ((rc = run_gemv<PRO_RMSNORM, EPI_SWIGLU>(p, M, di.sms, s, nullptr))) return rc;
+        }
+        {
+            GemvParams p = {};
+            p.W = w[HGD_W_DOWN]; p.N = d.D; p.K = d.I;
+            p.x = mlp; p.x_ld = d.I;
+            p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
+            if ((rc = run_gemv<PRO_COPY, EPI_RESID>(p, M, di.sms, s, nullptr))) return rc;
+        }
+    }
+    // final norm + tied LM head + per-CTA argmax, then the row argmax
+    {
+        GemvParams p = {};
+        p.W = m->embed; p.N = d.V; p.K = d.D;
+        p.x = resid; p.x_ld = d.D; p.norm_w = m->final_norm; p.eps = eps;
+        p.logits = logits; p.logits_ld = d.V; p.best_v = bestv; p.best_i = besti; p.status = status_dev;
+        if ((rc = run_gemv<PRO_RMSNORM, EPI_ARGMAX>(p, M, di.sms, s, nullptr))) return rc;
+        const int G = gemv_grid(d.V, GV_ROWS, di.sms);
+        cudaError_t e = launch_pdl(k_argmax_finalize, dim3(M), dim3(128), 0, s, (const float*)bestv,
+                                   (const int32_t*)besti, G, M, argmax, status_dev, pos, B, T);
+        if ((rc = launch_status(e))) return rc;
+    }
+    return HGD_OK;
+}
+
+}  // extern "C"

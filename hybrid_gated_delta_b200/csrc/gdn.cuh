@@ -1,0 +1,349 @@
+// gdn.cuh -- causal conv1d tail update and the gated-delta-rule state update.
+//
+// "qwen3_5 cuda: mixed-width MLX checkpoints ... #849", PR body: the gated delta
+// rule and the causal convolution, windows of rows that record each row's
+// recurrence and conv tail and equal one-row steps bit for bit.
+// "Running on Turing (sm_75)", What was checked: GDN decode kernels keep the
+// state [num_heads, V, K].
+//
+// State update per head, per row (beta, alpha scalars; k, q L2-normalised):
+//   w_i = S_i . k,   delta_i = beta (v_i - alpha w_i),   S_i <- alpha S_i + delta_i k,
+//   o_i = S_i . q
+// which is S <- alpha S (I - beta k k^T) + beta v k^T, o = S q, written as a rank-1
+// update so each of the dv rows of S is independent.  A warp owns RPW rows; lane
+// l holds KPL consecutive k-elements of each row (a 16-byte load when KPL = 4),
+// so every row of the fp32 state stays in registers across all T rows of a
+// call and is read and written once per call.  The arithmetic of a row depends
+// only on that row's inputs, so T-row calls equal T one-row calls bit for bit.
+#pragma once
+
+#include "common.cuh"
+
+namespace hgd {
+
+constexpr int GDN_WARPS = 4;
+constexpr int GDN_RPW = 4;                        // state rows per warp
+constexpr int GDN_ROWS = GDN_WARPS * GDN_RPW;     // state rows per CTA (16)
+
+template <int KPL>
+__device__ __forceinline__ void ld_vec(float (&d)[KPL], const float* p) {
+    if (KPL == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+    } else if (KPL == 8) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        const float4 u = *reinterpret_cast<const float4*>(p + 4);
+        d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+        d[4] = u.x; d[5] = u.y; d[6] = u.z; d[7] = u.w;
+    } else if (KPL == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(p);
+        d[0] = v.x; d[1] = v.y;
+    } else {
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) d[e] = p[e];
+    }
+}
+template <int KPL>
+__device__ __forceinline__ void st_vec(float* p, const float (&d)[KPL]) {
+    if (KPL == 4) {
+        *reinterpret_cast<float4*>(p) = make_float4(d[0], d[1], d[2], d[3]);
+    } else if (KPL == 8) {
+        *reinterpret_cast<float4*>(p) = make_float4(d[0], d[1], d[2], d[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(d[4], d[5], d[6], d[7]);
+    } else if (KPL == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(d[0], d[1]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) p[e] = d[e];
+    }
+}
+
+// One recurrent row for RPW state rows held by this warp.  kv/qv: this lane's
+// normalised key/query elements; vrow[r]: value of state row r; returns o in
+// every lane.
+template <int KPL>
+__device__ __forceinline__ void gdn_rows_step(float (&S)[GDN_RPW][KPL], const float (&kv)[KPL],
+                                              const float (&qv)[KPL], float alpha, float beta,
+                                              const float (&vrow)[GDN_RPW], float (&o)[GDN_RPW]) {
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) {
+        float w = 0.f;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) w = fmaf(S[r][e], kv[e], w);
+        w = warp_sum(w);
+        const float delta = beta * (vrow[r] - alpha * w);
+        float ov = 0.f;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            S[r][e] = fmaf(delta, kv[e], alpha * S[r][e]);
+            ov = fmaf(S[r][e], qv[e], ov);
+        }
+        o[r] = warp_sum(ov);
+    }
+}
+
+// L2 normalisation scale 1/sqrt(sum x^2 + 1e-6) of a dk-vector held in shared
+// memory, computed by one warp (lane-strided KPL chunks, then a butterfly).
+template <int KPL>
+__device__ __forceinline__ float l2_scale(const float* x, int lane) {
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+        const float a = x[lane * KPL + e];
+        ss = fmaf(a, a, ss);
+    }
+    ss = warp_sum(ss);
+    return rsqrtf(ss + 1e-6f);
+}
+
+// ------------------------------------------------------- standalone GDN step
+struct GdnParams {
+    const float* q; const float* k; const float* v; int64_t stride;
+    const float* g; const float* b;
+    float* S; float* o; bf16_t* o_bf16; float* S_rec;
+    int B, T, H, dk, dv, l2norm;
+};
+
+// grid (B*H, dv/16), block 128: a CTA owns 16 state rows of one (stream, head).
+template <int KPL>
+__global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_step(const __grid_constant__ GdnParams p) {
+    pdl_launch();
+    pdl_wait();
+    constexpr int DK = 32 * KPL;
+    __shared__ float qs[DK], ks[DK], coef[4];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int row0 = blockIdx.y * GDN_ROWS + warp * GDN_RPW;
+    float S[GDN_RPW][KPL];
+    float* Sbase = p.S + ((int64_t)(b * p.H + h) * p.dv + row0) * DK + lane * KPL;
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
+
+    for (int t = 0; t < p.T; ++t) {
+        const int64_t row = (int64_t)b * p.T + t;
+        const float* qp = p.q + row * p.stride + (int64_t)h * DK;
+        const float* kp = p.k + row * p.stride + (int64_t)h * DK;
+        __syncthreads();
+        for (int i = tid; i < DK; i += GDN_WARPS * 32) { qs[i] = qp[i]; ks[i] = kp[i]; }
+        __syncthreads();
+        if (warp == 0) { const float s = p.l2norm ? l2_scale<KPL>(qs, lane) : 1.f; if (lane == 0) coef[0] = s; }
+        if (warp == 1) { const float s = p.l2norm ? l2_scale<KPL>(ks, lane) : 1.f; if (lane == 0) coef[1] = s; }
+        if (warp == 2 && lane == 0) {
+            coef[2] = expf(p.g[row * p.H + h]);
+            coef[3] = sigmoid_f(p.b[row * p.H + h]);
+        }
+        __syncthreads();
+        float kv[KPL], qv[KPL];
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
+        float vrow[GDN_RPW], o[GDN_RPW];
+        const float* vp = p.v + row * p.stride + (int64_t)h * p.dv + row0;
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
+        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o);
+        const int64_t orow = (row * p.H + h) * p.dv + row0;
+        if (lane < GDN_RPW) {
+            float ov = o[0];
+#pragma unroll
+            for (int r = 1; r < GDN_RPW; ++r) if (lane == r) ov = o[r];
+            p.o[orow + lane] = ov;
+            if (p.o_bf16) p.o_bf16[orow + lane] = f2bf(ov);
+        }
+        if (p.S_rec) {
+            float* rp = p.S_rec + ((row * p.H + h) * p.dv + row0) * DK + lane * KPL;
+#pragma unroll
+            for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
+}
+
+// ---------------------------------------------------------- standalone conv
+struct ConvParams {
+    const float* x; float* tail; const bf16_t* w; float* y; float* tail_rec;
+    int B, T, C, kc, silu;
+};
+
+// One thread per (stream, channel); rows in order.
+__global__ void k_conv_tail(const __grid_constant__ ConvParams p) {
+    pdl_launch();
+    pdl_wait();
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)p.B * p.C) return;
+    const int b = (int)(idx / p.C), c = (int)(idx % p.C);
+    const int nt = p.kc - 1;
+    float tl[8], w[8];
+    for (int j = 0; j < p.kc; ++j) w[j] = bf2f(p.w[(int64_t)c * p.kc + j]);
+    float* tb = p.tail + (int64_t)b * nt * p.C + c;
+    for (int j = 0; j < nt; ++j) tl[j] = tb[(int64_t)j * p.C];
+    for (int t = 0; t < p.T; ++t) {
+        const int64_t row = (int64_t)b * p.T + t;
+        const float xv = p.x[row * p.C + c];
+        float s = 0.f;
+        for (int j = 0; j < nt; ++j) s = fmaf(w[j], tl[j], s);
+        s = fmaf(w[nt], xv, s);
+        p.y[row * p.C + c] = p.silu ? silu_f(s) : s;
+        for (int j = 0; j + 1 < nt; ++j) tl[j] = tl[j + 1];
+        if (nt > 0) tl[nt - 1] = xv;
+        if (p.tail_rec)
+            for (int j = 0; j < nt; ++j) p.tail_rec[(row * nt + j) * p.C + c] = tl[j];
+    }
+    for (int j = 0; j < nt; ++j) tb[(int64_t)j * p.C] = tl[j];
+}
+
+// ------------------------------------------------------- stack: GDN mixer
+// Conv (over q|k|v channels, SiLU), gates from a/b, L2 norm and the state
+// update for one GDN layer of the stack.  grid (B*H, dv/16), block 128.
+// The CTA with blockIdx.y == 0 also owns the q/k channels' conv tails; every
+// CTA owns the tails of its 16 value channels.  Rows (b, t) are token rows
+// b*T + t of the projection buffer [M][proj_ld] with columns
+// q (H*dk) | k (H*dk) | v (H*dv) | z (H*dv) | a (H) | b (H).
+struct GdnLayerParams {
+    const float* proj; int64_t proj_ld;
+    const bf16_t* conv_w;       // [C][kc]
+    const bf16_t* A_log; const bf16_t* dt_bias;  // [H]
+    float* S;                   // this layer: [B][H][dv][dk]
+    float* tail;                // this layer: [B][kc-1][C]
+    float* o; int64_t o_ld;     // [M][o_ld]
+    float* S_rec;               // this layer: [B][T][H][dv][dk] or null
+    float* tail_rec;            // this layer: [B][T][kc-1][C] or null
+    int B, T, H, dv;
+};
+
+template <int KPL, int KC>
+__global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_constant__ GdnLayerParams p) {
+    pdl_launch();
+    pdl_wait();
+    constexpr int DK = 32 * KPL;
+    constexpr int NT = GDN_WARPS * 32;
+    constexpr int kc = KC, nt = KC - 1;
+    __shared__ float qs[DK], ks[DK], vs[GDN_ROWS], coef[4];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H, dv = p.dv;
+    const int b = blockIdx.x / H, h = blockIdx.x % H;
+    const int vrow0 = blockIdx.y * GDN_ROWS;
+    const int row0 = vrow0 + warp * GDN_RPW;
+    const int64_t C = 2 * (int64_t)H * DK + (int64_t)H * dv;
+    const bool own_qk = (blockIdx.y == 0);
+
+    // channels handled by this thread: q channel and k channel (tid < DK, looped),
+    // and value channel tid (< 16)
+    constexpr int QK_PER_T = (DK + NT - 1) / NT;
+    float tq[QK_PER_T][nt], tk[QK_PER_T][nt], wq[QK_PER_T][kc], wk[QK_PER_T][kc];
+    float tv[nt], wv[kc];
+    float* tail_b = p.tail + (int64_t)b * nt * C;
+#pragma unroll
+    for (int u = 0; u < QK_PER_T; ++u) {
+        const int i = tid + u * NT;
+        if (i < DK) {
+            const int64_t cq = (int64_t)h * DK + i, ck = (int64_t)H * DK + h * DK + i;
+#pragma unroll
+            for (int j = 0; j < kc; ++j) { wq[u][j] = bf2f(p.conv_w[cq * kc + j]); wk[u][j] = bf2f(p.conv_w[ck * kc + j]); }
+#pragma unroll
+            for (int j = 0; j < nt; ++j) { tq[u][j] = tail_b[j * C + cq]; tk[u][j] = tail_b[j * C + ck]; }
+        }
+    }
+    const int64_t cv = 2 * (int64_t)H * DK + (int64_t)h * dv + vrow0 + tid;
+    if (tid < GDN_ROWS) {
+#pragma unroll
+        for (int j = 0; j < kc; ++j) wv[j] = bf2f(p.conv_w[cv * kc + j]);
+#pragma unroll
+        for (int j = 0; j < nt; ++j) tv[j] = tail_b[j * C + cv];
+    }
+    const float A = expf(bf2f(p.A_log[h])), dtb = bf2f(p.dt_bias[h]);
+
+    float S[GDN_RPW][KPL];
+    float* Sbase = p.S + ((int64_t)(b * H + h) * dv + row0) * DK + lane * KPL;
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
+
+    for (int t = 0; t < p.T; ++t) {
+        const int64_t row = (int64_t)b * p.T + t;
+        const float* pr = p.proj + row * p.proj_ld;
+        float* trec = p.tail_rec ? p.tail_rec + ((int64_t)b * p.T + t) * nt * C : nullptr;
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < QK_PER_T; ++u) {
+            const int i = tid + u * NT;
+            if (i < DK) {
+                const int64_t cq = (int64_t)h * DK + i, ck = (int64_t)H * DK + h * DK + i;
+                const float xq = pr[cq], xk = pr[ck];
+                float sq = 0.f, sk = 0.f;
+#pragma unroll
+                for (int j = 0; j < nt; ++j) { sq = fmaf(wq[u][j], tq[u][j], sq); sk = fmaf(wk[u][j], tk[u][j], sk); }
+                sq = fmaf(wq[u][nt], xq, sq);
+                sk = fmaf(wk[u][nt], xk, sk);
+                qs[i] = silu_f(sq);
+                ks[i] = silu_f(sk);
+#pragma unroll
+                for (int j = 0; j + 1 < nt; ++j) { tq[u][j] = tq[u][j + 1]; tk[u][j] = tk[u][j + 1]; }
+                tq[u][nt - 1] = xq;
+                tk[u][nt - 1] = xk;
+                if (trec && own_qk)
+#pragma unroll
+                    for (int j = 0; j < nt; ++j) { trec[j * C + cq] = tq[u][j]; trec[j * C + ck] = tk[u][j]; }
+            }
+        }
+        if (tid < GDN_ROWS) {
+            const float xv = pr[cv];
+            float sv = 0.f;
+#pragma unroll
+            for (int j = 0; j < nt; ++j) sv = fmaf(wv[j], tv[j], sv);
+            sv = fmaf(wv[nt], xv, sv);
+            vs[tid] = silu_f(sv);
+#pragma unroll
+            for (int j = 0; j + 1 < nt; ++j) tv[j] = tv[j + 1];
+            tv[nt - 1] = xv;
+            if (trec)
+#pragma unroll
+                for (int j = 0; j < nt; ++j) trec[j * C + cv] = tv[j];
+        }
+        __syncthreads();
+        if (warp == 0) { const float s = l2_scale<KPL>(qs, lane); if (lane == 0) coef[0] = s; }
+        if (warp == 1) { const float s = l2_scale<KPL>(ks, lane); if (lane == 0) coef[1] = s; }
+        if (warp == 2 && lane == 0) {
+            const float a = pr[C + (int64_t)H * dv + h];
+            const float braw = pr[C + (int64_t)H * dv + H + h];
+            const float g = -A * softplus_f(a + dtb);
+            coef[2] = expf(g);
+            coef[3] = sigmoid_f(braw);
+        }
+        __syncthreads();
+        float kv[KPL], qv[KPL];
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
+        float vrow[GDN_RPW], o[GDN_RPW];
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vs[warp * GDN_RPW + r];
+        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o);
+        if (lane < GDN_RPW) {
+            float ov = o[0];
+#pragma unroll
+            for (int r = 1; r < GDN_RPW; ++r) if (lane == r) ov = o[r];
+            p.o[row * p.o_ld + (int64_t)h * dv + row0 + lane] = ov;
+        }
+        if (p.S_rec) {
+            float* rp = p.S_rec + ((((int64_t)b * p.T + t) * H + h) * dv + row0) * DK + lane * KPL;
+#pragma unroll
+            for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
+    // conv tails back
+#pragma unroll
+    for (int u = 0; u < QK_PER_T; ++u) {
+        const int i = tid + u * NT;
+        if (i < DK && own_qk) {
+            const int64_t cq = (int64_t)h * DK + i, ck = (int64_t)H * DK + h * DK + i;
+#pragma unroll
+            for (int j = 0; j < nt; ++j) { tail_b[j * C + cq] = tq[u][j]; tail_b[j * C + ck] = tk[u][j]; }
+        }
+    }
+    if (tid < GDN_ROWS)
+#pragma unroll
+        for (int j = 0; j < nt; ++j) tail_b[j * C + cv] = tv[j];
+}
+
+}  // namespace hgd

@@ -1,0 +1,257 @@
+/*
+ * hgd.h -- C ABI of the B200 (sm_100a) hybrid gated-delta decode library.
+ *
+ * The library computes the small-batch decode step of a hybrid layer stack in
+ * which three gated-delta-rule (GDN, "DeltaNet") layers alternate with one gated
+ * full-attention layer, as the pages below describe it:
+ *   [LUCE] "luce-megakernel HANDOFF.md" -- Model: 24 layers, [DN,DN,DN,FA] x 6;
+ *          Architecture: one persistent decode kernel streaming all layers.
+ *   [TF]   "qwen3_5 cuda: mixed-width MLX checkpoints ... #849" -- PR body: gated
+ *          delta rule, causal convolution and gated attention at bf16 rounding
+ *          points; windows of up to 16 rows that record each row's recurrence
+ *          and convolution tail and equal one-row steps bit for bit; attention
+ *          partials over key chunks cut at logical positions, then a merge.
+ *   [FT]   "Running on Turing (sm_75)" -- What was checked: RMSNorm, causal conv,
+ *          GDN decode, gated RMSNorm, silu_and_mul, the 248k-row lm_head; the GDN
+ *          state is stored [num_heads, V, K]; debugging notes: an unchecked launch
+ *          left outputs uninitialised.
+ *   [AST]  "decode_linear_benchmark.md" -- commit message: BF16 GEMV and the fused
+ *          up/gate SwiGLU primitive for decode shapes, M = 1..32.
+ * The recurrence is the gated delta rule in its standard form (the pages name it
+ * without writing it out):
+ *   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t,
+ *   q, k L2-normalised, alpha = exp(g), beta = sigmoid(b).
+ *
+ * Conventions for every entry point:
+ *  - Every call returns an int status (HGD_OK = 0).  Nothing aborts or traps.  A
+ *    rejected call launches nothing and writes nothing.
+ *  - The caller owns every buffer.  The library allocates no device memory.
+ *    Device pointers are plain CUDA device addresses of the current device;
+ *    `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *  - Calls are asynchronous on `stream`; a launch failure is reported as
+ *    HGD_ERR_CUDA (cudaGetLastError is consumed).  Errors found inside a kernel
+ *    (a NaN logit, a wait that ran out) are written to a caller-provided device
+ *    status word, read after the stream synchronises.
+ *  - bf16 tensors are 16-bit bit patterns (uint16_t); row-major, contiguous.
+ *    Weights use the [out, in] (Linear) layout.
+ *  - Device pointers must be 16-byte aligned (HGD_ERR_MISALIGNED otherwise).
+ *  - Only sm_100 devices are supported (HGD_ERR_UNSUPPORTED_DEVICE otherwise).
+ */
+#ifndef HGD_H
+#define HGD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HGD_API __attribute__((visibility("default")))
+#else
+#define HGD_API
+#endif
+
+typedef struct CUstream_st* hgd_stream_t; /* same type as cudaStream_t */
+
+enum hgd_status {
+    HGD_OK = 0,
+    HGD_ERR_INVALID_ARG = 1,        /* NULL where a buffer is required, negative size */
+    HGD_ERR_UNSUPPORTED_SHAPE = 2,  /* a size outside what the kernels implement */
+    HGD_ERR_MISALIGNED = 3,         /* a pointer that is not 16-byte aligned */
+    HGD_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    HGD_ERR_TIMEOUT = 5,            /* a bounded in-kernel wait ran out (device status) */
+    HGD_ERR_NOT_CORESIDENT = 6,     /* a persistent launch cannot keep all CTAs resident */
+    HGD_ERR_NAN = 7,                /* a NaN logit reached the argmax (device status) */
+    HGD_ERR_UNSUPPORTED_DEVICE = 8, /* the current device is not sm_100 */
+    HGD_ERR_BUFFER_TOO_SMALL = 9    /* an arena smaller than the reported size */
+};
+
+/* Static text for a status code ("unknown status" for anything else). */
+HGD_API const char* hgd_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+HGD_API int hgd_version(void);
+
+/* ------------------------------------------------------------------ GEMV ---
+ * y[m][n] = sum_k x[m][k] * W[n][k]   ([AST] BF16 GEMV for decode shapes).
+ *   W  [N, K] bf16 device, x [M, K] bf16 device.
+ *   y  [M, N] device: fp32 if y_is_fp32, else bf16 (round to nearest even).
+ * fp32 accumulation.  Each output's arithmetic depends on K only, never on M,
+ * N or the device's SM count: a row computed in an M-row call equals the same
+ * row computed alone, bit for bit.
+ * Shapes: 1 <= M, 1 <= N, 32 <= K <= 65536 with K % 32 == 0
+ * (HGD_ERR_UNSUPPORTED_SHAPE otherwise).  y must not overlap W or x. */
+HGD_API int hgd_gemv_bf16(const uint16_t* W, const uint16_t* x, void* y, int y_is_fp32,
+                  int M, int N, int K, hgd_stream_t stream);
+
+/* h[m][i] = bf16( silu(g) * u ),  g = x . W_gate[i],  u = x . W_up[i]
+ * ([AST] fused BF16 up/gate SwiGLU; [FT] silu_and_mul), silu(t) = t/(1+exp(-t)).
+ *   W_gate, W_up [I, K] bf16 device; x [M, K] bf16 device; h [M, I] bf16 device.
+ * g and u are fp32 dot products computed exactly as hgd_gemv_bf16 computes them.
+ * Shapes as hgd_gemv_bf16 with N = I. */
+HGD_API int hgd_gemv_swiglu_bf16(const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* x,
+                         uint16_t* h, int M, int I, int K, hgd_stream_t stream);
+
+/* -------------------------------------------------------- conv1d tail ---
+ * Depthwise causal conv1d over a kept tail ([TF] causal convolution with each
+ * row's tail recorded).  For stream b, channel c and row t = 0..T-1:
+ *   s = sum_{j<kc-1} w[c][j] * tail[b][j][c] + w[c][kc-1] * x[b][t][c]
+ *   y[b][t][c] = apply_silu ? silu(s) : s
+ *   tail[b][:, c] shifts by one row and takes x[b][t][c] as its newest entry.
+ *   x [B, T, C] fp32, tail [B, kc-1, C] fp32 (oldest first, updated in place),
+ *   w [C, kc] bf16, y [B, T, C] fp32, tail_rec [B, T, kc-1, C] fp32 or NULL
+ *   (the tail after each row).  All device pointers.
+ * Shapes: B, T, C >= 1; 2 <= kc <= 8.  A T-row call equals T one-row calls
+ * bit for bit. */
+HGD_API int hgd_conv1d_tail_update(const float* x, float* tail, const uint16_t* w, float* y,
+                           float* tail_rec, int B, int T, int C, int kc, int apply_silu,
+                           hgd_stream_t stream);
+
+/* ---------------------------------------------------- gated delta rule ---
+ * One or more recurrent rows of the gated delta rule per (stream, head), state
+ * updated in place in fp32 ([FT] state layout [heads, V, K]).
+ * Row (b,t), head h reads
+ *   q = q_ptr + (b*T+t)*row_stride + h*dk,  k likewise,  v = v_ptr + (b*T+t)*row_stride + h*dv,
+ *   g[(b*T+t)*H + h], b[(b*T+t)*H + h]   (raw: alpha = exp(g), beta = sigmoid(b)),
+ * and computes, with q,k L2-normalised over dk (x / sqrt(sum x^2 + 1e-6)) when
+ * l2norm_qk is set:
+ *   S <- alpha S + beta (v - alpha S k) k^T     (= alpha S (I - beta k k^T) + beta v k^T)
+ *   o = S q                                     (with the updated S)
+ *   S [B, H, dv, dk] fp32 device, in place.
+ *   o [B, T, H, dv] fp32 device; o_bf16 the same shape in bf16, or NULL.
+ *   S_rec [B, T, H, dv, dk] fp32 device or NULL: S after each row.
+ * row_stride (elements, >= H*dk and >= H*dv) lets q|k|v come packed in one
+ * [B*T, row_stride] array (e.g. a conv output); for separate contiguous
+ * [B,T,H,d] arrays pass H*dk.
+ * Shapes: dk in {32, 64, 128, 256}; dv a multiple of 16 up to 1024; H, B, T >= 1.
+ * A T-row call equals T one-row calls bit for bit. */
+HGD_API int hgd_gdn_decode_step(const float* q, const float* k, const float* v, int64_t row_stride,
+                        const float* g, const float* b, float* S, float* o, uint16_t* o_bf16,
+                        float* S_rec, int B, int T, int H, int dk, int dv, int l2norm_qk,
+                        hgd_stream_t stream);
+
+/* ------------------------------------------------------ decode stack ---- */
+
+/* Geometry of the hybrid stack ([LUCE] Model).  Layer l is a gated-attention
+ * layer iff l % attn_every == attn_every - 1, otherwise a GDN layer. */
+typedef struct hgd_config {
+    int32_t n_layers;      /* 24 */
+    int32_t hidden;        /* D = 1024 */
+    int32_t vocab;         /* 248320; the LM head is tied to the embedding */
+    int32_t gdn_heads;     /* H = 16 */
+    int32_t gdn_dk;        /* 128 */
+    int32_t gdn_dv;        /* 128 */
+    int32_t conv_k;        /* 4 */
+    int32_t attn_q_heads;  /* 8 */
+    int32_t attn_kv_heads; /* 2 */
+    int32_t attn_head_dim; /* 256 */
+    int32_t mlp_inter;     /* I = 3584 */
+    int32_t attn_every;    /* 4 */
+    float norm_eps;        /* 1e-6 */
+    float rope_base;       /* 10000 */
+} hgd_config;
+
+#define HGD_MAX_LAYERS 64
+
+/* Tensors of the weight arena.  Per layer (layer >= 0):                 */
+enum hgd_weight_tensor {
+    HGD_W_IN_NORM = 0,   /* [D] gain (bf16) */
+    HGD_W_IN = 1,        /* GDN: [2*H*dk + 2*H*dv + 2*H, D], rows q|k|v|z|a|b
+                            attention: [2*nq*hd + 2*nkv*hd, D], rows q|gate|k|v */
+    HGD_W_CONV = 2,      /* GDN: [2*H*dk + H*dv, kc] over channels q|k|v */
+    HGD_W_A_LOG = 3,     /* GDN: [H] */
+    HGD_W_DT_BIAS = 4,   /* GDN: [H] */
+    HGD_W_GNORM = 5,     /* GDN: [dv] gated-RMSNorm gain shared by heads */
+    HGD_W_OUT = 6,       /* GDN: [D, H*dv]; attention: [D, nq*hd] */
+    HGD_W_POST_NORM = 7, /* [D] */
+    HGD_W_GATE = 8,      /* [I, D] */
+    HGD_W_UP = 9,        /* [I, D] */
+    HGD_W_DOWN = 10,     /* [D, I] */
+    HGD_W_LAYER_COUNT = 11,
+    /* model-level tensors (layer = -1) */
+    HGD_W_EMBED = 100,      /* [V, D], also the LM head */
+    HGD_W_FINAL_NORM = 101  /* [D] */
+};
+
+/* Model handle.  Filled by hgd_model_init from a caller-owned weight arena;
+ * holds only pointers into it and the configuration. */
+typedef struct hgd_model {
+    hgd_config cfg;
+    const uint16_t* embed;
+    const uint16_t* final_norm;
+    const uint16_t* w[HGD_MAX_LAYERS][HGD_W_LAYER_COUNT];
+    size_t arena_bytes;
+} hgd_model;
+
+/* Bytes of the weight arena for `cfg` (every tensor 256-byte aligned). */
+HGD_API int hgd_model_arena_bytes(const hgd_config* cfg, size_t* bytes);
+
+/* Byte offset and element count of one tensor in the weight arena.  A tensor
+ * the layer does not have (e.g. HGD_W_CONV in an attention layer) reports
+ * numel = 0.  HGD_ERR_INVALID_ARG for an unknown tensor or layer. */
+HGD_API int hgd_model_tensor(const hgd_config* cfg, int layer, int tensor, size_t* offset,
+                     size_t* numel);
+
+/* Validate cfg and point `m` at the arena (device memory the caller filled with
+ * bf16 weights at the offsets above).  No allocation, no launch. */
+HGD_API int hgd_model_init(hgd_model* m, const hgd_config* cfg, const void* weight_arena, size_t bytes);
+
+/* Tensors of the state arena (per-stream recurrent state, KV cache, position,
+ * and the activation scratch of one call). */
+enum hgd_state_tensor {
+    HGD_S_GDN = 0,    /* [n_gdn, B, H, dv, dk] fp32 recurrent state */
+    HGD_S_CONV = 1,   /* [n_gdn, B, kc-1, 2*H*dk + H*dv] fp32 conv tails, oldest first */
+    HGD_S_KV = 2,     /* [n_attn, 2, B, nkv, Lmax, hd] bf16 (0 = keys, rotated) */
+    HGD_S_POS = 3,    /* [B] int32 position of each stream's next row */
+    HGD_S_COUNT = 4
+};
+
+typedef struct hgd_state {
+    int32_t B, Tmax, Lmax;
+    void* arena;
+    size_t arena_bytes;
+    size_t off[32];  /* byte offsets of the state tensors and scratch buffers */
+} hgd_state;
+
+/* Bytes of the state arena for B streams, up to Tmax rows per call and Lmax
+ * cache positions.  Shapes: B*Tmax <= 256, Lmax <= 16384. */
+HGD_API int hgd_state_arena_bytes(const hgd_config* cfg, int B, int Tmax, int Lmax, size_t* bytes);
+
+/* Byte offset and element count of a caller-visible state tensor. */
+HGD_API int hgd_state_tensor(const hgd_config* cfg, int B, int Tmax, int Lmax, int tensor,
+                     size_t* offset, size_t* numel);
+
+/* Lay the state out in `state_arena` (caller-owned device memory of at least
+ * hgd_state_arena_bytes).  The caller initialises S, conv tails, KV rows below
+ * each stream's position and the positions themselves; nothing is written here. */
+HGD_API int hgd_state_init(hgd_state* st, const hgd_model* m, int B, int Tmax, int Lmax,
+                   void* state_arena, size_t bytes);
+
+/* One decode call over T rows of each of B streams ([LUCE] decode step;
+ * [TF] windows of rows that equal one-row steps):
+ *   tokens [B, T] int32 device; row (b,t) sits at position pos[b]+t and attends
+ *   its stream's keys 0..pos[b]+t.
+ *   logits [B*T, V] fp32 device or NULL; argmax [B*T] int32 device (first
+ *   maximum, lowest index on ties).
+ *   S_rec [n_gdn, B, T, H, dv, dk] and tail_rec [n_gdn, B, T, kc-1, C] fp32
+ *   device or NULL: the recurrent state and conv tail after each row.
+ *   status_dev: int32 device word; the kernels write a nonzero hgd_status there
+ *   on an in-kernel error (it is not cleared; zero it before the call).
+ * Every step is on `stream` and reads sizes from the device, so a call can be
+ * captured in a CUDA graph and replayed while positions advance.  pos[b] += T
+ * at the end.  Requires 1 <= T <= Tmax and pos[b]+T <= Lmax (checked on the
+ * device: violation sets HGD_ERR_INVALID_ARG in status_dev and skips the row). */
+HGD_API int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_t* tokens,
+                           int T, float* logits, int32_t* argmax, float* S_rec,
+                           float* tail_rec, int32_t* status_dev, hgd_stream_t stream);
+
+/* Number of kernel launches one hgd_decode_layer_stack call over B streams and
+ * T rows issues (-1 on bad arguments). */
+HGD_API int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HGD_H */
