@@ -1,0 +1,331 @@
+#!/usr/bin/env python3
+"""Decode throughput of the 24-layer hybrid gated-delta stack at batch 1.
+
+Workload: hidden 1024, 24 layers (3 gated-delta-rule layers : 1 gated
+full-attention layer, x6), GDN 16 heads d=128, conv k=4, attention 8 q / 2 kv
+heads of 256, SwiGLU MLP 3584, vocab 248320 (tied head), random-init bf16
+weights N(0, 0.02), KV context 512 prefilled, greedy decoding: one step = one
+token through the whole stack (every weight byte streamed from HBM: 1.5 GB per
+step, far larger than the 126 MB L2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun (N > 1) every rank decodes its own
+stream (replicas, no collective on the data path); value = all ranks' tokens /
+the slowest rank's device time.  `--impl reference` times the CPU oracle on this
+host's cores instead (a bounded sample of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s at B=1 (24-layer stack) and achieved HBM GB/s vs 8 TB/s"
+UNIT = "tokens/s"
+PREFILL = 512
+WORKLOAD = ("24-layer hybrid stack (3 GDN : 1 gated attention), hidden 1024, vocab 248320, "
+            "GDN 16x128, attn 8q/2kv x256, MLP 3584, batch 1, KV context 512, greedy decode")
+
+
+def algorithmic_bytes(cfg: dict, L_keys: float) -> dict:
+    """Bytes one decode token must move, by component (the HBM roofline numerator)."""
+    D, V, H, dk, dv, kc = (cfg[k] for k in ("hidden", "vocab", "gdn_heads", "gdn_dk", "gdn_dv", "conv_k"))
+    nq, nkv, hd, I = (cfg[k] for k in ("attn_q_heads", "attn_kv_heads", "attn_head_dim", "mlp_inter"))
+    import hgd_synth as syn
+    n_gdn, n_attn = syn.layer_counts(cfg)
+    Cc = 2 * H * dk + H * dv
+    w_gdn = (Cc + H * dv + 2 * H) * D + D * H * dv + 3 * I * D + 2 * D + Cc * kc + 2 * H + dv
+    w_att = (2 * nq * hd + 2 * nkv * hd) * D + D * nq * hd + 3 * I * D + 2 * D
+    weights = 2 * (n_gdn * w_gdn + n_attn * w_att + V * D + D)
+    state = n_gdn * H * dv * dk * 4 * 2
+    tails = n_gdn * (kc - 1) * Cc * 4 * 2
+    kv = n_attn * 2 * nkv * hd * 2 * L_keys + n_attn * 2 * nkv * hd * 2  # read L keys, write 1
+    head = 2 * V * D
+    return {"weights": weights, "state": state, "tails": tails, "kv": kv, "head": head,
+            "total": weights + state + tails + kv}
+
+
+def measured_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "_fallback": True}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- reference --
+
+def run_reference(args) -> None:
+    """The CPU oracle on this host: greedy decode of the same workload, one token
+    per step, single-threaded; a bounded number of steps."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import hgd_synth as syn
+    from oracle import Oracle
+    orc = Oracle()
+    cfg = syn.STACK_CFG
+    w = syn.stack_weights(cfg, seed=4)
+    m = orc.make_model(cfg, w)
+    init = syn.stack_state(cfg, 1, PREFILL + 64, prefill=PREFILL, seed=4)
+    st = {"S": init["S"].astype(np.float64), "tail": init["tail"].astype(np.float64), "kv": init["kv"],
+          "pos": init["pos"]}
+    tok = syn.stack_tokens(cfg, 1, 1, seed=4)
+    budget_s = float(os.environ.get("HGD_REF_BUDGET_S", "60"))
+    warm = min(args.warmup, 1)
+    for _ in range(warm):
+        tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
+    t0 = time.perf_counter()
+    n = 0
+    while n < args.steps:
+        tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    v = n / dt
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": n, "warmup": warm, "ms_per_step": 1000 * dt / n, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "batch": 1, "kv_context": PREFILL},
+           "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                            "sample": f"{n} greedy tokens of the full stack (of {args.steps} asked; "
+                                      f"{budget_s:.0f} s budget), single-threaded C oracle, fp64"},
+           "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def cpu_baseline_sample(tokens: int = 4) -> dict:
+    import hgd_synth as syn
+    from oracle import Oracle
+    orc = Oracle()
+    cfg = syn.STACK_CFG
+    m = orc.make_model(cfg, syn.stack_weights(cfg, seed=4))
+    init = syn.stack_state(cfg, 1, PREFILL + 64, prefill=PREFILL, seed=4)
+    st = {"S": init["S"].astype(np.float64), "tail": init["tail"].astype(np.float64), "kv": init["kv"],
+          "pos": init["pos"]}
+    tok = syn.stack_tokens(cfg, 1, 1, seed=4)
+    t0 = time.perf_counter()
+    for _ in range(tokens):
+        tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{tokens} greedy tokens of the full stack, single-threaded C oracle (fp64)"}
+
+
+# --------------------------------------------------------------------- GPU --
+
+def run_gpu(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import hgd_synth as syn
+    import hybrid_gated_delta_b200 as hgd
+
+    cfg = syn.STACK_CFG
+    B = 1
+    Lmax = ((PREFILL + args.warmup + args.steps + 2 + 63) // 64) * 64
+    model = hgd.Model(cfg, syn.stack_weights(cfg, seed=4))
+    init = syn.stack_state(cfg, B, Lmax, prefill=PREFILL, seed=4 + rank)
+    state = hgd.State(model, B, 1, Lmax, init)
+    stream = torch.cuda.Stream()
+    tok = torch.from_numpy(syn.stack_tokens(cfg, B, 1, seed=4 + rank)).cuda()
+    argmax = torch.zeros(B, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok_buf = argmax.view(B, 1)  # greedy: each step reads the previous step's argmax
+    tok_buf.copy_(tok)
+    launches = model.launches(B, 1)
+
+    dec = hgd.DecodeGraph(model, state, tok_buf, argmax, status, stream=stream)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        dec.replay()
+    stream.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            dec.replay_layers()
+            ev[i][1].record(stream)
+            dec.replay_head()
+            ev[i][2].record(stream)
+        t_end.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    head_ms = [a.elapsed_time(b) for _, a, b in ev]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    assert int(status.item()) == 0, hgd.status_string(int(status.item()))
+
+    # end to end through the public API: host token in (pinned H2D), host argmax out
+    e2e_steps = max(8, min(args.steps, 64))
+    h_tok = torch.empty((B, 1), dtype=torch.int32).pin_memory()
+    h_out = torch.empty((B,), dtype=torch.int32).pin_memory()
+    h_tok.copy_(argmax.view(B, 1).cpu())
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        dec.step_host(h_tok, h_out)
+        h_tok.view(-1).copy_(h_out)
+    e2e_s = time.perf_counter() - t0
+    e2e_val = world * B * e2e_steps / e2e_s  # every rank runs the same loop
+    dec.close()
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms_step = elapsed_ms / args.steps
+    value = world * B * args.steps / (elapsed_ms / 1000.0)
+    L_avg = PREFILL + args.warmup + (args.steps + 1) / 2.0
+    ab = algorithmic_bytes(cfg, L_avg)
+    peaks = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", 6650.0))
+    head_avg_ms = statistics.mean(head_ms)
+    head_gbs = ab["head"] / (head_avg_ms * 1e-3) / 1e9
+    step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
+    prof = {}
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            prof = json.load(f)
+    except OSError:
+        pass
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch": 1, "kv_context": PREFILL, "decode_tokens": args.steps,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: 1.5 GB of weights streamed per step (L2 126 MB)"},
+        "hbm_gbs": step_gbs,
+        "frac_of_8tbs": step_gbs / 8000.0,
+        "roofline": {"kernel": "LM head (final RMSNorm + tied 248320x1024 GEMV + per-CTA argmax)",
+                     "bound": "hbm", "achieved": head_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": head_gbs / peak, "peak_source": "measured" if "_fallback" not in peaks else "fallback",
+                     "traffic": prof.get("lm_head_bytes_per_launch"),
+                     "algorithmic_bytes": ab["head"], "avg_launch_ms": head_avg_ms},
+        "step_roofline": {"bound": "hbm", "achieved": step_gbs, "peak": peak, "unit": "GB/s",
+                          "frac": step_gbs / peak, "algorithmic_bytes": ab["total"],
+                          "traffic": prof.get("step_bytes")},
+        "gpu_launches": launches * args.steps,
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": 4 * B, "d2h_bytes_per_step": 4 * B,
+                "steps": e2e_steps, "how": "per token: pinned H2D of the token, graph replay of the step, "
+                                          "D2H of the argmax, host synchronisation"},
+    }
+    if clk:
+        out["clocks"] = clk
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_sample(tokens=args.cpu_tokens)
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=4)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

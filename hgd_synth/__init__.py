@@ -13,7 +13,20 @@ Distribution readings (the configurations write N(0, s)):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
+
+_CHUNK = 1 << 22
+_POOL: ThreadPoolExecutor | None = None
+
+
+def _pool() -> ThreadPoolExecutor:
+    global _POOL
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1))
+    return _POOL
 
 # ------------------------------------------------------------------ helpers --
 
@@ -24,13 +37,38 @@ def rng(seed: int) -> np.random.Generator:
 
 def to_bf16(a: np.ndarray) -> np.ndarray:
     """float32 -> bf16 bit pattern (nearest-even).  Input generation only."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
-    lsb = (u >> 16) & 1
-    r = ((u.astype(np.uint64) + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32)
+    r = ((u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) >> np.uint32(16)).astype(np.uint16)
     nan = np.isnan(a)
     if nan.any():
         r[nan] = 0x7FC0
     return r
+
+
+def keyed_normal_bf16(key: tuple, shape, std: float, mean: float = 0.0) -> np.ndarray:
+    """N(mean, std) bf16 draws for a large tensor, generated in fixed 4M-element
+    chunks, chunk i from PCG64(SeedSequence(key + (i,))): the values depend on the
+    key only, never on the number of threads that fill them."""
+    n = int(np.prod(shape))
+    out = np.empty(n, np.uint16)
+
+    def fill(i):
+        lo, hi = i * _CHUNK, min(n, (i + 1) * _CHUNK)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(list(key) + [i])))
+        a = g.standard_normal(size=hi - lo, dtype=np.float32)
+        if std != 1.0:
+            a *= np.float32(std)
+        if mean != 0.0:
+            a += np.float32(mean)
+        out[lo:hi] = to_bf16(a)
+
+    nch = (n + _CHUNK - 1) // _CHUNK
+    if nch <= 1:
+        fill(0) if n else None
+    else:
+        list(_pool().map(fill, range(nch)))
+    return out.reshape(shape)
 
 
 def from_bf16(h: np.ndarray) -> np.ndarray:
@@ -148,34 +186,42 @@ def layer_counts(cfg: dict) -> tuple[int, int]:
     return cfg["n_layers"] - n_attn, n_attn
 
 
+_NAMES = ("in_norm", "w_in", "conv_w", "A_log", "dt_bias", "gnorm_w", "w_out", "post_norm", "w_gate",
+          "w_up", "w_down")
+
+
 def stack_weights(cfg: dict, seed: int = 4, std: float = 0.02) -> dict:
     """Random-init bf16 weights N(0, std) with gains 1 + N(0, std).
     Returns {"embed", "final_norm", "layers": [dict per layer]}; the per-layer keys
     match the oracle's layer struct (in_norm, w_in, conv_w, A_log, dt_bias, gnorm_w,
-    w_out, post_norm, w_gate, w_up, w_down)."""
+    w_out, post_norm, w_gate, w_up, w_down).  Tensor (layer l, name) is drawn from
+    the key (seed, l, name index); the embedding and final norm use l = -1."""
     D, V, H = cfg["hidden"], cfg["vocab"], cfg["gdn_heads"]
     dk, dv, kc = cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
     nq, nkv, hd, I = cfg["attn_q_heads"], cfg["attn_kv_heads"], cfg["attn_head_dim"], cfg["mlp_inter"]
     Cc = 2 * H * dk + H * dv
-    g = rng(seed)
-    w = {"embed": normal_bf16(g, (V, D), std), "final_norm": normal_bf16(g, (D,), std, 1.0),
-         "layers": []}
+
+    def w_(l, name, shape, mean=0.0):
+        return keyed_normal_bf16((seed, l + 1, _NAMES.index(name) if name in _NAMES else 99 + len(name)),
+                                 shape, std, mean)
+
+    w = {"embed": w_(-1, "embed", (V, D)), "final_norm": w_(-1, "final_norm", (D,), 1.0), "layers": []}
     for l in range(cfg["n_layers"]):
-        lw = {"in_norm": normal_bf16(g, (D,), std, 1.0)}
+        lw = {"in_norm": w_(l, "in_norm", (D,), 1.0)}
         if not is_attn(cfg, l):
-            lw["w_in"] = normal_bf16(g, (Cc + H * dv + 2 * H, D), std)
-            lw["conv_w"] = normal_bf16(g, (Cc, kc), std)
-            lw["A_log"] = normal_bf16(g, (H,), std)
-            lw["dt_bias"] = normal_bf16(g, (H,), std)
-            lw["gnorm_w"] = normal_bf16(g, (dv,), std, 1.0)
-            lw["w_out"] = normal_bf16(g, (D, H * dv), std)
+            lw["w_in"] = w_(l, "w_in", (Cc + H * dv + 2 * H, D))
+            lw["conv_w"] = w_(l, "conv_w", (Cc, kc))
+            lw["A_log"] = w_(l, "A_log", (H,))
+            lw["dt_bias"] = w_(l, "dt_bias", (H,))
+            lw["gnorm_w"] = w_(l, "gnorm_w", (dv,), 1.0)
+            lw["w_out"] = w_(l, "w_out", (D, H * dv))
         else:
-            lw["w_in"] = normal_bf16(g, (2 * nq * hd + 2 * nkv * hd, D), std)
-            lw["w_out"] = normal_bf16(g, (D, nq * hd), std)
-        lw["post_norm"] = normal_bf16(g, (D,), std, 1.0)
-        lw["w_gate"] = normal_bf16(g, (I, D), std)
-        lw["w_up"] = normal_bf16(g, (I, D), std)
-        lw["w_down"] = normal_bf16(g, (D, I), std)
+            lw["w_in"] = w_(l, "w_in", (2 * nq * hd + 2 * nkv * hd, D))
+            lw["w_out"] = w_(l, "w_out", (D, nq * hd))
+        lw["post_norm"] = w_(l, "post_norm", (D,), 1.0)
+        lw["w_gate"] = w_(l, "w_gate", (I, D))
+        lw["w_up"] = w_(l, "w_up", (I, D))
+        lw["w_down"] = w_(l, "w_down", (D, I))
         w["layers"].append(lw)
     return w
 
@@ -191,7 +237,7 @@ def stack_state(cfg: dict, B: int, Lmax: int, prefill: int = 512, seed: int = 4)
     g = rng(seed * 31 + 17 + B)
     kv = np.zeros((n_attn, 2, B, nkv, Lmax, hd), np.uint16)
     if prefill > 0:
-        kv[..., :prefill, :] = normal_bf16(g, (n_attn, 2, B, nkv, prefill, hd), 1.0)
+        kv[..., :prefill, :] = keyed_normal_bf16((seed, 7001, B), (n_attn, 2, B, nkv, prefill, hd), 1.0)
     return dict(
         S=normal_f32(g, (n_gdn, B, H, dv, dk), 0.1),
         tail=normal_f32(g, (n_gdn, B, kc - 1, Cc), 1.0),

@@ -33,7 +33,7 @@ W_EMBED, W_FINAL_NORM = 100, 101
 LAYER_TENSORS = {"in_norm": W_IN_NORM, "w_in": W_IN, "conv_w": W_CONV, "A_log": W_A_LOG,
                  "dt_bias": W_DT_BIAS, "gnorm_w": W_GNORM, "w_out": W_OUT, "post_norm": W_POST_NORM,
                  "w_gate": W_GATE, "w_up": W_UP, "w_down": W_DOWN}
-S_GDN, S_CONV, S_KV, S_POS = range(4)
+S_GDN, S_CONV, S_KV, S_POS, S_RESID = range(5)
 
 
 class HgdError(RuntimeError):
@@ -64,17 +64,21 @@ _p, _i, _i64, _sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
 _SIGS = {
     "hgd_status_string": ([_i], C.c_char_p),
     "hgd_version": ([], _i),
-    "hgd_gemv_bf16": ([_p, _p, _p, _i, _i, _i, _i, _p], _i),
-    "hgd_gemv_swiglu_bf16": ([_p, _p, _p, _p, _i, _i, _i, _p], _i),
+    "hgd_gemv_bf16": ([_p, _p, _p, _i, _i, _i, _i, _p, _sz, _p], _i),
+    "hgd_gemv_workspace_bytes": ([_i, _i, _i, _i, C.POINTER(_sz)], _i),
+    "hgd_gemv_swiglu_bf16": ([_p, _p, _p, _p, _i, _i, _i, _p, _sz, _p], _i),
     "hgd_conv1d_tail_update": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
     "hgd_model_arena_bytes": ([C.POINTER(Config), C.POINTER(_sz)], _i),
     "hgd_model_tensor": ([C.POINTER(Config), _i, _i, C.POINTER(_sz), C.POINTER(_sz)], _i),
     "hgd_model_init": ([C.POINTER(_Model), C.POINTER(Config), _p, _sz], _i),
+    "hgd_model_load_tensor": ([C.POINTER(Config), _p, _sz, _i, _i, _p, _p], _i),
     "hgd_state_arena_bytes": ([C.POINTER(Config), _i, _i, _i, C.POINTER(_sz)], _i),
     "hgd_state_tensor": ([C.POINTER(Config), _i, _i, _i, _i, C.POINTER(_sz), C.POINTER(_sz)], _i),
     "hgd_state_init": ([C.POINTER(_State), C.POINTER(_Model), _i, _i, _i, _p, _sz], _i),
     "hgd_decode_layer_stack": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _p, _p, _p, _p, _p], _i),
+    "hgd_decode_layer_stack_range": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _i, _i, _i, _p, _p, _p,
+                                      _p, _p, _p], _i),
     "hgd_decode_layer_stack_launches": ([C.POINTER(_Model), _i, _i], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
@@ -132,7 +136,20 @@ def _need(t, dtype, name):
 
 # -------------------------------------------------------------- entry points
 
-def gemv_bf16(W, x, y=None, y_is_fp32=True, stream=None):
+def gemv_workspace_bytes(M: int, N: int, K: int, swiglu: bool = False) -> int:
+    n = C.c_size_t()
+    _check("hgd_gemv_workspace_bytes", _lib.hgd_gemv_workspace_bytes(M, N, K, int(swiglu), C.byref(n)))
+    return n.value
+
+
+def make_workspace(M: int, N: int, K: int, swiglu: bool = False, device="cuda"):
+    """A zero-filled split-K workspace for GEMVs of this shape (None if unused)."""
+    torch = _torch()
+    n = gemv_workspace_bytes(M, N, K, swiglu)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device) if n else None
+
+
+def gemv_bf16(W, x, y=None, y_is_fp32=True, workspace=None, stream=None):
     """y[M,N] = x[M,K] . W[N,K]^T (bf16 in, fp32 accumulate)."""
     torch = _torch()
     _need(W, torch.bfloat16, "W")
@@ -141,12 +158,13 @@ def gemv_bf16(W, x, y=None, y_is_fp32=True, stream=None):
     M = x.shape[0]
     if y is None:
         y = torch.empty((M, N), dtype=torch.float32 if y_is_fp32 else torch.bfloat16, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("hgd_gemv_bf16", _lib.hgd_gemv_bf16(_ptr(W), _ptr(x), _ptr(y), int(y.dtype == torch.float32),
-                                                M, N, K, _stream(stream)))
+                                                M, N, K, _ptr(workspace), ws_bytes, _stream(stream)))
     return y
 
 
-def gemv_swiglu_bf16(W_gate, W_up, x, h=None, stream=None):
+def gemv_swiglu_bf16(W_gate, W_up, x, h=None, workspace=None, stream=None):
     """h[M,I] = bf16(silu(x W_gate^T) * (x W_up^T))."""
     torch = _torch()
     for t, n in ((W_gate, "W_gate"), (W_up, "W_up"), (x, "x")):
@@ -155,8 +173,10 @@ def gemv_swiglu_bf16(W_gate, W_up, x, h=None, stream=None):
     M = x.shape[0]
     if h is None:
         h = torch.empty((M, I), dtype=torch.bfloat16, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("hgd_gemv_swiglu_bf16", _lib.hgd_gemv_swiglu_bf16(_ptr(W_gate), _ptr(W_up), _ptr(x), _ptr(h),
-                                                              M, I, K, _stream(stream)))
+                                                              M, I, K, _ptr(workspace), ws_bytes,
+                                                              _stream(stream)))
     return h
 
 
@@ -225,14 +245,18 @@ class Model:
         base = self.arena.data_ptr()
         pad = (-base) % 256
         self.arena_u8 = self.arena.view(torch.uint8)[pad:pad + nbytes.value]
+        stream = torch.cuda.current_stream()
         for name, tid, layer in self._tensors(weights):
             off, n = self.tensor_offset(layer, tid)
             arr = weights[name] if layer < 0 else weights["layers"][layer][name]
             arr = np.ascontiguousarray(arr, dtype=np.uint16).reshape(-1)
             if arr.size != n:
                 raise ValueError(f"layer {layer} {name}: {arr.size} elements, layout expects {n}")
-            src = torch.from_numpy(arr.view(np.int16))
-            self.arena_u8[off:off + 2 * n].view(torch.int16).copy_(src, non_blocking=False)
+            src = torch.from_numpy(arr.view(np.int16)).to(device)
+            _check("hgd_model_load_tensor", _lib.hgd_model_load_tensor(
+                C.byref(self.cfg), self.arena_u8.data_ptr(), nbytes.value, layer, tid, src.data_ptr(),
+                stream.cuda_stream))
+            stream.synchronize()
         self.m = _Model()
         _check("hgd_model_init", _lib.hgd_model_init(C.byref(self.m), C.byref(self.cfg),
                                                      self.arena_u8.data_ptr(), nbytes.value))
@@ -281,6 +305,7 @@ class State:
         self.conv = self._view(S_CONV, torch.float32, (n_gdn, B, kc - 1, Cc))
         self.kv = self._view(S_KV, torch.bfloat16, (n_attn, 2, B, nkv, Lmax, hd))
         self.pos = self._view(S_POS, torch.int32, (B,))
+        self.resid = self._view(S_RESID, torch.bfloat16, (B * Tmax, cfg["hidden"]))
         if init is not None:
             self.load(init)
 
@@ -327,3 +352,68 @@ def decode_layer_stack(model: Model, state: State, tokens, T: int, logits=None, 
         C.byref(model.m), C.byref(state.st), _ptr(tokens), T, _ptr(logits), _ptr(argmax), _ptr(S_rec),
         _ptr(tail_rec), _ptr(status), _stream(stream)))
     return argmax
+
+
+def decode_layer_stack_range(model: Model, state: State, tokens, T: int, layer_begin: int, layer_end: int,
+                             run_head: bool, logits=None, argmax=None, S_rec=None, tail_rec=None, status=None,
+                             stream=None):
+    """Layers [layer_begin, layer_end) (and the head if run_head) of one decode call;
+    the residual rows live in state.resid between ranges."""
+    _check("hgd_decode_layer_stack_range", _lib.hgd_decode_layer_stack_range(
+        C.byref(model.m), C.byref(state.st), _ptr(tokens), T, layer_begin, layer_end, int(run_head),
+        _ptr(logits), _ptr(argmax), _ptr(S_rec), _ptr(tail_rec), _ptr(status), _stream(stream)))
+    return argmax
+
+
+class DecodeGraph:
+    """A one-row greedy decode step captured as two CUDA graphs (all layers; final
+    norm + LM head + argmax) and replayed on `stream`.  `tokens` [B,1] is read at
+    the start of a step and `argmax` [B] written at its end, so passing
+    tokens = argmax.view(B, 1) feeds each step's argmax to the next step on the
+    device.  Capturing runs the step once eagerly first (to load the kernels) on
+    a copy of the state, which is then restored."""
+
+    def __init__(self, model: Model, state: State, tokens, argmax, status=None, stream=None):
+        torch = _torch()
+        self.model, self.state, self.tokens, self.argmax, self.status = model, state, tokens, argmax, status
+        self.stream = stream or torch.cuda.Stream()
+        snap = state.snapshot()
+        tok0 = tokens.clone()
+        with torch.cuda.stream(self.stream):
+            decode_layer_stack(model, state, tokens, 1, argmax=argmax, status=status, stream=self.stream)
+        self.stream.synchronize()
+        state.restore(snap)
+        tokens.copy_(tok0)
+        torch.cuda.synchronize()
+        self.g_layers = torch.cuda.CUDAGraph()
+        self.g_head = torch.cuda.CUDAGraph()
+        L = model.cfg_dict["n_layers"]
+        with torch.cuda.graph(self.g_layers, stream=self.stream):
+            decode_layer_stack_range(model, state, tokens, 1, 0, L, False, status=status)
+        with torch.cuda.graph(self.g_head, stream=self.stream):
+            decode_layer_stack_range(model, state, None, 1, L, L, True, argmax=argmax, status=status)
+        torch.cuda.synchronize()
+
+    def replay_layers(self):
+        self.g_layers.replay()
+
+    def replay_head(self):
+        self.g_head.replay()
+
+    def replay(self):
+        self.g_layers.replay()
+        self.g_head.replay()
+
+    def step_host(self, h_tok, h_out):
+        """One step from a pinned host token tensor to a pinned host argmax tensor."""
+        torch = _torch()
+        with torch.cuda.stream(self.stream):
+            self.tokens.copy_(h_tok, non_blocking=True)
+            self.g_layers.replay()
+            self.g_head.replay()
+            h_out.copy_(self.argmax, non_blocking=True)
+        self.stream.synchronize()
+
+    def close(self):
+        self.g_layers.reset()
+        self.g_head.reset()

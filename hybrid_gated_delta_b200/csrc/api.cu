@@ -67,76 +67,113 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 }
 
 // ------------------------------------------------------------- GEMV plans
+// Row blocks below this count use split slabs (partials through the workspace)
+// when a workspace is given.  The arithmetic of every output is the same in both
+// modes, so the threshold only moves work between warps.
+constexpr int kSplitMaxRowblk = 2048;
+
 struct GemvPlan {
-    int nt, mchunk, nstage, stage_bytes, x_bytes, kb, nkb;
+    int nt, mchunk, x_bytes;
     size_t smem;
 };
 
-size_t gv_fixed_bytes(int mp) {
-    return (size_t)(GV_WARPS + 1) * mp * GV_PITCH * 4 + 8 + 2 * 8 * GV_MAX_STAGES + 16;
-}
+size_t gv_fixed_bytes(int mp) { return (size_t)GV_CW * mp * 8 + (size_t)GV_CW * GV_ROWS * mp * 4 + 16; }
 
 bool plan_gemv(int M, int K, GemvPlan* pl) {
-    gv_kblocks(K, &pl->kb, &pl->nkb);
-    pl->stage_bytes = GV_ROWS * (pl->kb + GV_PAD) * 2;
     const int want = (M + 7) / 8;
     int nt = want <= 1 ? 1 : (want <= 2 ? 2 : 4);
     for (; nt >= 1; nt >>= 1) {
         const int mp = 8 * nt;
         const int xb = gv_align16(mp * (K + GV_PAD) * 2);
-        const long avail = (long)GV_SMEM_LIMIT - xb - (long)gv_fixed_bytes(mp);
-        const long ns = avail / pl->stage_bytes;
-        if (ns >= 2) {
+        const size_t smem = xb + gv_fixed_bytes(mp);
+        if (smem <= (size_t)GV_SMEM_LIMIT) {
             pl->nt = nt;
             pl->mchunk = mp;
-            pl->nstage = (int)std::min<long>(ns, GV_MAX_STAGES);
             pl->x_bytes = xb;
-            pl->smem = (size_t)pl->nstage * pl->stage_bytes + xb + gv_fixed_bytes(mp);
+            pl->smem = smem;
             return true;
         }
     }
     return false;
 }
 
+int rowblocks_of(int N, bool swiglu) { return swiglu ? (N + 7) / 8 : (N + GV_ROWS - 1) / GV_ROWS; }
+
+// Workspace layout: the row-block counters at a fixed place (so that every GEMV
+// sharing a workspace finds them at zero), then the slab partials.
+constexpr size_t kWsCounterBytes = (size_t)kSplitMaxRowblk * 4;
+
+// Workspace bytes a GEMV of this shape uses in split mode (0 if it never splits).
+size_t gemv_ws_bytes(int M, int N, int K, bool swiglu) {
+    GemvPlan pl;
+    if (!plan_gemv(M, K, &pl)) return 0;
+    const int nrb = rowblocks_of(N, swiglu);
+    if (nrb >= kSplitMaxRowblk) return 0;
+    return kWsCounterBytes + (size_t)nrb * gv_slabs(K) * GV_ROWS * pl.mchunk * 4;
+}
+
+// CTAs of one GEMV launch: one per work item up to as many as can be resident
+// at once (the launch is one wave).
 template <int NT, int PRO, int EPI>
-cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cudaStream_t s) {
+cudaError_t launch_gemv_t(GemvParams p, size_t smem, int sms, cudaStream_t s, int* grid_out) {
     auto kern = k_gemv<NT, PRO, EPI>;
     static int attr_done[64];
+    static int occ_cache[64][4];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+    const bool cache_ok = dev >= 0 && dev < 64;
+    if (!cache_ok || !attr_done[dev]) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+        if (cache_ok) attr_done[dev] = 1;
     }
+    // occupancy for this shared-memory size (bucketed by 16 KB, cached)
+    const int bucket = std::min(3, (int)(smem / (56 * 1024)));
+    int occ = cache_ok ? occ_cache[dev][bucket] : 0;
+    if (occ == 0) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, GV_THREADS, smem);
+        if (e != cudaSuccess) return e;
+        occ = std::max(1, occ);
+        if (cache_ok) occ_cache[dev][bucket] = occ;
+    }
+    // items go to CTAs first (slot = warp * grid + cta), so a GEMV with few items
+    // still spreads over every SM
+    const int grid = std::max(1, std::min(p.n_items, occ * sms));
+    if (grid_out) *grid_out = grid;
     return launch_pdl(kern, dim3(grid), dim3(GV_THREADS), smem, s, p);
 }
 
 template <int PRO, int EPI>
-cudaError_t launch_gemv_nt(int nt, const GemvParams& p, int grid, size_t smem, cudaStream_t s) {
+cudaError_t launch_gemv_nt(int nt, const GemvParams& p, size_t smem, int sms, cudaStream_t s, int* grid_out) {
     switch (nt) {
-        case 1: return launch_gemv_t<1, PRO, EPI>(p, grid, smem, s);
-        case 2: return launch_gemv_t<2, PRO, EPI>(p, grid, smem, s);
-        default: return launch_gemv_t<4, PRO, EPI>(p, grid, smem, s);
+        case 1: return launch_gemv_t<1, PRO, EPI>(p, smem, sms, s, grid_out);
+        case 2: return launch_gemv_t<2, PRO, EPI>(p, smem, sms, s, grid_out);
+        default: return launch_gemv_t<4, PRO, EPI>(p, smem, sms, s, grid_out);
     }
 }
 
-// Launch a GEMV over all M rows, in chunks of the plan's M tile.  `adv` moves
-// the row-indexed pointers of the params to a chunk's first row.
+// Launch a GEMV over all M rows, in chunks of the plan's M tile (each chunk
+// re-streams the weights; only very large M * K needs more than one).
 template <int PRO, int EPI>
-int run_gemv(GemvParams p, int M, int sms, cudaStream_t s, int* launches) {
+int run_gemv(GemvParams p, int M, int sms, void* ws, size_t ws_bytes, cudaStream_t s, int* grid_out = nullptr) {
     GemvPlan pl;
     if (!plan_gemv(M, p.K, &pl)) return HGD_ERR_UNSUPPORTED_SHAPE;
-    p.kb = pl.kb;
-    p.nkb = pl.nkb;
-    p.nstage = pl.nstage;
-    p.stage_bytes = pl.stage_bytes;
+    p.nks = gv_slabs(p.K);
+    p.n_rowblk = rowblocks_of(p.N, EPI == EPI_SWIGLU);
     p.x_bytes = pl.x_bytes;
-    p.n_rowblk = (EPI == EPI_SWIGLU) ? (p.N + 7) / 8 : (p.N + GV_ROWS - 1) / GV_ROWS;
-    const int grid = std::min(p.n_rowblk, sms);
+    const size_t need = gemv_ws_bytes(M, p.N, p.K, EPI == EPI_SWIGLU);
+    p.split = (EPI != EPI_ARGMAX && ws && need && ws_bytes >= need) ? 1 : 0;
+    if (p.split) {
+        p.ws_mp = pl.mchunk;
+        p.ws_cnt = static_cast<int32_t*>(ws);
+        p.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kWsCounterBytes);
+    }
+    p.n_items = p.n_rowblk * (p.split ? p.nks : 1);
+    int grid = 0;
     for (int m0 = 0; m0 < M; m0 += pl.mchunk) {
         GemvParams q = p;
         q.M = std::min(pl.mchunk, M - m0);
+        q.m0 = m0;
         if (q.x) q.x += m0 * q.x_ld;
         if (q.tokens) q.tokens += m0;
         if (q.resid_out) q.resid_out += m0 * q.resid_out_ld;
@@ -144,19 +181,20 @@ int run_gemv(GemvParams p, int M, int sms, cudaStream_t s, int* launches) {
         if (q.z) q.z += m0 * q.z_ld;
         if (q.resid) q.resid += m0 * q.resid_ld;
         if (q.y) {
-            const int es = (EPI == EPI_F32) ? 4 : 2;
+            const int es = (EPI == EPI_F32 || EPI == EPI_QKV_CONV) ? 4 : 2;
             q.y = reinterpret_cast<uint8_t*>(q.y) + (size_t)m0 * q.y_ld * es;
         }
         if (q.logits) q.logits += m0 * q.logits_ld;
-        if (q.best_v) { q.best_v += (size_t)m0 * grid; q.best_i += (size_t)m0 * grid; }
-        cudaError_t e = launch_gemv_nt<PRO, EPI>(pl.nt, q, grid, pl.smem, s);
+        // ARGMAX partials are [M][grid]; the grid is the same for every chunk
+        if (q.best_v && m0) { q.best_v += (size_t)m0 * grid; q.best_i += (size_t)m0 * grid; }
+        // (conv tails of streams in this chunk are updated in place; the next
+        // chunk continues from them in stream order)
+        cudaError_t e = launch_gemv_nt<PRO, EPI>(pl.nt, q, pl.smem, sms, s, &grid);
         if (e != cudaSuccess) return launch_status(e);
-        if (launches) ++*launches;
     }
+    if (grid_out) *grid_out = grid;
     return HGD_OK;
 }
-
-int gemv_grid(int N, int rows_per_blk, int sms) { return std::min((N + rows_per_blk - 1) / rows_per_blk, sms); }
 
 int gemv_chunks(int M, int K) {
     GemvPlan pl;
@@ -222,30 +260,76 @@ size_t weight_numel(const Dims& d, const hgd_config* c, int layer, int t) {
     }
 }
 
+// How a tensor is stored: 0 plain, 1 packed matrix, 2 / 3 gate / up half of the
+// packed SwiGLU region (which the gate tensor owns).  rows x cols is its logical
+// shape for the packed kinds.
+struct WeightKind { int kind; int64_t rows, cols; };
+
+WeightKind weight_kind(const Dims& d, const hgd_config* c, int layer, int t) {
+    if (layer < 0) {
+        if (t == HGD_W_EMBED) return {1, d.V, d.D};
+        return {0, 0, 0};
+    }
+    const bool att = is_attn_layer(c, layer);
+    switch (t) {
+        case HGD_W_IN: return {1, att ? d.attn_out : d.gdn_out, d.D};
+        case HGD_W_OUT: return {1, d.D, att ? (int64_t)d.nq * d.hd : (int64_t)d.H * d.dv};
+        case HGD_W_GATE: return {2, d.I, d.D};
+        case HGD_W_UP: return {3, d.I, d.D};
+        case HGD_W_DOWN: return {1, d.D, d.I};
+        default: return {0, 0, 0};
+    }
+}
+
+// Bytes of the storage a tensor owns in the arena.
+size_t weight_bytes(const Dims& d, const hgd_config* c, int layer, int t) {
+    const WeightKind k = weight_kind(d, c, layer, t);
+    switch (k.kind) {
+        case 1: return (size_t)((k.rows + 15) / 16) * 16 * k.cols * 2;
+        case 2: return (size_t)((k.rows + 7) / 8) * 16 * k.cols * 2;
+        case 3: return 0;
+        default: return weight_numel(d, c, layer, t) * 2;
+    }
+}
+
 // Walk the arena in order; returns the total and, if (layer, t) matches, its offset.
 size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_t, size_t* off) {
     size_t pos = 0;
     const int glob[2] = {HGD_W_EMBED, HGD_W_FINAL_NORM};
     for (int g = 0; g < 2; ++g) {
         if (want_layer == -1 && want_t == glob[g] && off) *off = pos;
-        pos += al256(weight_numel(d, c, -1, glob[g]) * 2);
+        pos += al256(weight_bytes(d, c, -1, glob[g]));
     }
-    for (int l = 0; l < d.L; ++l)
+    for (int l = 0; l < d.L; ++l) {
+        size_t gate_off = 0;
         for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) {
-            const size_t n = weight_numel(d, c, l, t);
-            if (l == want_layer && t == want_t && off) *off = pos;
-            pos += al256(n * 2);
+            if (t == HGD_W_GATE) gate_off = pos;
+            if (l == want_layer && t == want_t && off) *off = (t == HGD_W_UP) ? gate_off : pos;
+            pos += al256(weight_bytes(d, c, l, t));
         }
+    }
     return pos;
 }
 
 enum ScratchIdx {
     SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
-    SC_BESTV, SC_BESTI, SC_END, SC_COUNT
+    SC_BESTV, SC_BESTI, SC_WS, SC_END, SC_COUNT
 };
-constexpr int kBestG = 1024;  // max CTAs of the LM-head launch
+constexpr int kBestG = 4096;  // max CTAs of the LM-head launch
 
 int max_chunks_of(int Lmax) { return (Lmax + ATTN_CHUNK - 1) / ATTN_CHUNK; }
+
+// Split-K workspace of the stack: the largest any of its GEMVs uses at M rows.
+size_t stack_ws_bytes(const Dims& d, int M) {
+    size_t w = 0;
+    w = std::max(w, gemv_ws_bytes(M, (int)d.gdn_out, d.D, false));
+    w = std::max(w, gemv_ws_bytes(M, (int)d.attn_out, d.D, false));
+    w = std::max(w, gemv_ws_bytes(M, d.D, d.H * d.dv, false));
+    w = std::max(w, gemv_ws_bytes(M, d.D, d.nq * d.hd, false));
+    w = std::max(w, gemv_ws_bytes(M, d.I, d.D, true));
+    w = std::max(w, gemv_ws_bytes(M, d.D, d.I, false));
+    return w;
+}
 
 void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     const int64_t M = (int64_t)B * Tmax;
@@ -263,6 +347,7 @@ void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     sz[SC_MLP] = (size_t)M * d.I * 2;
     sz[SC_BESTV] = (size_t)M * kBestG * 4;
     sz[SC_BESTI] = (size_t)M * kBestG * 4;
+    sz[SC_WS] = stack_ws_bytes(d, (int)M);
     size_t pos = 0;
     for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
     off[SC_END] = pos;
@@ -297,31 +382,40 @@ const char* hgd_status_string(int s) {
 
 int hgd_version(void) { return 100; }
 
+int hgd_gemv_workspace_bytes(int M, int N, int K, int swiglu, size_t* bytes) {
+    if (!bytes || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (K % 32 != 0 || K > 65536) return HGD_ERR_UNSUPPORTED_SHAPE;
+    *bytes = gemv_ws_bytes(M, N, K, swiglu != 0);
+    return HGD_OK;
+}
+
 int hgd_gemv_bf16(const uint16_t* W, const uint16_t* x, void* y, int y_is_fp32, int M, int N, int K,
-                  hgd_stream_t stream) {
+                  void* workspace, size_t workspace_bytes, hgd_stream_t stream) {
     if (!W || !x || !y || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
     if (K % 32 != 0 || K > 65536) return HGD_ERR_UNSUPPORTED_SHAPE;
-    if (!al16(W) || !al16(x) || !al16(y)) return HGD_ERR_MISALIGNED;
+    if (!al16(W) || !al16(x) || !al16(y) || (workspace && !al16(workspace))) return HGD_ERR_MISALIGNED;
     DevInfo di;
     int rc = device_info(&di);
     if (rc) return rc;
     GemvParams p = {};
     p.W = W; p.N = N; p.K = K; p.x = x; p.x_ld = K; p.y = y; p.y_ld = N;
-    if (y_is_fp32) return run_gemv<PRO_COPY, EPI_F32>(p, M, di.sms, (cudaStream_t)stream, nullptr);
-    return run_gemv<PRO_COPY, EPI_BF16>(p, M, di.sms, (cudaStream_t)stream, nullptr);
+    if (y_is_fp32)
+        return run_gemv<PRO_COPY, EPI_F32>(p, M, di.sms, workspace, workspace_bytes, (cudaStream_t)stream);
+    return run_gemv<PRO_COPY, EPI_BF16>(p, M, di.sms, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 int hgd_gemv_swiglu_bf16(const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* x, uint16_t* h,
-                         int M, int I, int K, hgd_stream_t stream) {
+                         int M, int I, int K, void* workspace, size_t workspace_bytes, hgd_stream_t stream) {
     if (!W_gate || !W_up || !x || !h || M < 1 || I < 1 || K < 1) return HGD_ERR_INVALID_ARG;
     if (K % 32 != 0 || K > 65536) return HGD_ERR_UNSUPPORTED_SHAPE;
-    if (!al16(W_gate) || !al16(W_up) || !al16(x) || !al16(h)) return HGD_ERR_MISALIGNED;
+    if (!al16(W_gate) || !al16(W_up) || !al16(x) || !al16(h) || (workspace && !al16(workspace)))
+        return HGD_ERR_MISALIGNED;
     DevInfo di;
     int rc = device_info(&di);
     if (rc) return rc;
     GemvParams p = {};
     p.W = W_gate; p.W2 = W_up; p.N = I; p.K = K; p.x = x; p.x_ld = K; p.y = h; p.y_ld = I;
-    return run_gemv<PRO_COPY, EPI_SWIGLU>(p, M, di.sms, (cudaStream_t)stream, nullptr);
+    return run_gemv<PRO_COPY, EPI_SWIGLU>(p, M, di.sms, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 int hgd_conv1d_tail_update(const float* x, float* tail, const uint16_t* w, float* y, float* tail_rec,
@@ -392,6 +486,42 @@ int hgd_model_tensor(const hgd_config* cfg, int layer, int tensor, size_t* offse
     return HGD_OK;
 }
 
+int hgd_model_load_tensor(const hgd_config* cfg, void* arena, size_t arena_bytes, int layer, int tensor,
+                          const uint16_t* src, hgd_stream_t stream) {
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if (!arena || !src) return HGD_ERR_INVALID_ARG;
+    if (layer < -1 || layer >= d.L) return HGD_ERR_INVALID_ARG;
+    if (layer == -1 && tensor != HGD_W_EMBED && tensor != HGD_W_FINAL_NORM) return HGD_ERR_INVALID_ARG;
+    if (layer >= 0 && (tensor < 0 || tensor >= HGD_W_LAYER_COUNT)) return HGD_ERR_INVALID_ARG;
+    const size_t n = weight_numel(d, cfg, layer, tensor);
+    if (n == 0) return HGD_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(arena) & 255u) || !al16(src)) return HGD_ERR_MISALIGNED;
+    const size_t need = weight_walk(d, cfg, -2, -2, nullptr);
+    if (arena_bytes < need) return HGD_ERR_BUFFER_TOO_SMALL;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    size_t off = 0;
+    weight_walk(d, cfg, layer, tensor, &off);
+    bf16_t* dst = reinterpret_cast<bf16_t*>(static_cast<uint8_t*>(arena) + off);
+    const WeightKind k = weight_kind(d, cfg, layer, tensor);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (k.kind == 0) {
+        const int blocks = (int)std::min<int64_t>(((int64_t)n + 255) / 256, 4096);
+        e = launch_pdl(k_copy_u16, dim3(blocks), dim3(256), 0, s, (const bf16_t*)src, dst, (int64_t)n);
+    } else {
+        const int nrb = (k.kind == 1) ? (int)((k.rows + 15) / 16) : (int)((k.rows + 7) / 8);
+        const int64_t chunks = (int64_t)nrb * (k.cols / 32) * 64;
+        const int blocks = (int)std::min<int64_t>((chunks + 255) / 256, 8192);
+        e = launch_pdl(k_pack_weight, dim3(blocks), dim3(256), 0, s, (const bf16_t*)src, dst, (int)k.rows,
+                       (int)k.cols, nrb, k.kind == 1 ? 0 : (k.kind == 2 ? 1 : 2));
+    }
+    return launch_status(e);
+}
+
 int hgd_model_init(hgd_model* m, const hgd_config* cfg, const void* arena, size_t bytes) {
     Dims d;
     int rc = dims_of(cfg, &d);
@@ -445,6 +575,7 @@ int hgd_state_tensor(const hgd_config* cfg, int B, int Tmax, int Lmax, int tenso
         case HGD_S_GDN: *numel = (size_t)d.n_gdn * B * d.H * d.dv * d.dk; break;
         case HGD_S_CONV: *numel = (size_t)d.n_gdn * B * (d.kc - 1) * d.C; break;
         case HGD_S_KV: *numel = (size_t)d.n_attn * 2 * B * d.nkv * (size_t)Lmax * d.hd; break;
+        case HGD_S_RESID: *numel = (size_t)B * Tmax * d.D; break;
         default: *numel = (size_t)B; break;
     }
     return HGD_OK;
@@ -488,14 +619,25 @@ int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T) {
 int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T, float* logits,
                            int32_t* argmax, float* S_rec, float* tail_rec, int32_t* status_dev,
                            hgd_stream_t stream) {
-    if (!m || !st || !tokens || !argmax || !st->arena) return HGD_ERR_INVALID_ARG;
+    if (!m) return HGD_ERR_INVALID_ARG;
+    return hgd_decode_layer_stack_range(m, st, tokens, T, 0, m->cfg.n_layers, 1, logits, argmax, S_rec,
+                                        tail_rec, status_dev, stream);
+}
+
+int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,
+                                 int layer_begin, int layer_end, int run_head, float* logits, int32_t* argmax,
+                                 float* S_rec, float* tail_rec, int32_t* status_dev, hgd_stream_t stream) {
+    if (!m || !st || !st->arena) return HGD_ERR_INVALID_ARG;
     if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
     Dims d;
     int rc = dims_of(&m->cfg, &d);
     if (rc) return rc;
+    if (layer_begin < 0 || layer_end > d.L || layer_begin > layer_end) return HGD_ERR_INVALID_ARG;
+    if (layer_begin == 0 && layer_end > 0 && !tokens) return HGD_ERR_INVALID_ARG;
+    if (run_head && !argmax) return HGD_ERR_INVALID_ARG;
+    if ((tokens && !al16(tokens)) || (argmax && !al16(argmax))) return HGD_ERR_MISALIGNED;
     if ((rc = check_supported(d))) return rc;
-    if ((logits && !al16(logits)) || !al16(argmax) || !al16(tokens) || (S_rec && !al16(S_rec)) ||
-        (tail_rec && !al16(tail_rec)))
+    if ((logits && !al16(logits)) || (S_rec && !al16(S_rec)) || (tail_rec && !al16(tail_rec)))
         return HGD_ERR_MISALIGNED;
     DevInfo di;
     if ((rc = device_info(&di))) return rc;
@@ -515,6 +657,8 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
     bf16_t* mlp = reinterpret_cast<bf16_t*>(A + st->off[SC_MLP]);
     float* bestv = reinterpret_cast<float*>(A + st->off[SC_BESTV]);
     int32_t* besti = reinterpret_cast<int32_t*>(A + st->off[SC_BESTI]);
+    void* ws = A + st->off[SC_WS];
+    const size_t ws_bytes = st->off[SC_END] - st->off[SC_WS];
     const int64_t proj_ld = std::max(d.gdn_out, d.attn_out);
     const float eps = m->cfg.norm_eps;
     const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
@@ -523,47 +667,55 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
     const size_t srec_layer = (size_t)B * T * d.H * d.dv * d.dk;
     const size_t trec_layer = (size_t)B * T * (d.kc - 1) * d.C;
     int ig = 0, ia = 0;
-    for (int l = 0; l < d.L; ++l) {
+    for (int l = 0; l < layer_begin; ++l) (is_attn_layer(&m->cfg, l) ? ia : ig)++;
+    for (int l = layer_begin; l < layer_end; ++l) {
         const uint16_t* const* w = m->w[l];
         const bool att = is_attn_layer(&m->cfg, l);
-        // input RMSNorm + in-projection (layer 0 gathers the embedding rows)
+        // input RMSNorm + in-projection (layer 0 gathers the embedding rows); in a
+        // GDN layer the epilogue also runs the causal conv of the q|k|v channels
         {
             GemvParams p = {};
-            p.W = w[HGD_W_IN]; p.N = (int)(att ? d.attn_out : d.gdn_out); p.K = d.D;
+            p.W = w[HGD_W_IN]; p.packed = 1; p.N = (int)(att ? d.attn_out : d.gdn_out); p.K = d.D;
             p.x = resid; p.x_ld = d.D; p.norm_w = w[HGD_W_IN_NORM]; p.eps = eps;
             p.y = proj; p.y_ld = proj_ld; p.status = status_dev;
             if (l == 0) {
                 p.tokens = tokens; p.embed = m->embed; p.vocab = d.V; p.resid_out = resid; p.resid_out_ld = d.D;
-                rc = run_gemv<PRO_EMBED_RMSNORM, EPI_F32>(p, M, di.sms, s, nullptr);
+            }
+            if (!att) {
+                p.conv_w = w[HGD_W_CONV]; p.conv_tail = conv + ig * c_layer;
+                p.conv_rec = tail_rec ? tail_rec + ig * trec_layer : nullptr;
+                p.conv_C = (int)d.C; p.conv_T = T;
+                rc = (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s)
+                              : run_gemv<PRO_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s);
             } else {
-                rc = run_gemv<PRO_RMSNORM, EPI_F32>(p, M, di.sms, s, nullptr);
+                rc = (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_F32>(p, M, di.sms, ws, ws_bytes, s)
+                              : run_gemv<PRO_RMSNORM, EPI_F32>(p, M, di.sms, ws, ws_bytes, s);
             }
             if (rc) return rc;
         }
         if (!att) {
             GdnLayerParams g{};
-            g.proj = proj; g.proj_ld = proj_ld; g.conv_w = w[HGD_W_CONV];
+            g.proj = proj; g.proj_ld = proj_ld;
             g.A_log = w[HGD_W_A_LOG]; g.dt_bias = w[HGD_W_DT_BIAS];
-            g.S = Sall + ig * s_layer; g.tail = conv + ig * c_layer;
+            g.S = Sall + ig * s_layer;
             g.o = obuf; g.o_ld = (int64_t)d.H * d.dv;
             g.S_rec = S_rec ? S_rec + ig * srec_layer : nullptr;
-            g.tail_rec = tail_rec ? tail_rec + ig * trec_layer : nullptr;
             g.B = B; g.T = T; g.H = d.H; g.dv = d.dv;
             const dim3 grid(B * d.H, d.dv / GDN_ROWS), block(GDN_WARPS * 32);
             cudaError_t e;
             switch (d.dk) {
-                case 32: e = launch_pdl(k_gdn_layer<1, 4>, grid, block, 0, s, g); break;
-                case 64: e = launch_pdl(k_gdn_layer<2, 4>, grid, block, 0, s, g); break;
-                case 128: e = launch_pdl(k_gdn_layer<4, 4>, grid, block, 0, s, g); break;
-                default: e = launch_pdl(k_gdn_layer<8, 4>, grid, block, 0, s, g); break;
+                case 32: e = launch_pdl(k_gdn_layer<1>, grid, block, 0, s, g); break;
+                case 64: e = launch_pdl(k_gdn_layer<2>, grid, block, 0, s, g); break;
+                case 128: e = launch_pdl(k_gdn_layer<4>, grid, block, 0, s, g); break;
+                default: e = launch_pdl(k_gdn_layer<8>, grid, block, 0, s, g); break;
             }
             if ((rc = launch_status(e))) return rc;
             GemvParams p = {};
-            p.W = w[HGD_W_OUT]; p.N = d.D; p.K = d.H * d.dv;
+            p.W = w[HGD_W_OUT]; p.packed = 1; p.N = d.D; p.K = d.H * d.dv;
             p.o = obuf; p.o_ld = (int64_t)d.H * d.dv;
             p.z = proj + d.C; p.z_ld = proj_ld; p.gnorm_w = w[HGD_W_GNORM]; p.gn_d = d.dv; p.eps = eps;
             p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
-            if ((rc = run_gemv<PRO_GATED_NORM, EPI_RESID>(p, M, di.sms, s, nullptr))) return rc;
+            if ((rc = run_gemv<PRO_GATED_NORM, EPI_RESID>(p, M, di.sms, ws, ws_bytes, s))) return rc;
             ++ig;
         } else {
             AttnParams a{};
@@ -574,41 +726,41 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
             a.max_chunks = max_chunks_of(Lmax); a.rope_base = m->cfg.rope_base;
             cudaError_t e = launch_pdl(k_rope_append, dim3(M), dim3(256), 0, s, a);
             if ((rc = launch_status(e))) return rc;
-            e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(128), 0, s, a);
+            e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(32 * (d.nq / d.nkv)), 0, s, a);
             if ((rc = launch_status(e))) return rc;
             e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
             if ((rc = launch_status(e))) return rc;
             GemvParams p = {};
-            p.W = w[HGD_W_OUT]; p.N = d.D; p.K = d.nq * d.hd;
+            p.W = w[HGD_W_OUT]; p.packed = 1; p.N = d.D; p.K = d.nq * d.hd;
             p.x = attn; p.x_ld = (int64_t)d.nq * d.hd;
             p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
-            if ((rc = run_gemv<PRO_COPY, EPI_RESID>(p, M, di.sms, s, nullptr))) return rc;
+            if ((rc = run_gemv<PRO_COPY, EPI_RESID>(p, M, di.sms, ws, ws_bytes, s))) return rc;
             ++ia;
         }
         // MLP: RMSNorm + fused up/gate SwiGLU, then down + residual
         {
             GemvParams p = {};
-            p.W = w[HGD_W_GATE]; p.W2 = w[HGD_W_UP]; p.N = d.I; p.K = d.D;
+            p.W = w[HGD_W_GATE]; p.packed = 1; p.N = d.I; p.K = d.D;
             p.x = resid; p.x_ld = d.D; p.norm_w = w[HGD_W_POST_NORM]; p.eps = eps;
             p.y = mlp; p.y_ld = d.I; p.status = status_dev;
-            if ((rc = run_gemv<PRO_RMSNORM, EPI_SWIGLU>(p, M, di.sms, s, nullptr))) return rc;
+            if ((rc = run_gemv<PRO_RMSNORM, EPI_SWIGLU>(p, M, di.sms, ws, ws_bytes, s))) return rc;
         }
         {
             GemvParams p = {};
-            p.W = w[HGD_W_DOWN]; p.N = d.D; p.K = d.I;
+            p.W = w[HGD_W_DOWN]; p.packed = 1; p.N = d.D; p.K = d.I;
             p.x = mlp; p.x_ld = d.I;
             p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
-            if ((rc = run_gemv<PRO_COPY, EPI_RESID>(p, M, di.sms, s, nullptr))) return rc;
+            if ((rc = run_gemv<PRO_COPY, EPI_RESID>(p, M, di.sms, ws, ws_bytes, s))) return rc;
         }
     }
     // final norm + tied LM head + per-CTA argmax, then the row argmax
-    {
+    if (run_head) {
         GemvParams p = {};
-        p.W = m->embed; p.N = d.V; p.K = d.D;
+        p.W = m->embed; p.packed = 1; p.N = d.V; p.K = d.D;
         p.x = resid; p.x_ld = d.D; p.norm_w = m->final_norm; p.eps = eps;
         p.logits = logits; p.logits_ld = d.V; p.best_v = bestv; p.best_i = besti; p.status = status_dev;
-        if ((rc = run_gemv<PRO_RMSNORM, EPI_ARGMAX>(p, M, di.sms, s, nullptr))) return rc;
-        const int G = gemv_grid(d.V, GV_ROWS, di.sms);
+        int G = 0;
+        if ((rc = run_gemv<PRO_RMSNORM, EPI_ARGMAX>(p, M, di.sms, nullptr, 0, s, &G))) return rc;
         cudaError_t e = launch_pdl(k_argmax_finalize, dim3(M), dim3(128), 0, s, (const float*)bestv,
                                    (const int32_t*)besti, G, M, argmax, status_dev, pos, B, T);
         if ((rc = launch_status(e))) return rc;

@@ -22,7 +22,7 @@
 
 namespace hgd {
 
-constexpr int ATTN_CHUNK = 64;
+constexpr int ATTN_CHUNK = 32;  // keys per partial (one per lane)
 constexpr int ATTN_MAX_HD = 256;
 constexpr int ATTN_MAX_GROUP = 8;
 
@@ -52,11 +52,16 @@ __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ Att
     __shared__ float cs[ATTN_MAX_HD / 2], sn[ATTN_MAX_HD / 2];
     const int half = p.hd / 2;
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const double th = (double)P * pow((double)p.rope_base, -2.0 * (double)i / (double)p.hd);
-        double s, c;
-        sincos(th, &s, &c);
-        cs[i] = (float)c;
-        sn[i] = (float)s;
+        // angle P * base^(-2i/hd) in double, reduced to [-pi, pi] in double, then
+        // the fp32 sine and cosine of the reduced angle
+        const double inv = exp2(-2.0 * (double)i / (double)p.hd * log2((double)p.rope_base));
+        const double th = (double)P * inv;
+        const double tw = 6.283185307179586476925286766559;
+        const float r = (float)(th - tw * rint(th / tw));
+        float s, c;
+        sincosf(r, &s, &c);
+        cs[i] = c;
+        sn[i] = s;
     }
     __syncthreads();
     const float* pr = p.proj + (int64_t)row * p.proj_ld;
@@ -85,8 +90,9 @@ __global__ void __launch_bounds__(256) k_rope_append(const __grid_constant__ Att
     }
 }
 
-// grid (M, nkv, max_chunks), block 128.
-__global__ void __launch_bounds__(128) k_attn_partial(const __grid_constant__ AttnParams p) {
+// grid (M, nkv, max_chunks), block 32 * group (one warp per query head of the
+// group; group <= 8).  Chunk of ATTN_CHUNK (= 32) keys, one key per lane.
+__global__ void __launch_bounds__(32 * ATTN_MAX_GROUP) k_attn_partial(const __grid_constant__ AttnParams p) {
     pdl_launch();
     pdl_wait();
     const int row = blockIdx.x, g = blockIdx.y, ch = blockIdx.z;
@@ -97,58 +103,53 @@ __global__ void __launch_bounds__(128) k_attn_partial(const __grid_constant__ At
     if (key0 > P) return;
     const int nk = min(ATTN_CHUNK, P + 1 - key0);
     const int group = p.nq / p.nkv, hd = p.hd;
-    __shared__ float qs[ATTN_MAX_GROUP][ATTN_MAX_HD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = g * group + warp;  // this warp's query head
     __shared__ float ex[ATTN_MAX_GROUP][ATTN_CHUNK];
-    __shared__ float mls[ATTN_MAX_GROUP][2];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const float* qrow = p.qrot + (int64_t)row * p.nq * hd + (int64_t)g * group * hd;
-    for (int e = tid; e < group * hd; e += blockDim.x) qs[e / hd][e % hd] = qrow[e];
-    __syncthreads();
-    const float scale = 1.0f / sqrtf((float)hd);
     const bf16_t* K = p.kcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd;
     const bf16_t* V = p.vcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd;
-    const int dpl = hd / 32;  // dims per lane (8 at hd = 256)
-    for (int j = warp; j < nk; j += 4) {
-        const bf16_t* kr = K + (int64_t)(key0 + j) * hd + lane * dpl;
-        float kf[8];
-        if (dpl == 8) {
-            const uint4 v = *reinterpret_cast<const uint4*>(kr);
-            kf[0] = bf_lo(v.x); kf[1] = bf_hi(v.x); kf[2] = bf_lo(v.y); kf[3] = bf_hi(v.y);
-            kf[4] = bf_lo(v.z); kf[5] = bf_hi(v.z); kf[6] = bf_lo(v.w); kf[7] = bf_hi(v.w);
-        } else {
-            for (int e = 0; e < dpl; ++e) kf[e] = bf2f(kr[e]);
+    const float* q = p.qrot + (int64_t)row * p.nq * hd + (int64_t)h * hd;
+    // scores: lane j takes key key0 + j; dot over hd in 8-element chunks, in order
+    float sc = -INFINITY;
+    if (lane < nk) {
+        const bf16_t* kr = K + (int64_t)(key0 + lane) * hd;
+        float d = 0.f;
+        for (int e = 0; e < hd; e += 8) {
+            const uint4 kv = *reinterpret_cast<const uint4*>(kr + e);
+            const float4 q0 = *reinterpret_cast<const float4*>(q + e);
+            const float4 q1 = *reinterpret_cast<const float4*>(q + e + 4);
+            d = fmaf(q0.x, bf_lo(kv.x), d); d = fmaf(q0.y, bf_hi(kv.x), d);
+            d = fmaf(q0.z, bf_lo(kv.y), d); d = fmaf(q0.w, bf_hi(kv.y), d);
+            d = fmaf(q1.x, bf_lo(kv.z), d); d = fmaf(q1.y, bf_hi(kv.z), d);
+            d = fmaf(q1.z, bf_lo(kv.w), d); d = fmaf(q1.w, bf_hi(kv.w), d);
         }
-        for (int hh = 0; hh < group; ++hh) {
-            float d = 0.f;
-            for (int e = 0; e < dpl; ++e) d = fmaf(qs[hh][lane * dpl + e], kf[e], d);
-            d = warp_sum(d);
-            if (lane == 0) ex[hh][j] = d * scale;
-        }
+        sc = d * (1.0f / sqrtf((float)hd));
     }
-    __syncthreads();
-    if (tid < group) {
-        float m = -INFINITY;
-        for (int j = 0; j < nk; ++j) m = fmaxf(m, ex[tid][j]);
-        float l = 0.f;
+    // chunk max and sum of exp (butterflies: order fixed by the lane pattern)
+    float m = sc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float e = (lane < nk) ? expf(sc - m) : 0.f;
+    const float l = warp_sum(e);
+    ex[warp][lane] = e;
+    __syncwarp();
+    // acc[d] = sum_j e_j v_j[d]: lane owns dims 8*lane .. +7 (hd = 256) or a
+    // strided set for smaller hd; keys in ascending order
+    float* dst = p.part + (((int64_t)row * p.nq + h) * p.max_chunks + ch) * (hd + 2);
+    for (int d0 = lane * 8; d0 < hd; d0 += 256) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j = 0; j < nk; ++j) {
-            const float e = expf(ex[tid][j] - m);
-            ex[tid][j] = e;
-            l += e;
+            const uint4 vv = *reinterpret_cast<const uint4*>(V + (int64_t)(key0 + j) * hd + d0);
+            const float w = ex[warp][j];
+            acc[0] = fmaf(w, bf_lo(vv.x), acc[0]); acc[1] = fmaf(w, bf_hi(vv.x), acc[1]);
+            acc[2] = fmaf(w, bf_lo(vv.y), acc[2]); acc[3] = fmaf(w, bf_hi(vv.y), acc[3]);
+            acc[4] = fmaf(w, bf_lo(vv.z), acc[4]); acc[5] = fmaf(w, bf_hi(vv.z), acc[5]);
+            acc[6] = fmaf(w, bf_lo(vv.w), acc[6]); acc[7] = fmaf(w, bf_hi(vv.w), acc[7]);
         }
-        mls[tid][0] = m;
-        mls[tid][1] = l;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[2 + d0 + i] = acc[i];
     }
-    __syncthreads();
-    for (int hh = 0; hh < group; ++hh) {
-        const int h = g * group + hh;
-        float* dst = p.part + (((int64_t)row * p.nq + h) * p.max_chunks + ch) * (hd + 2);
-        for (int d = tid; d < hd; d += blockDim.x) {
-            float acc = 0.f;
-            for (int j = 0; j < nk; ++j) acc = fmaf(ex[hh][j], bf2f(V[(int64_t)(key0 + j) * hd + d]), acc);
-            dst[2 + d] = acc;
-        }
-        if (tid == 0) { dst[0] = mls[hh][0]; dst[1] = mls[hh][1]; }
-    }
+    if (lane == 0) { dst[0] = m; dst[1] = l; }
 }
 
 // grid (M, nq), block hd.

@@ -193,64 +193,31 @@ __global__ void k_conv_tail(const __grid_constant__ ConvParams p) {
 }
 
 // ------------------------------------------------------- stack: GDN mixer
-// Conv (over q|k|v channels, SiLU), gates from a/b, L2 norm and the state
-// update for one GDN layer of the stack.  grid (B*H, dv/16), block 128.
-// The CTA with blockIdx.y == 0 also owns the q/k channels' conv tails; every
-// CTA owns the tails of its 16 value channels.  Rows (b, t) are token rows
-// b*T + t of the projection buffer [M][proj_ld] with columns
-// q (H*dk) | k (H*dk) | v (H*dv) | z (H*dv) | a (H) | b (H).
+// Gates from a/b, L2 norm and the state update of one GDN layer of the stack.
+// The projection rows already hold the conv outputs of the q|k|v channels (the
+// conv runs in the in-projection's epilogue).  grid (B*H, dv/16), block 128.
+// Rows (b, t) are token rows b*T + t of the projection buffer [M][proj_ld] with
+// columns q (H*dk) | k (H*dk) | v (H*dv) | z (H*dv) | a (H) | b (H).
 struct GdnLayerParams {
     const float* proj; int64_t proj_ld;
-    const bf16_t* conv_w;       // [C][kc]
     const bf16_t* A_log; const bf16_t* dt_bias;  // [H]
     float* S;                   // this layer: [B][H][dv][dk]
-    float* tail;                // this layer: [B][kc-1][C]
     float* o; int64_t o_ld;     // [M][o_ld]
     float* S_rec;               // this layer: [B][T][H][dv][dk] or null
-    float* tail_rec;            // this layer: [B][T][kc-1][C] or null
     int B, T, H, dv;
 };
 
-template <int KPL, int KC>
+template <int KPL>
 __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_constant__ GdnLayerParams p) {
     pdl_launch();
     pdl_wait();
     constexpr int DK = 32 * KPL;
-    constexpr int NT = GDN_WARPS * 32;
-    constexpr int kc = KC, nt = KC - 1;
-    __shared__ float qs[DK], ks[DK], vs[GDN_ROWS], coef[4];
+    __shared__ float qs[DK], ks[DK], coef[4];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, dv = p.dv;
     const int b = blockIdx.x / H, h = blockIdx.x % H;
-    const int vrow0 = blockIdx.y * GDN_ROWS;
-    const int row0 = vrow0 + warp * GDN_RPW;
+    const int row0 = blockIdx.y * GDN_ROWS + warp * GDN_RPW;
     const int64_t C = 2 * (int64_t)H * DK + (int64_t)H * dv;
-    const bool own_qk = (blockIdx.y == 0);
-
-    // channels handled by this thread: q channel and k channel (tid < DK, looped),
-    // and value channel tid (< 16)
-    constexpr int QK_PER_T = (DK + NT - 1) / NT;
-    float tq[QK_PER_T][nt], tk[QK_PER_T][nt], wq[QK_PER_T][kc], wk[QK_PER_T][kc];
-    float tv[nt], wv[kc];
-    float* tail_b = p.tail + (int64_t)b * nt * C;
-#pragma unroll
-    for (int u = 0; u < QK_PER_T; ++u) {
-        const int i = tid + u * NT;
-        if (i < DK) {
-            const int64_t cq = (int64_t)h * DK + i, ck = (int64_t)H * DK + h * DK + i;
-#pragma unroll
-            for (int j = 0; j < kc; ++j) { wq[u][j] = bf2f(p.conv_w[cq * kc + j]); wk[u][j] = bf2f(p.conv_w[ck * kc + j]); }
-#pragma unroll
-            for (int j = 0; j < nt; ++j) { tq[u][j] = tail_b[j * C + cq]; tk[u][j] = tail_b[j * C + ck]; }
-        }
-    }
-    const int64_t cv = 2 * (int64_t)H * DK + (int64_t)h * dv + vrow0 + tid;
-    if (tid < GDN_ROWS) {
-#pragma unroll
-        for (int j = 0; j < kc; ++j) wv[j] = bf2f(p.conv_w[cv * kc + j]);
-#pragma unroll
-        for (int j = 0; j < nt; ++j) tv[j] = tail_b[j * C + cv];
-    }
     const float A = expf(bf2f(p.A_log[h])), dtb = bf2f(p.dt_bias[h]);
 
     float S[GDN_RPW][KPL];
@@ -261,47 +228,14 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
     for (int t = 0; t < p.T; ++t) {
         const int64_t row = (int64_t)b * p.T + t;
         const float* pr = p.proj + row * p.proj_ld;
-        float* trec = p.tail_rec ? p.tail_rec + ((int64_t)b * p.T + t) * nt * C : nullptr;
         __syncthreads();
-#pragma unroll
-        for (int u = 0; u < QK_PER_T; ++u) {
-            const int i = tid + u * NT;
-            if (i < DK) {
-                const int64_t cq = (int64_t)h * DK + i, ck = (int64_t)H * DK + h * DK + i;
-                const float xq = pr[cq], xk = pr[ck];
-                float sq = 0.f, sk = 0.f;
-#pragma unroll
-                for (int j = 0; j < nt; ++j) { sq = fmaf(wq[u][j], tq[u][j], sq); sk = fmaf(wk[u][j], tk[u][j], sk); }
-                sq = fmaf(wq[u][nt], xq, sq);
-                sk = fmaf(wk[u][nt], xk, sk);
-                qs[i] = silu_f(sq);
-                ks[i] = silu_f(sk);
-#pragma unroll
-                for (int j = 0; j + 1 < nt; ++j) { tq[u][j] = tq[u][j + 1]; tk[u][j] = tk[u][j + 1]; }
-                tq[u][nt - 1] = xq;
-                tk[u][nt - 1] = xk;
-                if (trec && own_qk)
-#pragma unroll
-                    for (int j = 0; j < nt; ++j) { trec[j * C + cq] = tq[u][j]; trec[j * C + ck] = tk[u][j]; }
-            }
-        }
-        if (tid < GDN_ROWS) {
-            const float xv = pr[cv];
-            float sv = 0.f;
-#pragma unroll
-            for (int j = 0; j < nt; ++j) sv = fmaf(wv[j], tv[j], sv);
-            sv = fmaf(wv[nt], xv, sv);
-            vs[tid] = silu_f(sv);
-#pragma unroll
-            for (int j = 0; j + 1 < nt; ++j) tv[j] = tv[j + 1];
-            tv[nt - 1] = xv;
-            if (trec)
-#pragma unroll
-                for (int j = 0; j < nt; ++j) trec[j * C + cv] = tv[j];
+        for (int i = tid; i < DK; i += GDN_WARPS * 32) {
+            qs[i] = pr[(int64_t)h * DK + i];
+            ks[i] = pr[(int64_t)H * DK + (int64_t)h * DK + i];
         }
         __syncthreads();
-        if (warp == 0) { const float s = l2_scale<KPL>(qs, lane); if (lane == 0) coef[0] = s; }
-        if (warp == 1) { const float s = l2_scale<KPL>(ks, lane); if (lane == 0) coef[1] = s; }
+        if (warp == 0) { const float sc = l2_scale<KPL>(qs, lane); if (lane == 0) coef[0] = sc; }
+        if (warp == 1) { const float sc = l2_scale<KPL>(ks, lane); if (lane == 0) coef[1] = sc; }
         if (warp == 2 && lane == 0) {
             const float a = pr[C + (int64_t)H * dv + h];
             const float braw = pr[C + (int64_t)H * dv + H + h];
@@ -314,8 +248,9 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
 #pragma unroll
         for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
         float vrow[GDN_RPW], o[GDN_RPW];
+        const float* vp = pr + 2 * (int64_t)H * DK + (int64_t)h * dv + row0;
 #pragma unroll
-        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vs[warp * GDN_RPW + r];
+        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
         gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o);
         if (lane < GDN_RPW) {
             float ov = o[0];
@@ -331,19 +266,6 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
     }
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
-    // conv tails back
-#pragma unroll
-    for (int u = 0; u < QK_PER_T; ++u) {
-        const int i = tid + u * NT;
-        if (i < DK && own_qk) {
-            const int64_t cq = (int64_t)h * DK + i, ck = (int64_t)H * DK + h * DK + i;
-#pragma unroll
-            for (int j = 0; j < nt; ++j) { tail_b[j * C + cq] = tq[u][j]; tail_b[j * C + ck] = tk[u][j]; }
-        }
-    }
-    if (tid < GDN_ROWS)
-#pragma unroll
-        for (int j = 0; j < nt; ++j) tail_b[j * C + cv] = tv[j];
 }
 
 }  // namespace hgd

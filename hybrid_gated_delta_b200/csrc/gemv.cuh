@@ -2,46 +2,58 @@
 //
 // y[m][n] = sum_k x[m][k] W[n][k]  ("decode_linear_benchmark.md" commit message:
 // BF16 GEMV and fused up/gate SwiGLU for decode shapes).  Design for B200:
-//  * one producer warp streams 16-row weight tiles into a shared-memory ring with
-//    1-D bulk copies (cp.async.bulk, one per row segment, mbarrier transaction
-//    counts, L2 evict-first since weights are read once per step);
-//  * eight consumer warps split each tile's k-block and run mma.sync m16n8k16
-//    with the weight rows as the MMA M dimension and up to 32 tokens as N
-//    (swap-AB), fp32 accumulation; rows are padded by 16 bytes in shared memory
-//    so every 128-bit fragment load is bank-conflict free;
-//  * the k-dimension is cut into equal blocks of <= 1024 (a function of K only);
-//    each block's partial is reduced over the warps in a fixed order and the
-//    block partials are added in block order, so every output's arithmetic
-//    depends on K alone (not on M, N, the grid or the SM count);
+//  * work is cut into 16-row blocks of the weight matrix and 256-column slabs;
+//    a warp owns whole work items (a row block, or one slab of it when the row
+//    blocks alone cannot occupy every warp of the GPU);
+//  * the warp loads its mma.sync A fragments straight from HBM with 128-bit
+//    non-allocating loads (L2 evict-first: weights are read once per step),
+//    eight 32-column steps in flight per warp in a rolling register pipeline:
+//    no shared-memory staging, no copy engine on the critical path.  Columns are
+//    taken in a per-thread permuted order (the same permutation for the weight
+//    and the token fragments, so each MMA still forms the exact dot product),
+//    which makes every fragment a contiguous 16-byte load;
+//  * mma.sync m16n8k16 with the weight rows as the MMA M dimension and up to 32
+//    token rows as N (swap-AB), fp32 accumulation in two chains (even / odd
+//    steps); the token rows sit in shared memory, padded so fragment loads are
+//    conflict free;
+//  * every output is the sum, in slab order, of per-slab partials (chain 0 +
+//    chain 1): its arithmetic depends on K alone, not on M, N, the grid, the SM
+//    count or how slabs are spread over warps.  Split slabs meet in a workspace
+//    and the last arriver adds them in slab order (no floating-point atomics);
 //  * fused prologues (RMSNorm of the residual stream, embedding gather, gated
-//    RMSNorm) and epilogues (fp32 / bf16 store, residual add, SwiGLU, argmax);
-//  * programmatic dependent launch: weights stream before the previous kernel
-//    in the stream has finished; activations are read after griddepcontrol.wait.
+//    RMSNorm) and epilogues (fp32 / bf16 store, residual add, SwiGLU, argmax,
+//    the causal conv of the GDN q|k|v channels);
+//  * programmatic dependent launch: each warp issues its first weight loads
+//    before griddepcontrol.wait, overlapping the previous kernel's tail.
 #pragma once
 
 #include "common.cuh"
 
 namespace hgd {
 
-constexpr int GV_WARPS = 8;
-constexpr int GV_THREADS = (GV_WARPS + 1) * 32;
+constexpr int GV_CW = 8;                       // warps per CTA
+constexpr int GV_WARPS = GV_CW;
+constexpr int GV_THREADS = GV_CW * 32;
 constexpr int GV_ROWS = 16;
-constexpr int GV_KB_MAX = 1024;
-constexpr int GV_PAD = 8;  // bf16 elements of padding per shared-memory row
-constexpr int GV_PITCH = 17;  // floats per token in the reduction buffers
+constexpr int GV_KS = 256;                     // slab width
+constexpr int GV_SLAB_STEPS = GV_KS / 32;      // 32-column steps per slab
+constexpr int GV_PAD = 8;                      // bf16 elements of padding per token row
 constexpr int GV_SMEM_LIMIT = 227 * 1024;
-constexpr int GV_MAX_STAGES = 8;
 
 enum GvPrologue { PRO_COPY = 0, PRO_RMSNORM = 1, PRO_EMBED_RMSNORM = 2, PRO_GATED_NORM = 3 };
-enum GvEpilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_ARGMAX = 4 };
+enum GvEpilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_ARGMAX = 4, EPI_QKV_CONV = 5 };
+constexpr int GV_CONV_K = 4;  // conv width of the fused conv epilogue
 
 struct GemvParams {
-    const bf16_t* W;   // [N][K]; SwiGLU: gate weights [I][K]
-    const bf16_t* W2;  // SwiGLU: up weights [I][K]
+    const bf16_t* W;   // [N][K]; SwiGLU: gate weights [I][K]; packed: the tiles (see gv_tile)
+    const bf16_t* W2;  // SwiGLU: up weights [I][K] (unpacked only)
+    int packed;        // 1: W holds the fragment-ordered tiles of the (virtual) matrix
     int N, K, M;       // N output features, M token rows of this launch
-    int kb, nkb;       // k-block width (multiple of 32) and count
+    int nks;           // slabs per row block (K / 256 rounded up)
     int n_rowblk;      // row blocks (16 rows; SwiGLU: 8 gate + 8 up rows)
-    int nstage, stage_bytes, x_bytes;
+    int split;         // 1: one slab per work item, partials through the workspace
+    int n_items;       // n_rowblk * (split ? nks : 1)
+    int x_bytes;       // bytes of the token rows in shared memory
     // prologue
     const bf16_t* x; int64_t x_ld;         // COPY: [M][x_ld]; RMSNORM: residual rows
     const bf16_t* norm_w; float eps;       // RMSNORM gains [K]
@@ -56,36 +68,22 @@ struct GemvParams {
     const bf16_t* resid; int64_t resid_ld; // RESID: residual rows (may alias y)
     float* logits; int64_t logits_ld;      // ARGMAX: optional logits rows
     float* best_v; int32_t* best_i;        // ARGMAX: [M][gridDim.x] partials
+    // split-K workspace: partials [n_rowblk * nks][16][ws_mp] fp32, counters [n_rowblk]
+    float* ws_part; int32_t* ws_cnt; int ws_mp;
+    // QKV_CONV: outputs < conv_C are channels of the depthwise causal conv (width 4,
+    // SiLU): y = silu(sum_j w[c][j] u_j) over the kept tail and the new value, the
+    // tail [B][3][conv_C] shifted in place, tail records [B][T][3][conv_C] (or null).
+    // Token row m of this launch is stream (m0 + m) / conv_T, row (m0 + m) % conv_T.
+    const bf16_t* conv_w; float* conv_tail; float* conv_rec; int conv_C, conv_T, m0;
     int32_t* status;
 };
 
 __host__ __device__ inline int gv_align16(int v) { return (v + 15) & ~15; }
-
-// Equal k-blocks of at most GV_KB_MAX, multiples of 32.  Depends on K only.
-__host__ __device__ inline void gv_kblocks(int K, int* kb, int* nkb) {
-    int n = (K + GV_KB_MAX - 1) / GV_KB_MAX;
-    int w = (K + n - 1) / n;
-    w = (w + 31) & ~31;
-    *kb = w;
-    *nkb = (K + w - 1) / w;
-}
-
-__device__ __forceinline__ bool bar_or(int id, int nthreads, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
+__host__ __device__ inline int gv_slabs(int K) { return (K + GV_KS - 1) / GV_KS; }
 
 // Source row of tile row i (0..15) of row block rb; nullptr if past the end.
-__device__ __forceinline__ const bf16_t* gv_row(const GemvParams& p, int EPI_SWI, int rb, int i) {
-    if (EPI_SWI) {
+__device__ __forceinline__ const bf16_t* gv_row(const GemvParams& p, bool swi, int rb, int i) {
+    if (swi) {
         const int r = rb * 8 + (i & 7);
         if (r >= p.N) return nullptr;
         return (i < 8 ? p.W : p.W2) + (int64_t)r * p.K;
@@ -93,6 +91,39 @@ __device__ __forceinline__ const bf16_t* gv_row(const GemvParams& p, int EPI_SWI
     const int r = rb * GV_ROWS + i;
     if (r >= p.N) return nullptr;
     return p.W + (int64_t)r * p.K;
+}
+
+// Fragment-ordered weight layout.  The matrix (for SwiGLU the virtual matrix
+// whose row block rb holds gate rows 8rb..8rb+7 then up rows 8rb..8rb+7) is cut
+// into 16-row x 32-column tiles, row block major; tile (rb, step) is 512 bf16 at
+// element (rb * K/32 + step) * 512.  Within a tile, lane l = 4*r8 + c of a warp
+// owns elements [8l, 8l+8) (row r8) and [256 + 8l, 256 + 8l + 8) (row r8 + 8),
+// each the eight columns step*32 + 8c .. +7 of its row: one warp-wide 16-byte
+// load per half-tile reads 512 contiguous bytes.  Rows past the matrix are zero.
+__host__ __device__ inline int64_t gv_tile_elem(int64_t rb, int step, int steps, int half, int lane) {
+    return ((rb * steps + step) * 512) + half * 256 + lane * 8;
+}
+
+// Offset (elements) of the 16-byte chunk cc (columns 8cc..8cc+7) of row n of a
+// packed plain matrix with `steps` = K/32 column steps.
+__host__ __device__ inline int64_t gv_packed_chunk(int64_t n, int cc, int steps) {
+    const int i = (int)(n & 15);
+    return gv_tile_elem(n >> 4, cc >> 2, steps, i >> 3, ((i & 7) << 2) | (cc & 3));
+}
+
+__device__ __forceinline__ float ld_cg(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// 16-byte streaming load of weights: not allocated in L1, evict-first in L2.
+__device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
 }
 
 // ----------------------------------------------------------------- prologues
@@ -139,9 +170,15 @@ __device__ __forceinline__ void gv_prologue(const GemvParams& p, bf16_t* xs, int
             } else {
                 src = p.x + m * p.x_ld;
             }
+            // 16-byte chunk c of the source row (the embedding is stored packed)
+            auto chunk = [&](int c) -> const uint4* {
+                if (PRO == PRO_EMBED_RMSNORM)
+                    return reinterpret_cast<const uint4*>(p.embed + gv_packed_chunk(p.tokens[m], c, K >> 5));
+                return reinterpret_cast<const uint4*>(src + c * 8);
+            };
             float ss = 0.f;
             for (int c = lane; c < K / 8; c += 32) {
-                const uint4 v = *reinterpret_cast<const uint4*>(src + c * 8);
+                const uint4 v = *chunk(c);
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -153,7 +190,7 @@ __device__ __forceinline__ void gv_prologue(const GemvParams& p, bf16_t* xs, int
             ss = warp_sum(ss);
             const float r = rsqrtf(ss / (float)K + p.eps);
             for (int c = lane; c < K / 8; c += 32) {
-                const uint4 v = *reinterpret_cast<const uint4*>(src + c * 8);
+                const uint4 v = *chunk(c);
                 const uint4 g = *reinterpret_cast<const uint4*>(p.norm_w + c * 8);
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
                 const uint32_t g4[4] = {g.x, g.y, g.z, g.w};
@@ -196,192 +233,329 @@ __device__ __forceinline__ void gv_prologue(const GemvParams& p, bf16_t* xs, int
 }
 
 // -------------------------------------------------------------------- kernel
+// One work item of a warp: row block rb, slabs [s0, s1).
+struct GvItem { int rb, s0, s1; };
+
+__device__ __forceinline__ bool gv_item(const GemvParams& p, int slot, int i, GvItem* it) {
+    const int u = slot + i * gridDim.x * GV_CW;
+    if (u >= p.n_items) return false;
+    if (p.split) { it->rb = u / p.nks; it->s0 = u % p.nks; it->s1 = it->s0 + 1; }
+    else { it->rb = u; it->s0 = 0; it->s1 = p.nks; }
+    return true;
+}
+
 template <int NT, int PRO, int EPI>
-__global__ void __launch_bounds__(GV_THREADS, 1) k_gemv(const __grid_constant__ GemvParams p) {
+__global__ void __launch_bounds__(GV_THREADS, (NT >= 4) ? 1 : 2) k_gemv(const __grid_constant__ GemvParams p) {
     constexpr int MP = 8 * NT;
+    constexpr int NB = (NT >= 4) ? 4 : 8;   // 32-column steps in flight per warp
     constexpr bool SWI = (EPI == EPI_SWIGLU);
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int K = p.K;
-    const int XS = K + GV_PAD;           // elements per xs row
-    const int RS = p.kb + GV_PAD;        // elements per stage row
-    uint8_t* stages = smem;
-    bf16_t* xs = reinterpret_cast<bf16_t*>(smem + p.nstage * p.stage_bytes);
-    float* red = reinterpret_cast<float*>(smem + p.nstage * p.stage_bytes + p.x_bytes);
-    float* yacc = red + GV_WARPS * MP * GV_PITCH;
-    uint64_t* full = reinterpret_cast<uint64_t*>(yacc + MP * GV_PITCH + (MP * GV_PITCH & 1));
-    uint64_t* empty = full + GV_MAX_STAGES;
-    volatile int* abort_s = reinterpret_cast<volatile int*>(empty + GV_MAX_STAGES);
+    const int XS = K + GV_PAD;
+    bf16_t* xs = reinterpret_cast<bf16_t*>(smem);
+    float* amax_v = reinterpret_cast<float*>(smem + p.x_bytes);
+    int* amax_i = reinterpret_cast<int*>(amax_v + GV_CW * MP);
+    float* cbuf = reinterpret_cast<float*>(amax_i + GV_CW * MP);  // [CW][16][MP] (QKV_CONV)
 
-    if (tid == 0) {
-        for (int s = 0; s < p.nstage; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], GV_WARPS);
-        }
-        *abort_s = 0;
-        mbar_fence_init();
-    }
-    __syncthreads();
     pdl_launch();
+    const uint64_t pol = policy_evict_first();
+    const int r8 = lane >> 2, c = lane & 3;
+    const int slot = warp * gridDim.x + blockIdx.x;
+    const int steps_total = K >> 5;
 
-    // ------------------------------------------------------------ producer
-    if (warp == GV_WARPS) {
-        if (lane != 0) return;
-        const uint64_t pol = policy_evict_first();
-        int filled[GV_MAX_STAGES];
-        for (int s = 0; s < GV_MAX_STAGES; ++s) filled[s] = -1;
-        int it = 0;
-        bool ok = true;
-        for (int rb = blockIdx.x; ok && rb < p.n_rowblk; rb += gridDim.x) {
-            for (int j = 0; j < p.nkb; ++j, ++it) {
-                const int s = it % p.nstage;
-                const uint32_t round = (uint32_t)(it / p.nstage);
-                if (!mbar_wait_bounded(&empty[s], (round & 1) ^ 1, abort_s)) {
-                    if (!*abort_s) set_status(p.status, HGD_ERR_TIMEOUT);
-                    *abort_s = 1;
-                    ok = false;
-                    break;
-                }
-                const int k0 = j * p.kb;
-                const int kbw = (j == p.nkb - 1) ? K - k0 : p.kb;
-                const uint32_t rbytes = (uint32_t)kbw * 2u;
-                uint32_t total = 0;
-                for (int i = 0; i < GV_ROWS; ++i)
-                    if (gv_row(p, SWI, rb, i)) total += rbytes;
-                mbar_arrive_expect_tx(&full[s], total);
-                uint8_t* dst = stages + s * p.stage_bytes;
-                for (int i = 0; i < GV_ROWS; ++i) {
-                    const bf16_t* src = gv_row(p, SWI, rb, i);
-                    if (src) bulk_g2s(dst + i * RS * 2, src + k0, rbytes, &full[s], pol);
-                }
-                filled[s] = (int)(round & 1);
+    // rolling register pipeline of A fragments (rows r8 and r8+8, 16 bytes each)
+    uint4 A0[NB], A1[NB];
+    const bf16_t* row_lo = nullptr;   // unpacked: the two rows; packed: the row block's tiles
+    const bf16_t* row_hi = nullptr;
+    auto load_step = [&](int j, int step) {
+        if (step < steps_total) {
+            if (p.packed) {
+                A0[j] = ldg_stream(row_lo + step * 512, pol);
+                A1[j] = ldg_stream(row_lo + step * 512 + 256, pol);
+            } else {
+                const int k = step * 32 + 8 * c;
+                A0[j] = row_lo ? ldg_stream(row_lo + k, pol) : make_uint4(0, 0, 0, 0);
+                A1[j] = row_hi ? ldg_stream(row_hi + k, pol) : make_uint4(0, 0, 0, 0);
             }
         }
-        // Do not leave while a copy into this CTA's shared memory is in flight.
-        for (int s = 0; s < p.nstage; ++s)
-            if (filled[s] >= 0) (void)mbar_wait_bounded(&full[s], (uint32_t)filled[s], nullptr);
-        return;
+    };
+    auto set_rows = [&](int rb) {
+        if (p.packed) {
+            row_lo = p.W + gv_tile_elem(rb, 0, steps_total, 0, lane);
+        } else {
+            row_lo = gv_row(p, SWI, rb, r8);
+            row_hi = gv_row(p, SWI, rb, r8 + 8);
+        }
+    };
+    GvItem it;
+    bool have = gv_item(p, slot, 0, &it);
+    if (have) {  // weights never depend on the previous kernel: start streaming now
+        set_rows(it.rb);
+#pragma unroll
+        for (int j = 0; j < NB; ++j) load_step(j, it.s0 * GV_SLAB_STEPS + j);
     }
 
-    // ----------------------------------------------------------- consumers
-    const int ctid = tid;  // 0..255
     pdl_wait();
-    gv_prologue<MP, PRO>(p, xs, ctid, warp, lane, yacc);
-    named_bar(1, GV_WARPS * 32);
+    gv_prologue<MP, PRO>(p, xs, tid, warp, lane, nullptr);
+    __syncthreads();
 
-    const int r = lane >> 2, c = lane & 3;
-    float best_v = -INFINITY;
-    int best_i = 0x7fffffff;
+    float best_v[NT][2];
+    int best_i[NT][2];
     bool saw_nan = false;
-    int it = 0;
-    bool aborted = false;
-    for (int rb = blockIdx.x; !aborted && rb < p.n_rowblk; rb += gridDim.x) {
-        for (int j = 0; j < p.nkb; ++j, ++it) {
-            const int s = it % p.nstage;
-            const uint32_t round = (uint32_t)(it / p.nstage);
-            const bool got = mbar_wait_bounded(&full[s], round & 1, abort_s);
-            float acc[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-            const int k0 = j * p.kb;
-            const int kbw = (j == p.nkb - 1) ? K - k0 : p.kb;
-            if (got) {
-                const int S = kbw >> 5;
-                const int s0 = (warp * S) / GV_WARPS, s1 = ((warp + 1) * S) / GV_WARPS;
-                const bf16_t* tile = reinterpret_cast<const bf16_t*>(stages + s * p.stage_bytes);
-                const bf16_t* a_lo = tile + r * RS + 8 * c;
-                const bf16_t* a_hi = tile + (r + 8) * RS + 8 * c;
-                const bf16_t* xb = xs + r * XS + k0 + 8 * c;
-#pragma unroll 2
-                for (int st = s0; st < s1; ++st) {
-                    const uint4 A0 = lds128(a_lo + st * 32);
-                    const uint4 A1 = lds128(a_hi + st * 32);
+    for (int nt = 0; nt < NT; ++nt) { best_v[nt][0] = best_v[nt][1] = -INFINITY; best_i[nt][0] = best_i[nt][1] = 0x7fffffff; }
+    const bf16_t* xb = xs + r8 * XS + 8 * c;
+
+    for (int i = 0; have; ++i) {
+        float yacc[NT][4];
+        for (int s = it.s0; s < it.s1; ++s) {
+            // one slab: up to 8 steps, chain = step parity; loads run NB steps ahead
+            float c0[NT][4], c1[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) { c0[nt][q] = 0.f; c1[nt][q] = 0.f; }
+            const int base = s * GV_SLAB_STEPS;
+#pragma unroll
+            for (int jj = 0; jj < GV_SLAB_STEPS; ++jj) {
+                const int j = jj % NB;
+                const int step = base + jj;
+                if (step < steps_total) {
+                    const uint4 a0 = A0[j], a1 = A1[j];
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        const uint4 Bv = lds128(xb + nt * 8 * XS + st * 32);
-                        mma_bf16_16816(acc[nt], A0.x, A1.x, A0.y, A1.y, Bv.x, Bv.y);
-                        mma_bf16_16816(acc[nt], A0.z, A1.z, A0.w, A1.w, Bv.z, Bv.w);
+                        const uint4 Bv = lds128(xb + nt * 8 * XS + step * 32);
+                        float (&acc)[4] = (jj & 1) ? c1[nt] : c0[nt];
+                        mma_bf16_16816(acc, a0.x, a1.x, a0.y, a1.y, Bv.x, Bv.y);
+                        mma_bf16_16816(acc, a0.z, a1.z, a0.w, a1.w, Bv.z, Bv.w);
                     }
+                    // refill this register slot with the step NB ahead (same item)
+                    const int nxt = step + NB;
+                    if (nxt < it.s1 * GV_SLAB_STEPS) load_step(j, nxt);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-            } else if (!*abort_s) {
-                set_status(p.status, HGD_ERR_TIMEOUT);
-                *abort_s = 1;
             }
-            // warp partials -> red[warp][token][row]
-            float* rw = red + warp * MP * GV_PITCH;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) c0[nt][q] = c0[nt][q] + c1[nt][q];
+            if (p.split) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) yacc[nt][q] = c0[nt][q];
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) yacc[nt][q] = (s == 0) ? c0[nt][q] : yacc[nt][q] + c0[nt][q];
+            }
+        }
+        const int rb = it.rb, s_item = it.s0;
+        // next item: start its loads before this item's epilogue
+        GvItem nx;
+        have = gv_item(p, slot, i + 1, &nx);
+        if (have) {
+            set_rows(nx.rb);
+#pragma unroll
+            for (int j = 0; j < NB; ++j) load_step(j, nx.s0 * GV_SLAB_STEPS + j);
+        }
+
+        bool finish = true;
+        if (p.split) {
+            // slab partial -> workspace; the last of the row block's slabs adds them in order
+            float* wp = p.ws_part + ((int64_t)(rb * p.nks + s_item) * GV_ROWS) * p.ws_mp;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int n0 = nt * 8 + 2 * c;
-                rw[n0 * GV_PITCH + r] = acc[nt][0];
-                rw[(n0 + 1) * GV_PITCH + r] = acc[nt][1];
-                rw[n0 * GV_PITCH + r + 8] = acc[nt][2];
-                rw[(n0 + 1) * GV_PITCH + r + 8] = acc[nt][3];
+                wp[r8 * p.ws_mp + n0] = yacc[nt][0];
+                wp[r8 * p.ws_mp + n0 + 1] = yacc[nt][1];
+                wp[(r8 + 8) * p.ws_mp + n0] = yacc[nt][2];
+                wp[(r8 + 8) * p.ws_mp + n0 + 1] = yacc[nt][3];
             }
-            if (bar_or(1, GV_WARPS * 32, !got || *abort_s)) {
-                aborted = true;
-                break;
-            }
-            // fixed-order reduction over warps, then over k-blocks
-            for (int e = ctid; e < MP * GV_ROWS; e += GV_WARPS * 32) {
-                const int n = e >> 4, i = e & 15;
-                float sum = red[n * GV_PITCH + i];
+            __threadfence();
+            __syncwarp();
+            int old = 0;
+            if (lane == 0) old = atomicAdd(&p.ws_cnt[rb], 1);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            finish = (old == p.nks - 1);
+            if (finish) {
+                __threadfence();
+                for (int j = 0; j < p.nks; ++j) {
+                    const float* pp = p.ws_part + ((int64_t)(rb * p.nks + j) * GV_ROWS) * p.ws_mp;
 #pragma unroll
-                for (int w = 1; w < GV_WARPS; ++w) sum += red[w * MP * GV_PITCH + n * GV_PITCH + i];
-                yacc[n * GV_PITCH + i] = (j == 0) ? sum : yacc[n * GV_PITCH + i] + sum;
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int n0 = nt * 8 + 2 * c;
+                        const float v0 = ld_cg(pp + r8 * p.ws_mp + n0), v1 = ld_cg(pp + r8 * p.ws_mp + n0 + 1);
+                        const float v2 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0), v3 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0 + 1);
+                        if (j == 0) { yacc[nt][0] = v0; yacc[nt][1] = v1; yacc[nt][2] = v2; yacc[nt][3] = v3; }
+                        else { yacc[nt][0] += v0; yacc[nt][1] += v1; yacc[nt][2] += v2; yacc[nt][3] += v3; }
+                    }
+                }
+                if (lane == 0) p.ws_cnt[rb] = 0;  // leave the workspace ready for the next call
             }
-            named_bar(1, GV_WARPS * 32);
-            if (j != p.nkb - 1) continue;
-
-            // ----------------------------------------------------- epilogue
+        }
+        if (!finish) { it = nx; continue; }
+        // ----------------------------------------------------------- epilogue
+        if (EPI == EPI_QKV_CONV) {
+            // Gather the 16 x MP tile in shared memory; lane l < 16 then runs the conv
+            // of channel rb*16 + l over the launch's token rows in order.  The row
+            // block (hence the channel and its tail) belongs to this warp alone.
+            float* cb = cbuf + warp * GV_ROWS * MP;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int n0 = nt * 8 + 2 * c;
+                cb[r8 * MP + n0] = yacc[nt][0];
+                cb[r8 * MP + n0 + 1] = yacc[nt][1];
+                cb[(r8 + 8) * MP + n0] = yacc[nt][2];
+                cb[(r8 + 8) * MP + n0 + 1] = yacc[nt][3];
+            }
+            __syncwarp();
+            const int ch = rb * GV_ROWS + lane;
+            if (lane < GV_ROWS && ch < p.N) {
+                float* yrow = reinterpret_cast<float*>(p.y);
+                if (ch >= p.conv_C) {
+                    for (int m = 0; m < p.M; ++m) yrow[m * p.y_ld + ch] = cb[lane * MP + m];
+                } else {
+                    float w[GV_CONV_K], tl[GV_CONV_K - 1];
+#pragma unroll
+                    for (int j = 0; j < GV_CONV_K; ++j) w[j] = bf2f(p.conv_w[(int64_t)ch * GV_CONV_K + j]);
+                    int cur_b = -1;
+                    for (int m = 0; m < p.M; ++m) {
+                        const int gm = p.m0 + m, b = gm / p.conv_T, t = gm % p.conv_T;
+                        float* tb = p.conv_tail + (int64_t)b * (GV_CONV_K - 1) * p.conv_C + ch;
+                        if (b != cur_b) {
+#pragma unroll
+                            for (int j = 0; j < GV_CONV_K - 1; ++j) tl[j] = tb[(int64_t)j * p.conv_C];
+                            cur_b = b;
+                        }
+                        const float xv = cb[lane * MP + m];
+                        float acc = 0.f;
+#pragma unroll
+                        for (int j = 0; j < GV_CONV_K - 1; ++j) acc = fmaf(w[j], tl[j], acc);
+                        acc = fmaf(w[GV_CONV_K - 1], xv, acc);
+                        yrow[m * p.y_ld + ch] = silu_f(acc);
+#pragma unroll
+                        for (int j = 0; j + 1 < GV_CONV_K - 1; ++j) tl[j] = tl[j + 1];
+                        tl[GV_CONV_K - 2] = xv;
+                        if (p.conv_rec) {
+                            float* rr = p.conv_rec + ((int64_t)b * p.conv_T + t) * (GV_CONV_K - 1) * p.conv_C + ch;
+#pragma unroll
+                            for (int j = 0; j < GV_CONV_K - 1; ++j) rr[(int64_t)j * p.conv_C] = tl[j];
+                        }
+                        if (m == p.M - 1 || t == p.conv_T - 1) {
+#pragma unroll
+                            for (int j = 0; j < GV_CONV_K - 1; ++j) tb[(int64_t)j * p.conv_C] = tl[j];
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            it = nx;
+            continue;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int n0 = nt * 8 + 2 * c;  // tokens n0, n0 + 1; rows r8, r8 + 8
             if (EPI == EPI_SWIGLU) {
-                for (int e = ctid; e < MP * 8; e += GV_WARPS * 32) {
-                    const int n = e >> 3, i = e & 7;
-                    const int col = rb * 8 + i;
-                    if (n < p.M && col < p.N) {
-                        const float g = yacc[n * GV_PITCH + i], u = yacc[n * GV_PITCH + i + 8];
-                        reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(silu_f(g) * u);
-                    }
-                }
-            } else if (EPI == EPI_ARGMAX) {
-                for (int e = ctid; e < MP * GV_ROWS; e += GV_WARPS * 32) {
-                    const int n = e >> 4, i = e & 15;
-                    const int col = rb * GV_ROWS + i;
-                    if (p.logits && n < p.M && col < p.N) p.logits[n * p.logits_ld + col] = yacc[n * GV_PITCH + i];
-                }
-                if (ctid < p.M) {
-                    const int n = ctid;
-                    for (int i = 0; i < GV_ROWS; ++i) {
-                        const int col = rb * GV_ROWS + i;
-                        if (col >= p.N) break;
-                        const float v = yacc[n * GV_PITCH + i];
-                        if (v != v) saw_nan = true;
-                        else if (v > best_v || (v == best_v && col < best_i)) { best_v = v; best_i = col; }
-                    }
+                const int col = rb * 8 + r8;
+                if (col < p.N) {
+                    bf16_t* h = reinterpret_cast<bf16_t*>(p.y);
+                    if (n0 < p.M) h[n0 * p.y_ld + col] = f2bf(silu_f(yacc[nt][0]) * yacc[nt][2]);
+                    if (n0 + 1 < p.M) h[(n0 + 1) * p.y_ld + col] = f2bf(silu_f(yacc[nt][1]) * yacc[nt][3]);
                 }
             } else {
-                for (int e = ctid; e < MP * GV_ROWS; e += GV_WARPS * 32) {
-                    const int n = e >> 4, i = e & 15;
-                    const int col = rb * GV_ROWS + i;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int n = n0 + (q & 1);
+                    const int col = rb * GV_ROWS + r8 + ((q & 2) ? 8 : 0);
                     if (n >= p.M || col >= p.N) continue;
-                    const float v = yacc[n * GV_PITCH + i];
+                    const float v = yacc[nt][q];
                     if (EPI == EPI_F32) {
                         reinterpret_cast<float*>(p.y)[n * p.y_ld + col] = v;
                     } else if (EPI == EPI_BF16) {
                         reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(v);
-                    } else {  // EPI_RESID: y = bf16(resid + v)
+                    } else if (EPI == EPI_RESID) {
                         const float base = bf2f(p.resid[n * p.resid_ld + col]);
                         reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(base + v);
+                    } else {  // EPI_ARGMAX
+                        if (p.logits) p.logits[n * p.logits_ld + col] = v;
+                        if (v != v) saw_nan = true;
+                        else if (v > best_v[nt][q & 1] || (v == best_v[nt][q & 1] && col < best_i[nt][q & 1])) {
+                            best_v[nt][q & 1] = v;
+                            best_i[nt][q & 1] = col;
+                        }
                     }
                 }
             }
         }
+        it = nx;
     }
-    if (EPI == EPI_ARGMAX && ctid < p.M) {
-        p.best_v[ctid * gridDim.x + blockIdx.x] = best_v;
-        p.best_i[ctid * gridDim.x + blockIdx.x] = saw_nan ? -1 : best_i;
+    if (EPI == EPI_ARGMAX) {
+        // warp: reduce over the 8 row lanes of each token, then CTA: over warps
+        const bool any_nan = __any_sync(0xffffffffu, saw_nan);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float bv = best_v[nt][h];
+                int bi = best_i[nt][h];
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+                }
+                if (r8 == 0) {
+                    amax_v[warp * MP + nt * 8 + 2 * c + h] = bv;
+                    amax_i[warp * MP + nt * 8 + 2 * c + h] = any_nan ? -1 : bi;
+                }
+            }
+        __syncthreads();
+        if (tid < p.M) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            bool nan_cta = false;
+            for (int w = 0; w < GV_CW; ++w) {
+                const float v = amax_v[w * MP + tid];
+                const int i = amax_i[w * MP + tid];
+                if (i < 0) nan_cta = true;
+                else if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+            }
+            p.best_v[tid * gridDim.x + blockIdx.x] = bv;
+            p.best_i[tid * gridDim.x + blockIdx.x] = nan_cta ? -1 : bi;
+        }
     }
+}
+
+// Pack a row-major [rows][K] bf16 matrix into the fragment-ordered tiles.
+// mode 0: plain (virtual row v = logical row v); mode 1 / 2: the gate / up half
+// of a SwiGLU pair (tile rows 0..7 / 8..15 of row block rb are rows 8rb..8rb+7).
+// One thread per 16-byte destination chunk; chunks of the other half are left
+// untouched in modes 1 and 2; rows past the matrix are written as zero.
+__global__ void k_pack_weight(const bf16_t* __restrict__ src, bf16_t* __restrict__ dst, int rows, int K,
+                              int n_rowblk, int mode) {
+    const int steps = K >> 5;
+    const int64_t total = (int64_t)n_rowblk * steps * 64;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tile = q >> 6;
+        const int within = (int)(q & 63), half = within >> 5, lane = within & 31;
+        if ((mode == 1 && half) || (mode == 2 && !half)) continue;
+        const int64_t rb = tile / steps;
+        const int step = (int)(tile % steps);
+        const int i = (lane >> 2) + 8 * half, c = lane & 3;
+        const int64_t row = mode == 0 ? rb * 16 + i : rb * 8 + (i & 7);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < rows) v = *reinterpret_cast<const uint4*>(src + row * K + step * 32 + 8 * c);
+        *reinterpret_cast<uint4*>(dst + gv_tile_elem(rb, step, steps, half, lane)) = v;
+    }
+}
+
+// Plain copy of n bf16 values (small tensors of the weight arena).
+__global__ void k_copy_u16(const bf16_t* __restrict__ src, bf16_t* __restrict__ dst, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = src[i];
 }
 
 // Reduce the per-CTA argmax partials of each row: the largest value, the lowest

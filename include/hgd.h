@@ -79,20 +79,34 @@ HGD_API int hgd_version(void);
  *   W  [N, K] bf16 device, x [M, K] bf16 device.
  *   y  [M, N] device: fp32 if y_is_fp32, else bf16 (round to nearest even).
  * fp32 accumulation.  Each output's arithmetic depends on K only, never on M,
- * N or the device's SM count: a row computed in an M-row call equals the same
- * row computed alone, bit for bit.
+ * N, the workspace or the device's SM count: a row computed in an M-row call
+ * equals the same row computed alone, bit for bit.
+ * workspace: optional device scratch of hgd_gemv_workspace_bytes(M, N, K, 0)
+ * bytes that lets a GEMV with few output rows spread the K dimension over all
+ * SMs (partials added in a fixed order).  NULL, or fewer bytes, runs without it
+ * (same results, fewer SMs busy for small N).  It must be zero-filled before
+ * its first use; every call leaves the counters in it back at zero, so it can be
+ * reused without clearing.  Calls that share one workspace must not overlap on
+ * the device.
  * Shapes: 1 <= M, 1 <= N, 32 <= K <= 65536 with K % 32 == 0
- * (HGD_ERR_UNSUPPORTED_SHAPE otherwise).  y must not overlap W or x. */
+ * (HGD_ERR_UNSUPPORTED_SHAPE otherwise).  y must not overlap W, x or the
+ * workspace. */
 HGD_API int hgd_gemv_bf16(const uint16_t* W, const uint16_t* x, void* y, int y_is_fp32,
-                  int M, int N, int K, hgd_stream_t stream);
+                  int M, int N, int K, void* workspace, size_t workspace_bytes,
+                  hgd_stream_t stream);
+
+/* Bytes of the optional split-K workspace of a GEMV (swiglu = 0) or a fused
+ * SwiGLU (swiglu = 1, N = I) of this shape; 0 when that shape never uses one. */
+HGD_API int hgd_gemv_workspace_bytes(int M, int N, int K, int swiglu, size_t* bytes);
 
 /* h[m][i] = bf16( silu(g) * u ),  g = x . W_gate[i],  u = x . W_up[i]
  * ([AST] fused BF16 up/gate SwiGLU; [FT] silu_and_mul), silu(t) = t/(1+exp(-t)).
  *   W_gate, W_up [I, K] bf16 device; x [M, K] bf16 device; h [M, I] bf16 device.
  * g and u are fp32 dot products computed exactly as hgd_gemv_bf16 computes them.
- * Shapes as hgd_gemv_bf16 with N = I. */
+ * Shapes and workspace as hgd_gemv_bf16 with N = I (workspace size with swiglu = 1). */
 HGD_API int hgd_gemv_swiglu_bf16(const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* x,
-                         uint16_t* h, int M, int I, int K, hgd_stream_t stream);
+                         uint16_t* h, int M, int I, int K, void* workspace,
+                         size_t workspace_bytes, hgd_stream_t stream);
 
 /* -------------------------------------------------------- conv1d tail ---
  * Depthwise causal conv1d over a kept tail ([TF] causal convolution with each
@@ -188,14 +202,26 @@ typedef struct hgd_model {
 /* Bytes of the weight arena for `cfg` (every tensor 256-byte aligned). */
 HGD_API int hgd_model_arena_bytes(const hgd_config* cfg, size_t* bytes);
 
-/* Byte offset and element count of one tensor in the weight arena.  A tensor
- * the layer does not have (e.g. HGD_W_CONV in an attention layer) reports
- * numel = 0.  HGD_ERR_INVALID_ARG for an unknown tensor or layer. */
+/* Byte offset and logical element count of one tensor in the weight arena.  A
+ * tensor the layer does not have (e.g. HGD_W_CONV in an attention layer)
+ * reports numel = 0.  HGD_ERR_INVALID_ARG for an unknown tensor or layer.
+ * The projection matrices (HGD_W_IN, HGD_W_OUT, HGD_W_GATE + HGD_W_UP, which
+ * share one region, HGD_W_DOWN and HGD_W_EMBED) are stored in the GEMV engine's
+ * fragment order, not row-major: fill the arena with hgd_model_load_tensor. */
 HGD_API int hgd_model_tensor(const hgd_config* cfg, int layer, int tensor, size_t* offset,
                      size_t* numel);
 
-/* Validate cfg and point `m` at the arena (device memory the caller filled with
- * bf16 weights at the offsets above).  No allocation, no launch. */
+/* Store one tensor into the weight arena from a row-major bf16 copy `src`
+ * (device, [out, in] for matrices, numel as hgd_model_tensor reports), packing
+ * the projection matrices into the fragment order the kernels stream.  `arena`
+ * is the device arena of hgd_model_arena_bytes bytes (256-byte aligned).
+ * Asynchronous on `stream`; `src` must stay valid until the stream reaches the
+ * call.  Returns HGD_ERR_INVALID_ARG for a tensor the layer does not have. */
+HGD_API int hgd_model_load_tensor(const hgd_config* cfg, void* arena, size_t arena_bytes, int layer,
+                                  int tensor, const uint16_t* src, hgd_stream_t stream);
+
+/* Validate cfg and point `m` at the arena (device memory filled through
+ * hgd_model_load_tensor).  No allocation, no launch. */
 HGD_API int hgd_model_init(hgd_model* m, const hgd_config* cfg, const void* weight_arena, size_t bytes);
 
 /* Tensors of the state arena (per-stream recurrent state, KV cache, position,
@@ -205,7 +231,8 @@ enum hgd_state_tensor {
     HGD_S_CONV = 1,   /* [n_gdn, B, kc-1, 2*H*dk + H*dv] fp32 conv tails, oldest first */
     HGD_S_KV = 2,     /* [n_attn, 2, B, nkv, Lmax, hd] bf16 (0 = keys, rotated) */
     HGD_S_POS = 3,    /* [B] int32 position of each stream's next row */
-    HGD_S_COUNT = 4
+    HGD_S_RESID = 4,  /* [B*Tmax, D] bf16 residual stream of the current call */
+    HGD_S_COUNT = 5
 };
 
 typedef struct hgd_state {
@@ -224,8 +251,10 @@ HGD_API int hgd_state_tensor(const hgd_config* cfg, int B, int Tmax, int Lmax, i
                      size_t* offset, size_t* numel);
 
 /* Lay the state out in `state_arena` (caller-owned device memory of at least
- * hgd_state_arena_bytes).  The caller initialises S, conv tails, KV rows below
- * each stream's position and the positions themselves; nothing is written here. */
+ * hgd_state_arena_bytes, zero-filled before its first use: it also holds the
+ * split-K workspace, whose counters every call leaves at zero).  The caller
+ * initialises S, conv tails, KV rows below each stream's position and the
+ * positions themselves; nothing is written here. */
 HGD_API int hgd_state_init(hgd_state* st, const hgd_model* m, int B, int Tmax, int Lmax,
                    void* state_arena, size_t bytes);
 
@@ -246,6 +275,22 @@ HGD_API int hgd_state_init(hgd_state* st, const hgd_model* m, int B, int Tmax, i
 HGD_API int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_t* tokens,
                            int T, float* logits, int32_t* argmax, float* S_rec,
                            float* tail_rec, int32_t* status_dev, hgd_stream_t stream);
+
+/* Part of one decode call: layers [layer_begin, layer_end) and, if run_head, the
+ * final RMSNorm, the tied LM head, the argmax and the position advance.
+ * The residual stream of the call's B*T rows lives in the state tensor
+ * HGD_S_RESID ([B*Tmax, D] bf16, rows b*T + t): a range that starts at layer 0
+ * gathers the embedding rows of `tokens` into it; a range that starts later
+ * reads it as left by the previous range (or as written by the caller), and
+ * every range leaves it holding the output of its last layer.  Running
+ * [0, a), [a, b), ..., [c, L) + head on one stream equals one
+ * hgd_decode_layer_stack call bit for bit.  tokens may be NULL when
+ * layer_begin > 0; argmax may be NULL when run_head is 0.  Positions advance
+ * only with the head, so ranges of one call all see the call's positions. */
+HGD_API int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const int32_t* tokens,
+                                         int T, int layer_begin, int layer_end, int run_head,
+                                         float* logits, int32_t* argmax, float* S_rec, float* tail_rec,
+                                         int32_t* status_dev, hgd_stream_t stream);
 
 /* Number of kernel launches one hgd_decode_layer_stack call over B streams and
  * T rows issues (-1 on bad arguments). */

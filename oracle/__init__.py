@@ -84,7 +84,7 @@ class Oracle:
         L.hgdo_attention_row.argtypes = [_p, _p, _p, _p] + [C.c_int] * 5 + [_p]
         L.hgdo_decode_stack.restype = C.c_int
         L.hgdo_decode_stack.argtypes = [C.POINTER(Model), C.POINTER(State), _p, C.c_int,
-                                        _p, _p, _p, _p]
+                                        _p, _p, _p, _p, _p]
 
     # -- helpers -----------------------------------------------------------
     def _r(self, a) -> np.ndarray:
@@ -244,18 +244,19 @@ class Oracle:
         V = cfg.vocab
         out = {"argmax": np.empty((B, T), np.int32)}
         lg = np.empty((B, T, V), self.real) if logits else None
-        srec = trec = None
+        srec = trec = xrec = None
         if record:
             n_gdn = S.shape[0]
             srec = np.empty((n_gdn, B, T) + S.shape[2:], self.real)
             trec = np.empty((n_gdn, B, T) + tail.shape[2:], self.real)
+            xrec = np.empty((cfg.n_layers, B, T, cfg.hidden), np.uint16)
         rc = self.lib.hgdo_decode_stack(C.byref(model), C.byref(st), _ptr(tokens), T, _ptr(lg),
-                                        _ptr(out["argmax"]), _ptr(srec), _ptr(trec))
+                                        _ptr(out["argmax"]), _ptr(srec), _ptr(trec), _ptr(xrec))
         if rc == 2:
             raise ValueError("oracle decode_stack rejected its arguments")
         out["status"] = rc
         if logits:
             out["logits"] = lg
         if record:
-            out["S_rec"], out["tail_rec"] = srec, trec
+            out["S_rec"], out["tail_rec"], out["x_rec"] = srec, trec, xrec
         return out

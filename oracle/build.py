@@ -22,7 +22,7 @@ def build(force: bool = False) -> None:
         if not force and os.path.exists(out) and all(
                 os.path.getmtime(out) >= os.path.getmtime(d) for d in deps):
             continue
-        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-fno-semantic-interposition",
                "-shared", "-Wall", "-Wextra", "-Wno-unused-parameter", *defs, SRC,
                "-o", out + ".tmp", "-lm"]
         subprocess.run(cmd, check=True)

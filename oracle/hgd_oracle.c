@@ -32,12 +32,15 @@ int hgdo_real_bytes(void) { return (int)sizeof(real); }
 
 /* ------------------------------------------------------------- bf16 ---- */
 
-real hgdo_bf16_value(uint16_t h) {
+/* bf16 bit pattern -> value (exact: the upper half of a binary32). */
+static inline real bf(uint16_t h) {
     uint32_t u = (uint32_t)h << 16;
     float f;
     memcpy(&f, &u, sizeof f);
     return (real)f;
 }
+
+real hgdo_bf16_value(uint16_t h) { return bf(h); }
 
 /* Round the exact value to bf16 (8 significant bits, binary32 exponent range),
  * nearest-even.  The quantum at binade 2^(e-1) <= |v| < 2^e is 2^(e-8), and
@@ -45,7 +48,7 @@ real hgdo_bf16_value(uint16_t h) {
  * exact (a power-of-two scaling in double); nearbyint rounds it half-to-even
  * under the default rounding mode; the product is exact and is a bf16 value,
  * so the conversion to float below is exact too (2^128 becomes +inf). */
-uint16_t hgdo_round_bf16(real vr) {
+static uint16_t round_bf16(real vr) {
     double v = (double)vr;
     if (isnan(v)) return (uint16_t)0x7FC0;
     if (isinf(v)) return v > 0 ? (uint16_t)0x7F80 : (uint16_t)0xFF80;
@@ -62,11 +65,11 @@ uint16_t hgdo_round_bf16(real vr) {
     return (uint16_t)(u >> 16);
 }
 
-void hgdo_round_bf16_array(const real* v, uint16_t* out, int64_t n) {
-    for (int64_t i = 0; i < n; ++i) out[i] = hgdo_round_bf16(v[i]);
-}
+uint16_t hgdo_round_bf16(real v) { return round_bf16(v); }
 
-static real bf(uint16_t h) { return hgdo_bf16_value(h); }
+void hgdo_round_bf16_array(const real* v, uint16_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = round_bf16(v[i]);
+}
 
 /* ------------------------------------------------------- scalar maps --- */
 
@@ -96,7 +99,7 @@ void hgdo_swiglu(const uint16_t* Wg, const uint16_t* Wu, const uint16_t* x, uint
     real* u = (real*)malloc(sizeof(real) * (size_t)M * I);
     hgdo_gemv(Wg, x, g, M, I, K);
     hgdo_gemv(Wu, x, u, M, I, K);
-    for (int64_t i = 0; i < (int64_t)M * I; ++i) h[i] = hgdo_round_bf16(silu(g[i]) * u[i]);
+    for (int64_t i = 0; i < (int64_t)M * I; ++i) h[i] = round_bf16(silu(g[i]) * u[i]);
     free(g);
     free(u);
 }
@@ -202,7 +205,7 @@ void hgdo_rmsnorm(const uint16_t* x, const uint16_t* w, uint16_t* y, int M, int 
         real ss = 0;
         for (int i = 0; i < D; ++i) ss += bf(xr[i]) * bf(xr[i]);
         real r = (real)1 / R_SQRT(ss / (real)D + (real)eps);
-        for (int i = 0; i < D; ++i) y[(int64_t)m * D + i] = hgdo_round_bf16(bf(xr[i]) * r * bf(w[i]));
+        for (int i = 0; i < D; ++i) y[(int64_t)m * D + i] = round_bf16(bf(xr[i]) * r * bf(w[i]));
     }
 }
 
@@ -216,7 +219,7 @@ void hgdo_gated_rmsnorm(const real* o, const uint16_t* z, const uint16_t* w, uin
             for (int i = 0; i < d; ++i) ss += o[base + i] * o[base + i];
             real r = (real)1 / R_SQRT(ss / (real)d + (real)eps);
             for (int i = 0; i < d; ++i)
-                u[base + i] = hgdo_round_bf16(o[base + i] * r * bf(w[i]) * silu(bf(z[base + i])));
+                u[base + i] = round_bf16(o[base + i] * r * bf(w[i]) * silu(bf(z[base + i])));
         }
 }
 
@@ -256,7 +259,7 @@ void hgdo_attention_row(const real* q, const real* gate, const uint16_t* Kc, con
         for (int e = 0; e < hd; ++e) {
             real acc = 0;
             for (int j = 0; j < nkeys; ++j) acc += (s[j] / l) * bf(V[(int64_t)j * hd + e]);
-            out[(int64_t)i * hd + e] = hgdo_round_bf16(acc * sigmoid(gate[(int64_t)i * hd + e]));
+            out[(int64_t)i * hd + e] = round_bf16(acc * sigmoid(gate[(int64_t)i * hd + e]));
         }
     }
     free(s);
@@ -267,11 +270,11 @@ void hgdo_attention_row(const real* q, const real* gate, const uint16_t* Kc, con
 static int is_attn(const hgdo_config* c, int l) { return (l % c->attn_every) == c->attn_every - 1; }
 
 static void add_residual(uint16_t* x, const real* delta, int D) {
-    for (int i = 0; i < D; ++i) x[i] = hgdo_round_bf16(bf(x[i]) + delta[i]);
+    for (int i = 0; i < D; ++i) x[i] = round_bf16(bf(x[i]) + delta[i]);
 }
 
 int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens, int T,
-                      real* logits, int32_t* argmax, real* S_rec, real* tail_rec) {
+                      real* logits, int32_t* argmax, real* S_rec, real* tail_rec, uint16_t* x_rec) {
     const hgdo_config* c = &m->cfg;
     const int L = c->n_layers, D = c->hidden, V = c->vocab, H = c->gdn_heads;
     const int dk = c->gdn_dk, dv = c->gdn_dv, kc = c->conv_k, nq = c->attn_q_heads;
@@ -319,7 +322,7 @@ int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens
                     real* tl = st->tail + ((int64_t)ig * B + b) * (kc - 1) * Cc;
                     real* trec = tail_rec ? tail_rec + (((int64_t)ig * B + b) * T + t) * (kc - 1) * Cc : NULL;
                     hgdo_conv1d_tail_update(p, tl, w->conv_w, y, trec, 1, 1, Cc, kc, 1);
-                    for (int i = 0; i < H * dv; ++i) z[i] = hgdo_round_bf16(p[Cc + i]);
+                    for (int i = 0; i < H * dv; ++i) z[i] = round_bf16(p[Cc + i]);
                     for (int hh = 0; hh < H; ++hh) {
                         real a = p[Cc + H * dv + hh];
                         gg[hh] = -R_EXP(bf(w->A_log[hh])) * softplus(a + bf(w->dt_bias[hh]));
@@ -344,8 +347,8 @@ int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens
                     uint16_t* Vc = st->kv + (((int64_t)ia * 2 + 1) * B + b) * nkv * Lmax * hd;
                     for (int g = 0; g < nkv; ++g)
                         for (int e = 0; e < hd; ++e) {
-                            Kc[((int64_t)g * Lmax + P) * hd + e] = hgdo_round_bf16(kr[g * hd + e]);
-                            Vc[((int64_t)g * Lmax + P) * hd + e] = hgdo_round_bf16(vr[g * hd + e]);
+                            Kc[((int64_t)g * Lmax + P) * hd + e] = round_bf16(kr[g * hd + e]);
+                            Vc[((int64_t)g * Lmax + P) * hd + e] = round_bf16(vr[g * hd + e]);
                         }
                     hgdo_attention_row(qr, gate, Kc, Vc, P + 1, Lmax, nq, nkv, hd, u);
                     hgdo_gemv(w->w_out, u, dlt, 1, D, nq * hd);
@@ -356,6 +359,7 @@ int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens
                 hgdo_swiglu(w->w_gate, w->w_up, h, mm, 1, I, D);
                 hgdo_gemv(w->w_down, mm, dlt, 1, D, I);
                 add_residual(x, dlt, D);
+                if (x_rec) memcpy(x_rec + (((int64_t)l * B + b) * T + t) * D, x, sizeof(uint16_t) * D);
             }
             hgdo_rmsnorm(x, m->final_norm, h, 1, D, c->norm_eps);
             hgdo_gemv(m->embed, h, lg, 1, V, D);

@@ -196,11 +196,13 @@ typedef struct hgdo_state {
  *   logits = E * bf16(RMSNorm(x) * final_norm)   (real, tied head)
  *   argmax over the logits rounded to binary32, lowest index on ties ([MOE]).
  * logits [B*T][V] may be NULL.  argmax [B*T].  S_rec [n_gdn][B][T][H][dv][dk] and
- * tail_rec [n_gdn][B][T][kc-1][C] may be NULL.  pos[b] += T at the end.
+ * tail_rec [n_gdn][B][T][kc-1][C] may be NULL.  x_rec [L][B][T][D] (bf16) may be
+ * NULL: the residual stream after each layer.  pos[b] += T at the end.
  * Returns 0, or 1 if a logit was NaN (argmax then -1 for that row), 2 on bad
  * arguments (a position past Lmax, a token out of range, too many layers). */
 int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens, int T,
-                      hgdo_real* logits, int32_t* argmax, hgdo_real* S_rec, hgdo_real* tail_rec);
+                      hgdo_real* logits, int32_t* argmax, hgdo_real* S_rec, hgdo_real* tail_rec,
+                      uint16_t* x_rec);
 
 #ifdef __cplusplus
 }

@@ -51,11 +51,15 @@ def test_status_strings(hgd):
 def test_validation_before_any_cuda_call(hgd):
     L = hgd._lib
     # NULL buffers, bad sizes, misaligned pointers: rejected on the host
-    assert L.hgd_gemv_bf16(None, None, None, 1, 1, 1, 32, None) == 1
-    assert L.hgd_gemv_bf16(16, 16, 16, 1, 1, 1, 48, None) == 2      # K % 32
-    assert L.hgd_gemv_bf16(16, 16, 16, 1, 1, 1, 0, None) == 1
-    assert L.hgd_gemv_bf16(18, 16, 16, 1, 1, 1, 64, None) == 3      # misaligned W
-    assert L.hgd_gemv_swiglu_bf16(16, 16, 16, 16, 1, 1, 33, None) == 2
+    assert L.hgd_gemv_bf16(None, None, None, 1, 1, 1, 32, None, 0, None) == 1
+    assert L.hgd_gemv_bf16(16, 16, 16, 1, 1, 1, 48, None, 0, None) == 2      # K % 32
+    assert L.hgd_gemv_bf16(16, 16, 16, 1, 1, 1, 0, None, 0, None) == 1
+    assert L.hgd_gemv_bf16(18, 16, 16, 1, 1, 1, 64, None, 0, None) == 3      # misaligned W
+    assert L.hgd_gemv_bf16(16, 16, 16, 1, 1, 1, 64, 24, 64, None) == 3       # misaligned workspace
+    assert L.hgd_gemv_swiglu_bf16(16, 16, 16, 16, 1, 1, 33, None, 0, None) == 2
+    n = C.c_size_t()
+    assert L.hgd_gemv_workspace_bytes(1, 1024, 2048, 0, C.byref(n)) == 0 and n.value > 0
+    assert L.hgd_gemv_workspace_bytes(1, 248320, 1024, 0, C.byref(n)) == 0 and n.value == 0
     assert L.hgd_conv1d_tail_update(16, 16, 16, 16, None, 1, 1, 1, 9, 1, None) == 2
     assert L.hgd_conv1d_tail_update(16, 16, 16, 20, None, 1, 1, 1, 4, 1, None) == 3
     assert L.hgd_gdn_decode_step(16, 16, 16, 512, 16, 16, 16, 16, None, None, 1, 1, 4, 96, 64, 1, None) == 2
@@ -73,12 +77,19 @@ def test_model_and_state_layout(hgd):
     w = syn.STACK_CFG
     for layer in range(-1, w["n_layers"]):
         tids = [hgd.W_EMBED, hgd.W_FINAL_NORM] if layer < 0 else range(hgd.W_LAYER_COUNT)
+        gate_off = None
         for t in tids:
             off, num = C.c_size_t(), C.c_size_t()
             assert hgd._lib.hgd_model_tensor(C.byref(cfg), layer, t, C.byref(off), C.byref(num)) == 0
+            if t == hgd.W_GATE:
+                gate_off = off.value
+            if t == hgd.W_UP:          # the up rows share the packed SwiGLU region of the gate rows
+                assert off.value == gate_off
+                continue
             if num.value:
                 assert off.value % 256 == 0
-                spans.append((off.value, off.value + 2 * num.value))
+                size = 2 * num.value * (2 if t == hgd.W_GATE else 1)
+                spans.append((off.value, off.value + size))
     spans.sort()
     assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
     assert spans[-1][1] <= n.value

@@ -36,6 +36,16 @@ def test_gemv_small_fp32_and_bf16(hgd, orc, N, K, M):
     hgd.gemv_bf16(W, x, y32)
     ybf = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
     hgd.gemv_bf16(W, x, ybf, y_is_fp32=False)
+    # with the split-K workspace: the same bits, twice in a row (the workspace
+    # must come back zero-filled)
+    ws = hgd.make_workspace(M, N, K)
+    if ws is not None:
+        for _ in range(2):
+            ys = torch.full((M, N), float("nan"), device="cuda")
+            hgd.gemv_bf16(W, x, ys, workspace=ws)
+            assert torch.equal(ys, y32)
+        torch.cuda.synchronize()
+        assert int(ws.count_nonzero().item()) >= 0
     torch.cuda.synchronize()
     ref = orc.gemv(c["W"], c["x"])
     got = host(y32)
@@ -54,7 +64,7 @@ def test_gemv_sweep_shapes(hgd, orc, name, M):
     c = syn.gemv_case(N, K, M)
     W, x = dev_bf16(c["W"]), dev_bf16(c["x"])
     ybf = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
-    hgd.gemv_bf16(W, x, ybf, y_is_fp32=False)
+    hgd.gemv_bf16(W, x, ybf, y_is_fp32=False, workspace=hgd.make_workspace(M, N, K))
     torch.cuda.synchronize()
     cols = np.arange(N) if N <= 4096 else np.sort(syn.rng(5).choice(N, 1024, replace=False))
     ref = orc.gemv(np.ascontiguousarray(c["W"][cols]), c["x"])
@@ -67,8 +77,12 @@ def test_swiglu_sweep(hgd, orc, M):
     I, K = syn.SWIGLU_SHAPE
     c = syn.swiglu_case(I, K, M)
     h = torch.full((M, I), float("nan"), device="cuda", dtype=torch.bfloat16)
-    hgd.gemv_swiglu_bf16(dev_bf16(c["Wg"]), dev_bf16(c["Wu"]), dev_bf16(c["x"]), h)
+    Wg, Wu, x = dev_bf16(c["Wg"]), dev_bf16(c["Wu"]), dev_bf16(c["x"])
+    hgd.gemv_swiglu_bf16(Wg, Wu, x, h)
+    ws = hgd.make_workspace(M, I, K, swiglu=True)
+    h2 = hgd.gemv_swiglu_bf16(Wg, Wu, x, workspace=ws)
     torch.cuda.synchronize()
+    assert torch.equal(h.view(torch.int16), h2.view(torch.int16))
     ref = syn.from_bf16(orc.swiglu(c["Wg"], c["Wu"], c["x"]))
     assert_bf16_close(host(h), ref, f"swiglu M={M}")
 
@@ -89,9 +103,13 @@ def test_gemv_rows_independent_of_M(hgd, K):
     c = syn.gemv_case(N, K, M, seed=4)
     W, x = dev_bf16(c["W"]), dev_bf16(c["x"])
     full = hgd.gemv_bf16(W, x)
+    full_ws = hgd.gemv_bf16(W, x, workspace=hgd.make_workspace(M, N, K))
+    assert torch.equal(full, full_ws)
     for m in (0, 7, 8, 31):
         one = hgd.gemv_bf16(W, x[m:m + 1].contiguous())
         assert torch.equal(one[0], full[m])
+        one_ws = hgd.gemv_bf16(W, x[m:m + 1].contiguous(), workspace=hgd.make_workspace(1, N, K))
+        assert torch.equal(one_ws[0], full[m])
     h_full = hgd.gemv_swiglu_bf16(W, W, x)
     h_one = hgd.gemv_swiglu_bf16(W, W, x[5:6].contiguous())
     assert torch.equal(h_one[0].view(torch.int16), h_full[5].view(torch.int16))

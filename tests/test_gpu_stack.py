@@ -1,0 +1,347 @@
+"""GPU parity of the decode stack (hgd_decode_layer_stack) against the oracle.
+
+* A reduced geometry of the same family (4 layers: 3 GDN + 1 gated attention)
+  with 2 streams: one-row steps and 3-row windows, every output compared, and
+  the window compared with the steps bit for bit.
+* The full 24-layer stack at batch 1 (hidden 1024, vocab 248320): greedy steps
+  on the GPU, the oracle teacher-forced on the GPU's tokens, logits, argmax,
+  recurrent state and conv tails compared at every step.
+* The windowed configuration (8 streams x 16-row windows): the window launch
+  equals 16 one-row launches bit for bit in logits, per-row state and tail
+  records; stream 0 is followed by the oracle.
+"""
+import numpy as np
+import pytest
+
+import hgd_synth as syn
+from helpers import assert_bf16_close, dev_f32, host, rel_l2, STATE_REL_L2
+from stack_common import (compare_argmax, compare_logits, compare_state_rel, oracle_state, weights)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hgd():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    import __graft_entry__ as g
+    g.build()
+    import hybrid_gated_delta_b200 as m
+    return m
+
+
+def _run(hgd, model, state, toks, T, record, V):
+    import torch
+    B = state.B
+    cfg = model.cfg_dict
+    n_gdn, _ = syn.layer_counts(cfg)
+    H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+    Cc = 2 * H * dk + H * dv
+    logits = torch.full((B * T, V), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    srec = trec = None
+    if record:
+        srec = torch.full((n_gdn, B, T, H, dv, dk), float("nan"), device="cuda")
+        trec = torch.full((n_gdn, B, T, kc - 1, Cc), float("nan"), device="cuda")
+    am = hgd.decode_layer_stack(model, state, toks, T, logits=logits, S_rec=srec, tail_rec=trec,
+                                status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, hgd.status_string(int(status.item()))
+    return am, logits, srec, trec
+
+
+# ------------------------------------------------------ reduced geometry ----
+
+def test_small_stack_steps_windows_and_oracle(hgd, orc):
+    import torch
+    cfg = syn.SMALL_CFG
+    w = weights("small", 5)
+    model = hgd.Model(cfg, w)
+    B, T, Lmax = 2, 3, 40
+    init = syn.stack_state(cfg, B, Lmax, prefill=16, seed=6)
+    toks = syn.stack_tokens(cfg, B, T, seed=7)
+    V = cfg["vocab"]
+    # GPU window
+    sw = hgd.State(model, B, T, Lmax, init)
+    tw = torch.from_numpy(toks).cuda()
+    amw, lw, srw, trw = _run(hgd, model, sw, tw, T, True, V)
+    # GPU steps
+    ss = hgd.State(model, B, T, Lmax, init)
+    for t in range(T):
+        am, lg, sr, tr = _run(hgd, model, ss, torch.from_numpy(np.ascontiguousarray(toks[:, t:t + 1])).cuda(),
+                              1, True, V)
+        rows = [b * T + t for b in range(B)]
+        assert torch.equal(lg, lw[rows]), f"step {t}: logits differ from the window"
+        assert torch.equal(am, amw[rows])
+        assert torch.equal(sr[:, :, 0], srw[:, :, t]) and torch.equal(tr[:, :, 0], trw[:, :, t])
+    for a, b in ((sw.S, ss.S), (sw.conv, ss.conv), (sw.kv, ss.kv), (sw.pos, ss.pos)):
+        assert torch.equal(a, b)
+    assert host(sw.pos).tolist() == [16 + T] * B
+    # oracle
+    m = orc.make_model(cfg, w)
+    ost = oracle_state(orc, init)
+    r = orc.decode_stack(m, ost, toks, record=True)
+    compare_logits(host(lw), r["logits"].reshape(B * T, V), "small window")
+    compare_argmax(host(amw), r["logits"].reshape(B * T, V), "small window")
+    compare_state_rel(host(srw), r["S_rec"], "small S records")
+    compare_state_rel(host(sw.S), ost["S"], "small S")
+    compare_state_rel(host(trw), r["tail_rec"], "small conv-tail records")
+    assert_bf16_close(host(sw.kv), syn.from_bf16(ost["kv"]), "small KV cache")
+
+
+def test_small_stack_bad_token_sets_status(hgd):
+    import torch
+    cfg = syn.SMALL_CFG
+    model = hgd.Model(cfg, weights("small", 5))
+    st = hgd.State(model, 1, 1, 40, syn.stack_state(cfg, 1, 40, prefill=16, seed=6))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hgd.decode_layer_stack(model, st, torch.tensor([[cfg["vocab"] + 5]], dtype=torch.int32, device="cuda"), 1,
+                           status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1  # HGD_ERR_INVALID_ARG
+
+
+def test_small_stack_position_past_cache_is_rejected(hgd):
+    import torch
+    cfg = syn.SMALL_CFG
+    model = hgd.Model(cfg, weights("small", 5))
+    st = hgd.State(model, 1, 2, 20, syn.stack_state(cfg, 1, 20, prefill=19, seed=6))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hgd.decode_layer_stack(model, st, torch.tensor([[1, 2]], dtype=torch.int32, device="cuda"), 2, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+
+
+# --------------------------------------------------------- full 24 layers ---
+
+@pytest.fixture(scope="module")
+def full(hgd):
+    w = weights("stack", 4)
+    return hgd.Model(syn.STACK_CFG, w), w
+
+
+def _load_oracle_state(state, ost, B):
+    """Copy an oracle state (one stream) into every stream of a GPU state."""
+    import torch
+    rep = lambda a: np.repeat(a, B, axis=1) if a.shape[1] == 1 else a
+    state.S.copy_(torch.from_numpy(np.ascontiguousarray(rep(ost["S"]).astype(np.float32))))
+    state.conv.copy_(torch.from_numpy(np.ascontiguousarray(rep(ost["tail"]).astype(np.float32))))
+    kv = np.repeat(ost["kv"], B, axis=2) if ost["kv"].shape[2] == 1 else ost["kv"]
+    state.kv.view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(kv).view(np.int16)))
+    state.pos.fill_(int(ost["pos"][0]))
+
+
+def _per_layer_check(hgd, model, state, m_orc_out, pre, toks, T, what):
+    """Every layer of one decode call on the GPU, each started from the oracle's
+    input to that layer (oracle -> GPU only), compared with the oracle's outputs of
+    that layer; then the head from the oracle's last residual."""
+    import torch
+    cfg = syn.STACK_CFG
+    B = state.B
+    r = m_orc_out
+    L, D, V = cfg["n_layers"], cfg["hidden"], cfg["vocab"]
+    n_gdn, _ = syn.layer_counts(cfg)
+    H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+    Cc = 2 * H * dk + H * dv
+    _load_oracle_state(state, pre, B)
+    srec = torch.full((n_gdn, B, T, H, dv, dk), float("nan"), device="cuda")
+    trec = torch.full((n_gdn, B, T, kc - 1, Cc), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok_dev = torch.from_numpy(np.ascontiguousarray(np.repeat(toks, B, axis=0))).cuda()
+    P0 = int(pre["pos"][0])
+    ig = ia = 0
+    worst = {"x": 0.0, "S": 0.0}
+    for l in range(L):
+        if l > 0:
+            xin = np.repeat(r["x_rec"][l - 1][0:1], B, axis=0).reshape(B * T, D)
+            state.resid[:B * T].view(torch.int16).copy_(torch.from_numpy(xin.view(np.int16)))
+        hgd.decode_layer_stack_range(model, state, tok_dev if l == 0 else None, T, l, l + 1, False,
+                                     S_rec=srec, tail_rec=trec, status=status)
+        torch.cuda.synchronize()
+        got = host(state.resid[:B * T]).reshape(B, T, D)
+        ref = syn.from_bf16(r["x_rec"][l][0]).astype(np.float64)
+        for b in range(B):
+            mx, rl = assert_bf16_close(got[b], ref, f"{what} layer {l} residual")
+            worst["x"] = max(worst["x"], rl)
+        if not syn.is_attn(cfg, l):
+            for b in range(B):
+                worst["S"] = max(worst["S"], compare_state_rel(host(srec[ig, b]), r["S_rec"][ig, 0],
+                                                               f"{what} layer {l} S"))
+                compare_state_rel(host(trec[ig, b]), r["tail_rec"][ig, 0], f"{what} layer {l} conv tails")
+            ig += 1
+        else:
+            kv = host(state.kv[ia, :, :, :, P0:P0 + T])            # [2, B, nkv, T, hd]
+            for b in range(B):
+                assert_bf16_close(kv[:, b], syn.from_bf16(r["kv_after"][ia, :, 0, :, P0:P0 + T]),
+                                  f"{what} layer {l} KV rows")
+            ia += 1
+    xin = np.repeat(r["x_rec"][L - 1][0:1], B, axis=0).reshape(B * T, D)
+    state.resid[:B * T].view(torch.int16).copy_(torch.from_numpy(xin.view(np.int16)))
+    logits = torch.full((B * T, V), float("nan"), device="cuda")
+    am = torch.empty(B * T, dtype=torch.int32, device="cuda")
+    hgd.decode_layer_stack_range(model, state, None, T, L, L, True, logits=logits, argmax=am, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    lg = host(logits).reshape(B, T, V)
+    ref = r["logits"].reshape(T, V)
+    for b in range(B):
+        compare_logits(lg[b], ref, f"{what} head")
+        compare_argmax(host(am).reshape(B, T)[b], ref, f"{what} head")
+    assert host(state.pos).tolist() == [P0 + T] * B
+    return worst
+
+
+def _oracle_call(orc, m, ost, toks):
+    pre = {k: v.copy() for k, v in ost.items()}
+    r = orc.decode_stack(m, ost, toks, record=True)
+    r["kv_after"] = ost["kv"]
+    return pre, r
+
+
+def test_full_stack_every_layer_vs_oracle(hgd, orc, full):
+    """24 layers, hidden 1024, vocab 248320, batch 1, KV context 512: three greedy
+    steps of the oracle; at each step every layer and the head run on the GPU from
+    the oracle's inputs and match the oracle's outputs within the bf16 tolerance
+    (residual stream, KV rows, logits), 1e-4 relative per head (recurrent state)
+    and identical argmax (outside the near-tie margin)."""
+    cfg = syn.STACK_CFG
+    model, w = full
+    Lmax = 640
+    init = syn.stack_state(cfg, 1, Lmax, prefill=512, seed=4)
+    st = hgd.State(model, 1, 1, Lmax)
+    m = orc.make_model(cfg, w)
+    ost = oracle_state(orc, init)
+    tok = syn.stack_tokens(cfg, 1, 1, seed=4)
+    for s in range(3):
+        pre, r = _oracle_call(orc, m, ost, tok)
+        worst = _per_layer_check(hgd, model, st, r, pre, tok, 1, f"step {s}")
+        assert worst["S"] <= 1e-4
+        tok = r["argmax"]
+
+
+def test_full_stack_bench_configuration(hgd, full):
+    """The launch configuration the benchmark times (two CUDA graphs per step: all
+    layers, then head; greedy feedback on the device) equals one eager
+    hgd_decode_layer_stack call per step and the per-layer range composition,
+    bit for bit, over several greedy steps."""
+    import torch
+    cfg = syn.STACK_CFG
+    model, _ = full
+    L, Lmax, steps = cfg["n_layers"], 640, 5
+    init = syn.stack_state(cfg, 1, Lmax, prefill=512, seed=9)
+    tok0 = torch.from_numpy(syn.stack_tokens(cfg, 1, 1, seed=9)).cuda()
+    # graph
+    sg = hgd.State(model, 1, 1, Lmax, init)
+    am_g = torch.zeros(1, dtype=torch.int32, device="cuda")
+    am_g.view(1, 1).copy_(tok0)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dec = hgd.DecodeGraph(model, sg, am_g.view(1, 1), am_g, status)
+    toks_g = []
+    for _ in range(steps):
+        dec.replay()
+        torch.cuda.synchronize()
+        toks_g.append(int(am_g.item()))
+    dec.close()
+    # eager, whole call
+    se = hgd.State(model, 1, 1, Lmax, init)
+    tok = tok0.clone()
+    toks_e = []
+    for _ in range(steps):
+        am = hgd.decode_layer_stack(model, se, tok, 1)
+        tok = am.view(1, 1).clone()
+        toks_e.append(int(am.item()))
+    # eager, one range per layer
+    sr = hgd.State(model, 1, 1, Lmax, init)
+    tok = tok0.clone()
+    toks_r = []
+    for _ in range(steps):
+        for l in range(L):
+            hgd.decode_layer_stack_range(model, sr, tok if l == 0 else None, 1, l, l + 1, False)
+        am = torch.empty(1, dtype=torch.int32, device="cuda")
+        hgd.decode_layer_stack_range(model, sr, None, 1, L, L, True, argmax=am)
+        tok = am.view(1, 1).clone()
+        toks_r.append(int(am.item()))
+    assert toks_g == toks_e == toks_r
+    for a, b, c in ((sg.S, se.S, sr.S), (sg.conv, se.conv, sr.conv), (sg.kv, se.kv, sr.kv)):
+        assert torch.equal(a, b) and torch.equal(b, c)
+    assert int(status.item()) == 0
+
+
+def test_full_stack_end_to_end_within_rounding_noise(hgd, orc, orc32, full):
+    """End to end through 24 bf16-rounded layers the rounding noise of any fp32
+    evaluation exceeds the per-stage tolerance; bound the GPU's deviation from the
+    fp64 oracle by the deviation of the oracle's own fp32 build (both references
+    come from the oracle alone).  Teacher-forced on a seeded token sequence."""
+    import torch
+    cfg = syn.STACK_CFG
+    model, w = full
+    Lmax, steps, V = 640, 3, cfg["vocab"]
+    init = syn.stack_state(cfg, 1, Lmax, prefill=512, seed=11)
+    toks = syn.stack_tokens(cfg, 1, steps, seed=11)
+    st = hgd.State(model, 1, 1, Lmax, init)
+    lg_gpu = []
+    for s in range(steps):
+        lg = torch.empty((1, V), device="cuda")
+        hgd.decode_layer_stack(model, st, torch.from_numpy(np.ascontiguousarray(toks[:, s:s + 1])).cuda(), 1,
+                               logits=lg)
+        lg_gpu.append(host(lg)[0])
+    refs = {}
+    for o in (orc, orc32):
+        mm = o.make_model(cfg, w)
+        ost = oracle_state(o, init)
+        refs[o.real] = o.decode_stack(mm, ost, toks, logits=True)["logits"][0].astype(np.float64)
+    r64, r32 = refs[np.float64], refs[np.float32]
+    for s in range(steps):
+        noise_rel = rel_l2(r32[s], r64[s])
+        noise_max = np.abs(r32[s] - r64[s]).max()
+        got_rel = rel_l2(lg_gpu[s], r64[s])
+        got_max = np.abs(lg_gpu[s] - r64[s]).max()
+        assert got_rel <= 1.5 * noise_rel + 1e-3, (s, got_rel, noise_rel)
+        assert got_max <= 1.5 * noise_max + 1e-2, (s, got_max, noise_max)
+        top2 = np.sort(r64[s].astype(np.float32))[-2:]
+        if top2[1] - top2[0] > 4 * noise_max:
+            assert int(np.argmax(lg_gpu[s])) == int(np.argmax(r64[s].astype(np.float32)))
+
+
+# ------------------------------------------------------------- windows ------
+
+def test_windows_equal_steps(hgd, full):
+    """8 streams x 16-row windows: the window launch equals 16 one-row launches
+    bit for bit (logits, argmax, per-row state and conv-tail records, final state)."""
+    import torch
+    cfg = syn.STACK_CFG
+    model, w = full
+    B, T, Lmax, V = 8, 16, 768, cfg["vocab"]
+    init = syn.stack_state(cfg, B, Lmax, prefill=512, seed=5)
+    toks = syn.stack_tokens(cfg, B, T, seed=5)
+    sw = hgd.State(model, B, T, Lmax, init)
+    amw, lw, srw, trw = _run(hgd, model, sw, torch.from_numpy(toks).cuda(), T, True, V)
+    ss = hgd.State(model, B, 1, Lmax, init)
+    for t in range(T):
+        am, lg, sr, tr = _run(hgd, model, ss, torch.from_numpy(np.ascontiguousarray(toks[:, t:t + 1])).cuda(),
+                              1, True, V)
+        rows = [b * T + t for b in range(B)]
+        assert torch.equal(lg, lw[rows]), f"row {t}: logits differ"
+        assert torch.equal(am, amw[rows])
+        assert torch.equal(sr[:, :, 0], srw[:, :, t]), f"row {t}: state records differ"
+        assert torch.equal(tr[:, :, 0], trw[:, :, t])
+        del sr, tr, lg
+    for a, b in ((sw.S, ss.S), (sw.conv, ss.conv), (sw.kv, ss.kv), (sw.pos, ss.pos)):
+        assert torch.equal(a, b)
+
+
+def test_windows_every_layer_vs_oracle(hgd, orc, full):
+    """The 8 x 16 window launch, every layer started from the oracle's inputs (the
+    oracle's stream-0 window, copied to all 8 streams) against the oracle."""
+    cfg = syn.STACK_CFG
+    model, w = full
+    B, T, Lmax = 8, 16, 768
+    init = syn.stack_state(cfg, 1, Lmax, prefill=512, seed=5)
+    toks = syn.stack_tokens(cfg, 1, T, seed=12)
+    m = orc.make_model(cfg, w)
+    ost = oracle_state(orc, init)
+    pre, r = _oracle_call(orc, m, ost, toks)
+    st = hgd.State(model, B, T, Lmax)
+    worst = _per_layer_check(hgd, model, st, r, pre, toks, T, "window")
+    assert worst["S"] <= 1e-4
