@@ -66,6 +66,7 @@ _SIGS = {
     "hgd_version": ([], _i),
     "hgd_gemv_bf16": ([_p, _p, _p, _i, _i, _i, _i, _p, _sz, _p], _i),
     "hgd_gemv_workspace_bytes": ([_i, _i, _i, _i, C.POINTER(_sz)], _i),
+    "hgd_gemv_bf16_static_ws": ([_p, _p, _p, _i, _i, _i, _i, _p], _i),
     "hgd_gemv_swiglu_bf16": ([_p, _p, _p, _p, _i, _i, _i, _p, _sz, _p], _i),
     "hgd_conv1d_tail_update": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),

@@ -769,3 +769,61 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
 }
 
 }  // extern "C"
+
+// ====================================================== allocation-free GEMV
+// Some callers cannot allocate device memory at all: a plugin hosted by a
+// framework that owns the device allocator and gives the plugin no handle to
+// it, or a latency-critical decode loop in which a cudaMalloc would synchronise
+// the device and stall every stream.  For them hgd_gemv_bf16_static_ws runs the
+// GEMV with its split-K scratch in a fixed array that is part of the library
+// image: nothing is allocated per call, and the caller passes only its inputs
+// and its output.  The array (kStaticWsBytes) lives on every device that loads
+// the library until the process exits, and every call shares it.
+
+namespace {
+
+constexpr size_t kStaticWsBytes = (size_t)4 << 20;  // 4 MiB of scratch per device
+static __device__ __align__(256) uint8_t g_gemv_static_ws[kStaticWsBytes];
+
+// Device address of the array on the current device, looked up once per device
+// (host code cannot use the symbol itself: it names a host-side stand-in).
+int static_ws_address(void** out) {
+    static void* addr[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HGD_ERR_CUDA; }
+    if (dev >= 0 && dev < 64 && addr[dev]) { *out = addr[dev]; return HGD_OK; }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gemv_static_ws) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
+    }
+    if (dev >= 0 && dev < 64) addr[dev] = p;
+    *out = p;
+    return HGD_OK;
+}
+
+}  // namespace
+
+extern "C" int hgd_gemv_bf16_static_ws(const uint16_t* W, const uint16_t* x, void* y, int y_is_fp32, int M,
+                                       int N, int K, hgd_stream_t stream) {
+    if (!W || !x || !y || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (K % 32 != 0 || K > 65536) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(W) || !al16(x) || !al16(y)) return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    const size_t need = gemv_ws_bytes(M, N, K, false);
+    if (need > kStaticWsBytes) return HGD_ERR_BUFFER_TOO_SMALL;
+    void* ws = nullptr;
+    if ((rc = static_ws_address(&ws))) return rc;
+    // the row-block counters must start at zero; the partials need no clearing
+    if (need && cudaMemsetAsync(ws, 0, kWsCounterBytes, (cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
+    }
+    GemvParams p = {};
+    p.W = W; p.N = N; p.K = K; p.x = x; p.x_ld = K; p.y = y; p.y_ld = N;
+    if (y_is_fp32)
+        return run_gemv<PRO_COPY, EPI_F32>(p, M, di.sms, need ? ws : nullptr, need, (cudaStream_t)stream);
+    return run_gemv<PRO_COPY, EPI_BF16>(p, M, di.sms, need ? ws : nullptr, need, (cudaStream_t)stream);
+}

@@ -99,6 +99,26 @@ HGD_API int hgd_gemv_bf16(const uint16_t* W, const uint16_t* x, void* y, int y_i
  * SwiGLU (swiglu = 1, N = I) of this shape; 0 when that shape never uses one. */
 HGD_API int hgd_gemv_workspace_bytes(int M, int N, int K, int swiglu, size_t* bytes);
 
+/* hgd_gemv_bf16 for callers that cannot allocate device memory (a plugin whose
+ * host framework owns the device allocator and offers it no handle; a decode
+ * loop that must never wait on the synchronisation a cudaMalloc brings).  The
+ * pages have no counterpart: it exists only so such callers need no workspace.
+ * Same inputs, output, shapes and results as hgd_gemv_bf16, but the split-K
+ * scratch is a 4 MiB array built into the library, present on every device that
+ * loads it until the process exits.  Nothing is allocated.
+ *  - The first call on a device looks the array's device address up (once per
+ *    device, with that device current); make that first call before capturing
+ *    any stream into a CUDA graph.
+ *  - A shape whose scratch would exceed 4 MiB returns HGD_ERR_BUFFER_TOO_SMALL
+ *    and launches nothing (hgd_gemv_workspace_bytes tells the size needed).
+ *  - Each call clears the part of the array that must start at zero (its
+ *    counters) on `stream` before the GEMV; the rest keeps the last call's data.
+ *  - All calls share the one array: calls that overlap on the device (other
+ *    streams, other host threads) race and corrupt each other's results.
+ *    Issue them on one stream, or order them. */
+HGD_API int hgd_gemv_bf16_static_ws(const uint16_t* W, const uint16_t* x, void* y, int y_is_fp32,
+                                    int M, int N, int K, hgd_stream_t stream);
+
 /* h[m][i] = bf16( silu(g) * u ),  g = x . W_gate[i],  u = x . W_up[i]
  * ([AST] fused BF16 up/gate SwiGLU; [FT] silu_and_mul), silu(t) = t/(1+exp(-t)).
  *   W_gate, W_up [I, K] bf16 device; x [M, K] bf16 device; h [M, I] bf16 device.
