@@ -38,6 +38,17 @@ WORKLOAD = ("24-layer hybrid stack (3 GDN : 1 gated attention), hidden 1024, voc
             "GDN 16x128, attn 8q/2kv x256, MLP 3584, batch 1, KV context 512, greedy decode")
 
 
+def chain_launches(cfg: dict) -> int:
+    """Kernels one B=1, T=1 step launches on the kernel-chain path: per GDN layer
+    in-projection (with the conv tail), mixer, out-projection, SwiGLU, down; per
+    attention layer the same with RoPE/append, partials and merge as the mixer;
+    then the LM head and the argmax finalisation."""
+    import hgd_synth as syn
+
+    n_gdn, n_att = syn.layer_counts(cfg)
+    return n_gdn * 5 + n_att * 7 + 2
+
+
 def algorithmic_bytes(cfg: dict, L_keys: float) -> dict:
     """Bytes one decode token must move, by component (the HBM roofline numerator)."""
     D, V, H, dk, dv, kc = (cfg[k] for k in ("hidden", "vocab", "gdn_heads", "gdn_dk", "gdn_dv", "conv_k"))
@@ -206,16 +217,17 @@ def run_gpu(args) -> None:
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     tok_buf = argmax.view(B, 1)  # greedy: each step reads the previous step's argmax
     tok_buf.copy_(tok)
-    launches = model.launches(B, 1)
+    split = args.path == "chain"
+    launches = chain_launches(cfg) if split else model.launches(B, 1)
 
-    dec = hgd.DecodeGraph(model, state, tok_buf, argmax, status, stream=stream)
+    dec = hgd.DecodeGraph(model, state, tok_buf, argmax, status, stream=stream, split=split)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
         dec.replay()
     stream.synchronize()
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -228,10 +240,8 @@ def run_gpu(args) -> None:
         t_start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
-            dec.replay_layers()
+            dec.replay()
             ev[i][1].record(stream)
-            dec.replay_head()
-            ev[i][2].record(stream)
         t_end.record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
@@ -239,7 +249,7 @@ def run_gpu(args) -> None:
     if world > 1:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    head_ms = [a.elapsed_time(b) for _, a, b in ev]
+    step_ms = [a.elapsed_time(b) for a, b in ev]
     if world > 1:
         t = torch.tensor([elapsed_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -272,8 +282,8 @@ def run_gpu(args) -> None:
     ab = algorithmic_bytes(cfg, L_avg)
     peaks = measured_peaks()
     peak = float(peaks.get("hbm_gbs", 6650.0))
-    head_avg_ms = statistics.mean(head_ms)
-    head_gbs = ab["head"] / (head_avg_ms * 1e-3) / 1e9
+    launch_ms = statistics.mean(step_ms)
+    kern_gbs = ab["total"] / (launch_ms * 1e-3) / 1e9
     step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
     prof = {}
     try:
@@ -290,15 +300,16 @@ def run_gpu(args) -> None:
                    "l2": "inputs larger than L2: 1.5 GB of weights streamed per step (L2 126 MB)"},
         "hbm_gbs": step_gbs,
         "frac_of_8tbs": step_gbs / 8000.0,
-        "roofline": {"kernel": "LM head (final RMSNorm + tied 248320x1024 GEMV + per-CTA argmax)",
-                     "bound": "hbm", "achieved": head_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": head_gbs / peak, "peak_source": "measured" if "_fallback" not in peaks else "fallback",
-                     "traffic": prof.get("lm_head_bytes_per_launch"),
-                     "algorithmic_bytes": ab["head"], "avg_launch_ms": head_avg_ms},
-        "step_roofline": {"bound": "hbm", "achieved": step_gbs, "peak": peak, "unit": "GB/s",
-                          "frac": step_gbs / peak, "algorithmic_bytes": ab["total"],
-                          "traffic": prof.get("step_bytes")},
+        "roofline": {"kernel": ("k_stack: the whole decode step in one cooperative launch" if not split else
+                                "the kernel chain of one decode step (GEMV, GDN, attention, argmax kernels)"),
+                     "bound": "hbm", "achieved": kern_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": kern_gbs / peak, "frac_of_8tbs": kern_gbs / 8000.0,
+                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if "_fallback" not in peaks
+                     else "fallback",
+                     "traffic": prof.get("k_stack_bytes_per_launch" if not split else "chain_bytes_per_step"),
+                     "algorithmic_bytes": ab["total"], "avg_launch_ms": launch_ms},
         "gpu_launches": launches * args.steps,
+        "path": "kernel chain" if split else "persistent",
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": 4 * B, "d2h_bytes_per_step": 4 * B,
                 "steps": e2e_steps, "how": "per token: pinned H2D of the token, graph replay of the step, "
                                           "D2H of the argmax, host synchronisation"},
@@ -317,6 +328,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="chain", choices=["chain", "persistent"],
+                    help="chain: one kernel per op, PDL-overlapped, in CUDA graphs; "
+                         "persistent: the whole step in one cooperative launch")
     ap.add_argument("--cpu-tokens", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -367,54 +367,68 @@ def decode_layer_stack_range(model: Model, state: State, tokens, T: int, layer_b
 
 
 class DecodeGraph:
-    """A one-row greedy decode step captured as two CUDA graphs (all layers; final
-    norm + LM head + argmax) and replayed on `stream`.  `tokens` [B,1] is read at
-    the start of a step and `argmax` [B] written at its end, so passing
-    tokens = argmax.view(B, 1) feeds each step's argmax to the next step on the
-    device.  Capturing runs the step once eagerly first (to load the kernels) on
-    a copy of the state, which is then restored."""
+    """A greedy decode step (T = 1) captured as a CUDA graph and replayed on
+    `stream`: one hgd_decode_layer_stack call, which is a single cooperative
+    launch when the call fits it.  `tokens` [B,1] is read at the start of a step
+    and `argmax` [B] written at its end, so tokens = argmax.view(B, 1) feeds each
+    step's argmax to the next on the device.  With split=True the step is
+    captured as two graphs (all layers; then the head) through the layer-range
+    entry point instead.  Capturing runs the step once eagerly first (to load the
+    kernels) on a copy of the state, which is then restored."""
 
-    def __init__(self, model: Model, state: State, tokens, argmax, status=None, stream=None):
+    def __init__(self, model: Model, state: State, tokens, argmax, status=None, stream=None, split=False):
         torch = _torch()
         self.model, self.state, self.tokens, self.argmax, self.status = model, state, tokens, argmax, status
         self.stream = stream or torch.cuda.Stream()
+        self.split = split
+        L = model.cfg_dict["n_layers"]
         snap = state.snapshot()
         tok0 = tokens.clone()
         with torch.cuda.stream(self.stream):
-            decode_layer_stack(model, state, tokens, 1, argmax=argmax, status=status, stream=self.stream)
+            if split:
+                decode_layer_stack_range(model, state, tokens, 1, 0, L, False, status=status, stream=self.stream)
+                decode_layer_stack_range(model, state, None, 1, L, L, True, argmax=argmax, status=status,
+                                         stream=self.stream)
+            else:
+                decode_layer_stack(model, state, tokens, 1, argmax=argmax, status=status, stream=self.stream)
         self.stream.synchronize()
         state.restore(snap)
         tokens.copy_(tok0)
         torch.cuda.synchronize()
         self.g_layers = torch.cuda.CUDAGraph()
-        self.g_head = torch.cuda.CUDAGraph()
-        L = model.cfg_dict["n_layers"]
-        with torch.cuda.graph(self.g_layers, stream=self.stream):
-            decode_layer_stack_range(model, state, tokens, 1, 0, L, False, status=status)
-        with torch.cuda.graph(self.g_head, stream=self.stream):
-            decode_layer_stack_range(model, state, None, 1, L, L, True, argmax=argmax, status=status)
+        self.g_head = torch.cuda.CUDAGraph() if split else None
+        if split:
+            with torch.cuda.graph(self.g_layers, stream=self.stream):
+                decode_layer_stack_range(model, state, tokens, 1, 0, L, False, status=status)
+            with torch.cuda.graph(self.g_head, stream=self.stream):
+                decode_layer_stack_range(model, state, None, 1, L, L, True, argmax=argmax, status=status)
+        else:
+            with torch.cuda.graph(self.g_layers, stream=self.stream):
+                decode_layer_stack(model, state, tokens, 1, argmax=argmax, status=status)
         torch.cuda.synchronize()
 
     def replay_layers(self):
         self.g_layers.replay()
 
     def replay_head(self):
-        self.g_head.replay()
+        if self.g_head is not None:
+            self.g_head.replay()
 
     def replay(self):
         self.g_layers.replay()
-        self.g_head.replay()
+        if self.g_head is not None:
+            self.g_head.replay()
 
     def step_host(self, h_tok, h_out):
         """One step from a pinned host token tensor to a pinned host argmax tensor."""
         torch = _torch()
         with torch.cuda.stream(self.stream):
             self.tokens.copy_(h_tok, non_blocking=True)
-            self.g_layers.replay()
-            self.g_head.replay()
+            self.replay()
             h_out.copy_(self.argmax, non_blocking=True)
         self.stream.synchronize()
 
     def close(self):
         self.g_layers.reset()
-        self.g_head.reset()
+        if self.g_head is not None:
+            self.g_head.reset()

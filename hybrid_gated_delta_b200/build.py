@@ -9,7 +9,10 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhgd.so")
 SOURCES = ["api.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+# -fmad=false: no multiply-add is fused implicitly, so an expression rounds the
+# same way in every kernel that evaluates it (all intended fused multiply-adds
+# are explicit fmaf calls).
+FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-fmad=false",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
          "-Xcompiler", "-fvisibility=hidden"]
 

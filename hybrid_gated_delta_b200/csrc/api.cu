@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "gdn.cuh"
 #include "gemv.cuh"
+#include "stack.cuh"
 
 using namespace hgd;
 
@@ -313,7 +314,7 @@ size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_
 
 enum ScratchIdx {
     SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
-    SC_BESTV, SC_BESTI, SC_WS, SC_END, SC_COUNT
+    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_END, SC_COUNT
 };
 constexpr int kBestG = 4096;  // max CTAs of the LM-head launch
 
@@ -348,6 +349,7 @@ void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     sz[SC_BESTV] = (size_t)M * kBestG * 4;
     sz[SC_BESTI] = (size_t)M * kBestG * 4;
     sz[SC_WS] = stack_ws_bytes(d, (int)M);
+    sz[SC_BAR] = 64 + 256 * 8;  // grid-barrier words and phase timestamps of the persistent launch
     size_t pos = 0;
     for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
     off[SC_END] = pos;
@@ -357,6 +359,55 @@ int check_state_dims(int B, int Tmax, int Lmax) {
     if (B < 1 || Tmax < 1 || Lmax < 1) return HGD_ERR_INVALID_ARG;
     if ((int64_t)B * Tmax > 256 || Lmax > 16384) return HGD_ERR_UNSUPPORTED_SHAPE;
     return HGD_OK;
+}
+
+// ------------------------------------------------------- persistent launch
+size_t sk_x_bytes(const Dims& d) {
+    const int kmax = std::max(std::max(d.D, d.H * d.dv), std::max(d.nq * d.hd, d.I));
+    return (size_t)gv_align16(8 * (kmax + GV_PAD) * 2);
+}
+
+size_t sk_smem_bytes(const Dims& d) {
+    return (size_t)SK_NSLOT * SK_SLAB_BYTES + sk_x_bytes(d) + (size_t)SK_CW * GV_ROWS * 8 * 4 +
+           (size_t)SK_CW * 8 * 8 + (size_t)SK_CW * 32 * 4 + 2 * 8 * SK_NSLOT + 32;
+}
+
+// The persistent launch covers calls of at most one MMA n-tile of token rows
+// with a GDN key width of 64 or 128 and a shared-memory footprint that fits.
+bool sk_supported(const Dims& d, int M) {
+    return M <= SK_MAXM && (d.dk == 64 || d.dk == 128) && sk_smem_bytes(d) <= (size_t)GV_SMEM_LIMIT;
+}
+
+template <int KPL>
+int sk_launch_t(const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
+    auto kern = k_stack<KPL>;
+    static int attr_done[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT) != cudaSuccess) {
+            cudaGetLastError();
+            return HGD_ERR_CUDA;
+        }
+        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    }
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, SK_THREADS, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
+    }
+    if (occ < 1) return HGD_ERR_NOT_CORESIDENT;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(SK_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return launch_status(cudaLaunchKernelEx(&cfg, kern, prm));
 }
 
 }  // namespace
@@ -604,6 +655,7 @@ int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T) {
     Dims d;
     if (dims_of(&m->cfg, &d)) return -1;
     const int M = B * T;
+    if (sk_supported(d, M)) return 1;  // one cooperative launch (plus a barrier reset)
     int n = 0;
     for (int l = 0; l < d.L; ++l) {
         const bool att = is_attn_layer(&m->cfg, l);
@@ -619,9 +671,57 @@ int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T) {
 int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T, float* logits,
                            int32_t* argmax, float* S_rec, float* tail_rec, int32_t* status_dev,
                            hgd_stream_t stream) {
-    if (!m) return HGD_ERR_INVALID_ARG;
-    return hgd_decode_layer_stack_range(m, st, tokens, T, 0, m->cfg.n_layers, 1, logits, argmax, S_rec,
-                                        tail_rec, status_dev, stream);
+    if (!m || !st || !st->arena || !tokens || !argmax) return HGD_ERR_INVALID_ARG;
+    if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if (!sk_supported(d, st->B * T))
+        return hgd_decode_layer_stack_range(m, st, tokens, T, 0, m->cfg.n_layers, 1, logits, argmax, S_rec,
+                                            tail_rec, status_dev, stream);
+    if (!al16(tokens) || !al16(argmax) || (logits && !al16(logits)) || (S_rec && !al16(S_rec)) ||
+        (tail_rec && !al16(tail_rec)))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    uint8_t* A = static_cast<uint8_t*>(st->arena);
+    SkParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.L = d.L; prm.D = d.D; prm.V = d.V; prm.H = d.H; prm.dk = d.dk; prm.dv = d.dv; prm.nq = d.nq;
+    prm.nkv = d.nkv; prm.hd = d.hd; prm.I = d.I; prm.every = d.every;
+    prm.C = (int)d.C; prm.gdn_out = (int)d.gdn_out; prm.attn_out = (int)d.attn_out;
+    prm.proj_ld = (int)std::max(d.gdn_out, d.attn_out);
+    prm.eps = m->cfg.norm_eps; prm.rope_base = m->cfg.rope_base;
+    prm.B = st->B; prm.T = T; prm.M = st->B * T; prm.Lmax = st->Lmax; prm.max_chunks = max_chunks_of(st->Lmax);
+    prm.embed = m->embed; prm.final_norm = m->final_norm;
+    prm.S = reinterpret_cast<float*>(A + st->off[SC_S]);
+    prm.conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
+    prm.kv = reinterpret_cast<bf16_t*>(A + st->off[SC_KV]);
+    prm.pos = reinterpret_cast<int32_t*>(A + st->off[SC_POS]);
+    prm.resid = reinterpret_cast<bf16_t*>(A + st->off[SC_RESID]);
+    prm.proj = reinterpret_cast<float*>(A + st->off[SC_PROJ]);
+    prm.obuf = reinterpret_cast<float*>(A + st->off[SC_O]);
+    prm.qrot = reinterpret_cast<float*>(A + st->off[SC_QROT]);
+    prm.attn = reinterpret_cast<bf16_t*>(A + st->off[SC_ATTN]);
+    prm.part = reinterpret_cast<float*>(A + st->off[SC_PART]);
+    prm.mlp = reinterpret_cast<bf16_t*>(A + st->off[SC_MLP]);
+    prm.bestv = reinterpret_cast<float*>(A + st->off[SC_BESTV]);
+    prm.besti = reinterpret_cast<int32_t*>(A + st->off[SC_BESTI]);
+    prm.ws_cnt = reinterpret_cast<int32_t*>(A + st->off[SC_WS]);
+    prm.ws_part = reinterpret_cast<float*>(A + st->off[SC_WS] + kWsCounterBytes);
+    prm.tokens = tokens; prm.logits = logits; prm.argmax = argmax; prm.S_rec = S_rec; prm.tail_rec = tail_rec;
+    prm.status = status_dev;
+    prm.bar = reinterpret_cast<unsigned*>(A + st->off[SC_BAR]);
+    prm.trace = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + 64);
+    prm.x_bytes = (int)sk_x_bytes(d);
+    for (int l = 0; l < d.L; ++l)
+        for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) prm.layer[l].w[t] = m->w[l][t];
+    cudaStream_t s = (cudaStream_t)stream;
+    // a fresh barrier for this call (an earlier call may have stopped on a timeout)
+    if (cudaMemsetAsync(prm.bar, 0, 64, s) != cudaSuccess) { cudaGetLastError(); return HGD_ERR_CUDA; }
+    const size_t smem = sk_smem_bytes(d);
+    return d.dk == 128 ? sk_launch_t<4>(prm, smem, di.sms, s) : sk_launch_t<2>(prm, smem, di.sms, s);
 }
 
 int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,

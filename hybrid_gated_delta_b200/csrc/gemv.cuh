@@ -244,6 +244,198 @@ __device__ __forceinline__ bool gv_item(const GemvParams& p, int slot, int i, Gv
     return true;
 }
 
+// Running argmax of a thread's tokens (nt*8 + 2c + h) over the rows it has seen.
+template <int NT>
+struct GvBest {
+    float v[NT][2];
+    int i[NT][2];
+    bool nan;
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) { v[nt][0] = v[nt][1] = -INFINITY; i[nt][0] = i[nt][1] = 0x7fffffff; }
+        nan = false;
+    }
+};
+
+// A finished slab partial (split) or row-block sum (unsplit) of row block rb:
+// in split mode add it to the workspace and, in the last of the row block's
+// slabs to arrive, add all partials in slab order; then run the epilogue.
+// `cb` is this warp's [16][MP] shared scratch (conv epilogue).
+template <int NT, int EPI>
+__device__ __forceinline__ void gv_finish(const GemvParams& p, int rb, int s_item, float (&yacc)[NT][4],
+                                          int lane, float* cb, GvBest<NT>& best) {
+    constexpr int MP = 8 * NT;
+    const int r8 = lane >> 2, c = lane & 3;
+        bool finish = true;
+        if (p.split) {
+            // slab partial -> workspace; the last of the row block's slabs adds them in order
+            float* wp = p.ws_part + ((int64_t)(rb * p.nks + s_item) * GV_ROWS) * p.ws_mp;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int n0 = nt * 8 + 2 * c;
+                wp[r8 * p.ws_mp + n0] = yacc[nt][0];
+                wp[r8 * p.ws_mp + n0 + 1] = yacc[nt][1];
+                wp[(r8 + 8) * p.ws_mp + n0] = yacc[nt][2];
+                wp[(r8 + 8) * p.ws_mp + n0 + 1] = yacc[nt][3];
+            }
+            __threadfence();
+            __syncwarp();
+            int old = 0;
+            if (lane == 0) old = atomicAdd(&p.ws_cnt[rb], 1);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            finish = (old == p.nks - 1);
+            if (finish) {
+                __threadfence();
+                for (int j = 0; j < p.nks; ++j) {
+                    const float* pp = p.ws_part + ((int64_t)(rb * p.nks + j) * GV_ROWS) * p.ws_mp;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int n0 = nt * 8 + 2 * c;
+                        const float v0 = ld_cg(pp + r8 * p.ws_mp + n0), v1 = ld_cg(pp + r8 * p.ws_mp + n0 + 1);
+                        const float v2 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0), v3 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0 + 1);
+                        if (j == 0) { yacc[nt][0] = v0; yacc[nt][1] = v1; yacc[nt][2] = v2; yacc[nt][3] = v3; }
+                        else { yacc[nt][0] += v0; yacc[nt][1] += v1; yacc[nt][2] += v2; yacc[nt][3] += v3; }
+                    }
+                }
+                if (lane == 0) p.ws_cnt[rb] = 0;  // leave the workspace ready for the next call
+            }
+        }
+        if (!finish) return;
+        // ----------------------------------------------------------- epilogue
+        if (EPI == EPI_QKV_CONV) {
+            // Gather the 16 x MP tile in shared memory; lane l < 16 then runs the conv
+            // of channel rb*16 + l over the launch's token rows in order.  The row
+            // block (hence the channel and its tail) belongs to this warp alone.
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int n0 = nt * 8 + 2 * c;
+                cb[r8 * MP + n0] = yacc[nt][0];
+                cb[r8 * MP + n0 + 1] = yacc[nt][1];
+                cb[(r8 + 8) * MP + n0] = yacc[nt][2];
+                cb[(r8 + 8) * MP + n0 + 1] = yacc[nt][3];
+            }
+            __syncwarp();
+            const int ch = rb * GV_ROWS + lane;
+            if (lane < GV_ROWS && ch < p.N) {
+                float* yrow = reinterpret_cast<float*>(p.y);
+                if (ch >= p.conv_C) {
+                    for (int m = 0; m < p.M; ++m) yrow[m * p.y_ld + ch] = cb[lane * MP + m];
+                } else {
+                    float w[GV_CONV_K], tl[GV_CONV_K - 1];
+#pragma unroll
+                    for (int j = 0; j < GV_CONV_K; ++j) w[j] = bf2f(p.conv_w[(int64_t)ch * GV_CONV_K + j]);
+                    int cur_b = -1;
+                    for (int m = 0; m < p.M; ++m) {
+                        const int gm = p.m0 + m, b = gm / p.conv_T, t = gm % p.conv_T;
+                        float* tb = p.conv_tail + (int64_t)b * (GV_CONV_K - 1) * p.conv_C + ch;
+                        if (b != cur_b) {
+#pragma unroll
+                            for (int j = 0; j < GV_CONV_K - 1; ++j) tl[j] = tb[(int64_t)j * p.conv_C];
+                            cur_b = b;
+                        }
+                        const float xv = cb[lane * MP + m];
+                        float acc = 0.f;
+#pragma unroll
+                        for (int j = 0; j < GV_CONV_K - 1; ++j) acc = fmaf(w[j], tl[j], acc);
+                        acc = fmaf(w[GV_CONV_K - 1], xv, acc);
+                        yrow[m * p.y_ld + ch] = silu_f(acc);
+#pragma unroll
+                        for (int j = 0; j + 1 < GV_CONV_K - 1; ++j) tl[j] = tl[j + 1];
+                        tl[GV_CONV_K - 2] = xv;
+                        if (p.conv_rec) {
+                            float* rr = p.conv_rec + ((int64_t)b * p.conv_T + t) * (GV_CONV_K - 1) * p.conv_C + ch;
+#pragma unroll
+                            for (int j = 0; j < GV_CONV_K - 1; ++j) rr[(int64_t)j * p.conv_C] = tl[j];
+                        }
+                        if (m == p.M - 1 || t == p.conv_T - 1) {
+#pragma unroll
+                            for (int j = 0; j < GV_CONV_K - 1; ++j) tb[(int64_t)j * p.conv_C] = tl[j];
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+        } else {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int n0 = nt * 8 + 2 * c;  // tokens n0, n0 + 1; rows r8, r8 + 8
+            if (EPI == EPI_SWIGLU) {
+                const int col = rb * 8 + r8;
+                if (col < p.N) {
+                    bf16_t* h = reinterpret_cast<bf16_t*>(p.y);
+                    if (n0 < p.M) h[n0 * p.y_ld + col] = f2bf(silu_f(yacc[nt][0]) * yacc[nt][2]);
+                    if (n0 + 1 < p.M) h[(n0 + 1) * p.y_ld + col] = f2bf(silu_f(yacc[nt][1]) * yacc[nt][3]);
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int n = n0 + (q & 1);
+                    const int col = rb * GV_ROWS + r8 + ((q & 2) ? 8 : 0);
+                    if (n >= p.M || col >= p.N) continue;
+                    const float v = yacc[nt][q];
+                    if (EPI == EPI_F32) {
+                        reinterpret_cast<float*>(p.y)[n * p.y_ld + col] = v;
+                    } else if (EPI == EPI_BF16) {
+                        reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(v);
+                    } else if (EPI == EPI_RESID) {
+                        const float base = bf2f(p.resid[n * p.resid_ld + col]);
+                        reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(base + v);
+                    } else {  // EPI_ARGMAX
+                        if (p.logits) p.logits[n * p.logits_ld + col] = v;
+                        if (v != v) best.nan = true;
+                        else if (v > best.v[nt][q & 1] || (v == best.v[nt][q & 1] && col < best.i[nt][q & 1])) {
+                            best.v[nt][q & 1] = v;
+                            best.i[nt][q & 1] = col;
+                        }
+                    }
+                }
+            }
+        }
+        }
+}
+
+// Per-CTA argmax partials: reduce each token over the row lanes of every warp,
+// then over the warps (`bar` synchronises the nthreads consumer threads).
+template <int NT>
+__device__ __forceinline__ void gv_argmax_cta(const GemvParams& p, GvBest<NT>& best, float* amax_v, int* amax_i,
+                                              int warp, int lane, int tid, int nwarps, int cta, int ncta,
+                                              bool named) {
+    constexpr int MP = 8 * NT;
+    const int r8 = lane >> 2, c = lane & 3;
+    const bool any_nan = __any_sync(0xffffffffu, best.nan);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float bv = best.v[nt][h];
+            int bi = best.i[nt][h];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (r8 == 0) {
+                amax_v[warp * MP + nt * 8 + 2 * c + h] = bv;
+                amax_i[warp * MP + nt * 8 + 2 * c + h] = any_nan ? -1 : bi;
+            }
+        }
+    if (named) named_bar(1, nwarps * 32); else __syncthreads();
+    if (tid < p.M) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        bool nan_cta = false;
+        for (int w = 0; w < nwarps; ++w) {
+            const float v = amax_v[w * MP + tid];
+            const int i = amax_i[w * MP + tid];
+            if (i < 0) nan_cta = true;
+            else if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+        }
+        p.best_v[tid * ncta + cta] = bv;
+        p.best_i[tid * ncta + cta] = nan_cta ? -1 : bi;
+    }
+}
+
 template <int NT, int PRO, int EPI>
 __global__ void __launch_bounds__(GV_THREADS, (NT >= 4) ? 1 : 2) k_gemv(const __grid_constant__ GemvParams p) {
     constexpr int MP = 8 * NT;
@@ -300,12 +492,10 @@ __global__ void __launch_bounds__(GV_THREADS, (NT >= 4) ? 1 : 2) k_gemv(const __
     gv_prologue<MP, PRO>(p, xs, tid, warp, lane, nullptr);
     __syncthreads();
 
-    float best_v[NT][2];
-    int best_i[NT][2];
-    bool saw_nan = false;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) { best_v[nt][0] = best_v[nt][1] = -INFINITY; best_i[nt][0] = best_i[nt][1] = 0x7fffffff; }
+    GvBest<NT> best;
+    best.init();
     const bf16_t* xb = xs + r8 * XS + 8 * c;
+    float* cb = cbuf + warp * GV_ROWS * MP;
 
     for (int i = 0; have; ++i) {
         float yacc[NT][4];
@@ -338,18 +528,10 @@ __global__ void __launch_bounds__(GV_THREADS, (NT >= 4) ? 1 : 2) k_gemv(const __
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) c0[nt][q] = c0[nt][q] + c1[nt][q];
-            if (p.split) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) yacc[nt][q] = c0[nt][q];
-            } else {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) yacc[nt][q] = (s == 0) ? c0[nt][q] : yacc[nt][q] + c0[nt][q];
-            }
+                for (int q = 0; q < 4; ++q) {
+                    const float part = c0[nt][q] + c1[nt][q];
+                    yacc[nt][q] = (p.split || s == 0) ? part : yacc[nt][q] + part;
+                }
         }
         const int rb = it.rb, s_item = it.s0;
         // next item: start its loads before this item's epilogue
@@ -360,172 +542,11 @@ __global__ void __launch_bounds__(GV_THREADS, (NT >= 4) ? 1 : 2) k_gemv(const __
 #pragma unroll
             for (int j = 0; j < NB; ++j) load_step(j, nx.s0 * GV_SLAB_STEPS + j);
         }
-
-        bool finish = true;
-        if (p.split) {
-            // slab partial -> workspace; the last of the row block's slabs adds them in order
-            float* wp = p.ws_part + ((int64_t)(rb * p.nks + s_item) * GV_ROWS) * p.ws_mp;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int n0 = nt * 8 + 2 * c;
-                wp[r8 * p.ws_mp + n0] = yacc[nt][0];
-                wp[r8 * p.ws_mp + n0 + 1] = yacc[nt][1];
-                wp[(r8 + 8) * p.ws_mp + n0] = yacc[nt][2];
-                wp[(r8 + 8) * p.ws_mp + n0 + 1] = yacc[nt][3];
-            }
-            __threadfence();
-            __syncwarp();
-            int old = 0;
-            if (lane == 0) old = atomicAdd(&p.ws_cnt[rb], 1);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            finish = (old == p.nks - 1);
-            if (finish) {
-                __threadfence();
-                for (int j = 0; j < p.nks; ++j) {
-                    const float* pp = p.ws_part + ((int64_t)(rb * p.nks + j) * GV_ROWS) * p.ws_mp;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int n0 = nt * 8 + 2 * c;
-                        const float v0 = ld_cg(pp + r8 * p.ws_mp + n0), v1 = ld_cg(pp + r8 * p.ws_mp + n0 + 1);
-                        const float v2 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0), v3 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0 + 1);
-                        if (j == 0) { yacc[nt][0] = v0; yacc[nt][1] = v1; yacc[nt][2] = v2; yacc[nt][3] = v3; }
-                        else { yacc[nt][0] += v0; yacc[nt][1] += v1; yacc[nt][2] += v2; yacc[nt][3] += v3; }
-                    }
-                }
-                if (lane == 0) p.ws_cnt[rb] = 0;  // leave the workspace ready for the next call
-            }
-        }
-        if (!finish) { it = nx; continue; }
-        // ----------------------------------------------------------- epilogue
-        if (EPI == EPI_QKV_CONV) {
-            // Gather the 16 x MP tile in shared memory; lane l < 16 then runs the conv
-            // of channel rb*16 + l over the launch's token rows in order.  The row
-            // block (hence the channel and its tail) belongs to this warp alone.
-            float* cb = cbuf + warp * GV_ROWS * MP;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int n0 = nt * 8 + 2 * c;
-                cb[r8 * MP + n0] = yacc[nt][0];
-                cb[r8 * MP + n0 + 1] = yacc[nt][1];
-                cb[(r8 + 8) * MP + n0] = yacc[nt][2];
-                cb[(r8 + 8) * MP + n0 + 1] = yacc[nt][3];
-            }
-            __syncwarp();
-            const int ch = rb * GV_ROWS + lane;
-            if (lane < GV_ROWS && ch < p.N) {
-                float* yrow = reinterpret_cast<float*>(p.y);
-                if (ch >= p.conv_C) {
-                    for (int m = 0; m < p.M; ++m) yrow[m * p.y_ld + ch] = cb[lane * MP + m];
-                } else {
-                    float w[GV_CONV_K], tl[GV_CONV_K - 1];
-#pragma unroll
-                    for (int j = 0; j < GV_CONV_K; ++j) w[j] = bf2f(p.conv_w[(int64_t)ch * GV_CONV_K + j]);
-                    int cur_b = -1;
-                    for (int m = 0; m < p.M; ++m) {
-                        const int gm = p.m0 + m, b = gm / p.conv_T, t = gm % p.conv_T;
-                        float* tb = p.conv_tail + (int64_t)b * (GV_CONV_K - 1) * p.conv_C + ch;
-                        if (b != cur_b) {
-#pragma unroll
-                            for (int j = 0; j < GV_CONV_K - 1; ++j) tl[j] = tb[(int64_t)j * p.conv_C];
-                            cur_b = b;
-                        }
-                        const float xv = cb[lane * MP + m];
-                        float acc = 0.f;
-#pragma unroll
-                        for (int j = 0; j < GV_CONV_K - 1; ++j) acc = fmaf(w[j], tl[j], acc);
-                        acc = fmaf(w[GV_CONV_K - 1], xv, acc);
-                        yrow[m * p.y_ld + ch] = silu_f(acc);
-#pragma unroll
-                        for (int j = 0; j + 1 < GV_CONV_K - 1; ++j) tl[j] = tl[j + 1];
-                        tl[GV_CONV_K - 2] = xv;
-                        if (p.conv_rec) {
-                            float* rr = p.conv_rec + ((int64_t)b * p.conv_T + t) * (GV_CONV_K - 1) * p.conv_C + ch;
-#pragma unroll
-                            for (int j = 0; j < GV_CONV_K - 1; ++j) rr[(int64_t)j * p.conv_C] = tl[j];
-                        }
-                        if (m == p.M - 1 || t == p.conv_T - 1) {
-#pragma unroll
-                            for (int j = 0; j < GV_CONV_K - 1; ++j) tb[(int64_t)j * p.conv_C] = tl[j];
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            it = nx;
-            continue;
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int n0 = nt * 8 + 2 * c;  // tokens n0, n0 + 1; rows r8, r8 + 8
-            if (EPI == EPI_SWIGLU) {
-                const int col = rb * 8 + r8;
-                if (col < p.N) {
-                    bf16_t* h = reinterpret_cast<bf16_t*>(p.y);
-                    if (n0 < p.M) h[n0 * p.y_ld + col] = f2bf(silu_f(yacc[nt][0]) * yacc[nt][2]);
-                    if (n0 + 1 < p.M) h[(n0 + 1) * p.y_ld + col] = f2bf(silu_f(yacc[nt][1]) * yacc[nt][3]);
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int n = n0 + (q & 1);
-                    const int col = rb * GV_ROWS + r8 + ((q & 2) ? 8 : 0);
-                    if (n >= p.M || col >= p.N) continue;
-                    const float v = yacc[nt][q];
-                    if (EPI == EPI_F32) {
-                        reinterpret_cast<float*>(p.y)[n * p.y_ld + col] = v;
-                    } else if (EPI == EPI_BF16) {
-                        reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(v);
-                    } else if (EPI == EPI_RESID) {
-                        const float base = bf2f(p.resid[n * p.resid_ld + col]);
-                        reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(base + v);
-                    } else {  // EPI_ARGMAX
-                        if (p.logits) p.logits[n * p.logits_ld + col] = v;
-                        if (v != v) saw_nan = true;
-                        else if (v > best_v[nt][q & 1] || (v == best_v[nt][q & 1] && col < best_i[nt][q & 1])) {
-                            best_v[nt][q & 1] = v;
-                            best_i[nt][q & 1] = col;
-                        }
-                    }
-                }
-            }
-        }
+        gv_finish<NT, EPI>(p, rb, s_item, yacc, lane, cb, best);
         it = nx;
     }
-    if (EPI == EPI_ARGMAX) {
-        // warp: reduce over the 8 row lanes of each token, then CTA: over warps
-        const bool any_nan = __any_sync(0xffffffffu, saw_nan);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float bv = best_v[nt][h];
-                int bi = best_i[nt][h];
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-                }
-                if (r8 == 0) {
-                    amax_v[warp * MP + nt * 8 + 2 * c + h] = bv;
-                    amax_i[warp * MP + nt * 8 + 2 * c + h] = any_nan ? -1 : bi;
-                }
-            }
-        __syncthreads();
-        if (tid < p.M) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            bool nan_cta = false;
-            for (int w = 0; w < GV_CW; ++w) {
-                const float v = amax_v[w * MP + tid];
-                const int i = amax_i[w * MP + tid];
-                if (i < 0) nan_cta = true;
-                else if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
-            }
-            p.best_v[tid * gridDim.x + blockIdx.x] = bv;
-            p.best_i[tid * gridDim.x + blockIdx.x] = nan_cta ? -1 : bi;
-        }
-    }
+    if (EPI == EPI_ARGMAX)
+        gv_argmax_cta<NT>(p, best, amax_v, amax_i, warp, lane, tid, GV_CW, blockIdx.x, gridDim.x, false);
 }
 
 // Pack a row-major [rows][K] bf16 matrix into the fragment-ordered tiles.

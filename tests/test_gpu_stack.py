@@ -231,7 +231,7 @@ def test_full_stack_bench_configuration(hgd, full):
     L, Lmax, steps = cfg["n_layers"], 640, 5
     init = syn.stack_state(cfg, 1, Lmax, prefill=512, seed=9)
     tok0 = torch.from_numpy(syn.stack_tokens(cfg, 1, 1, seed=9)).cuda()
-    # graph
+    # graph (the benchmark's launch configuration)
     sg = hgd.State(model, 1, 1, Lmax, init)
     am_g = torch.zeros(1, dtype=torch.int32, device="cuda")
     am_g.view(1, 1).copy_(tok0)
@@ -302,6 +302,57 @@ def test_full_stack_end_to_end_within_rounding_noise(hgd, orc, orc32, full):
         top2 = np.sort(r64[s].astype(np.float32))[-2:]
         if top2[1] - top2[0] > 4 * noise_max:
             assert int(np.argmax(lg_gpu[s])) == int(np.argmax(r64[s].astype(np.float32)))
+
+
+def _run_paths(hgd, model, cfg, B, T, Lmax, steps, seed):
+    """The same calls through hgd_decode_layer_stack (one persistent launch when
+    B*T <= 8) and through the per-layer range entry (a chain of kernels)."""
+    import torch
+    n_gdn, _ = syn.layer_counts(cfg)
+    H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+    Cc = 2 * H * dk + H * dv
+    V, L = cfg["vocab"], cfg["n_layers"]
+    init = syn.stack_state(cfg, B, Lmax, prefill=16 if Lmax < 100 else 512, seed=seed)
+    toks = syn.stack_tokens(cfg, B, T * steps, seed=seed)
+    outs = []
+    for path in ("persistent", "chain"):
+        st = hgd.State(model, B, T, Lmax, init)
+        res = []
+        for k in range(steps):
+            tk = torch.from_numpy(np.ascontiguousarray(toks[:, k * T:(k + 1) * T])).cuda()
+            lg = torch.full((B * T, V), float("nan"), device="cuda")
+            am = torch.full((B * T,), -7, dtype=torch.int32, device="cuda")
+            sr = torch.full((n_gdn, B, T, H, dv, dk), float("nan"), device="cuda")
+            tr = torch.full((n_gdn, B, T, kc - 1, Cc), float("nan"), device="cuda")
+            status = torch.zeros(1, dtype=torch.int32, device="cuda")
+            if path == "persistent":
+                hgd.decode_layer_stack(model, st, tk, T, logits=lg, argmax=am, S_rec=sr, tail_rec=tr, status=status)
+            else:
+                hgd.decode_layer_stack_range(model, st, tk, T, 0, L, True, logits=lg, argmax=am, S_rec=sr,
+                                             tail_rec=tr, status=status)
+            torch.cuda.synchronize()
+            assert int(status.item()) == 0
+            res.append((lg, am, sr, tr))
+        outs.append((res, st))
+    return outs
+
+
+@pytest.mark.parametrize("which", ["small", "full"])
+def test_persistent_launch_equals_kernel_chain(hgd, full, which):
+    """One cooperative launch per call equals the chain of per-phase kernels bit
+    for bit: logits, argmax, per-row state and conv-tail records, final state."""
+    import torch
+    if which == "small":
+        cfg, model, B, T, Lmax = syn.SMALL_CFG, hgd.Model(syn.SMALL_CFG, weights("small", 5)), 2, 3, 40
+    else:
+        cfg, model, B, T, Lmax = syn.STACK_CFG, full[0], 1, 1, 640
+    assert model.launches(B, T) == 1
+    (rp, sp), (rc, sc) = _run_paths(hgd, model, cfg, B, T, Lmax, 3, 13)
+    for k, ((l1, a1, s1, t1), (l2, a2, s2, t2)) in enumerate(zip(rp, rc)):
+        assert torch.equal(l1, l2), f"call {k}: logits differ"
+        assert torch.equal(a1, a2) and torch.equal(s1, s2) and torch.equal(t1, t2), f"call {k}"
+    for a, b in ((sp.S, sc.S), (sp.conv, sc.conv), (sp.kv, sc.kv), (sp.pos, sc.pos)):
+        assert torch.equal(a, b)
 
 
 # ------------------------------------------------------------- windows ------
