@@ -41,12 +41,13 @@ WORKLOAD = ("24-layer hybrid stack (3 GDN : 1 gated attention), hidden 1024, voc
 def chain_launches(cfg: dict) -> int:
     """Kernels one B=1, T=1 step launches on the kernel-chain path: per GDN layer
     in-projection (with the conv tail), mixer, out-projection, SwiGLU, down; per
-    attention layer the same with RoPE/append, partials and merge as the mixer;
-    then the LM head and the argmax finalisation."""
+    attention layer the same with partials and merge as the mixer (RoPE and the
+    KV append run in the in-projection); then the LM head and the argmax
+    finalisation."""
     import hgd_synth as syn
 
     n_gdn, n_att = syn.layer_counts(cfg)
-    return n_gdn * 5 + n_att * 7 + 2
+    return n_gdn * 5 + n_att * 6 + 2
 
 
 def algorithmic_bytes(cfg: dict, L_keys: float) -> dict:

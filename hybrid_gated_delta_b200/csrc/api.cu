@@ -181,8 +181,9 @@ int run_gemv(GemvParams p, int M, int sms, void* ws, size_t ws_bytes, cudaStream
         if (q.o) q.o += m0 * q.o_ld;
         if (q.z) q.z += m0 * q.z_ld;
         if (q.resid) q.resid += m0 * q.resid_ld;
+        if (q.rope_q) q.rope_q += (size_t)m0 * q.rope_nq * q.rope_hd;
         if (q.y) {
-            const int es = (EPI == EPI_F32 || EPI == EPI_QKV_CONV) ? 4 : 2;
+            const int es = (EPI == EPI_F32 || EPI == EPI_QKV_CONV || EPI == EPI_ROPE) ? 4 : 2;
             q.y = reinterpret_cast<uint8_t*>(q.y) + (size_t)m0 * q.y_ld * es;
         }
         if (q.logits) q.logits += m0 * q.logits_ld;
@@ -262,8 +263,9 @@ size_t weight_numel(const Dims& d, const hgd_config* c, int layer, int t) {
 }
 
 // How a tensor is stored: 0 plain, 1 packed matrix, 2 / 3 gate / up half of the
-// packed SwiGLU region (which the gate tensor owns).  rows x cols is its logical
-// shape for the packed kinds.
+// packed SwiGLU region (which the gate tensor owns), 4 packed attention
+// in-projection in rope_src_row's row order.  rows x cols is its logical shape
+// for the packed kinds.
 struct WeightKind { int kind; int64_t rows, cols; };
 
 WeightKind weight_kind(const Dims& d, const hgd_config* c, int layer, int t) {
@@ -273,7 +275,7 @@ WeightKind weight_kind(const Dims& d, const hgd_config* c, int layer, int t) {
     }
     const bool att = is_attn_layer(c, layer);
     switch (t) {
-        case HGD_W_IN: return {1, att ? d.attn_out : d.gdn_out, d.D};
+        case HGD_W_IN: return att ? WeightKind{4, d.attn_out, d.D} : WeightKind{1, d.gdn_out, d.D};
         case HGD_W_OUT: return {1, d.D, att ? (int64_t)d.nq * d.hd : (int64_t)d.H * d.dv};
         case HGD_W_GATE: return {2, d.I, d.D};
         case HGD_W_UP: return {3, d.I, d.D};
@@ -286,7 +288,7 @@ WeightKind weight_kind(const Dims& d, const hgd_config* c, int layer, int t) {
 size_t weight_bytes(const Dims& d, const hgd_config* c, int layer, int t) {
     const WeightKind k = weight_kind(d, c, layer, t);
     switch (k.kind) {
-        case 1: return (size_t)((k.rows + 15) / 16) * 16 * k.cols * 2;
+        case 1: case 4: return (size_t)((k.rows + 15) / 16) * 16 * k.cols * 2;
         case 2: return (size_t)((k.rows + 7) / 8) * 16 * k.cols * 2;
         case 3: return 0;
         default: return weight_numel(d, c, layer, t) * 2;
@@ -316,6 +318,18 @@ enum ScratchIdx {
     SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
     SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_END, SC_COUNT
 };
+// The persistent launch's control region: control words, one 128-byte line per
+// phase counter, then the phase timestamps.
+constexpr size_t kBarCtrlBytes = (size_t)(SK_CTRL_WORDS + SK_MCNT_WORDS) * 4;
+constexpr size_t kBarTraceOff = kBarCtrlBytes + (size_t)SK_MAX_PHASES * SK_CTR_STRIDE * 4;
+#ifdef HGD_TRACE_DETAIL
+// instrumented builds also keep every CTA's phase times after the timestamps
+constexpr size_t kBarDetailOff = kBarTraceOff + (size_t)SK_TRACE_SLOTS * 8;
+constexpr size_t kBarSlabOff = kBarDetailOff + (size_t)SK_MAX_PHASES * SK_TRACE_CTAS * 4 * 8;
+constexpr size_t kBarBytes = kBarSlabOff + (size_t)SK_TRACE_SLABS * 3 * 8;
+#else
+constexpr size_t kBarBytes = kBarTraceOff + (size_t)SK_TRACE_SLOTS * 8;
+#endif
 constexpr int kBestG = 4096;  // max CTAs of the LM-head launch
 
 int max_chunks_of(int Lmax) { return (Lmax + ATTN_CHUNK - 1) / ATTN_CHUNK; }
@@ -349,7 +363,7 @@ void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     sz[SC_BESTV] = (size_t)M * kBestG * 4;
     sz[SC_BESTI] = (size_t)M * kBestG * 4;
     sz[SC_WS] = stack_ws_bytes(d, (int)M);
-    sz[SC_BAR] = 64 + 256 * 8;  // grid-barrier words and phase timestamps of the persistent launch
+    sz[SC_BAR] = kBarBytes;
     size_t pos = 0;
     for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
     off[SC_END] = pos;
@@ -362,20 +376,29 @@ int check_state_dims(int B, int Tmax, int Lmax) {
 }
 
 // ------------------------------------------------------- persistent launch
-size_t sk_x_bytes(const Dims& d) {
-    const int kmax = std::max(std::max(d.D, d.H * d.dv), std::max(d.nq * d.hd, d.I));
-    return (size_t)gv_align16(8 * (kmax + GV_PAD) * 2);
+int sk_kmax(const Dims& d) { return std::max(std::max(d.D, d.H * d.dv), std::max(d.nq * d.hd, d.I)); }
+
+constexpr int kSkPartialSlabs = 32;  // slab partials of the non-split phases' rounds
+
+// Ring slots of the persistent launch for M token rows: the most (24, 16 or 8)
+// that fit beside the token rows and the fixed buffers; 0 if none fits.
+int sk_ring_slots(const Dims& d, int M) {
+    for (int ns = 24; ns >= 8; ns -= 8) {
+        const size_t smem = (size_t)ns * SK_SLAB_BYTES + sk_fixed_bytes(M, sk_kmax(d), d.D, kSkPartialSlabs, ns);
+        if (smem <= (size_t)GV_SMEM_LIMIT) return ns;
+    }
+    return 0;
 }
 
-size_t sk_smem_bytes(const Dims& d) {
-    return (size_t)SK_NSLOT * SK_SLAB_BYTES + sk_x_bytes(d) + (size_t)SK_CW * GV_ROWS * 8 * 4 +
-           (size_t)SK_CW * 8 * 8 + (size_t)SK_CW * 32 * 4 + 2 * 8 * SK_NSLOT + 32;
+size_t sk_smem_bytes(const Dims& d, int M, int ns) {
+    return (size_t)ns * SK_SLAB_BYTES + sk_fixed_bytes(M, sk_kmax(d), d.D, kSkPartialSlabs, ns);
 }
 
 // The persistent launch covers calls of at most one MMA n-tile of token rows
 // with a GDN key width of 64 or 128 and a shared-memory footprint that fits.
 bool sk_supported(const Dims& d, int M) {
-    return M <= SK_MAXM && (d.dk == 64 || d.dk == 128) && sk_smem_bytes(d) <= (size_t)GV_SMEM_LIMIT;
+    return M <= SK_MAXM && (d.dk == 64 || d.dk == 128) && d.L * SK_PHASES_PER_LAYER + 2 <= SK_MAX_PHASES &&
+           gv_slabs(sk_kmax(d)) <= kSkPartialSlabs && M * d.nq <= SK_MCNT_WORDS && sk_ring_slots(d, M) > 0;
 }
 
 template <int KPL>
@@ -564,11 +587,12 @@ int hgd_model_load_tensor(const hgd_config* cfg, void* arena, size_t arena_bytes
         const int blocks = (int)std::min<int64_t>(((int64_t)n + 255) / 256, 4096);
         e = launch_pdl(k_copy_u16, dim3(blocks), dim3(256), 0, s, (const bf16_t*)src, dst, (int64_t)n);
     } else {
-        const int nrb = (k.kind == 1) ? (int)((k.rows + 15) / 16) : (int)((k.rows + 7) / 8);
+        const int nrb = (k.kind == 1 || k.kind == 4) ? (int)((k.rows + 15) / 16) : (int)((k.rows + 7) / 8);
         const int64_t chunks = (int64_t)nrb * (k.cols / 32) * 64;
         const int blocks = (int)std::min<int64_t>((chunks + 255) / 256, 8192);
+        const int mode = k.kind == 1 ? 0 : k.kind == 2 ? 1 : k.kind == 3 ? 2 : 3;
         e = launch_pdl(k_pack_weight, dim3(blocks), dim3(256), 0, s, (const bf16_t*)src, dst, (int)k.rows,
-                       (int)k.cols, nrb, k.kind == 1 ? 0 : (k.kind == 2 ? 1 : 2));
+                       (int)k.cols, nrb, mode, d.nq, d.nkv, d.hd);
     }
     return launch_status(e);
 }
@@ -660,7 +684,7 @@ int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T) {
     for (int l = 0; l < d.L; ++l) {
         const bool att = is_attn_layer(&m->cfg, l);
         n += gemv_chunks(M, d.D);                                   // in-projection
-        n += att ? 3 : 1;                                           // rope/partial/merge or GDN mixer
+        n += att ? 2 : 1;                                           // partial/merge or GDN mixer
         n += gemv_chunks(M, att ? d.nq * d.hd : d.H * d.dv);        // out-projection
         n += gemv_chunks(M, d.D) + gemv_chunks(M, d.I);             // SwiGLU, down
     }
@@ -691,9 +715,10 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
     prm.L = d.L; prm.D = d.D; prm.V = d.V; prm.H = d.H; prm.dk = d.dk; prm.dv = d.dv; prm.nq = d.nq;
     prm.nkv = d.nkv; prm.hd = d.hd; prm.I = d.I; prm.every = d.every;
     prm.C = (int)d.C; prm.gdn_out = (int)d.gdn_out; prm.attn_out = (int)d.attn_out;
-    prm.proj_ld = (int)std::max(d.gdn_out, d.attn_out);
+    prm.proj_ld = (int)std::max(d.gdn_out, d.attn_out); prm.kmax = sk_kmax(d);
     prm.eps = m->cfg.norm_eps; prm.rope_base = m->cfg.rope_base;
     prm.B = st->B; prm.T = T; prm.M = st->B * T; prm.Lmax = st->Lmax; prm.max_chunks = max_chunks_of(st->Lmax);
+    prm.ns = sk_ring_slots(d, prm.M); prm.pb = kSkPartialSlabs;
     prm.embed = m->embed; prm.final_norm = m->final_norm;
     prm.S = reinterpret_cast<float*>(A + st->off[SC_S]);
     prm.conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
@@ -703,24 +728,31 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
     prm.proj = reinterpret_cast<float*>(A + st->off[SC_PROJ]);
     prm.obuf = reinterpret_cast<float*>(A + st->off[SC_O]);
     prm.qrot = reinterpret_cast<float*>(A + st->off[SC_QROT]);
-    prm.attn = reinterpret_cast<bf16_t*>(A + st->off[SC_ATTN]);
     prm.part = reinterpret_cast<float*>(A + st->off[SC_PART]);
     prm.mlp = reinterpret_cast<bf16_t*>(A + st->off[SC_MLP]);
+    prm.attn = reinterpret_cast<bf16_t*>(A + st->off[SC_ATTN]);
     prm.bestv = reinterpret_cast<float*>(A + st->off[SC_BESTV]);
     prm.besti = reinterpret_cast<int32_t*>(A + st->off[SC_BESTI]);
-    prm.ws_cnt = reinterpret_cast<int32_t*>(A + st->off[SC_WS]);
-    prm.ws_part = reinterpret_cast<float*>(A + st->off[SC_WS] + kWsCounterBytes);
     prm.tokens = tokens; prm.logits = logits; prm.argmax = argmax; prm.S_rec = S_rec; prm.tail_rec = tail_rec;
     prm.status = status_dev;
     prm.bar = reinterpret_cast<unsigned*>(A + st->off[SC_BAR]);
-    prm.trace = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + 64);
-    prm.x_bytes = (int)sk_x_bytes(d);
+    prm.mcnt = prm.bar + SK_CTRL_WORDS;
+    prm.trace = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarTraceOff);
+#ifdef HGD_TRACE_DETAIL
+    prm.tdetail = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarDetailOff);
+    prm.tslab = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarSlabOff);
+#endif
     for (int l = 0; l < d.L; ++l)
         for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) prm.layer[l].w[t] = m->w[l][t];
     cudaStream_t s = (cudaStream_t)stream;
-    // a fresh barrier for this call (an earlier call may have stopped on a timeout)
-    if (cudaMemsetAsync(prm.bar, 0, 64, s) != cudaSuccess) { cudaGetLastError(); return HGD_ERR_CUDA; }
-    const size_t smem = sk_smem_bytes(d);
+    // fresh control words and phase counters for this call (an earlier call may
+    // have stopped on a timeout)
+    const size_t nph = (size_t)d.L * SK_PHASES_PER_LAYER + 2;
+    if (cudaMemsetAsync(prm.bar, 0, kBarCtrlBytes + nph * SK_CTR_STRIDE * 4, s) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
+    }
+    const size_t smem = sk_smem_bytes(d, prm.M, prm.ns);
     return d.dk == 128 ? sk_launch_t<4>(prm, smem, di.sms, s) : sk_launch_t<2>(prm, smem, di.sms, s);
 }
 
@@ -778,6 +810,12 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             p.W = w[HGD_W_IN]; p.packed = 1; p.N = (int)(att ? d.attn_out : d.gdn_out); p.K = d.D;
             p.x = resid; p.x_ld = d.D; p.norm_w = w[HGD_W_IN_NORM]; p.eps = eps;
             p.y = proj; p.y_ld = proj_ld; p.status = status_dev;
+            if (att) {
+                p.rope_nq = d.nq; p.rope_nkv = d.nkv; p.rope_hd = d.hd; p.rope_Lmax = Lmax;
+                p.rope_base = m->cfg.rope_base; p.rope_q = qrot;
+                p.rope_k = kv + (size_t)ia * 2 * kv_half; p.rope_v = p.rope_k + kv_half;
+                p.rope_pos = pos; p.conv_T = T;
+            }
             if (l == 0) {
                 p.tokens = tokens; p.embed = m->embed; p.vocab = d.V; p.resid_out = resid; p.resid_out_ld = d.D;
             }
@@ -788,8 +826,8 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
                 rc = (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s)
                               : run_gemv<PRO_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s);
             } else {
-                rc = (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_F32>(p, M, di.sms, ws, ws_bytes, s)
-                              : run_gemv<PRO_RMSNORM, EPI_F32>(p, M, di.sms, ws, ws_bytes, s);
+                rc = (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_ROPE>(p, M, di.sms, ws, ws_bytes, s)
+                              : run_gemv<PRO_RMSNORM, EPI_ROPE>(p, M, di.sms, ws, ws_bytes, s);
             }
             if (rc) return rc;
         }
@@ -823,10 +861,8 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             a.kcache = kv + (size_t)ia * 2 * kv_half; a.vcache = a.kcache + kv_half;
             a.pos = pos; a.part = part; a.out = attn; a.status = status_dev;
             a.B = B; a.T = T; a.nq = d.nq; a.nkv = d.nkv; a.hd = d.hd; a.Lmax = Lmax;
-            a.max_chunks = max_chunks_of(Lmax); a.rope_base = m->cfg.rope_base;
-            cudaError_t e = launch_pdl(k_rope_append, dim3(M), dim3(256), 0, s, a);
-            if ((rc = launch_status(e))) return rc;
-            e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(32 * (d.nq / d.nkv)), 0, s, a);
+            a.max_chunks = max_chunks_of(Lmax);
+            cudaError_t e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(32 * (d.nq / d.nkv)), 0, s, a);
             if ((rc = launch_status(e))) return rc;
             e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
             if ((rc = launch_status(e))) return rc;

@@ -41,7 +41,8 @@ constexpr int GV_PAD = 8;                      // bf16 elements of padding per t
 constexpr int GV_SMEM_LIMIT = 227 * 1024;
 
 enum GvPrologue { PRO_COPY = 0, PRO_RMSNORM = 1, PRO_EMBED_RMSNORM = 2, PRO_GATED_NORM = 3 };
-enum GvEpilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_ARGMAX = 4, EPI_QKV_CONV = 5 };
+enum GvEpilogue { EPI_F32 = 0, EPI_BF16 = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_ARGMAX = 4, EPI_QKV_CONV = 5,
+                  EPI_ROPE = 6 };
 constexpr int GV_CONV_K = 4;  // conv width of the fused conv epilogue
 
 struct GemvParams {
@@ -75,6 +76,13 @@ struct GemvParams {
     // tail [B][3][conv_C] shifted in place, tail records [B][T][3][conv_C] (or null).
     // Token row m of this launch is stream (m0 + m) / conv_T, row (m0 + m) % conv_T.
     const bf16_t* conv_w; float* conv_tail; float* conv_rec; int conv_C, conv_T, m0;
+    // ROPE: the attention in-projection, packed with rope_src_row's row order:
+    // q rows are rotated and stored fp32 in rope_q [M][nq*hd]; gate rows go to y
+    // (fp32) at column nq*hd + g; k rows are rotated and v rows copied into the
+    // bf16 caches [B][nkv][Lmax][hd] at position pos[b] + t (row m0 + m is stream
+    // (m0 + m) / conv_T, row (m0 + m) % conv_T).
+    int rope_nq, rope_nkv, rope_hd, rope_Lmax; float rope_base;
+    float* rope_q; bf16_t* rope_k; bf16_t* rope_v; const int32_t* rope_pos;
     int32_t* status;
 };
 
@@ -109,6 +117,35 @@ __host__ __device__ inline int64_t gv_tile_elem(int64_t rb, int step, int steps,
 __host__ __device__ inline int64_t gv_packed_chunk(int64_t n, int cc, int steps) {
     const int i = (int)(n & 15);
     return gv_tile_elem(n >> 4, cc >> 2, steps, i >> 3, ((i & 7) << 2) | (cc & 3));
+}
+
+// Row order of the packed attention in-projection [q | gate | k | v] (rows of
+// nq*hd, nq*hd, nkv*hd, nkv*hd): within each q and k head the 16-row block j
+// holds dims 8j..8j+7 in its rows 0..7 and their rotate-half partners
+// hd/2 + 8j .. +7 in rows 8..15, so one lane's accumulators hold both halves of
+// a RoPE pair; gate and v rows keep their order.  Returns the source row of
+// virtual row v (a bijection on [0, 2*nq*hd + 2*nkv*hd)).
+__host__ __device__ inline int64_t rope_src_row(int64_t v, int nq, int nkv, int hd) {
+    const int64_t qw = (int64_t)nq * hd, kw = (int64_t)nkv * hd;
+    int64_t base, w;
+    if (v < qw) { base = 0; w = v; }
+    else if (v < 2 * qw) return v;
+    else if (v < 2 * qw + kw) { base = 2 * qw; w = v - 2 * qw; }
+    else return v;
+    const int64_t head = w / hd;
+    const int r = (int)(w % hd), j = r >> 4, i16 = r & 15;
+    const int dim = (i16 < 8) ? 8 * j + i16 : hd / 2 + 8 * j + (i16 - 8);
+    return base + head * hd + dim;
+}
+
+// sin and cos of the RoPE angle of dim pair i at position P: the angle
+// P * base^(-2i/hd) in double, reduced to [-pi, pi] in double, then fp32.
+__device__ __forceinline__ void rope_sincos(int P, int i, int hd, float base, float* sn, float* cs) {
+    const double inv = exp2(-2.0 * (double)i / (double)hd * log2((double)base));
+    const double th = (double)P * inv;
+    const double tw = 6.283185307179586476925286766559;
+    const float r = (float)(th - tw * rint(th / tw));
+    sincosf(r, sn, cs);
 }
 
 __device__ __forceinline__ float ld_cg(const float* p) {
@@ -355,6 +392,54 @@ __device__ __forceinline__ void gv_finish(const GemvParams& p, int rb, int s_ite
                 }
             }
             __syncwarp();
+        } else if (EPI == EPI_ROPE) {
+            const int hd = p.rope_hd, half = hd >> 1, hb = hd >> 4;  // 16-row blocks per head
+            const int qrb = p.rope_nq * hb, krb = p.rope_nkv * hb, qw = p.rope_nq * hd;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int n = nt * 8 + 2 * c + h2;
+                    if (n >= p.M) continue;
+                    const float a = yacc[nt][h2], bb = yacc[nt][2 + h2];  // rows r8 and r8 + 8
+                    const int gm = p.m0 + n, b = gm / p.conv_T, t = gm % p.conv_T;
+                    const int P = p.rope_pos[b] + t;
+                    const bool bad = P < 0 || P >= p.rope_Lmax;
+                    if (rb >= 2 * qrb + krb) {  // value rows: appended to the V cache
+                        if (bad) continue;
+                        const int vc = (rb - 2 * qrb - krb) * GV_ROWS + r8;
+                        const int g = vc / hd, d = vc % hd;  // vc and vc + 8 share a head (hd % 16 == 0)
+                        bf16_t* vo = p.rope_v + (((int64_t)b * p.rope_nkv + g) * p.rope_Lmax + P) * hd;
+                        vo[d] = f2bf(a);
+                        vo[d + 8] = f2bf(bb);
+                    } else if (rb >= qrb && rb < 2 * qrb) {  // output-gate rows
+                        const int gc = (rb - qrb) * GV_ROWS + r8;
+                        float* y = reinterpret_cast<float*>(p.y) + (int64_t)n * p.y_ld + qw;
+                        y[gc] = a;
+                        y[gc + 8] = bb;
+                    } else {  // q or k rows: the rotate-half pair (i, i + hd/2)
+                        const bool isk = rb >= qrb;
+                        const int rr = isk ? rb - 2 * qrb : rb;
+                        const int head = rr / hb, i = (rr % hb) * 8 + r8;
+                        if (bad) {
+                            if (isk) set_status(p.status, HGD_ERR_INVALID_ARG);
+                            continue;
+                        }
+                        float sn, cs;
+                        rope_sincos(P, i, hd, p.rope_base, &sn, &cs);
+                        const float x0 = a * cs - bb * sn, x1 = bb * cs + a * sn;
+                        if (!isk) {
+                            float* qo = p.rope_q + (int64_t)n * qw + (int64_t)head * hd;
+                            qo[i] = x0;
+                            qo[i + half] = x1;
+                        } else {
+                            bf16_t* ko = p.rope_k + (((int64_t)b * p.rope_nkv + head) * p.rope_Lmax + P) * hd;
+                            ko[i] = f2bf(x0);
+                            ko[i + half] = f2bf(x1);
+                        }
+                    }
+                }
+            }
         } else {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -551,11 +636,12 @@ __global__ void __launch_bounds__(GV_THREADS, (NT >= 4) ? 1 : 2) k_gemv(const __
 
 // Pack a row-major [rows][K] bf16 matrix into the fragment-ordered tiles.
 // mode 0: plain (virtual row v = logical row v); mode 1 / 2: the gate / up half
-// of a SwiGLU pair (tile rows 0..7 / 8..15 of row block rb are rows 8rb..8rb+7).
+// of a SwiGLU pair (tile rows 0..7 / 8..15 of row block rb are rows 8rb..8rb+7);
+// mode 3: the attention in-projection in rope_src_row's order.
 // One thread per 16-byte destination chunk; chunks of the other half are left
 // untouched in modes 1 and 2; rows past the matrix are written as zero.
 __global__ void k_pack_weight(const bf16_t* __restrict__ src, bf16_t* __restrict__ dst, int rows, int K,
-                              int n_rowblk, int mode) {
+                              int n_rowblk, int mode, int rope_nq, int rope_nkv, int rope_hd) {
     const int steps = K >> 5;
     const int64_t total = (int64_t)n_rowblk * steps * 64;
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total;
@@ -566,7 +652,9 @@ __global__ void k_pack_weight(const bf16_t* __restrict__ src, bf16_t* __restrict
         const int64_t rb = tile / steps;
         const int step = (int)(tile % steps);
         const int i = (lane >> 2) + 8 * half, c = lane & 3;
-        const int64_t row = mode == 0 ? rb * 16 + i : rb * 8 + (i & 7);
+        const int64_t row = mode == 0 ? rb * 16 + i
+                          : mode == 3 ? rope_src_row(rb * 16 + i, rope_nq, rope_nkv, rope_hd)
+                                      : rb * 8 + (i & 7);
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row < rows) v = *reinterpret_cast<const uint4*>(src + row * K + step * 32 + 8 * c);
         *reinterpret_cast<uint4*>(dst + gv_tile_elem(rb, step, steps, half, lane)) = v;

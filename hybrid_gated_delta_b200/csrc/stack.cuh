@@ -1,27 +1,38 @@
 // stack.cuh -- one cooperative launch for a whole decode step of the stack.
 //
 // "luce-megakernel HANDOFF.md", Architecture: all 24 layers of the decode step
-// in one persistent kernel with grid synchronisation between layers (and its
-// Known Issues: a grid sync deadlocks unless every block is resident, hence a
-// cooperative launch).  Built for B200 here:
+// in one persistent kernel with synchronisation between layers (and its Known
+// Issues: a grid-wide wait deadlocks unless every block is resident, hence a
+// cooperative launch).  Built for B200 here, as a dataflow of phases:
 //  * one CTA per SM: a producer warp and eight consumer warps;
-//  * the producer walks the CTA's share of every projection of the step, in
-//    order, and streams each 16-row x 256-column weight slab (8 KB, contiguous
-//    thanks to the fragment-ordered packing) with one bulk copy (cp.async.bulk,
-//    no multicast, L2 evict-first) into the two-slot ring of the consumer warp
-//    that owns it, feeding the warps slab by slab in turn.  Weights never depend
-//    on activations, so it runs ahead across phase boundaries and keeps HBM busy
-//    while the consumers wait at a grid barrier.  Each warp waits on its own
-//    slots strictly in order, so an mbarrier phase parity never aliases;
-//  * the consumers run the phases in order -- per GDN layer: in-projection with
-//    the fused causal conv, gated delta rule, out-projection with the gated
-//    RMSNorm, SwiGLU, down-projection; per attention layer: in-projection, RoPE
-//    and KV append, attention partials, merge, out-projection, SwiGLU, down; then
-//    the LM head with the argmax -- and meet at a grid barrier after each;
-//  * every phase runs the same per-row arithmetic as the per-kernel path (the
-//    same device functions, the same slab order), so the two agree bit for bit;
+//  * weights never depend on activations, so the producer walks the CTA's share
+//    of every projection of the step in order and streams each 16-row x
+//    256-column weight slab (8 KB, contiguous thanks to the fragment-ordered
+//    packing) with one bulk copy (cp.async.bulk, no multicast, L2 evict-first)
+//    into a CTA-wide ring of NS slots, across phase boundaries: HBM stays busy
+//    while the consumers wait for the previous phase.  Slab g of the CTA's
+//    sequence sits in slot g % NS and is consumed by warp g % 8 (NS is a
+//    multiple of 8), so each slot is only ever waited on by one warp, strictly
+//    in order, and an mbarrier phase parity never aliases;
+//  * per layer five phases -- GDN: in-projection with the fused causal conv,
+//    gated delta rule, out-projection with the gated RMSNorm, SwiGLU, down;
+//    attention: in-projection with the fused RoPE and KV append, attention
+//    partials, out-projection with the fused merge, SwiGLU, down -- then the LM
+//    head with the argmax and the final argmax reduction;
+//  * phases synchronise through monotonic counters, one per phase: each CTA
+//    adds 1 (red.release) once its writes of phase p are done, and phase p + 1
+//    starts when the counter of phase p reaches the grid size (ld.acquire);
+//  * a work item is a whole 16-row block (its slabs spread over the warps, the
+//    partials gathered in shared memory and added in slab order by the item's
+//    warp), so each projection's epilogue -- residual add included -- runs
+//    where the row is finished and the next phase reads only the residual
+//    rows.  Items go to CTA (phase rotation + item) % grid, so phases with
+//    fewer row blocks than CTAs land on different SMs from layer to layer and
+//    the weight stream stays spread over all of them;
+//  * every output has the arithmetic of the kernel chain (the same device
+//    functions, the same slab order), so the two agree bit for bit;
 //  * every wait is bounded; a wait that runs out sets HGD_ERR_TIMEOUT and a
-//    global abort flag, after which every CTA skips the remaining work.
+//    global abort word, after which every CTA skips the remaining work.
 #pragma once
 
 #include "attn.cuh"
@@ -31,40 +42,56 @@
 namespace hgd {
 
 constexpr int SK_CW = 8;                        // consumer warps
-constexpr int SK_THREADS = (SK_CW + 1) * 32;    // + the producer warp
+constexpr int SK_CT = SK_CW * 32;               // consumer threads
+constexpr int SK_THREADS = SK_CT + 32;          // + the producer warp
 constexpr int SK_SLAB_BYTES = GV_SLAB_STEPS * 1024;
-constexpr int SK_NSW = 2;                       // ring slots per consumer warp
-constexpr int SK_NSLOT = SK_CW * SK_NSW;        // 16 slots (128 KB)
+constexpr int SK_PB_SLAB = GV_ROWS * 8;         // floats of one slab partial in the partial buffer
 constexpr int SK_MAXM = 8;                      // token rows per call (one MMA n-tile)
+constexpr int SK_PHASES_PER_LAYER = 5;
+constexpr int SK_MAX_PHASES = SK_PHASES_PER_LAYER * HGD_MAX_LAYERS + 2;
+// control words: [0] abort, [1] what ran out first (1 phase counter, 2 weight
+// slab, 3 free ring slot), [2] its phase, [3] its CTA, [4] its sequence number;
+// then the attention merge counters [M][nq] (SK_MCNT_WORDS); the counter of
+// phase p is word SK_CTRL_WORDS + SK_MCNT_WORDS + p * SK_CTR_STRIDE (own 128 B)
+constexpr int SK_CTRL_WORDS = 32;
+constexpr int SK_MCNT_WORDS = 1024;
+constexpr int SK_CTR_STRIDE = 32;
+constexpr int SK_TRACE_SLOTS = 512;             // phase start times of CTA 0; the end in the last
+constexpr int SK_TRACE_CTAS = 256;              // CTAs the per-CTA phase times cover
+constexpr int SK_TRACE_SLABS = 4096;            // slabs of CTA 0 the slab times cover
 
-enum SkKind { SK_IN_GDN = 0, SK_GDN, SK_OUT_GDN, SK_IN_ATT, SK_ROPE, SK_PART, SK_MERGE, SK_OUT_ATT, SK_SWIGLU,
-              SK_DOWN, SK_HEAD, SK_FINAL };
+enum SkKind { SK_IN_GDN = 0, SK_GDN, SK_OUT_GDN, SK_IN_ATT, SK_PART, SK_OUT_ATT, SK_SWIGLU, SK_DOWN, SK_HEAD,
+              SK_FINAL };
 
 struct SkLayer { const bf16_t* w[HGD_W_LAYER_COUNT]; };
 
 struct SkParams {
     int L, D, V, H, dk, dv, nq, nkv, hd, I, every;
-    int C, gdn_out, attn_out, proj_ld;
+    int C, gdn_out, attn_out, proj_ld, kmax;
     float eps, rope_base;
     int B, T, M, Lmax, max_chunks;
+    int ns, pb;      // ring slots (a multiple of SK_CW), slab partials the partial buffer holds
     const bf16_t* embed; const bf16_t* final_norm;
     float* S; float* conv; bf16_t* kv; int32_t* pos;
-    bf16_t* resid; float* proj; float* obuf; float* qrot; bf16_t* attn; float* part; bf16_t* mlp;
-    float* bestv; int32_t* besti; float* ws_part; int32_t* ws_cnt;
+    bf16_t* resid;   // [M][D] residual rows (updated in place by the out- and down-projections)
+    float* proj; float* obuf; float* qrot; float* part; bf16_t* mlp;
+    bf16_t* attn;    // [M][nq*hd] merged attention output
+    unsigned* mcnt;  // [M][nq] chunks finished per (row, head), zero between layers
+    float* bestv; int32_t* besti;
     const int32_t* tokens; float* logits; int32_t* argmax; float* S_rec; float* tail_rec;
     int32_t* status;
-    unsigned* bar;   // [0] arrivals, [1] generation, [2] abort, [4..13] where the first wait ran out
-    unsigned long long* trace;  // %globaltimer at the start of each phase (CTA 0), or null
-    int x_bytes;
+    unsigned* bar;               // control words and phase counters (zeroed before the launch)
+    unsigned long long* trace;   // [SK_TRACE_SLOTS] %globaltimer, or null
+    unsigned long long* tdetail; // [SK_MAX_PHASES][SK_TRACE_CTAS][4] per-CTA phase times, or null
+    unsigned long long* tslab;   // CTA 0: [SK_TRACE_SLABS][3] slab issue / ready / release times, or null
     SkLayer layer[HGD_MAX_LAYERS];
 };
 
 __device__ __forceinline__ bool sk_attn(const SkParams& s, int l) { return l % s.every == s.every - 1; }
-__device__ __forceinline__ int sk_nphase(const SkParams& s, int l) { return sk_attn(s, l) ? 7 : 5; }
 __device__ __forceinline__ int sk_kind(const SkParams& s, int l, int j) {
     if (l == s.L) return j == 0 ? SK_HEAD : SK_FINAL;
     static constexpr int gdn[5] = {SK_IN_GDN, SK_GDN, SK_OUT_GDN, SK_SWIGLU, SK_DOWN};
-    static constexpr int att[7] = {SK_IN_ATT, SK_ROPE, SK_PART, SK_MERGE, SK_OUT_ATT, SK_SWIGLU, SK_DOWN};
+    static constexpr int att[5] = {SK_IN_ATT, SK_PART, SK_OUT_ATT, SK_SWIGLU, SK_DOWN};
     return sk_attn(s, l) ? att[j] : gdn[j];
 }
 __device__ __forceinline__ bool sk_is_gemv(int k) {
@@ -77,151 +104,489 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-
-// Record the first wait that ran out (what: 1 grid barrier, 2 weight slab,
-// 3 free ring slot) with its phase, CTA and ring sequence number; set the
-// status and the global abort flag.
-__device__ __forceinline__ void sk_timeout(unsigned* bar, int32_t* status, unsigned what, unsigned phase,
-                                           unsigned seq) {
-    if (atomicCAS(&bar[4], 0u, what) == 0u) {
-        bar[5] = phase;
-        bar[6] = blockIdx.x;
-        bar[7] = seq;
-    }
-    set_status(status, HGD_ERR_TIMEOUT);
-    atomicExch(&bar[2], 1u);
+// 16-byte load cached in L2 only (data written by other SMs during the launch).
+__device__ __forceinline__ float4 ld_cg4(const float* p) {
+    float4 v;
+    asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned* sk_ctr(const SkParams& s, int p) {
+    return s.bar + SK_CTRL_WORDS + SK_MCNT_WORDS + p * SK_CTR_STRIDE;
 }
 
-// The GEMV of a phase.  Row blocks below 2 per CTA split their slabs over CTAs.
-__device__ __forceinline__ void sk_gemv_params(const SkParams& s, int kind, int l, int ig, GemvParams& p) {
+// Record the first wait that ran out; set the status and the abort word.
+__device__ __forceinline__ void sk_timeout(const SkParams& s, unsigned what, unsigned phase, unsigned seq) {
+    if (atomicCAS(&s.bar[1], 0u, what) == 0u) {
+        s.bar[2] = phase;
+        s.bar[3] = blockIdx.x;
+        s.bar[4] = seq;
+    }
+    set_status(s.status, HGD_ERR_TIMEOUT);
+    atomicExch(&s.bar[0], 1u);
+}
+
+// End of phase p in this CTA: once every consumer warp's writes are done (the
+// CTA barrier orders them before thread 0's release), one release-add to the
+// phase's counter.
+__device__ __forceinline__ void sk_arrive(const SkParams& s, int p) {
+    named_bar(1, SK_CT);
+    if (threadIdx.x == 0) red_release_add(sk_ctr(s, p), 1u);
+}
+
+// Named barrier over the consumer threads that also ANDs a predicate: every
+// thread gets the same answer, so branches around later barriers stay uniform.
+__device__ __forceinline__ bool sk_bar_and(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(SK_CT)
+        : "memory");
+    return r != 0;
+}
+
+// Wait until every CTA has arrived at the end of phase p (thread 0 polls, the
+// consumer warps meet at a named barrier).  False, in every consumer thread,
+// on an abort or a timeout.
+__device__ bool sk_wait(const SkParams& s, volatile int* cta_abort, int p) {
+    if (threadIdx.x == 0 && !*cta_abort) {
+        const unsigned* c = sk_ctr(s, p);
+        const unsigned target = gridDim.x;
+        if (ld_acquire_u32(c) < target) {
+            const unsigned long long t0 = globaltimer();
+            unsigned it = 0;
+            while (ld_acquire_u32(c) < target) {
+                if ((++it & 31u) == 0u) {
+                    if (ld_acquire_u32(&s.bar[0])) { *cta_abort = 1; break; }
+                    if (globaltimer() - t0 > kWaitLimitNs) {
+                        sk_timeout(s, 1u, (unsigned)p, 0u);
+                        *cta_abort = 1;
+                        break;
+                    }
+                }
+            }
+        }
+    }
+    return sk_bar_and(!*cta_abort);
+}
+
+// GEMV parameters of a phase (the same fields the kernel chain's launch uses).
+__device__ __forceinline__ void sk_gemv_params(const SkParams& s, int kind, int l, int ig, int ia, GemvParams& p) {
     p = GemvParams{};
     const bf16_t* const* w = l < s.L ? s.layer[l].w : nullptr;
     p.packed = 1;
     p.M = s.M;
     p.eps = s.eps;
     p.status = s.status;
-    const size_t c_layer = (size_t)s.B * (GV_CONV_K - 1) * s.C;
-    const size_t trec_layer = (size_t)s.B * s.T * (GV_CONV_K - 1) * s.C;
     bool swi = false;
     switch (kind) {
-        case SK_IN_GDN: case SK_IN_ATT:
-            p.W = w[HGD_W_IN]; p.N = kind == SK_IN_GDN ? s.gdn_out : s.attn_out; p.K = s.D;
-            p.x = s.resid; p.x_ld = s.D; p.norm_w = w[HGD_W_IN_NORM];
+        case SK_IN_GDN: {
+            const size_t c_layer = (size_t)s.B * (GV_CONV_K - 1) * s.C;
+            const size_t trec_layer = (size_t)s.B * s.T * (GV_CONV_K - 1) * s.C;
+            p.W = w[HGD_W_IN]; p.N = s.gdn_out; p.K = s.D; p.norm_w = w[HGD_W_IN_NORM];
             p.y = s.proj; p.y_ld = s.proj_ld;
-            if (l == 0) { p.tokens = s.tokens; p.embed = s.embed; p.vocab = s.V; p.resid_out = s.resid; p.resid_out_ld = s.D; }
-            if (kind == SK_IN_GDN) {
-                p.conv_w = w[HGD_W_CONV]; p.conv_tail = s.conv + ig * c_layer;
-                p.conv_rec = s.tail_rec ? s.tail_rec + ig * trec_layer : nullptr;
-                p.conv_C = s.C; p.conv_T = s.T; p.m0 = 0;
-            }
+            p.conv_w = w[HGD_W_CONV]; p.conv_tail = s.conv + ig * c_layer;
+            p.conv_rec = s.tail_rec ? s.tail_rec + ig * trec_layer : nullptr;
+            p.conv_C = s.C; p.conv_T = s.T; p.m0 = 0;
             break;
+        }
+        case SK_IN_ATT: {
+            const size_t kv_half = (size_t)s.B * s.nkv * s.Lmax * s.hd;
+            p.W = w[HGD_W_IN]; p.N = s.attn_out; p.K = s.D; p.norm_w = w[HGD_W_IN_NORM];
+            p.y = s.proj; p.y_ld = s.proj_ld;
+            p.rope_nq = s.nq; p.rope_nkv = s.nkv; p.rope_hd = s.hd; p.rope_Lmax = s.Lmax; p.rope_base = s.rope_base;
+            p.rope_q = s.qrot; p.rope_k = s.kv + (size_t)ia * 2 * kv_half; p.rope_v = p.rope_k + kv_half;
+            p.rope_pos = s.pos; p.conv_T = s.T; p.m0 = 0;
+            break;
+        }
         case SK_OUT_GDN:
             p.W = w[HGD_W_OUT]; p.N = s.D; p.K = s.H * s.dv;
-            p.o = s.obuf; p.o_ld = (int64_t)s.H * s.dv; p.z = s.proj + s.C; p.z_ld = s.proj_ld;
             p.gnorm_w = w[HGD_W_GNORM]; p.gn_d = s.dv;
             p.y = s.resid; p.y_ld = s.D; p.resid = s.resid; p.resid_ld = s.D;
             break;
         case SK_OUT_ATT:
             p.W = w[HGD_W_OUT]; p.N = s.D; p.K = s.nq * s.hd;
-            p.x = s.attn; p.x_ld = (int64_t)s.nq * s.hd;
             p.y = s.resid; p.y_ld = s.D; p.resid = s.resid; p.resid_ld = s.D;
             break;
         case SK_SWIGLU:
-            p.W = w[HGD_W_GATE]; p.N = s.I; p.K = s.D; swi = true;
-            p.x = s.resid; p.x_ld = s.D; p.norm_w = w[HGD_W_POST_NORM];
+            p.W = w[HGD_W_GATE]; p.N = s.I; p.K = s.D; swi = true; p.norm_w = w[HGD_W_POST_NORM];
             p.y = s.mlp; p.y_ld = s.I;
             break;
         case SK_DOWN:
             p.W = w[HGD_W_DOWN]; p.N = s.D; p.K = s.I;
-            p.x = s.mlp; p.x_ld = s.I;
             p.y = s.resid; p.y_ld = s.D; p.resid = s.resid; p.resid_ld = s.D;
             break;
         default:  // SK_HEAD
-            p.W = s.embed; p.N = s.V; p.K = s.D;
-            p.x = s.resid; p.x_ld = s.D; p.norm_w = s.final_norm;
+            p.W = s.embed; p.N = s.V; p.K = s.D; p.norm_w = s.final_norm;
             p.logits = s.logits; p.logits_ld = s.V; p.best_v = s.bestv; p.best_i = s.besti;
             break;
     }
     p.nks = gv_slabs(p.K);
     p.n_rowblk = swi ? (p.N + 7) / 8 : (p.N + GV_ROWS - 1) / GV_ROWS;
-    p.split = (kind != SK_HEAD && p.n_rowblk < 2 * (int)gridDim.x) ? 1 : 0;
-    p.n_items = p.n_rowblk * (p.split ? p.nks : 1);
-    if (p.split) { p.ws_part = s.ws_part; p.ws_cnt = s.ws_cnt; p.ws_mp = 8; }
-    p.x_bytes = s.x_bytes;
+    p.split = 0;
+    p.n_items = p.n_rowblk;
 }
 
-// Items of this CTA in a phase of n items: c, c + G, c + 2G, ...
-__device__ __forceinline__ int sk_cta_items(int n) {
-    const int c = blockIdx.x, G = gridDim.x;
+// This CTA's place in phase `pid`'s item order (a rotation that moves from
+// phase to phase), and its items c, c + G, c + 2G, ... of n.
+__device__ __forceinline__ int sk_vcta(int pid) {
+    const int G = gridDim.x;
+    return (int)((blockIdx.x + (unsigned)pid * 37u) % (unsigned)G);
+}
+__device__ __forceinline__ int sk_cta_items(int n, int c) {
+    const int G = gridDim.x;
     return c < n ? (n - c + G - 1) / G : 0;
 }
 
-// Grid barrier among the consumer warps of all CTAs (the producer warps do not
-// take part).  Returns false if the wait ran out or an abort was raised.
-__device__ bool sk_grid_sync(const SkParams& s, volatile int* cta_abort, int phase) {
-    named_bar(1, SK_CW * 32);
-    if (threadIdx.x == 0) {
-        bool ok = !*cta_abort;
-        __threadfence();
-        const unsigned gen = ld_acquire_u32(&s.bar[1]);
-        const unsigned arrived = atomicAdd(&s.bar[0], 1u);
-        if (arrived == gridDim.x - 1) {
-            atomicExch(&s.bar[0], 0u);
-            __threadfence();
-            atomicAdd(&s.bar[1], 1u);
+// ------------------------------------------------------------------ prologues
+// xs rows hold the M token rows of the phase's GEMV input (bf16, row stride
+// K + GV_PAD); only rows < M exist.
+
+// The residual rows (bf16) into xs.
+__device__ void sk_pro_resid(const SkParams& s, bf16_t* xs) {
+    const int K = s.D, XS = K + GV_PAD, cpr = K / 8;
+    for (int e = threadIdx.x; e < s.M * cpr; e += SK_CT) {
+        const int m = e / cpr, c = e % cpr;
+        *reinterpret_cast<uint4*>(xs + m * XS + c * 8) =
+            *reinterpret_cast<const uint4*>(s.resid + (int64_t)m * K + c * 8);
+    }
+}
+
+// RMSNorm of the residual rows in xs, in place, one warp per row, with gains gb
+// (shared): the arithmetic of gv_prologue's RMSNorm.
+__device__ void sk_pro_rmsnorm(const SkParams& s, bf16_t* xs, const bf16_t* gb, int warp, int lane) {
+    const int K = s.D, XS = K + GV_PAD;
+    for (int m = warp; m < s.M; m += SK_CW) {
+        bf16_t* row = xs + m * XS;
+        float ss = 0.f;
+        for (int c = lane; c < K / 8; c += 32) {
+            const uint4 v = lds128(row + c * 8);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float a = bf_lo(w4[q]), b = bf_hi(w4[q]);
+                ss = fmaf(a, a, ss);
+                ss = fmaf(b, b, ss);
+            }
+        }
+        ss = warp_sum(ss);
+        const float r = rsqrtf(ss / (float)K + s.eps);
+        for (int c = lane; c < K / 8; c += 32) {
+            const uint4 v = lds128(row + c * 8);
+            const uint4 g = lds128(gb + c * 8);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t g4[4] = {g.x, g.y, g.z, g.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                o4[q] = pack_bf2(bf_lo(w4[q]) * r * bf_lo(g4[q]), bf_hi(w4[q]) * r * bf_hi(g4[q]));
+            *reinterpret_cast<uint4*>(row + c * 8) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+    }
+}
+
+// Layer 0: the embedding rows of the tokens (the packed embedding, gathered by
+// 16-byte chunks) into xs, CTA 0 writes them to the residual; a token outside
+// the vocabulary gives a zero row and HGD_ERR_INVALID_ARG.
+__device__ void sk_pro_embed(const SkParams& s, bf16_t* xs) {
+    const int K = s.D, XS = K + GV_PAD, cpr = K / 8;
+    for (int e = threadIdx.x; e < s.M * cpr; e += SK_CT) {
+        const int m = e / cpr, c = e % cpr;
+        const int tok = s.tokens[m];
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (tok < 0 || tok >= s.V) {
+            if (c == 0) set_status(s.status, HGD_ERR_INVALID_ARG);
         } else {
-            const unsigned long long t0 = globaltimer();
-            while (ld_acquire_u32(&s.bar[1]) == gen) {
-                if (ld_acquire_u32(&s.bar[2])) { ok = false; break; }
-                if (globaltimer() - t0 > kWaitLimitNs) {
-                    sk_timeout(s.bar, s.status, 1u, (unsigned)phase, arrived);
-                    ok = false;
-                    break;
+            v = *reinterpret_cast<const uint4*>(s.embed + gv_packed_chunk(tok, c, K >> 5));
+        }
+        *reinterpret_cast<uint4*>(xs + m * XS + c * 8) = v;
+        if (blockIdx.x == 0) *reinterpret_cast<uint4*>(s.resid + (int64_t)m * K + c * 8) = v;
+    }
+}
+
+// GDN out-projection input: per token row and head of width dv, the gated
+// RMSNorm o * rsqrt(mean(o^2) + eps) * w * silu(bf16(z)) (gv_prologue's), gains
+// gb in shared memory.  A warp takes its (row, head) pairs two at a time with
+// every load of both issued first (dv <= 128); wider heads loop.
+__device__ void sk_pro_gated(const SkParams& s, const GemvParams& p, const bf16_t* gb, bf16_t* xs, int warp,
+                             int lane) {
+    const int K = p.K, XS = K + GV_PAD, d = s.dv, nh = K / d, n = s.M * nh;
+    if (d <= 128) {
+        const int nk = d / 32;
+        for (int e0 = warp; e0 < n; e0 += 2 * SK_CW) {
+            float o[2][4], z[2][4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * SK_CW;
+                const int m = e / nh, h = e % nh;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    o[u][k] = 0.f;
+                    z[u][k] = 0.f;
+                    if (e < n && k < nk) {
+                        o[u][k] = s.obuf[(int64_t)m * K + h * d + lane + 32 * k];
+                        z[u][k] = s.proj[(int64_t)m * s.proj_ld + s.C + h * d + lane + 32 * k];
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * SK_CW;
+                if (e >= n) break;
+                const int m = e / nh, h = e % nh;
+                float ss = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < nk) ss = fmaf(o[u][k], o[u][k], ss);
+                ss = warp_sum(ss);
+                const float r = rsqrtf(ss / (float)d + s.eps);
+                bf16_t* dst = xs + m * XS + h * d;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < nk) {
+                        const int i = lane + 32 * k;
+                        const float zb = bf2f(f2bf(z[u][k]));
+                        dst[i] = f2bf(o[u][k] * r * bf2f(gb[i]) * silu_f(zb));
+                    }
+            }
+        }
+        return;
+    }
+    for (int e = warp; e < n; e += SK_CW) {
+        const int m = e / nh, h = e % nh;
+        bf16_t* dst = xs + m * XS + h * d;
+        const float* orow = s.obuf + (int64_t)m * K + h * d;
+        const float* zrow = s.proj + (int64_t)m * s.proj_ld + s.C + h * d;
+        float ss = 0.f;
+        for (int i = lane; i < d; i += 32) ss = fmaf(orow[i], orow[i], ss);
+        ss = warp_sum(ss);
+        const float r = rsqrtf(ss / (float)d + s.eps);
+        for (int i = lane; i < d; i += 32) {
+            const float zb = bf2f(f2bf(zrow[i]));
+            dst[i] = f2bf(orow[i] * r * bf2f(gb[i]) * silu_f(zb));
+        }
+    }
+}
+
+// Merge of the chunk partials of (row, query head h) -> out [hd] bf16, times
+// sigmoid(gate), by one warp.  Per dim d the arithmetic of attn_merge_dim:
+// M = max_c m_c, then in chunk order w_c = exp(m_c - M), L += w_c l_c,
+// acc_d += w_c acc_c[d].  Lane c % 32 loads chunk c's (m, l) and computes w_c
+// (shared by shuffles); lane j holds dims j, j + 32, ... (hd <= 256) and loads
+// them for SK_MB chunks at a time.
+constexpr int SK_MB = 4;
+__device__ void sk_merge_head(const float* base, int nch, int hd, const float* gate, bf16_t* out, int lane) {
+    const int nd = hd / 32;
+    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float Mx = -INFINITY;
+    for (int c = lane; c < nch; c += 32) Mx = fmaxf(Mx, __ldcg(base + (int64_t)c * (hd + 2)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, o));
+    for (int cb = 0; cb < nch; cb += 32) {
+        const int c = cb + lane;
+        float wl = 0.f, ll = 0.f;
+        if (c < nch) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(base + (int64_t)c * (hd + 2)));
+            wl = expf(ml.x - Mx);
+            ll = ml.y;
+        }
+        const int nb = min(32, nch - cb);
+        for (int j0 = 0; j0 < nb; j0 += SK_MB) {
+            float v[SK_MB][8];
+#pragma unroll
+            for (int u = 0; u < SK_MB; ++u) {
+                const float* pc = base + (int64_t)(cb + j0 + u) * (hd + 2) + 2;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[u][k] = (j0 + u < nb && k < nd) ? __ldcg(pc + lane + 32 * k) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < SK_MB; ++u) {
+                const float w = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
+                const float lc = __shfl_sync(0xffffffffu, ll, (j0 + u) & 31);
+                if (j0 + u < nb) {
+                    L = fmaf(w, lc, L);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        if (k < nd) acc[k] = fmaf(w, v[u][k], acc[k]);
                 }
             }
         }
-        __threadfence();
-        if (!ok) *cta_abort = 1;
     }
-    named_bar(1, SK_CW * 32);
-    return !*cta_abort;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        if (k < nd) {
+            const int dd = lane + 32 * k;
+            out[dd] = f2bf(acc[k] / L * sigmoid_f(gate[dd]));
+        }
 }
 
-// ------------------------------------------------------------ non-GEMV items
+// Down-projection input: the SwiGLU rows (bf16) as they are.
+__device__ void sk_pro_copy(const SkParams& s, const bf16_t* x, int K, bf16_t* xs) {
+    const int XS = K + GV_PAD, cpr = K / 8;
+    for (int e = threadIdx.x; e < s.M * cpr; e += SK_CT) {
+        const int m = e / cpr, c = e % cpr;
+        *reinterpret_cast<uint4*>(xs + m * XS + c * 8) = *reinterpret_cast<const uint4*>(x + (int64_t)m * K + c * 8);
+    }
+}
 
-// Gated delta rule for the 4 state rows row0..row0+3 (one warp) of stream b,
-// head h of GDN layer l (index ig), over the call's T rows.  The arithmetic of
-// every row is that of k_gdn_layer: the same norms, gates and gdn_rows_step.
+// ------------------------------------------------------------ GEMV consumer
+struct SkRing {
+    uint8_t* ring;
+    uint64_t* full;
+    uint64_t* empty;
+    int ns;
+};
+
+// Wait for the weight slab of CTA sequence number g (slot g % ns); false if the
+// wait ran out or the CTA aborted.  Every lane observes the completed phase.
+__device__ __forceinline__ bool sk_slab_wait(const SkParams& s, const SkRing& r, int g, volatile int* cta_abort,
+                                             int phase, int lane) {
+    const int slot = g % r.ns;
+    const uint32_t par = (uint32_t)((g / r.ns) & 1);
+    bool got = true;
+    if (lane == 0) got = mbar_wait_bounded(&r.full[slot], par, cta_abort);
+    got = __shfl_sync(0xffffffffu, got, 0);
+    if (got) got = __all_sync(0xffffffffu, mbar_try_wait(&r.full[slot], par));
+    if (!got && lane == 0 && !*cta_abort) {
+        sk_timeout(s, 2u, (unsigned)phase, (unsigned)g);
+        *cta_abort = 1;
+    }
+    if (s.tslab && blockIdx.x == 0 && lane == 0 && g < SK_TRACE_SLABS) s.tslab[g * 3 + 1] = globaltimer();
+    return got;
+}
+
+// 16 x 8 partial of one slab: chain 0 (even steps) + chain 1 (odd steps), the
+// per-slab arithmetic of k_gemv.
+__device__ __forceinline__ void sk_slab_mma(const bf16_t* tile, const bf16_t* xb, int sg, int nstep, bool has_x,
+                                            int lane, float (&part)[4]) {
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int jj = 0; jj < GV_SLAB_STEPS; ++jj) {
+        if (jj < nstep) {
+            const uint4 a0 = lds128(tile + jj * 512 + lane * 8);
+            const uint4 a1 = lds128(tile + jj * 512 + 256 + lane * 8);
+            const uint4 Bv = has_x ? lds128(xb + (sg * GV_SLAB_STEPS + jj) * 32) : make_uint4(0, 0, 0, 0);
+            float (&acc)[4] = (jj & 1) ? c1 : c0;
+            mma_bf16_16816(acc, a0.x, a1.x, a0.y, a1.y, Bv.x, Bv.y);
+            mma_bf16_16816(acc, a0.z, a1.z, a0.w, a1.w, Bv.z, Bv.w);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) part[q] = c0[q] + c1[q];
+}
+
+// The GEMV of one phase for this CTA's consumer warps.  gs: the CTA's slab
+// sequence number at the phase start (advanced past the phase's slabs); vc:
+// the CTA's place in the phase's item order.  Slab j of the phase (slab j % nks
+// of item j / nks) goes to warp (gs + j) % 8; the items' slab partials gather
+// in the partial buffer a round of items at a time, and item i's warp adds them
+// in slab order and runs the epilogue (gv_finish).
+template <int EPI>
+__device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const SkRing& r, const bf16_t* xs,
+                                float* pbuf, float* cbuf, GvBest<1>& best, int& gs, int vc,
+                                volatile int* cta_abort, int warp, int lane, int phase) {
+    const int G = gridDim.x;
+    const int XS = p.K + GV_PAD;
+    const int r8 = lane >> 2, c = lane & 3;
+    const bool has_x = r8 < s.M;
+    const bf16_t* xb = xs + (has_x ? r8 : 0) * XS + 8 * c;
+    const int steps_total = p.K >> 5;
+    const int nmine = sk_cta_items(p.n_items, vc);
+    const int first = ((warp - gs) % SK_CW + SK_CW) % SK_CW;  // this warp's first phase slab
+    const int nsl = p.nks;
+    const int R = max(1, s.pb / nsl);  // items per round
+    for (int i0 = 0; i0 < nmine; i0 += R) {
+        const int i1 = min(nmine, i0 + R);
+        const int jb = i0 * nsl, je = i1 * nsl;
+        // first slab >= jb of this warp
+        int j = jb + (((first - jb) % SK_CW) + SK_CW) % SK_CW;
+        for (; j < je; j += SK_CW) {
+            const int g = gs + j;
+            if (*cta_abort || !sk_slab_wait(s, r, g, cta_abort, phase, lane)) break;
+            const int sg = j % nsl;
+            const int nstep = min(GV_SLAB_STEPS, steps_total - sg * GV_SLAB_STEPS);
+            float part[4];
+            sk_slab_mma(reinterpret_cast<const bf16_t*>(r.ring + (g % r.ns) * SK_SLAB_BYTES), xb, sg, nstep, has_x,
+                        lane, part);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&r.empty[g % r.ns]);
+                if (s.tslab && blockIdx.x == 0 && g < SK_TRACE_SLABS) s.tslab[g * 3 + 2] = globaltimer();
+            }
+            float* pp = pbuf + (j - jb) * SK_PB_SLAB;
+            *reinterpret_cast<float2*>(pp + r8 * 8 + 2 * c) = make_float2(part[0], part[1]);
+            *reinterpret_cast<float2*>(pp + (r8 + 8) * 8 + 2 * c) = make_float2(part[2], part[3]);
+        }
+        named_bar(1, SK_CT);
+        if (!*cta_abort) {
+            for (int i = i0 + warp; i < i1; i += SK_CW) {
+                float yacc[1][4];
+                for (int sl = 0; sl < nsl; ++sl) {
+                    const float* pp = pbuf + ((i - i0) * nsl + sl) * SK_PB_SLAB;
+                    const float2 lo = *reinterpret_cast<const float2*>(pp + r8 * 8 + 2 * c);
+                    const float2 hi = *reinterpret_cast<const float2*>(pp + (r8 + 8) * 8 + 2 * c);
+                    if (sl == 0) { yacc[0][0] = lo.x; yacc[0][1] = lo.y; yacc[0][2] = hi.x; yacc[0][3] = hi.y; }
+                    else { yacc[0][0] += lo.x; yacc[0][1] += lo.y; yacc[0][2] += hi.x; yacc[0][3] += hi.y; }
+                }
+                gv_finish<1, EPI>(p, vc + i * G, 0, yacc, lane, cbuf + warp * GV_ROWS * 8, best);
+            }
+        }
+        named_bar(1, SK_CT);  // the partial buffer is reused by the next round
+    }
+    gs += nmine * nsl;
+}
+
+// ------------------------------------------------------------ GDN and attention
+
+// S rows row0..row0+3 of (stream b, head h) of GDN layer ig into registers.
 template <int KPL>
-__device__ void sk_gdn_item(const SkParams& s, int l, int ig, int b, int h, int row0, int lane) {
+__device__ __forceinline__ float* sk_gdn_rows(const SkParams& s, int ig, int it, float (&S)[GDN_RPW][KPL], int lane) {
     constexpr int DK = 32 * KPL;
-    const int H = s.H, dv = s.dv;
-    const bf16_t* const* w = s.layer[l].w;
-    const float A = expf(bf2f(w[HGD_W_A_LOG][h])), dtb = bf2f(w[HGD_W_DT_BIAS][h]);
-    float S[GDN_RPW][KPL];
-    float* Sbase = s.S + (size_t)ig * s.B * H * dv * DK + ((int64_t)(b * H + h) * dv + row0) * DK + lane * KPL;
+    const int rg = s.dv / GDN_RPW;
+    const int b = it / (s.H * rg), h = (it / rg) % s.H, row0 = (it % rg) * GDN_RPW;
+    float* Sbase = s.S + (size_t)ig * s.B * s.H * s.dv * DK + ((int64_t)(b * s.H + h) * s.dv + row0) * DK + lane * KPL;
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
+    return Sbase;
+}
+
+// Gated delta rule of GDN item `it` (4 state rows of one stream and head) over
+// the call's T rows, on state rows already in S: the arithmetic of k_gdn_layer.
+template <int KPL>
+__device__ void sk_gdn_item(const SkParams& s, int l, int ig, int it, float (&S)[GDN_RPW][KPL], float* Sbase,
+                            int lane) {
+    constexpr int DK = 32 * KPL;
+    const int H = s.H, dv = s.dv, rg = dv / GDN_RPW;
+    const int b = it / (H * rg), h = (it / rg) % H, row0 = (it % rg) * GDN_RPW;
+    const bf16_t* const* w = s.layer[l].w;
+    const float A = expf(bf2f(w[HGD_W_A_LOG][h])), dtb = bf2f(w[HGD_W_DT_BIAS][h]);
     for (int t = 0; t < s.T; ++t) {
         const int64_t row = (int64_t)b * s.T + t;
         const float* pr = s.proj + row * s.proj_ld;
         float qv[KPL], kv[KPL];
         ld_vec<KPL>(qv, pr + (int64_t)h * DK + lane * KPL);
         ld_vec<KPL>(kv, pr + (int64_t)H * DK + (int64_t)h * DK + lane * KPL);
+        const float a = pr[s.C + (int64_t)H * dv + h];
+        const float braw = pr[s.C + (int64_t)H * dv + H + h];
+        float vrow[GDN_RPW], o[GDN_RPW];
+        const float* vp = pr + 2 * (int64_t)H * DK + (int64_t)h * dv + row0;
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
         float sq = 0.f, sk = 0.f;
 #pragma unroll
         for (int e = 0; e < KPL; ++e) { sq = fmaf(qv[e], qv[e], sq); sk = fmaf(kv[e], kv[e], sk); }
         const float qsc = rsqrtf(warp_sum(sq) + 1e-6f), ksc = rsqrtf(warp_sum(sk) + 1e-6f);
 #pragma unroll
         for (int e = 0; e < KPL; ++e) { qv[e] = qv[e] * qsc; kv[e] = kv[e] * ksc; }
-        const float a = pr[s.C + (int64_t)H * dv + h];
-        const float braw = pr[s.C + (int64_t)H * dv + H + h];
-        const float alpha = expf(-A * softplus_f(a + dtb));
+        const float g = -A * softplus_f(a + dtb);
+        const float alpha = expf(g);
         const float beta = sigmoid_f(braw);
-        float vrow[GDN_RPW], o[GDN_RPW];
-        const float* vp = pr + 2 * (int64_t)H * DK + (int64_t)h * dv + row0;
-#pragma unroll
-        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
         gdn_rows_step<KPL>(S, kv, qv, alpha, beta, vrow, o);
         if (lane < GDN_RPW) {
             float ov = o[0];
@@ -238,130 +603,6 @@ __device__ void sk_gdn_item(const SkParams& s, int l, int ig, int b, int h, int 
     }
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
-}
-
-// RoPE of one head of one row (query heads: rotated q; key/value heads: the
-// rotated key and the value appended to the cache), as k_rope_append computes it.
-__device__ void sk_rope_item(const SkParams& s, int ia, int row, int head, int lane) {
-    const int b = row / s.T, t = row % s.T;
-    const int P = s.pos[b] + t;
-    if (P < 0 || P >= s.Lmax) {
-        if (lane == 0) set_status(s.status, HGD_ERR_INVALID_ARG);
-        return;
-    }
-    const int hd = s.hd, half = hd / 2, qw = s.nq * hd;
-    const float* pr = s.proj + (int64_t)row * s.proj_ld;
-    const size_t kv_half = (size_t)s.B * s.nkv * s.Lmax * hd;
-    bf16_t* kc = s.kv + (size_t)ia * 2 * kv_half;
-    bf16_t* vc = kc + kv_half;
-    for (int i = lane; i < half; i += 32) {
-        const double inv = exp2(-2.0 * (double)i / (double)hd * log2((double)s.rope_base));
-        const double th = (double)P * inv;
-        const double tw = 6.283185307179586476925286766559;
-        const float r = (float)(th - tw * rint(th / tw));
-        float sn, cs;
-        sincosf(r, &sn, &cs);
-        if (head < s.nq) {
-            const float a = pr[head * hd + i], bb = pr[head * hd + i + half];
-            float* qo = s.qrot + (int64_t)row * qw + head * hd;
-            qo[i] = a * cs - bb * sn;
-            qo[i + half] = bb * cs + a * sn;
-        } else {
-            const int g = head - s.nq;
-            const float* kp = pr + 2 * qw + g * hd;
-            bf16_t* ko = kc + (((int64_t)b * s.nkv + g) * s.Lmax + P) * hd;
-            ko[i] = f2bf(kp[i] * cs - kp[i + half] * sn);
-            ko[i + half] = f2bf(kp[i + half] * cs + kp[i] * sn);
-        }
-    }
-    if (head >= s.nq) {
-        const int g = head - s.nq;
-        const float* vp = pr + 2 * qw + s.nkv * hd + g * hd;
-        bf16_t* vo = vc + (((int64_t)b * s.nkv + g) * s.Lmax + P) * hd;
-        for (int d = lane; d < hd; d += 32) vo[d] = f2bf(vp[d]);
-    }
-}
-
-// One attention partial: query head h of one row over one chunk of keys (the
-// arithmetic of k_attn_partial's warps).  ex: this warp's 32 floats of scratch.
-__device__ void sk_partial_item(const SkParams& s, int ia, int row, int h, int ch, int lane, float* ex) {
-    const int b = row / s.T, t = row % s.T;
-    const int P = s.pos[b] + t;
-    if (P < 0 || P >= s.Lmax) return;
-    const int key0 = ch * ATTN_CHUNK;
-    if (key0 > P) return;
-    const int nk = min(ATTN_CHUNK, P + 1 - key0);
-    const int hd = s.hd, group = s.nq / s.nkv, g = h / group;
-    const size_t kv_half = (size_t)s.B * s.nkv * s.Lmax * hd;
-    const bf16_t* K = s.kv + (size_t)ia * 2 * kv_half + ((int64_t)b * s.nkv + g) * s.Lmax * hd;
-    const bf16_t* V = K + kv_half;
-    const float* q = s.qrot + (int64_t)row * s.nq * hd + (int64_t)h * hd;
-    float sc = -INFINITY;
-    if (lane < nk) {
-        const bf16_t* kr = K + (int64_t)(key0 + lane) * hd;
-        float d = 0.f;
-        for (int e = 0; e < hd; e += 8) {
-            const uint4 kv = *reinterpret_cast<const uint4*>(kr + e);
-            const float4 q0 = *reinterpret_cast<const float4*>(q + e);
-            const float4 q1 = *reinterpret_cast<const float4*>(q + e + 4);
-            d = fmaf(q0.x, bf_lo(kv.x), d); d = fmaf(q0.y, bf_hi(kv.x), d);
-            d = fmaf(q0.z, bf_lo(kv.y), d); d = fmaf(q0.w, bf_hi(kv.y), d);
-            d = fmaf(q1.x, bf_lo(kv.z), d); d = fmaf(q1.y, bf_hi(kv.z), d);
-            d = fmaf(q1.z, bf_lo(kv.w), d); d = fmaf(q1.w, bf_hi(kv.w), d);
-        }
-        sc = d * (1.0f / sqrtf((float)hd));
-    }
-    float m = sc;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float e = (lane < nk) ? expf(sc - m) : 0.f;
-    const float l = warp_sum(e);
-    ex[lane] = e;
-    __syncwarp();
-    float* dst = s.part + (((int64_t)row * s.nq + h) * s.max_chunks + ch) * (hd + 2);
-    for (int d0 = lane * 8; d0 < hd; d0 += 256) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < nk; ++j) {
-            const uint4 vv = *reinterpret_cast<const uint4*>(V + (int64_t)(key0 + j) * hd + d0);
-            const float wgt = ex[j];
-            acc[0] = fmaf(wgt, bf_lo(vv.x), acc[0]); acc[1] = fmaf(wgt, bf_hi(vv.x), acc[1]);
-            acc[2] = fmaf(wgt, bf_lo(vv.y), acc[2]); acc[3] = fmaf(wgt, bf_hi(vv.y), acc[3]);
-            acc[4] = fmaf(wgt, bf_lo(vv.z), acc[4]); acc[5] = fmaf(wgt, bf_hi(vv.z), acc[5]);
-            acc[6] = fmaf(wgt, bf_lo(vv.w), acc[6]); acc[7] = fmaf(wgt, bf_hi(vv.w), acc[7]);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dst[2 + d0 + i] = acc[i];
-    }
-    if (lane == 0) { dst[0] = m; dst[1] = l; }
-    __syncwarp();
-}
-
-// Merge the chunk partials of query head h of one row, times sigmoid(gate)
-// (per dimension, the arithmetic of k_attn_merge).
-__device__ void sk_merge_item(const SkParams& s, int row, int h, int lane) {
-    const int b = row / s.T, t = row % s.T;
-    const int P = s.pos[b] + t;
-    const int hd = s.hd;
-    bf16_t* out = s.attn + (int64_t)row * s.nq * hd + (int64_t)h * hd;
-    if (P < 0 || P >= s.Lmax) {
-        for (int d = lane; d < hd; d += 32) out[d] = 0;
-        return;
-    }
-    const int nch = P / ATTN_CHUNK + 1;
-    const float* base = s.part + ((int64_t)row * s.nq + h) * s.max_chunks * (hd + 2);
-    float M = -INFINITY;
-    for (int c = 0; c < nch; ++c) M = fmaxf(M, base[c * (hd + 2)]);
-    for (int d = lane; d < hd; d += 32) {
-        float L = 0.f, acc = 0.f;
-        for (int c = 0; c < nch; ++c) {
-            const float* pc = base + c * (hd + 2);
-            const float wgt = expf(pc[0] - M);
-            L = fmaf(wgt, pc[1], L);
-            acc = fmaf(wgt, pc[2 + d], acc);
-        }
-        const float gate = s.proj[(int64_t)row * s.proj_ld + s.nq * hd + (int64_t)h * hd + d];
-        out[d] = f2bf(acc / L * sigmoid_f(gate));
-    }
 }
 
 // Argmax of each row over the CTAs' partials; positions advance by T.
@@ -393,252 +634,268 @@ __device__ void sk_final(const SkParams& s, int lane) {
 }
 
 // ------------------------------------------------------------------ kernel
+// Shared memory: ring [ns][8 KB] | xs [M][kmax + 8] bf16 | gains [D] bf16 |
+// partial buffer [pb][16][8] f32 | conv scratch [8][16][8] f32 | argmax [8][8] x2 |
+// attention scratch [8][32] f32 | full[ns], empty[ns] mbarriers | flags.
+struct SkSmem {
+    uint8_t* ring; bf16_t* xs; bf16_t* gb; float* pbuf; float* cbuf; float* amax_v; int* amax_i; float* ex;
+    uint64_t* full; uint64_t* empty; volatile int* flags;
+};
 
-// Consumer side of one GEMV phase: prologue, this CTA's items, epilogue.
-template <int PRO, int EPI>
-__device__ void sk_gemv_phase(const SkParams& s, const GemvParams& p, uint8_t* ring, uint64_t* full,
-                              uint64_t* empty, bf16_t* xs, float* cbuf, float* amax_v, int* amax_i,
-                              int& wseq, volatile int* cta_abort, int warp, int lane, int phase) {
-    const int seq_base = wseq;
-    const int tid = threadIdx.x;
-    if (!*cta_abort) gv_prologue<8, PRO>(p, xs, tid, warp, lane, nullptr);
-    named_bar(1, SK_CW * 32);
-    const int XS = p.K + GV_PAD;
-    const int r8 = lane >> 2, c = lane & 3;
-    const int steps_total = p.K >> 5;
-    const int nsl = p.split ? 1 : p.nks;
-    const int nmine = sk_cta_items(p.n_items);
-    const bf16_t* xb = xs + r8 * XS + 8 * c;
-    float* cb = cbuf + warp * GV_ROWS * 8;
-    GvBest<1> best;
-    best.init();
-    for (int i = warp; i < nmine; i += SK_CW) {
-        const int u = blockIdx.x + i * gridDim.x;
-        const int rb = p.split ? u / p.nks : u;
-        const int s0 = p.split ? u % p.nks : 0;
-        float yacc[1][4];
-        bool ok = !*cta_abort;
-        for (int sl = 0; sl < nsl; ++sl) {
-            const int seq = wseq++;  // this warp's slab sequence number
-            const int slot = warp * SK_NSW + seq % SK_NSW;
-            const uint32_t par = (uint32_t)((seq / SK_NSW) & 1);
-            if (ok) {
-                bool got = true;
-                if (lane == 0) got = mbar_wait_bounded(&full[slot], par, cta_abort);
-                got = __shfl_sync(0xffffffffu, got, 0);
-                if (got) got = __all_sync(0xffffffffu, mbar_try_wait(&full[slot], par));
-                if (!got) {
-                    if (lane == 0) {
-                        if (!*cta_abort && atomicCAS(&s.bar[4], 0u, 2u) == 0u) {
-                            const volatile int* pr = reinterpret_cast<const volatile int*>(cta_abort) + 1;
-                            s.bar[5] = (unsigned)phase;
-                            s.bar[6] = blockIdx.x;
-                            s.bar[7] = (unsigned)seq;
-                            s.bar[8] = (unsigned)pr[0];
-                            s.bar[9] = (unsigned)pr[1];
-                            s.bar[10] = (unsigned)warp;
-                            s.bar[12] = (unsigned)seq_base;
-                            unsigned fb = 0, eb = 0;
-                            for (int q = 0; q < SK_NSLOT; ++q) {
-                                fb |= (mbar_try_wait(&full[q], 0) ? 1u : 0u) << (2 * q);
-                                fb |= (mbar_try_wait(&full[q], 1) ? 2u : 0u) << (2 * q);
-                                eb |= (mbar_try_wait(&empty[q], 0) ? 1u : 0u) << (2 * q);
-                                eb |= (mbar_try_wait(&empty[q], 1) ? 2u : 0u) << (2 * q);
-                            }
-                            s.bar[11] = fb;
-                            s.bar[13] = eb;
-                        }
-                        sk_timeout(s.bar, s.status, 2u, (unsigned)phase, (unsigned)seq);
-                        *cta_abort = 1;
-                    }
-                    ok = false;
-                }
-            }
-            const int sg = s0 + sl;  // slab index within the row block
-            const int nstep = min(GV_SLAB_STEPS, steps_total - sg * GV_SLAB_STEPS);
-            float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-            if (ok) {
-                const bf16_t* tile = reinterpret_cast<const bf16_t*>(ring + slot * SK_SLAB_BYTES);
-#pragma unroll
-                for (int jj = 0; jj < GV_SLAB_STEPS; ++jj) {
-                    if (jj < nstep) {
-                        const uint4 a0 = lds128(tile + jj * 512 + lane * 8);
-                        const uint4 a1 = lds128(tile + jj * 512 + 256 + lane * 8);
-                        const uint4 Bv = lds128(xb + (sg * GV_SLAB_STEPS + jj) * 32);
-                        float (&acc)[4] = (jj & 1) ? c1 : c0;
-                        mma_bf16_16816(acc, a0.x, a1.x, a0.y, a1.y, Bv.x, Bv.y);
-                        mma_bf16_16816(acc, a0.z, a1.z, a0.w, a1.w, Bv.z, Bv.w);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[slot]);
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float part = c0[q] + c1[q];
-                yacc[0][q] = (p.split || sl == 0) ? part : yacc[0][q] + part;
-            }
-        }
-        if (ok) gv_finish<1, EPI>(p, rb, s0, yacc, lane, cb, best);
-    }
-    if (EPI == EPI_ARGMAX)
-        gv_argmax_cta<1>(p, best, amax_v, amax_i, warp, lane, tid, SK_CW, blockIdx.x, gridDim.x, true);
+__host__ __device__ inline size_t sk_al128(size_t v) { return (v + 127) & ~(size_t)127; }
+__host__ __device__ inline size_t sk_xs_bytes(int M, int kmax) { return sk_al128((size_t)M * (kmax + GV_PAD) * 2); }
+__host__ __device__ inline size_t sk_fixed_bytes(int M, int kmax, int D, int pb, int ns) {
+    return sk_xs_bytes(M, kmax) + sk_al128((size_t)D * 2) + (size_t)pb * SK_PB_SLAB * 4 +
+           (size_t)SK_CW * GV_ROWS * 8 * 4 + (size_t)SK_CW * 8 * 8 + (size_t)SK_CW * 32 * 4 + (size_t)ns * 16 + 64;
+}
+
+__device__ __forceinline__ SkSmem sk_smem(const SkParams& s, uint8_t* base) {
+    SkSmem m;
+    size_t o = 0;
+    m.ring = base; o += (size_t)s.ns * SK_SLAB_BYTES;
+    m.xs = reinterpret_cast<bf16_t*>(base + o); o += sk_xs_bytes(s.M, s.kmax);
+    m.gb = reinterpret_cast<bf16_t*>(base + o); o += sk_al128((size_t)s.D * 2);
+    m.pbuf = reinterpret_cast<float*>(base + o); o += (size_t)s.pb * SK_PB_SLAB * 4;
+    m.cbuf = reinterpret_cast<float*>(base + o); o += (size_t)SK_CW * GV_ROWS * 8 * 4;
+    m.amax_v = reinterpret_cast<float*>(base + o); o += SK_CW * 8 * 4;
+    m.amax_i = reinterpret_cast<int*>(base + o); o += SK_CW * 8 * 4;
+    m.ex = reinterpret_cast<float*>(base + o); o += SK_CW * 32 * 4;
+    m.full = reinterpret_cast<uint64_t*>(base + o); o += (size_t)s.ns * 8;
+    m.empty = reinterpret_cast<uint64_t*>(base + o); o += (size_t)s.ns * 8;
+    m.flags = reinterpret_cast<volatile int*>(base + o);
+    return m;
 }
 
 template <int KPL>
 __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__ SkParams s) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint8_t* ring = smem;
-    bf16_t* xs = reinterpret_cast<bf16_t*>(smem + SK_NSLOT * SK_SLAB_BYTES);
-    float* cbuf = reinterpret_cast<float*>(smem + SK_NSLOT * SK_SLAB_BYTES + s.x_bytes);  // [CW][16][8]
-    float* amax_v = cbuf + SK_CW * GV_ROWS * 8;
-    int* amax_i = reinterpret_cast<int*>(amax_v + SK_CW * 8);
-    float* exbuf = reinterpret_cast<float*>(amax_i + SK_CW * 8);  // [CW][32]
-    uint64_t* full = reinterpret_cast<uint64_t*>(exbuf + SK_CW * 32);
-    uint64_t* empty = full + SK_NSLOT;
-    volatile int* cta_abort = reinterpret_cast<volatile int*>(empty + SK_NSLOT);
-    volatile int* prod = cta_abort + 1;  // [0] producer's next sequence number, [1] 1 while it waits
+    const SkSmem sm = sk_smem(s, smem);
+    volatile int* cta_abort = sm.flags;
+    const SkRing ring{sm.ring, sm.full, sm.empty, s.ns};
+    const int G = gridDim.x;
 
     if (tid == 0) {
-        for (int i = 0; i < SK_NSLOT; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < s.ns; ++i) { mbar_init(&sm.full[i], 1); mbar_init(&sm.empty[i], 1); }
         *cta_abort = 0;
-        prod[0] = 0;
-        prod[1] = 0;
         mbar_fence_init();
     }
     __syncthreads();
 
     // ---------------------------------------------------------------- producer
+    // The CTA's slabs of a phase, j = 0 .. nmine * nks - 1 (slab j % nks of item
+    // j / nks), go out eight at a time: lane l of the producer warp takes slab
+    // j0 + l, waits for its ring slot to be released and issues its bulk copy.
     if (warp == SK_CW) {
-        if (lane != 0) return;
+        constexpr int PB = 8;  // copies issued together (<= ring slots)
         const uint64_t pol = policy_evict_first();
-        int wseq[SK_CW];
-        for (int w = 0; w < SK_CW; ++w) wseq[w] = 0;
-        int pid = -1;
+        int g = 0;  // the CTA's slab sequence number at the start of the batch
         bool ok = true;
+        int pid = -1;
         for (int l = 0; l <= s.L && ok; ++l) {
-            const int nph = (l == s.L) ? 1 : sk_nphase(s, l);
-            for (int j = 0; j < nph && ok; ++j) {
+            const int nph = (l == s.L) ? 1 : SK_PHASES_PER_LAYER;
+            for (int jph = 0; jph < nph && ok; ++jph) {
                 ++pid;
-                const int kind = sk_kind(s, l, j);
+                const int kind = sk_kind(s, l, jph);
                 if (!sk_is_gemv(kind)) continue;
                 GemvParams p;
-                sk_gemv_params(s, kind, l, 0, p);
+                sk_gemv_params(s, kind, l, 0, 0, p);
                 const int steps_total = p.K >> 5;
-                const int nsl = p.split ? 1 : p.nks;
-                const int nmine = sk_cta_items(p.n_items);
-                // warp w owns items w, w + CW, ...; its k-th slab of the phase is slab
-                // k % nsl of its (k / nsl)-th item.  Feed the warps one slab each in turn.
-                const int per_warp_max = ((nmine + SK_CW - 1) / SK_CW) * nsl;
-                for (int k = 0; k < per_warp_max && ok; ++k) {
-                    for (int w = 0; w < SK_CW && ok; ++w) {
-                        const int i = w + (k / nsl) * SK_CW;
-                        if (i >= nmine) continue;
-                        const int sl = k % nsl;
-                        const int u = blockIdx.x + i * gridDim.x;
-                        const int rb = p.split ? u / p.nks : u;
-                        const int s0 = p.split ? u % p.nks : 0;
-                        const int q = wseq[w]++;
-                        const int slot = w * SK_NSW + q % SK_NSW;
-                        const uint32_t par = (uint32_t)((q / SK_NSW) & 1);
-                        prod[0] = q;
-                        prod[1] = 1;
-                        const bool free_slot = mbar_wait_bounded(&empty[slot], par ^ 1, cta_abort);
-                        prod[1] = 0;
-                        if (!free_slot || ld_acquire_u32(&s.bar[2])) {
-                            if (!ld_acquire_u32(&s.bar[2])) sk_timeout(s.bar, s.status, 3u, (unsigned)pid, (unsigned)q);
-                            wseq[w]--;
-                            ok = false;
-                            break;
+                const int vc = sk_vcta(pid);
+                const int J = sk_cta_items(p.n_items, vc) * p.nks;
+                for (int j0 = 0; j0 < J && ok; j0 += PB) {
+                    const int j = j0 + lane;
+                    bool lane_ok = true, sent = false;
+                    if (lane < PB && j < J) {
+                        const int gj = g + lane;
+                        const int slot = gj % s.ns;
+                        if (gj >= s.ns &&
+                            !mbar_wait_bounded(&sm.empty[slot], (uint32_t)(((gj / s.ns) - 1) & 1), cta_abort)) {
+                            // (an abort raised elsewhere reaches this CTA through its consumers' waits)
+                            if (!*cta_abort) sk_timeout(s, 3u, (unsigned)pid, (unsigned)gj);
+                            lane_ok = false;
+                        } else {
+                            const int i = j / p.nks, sg = j % p.nks;
+                            const int rb = vc + i * G;
+                            const int nstep = min(GV_SLAB_STEPS, steps_total - sg * GV_SLAB_STEPS);
+                            const uint32_t bytes = (uint32_t)nstep * 1024u;
+                            if (s.tslab && blockIdx.x == 0 && gj < SK_TRACE_SLABS) s.tslab[gj * 3] = globaltimer();
+                            mbar_arrive_expect_tx(&sm.full[slot], bytes);
+                            bulk_g2s(ring.ring + (size_t)slot * SK_SLAB_BYTES,
+                                     p.W + gv_tile_elem(rb, sg * GV_SLAB_STEPS, steps_total, 0, 0), bytes,
+                                     &sm.full[slot], pol);
+                            sent = true;
                         }
-                        const int sg = s0 + sl;
-                        const int nstep = min(GV_SLAB_STEPS, steps_total - sg * GV_SLAB_STEPS);
-                        const uint32_t bytes = (uint32_t)nstep * 1024u;
-                        mbar_arrive_expect_tx(&full[slot], bytes);
-                        bulk_g2s(ring + slot * SK_SLAB_BYTES,
-                                 p.W + gv_tile_elem(rb, sg * GV_SLAB_STEPS, steps_total, 0, 0), bytes, &full[slot],
-                                 pol);
                     }
+                    ok = __all_sync(0xffffffffu, lane_ok);
+                    if (!ok) {
+                        // a wait ran out: the copies this batch did send land before the
+                        // warp leaves; g stays at the batch start for the drain below
+                        if (sent) {
+                            const int gj = g + lane;
+                            (void)mbar_wait_bounded(&sm.full[gj % s.ns], (uint32_t)((gj / s.ns) & 1), nullptr);
+                        }
+                        break;
+                    }
+                    g += min(PB, J - j0);
                 }
             }
         }
-        // Do not leave while a copy into this CTA's shared memory is in flight.
-        for (int w = 0; w < SK_CW; ++w)
-            for (int q = max(0, wseq[w] - SK_NSW); q < wseq[w]; ++q)
-                (void)mbar_wait_bounded(&full[w * SK_NSW + q % SK_NSW], (uint32_t)((q / SK_NSW) & 1), nullptr);
+        // Do not leave while a copy into this CTA's shared memory is in flight:
+        // wait for the fills of the last ns slabs issued (a slot whose copy was
+        // never issued after a failed wait completed its earlier fill already).
+        if (lane == 0)
+            for (int q = max(0, g - s.ns); q < g; ++q)
+                (void)mbar_wait_bounded(&sm.full[q % s.ns], (uint32_t)((q / s.ns) & 1), nullptr);
         return;
     }
 
     // --------------------------------------------------------------- consumers
-    int wseq = 0;  // this warp's slab sequence number across all phases
+    int gs = 0;       // the CTA's slab sequence number (same in every consumer warp)
     int ig = 0, ia = 0, pid = -1;
-    bool first = true;
+    GvBest<1> best;
+    best.init();
     for (int l = 0; l <= s.L; ++l) {
-        const bool att = l < s.L && sk_attn(s, l);
-        const int nph = (l == s.L) ? 2 : sk_nphase(s, l);
+        const int nph = (l == s.L) ? 2 : SK_PHASES_PER_LAYER;
         for (int j = 0; j < nph; ++j) {
             const int kind = sk_kind(s, l, j);
             ++pid;
-            if (!first) sk_grid_sync(s, cta_abort, pid);
-            first = false;
-            if (s.trace && blockIdx.x == 0 && threadIdx.x == 0 && pid < 256) s.trace[pid] = globaltimer();
-            const bool live = !*cta_abort;
-            if (sk_is_gemv(kind)) {
-                GemvParams p;
-                sk_gemv_params(s, kind, l, ig, p);
-                switch (kind) {
-                    case SK_IN_GDN:
-                        if (l == 0) sk_gemv_phase<PRO_EMBED_RMSNORM, EPI_QKV_CONV>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        else sk_gemv_phase<PRO_RMSNORM, EPI_QKV_CONV>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        break;
-                    case SK_IN_ATT:
-                        if (l == 0) sk_gemv_phase<PRO_EMBED_RMSNORM, EPI_F32>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        else sk_gemv_phase<PRO_RMSNORM, EPI_F32>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        break;
-                    case SK_OUT_GDN:
-                        sk_gemv_phase<PRO_GATED_NORM, EPI_RESID>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        break;
-                    case SK_OUT_ATT: case SK_DOWN:
-                        sk_gemv_phase<PRO_COPY, EPI_RESID>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        break;
-                    case SK_SWIGLU:
-                        sk_gemv_phase<PRO_RMSNORM, EPI_SWIGLU>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        break;
-                    default:
-                        sk_gemv_phase<PRO_RMSNORM, EPI_ARGMAX>(s, p, ring, full, empty, xs, cbuf, amax_v, amax_i, wseq, cta_abort, warp, lane, pid);
-                        break;
+            if (kind == SK_FINAL) {
+                if (blockIdx.x == 0) {
+                    const bool live = sk_wait(s, cta_abort, pid - 1);
+                    if (live && warp == 0) sk_final(s, lane);
                 }
                 continue;
             }
-            // the phases without weights: items spread over the warps of all CTAs
-            const int gw = warp * gridDim.x + blockIdx.x, nw = gridDim.x * SK_CW;
-            if (kind == SK_GDN) {
-                const int rg = s.dv / GDN_RPW;
-                const int n = s.B * s.H * rg;
-                for (int it = gw; live && it < n; it += nw) {
-                    const int b = it / (s.H * rg), h = (it / rg) % s.H, r = it % rg;
-                    sk_gdn_item<KPL>(s, l, ig, b, h, r * GDN_RPW, lane);
-                }
-            } else if (kind == SK_ROPE) {
-                const int nh = s.nq + s.nkv, n = s.M * nh;
-                for (int it = gw; live && it < n; it += nw) sk_rope_item(s, ia, it / nh, it % nh, lane);
-            } else if (kind == SK_PART) {
-                const int n = s.M * s.nq * s.max_chunks;
-                for (int it = gw; live && it < n; it += nw) {
-                    const int row = it / (s.nq * s.max_chunks), h = (it / s.max_chunks) % s.nq;
-                    sk_partial_item(s, ia, row, h, it % s.max_chunks, lane, exbuf + warp * 32);
-                }
-            } else if (kind == SK_MERGE) {
-                const int n = s.M * s.nq;
-                for (int it = gw; live && it < n; it += nw) sk_merge_item(s, it / s.nq, it % s.nq, lane);
-            } else if (kind == SK_FINAL) {
-                if (live && blockIdx.x == 0 && warp == 0) sk_final(s, lane);
+            GemvParams p;
+            const bool gemv = sk_is_gemv(kind);
+            const int vc = sk_vcta(pid);
+            int nmine = 0;
+            if (gemv) {
+                sk_gemv_params(s, kind, l, ig, ia, p);
+                nmine = sk_cta_items(p.n_items, vc);
             }
+            // work that does not depend on the previous phase: gains, GDN state rows
+            float S[GDN_RPW][KPL];
+            float* Sbase = nullptr;
+            const int gw = warp * G + blockIdx.x, nw = G * SK_CW;
+            const int n_gdn = s.B * s.H * (s.dv / GDN_RPW);
+            if (nmine > 0 && (kind == SK_IN_GDN || kind == SK_IN_ATT || kind == SK_SWIGLU || kind == SK_HEAD)) {
+                for (int c = tid; c < s.D / 8; c += SK_CT)
+                    *reinterpret_cast<uint4*>(sm.gb + c * 8) = *reinterpret_cast<const uint4*>(p.norm_w + c * 8);
+            } else if (nmine > 0 && kind == SK_OUT_GDN) {
+                for (int c = tid; c < s.dv / 8; c += SK_CT)
+                    *reinterpret_cast<uint4*>(sm.gb + c * 8) = *reinterpret_cast<const uint4*>(p.gnorm_w + c * 8);
+            } else if (kind == SK_GDN && gw < n_gdn) {
+                Sbase = sk_gdn_rows<KPL>(s, ig, gw, S, lane);
+            }
+            const bool live = (pid == 0) ? sk_bar_and(!*cta_abort) : sk_wait(s, cta_abort, pid - 1);
+            if (s.trace && blockIdx.x == 0 && tid == 0 && pid < SK_TRACE_SLOTS - 1) s.trace[pid] = globaltimer();
+            // per-CTA phase times: wait done, prologue done, GEMV or items done, arrival
+            unsigned long long* td = (s.tdetail && tid == 0 && blockIdx.x < SK_TRACE_CTAS)
+                                         ? s.tdetail + ((size_t)pid * SK_TRACE_CTAS + blockIdx.x) * 4
+                                         : nullptr;
+            if (td) td[0] = globaltimer();
+            if (live && (!gemv || nmine > 0)) {
+                switch (kind) {
+                    case SK_IN_GDN: case SK_IN_ATT: case SK_SWIGLU: case SK_HEAD: {
+                        if (kind != SK_SWIGLU && l == 0) sk_pro_embed(s, sm.xs);
+                        else sk_pro_resid(s, sm.xs);
+                        named_bar(1, SK_CT);
+                        sk_pro_rmsnorm(s, sm.xs, sm.gb, warp, lane);
+                        break;
+                    }
+                    case SK_OUT_GDN: sk_pro_gated(s, p, sm.gb, sm.xs, warp, lane); break;
+                    case SK_OUT_ATT: sk_pro_copy(s, s.attn, s.nq * s.hd, sm.xs); break;
+                    case SK_DOWN: sk_pro_copy(s, s.mlp, s.I, sm.xs); break;
+                    default: break;
+                }
+                named_bar(1, SK_CT);
+                if (td) td[1] = globaltimer();
+                switch (kind) {
+                    case SK_IN_GDN:
+                        sk_gemv_consume<EPI_QKV_CONV>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
+                                                      warp, lane, pid);
+                        break;
+                    case SK_IN_ATT:
+                        sk_gemv_consume<EPI_ROPE>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort, warp,
+                                                  lane, pid);
+                        break;
+                    case SK_SWIGLU:
+                        sk_gemv_consume<EPI_SWIGLU>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
+                                                    warp, lane, pid);
+                        break;
+                    case SK_HEAD:
+                        sk_gemv_consume<EPI_ARGMAX>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
+                                                    warp, lane, pid);
+                        gv_argmax_cta<1>(p, best, sm.amax_v, sm.amax_i, warp, lane, tid, SK_CW, blockIdx.x, G, true);
+                        break;
+                    case SK_OUT_GDN: case SK_OUT_ATT: case SK_DOWN:
+                        sk_gemv_consume<EPI_RESID>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
+                                                   warp, lane, pid);
+                        break;
+                    case SK_GDN:
+                        for (int it = gw; it < n_gdn; it += nw) {
+                            if (it != gw) Sbase = sk_gdn_rows<KPL>(s, ig, it, S, lane);
+                            sk_gdn_item<KPL>(s, l, ig, it, S, Sbase, lane);
+                        }
+                        break;
+                    case SK_PART: {
+                        const int n = s.M * s.nq * s.max_chunks;
+                        const size_t kv_half = (size_t)s.B * s.nkv * s.Lmax * s.hd;
+                        const int group = s.nq / s.nkv;
+                        for (int it = gw; it < n; it += nw) {
+                            const int row = it / (s.nq * s.max_chunks), h = (it / s.max_chunks) % s.nq;
+                            const int ch = it % s.max_chunks;
+                            const int b = row / s.T, t = row % s.T;
+                            const int P = s.pos[b] + t;
+                            if (P < 0 || P >= s.Lmax) {  // the merged output of the row is zero
+                                if (ch == 0)
+                                    for (int d = lane; d < s.hd; d += 32)
+                                        s.attn[(int64_t)row * s.nq * s.hd + (int64_t)h * s.hd + d] = 0;
+                                continue;
+                            }
+                            const int key0 = ch * ATTN_CHUNK;
+                            if (key0 > P) continue;
+                            const int g = h / group;
+                            const bf16_t* K = s.kv + (size_t)ia * 2 * kv_half + ((int64_t)b * s.nkv + g) * s.Lmax * s.hd;
+                            const float* q = s.qrot + (int64_t)row * s.nq * s.hd + (int64_t)h * s.hd;
+                            float* dst = s.part + (((int64_t)row * s.nq + h) * s.max_chunks + ch) * (s.hd + 2);
+                            attn_partial_warp(q, K, K + kv_half, key0, min(ATTN_CHUNK, P + 1 - key0), s.hd, dst,
+                                              sm.ex + warp * 32, lane);
+                            // the last of the row's chunks of this head merges them
+                            const int nch = P / ATTN_CHUNK + 1;
+                            unsigned* cnt = s.mcnt + row * s.nq + h;
+                            unsigned old = 0;
+                            if (lane == 0) {
+                                __threadfence();
+                                old = atomicAdd(cnt, 1u);
+                            }
+                            old = __shfl_sync(0xffffffffu, old, 0);
+                            if (old == (unsigned)nch - 1u) {
+                                __threadfence();
+                                const float* base = s.part + ((int64_t)row * s.nq + h) * s.max_chunks * (s.hd + 2);
+                                const float* gate = s.proj + (int64_t)row * s.proj_ld + s.nq * s.hd + (int64_t)h * s.hd;
+                                sk_merge_head(base, nch, s.hd, gate, s.attn + (int64_t)row * s.nq * s.hd + (int64_t)h * s.hd,
+                                              lane);
+                                if (lane == 0) *cnt = 0u;  // ready for the next attention layer
+                            }
+                        }
+                        break;
+                    }
+                    default: break;
+                }
+            } else if (gemv) {
+                // keep the slab count in step with the producer (nothing is consumed)
+                gs += nmine * p.nks;
+            }
+            if (td) td[2] = globaltimer();
+            sk_arrive(s, pid);
+            if (td) td[3] = globaltimer();
         }
-        if (l < s.L) (att ? ia : ig)++;
+        if (l < s.L) (sk_attn(s, l) ? ia : ig)++;
     }
-    if (s.trace && blockIdx.x == 0 && threadIdx.x == 0) s.trace[255] = globaltimer();
+    if (s.trace && blockIdx.x == 0 && tid == 0) s.trace[SK_TRACE_SLOTS - 1] = globaltimer();
 }
 
 }  // namespace hgd

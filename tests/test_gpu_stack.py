@@ -351,7 +351,7 @@ def test_persistent_launch_equals_kernel_chain(hgd, full, which):
     for k, ((l1, a1, s1, t1), (l2, a2, s2, t2)) in enumerate(zip(rp, rc)):
         assert torch.equal(l1, l2), f"call {k}: logits differ"
         assert torch.equal(a1, a2) and torch.equal(s1, s2) and torch.equal(t1, t2), f"call {k}"
-    for a, b in ((sp.S, sc.S), (sp.conv, sc.conv), (sp.kv, sc.kv), (sp.pos, sc.pos)):
+    for a, b in ((sp.S, sc.S), (sp.conv, sc.conv), (sp.kv, sc.kv), (sp.pos, sc.pos), (sp.resid, sc.resid)):
         assert torch.equal(a, b)
 
 
