@@ -329,7 +329,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="chain", choices=["chain", "persistent"],
+    ap.add_argument("--path", default="persistent", choices=["chain", "persistent"],
                     help="chain: one kernel per op, PDL-overlapped, in CUDA graphs; "
                          "persistent: the whole step in one cooperative launch")
     ap.add_argument("--cpu-tokens", type=int, default=4)

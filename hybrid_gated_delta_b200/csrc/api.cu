@@ -234,7 +234,8 @@ int check_supported(const Dims& d) {
     const bool ok =
         d.D % 32 == 0 && d.D <= 65536 && (d.H * d.dv) % 32 == 0 && (d.nq * d.hd) % 32 == 0 &&
         d.I % 32 == 0 && (d.dk == 32 || d.dk == 64 || d.dk == 128 || d.dk == 256) && d.dv % 16 == 0 &&
-        d.dv <= 1024 && d.kc == 4 && d.hd % 32 == 0 && d.hd <= ATTN_MAX_HD && d.nq % d.nkv == 0 &&
+        d.dv <= 1024 && d.kc == 4 && (d.hd == 32 || d.hd == 64 || d.hd == 128 || d.hd == 256) &&
+        d.nq % d.nkv == 0 &&
         d.nq / d.nkv <= ATTN_MAX_GROUP;
     return ok ? HGD_OK : HGD_ERR_UNSUPPORTED_SHAPE;
 }
@@ -325,7 +326,7 @@ constexpr size_t kBarTraceOff = kBarCtrlBytes + (size_t)SK_MAX_PHASES * SK_CTR_S
 #ifdef HGD_TRACE_DETAIL
 // instrumented builds also keep every CTA's phase times after the timestamps
 constexpr size_t kBarDetailOff = kBarTraceOff + (size_t)SK_TRACE_SLOTS * 8;
-constexpr size_t kBarSlabOff = kBarDetailOff + (size_t)SK_MAX_PHASES * SK_TRACE_CTAS * 4 * 8;
+constexpr size_t kBarSlabOff = kBarDetailOff + (size_t)SK_MAX_PHASES * SK_TRACE_CTAS * 8 * 8;
 constexpr size_t kBarBytes = kBarSlabOff + (size_t)SK_TRACE_SLABS * 3 * 8;
 #else
 constexpr size_t kBarBytes = kBarTraceOff + (size_t)SK_TRACE_SLOTS * 8;

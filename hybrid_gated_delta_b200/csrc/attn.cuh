@@ -9,9 +9,10 @@
 // RoPE of q and k at P and the append of K and V to the bf16 cache run in the
 // in-projection's epilogue, gemv.cuh EPI_ROPE):
 //   k_attn_partial:  per (row, kv head, chunk of CHUNK keys), the four query
-//                    heads of the group: s = q.k / sqrt(hd), chunk max m,
-//                    l = sum exp(s - m), acc = sum exp(s - m) v, all fp32 in
-//                    ascending key order;
+//                    heads of the group: s = q.k / sqrt(hd) (each lane's share
+//                    of the dims, then a butterfly over the lanes), chunk max
+//                    m, l = sum exp(s - m), acc = sum exp(s - m) v, fp32, the
+//                    sums over keys in ascending key order;
 //   k_attn_merge:    per (row, query head): M = max m_c, L = sum exp(m_c - M) l_c,
 //                    out = (sum exp(m_c - M) acc_c) / L * sigmoid(gate) -> bf16.
 // The chunk width is a constant, so the partials of a row depend only on its
@@ -38,54 +39,111 @@ struct AttnParams {
 };
 
 // One attention partial, computed by one warp: query q (fp32, rotated) over
-// the nk keys key0 .. key0 + nk - 1 of one (stream, kv head) cache (K, V at
-// position 0, rows of hd bf16).  Lane j scores key key0 + j (dot product over
-// hd in ascending order, 8 elements at a time); chunk max m, l = sum exp(s - m),
-// acc[d] = sum_j exp(s_j - m) v_j[d] in ascending key order.  dst: [hd + 2] =
-// m, l, acc.  ex: 32 floats of this warp's shared scratch.
-__device__ __forceinline__ void attn_partial_warp(const float* q, const bf16_t* K, const bf16_t* V, int key0,
-                                                  int nk, int hd, float* dst, float* ex, int lane) {
-    float sc = -INFINITY;
-    if (lane < nk) {
-        const bf16_t* kr = K + (int64_t)(key0 + lane) * hd;
-        float d = 0.f;
-#pragma unroll 8
-        for (int e = 0; e < hd; e += 8) {
-            const uint4 kv = *reinterpret_cast<const uint4*>(kr + e);
-            const float4 q0 = *reinterpret_cast<const float4*>(q + e);
-            const float4 q1 = *reinterpret_cast<const float4*>(q + e + 4);
-            d = fmaf(q0.x, bf_lo(kv.x), d); d = fmaf(q0.y, bf_hi(kv.x), d);
-            d = fmaf(q0.z, bf_lo(kv.y), d); d = fmaf(q0.w, bf_hi(kv.y), d);
-            d = fmaf(q1.x, bf_lo(kv.z), d); d = fmaf(q1.y, bf_hi(kv.z), d);
-            d = fmaf(q1.z, bf_lo(kv.w), d); d = fmaf(q1.w, bf_hi(kv.w), d);
-        }
-        sc = d * (1.0f / sqrtf((float)hd));
+// the nk <= 32 keys key0 .. key0 + nk - 1 of one (stream, kv head) cache (K, V
+// at position 0, rows of hd bf16).  Lane l owns the DPL = hd / 32 contiguous
+// dims [l*DPL, (l+1)*DPL): per key it forms its share of q.k (fmaf over its
+// dims in order) and a butterfly over the lanes completes the dot product;
+// s_j = dot / sqrt(hd), chunk max m, l = sum_j exp(s_j - m) (butterfly),
+// acc[d] = sum_j exp(s_j - m) v_j[d] in ascending key order.  Key and value
+// rows load coalesced, 16 keys at a time.  dst: [hd + 2] = m, l, acc.
+// DPL consecutive bf16 of a cache row, packed two per word (DPL = 1: one).
+template <int DPL>
+struct AttnRow { uint32_t w[(DPL + 1) / 2]; };
+template <int DPL>
+__device__ __forceinline__ AttnRow<DPL> attn_rowload(const bf16_t* row) {
+    AttnRow<DPL> r;
+    if (DPL == 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(row);
+        r.w[0] = u.x; r.w[1] = u.y; r.w[2] = u.z; r.w[3] = u.w;
+    } else if (DPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(row);
+        r.w[0] = u.x; r.w[1] = u.y;
+    } else if (DPL == 2) {
+        r.w[0] = *reinterpret_cast<const uint32_t*>(row);
+    } else {
+        r.w[0] = (uint32_t)row[0];
     }
-    // chunk max and sum of exp (butterflies: order fixed by the lane pattern)
+    return r;
+}
+template <int DPL>
+__device__ __forceinline__ float attn_elem(const AttnRow<DPL>& r, int i) {
+    return (i & 1) ? bf_hi(r.w[i >> 1]) : bf_lo(r.w[i >> 1]);
+}
+
+template <int DPL>
+__device__ void attn_partial_warp_t(const float* q, const bf16_t* K, const bf16_t* V, int key0, int nk, float* dst,
+                                    int lane) {
+    constexpr int hd = 32 * DPL, KB = 16;
+    const int d0 = lane * DPL;
+    float qv[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) qv[i] = q[d0 + i];
+    float sc = -INFINITY;  // lane j: key j's scaled score
+#pragma unroll
+    for (int b = 0; b < 32; b += KB) {
+        if (b >= nk) break;
+        AttnRow<DPL> kr[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            if (b + j < nk) kr[j] = attn_rowload<DPL>(K + (int64_t)(key0 + b + j) * hd + d0);
+            else {
+#pragma unroll
+                for (int i = 0; i < (DPL + 1) / 2; ++i) kr[j].w[i] = 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            float dd = 0.f;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) dd = fmaf(qv[i], attn_elem<DPL>(kr[j], i), dd);
+            dd = warp_sum(dd);
+            if (lane == b + j && b + j < nk) sc = dd * (1.0f / sqrtf((float)hd));
+        }
+    }
     float m = sc;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const float e = (lane < nk) ? expf(sc - m) : 0.f;
     const float l = warp_sum(e);
-    ex[lane] = e;
-    __syncwarp();
-    // acc[d]: lane owns dims 8*lane .. +7 (and +256 .. for larger hd); keys in order
-    for (int d0 = lane * 8; d0 < hd; d0 += 256) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int j = 0; j < nk; ++j) {
-            const uint4 vv = *reinterpret_cast<const uint4*>(V + (int64_t)(key0 + j) * hd + d0);
-            const float w = ex[j];
-            acc[0] = fmaf(w, bf_lo(vv.x), acc[0]); acc[1] = fmaf(w, bf_hi(vv.x), acc[1]);
-            acc[2] = fmaf(w, bf_lo(vv.y), acc[2]); acc[3] = fmaf(w, bf_hi(vv.y), acc[3]);
-            acc[4] = fmaf(w, bf_lo(vv.z), acc[4]); acc[5] = fmaf(w, bf_hi(vv.z), acc[5]);
-            acc[6] = fmaf(w, bf_lo(vv.w), acc[6]); acc[7] = fmaf(w, bf_hi(vv.w), acc[7]);
+    float acc[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int b = 0; b < 32; b += KB) {
+        if (b >= nk) break;
+        AttnRow<DPL> vr[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            if (b + j < nk) vr[j] = attn_rowload<DPL>(V + (int64_t)(key0 + b + j) * hd + d0);
+            else {
+#pragma unroll
+                for (int i = 0; i < (DPL + 1) / 2; ++i) vr[j].w[i] = 0u;
+            }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dst[2 + d0 + i] = acc[i];
+        for (int j = 0; j < KB; ++j) {
+            const float w = __shfl_sync(0xffffffffu, e, b + j);
+            if (b + j < nk) {
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, attn_elem<DPL>(vr[j], i), acc[i]);
+            }
+        }
     }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) dst[2 + d0 + i] = acc[i];
     if (lane == 0) { dst[0] = m; dst[1] = l; }
     __syncwarp();
+}
+
+// hd = 32 * DPL with DPL one of 1, 2, 4, 8 (the shapes check_supported admits).
+__device__ __forceinline__ void attn_partial_warp(const float* q, const bf16_t* K, const bf16_t* V, int key0,
+                                                  int nk, int hd, float* dst, int lane) {
+    switch (hd) {
+        case 256: attn_partial_warp_t<8>(q, K, V, key0, nk, dst, lane); break;
+        case 128: attn_partial_warp_t<4>(q, K, V, key0, nk, dst, lane); break;
+        case 64: attn_partial_warp_t<2>(q, K, V, key0, nk, dst, lane); break;
+        default: attn_partial_warp_t<1>(q, K, V, key0, nk, dst, lane); break;
+    }
 }
 
 // Merge of the nch chunk partials (rows of hd + 2 floats: m, l, acc) of one query
@@ -123,12 +181,11 @@ __global__ void __launch_bounds__(32 * ATTN_MAX_GROUP) k_attn_partial(const __gr
     const int group = p.nq / p.nkv, hd = p.hd;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = g * group + warp;  // this warp's query head
-    __shared__ float ex[ATTN_MAX_GROUP][ATTN_CHUNK];
     const bf16_t* K = p.kcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd;
     const bf16_t* V = p.vcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd;
     const float* q = p.qrot + (int64_t)row * p.nq * hd + (int64_t)h * hd;
     float* dst = p.part + (((int64_t)row * p.nq + h) * p.max_chunks + ch) * (hd + 2);
-    attn_partial_warp(q, K, V, key0, nk, hd, dst, ex[warp], lane);
+    attn_partial_warp(q, K, V, key0, nk, hd, dst, lane);
 }
 
 // grid (M, nq), block hd.

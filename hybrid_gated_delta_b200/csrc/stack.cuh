@@ -82,7 +82,7 @@ struct SkParams {
     int32_t* status;
     unsigned* bar;               // control words and phase counters (zeroed before the launch)
     unsigned long long* trace;   // [SK_TRACE_SLOTS] %globaltimer, or null
-    unsigned long long* tdetail; // [SK_MAX_PHASES][SK_TRACE_CTAS][4] per-CTA phase times, or null
+    unsigned long long* tdetail; // [SK_MAX_PHASES][SK_TRACE_CTAS][8] per-CTA phase times, or null
     unsigned long long* tslab;   // CTA 0: [SK_TRACE_SLABS][3] slab issue / ready / release times, or null
     SkLayer layer[HGD_MAX_LAYERS];
 };
@@ -378,12 +378,17 @@ __device__ void sk_pro_gated(const SkParams& s, const GemvParams& p, const bf16_
 // sigmoid(gate), by one warp.  Per dim d the arithmetic of attn_merge_dim:
 // M = max_c m_c, then in chunk order w_c = exp(m_c - M), L += w_c l_c,
 // acc_d += w_c acc_c[d].  Lane c % 32 loads chunk c's (m, l) and computes w_c
-// (shared by shuffles); lane j holds dims j, j + 32, ... (hd <= 256) and loads
-// them for SK_MB chunks at a time.
-constexpr int SK_MB = 4;
-__device__ void sk_merge_head(const float* base, int nch, int hd, const float* gate, bf16_t* out, int lane) {
-    const int nd = hd / 32;
-    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+// (shared by shuffles); lane j holds the hd / 32 contiguous dims from
+// j * hd / 32 (hd one of 32, 64, 128, 256) and loads them for SK_MB chunks at
+// a time.
+constexpr int SK_MB = 8;
+template <int DPL>
+__device__ void sk_merge_head_t(const float* base, int nch, const float* gate, bf16_t* out, int lane) {
+    constexpr int hd = 32 * DPL, NV = (DPL + 3) / 4;  // float4s per lane per chunk
+    const int d0 = lane * DPL;
+    float L = 0.f, acc[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
     float Mx = -INFINITY;
     for (int c = lane; c < nch; c += 32) Mx = fmaxf(Mx, __ldcg(base + (int64_t)c * (hd + 2)));
 #pragma unroll
@@ -398,12 +403,26 @@ __device__ void sk_merge_head(const float* base, int nch, int hd, const float* g
         }
         const int nb = min(32, nch - cb);
         for (int j0 = 0; j0 < nb; j0 += SK_MB) {
-            float v[SK_MB][8];
+            float v[SK_MB][DPL];
 #pragma unroll
             for (int u = 0; u < SK_MB; ++u) {
-                const float* pc = base + (int64_t)(cb + j0 + u) * (hd + 2) + 2;
+                const float* pc = base + (int64_t)(cb + j0 + u) * (hd + 2) + 2 + d0;
+                if (j0 + u < nb) {
+                    if (DPL >= 4) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) v[u][k] = (j0 + u < nb && k < nd) ? __ldcg(pc + lane + 32 * k) : 0.f;
+                        for (int k = 0; k < NV; ++k) {
+                            const float2 a = __ldcg(reinterpret_cast<const float2*>(pc + 4 * k));
+                            const float2 b = __ldcg(reinterpret_cast<const float2*>(pc + 4 * k + 2));
+                            v[u][4 * k] = a.x; v[u][4 * k + 1] = a.y; v[u][4 * k + 2] = b.x; v[u][4 * k + 3] = b.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < DPL; ++i) v[u][i] = __ldcg(pc + i);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < DPL; ++i) v[u][i] = 0.f;
+                }
             }
 #pragma unroll
             for (int u = 0; u < SK_MB; ++u) {
@@ -412,18 +431,22 @@ __device__ void sk_merge_head(const float* base, int nch, int hd, const float* g
                 if (j0 + u < nb) {
                     L = fmaf(w, lc, L);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        if (k < nd) acc[k] = fmaf(w, v[u][k], acc[k]);
+                    for (int i = 0; i < DPL; ++i) acc[i] = fmaf(w, v[u][i], acc[i]);
                 }
             }
         }
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-        if (k < nd) {
-            const int dd = lane + 32 * k;
-            out[dd] = f2bf(acc[k] / L * sigmoid_f(gate[dd]));
-        }
+    for (int i = 0; i < DPL; ++i) out[d0 + i] = f2bf(acc[i] / L * sigmoid_f(gate[d0 + i]));
+}
+__device__ __forceinline__ void sk_merge_head(const float* base, int nch, int hd, const float* gate, bf16_t* out,
+                                              int lane) {
+    switch (hd) {
+        case 256: sk_merge_head_t<8>(base, nch, gate, out, lane); break;
+        case 128: sk_merge_head_t<4>(base, nch, gate, out, lane); break;
+        case 64: sk_merge_head_t<2>(base, nch, gate, out, lane); break;
+        default: sk_merge_head_t<1>(base, nch, gate, out, lane); break;
+    }
 }
 
 // Down-projection input: the SwiGLU rows (bf16) as they are.
@@ -490,7 +513,8 @@ __device__ __forceinline__ void sk_slab_mma(const bf16_t* tile, const bf16_t* xb
 template <int EPI>
 __device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const SkRing& r, const bf16_t* xs,
                                 float* pbuf, float* cbuf, GvBest<1>& best, int& gs, int vc,
-                                volatile int* cta_abort, int warp, int lane, int phase) {
+                                volatile int* cta_abort, int warp, int lane, int phase,
+                                unsigned long long* td = nullptr) {
     const int G = gridDim.x;
     const int XS = p.K + GV_PAD;
     const int r8 = lane >> 2, c = lane & 3;
@@ -523,7 +547,9 @@ __device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const Sk
             *reinterpret_cast<float2*>(pp + r8 * 8 + 2 * c) = make_float2(part[0], part[1]);
             *reinterpret_cast<float2*>(pp + (r8 + 8) * 8 + 2 * c) = make_float2(part[2], part[3]);
         }
+        if (td && i0 == 0) td[4] = globaltimer();
         named_bar(1, SK_CT);
+        if (td && i0 == 0) td[5] = globaltimer();
         if (!*cta_abort) {
             for (int i = i0 + warp; i < i1; i += SK_CW) {
                 float yacc[1][4];
@@ -537,7 +563,9 @@ __device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const Sk
                 gv_finish<1, EPI>(p, vc + i * G, 0, yacc, lane, cbuf + warp * GV_ROWS * 8, best);
             }
         }
+        if (td && i0 == 0) td[6] = globaltimer();
         named_bar(1, SK_CT);  // the partial buffer is reused by the next round
+        if (td && i0 == 0) td[7] = globaltimer();
     }
     gs += nmine * nsl;
 }
@@ -793,7 +821,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
             if (s.trace && blockIdx.x == 0 && tid == 0 && pid < SK_TRACE_SLOTS - 1) s.trace[pid] = globaltimer();
             // per-CTA phase times: wait done, prologue done, GEMV or items done, arrival
             unsigned long long* td = (s.tdetail && tid == 0 && blockIdx.x < SK_TRACE_CTAS)
-                                         ? s.tdetail + ((size_t)pid * SK_TRACE_CTAS + blockIdx.x) * 4
+                                         ? s.tdetail + ((size_t)pid * SK_TRACE_CTAS + blockIdx.x) * 8
                                          : nullptr;
             if (td) td[0] = globaltimer();
             if (live && (!gemv || nmine > 0)) {
@@ -815,24 +843,24 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                 switch (kind) {
                     case SK_IN_GDN:
                         sk_gemv_consume<EPI_QKV_CONV>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
-                                                      warp, lane, pid);
+                                                      warp, lane, pid, td);
                         break;
                     case SK_IN_ATT:
                         sk_gemv_consume<EPI_ROPE>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort, warp,
-                                                  lane, pid);
+                                                  lane, pid, td);
                         break;
                     case SK_SWIGLU:
                         sk_gemv_consume<EPI_SWIGLU>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
-                                                    warp, lane, pid);
+                                                    warp, lane, pid, td);
                         break;
                     case SK_HEAD:
                         sk_gemv_consume<EPI_ARGMAX>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
-                                                    warp, lane, pid);
+                                                    warp, lane, pid, td);
                         gv_argmax_cta<1>(p, best, sm.amax_v, sm.amax_i, warp, lane, tid, SK_CW, blockIdx.x, G, true);
                         break;
                     case SK_OUT_GDN: case SK_OUT_ATT: case SK_DOWN:
                         sk_gemv_consume<EPI_RESID>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
-                                                   warp, lane, pid);
+                                                   warp, lane, pid, td);
                         break;
                     case SK_GDN:
                         for (int it = gw; it < n_gdn; it += nw) {
@@ -862,7 +890,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                             const float* q = s.qrot + (int64_t)row * s.nq * s.hd + (int64_t)h * s.hd;
                             float* dst = s.part + (((int64_t)row * s.nq + h) * s.max_chunks + ch) * (s.hd + 2);
                             attn_partial_warp(q, K, K + kv_half, key0, min(ATTN_CHUNK, P + 1 - key0), s.hd, dst,
-                                              sm.ex + warp * 32, lane);
+                                              lane);
                             // the last of the row's chunks of this head merges them
                             const int nch = P / ATTN_CHUNK + 1;
                             unsigned* cnt = s.mcnt + row * s.nq + h;
