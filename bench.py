@@ -207,6 +207,8 @@ def run_gpu(args) -> None:
     import hybrid_gated_delta_b200 as hgd
 
     cfg = syn.STACK_CFG
+    if args.layers and args.layers != cfg["n_layers"]:
+        cfg = dict(cfg, n_layers=args.layers)
     B = 1
     Lmax = ((PREFILL + args.warmup + args.steps + 2 + 63) // 64) * 64
     model = hgd.Model(cfg, syn.stack_weights(cfg, seed=4))
@@ -296,7 +298,9 @@ def run_gpu(args) -> None:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch": 1, "kv_context": PREFILL, "decode_tokens": args.steps,
+        "config": {"workload": WORKLOAD if cfg is syn.STACK_CFG else
+                   f"PROFILING ONLY, not a bench line: {cfg['n_layers']}-layer stack of the same width",
+                   "batch": 1, "kv_context": PREFILL, "decode_tokens": args.steps,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2: 1.5 GB of weights streamed per step (L2 126 MB)"},
         "hbm_gbs": step_gbs,
@@ -329,6 +333,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling aid: a stack of this many layers of the same width (the line it prints "
+                         "is marked as not a bench line); 0 = the benchmark's 24")
     ap.add_argument("--path", default="persistent", choices=["chain", "persistent"],
                     help="chain: one kernel per op, PDL-overlapped, in CUDA graphs; "
                          "persistent: the whole step in one cooperative launch")
