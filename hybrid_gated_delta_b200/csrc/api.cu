@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <utility>
 #include <cstdio>
+#include <cmath>
 #include <cstring>
 
 #include "attn.cuh"
@@ -242,6 +243,9 @@ int check_supported(const Dims& d) {
 
 size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
 
+// base^(-2/hd): the RoPE frequency ratio between neighbouring dim pairs.
+double rope_inv1_of(const Dims& d, float base) { return std::pow((double)base, -2.0 / (double)d.hd); }
+
 // numel of one weight tensor (0 if absent)
 size_t weight_numel(const Dims& d, const hgd_config* c, int layer, int t) {
     if (layer < 0) {
@@ -327,7 +331,7 @@ constexpr size_t kBarTraceOff = kBarCtrlBytes + (size_t)SK_MAX_PHASES * SK_CTR_S
 // instrumented builds also keep every CTA's phase times after the timestamps
 constexpr size_t kBarDetailOff = kBarTraceOff + (size_t)SK_TRACE_SLOTS * 8;
 constexpr size_t kBarSlabOff = kBarDetailOff + (size_t)SK_MAX_PHASES * SK_TRACE_CTAS * 8 * 8;
-constexpr size_t kBarBytes = kBarSlabOff + (size_t)SK_TRACE_SLABS * 3 * 8;
+constexpr size_t kBarBytes = kBarSlabOff + (size_t)SK_TRACE_SLABS * 4 * 8;
 #else
 constexpr size_t kBarBytes = kBarTraceOff + (size_t)SK_TRACE_SLOTS * 8;
 #endif
@@ -384,7 +388,7 @@ constexpr int kSkPartialSlabs = 32;  // slab partials of the non-split phases' r
 // Ring slots of the persistent launch for M token rows: the most (24, 16 or 8)
 // that fit beside the token rows and the fixed buffers; 0 if none fits.
 int sk_ring_slots(const Dims& d, int M) {
-    for (int ns = 24; ns >= 8; ns -= 8) {
+    for (int ns = 3 * SK_CW; ns >= SK_CW; ns -= SK_CW) {
         const size_t smem = (size_t)ns * SK_SLAB_BYTES + sk_fixed_bytes(M, sk_kmax(d), d.D, kSkPartialSlabs, ns);
         if (smem <= (size_t)GV_SMEM_LIMIT) return ns;
     }
@@ -402,9 +406,9 @@ bool sk_supported(const Dims& d, int M) {
            gv_slabs(sk_kmax(d)) <= kSkPartialSlabs && M * d.nq <= SK_MCNT_WORDS && sk_ring_slots(d, M) > 0;
 }
 
-template <int KPL>
+template <int KPL, int DPL>
 int sk_launch_t(const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
-    auto kern = k_stack<KPL>;
+    auto kern = k_stack<KPL, DPL>;
     static int attr_done[64];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -432,6 +436,25 @@ int sk_launch_t(const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return launch_status(cudaLaunchKernelEx(&cfg, kern, prm));
+}
+
+// The persistent kernel for this model's GDN key width (64 or 128) and
+// attention head width (32, 64, 128 or 256).
+int sk_launch(const Dims& d, const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
+    if (d.dk == 128) {
+        switch (d.hd) {
+            case 256: return sk_launch_t<4, 8>(prm, smem, sms, s);
+            case 128: return sk_launch_t<4, 4>(prm, smem, sms, s);
+            case 64: return sk_launch_t<4, 2>(prm, smem, sms, s);
+            default: return sk_launch_t<4, 1>(prm, smem, sms, s);
+        }
+    }
+    switch (d.hd) {
+        case 256: return sk_launch_t<2, 8>(prm, smem, sms, s);
+        case 128: return sk_launch_t<2, 4>(prm, smem, sms, s);
+        case 64: return sk_launch_t<2, 2>(prm, smem, sms, s);
+        default: return sk_launch_t<2, 1>(prm, smem, sms, s);
+    }
 }
 
 }  // namespace
@@ -717,7 +740,7 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
     prm.nkv = d.nkv; prm.hd = d.hd; prm.I = d.I; prm.every = d.every;
     prm.C = (int)d.C; prm.gdn_out = (int)d.gdn_out; prm.attn_out = (int)d.attn_out;
     prm.proj_ld = (int)std::max(d.gdn_out, d.attn_out); prm.kmax = sk_kmax(d);
-    prm.eps = m->cfg.norm_eps; prm.rope_base = m->cfg.rope_base;
+    prm.eps = m->cfg.norm_eps; prm.rope_inv1 = rope_inv1_of(d, m->cfg.rope_base);
     prm.B = st->B; prm.T = T; prm.M = st->B * T; prm.Lmax = st->Lmax; prm.max_chunks = max_chunks_of(st->Lmax);
     prm.ns = sk_ring_slots(d, prm.M); prm.pb = kSkPartialSlabs;
     prm.embed = m->embed; prm.final_norm = m->final_norm;
@@ -754,7 +777,7 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
         return HGD_ERR_CUDA;
     }
     const size_t smem = sk_smem_bytes(d, prm.M, prm.ns);
-    return d.dk == 128 ? sk_launch_t<4>(prm, smem, di.sms, s) : sk_launch_t<2>(prm, smem, di.sms, s);
+    return sk_launch(d, prm, smem, di.sms, s);
 }
 
 int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,
@@ -813,7 +836,7 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             p.y = proj; p.y_ld = proj_ld; p.status = status_dev;
             if (att) {
                 p.rope_nq = d.nq; p.rope_nkv = d.nkv; p.rope_hd = d.hd; p.rope_Lmax = Lmax;
-                p.rope_base = m->cfg.rope_base; p.rope_q = qrot;
+                p.rope_inv1 = rope_inv1_of(d, m->cfg.rope_base); p.rope_q = qrot;
                 p.rope_k = kv + (size_t)ia * 2 * kv_half; p.rope_v = p.rope_k + kv_half;
                 p.rope_pos = pos; p.conv_T = T;
             }

@@ -98,6 +98,21 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// As mbar_wait_bounded, sleeping `ns` nanoseconds between tests: for a waiter
+// that is not on a critical path and should leave the issue slots of its SM
+// sub-partition to the warps that are.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                 unsigned ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        __nanosleep(ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (abort_flag && *abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+    }
+}
+
 // ----------------------------------------------------------- bulk (TMA) copy
 // 1-D bulk copy global -> shared, completing `bytes` of transaction count on
 // `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.  No multicast.
@@ -108,6 +123,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
         " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst_smem)),
         "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
+}
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned start) into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;

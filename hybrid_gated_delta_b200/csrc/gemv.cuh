@@ -81,7 +81,7 @@ struct GemvParams {
     // (fp32) at column nq*hd + g; k rows are rotated and v rows copied into the
     // bf16 caches [B][nkv][Lmax][hd] at position pos[b] + t (row m0 + m is stream
     // (m0 + m) / conv_T, row (m0 + m) % conv_T).
-    int rope_nq, rope_nkv, rope_hd, rope_Lmax; float rope_base;
+    int rope_nq, rope_nkv, rope_hd, rope_Lmax; double rope_inv1;  // inv1 = base^(-2/hd)
     float* rope_q; bf16_t* rope_k; bf16_t* rope_v; const int32_t* rope_pos;
     int32_t* status;
 };
@@ -139,12 +139,19 @@ __host__ __device__ inline int64_t rope_src_row(int64_t v, int nq, int nkv, int 
 }
 
 // sin and cos of the RoPE angle of dim pair i at position P: the angle
-// P * base^(-2i/hd) in double, reduced to [-pi, pi] in double, then fp32.
-__device__ __forceinline__ void rope_sincos(int P, int i, int hd, float base, float* sn, float* cs) {
-    const double inv = exp2(-2.0 * (double)i / (double)hd * log2((double)base));
+// P * base^(-2i/hd) in double, with base^(-2i/hd) = inv1^i (inv1 = base^(-2/hd),
+// computed once in double on the host; the power by repeated squaring in
+// double, relative error ~1e-15), reduced to [-pi, pi] in double, then the fp32
+// sine and cosine of the reduced angle.
+__device__ __forceinline__ void rope_sincos(int P, int i, double inv1, float* sn, float* cs) {
+    double inv = 1.0, b = inv1;
+    for (int e = i; e; e >>= 1) {
+        if (e & 1) inv *= b;
+        b *= b;
+    }
     const double th = (double)P * inv;
-    const double tw = 6.283185307179586476925286766559;
-    const float r = (float)(th - tw * rint(th / tw));
+    const double tw = 6.283185307179586476925286766559, itw = 0.15915494309189533576888376337251;
+    const float r = (float)(th - tw * rint(th * itw));
     sincosf(r, sn, cs);
 }
 
@@ -426,7 +433,7 @@ __device__ __forceinline__ void gv_finish(const GemvParams& p, int rb, int s_ite
                             continue;
                         }
                         float sn, cs;
-                        rope_sincos(P, i, hd, p.rope_base, &sn, &cs);
+                        rope_sincos(P, i, p.rope_inv1, &sn, &cs);
                         const float x0 = a * cs - bb * sn, x1 = bb * cs + a * sn;
                         if (!isk) {
                             float* qo = p.rope_q + (int64_t)n * qw + (int64_t)head * hd;

@@ -68,7 +68,8 @@ struct SkLayer { const bf16_t* w[HGD_W_LAYER_COUNT]; };
 struct SkParams {
     int L, D, V, H, dk, dv, nq, nkv, hd, I, every;
     int C, gdn_out, attn_out, proj_ld, kmax;
-    float eps, rope_base;
+    float eps;
+    double rope_inv1;  // base^(-2/hd)
     int B, T, M, Lmax, max_chunks;
     int ns, pb;      // ring slots (a multiple of SK_CW), slab partials the partial buffer holds
     const bf16_t* embed; const bf16_t* final_norm;
@@ -83,7 +84,7 @@ struct SkParams {
     unsigned* bar;               // control words and phase counters (zeroed before the launch)
     unsigned long long* trace;   // [SK_TRACE_SLOTS] %globaltimer, or null
     unsigned long long* tdetail; // [SK_MAX_PHASES][SK_TRACE_CTAS][8] per-CTA phase times, or null
-    unsigned long long* tslab;   // CTA 0: [SK_TRACE_SLABS][3] slab issue / ready / release times, or null
+    unsigned long long* tslab;   // CTA 0: [SK_TRACE_SLABS][4] slab issue / ready / release / wait-start times, or null
     SkLayer layer[HGD_MAX_LAYERS];
 };
 
@@ -118,14 +119,18 @@ __device__ __forceinline__ unsigned* sk_ctr(const SkParams& s, int p) {
 }
 
 // Record the first wait that ran out; set the status and the abort word.
-__device__ __forceinline__ void sk_timeout(const SkParams& s, unsigned what, unsigned phase, unsigned seq) {
-    if (atomicCAS(&s.bar[1], 0u, what) == 0u) {
-        s.bar[2] = phase;
-        s.bar[3] = blockIdx.x;
-        s.bar[4] = seq;
+__device__ __forceinline__ void sk_timeout_w(unsigned* bar, int32_t* status, unsigned what, unsigned phase,
+                                             unsigned seq) {
+    if (atomicCAS(&bar[1], 0u, what) == 0u) {
+        bar[2] = phase;
+        bar[3] = blockIdx.x;
+        bar[4] = seq;
     }
-    set_status(s.status, HGD_ERR_TIMEOUT);
-    atomicExch(&s.bar[0], 1u);
+    set_status(status, HGD_ERR_TIMEOUT);
+    atomicExch(&bar[0], 1u);
+}
+__device__ __forceinline__ void sk_timeout(const SkParams& s, unsigned what, unsigned phase, unsigned seq) {
+    sk_timeout_w(s.bar, s.status, what, phase, seq);
 }
 
 // End of phase p in this CTA: once every consumer warp's writes are done (the
@@ -151,27 +156,33 @@ __device__ __forceinline__ bool sk_bar_and(bool pred) {
     return r != 0;
 }
 
-// Wait until every CTA has arrived at the end of phase p (thread 0 polls, the
-// consumer warps meet at a named barrier).  False, in every consumer thread,
-// on an abort or a timeout.
-__device__ bool sk_wait(const SkParams& s, volatile int* cta_abort, int p) {
-    if (threadIdx.x == 0 && !*cta_abort) {
+// Wait until every CTA has arrived at the end of phase p.  Lane 0 of warps
+// 0..SK_POLLERS-1 poll the counter, started a fraction of a round trip apart so
+// that the completion is seen soon after it lands; the first to see it raises
+// `seen` (shared) for the others; the consumer warps then meet at a named
+// barrier.  False, in every consumer thread, on an abort or a timeout.
+constexpr int SK_POLLERS = 4;
+__device__ bool sk_wait(const SkParams& s, volatile int* cta_abort, volatile int* seen, int p) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0 && warp < SK_POLLERS && !*cta_abort) {
         const unsigned* c = sk_ctr(s, p);
         const unsigned target = gridDim.x;
-        if (ld_acquire_u32(c) < target) {
+        if (warp) __nanosleep(120u * (unsigned)warp);
+        if (*seen != p && ld_acquire_u32(c) < target) {
             const unsigned long long t0 = globaltimer();
             unsigned it = 0;
-            while (ld_acquire_u32(c) < target) {
+            while (*seen != p && ld_acquire_u32(c) < target) {
                 if ((++it & 31u) == 0u) {
                     if (ld_acquire_u32(&s.bar[0])) { *cta_abort = 1; break; }
                     if (globaltimer() - t0 > kWaitLimitNs) {
-                        sk_timeout(s, 1u, (unsigned)p, 0u);
+                        if (warp == 0) sk_timeout(s, 1u, (unsigned)p, 0u);
                         *cta_abort = 1;
                         break;
                     }
                 }
             }
         }
+        *seen = p;
     }
     return sk_bar_and(!*cta_abort);
 }
@@ -200,7 +211,7 @@ __device__ __forceinline__ void sk_gemv_params(const SkParams& s, int kind, int 
             const size_t kv_half = (size_t)s.B * s.nkv * s.Lmax * s.hd;
             p.W = w[HGD_W_IN]; p.N = s.attn_out; p.K = s.D; p.norm_w = w[HGD_W_IN_NORM];
             p.y = s.proj; p.y_ld = s.proj_ld;
-            p.rope_nq = s.nq; p.rope_nkv = s.nkv; p.rope_hd = s.hd; p.rope_Lmax = s.Lmax; p.rope_base = s.rope_base;
+            p.rope_nq = s.nq; p.rope_nkv = s.nkv; p.rope_hd = s.hd; p.rope_Lmax = s.Lmax; p.rope_inv1 = s.rope_inv1;
             p.rope_q = s.qrot; p.rope_k = s.kv + (size_t)ia * 2 * kv_half; p.rope_v = p.rope_k + kv_half;
             p.rope_pos = s.pos; p.conv_T = s.T; p.m0 = 0;
             break;
@@ -468,40 +479,83 @@ struct SkRing {
 
 // Wait for the weight slab of CTA sequence number g (slot g % ns); false if the
 // wait ran out or the CTA aborted.  Every lane observes the completed phase.
-__device__ __forceinline__ bool sk_slab_wait(const SkParams& s, const SkRing& r, int g, volatile int* cta_abort,
-                                             int phase, int lane) {
+__device__ __forceinline__ bool sk_slab_wait(unsigned* bar, int32_t* status, unsigned long long* tslab,
+                                             const SkRing& r, int g, volatile int* cta_abort, int phase, int lane) {
     const int slot = g % r.ns;
     const uint32_t par = (uint32_t)((g / r.ns) & 1);
+    if (tslab && blockIdx.x == 0 && lane == 0 && g < SK_TRACE_SLABS) tslab[g * 4 + 3] = globaltimer();
     bool got = true;
     if (lane == 0) got = mbar_wait_bounded(&r.full[slot], par, cta_abort);
     got = __shfl_sync(0xffffffffu, got, 0);
     if (got) got = __all_sync(0xffffffffu, mbar_try_wait(&r.full[slot], par));
     if (!got && lane == 0 && !*cta_abort) {
-        sk_timeout(s, 2u, (unsigned)phase, (unsigned)g);
+        sk_timeout_w(bar, status, 2u, (unsigned)phase, (unsigned)g);
         *cta_abort = 1;
     }
-    if (s.tslab && blockIdx.x == 0 && lane == 0 && g < SK_TRACE_SLABS) s.tslab[g * 3 + 1] = globaltimer();
+    if (tslab && blockIdx.x == 0 && lane == 0 && g < SK_TRACE_SLABS) tslab[g * 4 + 1] = globaltimer();
     return got;
 }
 
 // 16 x 8 partial of one slab: chain 0 (even steps) + chain 1 (odd steps), the
-// per-slab arithmetic of k_gemv.
-__device__ __forceinline__ void sk_slab_mma(const bf16_t* tile, const bf16_t* xb, int sg, int nstep, bool has_x,
-                                            int lane, float (&part)[4]) {
+// per-slab arithmetic of k_gemv.  A full slab (every slab of a K that is a
+// multiple of 256) takes a loop without per-step guards, which lets every
+// shared-memory load of the slab issue ahead of the MMAs; a ragged last slab
+// takes the guarded loop, out of line.
+__device__ __noinline__ float4 sk_slab_mma_ragged(const bf16_t* tile, const bf16_t* xs0, int nstep, bool has_x,
+                                                  int lane) {
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int jj = 0; jj < nstep; ++jj) {
+        const uint4 a0 = lds128(tile + jj * 512 + lane * 8);
+        const uint4 a1 = lds128(tile + jj * 512 + 256 + lane * 8);
+        const uint4 Bv = has_x ? lds128(xs0 + jj * 32) : make_uint4(0, 0, 0, 0);
+        float (&acc)[4] = (jj & 1) ? c1 : c0;
+        mma_bf16_16816(acc, a0.x, a1.x, a0.y, a1.y, Bv.x, Bv.y);
+        mma_bf16_16816(acc, a0.z, a1.z, a0.w, a1.w, Bv.z, Bv.w);
+    }
+    return make_float4(c0[0] + c1[0], c0[1] + c1[1], c0[2] + c1[2], c0[3] + c1[3]);
+}
+__device__ __forceinline__ float4 sk_slab_mma(const bf16_t* tile, const bf16_t* xb, int sg, int nstep, bool has_x,
+                                              int lane) {
+    const bf16_t* xs0 = xb + sg * GV_SLAB_STEPS * 32;
+    if (nstep != GV_SLAB_STEPS) return sk_slab_mma_ragged(tile, xs0, nstep, has_x, lane);
     float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int jj = 0; jj < GV_SLAB_STEPS; ++jj) {
-        if (jj < nstep) {
-            const uint4 a0 = lds128(tile + jj * 512 + lane * 8);
-            const uint4 a1 = lds128(tile + jj * 512 + 256 + lane * 8);
-            const uint4 Bv = has_x ? lds128(xb + (sg * GV_SLAB_STEPS + jj) * 32) : make_uint4(0, 0, 0, 0);
-            float (&acc)[4] = (jj & 1) ? c1 : c0;
-            mma_bf16_16816(acc, a0.x, a1.x, a0.y, a1.y, Bv.x, Bv.y);
-            mma_bf16_16816(acc, a0.z, a1.z, a0.w, a1.w, Bv.z, Bv.w);
-        }
+        const uint4 a0 = lds128(tile + jj * 512 + lane * 8);
+        const uint4 a1 = lds128(tile + jj * 512 + 256 + lane * 8);
+        const uint4 bv = has_x ? lds128(xs0 + jj * 32) : make_uint4(0, 0, 0, 0);
+        float (&acc)[4] = (jj & 1) ? c1 : c0;
+        mma_bf16_16816(acc, a0.x, a1.x, a0.y, a1.y, bv.x, bv.y);
+        mma_bf16_16816(acc, a0.z, a1.z, a0.w, a1.w, bv.z, bv.w);
     }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) part[q] = c0[q] + c1[q];
+    return make_float4(c0[0] + c1[0], c0[1] + c1[1], c0[2] + c1[2], c0[3] + c1[3]);
+}
+
+// This warp's slabs j in [jb, je) of a phase round (j congruent to `first`
+// mod 8): wait, partial sums, release the slot, partials to the partial
+// buffer (slab j at pbuf[(j - jb) * 128]).
+__device__ __forceinline__ void sk_round_slabs(const SkRing r, const bf16_t* xb, bool has_x, float* pbuf, int gs,
+                                            int jb, int je, int first, int nsl, int steps_total,
+                                            volatile int* cta_abort, int phase, int lane, unsigned* bar,
+                                            int32_t* status, unsigned long long* tslab) {
+    const int r8 = lane >> 2, c = lane & 3;
+    for (int j = jb + (((first - jb) % SK_CW) + SK_CW) % SK_CW; j < je; j += SK_CW) {
+        const int g = gs + j;
+        const int slot = g % r.ns;
+        if (*cta_abort || !sk_slab_wait(bar, status, tslab, r, g, cta_abort, phase, lane)) break;
+        const int sg = j % nsl;
+        const int nstep = min(GV_SLAB_STEPS, steps_total - sg * GV_SLAB_STEPS);
+        const float4 part = sk_slab_mma(reinterpret_cast<const bf16_t*>(r.ring + slot * SK_SLAB_BYTES), xb, sg,
+                                        nstep, has_x, lane);
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&r.empty[slot]);
+            if (tslab && blockIdx.x == 0 && g < SK_TRACE_SLABS) tslab[g * 4 + 2] = globaltimer();
+        }
+        float* pp = pbuf + (j - jb) * SK_PB_SLAB;
+        *reinterpret_cast<float2*>(pp + r8 * 8 + 2 * c) = make_float2(part.x, part.y);
+        *reinterpret_cast<float2*>(pp + (r8 + 8) * 8 + 2 * c) = make_float2(part.z, part.w);
+    }
 }
 
 // The GEMV of one phase for this CTA's consumer warps.  gs: the CTA's slab
@@ -514,7 +568,7 @@ template <int EPI>
 __device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const SkRing& r, const bf16_t* xs,
                                 float* pbuf, float* cbuf, GvBest<1>& best, int& gs, int vc,
                                 volatile int* cta_abort, int warp, int lane, int phase,
-                                unsigned long long* td = nullptr) {
+                                unsigned long long* td = nullptr, const float* rpre = nullptr) {
     const int G = gridDim.x;
     const int XS = p.K + GV_PAD;
     const int r8 = lane >> 2, c = lane & 3;
@@ -527,26 +581,8 @@ __device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const Sk
     const int R = max(1, s.pb / nsl);  // items per round
     for (int i0 = 0; i0 < nmine; i0 += R) {
         const int i1 = min(nmine, i0 + R);
-        const int jb = i0 * nsl, je = i1 * nsl;
-        // first slab >= jb of this warp
-        int j = jb + (((first - jb) % SK_CW) + SK_CW) % SK_CW;
-        for (; j < je; j += SK_CW) {
-            const int g = gs + j;
-            if (*cta_abort || !sk_slab_wait(s, r, g, cta_abort, phase, lane)) break;
-            const int sg = j % nsl;
-            const int nstep = min(GV_SLAB_STEPS, steps_total - sg * GV_SLAB_STEPS);
-            float part[4];
-            sk_slab_mma(reinterpret_cast<const bf16_t*>(r.ring + (g % r.ns) * SK_SLAB_BYTES), xb, sg, nstep, has_x,
-                        lane, part);
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&r.empty[g % r.ns]);
-                if (s.tslab && blockIdx.x == 0 && g < SK_TRACE_SLABS) s.tslab[g * 3 + 2] = globaltimer();
-            }
-            float* pp = pbuf + (j - jb) * SK_PB_SLAB;
-            *reinterpret_cast<float2*>(pp + r8 * 8 + 2 * c) = make_float2(part[0], part[1]);
-            *reinterpret_cast<float2*>(pp + (r8 + 8) * 8 + 2 * c) = make_float2(part[2], part[3]);
-        }
+        sk_round_slabs(r, xb, has_x, pbuf, gs, i0 * nsl, i1 * nsl, first, nsl, steps_total, cta_abort, phase, lane,
+                       s.bar, s.status, s.tslab);
         if (td && i0 == 0) td[4] = globaltimer();
         named_bar(1, SK_CT);
         if (td && i0 == 0) td[5] = globaltimer();
@@ -560,7 +596,18 @@ __device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const Sk
                     if (sl == 0) { yacc[0][0] = lo.x; yacc[0][1] = lo.y; yacc[0][2] = hi.x; yacc[0][3] = hi.y; }
                     else { yacc[0][0] += lo.x; yacc[0][1] += lo.y; yacc[0][2] += hi.x; yacc[0][3] += hi.y; }
                 }
-                gv_finish<1, EPI>(p, vc + i * G, 0, yacc, lane, cbuf + warp * GV_ROWS * 8, best);
+                if (EPI == EPI_RESID && rpre && i == warp) {
+                    // the residual add of gv_finish, on the rows loaded before the phase
+                    const int rb = vc + i * G;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int n = 2 * c + (q & 1), col = rb * GV_ROWS + r8 + ((q & 2) ? 8 : 0);
+                        if (n < p.M && col < p.N)
+                            reinterpret_cast<bf16_t*>(p.y)[n * p.y_ld + col] = f2bf(rpre[q] + yacc[0][q]);
+                    }
+                } else {
+                    gv_finish<1, EPI>(p, vc + i * G, 0, yacc, lane, cbuf + warp * GV_ROWS * 8, best);
+                }
             }
         }
         if (td && i0 == 0) td[6] = globaltimer();
@@ -572,12 +619,17 @@ __device__ void sk_gemv_consume(const SkParams& s, const GemvParams& p, const Sk
 
 // ------------------------------------------------------------ GDN and attention
 
-// S rows row0..row0+3 of (stream b, head h) of GDN layer ig into registers.
+// S rows row0..row0+3 of (stream b, head h) of GDN layer ig into registers,
+// with the head's A = exp(A_log) and dt_bias.
 template <int KPL>
-__device__ __forceinline__ float* sk_gdn_rows(const SkParams& s, int ig, int it, float (&S)[GDN_RPW][KPL], int lane) {
+__device__ __forceinline__ float* sk_gdn_rows(const SkParams& s, int l, int ig, int it, float (&S)[GDN_RPW][KPL],
+                                              float& A, float& dtb, int lane) {
     constexpr int DK = 32 * KPL;
     const int rg = s.dv / GDN_RPW;
     const int b = it / (s.H * rg), h = (it / rg) % s.H, row0 = (it % rg) * GDN_RPW;
+    const bf16_t* const* w = s.layer[l].w;
+    A = expf(bf2f(w[HGD_W_A_LOG][h]));
+    dtb = bf2f(w[HGD_W_DT_BIAS][h]);
     float* Sbase = s.S + (size_t)ig * s.B * s.H * s.dv * DK + ((int64_t)(b * s.H + h) * s.dv + row0) * DK + lane * KPL;
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
@@ -587,13 +639,11 @@ __device__ __forceinline__ float* sk_gdn_rows(const SkParams& s, int ig, int it,
 // Gated delta rule of GDN item `it` (4 state rows of one stream and head) over
 // the call's T rows, on state rows already in S: the arithmetic of k_gdn_layer.
 template <int KPL>
-__device__ void sk_gdn_item(const SkParams& s, int l, int ig, int it, float (&S)[GDN_RPW][KPL], float* Sbase,
-                            int lane) {
+__device__ void sk_gdn_item(const SkParams& s, int ig, int it, float (&S)[GDN_RPW][KPL], float* Sbase, float A,
+                            float dtb, int lane) {
     constexpr int DK = 32 * KPL;
     const int H = s.H, dv = s.dv, rg = dv / GDN_RPW;
     const int b = it / (H * rg), h = (it / rg) % H, row0 = (it % rg) * GDN_RPW;
-    const bf16_t* const* w = s.layer[l].w;
-    const float A = expf(bf2f(w[HGD_W_A_LOG][h])), dtb = bf2f(w[HGD_W_DT_BIAS][h]);
     for (int t = 0; t < s.T; ++t) {
         const int64_t row = (int64_t)b * s.T + t;
         const float* pr = s.proj + row * s.proj_ld;
@@ -694,18 +744,21 @@ __device__ __forceinline__ SkSmem sk_smem(const SkParams& s, uint8_t* base) {
     return m;
 }
 
-template <int KPL>
+// KPL: GDN key elements per lane (dk / 32); DPL: attention dims per lane (hd / 32).
+template <int KPL, int DPL>
 __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__ SkParams s) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const SkSmem sm = sk_smem(s, smem);
     volatile int* cta_abort = sm.flags;
+    volatile int* seen = sm.flags + 1;  // the last phase whose completion a poller saw
     const SkRing ring{sm.ring, sm.full, sm.empty, s.ns};
     const int G = gridDim.x;
 
     if (tid == 0) {
         for (int i = 0; i < s.ns; ++i) { mbar_init(&sm.full[i], 1); mbar_init(&sm.empty[i], 1); }
         *cta_abort = 0;
+        seen[0] = -1;
         mbar_fence_init();
     }
     __syncthreads();
@@ -737,8 +790,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                     if (lane < PB && j < J) {
                         const int gj = g + lane;
                         const int slot = gj % s.ns;
-                        if (gj >= s.ns &&
-                            !mbar_wait_bounded(&sm.empty[slot], (uint32_t)(((gj / s.ns) - 1) & 1), cta_abort)) {
+                        if (gj >= s.ns && !mbar_wait_sleepy(&sm.empty[slot], (uint32_t)(((gj / s.ns) - 1) & 1),
+                                                            cta_abort, 64u)) {
                             // (an abort raised elsewhere reaches this CTA through its consumers' waits)
                             if (!*cta_abort) sk_timeout(s, 3u, (unsigned)pid, (unsigned)gj);
                             lane_ok = false;
@@ -747,7 +800,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                             const int rb = vc + i * G;
                             const int nstep = min(GV_SLAB_STEPS, steps_total - sg * GV_SLAB_STEPS);
                             const uint32_t bytes = (uint32_t)nstep * 1024u;
-                            if (s.tslab && blockIdx.x == 0 && gj < SK_TRACE_SLABS) s.tslab[gj * 3] = globaltimer();
+                            if (s.tslab && blockIdx.x == 0 && gj < SK_TRACE_SLABS) s.tslab[gj * 4] = globaltimer();
                             mbar_arrive_expect_tx(&sm.full[slot], bytes);
                             bulk_g2s(ring.ring + (size_t)slot * SK_SLAB_BYTES,
                                      p.W + gv_tile_elem(rb, sg * GV_SLAB_STEPS, steps_total, 0, 0), bytes,
@@ -790,7 +843,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
             ++pid;
             if (kind == SK_FINAL) {
                 if (blockIdx.x == 0) {
-                    const bool live = sk_wait(s, cta_abort, pid - 1);
+                    const bool live = sk_wait(s, cta_abort, seen, pid - 1);
                     if (live && warp == 0) sk_final(s, lane);
                 }
                 continue;
@@ -806,6 +859,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
             // work that does not depend on the previous phase: gains, GDN state rows
             float S[GDN_RPW][KPL];
             float* Sbase = nullptr;
+            float gA = 0.f, gdtb = 0.f, rpre[4] = {0.f, 0.f, 0.f, 0.f};
             const int gw = warp * G + blockIdx.x, nw = G * SK_CW;
             const int n_gdn = s.B * s.H * (s.dv / GDN_RPW);
             if (nmine > 0 && (kind == SK_IN_GDN || kind == SK_IN_ATT || kind == SK_SWIGLU || kind == SK_HEAD)) {
@@ -815,9 +869,38 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                 for (int c = tid; c < s.dv / 8; c += SK_CT)
                     *reinterpret_cast<uint4*>(sm.gb + c * 8) = *reinterpret_cast<const uint4*>(p.gnorm_w + c * 8);
             } else if (kind == SK_GDN && gw < n_gdn) {
-                Sbase = sk_gdn_rows<KPL>(s, ig, gw, S, lane);
+                Sbase = sk_gdn_rows<KPL>(s, l, ig, gw, S, gA, gdtb, lane);
             }
-            const bool live = (pid == 0) ? sk_bar_and(!*cta_abort) : sk_wait(s, cta_abort, pid - 1);
+            if (nmine > 0 && (kind == SK_OUT_GDN || kind == SK_OUT_ATT || kind == SK_DOWN)) {
+                // the residual rows this warp's first item adds to (written two or
+                // more phases ago, stable until this phase writes them)
+                const int R = max(1, s.pb / p.nks);
+                if (warp < min(R, nmine)) {
+                    const int rb = vc + warp * G, r8 = lane >> 2, c = lane & 3;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int n = 2 * c + (q & 1), col = rb * GV_ROWS + r8 + ((q & 2) ? 8 : 0);
+                        rpre[q] = (n < s.M && col < p.N) ? bf2f(s.resid[(int64_t)n * s.D + col]) : 0.f;
+                    }
+                }
+            }
+            if (kind == SK_IN_ATT) {
+                // warm L2 with the key and value chunks of this warp's coming attention partials
+                const int n = s.M * s.nq * s.max_chunks;
+                const size_t kv_half = (size_t)s.B * s.nkv * s.Lmax * s.hd;
+                for (int it = gw; lane == 0 && it < n; it += nw) {
+                    const int row = it / (s.nq * s.max_chunks), h = (it / s.max_chunks) % s.nq;
+                    const int ch = it % s.max_chunks, b = row / s.T, t = row % s.T;
+                    const int P = s.pos[b] + t, key0 = ch * ATTN_CHUNK;
+                    if (P < 0 || P >= s.Lmax || key0 > P) continue;
+                    const int nk = min(ATTN_CHUNK, P + 1 - key0);
+                    const bf16_t* K = s.kv + (size_t)ia * 2 * kv_half +
+                                      (((int64_t)b * s.nkv + h / (s.nq / s.nkv)) * s.Lmax + key0) * s.hd;
+                    prefetch_l2_bulk(K, (uint32_t)nk * s.hd * 2);
+                    prefetch_l2_bulk(K + kv_half, (uint32_t)nk * s.hd * 2);
+                }
+            }
+            const bool live = (pid == 0) ? sk_bar_and(!*cta_abort) : sk_wait(s, cta_abort, seen, pid - 1);
             if (s.trace && blockIdx.x == 0 && tid == 0 && pid < SK_TRACE_SLOTS - 1) s.trace[pid] = globaltimer();
             // per-CTA phase times: wait done, prologue done, GEMV or items done, arrival
             unsigned long long* td = (s.tdetail && tid == 0 && blockIdx.x < SK_TRACE_CTAS)
@@ -860,12 +943,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                         break;
                     case SK_OUT_GDN: case SK_OUT_ATT: case SK_DOWN:
                         sk_gemv_consume<EPI_RESID>(s, p, ring, sm.xs, sm.pbuf, sm.cbuf, best, gs, vc, cta_abort,
-                                                   warp, lane, pid, td);
+                                                   warp, lane, pid, td, rpre);
                         break;
                     case SK_GDN:
                         for (int it = gw; it < n_gdn; it += nw) {
-                            if (it != gw) Sbase = sk_gdn_rows<KPL>(s, ig, it, S, lane);
-                            sk_gdn_item<KPL>(s, l, ig, it, S, Sbase, lane);
+                            if (it != gw) Sbase = sk_gdn_rows<KPL>(s, l, ig, it, S, gA, gdtb, lane);
+                            sk_gdn_item<KPL>(s, ig, it, S, Sbase, gA, gdtb, lane);
                         }
                         break;
                     case SK_PART: {
@@ -889,8 +972,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                             const bf16_t* K = s.kv + (size_t)ia * 2 * kv_half + ((int64_t)b * s.nkv + g) * s.Lmax * s.hd;
                             const float* q = s.qrot + (int64_t)row * s.nq * s.hd + (int64_t)h * s.hd;
                             float* dst = s.part + (((int64_t)row * s.nq + h) * s.max_chunks + ch) * (s.hd + 2);
-                            attn_partial_warp(q, K, K + kv_half, key0, min(ATTN_CHUNK, P + 1 - key0), s.hd, dst,
-                                              lane);
+                            attn_partial_warp_t<DPL>(q, K, K + kv_half, key0, min(ATTN_CHUNK, P + 1 - key0), dst,
+                                                     lane);
                             // the last of the row's chunks of this head merges them
                             const int nch = P / ATTN_CHUNK + 1;
                             unsigned* cnt = s.mcnt + row * s.nq + h;
@@ -904,8 +987,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                                 __threadfence();
                                 const float* base = s.part + ((int64_t)row * s.nq + h) * s.max_chunks * (s.hd + 2);
                                 const float* gate = s.proj + (int64_t)row * s.proj_ld + s.nq * s.hd + (int64_t)h * s.hd;
-                                sk_merge_head(base, nch, s.hd, gate, s.attn + (int64_t)row * s.nq * s.hd + (int64_t)h * s.hd,
-                                              lane);
+                                sk_merge_head_t<DPL>(base, nch, gate,
+                                                     s.attn + (int64_t)row * s.nq * s.hd + (int64_t)h * s.hd, lane);
                                 if (lane == 0) *cnt = 0u;  // ready for the next attention layer
                             }
                         }
