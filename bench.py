@@ -189,6 +189,26 @@ def cpu_baseline_sample(tokens: int = 4) -> dict:
             "sample": f"{tokens} greedy tokens of the full stack, single-threaded C oracle (fp64)"}
 
 
+# ---------------------------------------------------------------- replicas --
+
+def replica_reduce(vals: list, device: str) -> list:
+    """Max over the ranks of each value (device-timed milliseconds, end-to-end
+    seconds, status word): the job takes as long as its slowest replica, and an
+    error on any rank is the job's.  One all-reduce, which every rank issues at
+    the same point."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def aggregate_rate(world: int, units_per_rank: float, seconds: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed
+    `units_per_rank` units in at most `seconds`."""
+    return world * units_per_rank / seconds
+
+
 # --------------------------------------------------------------------- GPU --
 
 def run_gpu(args) -> None:
@@ -253,11 +273,6 @@ def run_gpu(args) -> None:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-    assert int(status.item()) == 0, hgd.status_string(int(status.item()))
 
     # end to end through the public API: host token in (pinned H2D), host argmax out
     e2e_steps = max(8, min(args.steps, 64))
@@ -270,17 +285,21 @@ def run_gpu(args) -> None:
         dec.step_host(h_tok, h_out)
         h_tok.view(-1).copy_(h_out)
     e2e_s = time.perf_counter() - t0
-    e2e_val = world * B * e2e_steps / e2e_s  # every rank runs the same loop
     dec.close()
+    st = int(status.item())
 
     if world > 1:
+        elapsed_ms, e2e_s, st_max = replica_reduce([elapsed_ms, e2e_s, st], "cuda")
+        st = int(st_max)
         dist.barrier()
         dist.destroy_process_group()
+    assert st == 0, hgd.status_string(st)
     if rank != 0:
         return
 
     ms_step = elapsed_ms / args.steps
-    value = world * B * args.steps / (elapsed_ms / 1000.0)
+    value = aggregate_rate(world, B * args.steps, elapsed_ms / 1000.0)
+    e2e_val = aggregate_rate(world, B * e2e_steps, e2e_s)  # every rank runs the same loop
     L_avg = PREFILL + args.warmup + (args.steps + 1) / 2.0
     ab = algorithmic_bytes(cfg, L_avg)
     peaks = measured_peaks()
