@@ -230,7 +230,9 @@ def run_gpu(args) -> None:
     if args.layers and args.layers != cfg["n_layers"]:
         cfg = dict(cfg, n_layers=args.layers)
     B = 1
-    Lmax = ((PREFILL + args.warmup + args.steps + 2 + 63) // 64) * 64
+    e2e_steps = max(8, min(args.steps, 64))
+    # cache positions for every token this run decodes: warm-up, timed and end-to-end steps
+    Lmax = ((PREFILL + args.warmup + args.steps + e2e_steps + 2 + 63) // 64) * 64
     model = hgd.Model(cfg, syn.stack_weights(cfg, seed=4))
     init = syn.stack_state(cfg, B, Lmax, prefill=PREFILL, seed=4 + rank)
     state = hgd.State(model, B, 1, Lmax, init)
@@ -275,7 +277,6 @@ def run_gpu(args) -> None:
     step_ms = [a.elapsed_time(b) for a, b in ev]
 
     # end to end through the public API: host token in (pinned H2D), host argmax out
-    e2e_steps = max(8, min(args.steps, 64))
     h_tok = torch.empty((B, 1), dtype=torch.int32).pin_memory()
     h_out = torch.empty((B,), dtype=torch.int32).pin_memory()
     h_tok.copy_(argmax.view(B, 1).cpu())
@@ -332,6 +333,8 @@ def run_gpu(args) -> None:
                      else "fallback",
                      "traffic": prof.get("k_stack_bytes_per_launch" if not split else "chain_bytes_per_step"),
                      "algorithmic_bytes": ab["total"], "avg_launch_ms": launch_ms},
+        "step_ms": {"median": float(np.median(step_ms)), "p90": float(np.percentile(step_ms, 90)),
+                    "p99": float(np.percentile(step_ms, 99)), "how": "CUDA events around each step's graph replay"},
         "gpu_launches": launches * args.steps,
         "path": "kernel chain" if split else "persistent",
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": 4 * B, "d2h_bytes_per_step": 4 * B,
@@ -345,10 +348,90 @@ def run_gpu(args) -> None:
     print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------------- standalone kernels --
+
+def run_kernels(args) -> None:
+    """Per-kernel rooflines of the standalone entry points at the GEMV sweep's
+    shapes (K = 1536 projections, fused up/gate, down, a 100000-row head; M = 1,
+    8, 32) and the GDN sweep's batches (B = 1, 4, 16, 64; 16 heads of 128).
+    Each call streams a different copy of its weights or state (copies totalling
+    more than twice the L2), timed with CUDA events; GB/s counts algorithmic
+    bytes.  One JSON line per kernel shape; these are not the benchmark line."""
+    import torch
+    import hybrid_gated_delta_b200 as hgd
+
+    peak = float(measured_peaks().get("hbm_gbs", 6650.0))
+    rot_bytes = 256 << 20  # > 2 x the 126 MB L2
+    gen = torch.Generator(device="cuda").manual_seed(2)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, ncopies, iters):
+        for i in range(3 * ncopies if ncopies < 8 else ncopies):
+            fn(i % ncopies)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(iters):
+            fn(i % ncopies)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3 / iters  # us per call
+
+    def line(kernel, shape, us, nbytes):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        print(json.dumps({"kernel": kernel, "shape": shape, "us": us, "algorithmic_bytes": nbytes, "gb_s": gbs,
+                          "frac_of_measured_peak": gbs / peak, "frac_of_8tbs": gbs / 8000.0,
+                          "note": "standalone kernel roofline, not the benchmark line"}), flush=True)
+
+    K = 1536
+    shapes = [("q/k/v/o", 1536, 1536, False), ("up+gate SwiGLU", 4096, 1536, True), ("down", 1536, 4096, False),
+              ("LM head", 100000, 1536, False)]
+    for name, N, KK, swi in shapes:
+        wbytes = (2 if swi else 1) * 2 * N * KK
+        ncopies = max(1, min(64, rot_bytes // wbytes))
+        Ws = [torch.randn(N, KK, device="cuda", generator=gen).mul_(KK ** -0.5).to(torch.bfloat16)
+              for _ in range(ncopies)]
+        Us = [torch.randn(N, KK, device="cuda", generator=gen).mul_(KK ** -0.5).to(torch.bfloat16)
+              for _ in range(ncopies)] if swi else None
+        for M in (1, 8, 32):
+            x = torch.randn(M, KK, device="cuda", generator=gen).to(torch.bfloat16)
+            ws = hgd.make_workspace(M, N, KK, swiglu=swi)
+            if swi:
+                h = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+                us = timed(lambda i: hgd.gemv_swiglu_bf16(Ws[i], Us[i], x, h=h, workspace=ws), ncopies, 200)
+                nbytes = 2 * 2 * N * KK + 2 * M * KK + 2 * M * N
+                line("hgd_gemv_swiglu_bf16 (k_gemv, SwiGLU epilogue)", {"M": M, "I": N, "K": KK}, us, nbytes)
+            else:
+                y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+                us = timed(lambda i: hgd.gemv_bf16(Ws[i], x, y=y, y_is_fp32=True, workspace=ws), ncopies,
+                           200 if N < 50000 else 50)
+                nbytes = 2 * N * KK + 2 * M * KK + 4 * M * N
+                line(f"hgd_gemv_bf16 (k_gemv) {name}", {"M": M, "N": N, "K": KK}, us, nbytes)
+        del Ws, Us
+        torch.cuda.empty_cache()
+
+    H, d = 16, 128
+    for B in (1, 4, 16, 64):
+        sbytes = B * H * d * d * 4
+        ncopies = max(4, min(256, rot_bytes // sbytes))
+        Ss = [torch.randn(B, H, d, d, device="cuda", generator=gen).mul_(0.1) for _ in range(ncopies)]
+        q = torch.randn(B, 1, H, d, device="cuda", generator=gen)
+        k = torch.randn(B, 1, H, d, device="cuda", generator=gen)
+        v = torch.randn(B, 1, H, d, device="cuda", generator=gen)
+        g = -torch.nn.functional.softplus(torch.randn(B, 1, H, device="cuda", generator=gen))
+        bb = torch.randn(B, 1, H, device="cuda", generator=gen)
+        o = torch.empty(B, 1, H, d, device="cuda")
+        us = timed(lambda i: hgd.gdn_decode_step(q, k, v, g, bb, Ss[i], o=o), ncopies, 400)
+        nbytes = 2 * sbytes + 4 * B * H * d * 4 + 2 * B * H * 4
+        line("hgd_gdn_decode_step (k_gdn_step)", {"B": B, "H": H, "dk": d, "dv": d, "T": 1}, us, nbytes)
+        del Ss
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -359,11 +442,16 @@ def main():
                     help="chain: one kernel per op, PDL-overlapped, in CUDA graphs; "
                          "persistent: the whole step in one cooperative launch")
     ap.add_argument("--cpu-tokens", type=int, default=4)
+    ap.add_argument("--kernels", action="store_true",
+                    help="instead of the benchmark line: per-kernel rooflines of the standalone GEMV and GDN "
+                         "entry points at the sweep shapes")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.kernels:
+        run_kernels(args)
     else:
         run_gpu(args)
 

@@ -952,6 +952,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                         }
                         break;
                     case SK_PART: {
+                        // partials per (row, head, 32-key chunk), one warp each; the last
+                        // chunk of a (row, head) to finish queues its merge, which the whole
+                        // CTA then runs with one dim per thread
+                        volatile int* mlist = reinterpret_cast<volatile int*>(sm.ex);  // count, (row*nq+h, nch)...
+                        const int mcap = (SK_CW * 32 - 1) / 2;
+                        if (tid == 0) mlist[0] = 0;
+                        named_bar(1, SK_CT);
                         const int n = s.M * s.nq * s.max_chunks;
                         const size_t kv_half = (size_t)s.B * s.nkv * s.Lmax * s.hd;
                         const int group = s.nq / s.nkv;
@@ -974,23 +981,53 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                             float* dst = s.part + (((int64_t)row * s.nq + h) * s.max_chunks + ch) * (s.hd + 2);
                             attn_partial_warp_t<DPL>(q, K, K + kv_half, key0, min(ATTN_CHUNK, P + 1 - key0), dst,
                                                      lane);
-                            // the last of the row's chunks of this head merges them
                             const int nch = P / ATTN_CHUNK + 1;
-                            unsigned* cnt = s.mcnt + row * s.nq + h;
-                            unsigned old = 0;
+                            int k = -1;  // this warp's place in the merge queue, or -1
                             if (lane == 0) {
                                 __threadfence();
-                                old = atomicAdd(cnt, 1u);
+                                const unsigned old = atomicAdd(s.mcnt + row * s.nq + h, 1u);
+                                if (old == (unsigned)nch - 1u) {
+                                    __threadfence();  // the other chunks' partials are visible from here on
+                                    k = atomicAdd(const_cast<int*>(mlist), 1);
+                                    if (k < mcap) {
+                                        mlist[1 + 2 * k] = row * s.nq + h;
+                                        mlist[2 + 2 * k] = nch;
+                                    }
+                                }
                             }
-                            old = __shfl_sync(0xffffffffu, old, 0);
-                            if (old == (unsigned)nch - 1u) {
-                                __threadfence();
+                            k = __shfl_sync(0xffffffffu, k, 0);
+                            if (k >= mcap) {  // queue full: this warp merges the head itself
                                 const float* base = s.part + ((int64_t)row * s.nq + h) * s.max_chunks * (s.hd + 2);
                                 const float* gate = s.proj + (int64_t)row * s.proj_ld + s.nq * s.hd + (int64_t)h * s.hd;
                                 sk_merge_head_t<DPL>(base, nch, gate,
                                                      s.attn + (int64_t)row * s.nq * s.hd + (int64_t)h * s.hd, lane);
-                                if (lane == 0) *cnt = 0u;  // ready for the next attention layer
+                                if (lane == 0) s.mcnt[row * s.nq + h] = 0u;
                             }
+                        }
+                        named_bar(1, SK_CT);
+                        const int nm = min((int)mlist[0], mcap);
+                        for (int e = 0; e < nm; ++e) {
+                            const int rh = mlist[1 + 2 * e], nch = mlist[2 + 2 * e];
+                            const int row = rh / s.nq, h = rh % s.nq, hd = s.hd;
+                            const float* base = s.part + (int64_t)rh * s.max_chunks * (hd + 2);
+                            const float* gate = s.proj + (int64_t)row * s.proj_ld + s.nq * hd + (int64_t)h * hd;
+                            bf16_t* out = s.attn + (int64_t)row * s.nq * hd + (int64_t)h * hd;
+                            for (int d = tid; d < hd; d += SK_CT) {
+                                // the arithmetic of attn_merge_dim for dim d
+                                float Mx = -INFINITY;
+#pragma unroll 8
+                                for (int c = 0; c < nch; ++c) Mx = fmaxf(Mx, __ldcg(base + (int64_t)c * (hd + 2)));
+                                float L = 0.f, acc = 0.f;
+#pragma unroll 8
+                                for (int c = 0; c < nch; ++c) {
+                                    const float* pc = base + (int64_t)c * (hd + 2);
+                                    const float w = expf(__ldcg(pc) - Mx);
+                                    L = fmaf(w, __ldcg(pc + 1), L);
+                                    acc = fmaf(w, __ldcg(pc + 2 + d), acc);
+                                }
+                                out[d] = f2bf(acc / L * sigmoid_f(gate[d]));
+                            }
+                            if (tid == 0) s.mcnt[rh] = 0u;  // ready for the next attention layer
                         }
                         break;
                     }
