@@ -862,12 +862,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
             float gA = 0.f, gdtb = 0.f, rpre[4] = {0.f, 0.f, 0.f, 0.f};
             const int gw = warp * G + blockIdx.x, nw = G * SK_CW;
             const int n_gdn = s.B * s.H * (s.dv / GDN_RPW);
+            // (gains go to shared memory asynchronously; the prologue waits for them)
             if (nmine > 0 && (kind == SK_IN_GDN || kind == SK_IN_ATT || kind == SK_SWIGLU || kind == SK_HEAD)) {
-                for (int c = tid; c < s.D / 8; c += SK_CT)
-                    *reinterpret_cast<uint4*>(sm.gb + c * 8) = *reinterpret_cast<const uint4*>(p.norm_w + c * 8);
+                for (int c = tid; c < s.D / 8; c += SK_CT) cp_async16(sm.gb + c * 8, p.norm_w + c * 8);
             } else if (nmine > 0 && kind == SK_OUT_GDN) {
-                for (int c = tid; c < s.dv / 8; c += SK_CT)
-                    *reinterpret_cast<uint4*>(sm.gb + c * 8) = *reinterpret_cast<const uint4*>(p.gnorm_w + c * 8);
+                for (int c = tid; c < s.dv / 8; c += SK_CT) cp_async16(sm.gb + c * 8, p.gnorm_w + c * 8);
             } else if (kind == SK_GDN && gw < n_gdn) {
                 Sbase = sk_gdn_rows<KPL>(s, l, ig, gw, S, gA, gdtb, lane);
             }
@@ -912,11 +911,16 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                     case SK_IN_GDN: case SK_IN_ATT: case SK_SWIGLU: case SK_HEAD: {
                         if (kind != SK_SWIGLU && l == 0) sk_pro_embed(s, sm.xs);
                         else sk_pro_resid(s, sm.xs);
+                        cp_async_wait_all();
                         named_bar(1, SK_CT);
                         sk_pro_rmsnorm(s, sm.xs, sm.gb, warp, lane);
                         break;
                     }
-                    case SK_OUT_GDN: sk_pro_gated(s, p, sm.gb, sm.xs, warp, lane); break;
+                    case SK_OUT_GDN:
+                        cp_async_wait_all();
+                        named_bar(1, SK_CT);
+                        sk_pro_gated(s, p, sm.gb, sm.xs, warp, lane);
+                        break;
                     case SK_OUT_ATT: sk_pro_copy(s, s.attn, s.nq * s.hd, sm.xs); break;
                     case SK_DOWN: sk_pro_copy(s, s.mlp, s.I, sm.xs); break;
                     default: break;
@@ -1038,6 +1042,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                 gs += nmine * p.nks;
             }
             if (td) td[2] = globaltimer();
+            cp_async_wait_all();  // (a gains copy of a skipped phase lands before the slot is reused)
             sk_arrive(s, pid);
             if (td) td[3] = globaltimer();
         }
