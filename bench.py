@@ -428,6 +428,52 @@ def run_kernels(args) -> None:
         torch.cuda.empty_cache()
 
 
+def run_windows(args) -> None:
+    """Throughput of the window workload: 8 streams x 16 rows per decode call
+    (128 token rows through the 24-layer stack, the kernel chain's path for more
+    than 8 rows), replayed from a CUDA graph; 16 windows per stream after the
+    512-key prefill.  Not the benchmark line."""
+    import torch
+    import hgd_synth as syn
+    import hybrid_gated_delta_b200 as hgd
+
+    cfg = syn.STACK_CFG
+    B, T, n_win, warm = 8, 16, 16, 2
+    Lmax = ((PREFILL + (n_win + warm + 1) * T + 63) // 64) * 64
+    model = hgd.Model(cfg, syn.stack_weights(cfg, seed=5))
+    state = hgd.State(model, B, T, Lmax, syn.stack_state(cfg, B, Lmax, prefill=PREFILL, seed=5))
+    toks = torch.from_numpy(syn.stack_tokens(cfg, B, T, seed=5)).cuda()
+    am = torch.zeros(B * T, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        hgd.decode_layer_stack(model, state, toks, T, argmax=am, status=status, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        hgd.decode_layer_stack(model, state, toks, T, argmax=am, status=status)
+    for _ in range(warm):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(n_win - warm - 1):
+            g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, hgd.status_string(int(status.item()))
+    n = n_win - warm - 1
+    ms = a.elapsed_time(b) / n
+    ab = algorithmic_bytes(cfg, PREFILL + (warm + 1 + n / 2.0) * T)
+    nbytes = ab["weights"] + B * (ab["total"] - ab["weights"])  # weights once, state and cache per stream
+    print(json.dumps({"workload": "8 streams x 16-row windows (128 token rows per call), 24-layer stack",
+                      "calls": n, "ms_per_call": ms, "tokens_per_s": B * T / (ms * 1e-3),
+                      "algorithmic_bytes_per_call": nbytes, "gb_s": nbytes / (ms * 1e-3) / 1e9,
+                      "launches_per_call": model.launches(B, T),
+                      "note": "window throughput, not the benchmark line"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -442,6 +488,8 @@ def main():
                     help="chain: one kernel per op, PDL-overlapped, in CUDA graphs; "
                          "persistent: the whole step in one cooperative launch")
     ap.add_argument("--cpu-tokens", type=int, default=4)
+    ap.add_argument("--windows", action="store_true",
+                    help="instead of the benchmark line: throughput of 8 streams x 16-row windows")
     ap.add_argument("--kernels", action="store_true",
                     help="instead of the benchmark line: per-kernel rooflines of the standalone GEMV and GDN "
                          "entry points at the sweep shapes")
@@ -452,6 +500,8 @@ def main():
         run_reference(args)
     elif args.kernels:
         run_kernels(args)
+    elif args.windows:
+        run_windows(args)
     else:
         run_gpu(args)
 

@@ -330,13 +330,16 @@ __device__ __forceinline__ void gv_finish(const GemvParams& p, int rb, int s_ite
             finish = (old == p.nks - 1);
             if (finish) {
                 __threadfence();
+                // partials in slab order; L2-only loads the compiler may issue ahead
+#pragma unroll 4
                 for (int j = 0; j < p.nks; ++j) {
                     const float* pp = p.ws_part + ((int64_t)(rb * p.nks + j) * GV_ROWS) * p.ws_mp;
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
                         const int n0 = nt * 8 + 2 * c;
-                        const float v0 = ld_cg(pp + r8 * p.ws_mp + n0), v1 = ld_cg(pp + r8 * p.ws_mp + n0 + 1);
-                        const float v2 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0), v3 = ld_cg(pp + (r8 + 8) * p.ws_mp + n0 + 1);
+                        const float2 lo = __ldcg(reinterpret_cast<const float2*>(pp + r8 * p.ws_mp + n0));
+                        const float2 hi = __ldcg(reinterpret_cast<const float2*>(pp + (r8 + 8) * p.ws_mp + n0));
+                        const float v0 = lo.x, v1 = lo.y, v2 = hi.x, v3 = hi.y;
                         if (j == 0) { yacc[nt][0] = v0; yacc[nt][1] = v1; yacc[nt][2] = v2; yacc[nt][3] = v3; }
                         else { yacc[nt][0] += v0; yacc[nt][1] += v1; yacc[nt][2] += v2; yacc[nt][3] += v3; }
                     }

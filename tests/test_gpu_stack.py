@@ -337,15 +337,21 @@ def _run_paths(hgd, model, cfg, B, T, Lmax, steps, seed):
     return outs
 
 
-@pytest.mark.parametrize("which", ["small", "full"])
+@pytest.mark.parametrize("which", ["small", "full", "full_b8", "full_b2t4"])
 def test_persistent_launch_equals_kernel_chain(hgd, full, which):
     """One cooperative launch per call equals the chain of per-phase kernels bit
-    for bit: logits, argmax, per-row state and conv-tail records, final state."""
+    for bit: logits, argmax, per-row state and conv-tail records, final state.
+    At full size: one row; 8 streams of one row and 2 streams of 4-row windows
+    (8 token rows: the launch's largest, with its smaller weight ring)."""
     import torch
     if which == "small":
         cfg, model, B, T, Lmax = syn.SMALL_CFG, hgd.Model(syn.SMALL_CFG, weights("small", 5)), 2, 3, 40
-    else:
+    elif which == "full":
         cfg, model, B, T, Lmax = syn.STACK_CFG, full[0], 1, 1, 640
+    elif which == "full_b8":
+        cfg, model, B, T, Lmax = syn.STACK_CFG, full[0], 8, 1, 640
+    else:
+        cfg, model, B, T, Lmax = syn.STACK_CFG, full[0], 2, 4, 640
     assert model.launches(B, T) == 1
     (rp, sp), (rc, sc) = _run_paths(hgd, model, cfg, B, T, Lmax, 3, 13)
     for k, ((l1, a1, s1, t1), (l2, a2, s2, t2)) in enumerate(zip(rp, rc)):
