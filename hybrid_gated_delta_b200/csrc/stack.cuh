@@ -244,6 +244,21 @@ __device__ __forceinline__ void sk_gemv_params(const SkParams& s, int kind, int 
     p.n_items = p.n_rowblk;
 }
 
+// The norm gains the prologue of phase `kind` of layer l reads (the RMSNorm
+// before the in-projections, the SwiGLU and the LM head; the gated norm before
+// the GDN out-projection), or null; n: their count.
+__device__ __forceinline__ const bf16_t* sk_gains(const SkParams& s, int kind, int l, int& n) {
+    n = s.D;
+    switch (kind) {
+        case SK_IN_GDN: case SK_IN_ATT: return s.layer[l].w[HGD_W_IN_NORM];
+        case SK_SWIGLU: return s.layer[l].w[HGD_W_POST_NORM];
+        case SK_HEAD: return s.final_norm;
+        case SK_OUT_GDN: n = s.dv; return s.layer[l].w[HGD_W_GNORM];
+        default: n = 0; return nullptr;
+    }
+}
+
+
 // This CTA's place in phase `pid`'s item order (a rotation that moves from
 // phase to phase), and its items c, c + G, c + 2G, ... of n.
 __device__ __forceinline__ int sk_vcta(int pid) {
@@ -716,14 +731,14 @@ __device__ void sk_final(const SkParams& s, int lane) {
 // partial buffer [pb][16][8] f32 | conv scratch [8][16][8] f32 | argmax [8][8] x2 |
 // attention scratch [8][32] f32 | full[ns], empty[ns] mbarriers | flags.
 struct SkSmem {
-    uint8_t* ring; bf16_t* xs; bf16_t* gb; float* pbuf; float* cbuf; float* amax_v; int* amax_i; float* ex;
+    uint8_t* ring; bf16_t* xs; bf16_t* gb[2]; float* pbuf; float* cbuf; float* amax_v; int* amax_i; float* ex;
     uint64_t* full; uint64_t* empty; volatile int* flags;
 };
 
 __host__ __device__ inline size_t sk_al128(size_t v) { return (v + 127) & ~(size_t)127; }
 __host__ __device__ inline size_t sk_xs_bytes(int M, int kmax) { return sk_al128((size_t)M * (kmax + GV_PAD) * 2); }
 __host__ __device__ inline size_t sk_fixed_bytes(int M, int kmax, int D, int pb, int ns) {
-    return sk_xs_bytes(M, kmax) + sk_al128((size_t)D * 2) + (size_t)pb * SK_PB_SLAB * 4 +
+    return sk_xs_bytes(M, kmax) + 2 * sk_al128((size_t)D * 2) + (size_t)pb * SK_PB_SLAB * 4 +
            (size_t)SK_CW * GV_ROWS * 8 * 4 + (size_t)SK_CW * 8 * 8 + (size_t)SK_CW * 32 * 4 + (size_t)ns * 16 + 64;
 }
 
@@ -732,7 +747,8 @@ __device__ __forceinline__ SkSmem sk_smem(const SkParams& s, uint8_t* base) {
     size_t o = 0;
     m.ring = base; o += (size_t)s.ns * SK_SLAB_BYTES;
     m.xs = reinterpret_cast<bf16_t*>(base + o); o += sk_xs_bytes(s.M, s.kmax);
-    m.gb = reinterpret_cast<bf16_t*>(base + o); o += sk_al128((size_t)s.D * 2);
+    m.gb[0] = reinterpret_cast<bf16_t*>(base + o); o += sk_al128((size_t)s.D * 2);
+    m.gb[1] = reinterpret_cast<bf16_t*>(base + o); o += sk_al128((size_t)s.D * 2);
     m.pbuf = reinterpret_cast<float*>(base + o); o += (size_t)s.pb * SK_PB_SLAB * 4;
     m.cbuf = reinterpret_cast<float*>(base + o); o += (size_t)SK_CW * GV_ROWS * 8 * 4;
     m.amax_v = reinterpret_cast<float*>(base + o); o += SK_CW * 8 * 4;
@@ -742,6 +758,20 @@ __device__ __forceinline__ SkSmem sk_smem(const SkParams& s, uint8_t* base) {
     m.empty = reinterpret_cast<uint64_t*>(base + o); o += (size_t)s.ns * 8;
     m.flags = reinterpret_cast<volatile int*>(base + o);
     return m;
+}
+
+// Gains of phase pid (layer l, phase j of the layer) into gains buffer pid & 1,
+// by cp.async, as one committed group (empty if the phase reads none): each
+// phase's gains are issued one phase ahead, so they land while the phase
+// before runs.
+__device__ __forceinline__ void sk_issue_gains(const SkParams& s, const SkSmem& sm, int pid, int l, int j, int tid) {
+    if (l <= s.L && j < ((l == s.L) ? 2 : SK_PHASES_PER_LAYER)) {
+        int n = 0;
+        const bf16_t* g = sk_gains(s, sk_kind(s, l, j), l, n);
+        if (g)
+            for (int c = tid; c < n / 8; c += SK_CT) cp_async16(((pid & 1) ? sm.gb[1] : sm.gb[0]) + c * 8, g + c * 8);
+    }
+    cp_async_commit();
 }
 
 // KPL: GDN key elements per lane (dk / 32); DPL: attention dims per lane (hd / 32).
@@ -836,6 +866,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
     int ig = 0, ia = 0, pid = -1;
     GvBest<1> best;
     best.init();
+    sk_issue_gains(s, sm, 0, 0, 0, tid);
     for (int l = 0; l <= s.L; ++l) {
         const int nph = (l == s.L) ? 2 : SK_PHASES_PER_LAYER;
         for (int j = 0; j < nph; ++j) {
@@ -862,12 +893,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
             float gA = 0.f, gdtb = 0.f, rpre[4] = {0.f, 0.f, 0.f, 0.f};
             const int gw = warp * G + blockIdx.x, nw = G * SK_CW;
             const int n_gdn = s.B * s.H * (s.dv / GDN_RPW);
-            // (gains go to shared memory asynchronously; the prologue waits for them)
-            if (nmine > 0 && (kind == SK_IN_GDN || kind == SK_IN_ATT || kind == SK_SWIGLU || kind == SK_HEAD)) {
-                for (int c = tid; c < s.D / 8; c += SK_CT) cp_async16(sm.gb + c * 8, p.norm_w + c * 8);
-            } else if (nmine > 0 && kind == SK_OUT_GDN) {
-                for (int c = tid; c < s.dv / 8; c += SK_CT) cp_async16(sm.gb + c * 8, p.gnorm_w + c * 8);
-            } else if (kind == SK_GDN && gw < n_gdn) {
+            // the next phase's gains go to shared memory asynchronously (this
+            // phase's were issued one phase ago; the prologue waits for them)
+            if (j + 1 < nph) sk_issue_gains(s, sm, pid + 1, l, j + 1, tid);
+            else sk_issue_gains(s, sm, pid + 1, l + 1, 0, tid);
+            if (kind == SK_GDN && gw < n_gdn) {
                 Sbase = sk_gdn_rows<KPL>(s, l, ig, gw, S, gA, gdtb, lane);
             }
             if (nmine > 0 && (kind == SK_OUT_GDN || kind == SK_OUT_ATT || kind == SK_DOWN)) {
@@ -911,15 +941,15 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                     case SK_IN_GDN: case SK_IN_ATT: case SK_SWIGLU: case SK_HEAD: {
                         if (kind != SK_SWIGLU && l == 0) sk_pro_embed(s, sm.xs);
                         else sk_pro_resid(s, sm.xs);
-                        cp_async_wait_all();
+                        cp_async_wait_prior();
                         named_bar(1, SK_CT);
-                        sk_pro_rmsnorm(s, sm.xs, sm.gb, warp, lane);
+                        sk_pro_rmsnorm(s, sm.xs, (pid & 1) ? sm.gb[1] : sm.gb[0], warp, lane);
                         break;
                     }
                     case SK_OUT_GDN:
-                        cp_async_wait_all();
+                        cp_async_wait_prior();
                         named_bar(1, SK_CT);
-                        sk_pro_gated(s, p, sm.gb, sm.xs, warp, lane);
+                        sk_pro_gated(s, p, (pid & 1) ? sm.gb[1] : sm.gb[0], sm.xs, warp, lane);
                         break;
                     case SK_OUT_ATT: sk_pro_copy(s, s.attn, s.nq * s.hd, sm.xs); break;
                     case SK_DOWN: sk_pro_copy(s, s.mlp, s.I, sm.xs); break;
@@ -1042,7 +1072,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
                 gs += nmine * p.nks;
             }
             if (td) td[2] = globaltimer();
-            cp_async_wait_all();  // (a gains copy of a skipped phase lands before the slot is reused)
+            // this phase's gains have landed even where the phase read none, so the
+            // buffer takes the copy issued two phases on (the next phase's may fly)
+            cp_async_wait_prior();
             sk_arrive(s, pid);
             if (td) td[3] = globaltimer();
         }
