@@ -68,6 +68,10 @@ _SIGS = {
     "hgd_gemv_workspace_bytes": ([_i, _i, _i, _i, C.POINTER(_sz)], _i),
     "hgd_gemv_bf16_static_ws": ([_p, _p, _p, _i, _i, _i, _i, _p], _i),
     "hgd_gemv_swiglu_bf16": ([_p, _p, _p, _p, _i, _i, _i, _p, _sz, _p], _i),
+    "hgd_gemm_tc_weight_bytes": ([_i, _i, C.POINTER(_sz)], _i),
+    "hgd_gemm_tc_pack_weight": ([_p, _p, _i, _i, _p], _i),
+    "hgd_gemm_tc_workspace_bytes": ([_i, _i, _i, C.POINTER(_sz)], _i),
+    "hgd_gemm_tc_bf16": ([_p, _p, _p, _i, _i, _i, _p, _sz, _p, _p], _i),
     "hgd_conv1d_tail_update": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
     "hgd_model_arena_bytes": ([C.POINTER(Config), C.POINTER(_sz)], _i),
@@ -162,6 +166,39 @@ def gemv_bf16(W, x, y=None, y_is_fp32=True, workspace=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("hgd_gemv_bf16", _lib.hgd_gemv_bf16(_ptr(W), _ptr(x), _ptr(y), int(y.dtype == torch.float32),
                                                 M, N, K, _ptr(workspace), ws_bytes, _stream(stream)))
+    return y
+
+
+def gemm_tc_pack_weight(W, stream=None):
+    """W [N,K] bf16 -> the tensor-core GEMM's packed weight (uint8 device tensor)."""
+    torch = _torch()
+    _need(W, torch.bfloat16, "W")
+    N, K = W.shape
+    n = C.c_size_t()
+    _check("hgd_gemm_tc_weight_bytes", _lib.hgd_gemm_tc_weight_bytes(N, K, C.byref(n)))
+    Wp = torch.empty(n.value, dtype=torch.uint8, device=W.device)
+    _check("hgd_gemm_tc_pack_weight", _lib.hgd_gemm_tc_pack_weight(_ptr(W), _ptr(Wp), N, K, _stream(stream)))
+    return Wp
+
+
+def gemm_tc_workspace_bytes(M: int, N: int, K: int) -> int:
+    n = C.c_size_t()
+    _check("hgd_gemm_tc_workspace_bytes", _lib.hgd_gemm_tc_workspace_bytes(M, N, K, C.byref(n)))
+    return n.value
+
+
+def gemm_tc_bf16(Wp, x, N, y=None, workspace=None, status=None, stream=None):
+    """y[M,N] fp32 = x[M,K] . W[N,K]^T on the tensor cores; Wp from gemm_tc_pack_weight."""
+    torch = _torch()
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(gemm_tc_workspace_bytes(M, N, K), dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("hgd_gemm_tc_bf16", _lib.hgd_gemm_tc_bf16(_ptr(Wp), _ptr(x), _ptr(y), M, N, K, _ptr(workspace),
+                                                      ws_bytes, _ptr(status), _stream(stream)))
     return y
 
 

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "gdn.cuh"
 #include "gemv.cuh"
+#include "gemm_tc.cuh"
 #include "stack.cuh"
 
 using namespace hgd;
@@ -457,6 +458,65 @@ int sk_launch(const Dims& d, const SkParams& prm, size_t smem, int sms, cudaStre
     }
 }
 
+// ------------------------------------------------------- tensor-core GEMM plan
+// A fixed function of (M, N, K): token rows padded to the MMA's N, 128-row
+// weight tiles, a split of the K blocks that brings the CTA count near one wave
+// (it depends on N and K only), as many shared-memory stages as fit.
+struct TcPlan {
+    int NTp, n_blocks, kb_per_split, splits, stages;
+    uint32_t tmem_cols;
+    size_t xp_bytes, part_bytes;
+};
+TcPlan tc_plan(int M, int N, int K) {
+    TcPlan q{};
+    q.NTp = tc_ntp(M);
+    q.n_blocks = tc_nblocks(N);
+    const int nkb = K / TC_BK;
+    const int want = std::max(1, std::min(nkb, TC_TARGET_CTAS / q.n_blocks));
+    q.kb_per_split = (nkb + want - 1) / want;
+    q.splits = (nkb + q.kb_per_split - 1) / q.kb_per_split;
+    const size_t avail = (size_t)GV_SMEM_LIMIT - tc_smem_bytes(q.NTp, 0);
+    q.stages = (int)std::min<size_t>(TC_MAX_STAGES, avail / tc_stage_bytes(q.NTp));
+    uint32_t c = 32;
+    while ((int)c < q.NTp) c <<= 1;
+    q.tmem_cols = c;
+    q.xp_bytes = ((size_t)q.NTp * K * 2 + 255) / 256 * 256;
+    q.part_bytes = q.splits > 1 ? (size_t)q.splits * M * N * 4 : 0;
+    return q;
+}
+bool tc_shape_ok(int M, int N, int K) { return M >= 1 && M <= TC_MAXN && N >= 1 && K >= TC_BK && K % TC_BK == 0 && K <= 65536; }
+
+int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int N, int K, void* ws,
+           int32_t* status, cudaStream_t s) {
+    const TcPlan q = tc_plan(M, N, K);
+    static int attr_done[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        if (cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return HGD_ERR_CUDA;
+        }
+        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    }
+    bf16_t* Xp = static_cast<bf16_t*>(ws);
+    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + q.xp_bytes);
+    const int chunks = q.NTp * (K / 8);
+    cudaError_t e = launch_pdl(k_tc_pack_x, dim3(std::min(1184, (chunks + 255) / 256)), dim3(256), 0, s, x, x_ld, Xp,
+                               M, K, q.NTp);
+    if (e != cudaSuccess) return launch_status(e);
+    TcParams prm{};
+    prm.Wp = Wp; prm.Xp = Xp; prm.out = q.splits > 1 ? part : y; prm.status = status;
+    prm.M = M; prm.N = N; prm.K = K; prm.NTp = q.NTp; prm.ldo = N;
+    prm.n_blocks = q.n_blocks; prm.kb_per_split = q.kb_per_split; prm.stages = q.stages; prm.tmem_cols = q.tmem_cols;
+    e = launch_pdl(k_gemm_tc, dim3(q.n_blocks * q.splits), dim3(TC_THREADS), tc_smem_bytes(q.NTp, q.stages), s, prm);
+    if (e != cudaSuccess || q.splits == 1) return launch_status(e);
+    const int64_t n = (int64_t)M * N;
+    return launch_status(launch_pdl(k_tc_reduce, dim3((unsigned)std::min<int64_t>(1184, (n + 255) / 256)), dim3(256),
+                                    0, s, (const float*)part, y, q.splits, n));
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -514,6 +574,47 @@ int hgd_gemv_swiglu_bf16(const uint16_t* W_gate, const uint16_t* W_up, const uin
     GemvParams p = {};
     p.W = W_gate; p.W2 = W_up; p.N = I; p.K = K; p.x = x; p.x_ld = K; p.y = h; p.y_ld = I;
     return run_gemv<PRO_COPY, EPI_SWIGLU>(p, M, di.sms, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+int hgd_gemm_tc_weight_bytes(int N, int K, size_t* bytes) {
+    if (!bytes || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (!tc_shape_ok(1, N, K)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    *bytes = (size_t)tc_nblocks(N) * TC_BM * K * 2;
+    return HGD_OK;
+}
+
+int hgd_gemm_tc_pack_weight(const uint16_t* W, uint16_t* Wp, int N, int K, hgd_stream_t stream) {
+    if (!W || !Wp || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (!tc_shape_ok(1, N, K)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(W) || !al16(Wp)) return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    const int64_t chunks = (int64_t)tc_nblocks(N) * TC_BM * (K / 8);
+    k_tc_pack_w<<<(unsigned)std::min<int64_t>(4736, (chunks + 255) / 256), 256, 0, (cudaStream_t)stream>>>(W, Wp, N, K);
+    return launch_status(cudaGetLastError());
+}
+
+int hgd_gemm_tc_workspace_bytes(int M, int N, int K, size_t* bytes) {
+    if (!bytes || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (!tc_shape_ok(M, N, K)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    const TcPlan q = tc_plan(M, N, K);
+    *bytes = q.xp_bytes + q.part_bytes;
+    return HGD_OK;
+}
+
+int hgd_gemm_tc_bf16(const uint16_t* Wp, const uint16_t* x, float* y, int M, int N, int K, void* workspace,
+                     size_t workspace_bytes, int32_t* status, hgd_stream_t stream) {
+    if (!Wp || !x || !y || !workspace || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (!tc_shape_ok(M, N, K)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(Wp) || !al16(x) || !al16(y) || !al16(workspace)) return HGD_ERR_MISALIGNED;
+    const TcPlan q = tc_plan(M, N, K);
+    if (workspace_bytes < q.xp_bytes + q.part_bytes) return HGD_ERR_BUFFER_TOO_SMALL;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    return tc_run(reinterpret_cast<const bf16_t*>(Wp), reinterpret_cast<const bf16_t*>(x), K, y, M, N, K, workspace,
+                  status, (cudaStream_t)stream);
 }
 
 int hgd_conv1d_tail_update(const float* x, float* tail, const uint16_t* w, float* y, float* tail_rec,

@@ -1,0 +1,268 @@
+// Tensor-core GEMM for windows of token rows (tcgen05, sm_100a):
+//
+//   Y[t][n] = sum_k X[t][k] * W[n][k]     t < M <= 256 token rows, fp32 sums
+//
+// The decode-step projections of the hybrid stack (Qwen3.5-style gated-delta /
+// gated-attention decoder; the projection GEMVs of the decode step) become real
+// GEMMs once a call carries a window of many token rows: at 128 rows a weight
+// byte feeds 128 multiply-adds, which the legacy mma.sync path cannot sustain.
+// Here one CTA owns a 128-row block of W (the MMA's M), takes every token row
+// of the call as the MMA's N (16..256), and streams its K range through a ring
+// of shared-memory stages:
+//   - one lane issues the bulk copies (cp.async.bulk, no multicast) of a
+//     stage's weight tile (128 x 64, 16 KB) and token tile (NTp x 64),
+//     completing on the stage's `full` mbarrier;
+//   - one lane issues four tcgen05.mma (K = 16 each) per stage into a TMEM
+//     accumulator of 128 lanes x NTp fp32 columns, and tcgen05.commit frees the
+//     stage (`empty`) once they complete;
+//   - after the last stage, the four warps read the accumulator back with
+//     tcgen05.ld (warp w owns TMEM lanes 32w..32w+31 = W rows) and write fp32.
+// Operands are packed once into the canonical no-swizzle K-major layout the
+// shared-memory descriptors describe: 8 x 8 core matrices (8 rows of 16 bytes,
+// 128 contiguous bytes), core (row group g, k group j) of a tile at byte
+// (g * 8 + j) * 128, so the leading-dimension (k) stride is 128 bytes and the
+// stride-dimension (8-row group) stride is 1024 bytes.  A fixed split of K over
+// CTAs (a function of N and K only) fills the SMs for short-N projections; its
+// partials are added in split order by a second kernel.
+//
+// Every wait is bounded (HGD_ERR_TIMEOUT in *status), the producer waits for
+// its copies before the CTA leaves, the issuer's final commit covers every MMA
+// it issued, and the TMEM columns are freed on every path.
+#pragma once
+#include "common.cuh"
+
+namespace hgd {
+
+constexpr int TC_BM = 128;                    // W rows per tile (the MMA's M)
+constexpr int TC_BK = 64;                     // K per stage (four MMAs of K = 16)
+constexpr int TC_MAXN = 256;                  // token rows per call (the MMA's N)
+constexpr int TC_THREADS = 128;
+constexpr int TC_WTILE = TC_BM * TC_BK;       // elements of a weight tile (16 KB)
+constexpr int TC_MAX_STAGES = 8;
+constexpr int TC_TARGET_CTAS = 148;           // split-K target: one wave of B200 SMs
+
+__host__ __device__ inline int tc_ntp(int M) { return M <= 16 ? 16 : (M + 15) / 16 * 16; }
+__host__ __device__ inline int tc_nblocks(int N) { return (N + TC_BM - 1) / TC_BM; }
+
+// Packed weight: tile (n / 128, k / 64) at tile index nb * (K / 64) + kb, each
+// tile in core-matrix order.  Element offset of W[n][k]:
+__host__ __device__ inline size_t tc_w_elem(int n, int k, int K) {
+    const int r = n & (TC_BM - 1), kk = k & (TC_BK - 1);
+    const size_t tile = (size_t)(n >> 7) * (K / TC_BK) + (k >> 6);
+    return tile * TC_WTILE + (size_t)(((r >> 3) * 8 + (kk >> 3)) * 64 + (r & 7) * 8 + (kk & 7));
+}
+// Packed token rows: for each k block a tile of NTp rows x 64 in the same core order.
+__host__ __device__ inline size_t tc_x_elem(int t, int k, int NTp) {
+    const int kk = k & (TC_BK - 1);
+    return (size_t)(k >> 6) * NTp * TC_BK + (size_t)(((t >> 3) * 8 + (kk >> 3)) * 64 + (t & 7) * 8 + (kk & 7));
+}
+
+// One 16-byte chunk (8 consecutive k) per thread: rows n >= N are zero.
+__global__ void k_tc_pack_w(const bf16_t* __restrict__ W, bf16_t* __restrict__ Wp, int N, int K) {
+    const int cpr = K / 8;
+    const int64_t total = (int64_t)tc_nblocks(N) * TC_BM * cpr;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int n = (int)(e / cpr), k = (int)(e % cpr) * 8;
+        const uint4 v = n < N ? *reinterpret_cast<const uint4*>(W + (int64_t)n * K + k) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(Wp + tc_w_elem(n, k, K)) = v;
+    }
+}
+__global__ void k_tc_pack_x(const bf16_t* __restrict__ X, int64_t x_ld, bf16_t* __restrict__ Xp, int M, int K,
+                            int NTp) {
+    pdl_launch();
+    pdl_wait();
+    const int cpr = K / 8;
+    const int total = NTp * cpr;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+        const int t = e / cpr, k = (e % cpr) * 8;
+        const uint4 v = t < M ? *reinterpret_cast<const uint4*>(X + (int64_t)t * x_ld + k) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(Xp + tc_x_elem(t, k, NTp)) = v;
+    }
+}
+
+// ------------------------------------------------------------- tcgen05 PTX
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Shared-memory matrix descriptor: no swizzle, K-major, start / leading (k) /
+// stride (8-row group) byte offsets in 16-byte units, descriptor version 1.
+__device__ __forceinline__ uint64_t tc_desc(const void* smem, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((smem_addr(smem) >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// Instruction descriptor of kind::f16: bf16 A and B, both K-major, fp32 D,
+// M = 128, N = n.
+__host__ __device__ inline uint32_t tc_idesc(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on `bar` once every MMA this thread issued before has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+struct TcParams {
+    const bf16_t* Wp;   // packed weight (tc_w_elem), N padded to 128-row tiles
+    const bf16_t* Xp;   // packed token rows (tc_x_elem), NTp rows
+    float* out;         // splits == 1: Y [M][ldo]; else partials [splits][M][ldo]
+    int32_t* status;    // optional: HGD_ERR_TIMEOUT if a wait ran out
+    int M, N, K, NTp, ldo;
+    int n_blocks, kb_per_split, stages;
+    uint32_t tmem_cols;
+};
+
+// Shared memory: stages x (weight tile 16 KB, token tile NTp x 128 B), then the
+// full / empty / done mbarriers, the TMEM address and the abort flag.
+__host__ __device__ inline size_t tc_stage_bytes(int NTp) { return (size_t)TC_WTILE * 2 + (size_t)NTp * TC_BK * 2; }
+__host__ __device__ inline size_t tc_smem_bytes(int NTp, int stages) {
+    return (size_t)stages * tc_stage_bytes(NTp) + (2 * TC_MAX_STAGES + 1) * 8 + 16;
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int S = p.stages;
+    const size_t sb = tc_stage_bytes(p.NTp);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * sb);
+    uint64_t* empty = full + TC_MAX_STAGES;
+    uint64_t* done = empty + TC_MAX_STAGES;
+    volatile uint32_t* tslot = reinterpret_cast<volatile uint32_t*>(done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1) + 1;
+    const int nb = blockIdx.x % p.n_blocks, sp = blockIdx.x / p.n_blocks;
+    const int nkb_all = p.K / TC_BK;
+    const int kb0 = sp * p.kb_per_split, nkb = min(nkb_all, kb0 + p.kb_per_split) - kb0;
+
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(const_cast<uint32_t*>(tslot))),
+                     "r"(p.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    pdl_launch();
+
+    if (warp == 0 && lane == 0) {
+        // producer: the first stages' weight tiles go out before the wait for the
+        // previous kernel on the stream (weights are never written by it), their
+        // token tiles after it; then stage by stage as the MMAs free them
+        const uint32_t xbytes = (uint32_t)p.NTp * TC_BK * 2, wbytes = (uint32_t)TC_WTILE * 2;
+        const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+        const int pre = min(S, nkb);
+        for (int i = 0; i < pre; ++i) {
+            mbar_arrive_expect_tx(&full[i], wbytes + xbytes);
+            bulk_g2s(smem + (size_t)i * sb, p.Wp + ((size_t)nb * nkb_all + kb0 + i) * TC_WTILE, wbytes, &full[i],
+                     pol_w);
+        }
+        pdl_wait();
+        for (int i = 0; i < pre; ++i)
+            bulk_g2s(smem + (size_t)i * sb + wbytes, p.Xp + (size_t)(kb0 + i) * p.NTp * TC_BK, xbytes, &full[i],
+                     pol_x);
+        int issued = pre;
+        bool ok = true;
+        for (int i = pre; i < nkb; ++i) {
+            const int st = i % S;
+            if (!mbar_wait_bounded(&empty[st], (uint32_t)(((i / S) & 1) ^ 1), abort_flag)) {
+                ok = false;
+                break;
+            }
+            mbar_arrive_expect_tx(&full[st], wbytes + xbytes);
+            uint8_t* dst = smem + (size_t)st * sb;
+            bulk_g2s(dst, p.Wp + ((size_t)nb * nkb_all + kb0 + i) * TC_WTILE, wbytes, &full[st], pol_w);
+            bulk_g2s(dst + wbytes, p.Xp + (size_t)(kb0 + i) * p.NTp * TC_BK, xbytes, &full[st], pol_x);
+            issued = i + 1;
+        }
+        if (!ok) {
+            if (p.status) set_status(p.status, HGD_ERR_TIMEOUT);
+            *abort_flag = 1;
+        }
+        // the copies still in flight land before this CTA's shared memory goes away
+        for (int q = max(0, issued - S); q < issued; ++q)
+            (void)mbar_wait_bounded(&full[q % S], (uint32_t)((q / S) & 1), nullptr);
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer
+        const uint32_t idesc = tc_idesc(p.NTp);
+        for (int i = 0; i < nkb; ++i) {
+            const int st = i % S;
+            if (!mbar_wait_bounded(&full[st], (uint32_t)((i / S) & 1), abort_flag)) {
+                if (p.status) set_status(p.status, HGD_ERR_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint8_t* a = smem + (size_t)st * sb;
+            const uint8_t* b = a + (size_t)TC_WTILE * 2;
+#pragma unroll
+            for (int s = 0; s < TC_BK / 16; ++s)
+                tc_mma(tmem, tc_desc(a + s * 256, 128, 1024), tc_desc(b + s * 256, 128, 1024), idesc,
+                       (i > 0 || s > 0) ? 1u : 0u);
+            tc_commit(&empty[st]);
+        }
+        tc_commit(done);  // covers every MMA issued above
+    }
+    __syncwarp();
+
+    // epilogue: warp w reads TMEM lanes 32w.. (W rows nb*128 + 32w + lane)
+    const bool got = mbar_wait_bounded(done, 0u, nullptr);
+    tc_fence_after();
+    if (!got && lane == 0 && p.status) set_status(p.status, HGD_ERR_TIMEOUT);
+    const bool live = __all_sync(0xffffffffu, got) && !*abort_flag && nkb > 0;
+    if (live) {
+        const int n = nb * TC_BM + warp * 32 + lane;
+        float* out = p.out + (size_t)sp * p.M * p.ldo;
+        for (int c0 = 0; c0 < p.NTp; c0 += 16) {
+            uint32_t v[16];
+            tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int t = c0 + j;
+                if (t < p.M && n < p.N) out[(size_t)t * p.ldo + n] = __uint_as_float(v[j]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols) : "memory");
+    }
+}
+
+// Y[t][n] = sum over splits, in split order, of the partials.
+__global__ void k_tc_reduce(const float* __restrict__ part, float* __restrict__ y, int splits, int64_t n_elem) {
+    pdl_launch();
+    pdl_wait();
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n_elem;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        float acc = part[e];
+        for (int s = 1; s < splits; ++s) acc += part[(int64_t)s * n_elem + e];
+        y[e] = acc;
+    }
+}
+
+}  // namespace hgd

@@ -99,6 +99,38 @@ HGD_API int hgd_gemv_bf16(const uint16_t* W, const uint16_t* x, void* y, int y_i
  * SwiGLU (swiglu = 1, N = I) of this shape; 0 when that shape never uses one. */
 HGD_API int hgd_gemv_workspace_bytes(int M, int N, int K, int swiglu, size_t* bytes);
 
+/* ------------------------------------------------------- tensor-core GEMM ---
+ * The same product for windows of many token rows ([TF] PR body: windows of up
+ * to 16 rows per stream, several streams per call; [AST] commit message: the
+ * decode projections as GEMVs): at 16..256 rows the projection is a dense
+ * contraction and runs on the 5th-generation tensor cores (tcgen05.mma, fp32
+ * accumulators in tensor memory).
+ *   y[m][n] = sum_k x[m][k] * W[n][k],  fp32 out [M, N] (row-major).
+ * The weight is packed once (hgd_gemm_tc_pack_weight) into 128 x 64 tiles in the
+ * tensor core's core-matrix order; the call packs x into its workspace, streams
+ * each tile once, and splits K over CTAs by a fixed function of N and K (the
+ * partials are added in split order), so results do not depend on the device
+ * or the call's neighbours.  The sums follow the tensor core's order, not the
+ * GEMV's: results agree with hgd_gemv_bf16 to fp32 rounding, not bit for bit.
+ * Shapes: 1 <= M <= 256, 1 <= N, 64 <= K <= 65536 with K % 64 == 0
+ * (HGD_ERR_UNSUPPORTED_SHAPE otherwise). */
+/* Bytes of the packed weight of an [N, K] matrix (N rounded up to 128 rows). */
+HGD_API int hgd_gemm_tc_weight_bytes(int N, int K, size_t* bytes);
+/* W [N, K] bf16 (device) -> Wp (device, hgd_gemm_tc_weight_bytes bytes; the
+ * rows past N are zero).  Wp must be complete before a GEMM reads it: the GEMM
+ * starts streaming it before it waits for the kernel that precedes it on the
+ * stream, so that kernel must not be the one writing Wp. */
+HGD_API int hgd_gemm_tc_pack_weight(const uint16_t* W, uint16_t* Wp, int N, int K, hgd_stream_t stream);
+/* Bytes of the workspace of a GEMM of this shape (packed x and split partials). */
+HGD_API int hgd_gemm_tc_workspace_bytes(int M, int N, int K, size_t* bytes);
+/* Wp: packed weight; x [M, K] bf16; y [M, N] fp32; workspace of at least
+ * hgd_gemm_tc_workspace_bytes bytes (HGD_ERR_BUFFER_TOO_SMALL otherwise; no
+ * initial contents needed; calls sharing one must not overlap on the device);
+ * status: optional device int32, set to HGD_ERR_TIMEOUT if an in-kernel wait ran
+ * out (y is then not written).  y must not overlap the other buffers. */
+HGD_API int hgd_gemm_tc_bf16(const uint16_t* Wp, const uint16_t* x, float* y, int M, int N, int K,
+                     void* workspace, size_t workspace_bytes, int32_t* status, hgd_stream_t stream);
+
 /* hgd_gemv_bf16 for callers that cannot allocate device memory (a plugin whose
  * host framework owns the device allocator and offers it no handle; a decode
  * loop that must never wait on the synchronisation a cudaMalloc brings).  The

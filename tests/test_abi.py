@@ -65,6 +65,18 @@ def test_validation_before_any_cuda_call(hgd):
     assert L.hgd_gdn_decode_step(16, 16, 16, 512, 16, 16, 16, 16, None, None, 1, 1, 4, 96, 64, 1, None) == 2
     assert L.hgd_gdn_decode_step(16, 16, 16, 512, 16, 16, 16, 16, None, None, 1, 1, 4, 128, 24, 1, None) == 2
     assert L.hgd_gdn_decode_step(16, 16, 16, 100, 16, 16, 16, 16, None, None, 1, 1, 4, 64, 64, 1, None) == 1
+    # tensor-core GEMM: shapes, alignment and workspace size checked on the host
+    assert L.hgd_gemm_tc_weight_bytes(128, 96, C.byref(n)) == 2                    # K % 64
+    assert L.hgd_gemm_tc_weight_bytes(0, 64, C.byref(n)) == 1
+    assert L.hgd_gemm_tc_weight_bytes(129, 128, C.byref(n)) == 0 and n.value == 256 * 128 * 2
+    assert L.hgd_gemm_tc_workspace_bytes(257, 128, 128, C.byref(n)) == 2           # M > 256
+    assert L.hgd_gemm_tc_workspace_bytes(128, 8224, 1024, C.byref(n)) == 0 and n.value >= 128 * 1024 * 2
+    assert L.hgd_gemm_tc_pack_weight(16, 16, 128, 96, None) == 2
+    assert L.hgd_gemm_tc_pack_weight(18, 16, 128, 128, None) == 3
+    assert L.hgd_gemm_tc_bf16(16, 16, 16, 1, 128, 96, 16, 1 << 20, None, None) == 2
+    assert L.hgd_gemm_tc_bf16(16, 18, 16, 1, 128, 128, 16, 1 << 20, None, None) == 3   # misaligned x
+    assert L.hgd_gemm_tc_bf16(16, 16, 16, 1, 128, 128, None, 1 << 20, None, None) == 1
+    assert L.hgd_gemm_tc_bf16(16, 16, 16, 1, 128, 128, 16, 16, None, None) == 9        # workspace too small
 
 
 def test_model_and_state_layout(hgd):
