@@ -410,6 +410,34 @@ def run_kernels(args) -> None:
         del Ws, Us
         torch.cuda.empty_cache()
 
+    # the tensor-core GEMM at 128 token rows (an 8 x 16 window) on the stack's
+    # projection shapes: bytes and flops per call, against the copy and bf16 peaks
+    tflops_peak = float(measured_peaks().get("bf16_tflops", 1590.0))
+    for name, N, KK in (("GDN in-projection", 8224, 1024), ("up+gate", 7168, 1024), ("down", 1024, 3584),
+                        ("LM head", 248320, 1024)):
+        M = 128
+        wbytes = 2 * N * KK
+        ncopies = max(1, min(64, rot_bytes // wbytes))
+        Wps = []
+        for _ in range(ncopies):
+            W = torch.randn(N, KK, device="cuda", generator=gen).mul_(KK ** -0.5).to(torch.bfloat16)
+            Wps.append(hgd.gemm_tc_pack_weight(W))
+            del W
+        torch.cuda.synchronize()
+        x = torch.randn(M, KK, device="cuda", generator=gen).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+        ws = torch.empty(hgd.gemm_tc_workspace_bytes(M, N, KK), dtype=torch.uint8, device="cuda")
+        us = timed(lambda i: hgd.gemm_tc_bf16(Wps[i], x, N, y=y, workspace=ws), ncopies, 50 if N > 50000 else 200)
+        nbytes = wbytes + 2 * M * KK + 4 * M * N
+        line(f"hgd_gemm_tc_bf16 (k_tc_pack_x + k_gemm_tc + k_tc_reduce) {name}", {"M": M, "N": N, "K": KK}, us,
+             nbytes)
+        tf = 2.0 * M * N * KK / (us * 1e-6) / 1e12
+        print(json.dumps({"kernel": f"hgd_gemm_tc_bf16 {name}", "shape": {"M": M, "N": N, "K": KK}, "tflops": tf,
+                          "frac_of_measured_bf16_peak": tf / tflops_peak,
+                          "note": "standalone kernel, tensor-core throughput"}), flush=True)
+        del Wps
+        torch.cuda.empty_cache()
+
     H, d = 16, 128
     for B in (1, 4, 16, 64):
         sbytes = B * H * d * d * 4

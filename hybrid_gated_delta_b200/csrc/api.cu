@@ -475,8 +475,13 @@ TcPlan tc_plan(int M, int N, int K) {
     const int want = std::max(1, std::min(nkb, TC_TARGET_CTAS / q.n_blocks));
     q.kb_per_split = (nkb + want - 1) / want;
     q.splits = (nkb + q.kb_per_split - 1) / q.kb_per_split;
-    const size_t avail = (size_t)GV_SMEM_LIMIT - tc_smem_bytes(q.NTp, 0);
+    // more than one wave of CTAs: stages for two CTAs per SM, so one's epilogue
+    // overlaps the other's stream; otherwise every stage that fits
+    const int per_sm = q.n_blocks * q.splits > TC_TARGET_CTAS ? 2 : 1;
+    const size_t avail = (size_t)GV_SMEM_LIMIT / per_sm - tc_smem_bytes(q.NTp, 0);
     q.stages = (int)std::min<size_t>(TC_MAX_STAGES, avail / tc_stage_bytes(q.NTp));
+    if (q.stages < 2) q.stages = (int)std::min<size_t>(TC_MAX_STAGES, ((size_t)GV_SMEM_LIMIT - tc_smem_bytes(q.NTp, 0)) /
+                                                                      tc_stage_bytes(q.NTp));
     uint32_t c = 32;
     while ((int)c < q.NTp) c <<= 1;
     q.tmem_cols = c;
