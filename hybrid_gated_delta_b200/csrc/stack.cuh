@@ -317,6 +317,58 @@ __device__ void sk_pro_rmsnorm(const SkParams& s, bf16_t* xs, const bf16_t* gb, 
     }
 }
 
+// RMSNorm of the residual rows straight from global memory into xs, with gains
+// gb (shared; this thread's copies of them waited for here): the arithmetic of
+// gv_prologue's RMSNorm.  Every warp loads its lanes' chunks (chunk c = lane +
+// 32 j) of a row and forms the same sum of squares in the same order, so every
+// warp holds the same scale; the lanes l with l % 8 == warp write their chunks.
+// Needs D % 256 == 0 and D <= 1024.
+constexpr int SK_NORM_MAXJ = 4;
+__device__ void sk_pro_resid_rmsnorm(const SkParams& s, bf16_t* xs, const bf16_t* gb, int warp, int lane) {
+    const int K = s.D, XS = K + GV_PAD, nj = K / 256;
+    uint4 v[SK_NORM_MAXJ][1];
+    for (int m = 0; m < s.M; ++m) {
+        const bf16_t* src = s.resid + (int64_t)m * K;
+#pragma unroll
+        for (int j = 0; j < SK_NORM_MAXJ; ++j)
+            if (j < nj) v[j][0] = *reinterpret_cast<const uint4*>(src + (lane + 32 * j) * 8);
+        if (m == 0) {
+            cp_async_wait_prior();
+            named_bar(1, SK_CT);
+        }
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < SK_NORM_MAXJ; ++j)
+            if (j < nj) {
+                const uint32_t w4[4] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float a = bf_lo(w4[q]), b = bf_hi(w4[q]);
+                    ss = fmaf(a, a, ss);
+                    ss = fmaf(b, b, ss);
+                }
+            }
+        ss = warp_sum(ss);
+        const float r = rsqrtf(ss / (float)K + s.eps);
+        if ((lane & (SK_CW - 1)) == warp) {
+            bf16_t* row = xs + m * XS;
+#pragma unroll
+            for (int j = 0; j < SK_NORM_MAXJ; ++j)
+                if (j < nj) {
+                    const int c = lane + 32 * j;
+                    const uint4 g = lds128(gb + c * 8);
+                    const uint32_t w4[4] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w};
+                    const uint32_t g4[4] = {g.x, g.y, g.z, g.w};
+                    uint32_t o4[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        o4[q] = pack_bf2(bf_lo(w4[q]) * r * bf_lo(g4[q]), bf_hi(w4[q]) * r * bf_hi(g4[q]));
+                    *reinterpret_cast<uint4*>(row + c * 8) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                }
+        }
+    }
+}
+
 // Layer 0: the embedding rows of the tokens (the packed embedding, gathered by
 // 16-byte chunks) into xs, CTA 0 writes them to the residual; a token outside
 // the vocabulary gives a zero row and HGD_ERR_INVALID_ARG.
@@ -939,11 +991,16 @@ __global__ void __launch_bounds__(SK_THREADS, 1) k_stack(const __grid_constant__
             if (live && (!gemv || nmine > 0)) {
                 switch (kind) {
                     case SK_IN_GDN: case SK_IN_ATT: case SK_SWIGLU: case SK_HEAD: {
+                        const bf16_t* gb = (pid & 1) ? sm.gb[1] : sm.gb[0];
+                        if ((kind == SK_SWIGLU || l > 0) && s.D % 256 == 0 && s.D <= 256 * SK_NORM_MAXJ) {
+                            sk_pro_resid_rmsnorm(s, sm.xs, gb, warp, lane);
+                            break;
+                        }
                         if (kind != SK_SWIGLU && l == 0) sk_pro_embed(s, sm.xs);
                         else sk_pro_resid(s, sm.xs);
                         cp_async_wait_prior();
                         named_bar(1, SK_CT);
-                        sk_pro_rmsnorm(s, sm.xs, (pid & 1) ? sm.gb[1] : sm.gb[0], warp, lane);
+                        sk_pro_rmsnorm(s, sm.xs, gb, warp, lane);
                         break;
                     }
                     case SK_OUT_GDN:
