@@ -304,16 +304,21 @@ def test_full_stack_end_to_end_within_rounding_noise(hgd, orc, orc32, full):
             assert int(np.argmax(lg_gpu[s])) == int(np.argmax(r64[s].astype(np.float32)))
 
 
-def _run_paths(hgd, model, cfg, B, T, Lmax, steps, seed):
+def _run_paths(hgd, model, cfg, B, T, Lmax, steps, seed, prefill=None, inputs=None):
     """The same calls through hgd_decode_layer_stack (one persistent launch when
-    B*T <= 8) and through the per-layer range entry (a chain of kernels)."""
+    B*T <= 8) and through the per-layer range entry (a chain of kernels).  With
+    `inputs` (a dict), the initial state and the tokens are left there."""
     import torch
     n_gdn, _ = syn.layer_counts(cfg)
     H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
     Cc = 2 * H * dk + H * dv
     V, L = cfg["vocab"], cfg["n_layers"]
-    init = syn.stack_state(cfg, B, Lmax, prefill=16 if Lmax < 100 else 512, seed=seed)
+    if prefill is None:
+        prefill = 16 if Lmax < 100 else 512
+    init = syn.stack_state(cfg, B, Lmax, prefill=prefill, seed=seed)
     toks = syn.stack_tokens(cfg, B, T * steps, seed=seed)
+    if inputs is not None:
+        inputs.update(init=init, toks=toks)
     outs = []
     for path in ("persistent", "chain"):
         st = hgd.State(model, B, T, Lmax, init)
@@ -359,6 +364,62 @@ def test_persistent_launch_equals_kernel_chain(hgd, full, which):
         assert torch.equal(a1, a2) and torch.equal(s1, s2) and torch.equal(t1, t2), f"call {k}"
     for a, b in ((sp.S, sc.S), (sp.conv, sc.conv), (sp.kv, sc.kv), (sp.pos, sc.pos), (sp.resid, sc.resid)):
         assert torch.equal(a, b)
+
+
+def _assert_paths_equal(rp, sp, rc, sc):
+    import torch
+    for k, ((l1, a1, s1, t1), (l2, a2, s2, t2)) in enumerate(zip(rp, rc)):
+        assert torch.equal(l1, l2), f"call {k}: logits differ"
+        assert torch.equal(a1, a2) and torch.equal(s1, s2) and torch.equal(t1, t2), f"call {k}"
+    for a, b in ((sp.S, sc.S), (sp.conv, sc.conv), (sp.kv, sc.kv), (sp.pos, sc.pos), (sp.resid, sc.resid)):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("prefill,steps,Lmax,B", [(30, 4, 64, 2), (16381, 3, 16384, 1)])
+def test_small_stack_context_edges(hgd, orc, prefill, steps, Lmax, B):
+    """Attention at the edges of its chunking and of the cache, reduced geometry
+    (64-dim heads): positions 30..33 of two streams cross the first 32-key chunk
+    (the new chunk holds one key, then two, ...); the last three positions of the
+    largest cache, 16384 keys (512 chunk partials per query head in one merge).
+    One-row calls through the persistent launch and the kernel chain agree bit
+    for bit, and with the oracle run over the same tokens."""
+    cfg, w = syn.SMALL_CFG, weights("small", 5)
+    model = hgd.Model(cfg, w)
+    assert model.launches(B, 1) == 1
+    inp = {}
+    (rp, sp), (rc, sc) = _run_paths(hgd, model, cfg, B, 1, Lmax, steps, 21, prefill=prefill, inputs=inp)
+    _assert_paths_equal(rp, sp, rc, sc)
+    assert host(sp.pos).tolist() == [prefill + steps] * B
+    V = cfg["vocab"]
+    got = np.stack([host(lg) for (lg, _, _, _) in rp], axis=1).reshape(B * steps, V)
+    am = np.stack([host(a) for (_, a, _, _) in rp], axis=1).reshape(B * steps)
+    m = orc.make_model(cfg, w)
+    ost = oracle_state(orc, inp["init"])
+    r = orc.decode_stack(m, ost, inp["toks"], record=False)
+    compare_logits(got, r["logits"].reshape(B * steps, V), f"context edge {prefill}+{steps}")
+    compare_argmax(am, r["logits"].reshape(B * steps, V), f"context edge {prefill}+{steps}")
+    assert_bf16_close(host(sp.kv), syn.from_bf16(ost["kv"]), "KV cache")
+
+
+def test_full_stack_max_context(hgd, orc, full):
+    """Full size (256-dim heads) at the largest cache: the last two positions of
+    16384 keys.  The persistent launch equals the kernel chain bit for bit, and
+    every layer matches the oracle from the oracle's inputs (two greedy steps)."""
+    cfg = syn.STACK_CFG
+    model, w = full
+    Lmax, prefill = 16384, 16382
+    (rp, sp), (rc, sc) = _run_paths(hgd, model, cfg, 1, 1, Lmax, 2, 22, prefill=prefill)
+    _assert_paths_equal(rp, sp, rc, sc)
+    init = syn.stack_state(cfg, 1, Lmax, prefill=prefill, seed=23)
+    st = hgd.State(model, 1, 1, Lmax)
+    m = orc.make_model(cfg, w)
+    ost = oracle_state(orc, init)
+    tok = syn.stack_tokens(cfg, 1, 1, seed=23)
+    for s in range(2):
+        pre, r = _oracle_call(orc, m, ost, tok)
+        worst = _per_layer_check(hgd, model, st, r, pre, tok, 1, f"max context step {s}")
+        assert worst["S"] <= 1e-4
+        tok = r["argmax"]
 
 
 # ------------------------------------------------------------- windows ------
