@@ -322,7 +322,7 @@ size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_
 
 enum ScratchIdx {
     SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
-    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_END, SC_COUNT
+    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_GN, SC_END, SC_COUNT
 };
 // The persistent launch's control region: control words, one 128-byte line per
 // phase counter, then the phase timestamps.
@@ -370,6 +370,7 @@ void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     sz[SC_BESTI] = (size_t)M * kBestG * 4;
     sz[SC_WS] = stack_ws_bytes(d, (int)M);
     sz[SC_BAR] = kBarBytes;
+    sz[SC_GN] = (size_t)M * d.H * d.dv * 2;  // the chain's gated-norm rows for calls of many rows
     size_t pos = 0;
     for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
     off[SC_END] = pos;
@@ -816,6 +817,7 @@ int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T) {
         n += gemv_chunks(M, d.D);                                   // in-projection
         n += att ? 2 : 1;                                           // partial/merge or GDN mixer
         n += gemv_chunks(M, att ? d.nq * d.hd : d.H * d.dv);        // out-projection
+        if (!att && M > SK_MAXM) n += 1;                            // its gated norm, once per row
         n += gemv_chunks(M, d.D) + gemv_chunks(M, d.I);             // SwiGLU, down
     }
     n += gemv_chunks(M, d.D) + 1;                                   // LM head, argmax
@@ -920,7 +922,8 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
     float* bestv = reinterpret_cast<float*>(A + st->off[SC_BESTV]);
     int32_t* besti = reinterpret_cast<int32_t*>(A + st->off[SC_BESTI]);
     void* ws = A + st->off[SC_WS];
-    const size_t ws_bytes = st->off[SC_END] - st->off[SC_WS];
+    const size_t ws_bytes = st->off[SC_BAR] - st->off[SC_WS];
+    bf16_t* gn_rows = reinterpret_cast<bf16_t*>(A + st->off[SC_GN]);
     const int64_t proj_ld = std::max(d.gdn_out, d.attn_out);
     const float eps = m->cfg.norm_eps;
     const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
@@ -980,10 +983,21 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             if ((rc = launch_status(e))) return rc;
             GemvParams p = {};
             p.W = w[HGD_W_OUT]; p.packed = 1; p.N = d.D; p.K = d.H * d.dv;
-            p.o = obuf; p.o_ld = (int64_t)d.H * d.dv;
-            p.z = proj + d.C; p.z_ld = proj_ld; p.gnorm_w = w[HGD_W_GNORM]; p.gn_d = d.dv; p.eps = eps;
             p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
-            if ((rc = run_gemv<PRO_GATED_NORM, EPI_RESID>(p, M, di.sms, ws, ws_bytes, s))) return rc;
+            if (M > SK_MAXM) {
+                // many rows: the gated norm once per (row, head), then a plain-input GEMV
+                // (the same values reach the MMAs as from the fused prologue)
+                GatedNormParams g{obuf, (int64_t)d.H * d.dv, proj + d.C, proj_ld, w[HGD_W_GNORM], gn_rows,
+                                  (int64_t)d.H * d.dv, M, d.H, d.dv, eps};
+                cudaError_t e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, g);
+                if (e != cudaSuccess) return launch_status(e);
+                p.x = gn_rows; p.x_ld = (int64_t)d.H * d.dv;
+                if ((rc = run_gemv<PRO_COPY, EPI_RESID>(p, M, di.sms, ws, ws_bytes, s))) return rc;
+            } else {
+                p.o = obuf; p.o_ld = (int64_t)d.H * d.dv;
+                p.z = proj + d.C; p.z_ld = proj_ld; p.gnorm_w = w[HGD_W_GNORM]; p.gn_d = d.dv; p.eps = eps;
+                if ((rc = run_gemv<PRO_GATED_NORM, EPI_RESID>(p, M, di.sms, ws, ws_bytes, s))) return rc;
+            }
             ++ig;
         } else {
             AttnParams a{};

@@ -489,6 +489,36 @@ __device__ __forceinline__ void gv_finish(const GemvParams& p, int rb, int s_ite
         }
 }
 
+// The GDN out-projection's input for calls of many token rows, computed once per
+// (token row, head) instead of in every CTA's prologue: the arithmetic of the
+// PRO_GATED_NORM prologue, one warp per (row, head), into u [M][u_ld] (bf16).
+struct GatedNormParams {
+    const float* o; int64_t o_ld;
+    const float* z; int64_t z_ld;
+    const bf16_t* w;
+    bf16_t* u; int64_t u_ld;
+    int M, nh, d;
+    float eps;
+};
+__global__ void __launch_bounds__(256) k_gated_norm(const __grid_constant__ GatedNormParams p) {
+    pdl_launch();
+    pdl_wait();
+    const int e = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (e >= p.M * p.nh) return;
+    const int m = e / p.nh, h = e % p.nh, d = p.d;
+    const float* orow = p.o + m * p.o_ld + h * d;
+    const float* zrow = p.z + m * p.z_ld + h * d;
+    bf16_t* dst = p.u + m * p.u_ld + h * d;
+    float ss = 0.f;
+    for (int i = lane; i < d; i += 32) ss = fmaf(orow[i], orow[i], ss);
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)d + p.eps);
+    for (int i = lane; i < d; i += 32) {
+        const float zb = bf2f(f2bf(zrow[i]));
+        dst[i] = f2bf(orow[i] * r * bf2f(p.w[i]) * silu_f(zb));
+    }
+}
+
 // Per-CTA argmax partials: reduce each token over the row lanes of every warp,
 // then over the warps (`bar` synchronises the nthreads consumer threads).
 template <int NT>
