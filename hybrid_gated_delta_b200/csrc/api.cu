@@ -322,7 +322,7 @@ size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_
 
 enum ScratchIdx {
     SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
-    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_GN, SC_END, SC_COUNT
+    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_GN, SC_XN, SC_END, SC_COUNT
 };
 // The persistent launch's control region: control words, one 128-byte line per
 // phase counter, then the phase timestamps.
@@ -371,6 +371,7 @@ void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     sz[SC_WS] = stack_ws_bytes(d, (int)M);
     sz[SC_BAR] = kBarBytes;
     sz[SC_GN] = (size_t)M * d.H * d.dv * 2;  // the chain's gated-norm rows for calls of many rows
+    sz[SC_XN] = (size_t)M * d.D * 2;         // the chain's RMSNorm rows for calls of many rows
     size_t pos = 0;
     for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
     off[SC_END] = pos;
@@ -817,10 +818,11 @@ int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T) {
         n += gemv_chunks(M, d.D);                                   // in-projection
         n += att ? 2 : 1;                                           // partial/merge or GDN mixer
         n += gemv_chunks(M, att ? d.nq * d.hd : d.H * d.dv);        // out-projection
-        if (!att && M > SK_MAXM) n += 1;                            // its gated norm, once per row
+        if (M > SK_MAXM) n += att ? 2 : 3;                          // norms once per row (in, gated, post)
         n += gemv_chunks(M, d.D) + gemv_chunks(M, d.I);             // SwiGLU, down
     }
     n += gemv_chunks(M, d.D) + 1;                                   // LM head, argmax
+    if (M > SK_MAXM) n += 1;                                        // its norm, once per row
     return n;
 }
 
@@ -924,8 +926,16 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
     void* ws = A + st->off[SC_WS];
     const size_t ws_bytes = st->off[SC_BAR] - st->off[SC_WS];
     bf16_t* gn_rows = reinterpret_cast<bf16_t*>(A + st->off[SC_GN]);
+    bf16_t* xn_rows = reinterpret_cast<bf16_t*>(A + st->off[SC_XN]);
     const int64_t proj_ld = std::max(d.gdn_out, d.attn_out);
     const float eps = m->cfg.norm_eps;
+    const bool many = M > SK_MAXM;  // norms once per row, then plain-input GEMVs
+    auto norm_rows = [&](const bf16_t* gains, bool embed) -> int {
+        NormRowsParams q{resid, d.D, tokens, m->embed, d.V, resid, d.D, gains, eps, xn_rows, d.D, M, d.D, status_dev};
+        cudaError_t e = embed ? launch_pdl(k_norm_rows<true>, dim3((M + 7) / 8), dim3(256), 0, s, q)
+                              : launch_pdl(k_norm_rows<false>, dim3((M + 7) / 8), dim3(256), 0, s, q);
+        return launch_status(e);
+    };
     const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
     const size_t c_layer = (size_t)B * (d.kc - 1) * d.C;
     const size_t kv_half = (size_t)B * d.nkv * Lmax * d.hd;
@@ -952,15 +962,21 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             if (l == 0) {
                 p.tokens = tokens; p.embed = m->embed; p.vocab = d.V; p.resid_out = resid; p.resid_out_ld = d.D;
             }
+            if (many) {
+                if ((rc = norm_rows(w[HGD_W_IN_NORM], l == 0))) return rc;
+                p.x = xn_rows;
+            }
             if (!att) {
                 p.conv_w = w[HGD_W_CONV]; p.conv_tail = conv + ig * c_layer;
                 p.conv_rec = tail_rec ? tail_rec + ig * trec_layer : nullptr;
                 p.conv_C = (int)d.C; p.conv_T = T;
-                rc = (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s)
-                              : run_gemv<PRO_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s);
+                rc = many     ? run_gemv<PRO_COPY, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s)
+                     : (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s)
+                                : run_gemv<PRO_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s);
             } else {
-                rc = (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_ROPE>(p, M, di.sms, ws, ws_bytes, s)
-                              : run_gemv<PRO_RMSNORM, EPI_ROPE>(p, M, di.sms, ws, ws_bytes, s);
+                rc = many     ? run_gemv<PRO_COPY, EPI_ROPE>(p, M, di.sms, ws, ws_bytes, s)
+                     : (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_ROPE>(p, M, di.sms, ws, ws_bytes, s)
+                                : run_gemv<PRO_RMSNORM, EPI_ROPE>(p, M, di.sms, ws, ws_bytes, s);
             }
             if (rc) return rc;
         }
@@ -1023,7 +1039,13 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             p.W = w[HGD_W_GATE]; p.packed = 1; p.N = d.I; p.K = d.D;
             p.x = resid; p.x_ld = d.D; p.norm_w = w[HGD_W_POST_NORM]; p.eps = eps;
             p.y = mlp; p.y_ld = d.I; p.status = status_dev;
-            if ((rc = run_gemv<PRO_RMSNORM, EPI_SWIGLU>(p, M, di.sms, ws, ws_bytes, s))) return rc;
+            if (many) {
+                if ((rc = norm_rows(w[HGD_W_POST_NORM], false))) return rc;
+                p.x = xn_rows;
+                if ((rc = run_gemv<PRO_COPY, EPI_SWIGLU>(p, M, di.sms, ws, ws_bytes, s))) return rc;
+            } else if ((rc = run_gemv<PRO_RMSNORM, EPI_SWIGLU>(p, M, di.sms, ws, ws_bytes, s))) {
+                return rc;
+            }
         }
         {
             GemvParams p = {};
@@ -1040,7 +1062,13 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
         p.x = resid; p.x_ld = d.D; p.norm_w = m->final_norm; p.eps = eps;
         p.logits = logits; p.logits_ld = d.V; p.best_v = bestv; p.best_i = besti; p.status = status_dev;
         int G = 0;
-        if ((rc = run_gemv<PRO_RMSNORM, EPI_ARGMAX>(p, M, di.sms, nullptr, 0, s, &G))) return rc;
+        if (many) {
+            if ((rc = norm_rows(m->final_norm, false))) return rc;
+            p.x = xn_rows;
+            if ((rc = run_gemv<PRO_COPY, EPI_ARGMAX>(p, M, di.sms, nullptr, 0, s, &G))) return rc;
+        } else if ((rc = run_gemv<PRO_RMSNORM, EPI_ARGMAX>(p, M, di.sms, nullptr, 0, s, &G))) {
+            return rc;
+        }
         cudaError_t e = launch_pdl(k_argmax_finalize, dim3(M), dim3(128), 0, s, (const float*)bestv,
                                    (const int32_t*)besti, G, M, argmax, status_dev, pos, B, T);
         if ((rc = launch_status(e))) return rc;

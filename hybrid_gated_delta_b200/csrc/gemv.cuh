@@ -489,6 +489,72 @@ __device__ __forceinline__ void gv_finish(const GemvParams& p, int rb, int s_ite
         }
 }
 
+// The RMSNorm input of a projection for calls of many token rows, once per row
+// instead of in every CTA's prologue: the arithmetic of the PRO_RMSNORM /
+// PRO_EMBED_RMSNORM prologue, one warp per row, into out [M][out_ld] (bf16).
+// EMBED: the row is the token's (packed) embedding row, also written to the
+// residual; a token outside the vocabulary gives zero rows and
+// HGD_ERR_INVALID_ARG.
+struct NormRowsParams {
+    const bf16_t* x; int64_t x_ld;
+    const int32_t* tokens; const bf16_t* embed; int vocab;
+    bf16_t* resid_out; int64_t resid_out_ld;
+    const bf16_t* norm_w; float eps;
+    bf16_t* out; int64_t out_ld;
+    int M, K;
+    int32_t* status;
+};
+template <bool EMBED>
+__global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormRowsParams p) {
+    pdl_launch();
+    pdl_wait();
+    const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (m >= p.M) return;
+    const int K = p.K;
+    bf16_t* dst = p.out + m * p.out_ld;
+    int tok = 0;
+    if (EMBED) {
+        tok = p.tokens[m];
+        if (tok < 0 || tok >= p.vocab) {
+            if (lane == 0) set_status(p.status, HGD_ERR_INVALID_ARG);
+            for (int c = lane; c < K / 8; c += 32) {
+                *reinterpret_cast<uint4*>(dst + c * 8) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(p.resid_out + m * p.resid_out_ld + c * 8) = make_uint4(0, 0, 0, 0);
+            }
+            return;
+        }
+    }
+    auto chunk = [&](int c) -> uint4 {
+        if (EMBED) return *reinterpret_cast<const uint4*>(p.embed + gv_packed_chunk(tok, c, K >> 5));
+        return *reinterpret_cast<const uint4*>(p.x + m * p.x_ld + c * 8);
+    };
+    float ss = 0.f;
+    for (int c = lane; c < K / 8; c += 32) {
+        const uint4 v = chunk(c);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float a = bf_lo(w4[q]), b = bf_hi(w4[q]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
+    }
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)K + p.eps);
+    for (int c = lane; c < K / 8; c += 32) {
+        const uint4 v = chunk(c);
+        const uint4 g = *reinterpret_cast<const uint4*>(p.norm_w + c * 8);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t g4[4] = {g.x, g.y, g.z, g.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            o4[q] = pack_bf2(bf_lo(w4[q]) * r * bf_lo(g4[q]), bf_hi(w4[q]) * r * bf_hi(g4[q]));
+        *reinterpret_cast<uint4*>(dst + c * 8) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        if (EMBED) *reinterpret_cast<uint4*>(p.resid_out + m * p.resid_out_ld + c * 8) = v;
+    }
+}
+
 // The GDN out-projection's input for calls of many token rows, computed once per
 // (token row, head) instead of in every CTA's prologue: the arithmetic of the
 // PRO_GATED_NORM prologue, one warp per (row, head), into u [M][u_ld] (bf16).
