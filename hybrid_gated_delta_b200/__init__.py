@@ -68,6 +68,7 @@ _SIGS = {
     "hgd_gemv_workspace_bytes": ([_i, _i, _i, _i, C.POINTER(_sz)], _i),
     "hgd_gemv_bf16_static_ws": ([_p, _p, _p, _i, _i, _i, _i, _p], _i),
     "hgd_gemv_swiglu_bf16": ([_p, _p, _p, _p, _i, _i, _i, _p, _sz, _p], _i),
+    "hgd_check_bounded_wait": ([_p, _p], _i),
     "hgd_gemm_tc_weight_bytes": ([_i, _i, C.POINTER(_sz)], _i),
     "hgd_gemm_tc_pack_weight": ([_p, _p, _i, _i, _p], _i),
     "hgd_gemm_tc_workspace_bytes": ([_i, _i, _i, C.POINTER(_sz)], _i),
@@ -167,6 +168,11 @@ def gemv_bf16(W, x, y=None, y_is_fp32=True, workspace=None, stream=None):
     _check("hgd_gemv_bf16", _lib.hgd_gemv_bf16(_ptr(W), _ptr(x), _ptr(y), int(y.dtype == torch.float32),
                                                 M, N, K, _ptr(workspace), ws_bytes, _stream(stream)))
     return y
+
+
+def check_bounded_wait(status, stream=None):
+    """Run a bounded in-kernel wait that nothing completes; HGD_ERR_TIMEOUT lands in status."""
+    _check("hgd_check_bounded_wait", _lib.hgd_check_bounded_wait(_ptr(status), _stream(stream)))
 
 
 def gemm_tc_pack_weight(W, stream=None):

@@ -524,6 +524,19 @@ int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int
                                     0, s, (const float*)part, y, q.splits, n));
 }
 
+// A wait that nothing completes: the bounded mbarrier wait of the slab rings and
+// the tensor-core GEMM, on a barrier no thread arrives at.  It runs out after
+// kWaitLimitNs and the kernel reports HGD_ERR_TIMEOUT in *status.
+__global__ void k_check_bounded_wait(int32_t* status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0u, nullptr)) set_status(status, HGD_ERR_TIMEOUT);
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -581,6 +594,16 @@ int hgd_gemv_swiglu_bf16(const uint16_t* W_gate, const uint16_t* W_up, const uin
     GemvParams p = {};
     p.W = W_gate; p.W2 = W_up; p.N = I; p.K = K; p.x = x; p.x_ld = K; p.y = h; p.y_ld = I;
     return run_gemv<PRO_COPY, EPI_SWIGLU>(p, M, di.sms, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+int hgd_check_bounded_wait(int32_t* status, hgd_stream_t stream) {
+    if (!status) return HGD_ERR_INVALID_ARG;
+    if (!al16(status)) return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    k_check_bounded_wait<<<1, 32, 0, (cudaStream_t)stream>>>(status);
+    return launch_status(cudaGetLastError());
 }
 
 int hgd_gemm_tc_weight_bytes(int N, int K, size_t* bytes) {

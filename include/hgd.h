@@ -99,6 +99,15 @@ HGD_API int hgd_gemv_bf16(const uint16_t* W, const uint16_t* x, void* y, int y_i
  * SwiGLU (swiglu = 1, N = I) of this shape; 0 when that shape never uses one. */
 HGD_API int hgd_gemv_workspace_bytes(int M, int N, int K, int swiglu, size_t* bytes);
 
+/* ------------------------------------------------------------ diagnostics ---
+ * Check that a stuck in-kernel wait ends with a status rather than a hang (the
+ * conventions above: errors found inside a kernel go to a device status word):
+ * one kernel runs the bounded mbarrier wait the weight rings and the tensor-core
+ * GEMM use, on a barrier that nothing completes.  About 2 s later the wait runs
+ * out and the kernel writes HGD_ERR_TIMEOUT to *status (device int32, 16-byte
+ * aligned; not cleared first).  Launches nothing else; the context stays usable. */
+HGD_API int hgd_check_bounded_wait(int32_t* status, hgd_stream_t stream);
+
 /* ------------------------------------------------------- tensor-core GEMM ---
  * The same product for windows of many token rows ([TF] PR body: windows of up
  * to 16 rows per stream, several streams per call; [AST] commit message: the

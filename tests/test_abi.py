@@ -77,6 +77,8 @@ def test_validation_before_any_cuda_call(hgd):
     assert L.hgd_gemm_tc_bf16(16, 18, 16, 1, 128, 128, 16, 1 << 20, None, None) == 3   # misaligned x
     assert L.hgd_gemm_tc_bf16(16, 16, 16, 1, 128, 128, None, 1 << 20, None, None) == 1
     assert L.hgd_gemm_tc_bf16(16, 16, 16, 1, 128, 128, 16, 16, None, None) == 9        # workspace too small
+    assert L.hgd_check_bounded_wait(None, None) == 1
+    assert L.hgd_check_bounded_wait(20, None) == 3
 
 
 def test_model_and_state_layout(hgd):

@@ -108,3 +108,22 @@ def test_gemm_tc_window_shapes(hgd, orc, name):
     err = np.abs(got - ref)
     bound = fp32_dot_bound(Ws, c["x"])
     assert np.all(err <= 2 * bound + 1e-30), (name, err.max(), (err / (bound + 1e-30)).max())
+
+
+def test_stuck_wait_reports_timeout_and_context_survives(hgd, orc):
+    """A bounded in-kernel wait that nothing completes ends after its limit with
+    HGD_ERR_TIMEOUT in the status word; the next calls still compute correctly."""
+    import time
+    import torch
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    hgd.check_bounded_wait(status)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert int(status[0].item()) == 5  # HGD_ERR_TIMEOUT
+    assert 1.0 < elapsed < 30.0, elapsed
+    c = syn.gemv_case(257, 1024, 16, seed=14)
+    y, guard_ok, _, _ = _run(hgd, dev_bf16(c["W"]), dev_bf16(c["x"]), 257)
+    assert guard_ok
+    err = np.abs(host(y) - orc.gemv(c["W"], c["x"]))
+    assert np.all(err <= 2 * fp32_dot_bound(c["W"], c["x"]) + 1e-30)
