@@ -115,7 +115,8 @@ __device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity,
 
 // ----------------------------------------------------------- bulk (TMA) copy
 // 1-D bulk copy global -> shared, completing `bytes` of transaction count on
-// `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.  No multicast.
+// `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.  The copy lands in
+// this CTA's own shared memory only.
 __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes,
                                          uint64_t* bar, uint64_t policy) {
     asm volatile(

@@ -9,7 +9,7 @@
 // Here one CTA owns a 128-row block of W (the MMA's M), takes every token row
 // of the call as the MMA's N (16..256), and streams its K range through a ring
 // of shared-memory stages:
-//   - one lane issues the bulk copies (cp.async.bulk, no multicast) of a
+//   - one lane issues the bulk copies (cp.async.bulk, into this CTA only) of a
 //     stage's weight tile (128 x 64, 16 KB) and token tile (NTp x 64),
 //     completing on the stage's `full` mbarrier;
 //   - one lane issues four tcgen05.mma (K = 16 each) per stage into a TMEM

@@ -8,7 +8,7 @@
 //  * weights never depend on activations, so the producer walks the CTA's share
 //    of every projection of the step in order and streams each 16-row x
 //    256-column weight slab (8 KB, contiguous thanks to the fragment-ordered
-//    packing) with one bulk copy (cp.async.bulk, no multicast, L2 evict-first)
+//    packing) with one bulk copy (cp.async.bulk into this CTA's own shared memory, L2 evict-first)
 //    into a CTA-wide ring of NS slots, across phase boundaries: HBM stays busy
 //    while the consumers wait for the previous phase.  Slab g of the CTA's
 //    sequence sits in slot g % NS and is consumed by warp g % 8 (NS is a
