@@ -630,7 +630,7 @@ __device__ __forceinline__ void gv_argmax_cta(const GemvParams& p, GvBest<NT>& b
 template <int NT, int PRO, int EPI>
 __global__ void __launch_bounds__(GV_THREADS, (NT >= 4) ? 1 : 2) k_gemv(const __grid_constant__ GemvParams p) {
     constexpr int MP = 8 * NT;
-    constexpr int NB = (NT >= 4) ? 4 : 8;   // 32-column steps in flight per warp
+    constexpr int NB = 8;  // 32-column steps in flight per warp
     constexpr bool SWI = (EPI == EPI_SWIGLU);
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
