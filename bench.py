@@ -129,6 +129,39 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------ host cores --
+
+def host_info() -> dict:
+    """The host the oracle is timed on: online cores and the CPU model."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+class one_core:
+    """Pin this process to one of its allowed cores while timing the oracle
+    (single-threaded), and restore the previous set afterwards."""
+
+    def __enter__(self):
+        self.prev = None
+        if hasattr(os, "sched_getaffinity"):
+            self.prev = os.sched_getaffinity(0)
+            os.sched_setaffinity(0, {min(self.prev)})
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            os.sched_setaffinity(0, self.prev)
+        return False
+
+
 # ---------------------------------------------------------------- reference --
 
 def run_reference(args) -> None:
@@ -149,16 +182,17 @@ def run_reference(args) -> None:
     tok = syn.stack_tokens(cfg, 1, 1, seed=4)
     budget_s = float(os.environ.get("HGD_REF_BUDGET_S", "60"))
     warm = min(args.warmup, 1)
-    for _ in range(warm):
-        tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
-    t0 = time.perf_counter()
-    n = 0
-    while n < args.steps:
-        tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
-        n += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
+    with one_core():
+        for _ in range(warm):
+            tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
+        t0 = time.perf_counter()
+        n = 0
+        while n < args.steps:
+            tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
     v = n / dt
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
            "steps": n, "warmup": warm, "ms_per_step": 1000 * dt / n, "higher_is_better": True,
@@ -166,7 +200,8 @@ def run_reference(args) -> None:
            "config": {"workload": WORKLOAD, "batch": 1, "kv_context": PREFILL},
            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                             "sample": f"{n} greedy tokens of the full stack (of {args.steps} asked; "
-                                      f"{budget_s:.0f} s budget), single-threaded C oracle, fp64"},
+                                      f"{budget_s:.0f} s budget), single-threaded C oracle, fp64, pinned "
+                                      f"to one core", **host_info()},
            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
@@ -181,12 +216,14 @@ def cpu_baseline_sample(tokens: int = 4) -> dict:
     st = {"S": init["S"].astype(np.float64), "tail": init["tail"].astype(np.float64), "kv": init["kv"],
           "pos": init["pos"]}
     tok = syn.stack_tokens(cfg, 1, 1, seed=4)
-    t0 = time.perf_counter()
-    for _ in range(tokens):
-        tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
-    dt = time.perf_counter() - t0
+    with one_core():
+        t0 = time.perf_counter()
+        for _ in range(tokens):
+            tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
+        dt = time.perf_counter() - t0
     return {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{tokens} greedy tokens of the full stack, single-threaded C oracle (fp64)"}
+            "sample": f"{tokens} greedy tokens of the full stack, single-threaded C oracle (fp64), pinned to one core",
+            **host_info()}
 
 
 # ---------------------------------------------------------------- replicas --
