@@ -137,3 +137,29 @@ def test_model_init_rejects_unsupported(hgd):
     assert hgd._lib.hgd_model_init(C.byref(m), C.byref(cfg), 272, 1 << 40) == 3
     assert hgd._lib.hgd_model_init(C.byref(m), C.byref(cfg), 256, 1 << 40) == 0
     assert m.embed == 256
+
+
+def test_tensor_core_split_depends_on_n_and_k_only(hgd):
+    """The tensor-core GEMM splits K over CTAs by a fixed function of N and K (a
+    split never depends on M or on the device): its workspace is the packed x
+    plus splits x M x N fp32 partials, with the same split count at every M, and
+    no partials once the row tiles alone fill the device (N = 248320)."""
+    L = hgd._lib
+    n = C.c_size_t()
+
+    def ws(M, N, K):
+        assert L.hgd_gemm_tc_workspace_bytes(M, N, K, C.byref(n)) == 0
+        return n.value
+
+    def xp(M, K):
+        ntp = 16 if M <= 16 else (M + 15) // 16 * 16
+        return (ntp * K * 2 + 255) // 256 * 256
+
+    for N, K in ((1024, 3584), (1024, 2048), (8224, 1024), (300, 640)):
+        splits = {(ws(M, N, K) - xp(M, K)) // (M * N * 4) for M in (1, 16, 33, 128, 256)}
+        assert len(splits) == 1, (N, K, splits)
+        s = splits.pop()
+        assert 1 <= s <= K // 64
+        for M in (1, 16, 33, 128, 256):
+            assert ws(M, N, K) == xp(M, K) + (s * M * N * 4 if s > 1 else 0)
+    assert ws(128, 248320, 1024) == xp(128, 1024)
