@@ -552,7 +552,7 @@ def main():
     ap.add_argument("--path", default="persistent", choices=["chain", "persistent"],
                     help="chain: one kernel per op, PDL-overlapped, in CUDA graphs; "
                          "persistent: the whole step in one cooperative launch")
-    ap.add_argument("--cpu-tokens", type=int, default=12)  # about 13 s of oracle work on the B200 host
+    ap.add_argument("--cpu-tokens", type=int, default=12)  # about 13 s of oracle work at ~1 token/s
     ap.add_argument("--windows", action="store_true",
                     help="instead of the benchmark line: throughput of 8 streams x 16-row windows")
     ap.add_argument("--kernels", action="store_true",
