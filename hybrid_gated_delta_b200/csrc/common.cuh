@@ -125,12 +125,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
         "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
 }
-// 16-byte asynchronous copy global -> shared (cp.async, L2 only), and the wait
-// for this thread's outstanding copies.
+// 16-byte asynchronous copy global -> shared (cp.async, L2 only), committed in
+// groups; a thread waits for all but its newest group.
 __device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)), "l"(src_gmem) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 // Wait until at most the newest committed group of this thread is in flight.
 __device__ __forceinline__ void cp_async_wait_prior() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }

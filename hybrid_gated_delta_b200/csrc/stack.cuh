@@ -105,12 +105,6 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// 16-byte load cached in L2 only (data written by other SMs during the launch).
-__device__ __forceinline__ float4 ld_cg4(const float* p) {
-    float4 v;
-    asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
-    return v;
-}
 __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -516,15 +510,6 @@ __device__ void sk_merge_head_t(const float* base, int nch, const float* gate, b
     }
 #pragma unroll
     for (int i = 0; i < DPL; ++i) out[d0 + i] = f2bf(acc[i] / L * sigmoid_f(gate[d0 + i]));
-}
-__device__ __forceinline__ void sk_merge_head(const float* base, int nch, int hd, const float* gate, bf16_t* out,
-                                              int lane) {
-    switch (hd) {
-        case 256: sk_merge_head_t<8>(base, nch, gate, out, lane); break;
-        case 128: sk_merge_head_t<4>(base, nch, gate, out, lane); break;
-        case 64: sk_merge_head_t<2>(base, nch, gate, out, lane); break;
-        default: sk_merge_head_t<1>(base, nch, gate, out, lane); break;
-    }
 }
 
 // Down-projection input: the SwiGLU rows (bf16) as they are.
