@@ -78,6 +78,9 @@ class Oracle:
         L.hgdo_swiglu.argtypes = [_p, _p, _p, _p, C.c_int, C.c_int, C.c_int]
         L.hgdo_conv1d_tail_update.argtypes = [_p, _p, _p, _p, _p] + [C.c_int] * 5
         L.hgdo_gdn_step.argtypes = [_p, _p, _p, C.c_int64, _p, _p, _p, _p, _p] + [C.c_int] * 6
+        L.hgdo_softplus.restype = C.c_double if nb == 8 else C.c_float
+        L.hgdo_softplus.argtypes = [C.c_double if nb == 8 else C.c_float]
+        L.hgdo_gdn_gates.argtypes = [_p, _p, _p, _p, C.c_int]
         L.hgdo_rmsnorm.argtypes = [_p, _p, _p, C.c_int, C.c_int, C.c_double]
         L.hgdo_gated_rmsnorm.argtypes = [_p, _p, _p, _p, C.c_int, C.c_int, C.c_int, C.c_double]
         L.hgdo_rope.argtypes = [_p, C.c_int, C.c_int, C.c_double]
@@ -175,6 +178,19 @@ class Oracle:
                                stride, _ptr(g), _ptr(b), _ptr(S), _ptr(o), _ptr(rec),
                                B, T, H, dk, dv, int(l2norm))
         return (o, rec) if record else o
+
+    def softplus(self, t) -> float:
+        return float(self.lib.hgdo_softplus(float(t)))
+
+    def gdn_gates(self, a, A_log, dt_bias) -> np.ndarray:
+        """a [H] real; A_log, dt_bias [H] bf16.  Returns g [H] (log-decay)."""
+        a = self._r(a)
+        A_log, dt_bias = self._u16(A_log), self._u16(dt_bias)
+        H = a.shape[0]
+        assert A_log.shape == (H,) and dt_bias.shape == (H,)
+        g = np.empty(H, self.real)
+        self.lib.hgdo_gdn_gates(_ptr(a), _ptr(A_log), _ptr(dt_bias), _ptr(g), H)
+        return g
 
     def rmsnorm(self, x, w, eps=1e-6) -> np.ndarray:
         x, w = self._u16(x), self._u16(w)

@@ -78,6 +78,15 @@ static real sigmoid(real t) { return (real)1 / ((real)1 + R_EXP(-t)); }
 /* [MOE] activation_topk: max(x,0) + log1p(exp(-|x|)). */
 static real softplus(real t) { return (t > 0 ? t : (real)0) + R_LOG1P(R_EXP(-R_FABS(t))); }
 
+real hgdo_softplus(real t) { return softplus(t); }
+
+/* Log-decay of the GDN layers of the stack, one per head ([TF] PR body: the
+ * gated delta rule; commit on config.json widths: A_log stored as bf16):
+ *   g[h] = -exp(A_log[h]) * softplus(a[h] + dt_bias[h]),  so alpha = exp(g) in (0, 1]. */
+void hgdo_gdn_gates(const real* a, const uint16_t* A_log, const uint16_t* dt_bias, real* g, int H) {
+    for (int h = 0; h < H; ++h) g[h] = -R_EXP(bf(A_log[h])) * softplus(a[h] + bf(dt_bias[h]));
+}
+
 /* ------------------------------------------------------------ GEMV ----- */
 
 /* [AST] BF16 GEMV: y = x W^T with W in the [N,K] (Linear) layout. */
@@ -323,11 +332,8 @@ int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens
                     real* trec = tail_rec ? tail_rec + (((int64_t)ig * B + b) * T + t) * (kc - 1) * Cc : NULL;
                     hgdo_conv1d_tail_update(p, tl, w->conv_w, y, trec, 1, 1, Cc, kc, 1);
                     for (int i = 0; i < H * dv; ++i) z[i] = round_bf16(p[Cc + i]);
-                    for (int hh = 0; hh < H; ++hh) {
-                        real a = p[Cc + H * dv + hh];
-                        gg[hh] = -R_EXP(bf(w->A_log[hh])) * softplus(a + bf(w->dt_bias[hh]));
-                        bb[hh] = p[Cc + H * dv + H + hh];
-                    }
+                    hgdo_gdn_gates(p + Cc + H * dv, w->A_log, w->dt_bias, gg, H);
+                    for (int hh = 0; hh < H; ++hh) bb[hh] = p[Cc + H * dv + H + hh];
                     real* srec = S_rec ? S_rec + (((int64_t)ig * B + b) * T + t) * H * dv * dk : NULL;
                     hgdo_gdn_step(y, y + H * dk, y + 2 * H * dk, Cc, gg, bb, S, o, srec,
                                   1, 1, H, dk, dv, 1);

@@ -92,6 +92,16 @@ void hgdo_gdn_step(const hgdo_real* q, const hgdo_real* k, const hgdo_real* v, i
                    const hgdo_real* g, const hgdo_real* braw, hgdo_real* S, hgdo_real* o,
                    hgdo_real* S_rec, int B, int T, int H, int dk, int dv, int l2norm);
 
+/* softplus(t) = max(t,0) + log1p(exp(-|t|))  ([MOE] activation_topk's stable form). */
+hgdo_real hgdo_softplus(hgdo_real t);
+
+/* Log-decay of the stack's GDN layers, per head h < H:
+ *   g[h] = -exp(A_log[h]) * softplus(a[h] + dt_bias[h])
+ * a[h] is the head's "a" projection output (real); A_log and dt_bias are the
+ * layer's bf16 parameters.  The state update then uses alpha = exp(g). */
+void hgdo_gdn_gates(const hgdo_real* a, const uint16_t* A_log, const uint16_t* dt_bias,
+                    hgdo_real* g, int H);
+
 /* y[m] = bf16( x[m] * (1/sqrt(mean(x[m]^2) + eps)) * w )   ([FT] RMSNorm). */
 void hgdo_rmsnorm(const uint16_t* x, const uint16_t* w, uint16_t* y, int M, int D, double eps);
 
@@ -185,7 +195,7 @@ typedef struct hgdo_state {
  *   x = E[token]                                            (bf16 residual stream)
  *   per layer:  h = bf16(RMSNorm(x) * in_norm)
  *     GDN:  p = W_in h;  conv(q|k|v) with SiLU;  z = bf16(p_z)
- *           g = -exp(A_log) * softplus(a + dt_bias),  beta from b
+ *           g = hgdo_gdn_gates(a, A_log, dt_bias),  beta from b
  *           gated delta rule per head (dense form);  u = bf16(gatedRMSNorm(o, z))
  *           x = bf16(x + W_out u)
  *     attn: p = W_in h;  RoPE(q), RoPE(k) at the row's position;

@@ -321,6 +321,107 @@ def test_gdn_packed_rows_match_separate(orc):
 
 # --------------------------------------------------------------- norms -----
 
+# --------------------------------------------------------- GDN gates -----
+# North_star: alpha_t = exp(g_t).  The stack's log-decay is
+# g = -exp(A_log) * softplus(a + dt_bias) with the stable softplus
+# max(x,0) + log1p(exp(-|x|)) ("nvfp4-megamoe-kernel commit log", activation_topk).
+# The references below are evaluated with mpmath at 50 digits from the closed
+# form log(1 + e^x), not from the oracle's formula.
+
+def _mp_softplus(x):
+    import mpmath
+    mpmath.mp.dps = 50
+    return mpmath.log1p(mpmath.exp(mpmath.mpf(x)))
+
+
+def _mp_gate(a, A_log, dt):
+    import mpmath
+    mpmath.mp.dps = 50
+    return -mpmath.exp(mpmath.mpf(A_log)) * _mp_softplus(mpmath.mpf(a) + mpmath.mpf(dt))
+
+
+def test_softplus_closed_forms(orc):
+    pytest.importorskip("mpmath")
+    assert abs(orc.softplus(0.0) - math.log(2.0)) <= 2 * EPS_D * math.log(2.0)
+    # softplus(x) - softplus(-x) = x, and the limits at both ends: the unstable
+    # log(1 + exp(x)) gives 0 at -40 (1 + e^-40 rounds to 1) and inf past 709,
+    # the stable form e^x and x to full relative precision
+    for x in (-700.0, -40.0, -7.25, -1.0, -1e-3, 1e-3, 0.5, 3.0, 40.0, 700.0):
+        ref = float(_mp_softplus(x))
+        got = orc.softplus(x)
+        assert got > 0 and abs(got - ref) <= 4 * EPS_D * ref, (x, got, ref)
+        assert abs((orc.softplus(x) - orc.softplus(-x)) - x) <= 8 * EPS_D * max(1.0, abs(x))
+    assert orc.softplus(800.0) == 800.0
+
+
+def test_gdn_gates_match_closed_form(orc):
+    """g = -exp(A_log) softplus(a + dt_bias) per head, against the closed form in
+    50-digit arithmetic: a dropped exp on A_log, a wrong sign or a missing
+    dt_bias each miss by far more than the tolerance."""
+    pytest.importorskip("mpmath")
+    g = syn.rng(41)
+    H = 64
+    a = g.standard_normal(H) * 3.0
+    A_log = syn.to_bf16((g.standard_normal(H) * 0.7).astype(np.float32))
+    dt = syn.to_bf16((g.standard_normal(H) * 1.5).astype(np.float32))
+    got = orc.gdn_gates(a, A_log, dt)
+    ref = np.array([float(_mp_gate(a[h], bfv(A_log[h]), bfv(dt[h]))) for h in range(H)])
+    assert np.all(got < 0)
+    assert np.all(np.abs(got - ref) <= 8 * EPS_D * np.abs(ref))
+    # special cases: A_log = 0, dt_bias = 0 give g = -softplus(a); A_log = bf16(ln 2)
+    # scales |g| by exp(bf16(ln 2)) (= 1.9965, the bf16 value of ln 2 being 0.69140625)
+    z = np.zeros(H, np.uint16)
+    g0 = orc.gdn_gates(a, z, z)
+    assert np.all(np.abs(g0 + np.array([float(_mp_softplus(v)) for v in a])) <= 4 * EPS_D * np.abs(g0))
+    ln2 = np.full(H, syn.to_bf16(np.array([math.log(2.0)], np.float32))[0], np.uint16)
+    assert bfv(ln2[0]) == 0.69140625
+    g2 = orc.gdn_gates(a, ln2, z)
+    assert np.all(np.abs(g2 / g0 - math.exp(0.69140625)) <= 8 * EPS_D)
+    # dt_bias enters as a shift of a
+    gd = orc.gdn_gates(a, z, dt)
+    assert np.allclose(gd, orc.gdn_gates(a + bfv(dt), z, z), rtol=8 * EPS_D, atol=0)
+
+
+def test_stack_gdn_decay_follows_the_gates(orc):
+    """One GDN layer of the stack with its key rows zeroed and zero conv tails: the
+    key is 0, so the layer's update reduces to S <- alpha S with
+    alpha = exp(-exp(A_log[h]) softplus(a_h + dt_bias[h])).  The a-row of head h is
+    the unit vector e_{j_h}, so a_h is the normalised input's element j_h (from the
+    oracle's RMSNorm, pinned above).  The recorded state after the row is compared
+    with alpha * S0 per head, alpha from the closed form in 50-digit arithmetic:
+    this ties the stack to the gate formula, to its a/b row order and to the
+    per-head A_log and dt_bias."""
+    pytest.importorskip("mpmath")
+    cfg = dict(syn.SMALL_CFG, n_layers=1, attn_every=8)
+    w = syn.stack_weights(cfg, seed=42)
+    H, dk, dv, D = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["hidden"]
+    Cc = 2 * H * dk + H * dv
+    lw = w["layers"][0]
+    w_in = lw["w_in"].copy()
+    w_in[H * dk:2 * H * dk] = 0                        # key rows: k = conv(0) = silu(0) = 0
+    cols = [3, 200]
+    for h in range(H):
+        w_in[Cc + H * dv + h] = 0
+        w_in[Cc + H * dv + h, cols[h]] = 0x3F80          # a_h = 1.0 * hnorm[cols[h]]
+    lw["w_in"] = w_in
+    lw["A_log"] = syn.to_bf16(np.array([0.6, -0.9], np.float32))
+    lw["dt_bias"] = syn.to_bf16(np.array([-1.25, 2.0], np.float32))
+    m = orc.make_model(cfg, w)
+    st = syn.stack_state(cfg, 1, 8, prefill=0, seed=43)
+    st["S"] = st["S"].astype(orc.real)
+    st["tail"] = np.zeros_like(st["tail"], dtype=orc.real)
+    S0 = st["S"].copy()
+    tok = np.array([[17]], np.int32)
+    r = orc.decode_stack(m, st, tok, record=True)
+    hn = bfv(orc.rmsnorm(w["embed"][17][None], lw["in_norm"]))[0]
+    for h in range(H):
+        alpha = float(__import__("mpmath").exp(_mp_gate(hn[cols[h]], bfv(lw["A_log"][h]),
+                                                           bfv(lw["dt_bias"][h]))))
+        ratio = r["S_rec"][0, 0, 0, h] / S0[0, 0, h]
+        assert 0 < alpha < 1
+        assert np.all(np.abs(ratio - alpha) <= 4 * EPS_D * alpha), (h, ratio.min(), ratio.max(), alpha)
+
+
 def test_rmsnorm_unit_gain_gives_unit_rms(orc):
     g = syn.rng(31)
     x = syn.normal_bf16(g, (5, 512), 3.0)
