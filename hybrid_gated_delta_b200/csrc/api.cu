@@ -5,10 +5,12 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <utility>
 #include <cstdio>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "attn.cuh"
 #include "common.cuh"
@@ -21,18 +23,99 @@ using namespace hgd;
 
 namespace {
 
+// ------------------------------------------------------------ context identity
+// What the library caches per device (a kernel's shared-memory attribute, its
+// occupancy, the device address of a built-in array) belongs to a CUDA context,
+// not to the device ordinal: after a device reset the next call runs in a new
+// context, where attributes are unset and a module variable may sit at another
+// address.  Every such cache is therefore keyed on the current context's id
+// (cuCtxGetId: unique within the process, never reused), read through the
+// runtime's driver entry points so the library links no driver stub.
+typedef int (*CtxGetCurrentFn)(void**);
+typedef int (*CtxGetIdFn)(void*, unsigned long long*);
+
+// Id of the calling thread's current context; 0 when there is none yet or the
+// driver cannot tell (callers then cache nothing).
+unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+        cudaGetLastError();
+    });
+    if (!get_cur || !get_id) return 0;
+    void* ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_cur(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+    return id;
+}
+
+// A value cached per context: a few slots, each holding (context id, value),
+// read and written under one mutex.  Lookups from concurrent host threads are
+// safe; a context that is not found is simply computed again.
+template <typename V, int N = 8>
+struct CtxCache {
+    std::mutex mu;
+    unsigned long long id[N] = {};
+    V val[N] = {};
+    int next = 0;
+    bool get(unsigned long long ctx, V* out) {
+        if (!ctx) return false;
+        std::lock_guard<std::mutex> g(mu);
+        for (int i = 0; i < N; ++i)
+            if (id[i] == ctx) { *out = val[i]; return true; }
+        return false;
+    }
+    void put(unsigned long long ctx, const V& v) {
+        if (!ctx) return;
+        std::lock_guard<std::mutex> g(mu);
+        for (int i = 0; i < N; ++i)
+            if (id[i] == ctx) { val[i] = v; return; }
+        id[next] = ctx;
+        val[next] = v;
+        next = (next + 1) % N;
+    }
+};
+
+// Sets the dynamic shared-memory limit of `kern` once per context.
+template <typename K>
+cudaError_t ensure_smem_attr(K kern, CtxCache<int>& done) {
+    const unsigned long long ctx = current_ctx_id();
+    int v = 0;
+    if (done.get(ctx, &v)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT);
+    if (e != cudaSuccess) return e;
+    done.put(ctx, 1);
+    return cudaSuccess;
+}
+
 // ------------------------------------------------------------ device info
 struct DevInfo {
     int ok;    // 1 = sm_100, 0 = unsupported, -1 = cuda error
     int sms;
 };
 
+// The architecture and SM count of the current device (properties of the
+// device, so cached per ordinal; packed in one atomic word: bit 31 set = known).
 int device_info(DevInfo* di) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HGD_ERR_CUDA; }
-    static DevInfo cache[64];
-    static int have[64];
-    if (dev >= 0 && dev < 64 && have[dev]) { *di = cache[dev]; return di->ok == 1 ? HGD_OK : HGD_ERR_UNSUPPORTED_DEVICE; }
+    static std::atomic<unsigned> cache[64];
+    const bool cache_ok = dev >= 0 && dev < 64;
+    const unsigned c = cache_ok ? cache[dev].load(std::memory_order_relaxed) : 0u;
+    if (c & 0x80000000u) {
+        *di = DevInfo{(int)((c >> 30) & 1u), (int)(c & 0xFFFFu)};
+        return di->ok == 1 ? HGD_OK : HGD_ERR_UNSUPPORTED_DEVICE;
+    }
     int major = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
@@ -40,7 +123,8 @@ int device_info(DevInfo* di) {
         return HGD_ERR_CUDA;
     }
     DevInfo d{major == 10 ? 1 : 0, sms};
-    if (dev >= 0 && dev < 64) { cache[dev] = d; have[dev] = 1; }
+    if (cache_ok)
+        cache[dev].store(0x80000000u | ((unsigned)d.ok << 30) | ((unsigned)sms & 0xFFFFu), std::memory_order_relaxed);
     *di = d;
     return d.ok == 1 ? HGD_OK : HGD_ERR_UNSUPPORTED_DEVICE;
 }
@@ -120,24 +204,24 @@ size_t gemv_ws_bytes(int M, int N, int K, bool swiglu) {
 template <int NT, int PRO, int EPI>
 cudaError_t launch_gemv_t(GemvParams p, size_t smem, int sms, cudaStream_t s, int* grid_out) {
     auto kern = k_gemv<NT, PRO, EPI>;
-    static int attr_done[64];
-    static int occ_cache[64][4];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const bool cache_ok = dev >= 0 && dev < 64;
-    if (!cache_ok || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT);
-        if (e != cudaSuccess) return e;
-        if (cache_ok) attr_done[dev] = 1;
-    }
-    // occupancy for this shared-memory size (bucketed by 16 KB, cached)
+    static CtxCache<int> attr_done;
+    struct Occ { int v[4]; };
+    static CtxCache<Occ> occ_cache;
+    cudaError_t e = ensure_smem_attr(kern, attr_done);
+    if (e != cudaSuccess) return e;
+    // occupancy for this shared-memory size (bucketed by 56 KB, cached per context)
+    const unsigned long long ctx = current_ctx_id();
     const int bucket = std::min(3, (int)(smem / (56 * 1024)));
-    int occ = cache_ok ? occ_cache[dev][bucket] : 0;
+    Occ oc{};
+    occ_cache.get(ctx, &oc);
+    int occ = oc.v[bucket];
     if (occ == 0) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, GV_THREADS, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, GV_THREADS, smem);
         if (e != cudaSuccess) return e;
         occ = std::max(1, occ);
-        if (cache_ok) occ_cache[dev][bucket] = occ;
+        occ_cache.get(ctx, &oc);
+        oc.v[bucket] = occ;
+        occ_cache.put(ctx, oc);
     }
     // items go to CTAs first (slot = warp * grid + cta), so a GEMV with few items
     // still spreads over every SM
@@ -412,15 +496,10 @@ bool sk_supported(const Dims& d, int M) {
 template <int KPL, int DPL>
 int sk_launch_t(const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
     auto kern = k_stack<KPL, DPL>;
-    static int attr_done[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT) != cudaSuccess) {
-            cudaGetLastError();
-            return HGD_ERR_CUDA;
-        }
-        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    static CtxCache<int> attr_done;
+    if (ensure_smem_attr(kern, attr_done) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
     }
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, SK_THREADS, smem) != cudaSuccess) {
@@ -496,16 +575,10 @@ bool tc_shape_ok(int M, int N, int K) { return M >= 1 && M <= TC_MAXN && N >= 1 
 int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int N, int K, void* ws,
            int32_t* status, cudaStream_t s) {
     const TcPlan q = tc_plan(M, N, K);
-    static int attr_done[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        if (cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM_LIMIT) !=
-            cudaSuccess) {
-            cudaGetLastError();
-            return HGD_ERR_CUDA;
-        }
-        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    static CtxCache<int> attr_done;
+    if (ensure_smem_attr(k_gemm_tc, attr_done) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
     }
     bf16_t* Xp = static_cast<bf16_t*>(ws);
     float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + q.xp_bytes);
@@ -1116,19 +1189,21 @@ namespace {
 constexpr size_t kStaticWsBytes = (size_t)4 << 20;  // 4 MiB of scratch per device
 static __device__ __align__(256) uint8_t g_gemv_static_ws[kStaticWsBytes];
 
-// Device address of the array on the current device, looked up once per device
-// (host code cannot use the symbol itself: it names a host-side stand-in).
+// Device address of the array in the current context, looked up once per
+// context with that context current (host code cannot use the symbol itself: it
+// names a host-side stand-in).  Keyed on the context, not the device: after a
+// device reset the array is loaded again, possibly elsewhere, and the next call
+// looks it up afresh.  The cache is guarded by a mutex, so first calls from
+// several host threads are safe.
 int static_ws_address(void** out) {
-    static void* addr[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return HGD_ERR_CUDA; }
-    if (dev >= 0 && dev < 64 && addr[dev]) { *out = addr[dev]; return HGD_OK; }
+    static CtxCache<void*> addr;
     void* p = nullptr;
+    if (addr.get(current_ctx_id(), &p) && p) { *out = p; return HGD_OK; }
     if (cudaGetSymbolAddress(&p, g_gemv_static_ws) != cudaSuccess || !p) {
         cudaGetLastError();
         return HGD_ERR_CUDA;
     }
-    if (dev >= 0 && dev < 64) addr[dev] = p;
+    addr.put(current_ctx_id(), p);  // the lookup has made the context current if it was not
     *out = p;
     return HGD_OK;
 }

@@ -147,9 +147,11 @@ HGD_API int hgd_gemm_tc_bf16(const uint16_t* Wp, const uint16_t* x, float* y, in
  * Same inputs, output, shapes and results as hgd_gemv_bf16, but the split-K
  * scratch is a 4 MiB array built into the library, present on every device that
  * loads it until the process exits.  Nothing is allocated.
- *  - The first call on a device looks the array's device address up (once per
- *    device, with that device current); make that first call before capturing
- *    any stream into a CUDA graph.
+ *  - The first call in a CUDA context looks the array's device address up (once
+ *    per context, with that context current: once per device in the usual
+ *    runtime use, and again after a device reset, which starts a new context);
+ *    make that first call before capturing any stream into a CUDA graph.
+ *    Concurrent first calls from several host threads are safe.
  *  - A shape whose scratch would exceed 4 MiB returns HGD_ERR_BUFFER_TOO_SMALL
  *    and launches nothing (hgd_gemv_workspace_bytes tells the size needed).
  *  - Each call clears the part of the array that must start at zero (its

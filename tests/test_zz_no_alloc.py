@@ -68,9 +68,13 @@ def test_static_scratch_rejects_shapes_beyond_its_size(hgd):
     n = C.c_size_t()
     assert hgd._lib.hgd_gemv_workspace_bytes(M, N, K, 0, C.byref(n)) == 0
     assert n.value > (4 << 20)
-    W = torch.zeros((16, 32), dtype=torch.bfloat16, device="cuda")  # never read: rejected first
-    x = torch.zeros((1, 32), dtype=torch.bfloat16, device="cuda")
-    y = torch.zeros((1, 16), device="cuda")
+    # buffers of the declared shape (W is 268 MB), so that even if the size check
+    # ever stopped rejecting this shape, the launch would stay inside them
+    W = torch.zeros((N, K), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((M, N), 7.0, device="cuda")
     rc = hgd._lib.hgd_gemv_bf16_static_ws(W.data_ptr(), x.data_ptr(), y.data_ptr(), 1, M, N, K,
                                           torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
     assert rc == 9  # HGD_ERR_BUFFER_TOO_SMALL
+    assert bool((y == 7.0).all())  # a rejected call writes nothing
