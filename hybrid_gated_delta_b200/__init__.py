@@ -86,6 +86,8 @@ _SIGS = {
     "hgd_decode_layer_stack_range": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _i, _i, _i, _p, _p, _p,
                                       _p, _p, _p], _i),
     "hgd_decode_layer_stack_launches": ([C.POINTER(_Model), _i, _i], _i),
+    "hgd_check_stack_timeout": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _i, _i, _i, _p, _p, _p], _i),
+    "hgd_check_not_coresident": ([C.POINTER(_Model), C.POINTER(_State), _i], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -407,6 +409,25 @@ def decode_layer_stack_range(model: Model, state: State, tokens, T: int, layer_b
         C.byref(model.m), C.byref(state.st), _ptr(tokens), T, layer_begin, layer_end, int(run_head),
         _ptr(logits), _ptr(argmax), _ptr(S_rec), _ptr(tail_rec), _ptr(status), _stream(stream)))
     return argmax
+
+
+def check_stack_timeout(model: Model, state: State, tokens, T: int, skip_cta: int, skip_phase: int,
+                        wait_ms: int, status, report=None, argmax=None, stream=None):
+    """One persistent decode call in which CTA skip_cta leaves out its arrival at
+    phase skip_phase and phase waits are limited to wait_ms: HGD_ERR_TIMEOUT lands
+    in status, what ran out first in report (uint32 [4] device, or None)."""
+    torch = _torch()
+    if argmax is None:
+        argmax = torch.empty((state.B * T,), dtype=torch.int32, device=tokens.device)
+    _check("hgd_check_stack_timeout", _lib.hgd_check_stack_timeout(
+        C.byref(model.m), C.byref(state.st), _ptr(tokens), T, _ptr(argmax), skip_cta, skip_phase, wait_ms,
+        _ptr(status), _ptr(report), _stream(stream)))
+
+
+def check_not_coresident(model: Model, state: State, T: int) -> int:
+    """The status the persistent launch's co-residency check returns when the
+    device can hold none of its CTAs (HGD_ERR_NOT_CORESIDENT); nothing is run."""
+    return _lib.hgd_check_not_coresident(C.byref(model.m), C.byref(state.st), T)
 
 
 class DecodeGraph:

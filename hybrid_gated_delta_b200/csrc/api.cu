@@ -494,19 +494,23 @@ bool sk_supported(const Dims& d, int M) {
 }
 
 template <int KPL, int DPL>
-int sk_launch_t(const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
+int sk_launch_t(const SkParams& prm, size_t smem, int sms, cudaStream_t s, bool launch, int occ_override) {
     auto kern = k_stack<KPL, DPL>;
     static CtxCache<int> attr_done;
     if (ensure_smem_attr(kern, attr_done) != cudaSuccess) {
         cudaGetLastError();
         return HGD_ERR_CUDA;
     }
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, SK_THREADS, smem) != cudaSuccess) {
-        cudaGetLastError();
-        return HGD_ERR_CUDA;
+    if (!launch) {
+        // every CTA must be resident at once: the phases wait on one another
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, SK_THREADS, smem) != cudaSuccess) {
+            cudaGetLastError();
+            return HGD_ERR_CUDA;
+        }
+        if (occ_override >= 0) occ = occ_override;
+        return occ < 1 ? HGD_ERR_NOT_CORESIDENT : HGD_OK;
     }
-    if (occ < 1) return HGD_ERR_NOT_CORESIDENT;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(SK_THREADS);
@@ -522,20 +526,23 @@ int sk_launch_t(const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
 
 // The persistent kernel for this model's GDN key width (64 or 128) and
 // attention head width (32, 64, 128 or 256).
-int sk_launch(const Dims& d, const SkParams& prm, size_t smem, int sms, cudaStream_t s) {
+// launch = false: only the co-residency check (occ_override >= 0 stands in for
+// the occupancy the runtime reports); launch = true: the cooperative launch.
+int sk_launch(const Dims& d, const SkParams& prm, size_t smem, int sms, cudaStream_t s, bool launch,
+              int occ_override = -1) {
     if (d.dk == 128) {
         switch (d.hd) {
-            case 256: return sk_launch_t<4, 8>(prm, smem, sms, s);
-            case 128: return sk_launch_t<4, 4>(prm, smem, sms, s);
-            case 64: return sk_launch_t<4, 2>(prm, smem, sms, s);
-            default: return sk_launch_t<4, 1>(prm, smem, sms, s);
+            case 256: return sk_launch_t<4, 8>(prm, smem, sms, s, launch, occ_override);
+            case 128: return sk_launch_t<4, 4>(prm, smem, sms, s, launch, occ_override);
+            case 64: return sk_launch_t<4, 2>(prm, smem, sms, s, launch, occ_override);
+            default: return sk_launch_t<4, 1>(prm, smem, sms, s, launch, occ_override);
         }
     }
     switch (d.hd) {
-        case 256: return sk_launch_t<2, 8>(prm, smem, sms, s);
-        case 128: return sk_launch_t<2, 4>(prm, smem, sms, s);
-        case 64: return sk_launch_t<2, 2>(prm, smem, sms, s);
-        default: return sk_launch_t<2, 1>(prm, smem, sms, s);
+        case 256: return sk_launch_t<2, 8>(prm, smem, sms, s, launch, occ_override);
+        case 128: return sk_launch_t<2, 4>(prm, smem, sms, s, launch, occ_override);
+        case 64: return sk_launch_t<2, 2>(prm, smem, sms, s, launch, occ_override);
+        default: return sk_launch_t<2, 1>(prm, smem, sms, s, launch, occ_override);
     }
 }
 
@@ -608,6 +615,73 @@ __global__ void k_check_bounded_wait(int32_t* status) {
     }
     __syncthreads();
     if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0u, nullptr)) set_status(status, HGD_ERR_TIMEOUT);
+}
+
+// Diagnostic settings of one persistent launch (defaults: none).
+struct SkDebug {
+    unsigned long long wait_ns = kWaitLimitNs;
+    int skip_cta = -1, skip_phase = -1;
+};
+
+// One call through the persistent launch: parameters, co-residency check, fresh
+// control words, launch.  Nothing is enqueued if the check fails.
+int sk_run(const hgd_model* m, const hgd_state* st, const Dims& d, const int32_t* tokens, int T, float* logits,
+           int32_t* argmax, float* S_rec, float* tail_rec, int32_t* status_dev, cudaStream_t s,
+           const SkDebug& dbg) {
+    int rc;
+    if (!al16(tokens) || !al16(argmax) || (logits && !al16(logits)) || (S_rec && !al16(S_rec)) ||
+        (tail_rec && !al16(tail_rec)))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    uint8_t* A = static_cast<uint8_t*>(st->arena);
+    SkParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.L = d.L; prm.D = d.D; prm.V = d.V; prm.H = d.H; prm.dk = d.dk; prm.dv = d.dv; prm.nq = d.nq;
+    prm.nkv = d.nkv; prm.hd = d.hd; prm.I = d.I; prm.every = d.every;
+    prm.C = (int)d.C; prm.gdn_out = (int)d.gdn_out; prm.attn_out = (int)d.attn_out;
+    prm.proj_ld = (int)std::max(d.gdn_out, d.attn_out); prm.kmax = sk_kmax(d);
+    prm.eps = m->cfg.norm_eps; prm.rope_inv1 = rope_inv1_of(d, m->cfg.rope_base);
+    prm.B = st->B; prm.T = T; prm.M = st->B * T; prm.Lmax = st->Lmax; prm.max_chunks = max_chunks_of(st->Lmax);
+    prm.ns = sk_ring_slots(d, prm.M); prm.pb = kSkPartialSlabs;
+    prm.embed = m->embed; prm.final_norm = m->final_norm;
+    prm.S = reinterpret_cast<float*>(A + st->off[SC_S]);
+    prm.conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
+    prm.kv = reinterpret_cast<bf16_t*>(A + st->off[SC_KV]);
+    prm.pos = reinterpret_cast<int32_t*>(A + st->off[SC_POS]);
+    prm.resid = reinterpret_cast<bf16_t*>(A + st->off[SC_RESID]);
+    prm.proj = reinterpret_cast<float*>(A + st->off[SC_PROJ]);
+    prm.obuf = reinterpret_cast<float*>(A + st->off[SC_O]);
+    prm.qrot = reinterpret_cast<float*>(A + st->off[SC_QROT]);
+    prm.part = reinterpret_cast<float*>(A + st->off[SC_PART]);
+    prm.mlp = reinterpret_cast<bf16_t*>(A + st->off[SC_MLP]);
+    prm.attn = reinterpret_cast<bf16_t*>(A + st->off[SC_ATTN]);
+    prm.bestv = reinterpret_cast<float*>(A + st->off[SC_BESTV]);
+    prm.besti = reinterpret_cast<int32_t*>(A + st->off[SC_BESTI]);
+    prm.tokens = tokens; prm.logits = logits; prm.argmax = argmax; prm.S_rec = S_rec; prm.tail_rec = tail_rec;
+    prm.status = status_dev;
+    prm.bar = reinterpret_cast<unsigned*>(A + st->off[SC_BAR]);
+    prm.mcnt = prm.bar + SK_CTRL_WORDS;
+    prm.trace = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarTraceOff);
+#ifdef HGD_TRACE_DETAIL
+    prm.tdetail = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarDetailOff);
+    prm.tslab = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarSlabOff);
+#endif
+    for (int l = 0; l < d.L; ++l)
+        for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) prm.layer[l].w[t] = m->w[l][t];
+    prm.wait_ns = dbg.wait_ns;
+    prm.dbg_skip_cta = dbg.skip_cta;
+    prm.dbg_skip_phase = dbg.skip_phase;
+    const size_t smem = sk_smem_bytes(d, prm.M, prm.ns);
+    if ((rc = sk_launch(d, prm, smem, di.sms, s, false))) return rc;
+    // fresh control words and phase counters for this call (an earlier call may
+    // have stopped on a timeout)
+    const size_t nph = (size_t)d.L * SK_PHASES_PER_LAYER + 2;
+    if (cudaMemsetAsync(prm.bar, 0, kBarCtrlBytes + nph * SK_CTR_STRIDE * 4, s) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
+    }
+    return sk_launch(d, prm, smem, di.sms, s, true);
 }
 
 }  // namespace
@@ -934,56 +1008,57 @@ int hgd_decode_layer_stack(const hgd_model* m, const hgd_state* st, const int32_
     if (!sk_supported(d, st->B * T))
         return hgd_decode_layer_stack_range(m, st, tokens, T, 0, m->cfg.n_layers, 1, logits, argmax, S_rec,
                                             tail_rec, status_dev, stream);
-    if (!al16(tokens) || !al16(argmax) || (logits && !al16(logits)) || (S_rec && !al16(S_rec)) ||
-        (tail_rec && !al16(tail_rec)))
-        return HGD_ERR_MISALIGNED;
+    return sk_run(m, st, d, tokens, T, logits, argmax, S_rec, tail_rec, status_dev, (cudaStream_t)stream,
+                  SkDebug{});
+}
+
+int hgd_check_stack_timeout(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,
+                            int32_t* argmax, int skip_cta, int skip_phase, int wait_ms, int32_t* status_dev,
+                            uint32_t* report_dev, hgd_stream_t stream) {
+    if (!m || !st || !st->arena || !tokens || !argmax || !status_dev) return HGD_ERR_INVALID_ARG;
+    if (T < 1 || T > st->Tmax || skip_cta < 0 || skip_phase < 0 || wait_ms < 1 || wait_ms > 2000)
+        return HGD_ERR_INVALID_ARG;
+    if (report_dev && !al16(report_dev)) return HGD_ERR_MISALIGNED;
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if (!sk_supported(d, st->B * T)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (skip_phase > d.L * SK_PHASES_PER_LAYER) return HGD_ERR_INVALID_ARG;  // the LM head phase at most
     DevInfo di;
     if ((rc = device_info(&di))) return rc;
-    uint8_t* A = static_cast<uint8_t*>(st->arena);
-    SkParams prm;
-    std::memset(&prm, 0, sizeof(prm));
-    prm.L = d.L; prm.D = d.D; prm.V = d.V; prm.H = d.H; prm.dk = d.dk; prm.dv = d.dv; prm.nq = d.nq;
-    prm.nkv = d.nkv; prm.hd = d.hd; prm.I = d.I; prm.every = d.every;
-    prm.C = (int)d.C; prm.gdn_out = (int)d.gdn_out; prm.attn_out = (int)d.attn_out;
-    prm.proj_ld = (int)std::max(d.gdn_out, d.attn_out); prm.kmax = sk_kmax(d);
-    prm.eps = m->cfg.norm_eps; prm.rope_inv1 = rope_inv1_of(d, m->cfg.rope_base);
-    prm.B = st->B; prm.T = T; prm.M = st->B * T; prm.Lmax = st->Lmax; prm.max_chunks = max_chunks_of(st->Lmax);
-    prm.ns = sk_ring_slots(d, prm.M); prm.pb = kSkPartialSlabs;
-    prm.embed = m->embed; prm.final_norm = m->final_norm;
-    prm.S = reinterpret_cast<float*>(A + st->off[SC_S]);
-    prm.conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
-    prm.kv = reinterpret_cast<bf16_t*>(A + st->off[SC_KV]);
-    prm.pos = reinterpret_cast<int32_t*>(A + st->off[SC_POS]);
-    prm.resid = reinterpret_cast<bf16_t*>(A + st->off[SC_RESID]);
-    prm.proj = reinterpret_cast<float*>(A + st->off[SC_PROJ]);
-    prm.obuf = reinterpret_cast<float*>(A + st->off[SC_O]);
-    prm.qrot = reinterpret_cast<float*>(A + st->off[SC_QROT]);
-    prm.part = reinterpret_cast<float*>(A + st->off[SC_PART]);
-    prm.mlp = reinterpret_cast<bf16_t*>(A + st->off[SC_MLP]);
-    prm.attn = reinterpret_cast<bf16_t*>(A + st->off[SC_ATTN]);
-    prm.bestv = reinterpret_cast<float*>(A + st->off[SC_BESTV]);
-    prm.besti = reinterpret_cast<int32_t*>(A + st->off[SC_BESTI]);
-    prm.tokens = tokens; prm.logits = logits; prm.argmax = argmax; prm.S_rec = S_rec; prm.tail_rec = tail_rec;
-    prm.status = status_dev;
-    prm.bar = reinterpret_cast<unsigned*>(A + st->off[SC_BAR]);
-    prm.mcnt = prm.bar + SK_CTRL_WORDS;
-    prm.trace = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarTraceOff);
-#ifdef HGD_TRACE_DETAIL
-    prm.tdetail = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarDetailOff);
-    prm.tslab = reinterpret_cast<unsigned long long*>(A + st->off[SC_BAR] + kBarSlabOff);
-#endif
-    for (int l = 0; l < d.L; ++l)
-        for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) prm.layer[l].w[t] = m->w[l][t];
+    if (skip_cta >= di.sms) return HGD_ERR_INVALID_ARG;
+    SkDebug dbg;
+    dbg.wait_ns = (unsigned long long)wait_ms * 1000000ull;
+    dbg.skip_cta = skip_cta;
+    dbg.skip_phase = skip_phase;
     cudaStream_t s = (cudaStream_t)stream;
-    // fresh control words and phase counters for this call (an earlier call may
-    // have stopped on a timeout)
-    const size_t nph = (size_t)d.L * SK_PHASES_PER_LAYER + 2;
-    if (cudaMemsetAsync(prm.bar, 0, kBarCtrlBytes + nph * SK_CTR_STRIDE * 4, s) != cudaSuccess) {
+    rc = sk_run(m, st, d, tokens, T, nullptr, argmax, nullptr, nullptr, status_dev, s, dbg);
+    if (rc || !report_dev) return rc;
+    // what ran out first, its phase and its CTA: control words 1..3
+    const uint8_t* A = static_cast<const uint8_t*>(st->arena);
+    if (cudaMemsetAsync(report_dev, 0, 16, s) != cudaSuccess ||
+        cudaMemcpyAsync(report_dev, A + st->off[SC_BAR] + 4, 12, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
         cudaGetLastError();
         return HGD_ERR_CUDA;
     }
-    const size_t smem = sk_smem_bytes(d, prm.M, prm.ns);
-    return sk_launch(d, prm, smem, di.sms, s);
+    return HGD_OK;
+}
+
+int hgd_check_not_coresident(const hgd_model* m, const hgd_state* st, int T) {
+    if (!m || !st || !st->arena) return HGD_ERR_INVALID_ARG;
+    if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if (!sk_supported(d, st->B * T)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    const int M = st->B * T;
+    SkParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    return sk_launch(d, prm, sk_smem_bytes(d, M, sk_ring_slots(d, M)), di.sms, nullptr, false, 0);
 }
 
 int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,

@@ -85,6 +85,8 @@ struct SkParams {
     unsigned long long* trace;   // [SK_TRACE_SLOTS] %globaltimer, or null
     unsigned long long* tdetail; // [SK_MAX_PHASES][SK_TRACE_CTAS][8] per-CTA phase times, or null
     unsigned long long* tslab;   // CTA 0: [SK_TRACE_SLABS][4] slab issue / ready / release / wait-start times, or null
+    unsigned long long wait_ns;  // limit of each phase wait (kWaitLimitNs in normal calls)
+    int dbg_skip_cta, dbg_skip_phase;  // diagnostic: this CTA leaves out its arrival at this phase (-1: none)
     SkLayer layer[HGD_MAX_LAYERS];
 };
 
@@ -132,7 +134,8 @@ __device__ __forceinline__ void sk_timeout(const SkParams& s, unsigned what, uns
 // phase's counter.
 __device__ __forceinline__ void sk_arrive(const SkParams& s, int p) {
     named_bar(1, SK_CT);
-    if (threadIdx.x == 0) red_release_add(sk_ctr(s, p), 1u);
+    if (threadIdx.x == 0 && !((int)blockIdx.x == s.dbg_skip_cta && p == s.dbg_skip_phase))
+        red_release_add(sk_ctr(s, p), 1u);
 }
 
 // Named barrier over the consumer threads that also ANDs a predicate: every
@@ -168,7 +171,7 @@ __device__ bool sk_wait(const SkParams& s, volatile int* cta_abort, volatile int
             while (*seen != p && ld_acquire_u32(c) < target) {
                 if ((++it & 31u) == 0u) {
                     if (ld_acquire_u32(&s.bar[0])) { *cta_abort = 1; break; }
-                    if (globaltimer() - t0 > kWaitLimitNs) {
+                    if (globaltimer() - t0 > s.wait_ns) {
                         if (warp == 0) sk_timeout(s, 1u, (unsigned)p, 0u);
                         *cta_abort = 1;
                         break;

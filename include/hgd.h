@@ -359,6 +359,31 @@ HGD_API int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st
  * T rows issues (-1 on bad arguments). */
 HGD_API int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T);
 
+/* ------------------------------------------------------ stack diagnostics --
+ * The same check on the persistent decode launch itself ([LUCE] Known issues:
+ * a grid-wide wait that can never complete deadlocks the whole kernel).  One
+ * hgd_decode_layer_stack call over T rows that takes the persistent launch, in
+ * which CTA `skip_cta` leaves out its arrival at the end of phase `skip_phase`
+ * (phases count from 0: five per layer, then the LM head) and every phase wait
+ * is limited to `wait_ms` (1..2000) instead of 2 s.  The waits for that phase
+ * then run out: the kernel writes HGD_ERR_TIMEOUT to *status_dev (zero it
+ * first), and every CTA skips the rest of the call, so the call ends.
+ * report_dev (device uint32[4], 16-byte aligned, or NULL) receives what ran out
+ * first {1 = a phase counter, 2 = a weight slab, 3 = a ring slot}, its phase,
+ * the CTA that saw it, and 0.  The call leaves the state partly advanced (the
+ * phases before the skipped arrival ran; positions do not advance) and argmax
+ * unwritten: restore the state before decoding on.  HGD_ERR_UNSUPPORTED_SHAPE
+ * if the call would not take the persistent launch. */
+HGD_API int hgd_check_stack_timeout(const hgd_model* m, const hgd_state* st, const int32_t* tokens,
+                                    int T, int32_t* argmax, int skip_cta, int skip_phase, int wait_ms,
+                                    int32_t* status_dev, uint32_t* report_dev, hgd_stream_t stream);
+
+/* The persistent launch's co-residency refusal: runs the host-side check that
+ * precedes every persistent launch with the occupancy query's answer replaced
+ * by zero resident CTAs per SM, and returns what hgd_decode_layer_stack returns
+ * then (HGD_ERR_NOT_CORESIDENT).  Enqueues nothing. */
+HGD_API int hgd_check_not_coresident(const hgd_model* m, const hgd_state* st, int T);
+
 #ifdef __cplusplus
 }
 #endif

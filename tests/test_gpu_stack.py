@@ -463,3 +463,57 @@ def test_windows_every_layer_vs_oracle(hgd, orc, full):
     st = hgd.State(model, B, T, Lmax)
     worst = _per_layer_check(hgd, model, st, r, pre, toks, T, "window")
     assert worst["S"] <= 1e-4
+
+
+# ------------------------------------------------- failure detection --------
+
+@pytest.mark.parametrize("skip_phase", [0, 6, 20])
+def test_persistent_phase_wait_runs_out_and_context_survives(hgd, skip_phase):
+    """The persistent launch's own bounded phase wait ("luce-megakernel HANDOFF.md",
+    Known issues: a grid-wide wait that never completes deadlocks the kernel):
+    CTA 5 leaves out its arrival at the end of one phase (layer 0's in-projection,
+    layer 1's gated delta rule, the LM head) and waits are limited to 50 ms.  The
+    call ends with HGD_ERR_TIMEOUT in the status word and a report of the phase
+    whose counter ran out; afterwards persistent calls on the same context still
+    equal the kernel chain bit for bit."""
+    import time
+    import torch
+    cfg = syn.SMALL_CFG
+    model = hgd.Model(cfg, weights("small", 5))
+    B, T, Lmax = 1, 1, 40
+    st = hgd.State(model, B, T, Lmax, syn.stack_state(cfg, B, Lmax, prefill=16, seed=6))
+    assert model.launches(B, T) == 1
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    report = torch.full((4,), 0xAB, dtype=torch.int32, device="cuda")
+    tok = torch.tensor([[3]], dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    hgd.check_stack_timeout(model, st, tok, T, 5, skip_phase, 50, status, report)
+    torch.cuda.synchronize()
+    dt = time.time() - t0
+    rep = report.cpu().tolist()
+    assert int(status.item()) == 5, hgd.status_string(int(status.item()))  # HGD_ERR_TIMEOUT
+    assert rep[0] == 1 and rep[1] == skip_phase and 0 <= rep[2] < torch.cuda.get_device_properties(0).multi_processor_count
+    assert rep[3] == 0
+    assert dt < 10.0
+    assert host(st.pos).tolist() == [16]  # the final phase did not run
+    # the context is usable: persistent calls still equal the chain
+    (rp, sp), (rc, sc) = _run_paths(hgd, model, cfg, 2, 3, 40, 2, 13)
+    _assert_paths_equal(rp, sp, rc, sc)
+
+
+def test_not_coresident_is_refused_on_the_host(hgd):
+    """With the occupancy query's answer replaced by zero resident CTAs, the
+    persistent launch's check returns HGD_ERR_NOT_CORESIDENT and enqueues nothing."""
+    import torch
+    cfg = syn.SMALL_CFG
+    model = hgd.Model(cfg, weights("small", 5))
+    st = hgd.State(model, 1, 1, 40, syn.stack_state(cfg, 1, 40, prefill=16, seed=6))
+    snap = st.snapshot()
+    assert hgd.check_not_coresident(model, st, 1) == 6
+    torch.cuda.synchronize()
+    for k, v in snap.items():
+        assert torch.equal(v, getattr(st, k))
+    # and the real check passes on this device
+    am = hgd.decode_layer_stack(model, st, torch.tensor([[3]], dtype=torch.int32, device="cuda"), 1)
+    torch.cuda.synchronize()
+    assert 0 <= int(am.item()) < cfg["vocab"]
