@@ -75,6 +75,9 @@ _SIGS = {
     "hgd_gemm_tc_bf16": ([_p, _p, _p, _i, _i, _i, _p, _sz, _p, _p], _i),
     "hgd_conv1d_tail_update": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
+    "hgd_gdn_window_log": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
+    "hgd_gdn_keep": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
+    "hgd_conv1d_keep": ([_p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
     "hgd_model_arena_bytes": ([C.POINTER(Config), C.POINTER(_sz)], _i),
     "hgd_model_tensor": ([C.POINTER(Config), _i, _i, C.POINTER(_sz), C.POINTER(_sz)], _i),
     "hgd_model_init": ([C.POINTER(_Model), C.POINTER(Config), _p, _sz], _i),
@@ -86,6 +89,9 @@ _SIGS = {
     "hgd_decode_layer_stack_range": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _i, _i, _i, _p, _p, _p,
                                       _p, _p, _p], _i),
     "hgd_decode_layer_stack_launches": ([C.POINTER(_Model), _i, _i], _i),
+    "hgd_verify_log_bytes": ([C.POINTER(Config), _i, _i, C.POINTER(_sz)], _i),
+    "hgd_decode_layer_stack_verify": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _p, _p, _sz, _p, _p], _i),
+    "hgd_decode_layer_stack_keep": ([C.POINTER(_Model), C.POINTER(_State), _i, _p, _sz, _p, _p, _p], _i),
     "hgd_check_stack_timeout": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _i, _i, _i, _p, _p, _p], _i),
     "hgd_check_not_coresident": ([C.POINTER(_Model), C.POINTER(_State), _i], _i),
 }
@@ -269,6 +275,55 @@ def gdn_decode_step(q, k, v, g, b, S, o=None, o_bf16=None, S_rec=None, l2norm_qk
     return o
 
 
+def gdn_window_log(q, k, v, g, b, S, o=None, o_bf16=None, l2norm_qk=True, row_stride=None, B=None, T=None,
+                   stream=None):
+    """The rows of gdn_decode_step with S only read; returns (o, log_alpha [B,T,H],
+    log_delta [B,T,H,dv], log_k [B,T,H,dk])."""
+    torch = _torch()
+    _need(S, torch.float32, "S")
+    Bs, H, dv, dk = S.shape
+    Tn = g.shape[1] if T is None else T
+    Bn = Bs if B is None else B
+    if row_stride is None:
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _need(t, torch.float32, n)
+            if not t.is_contiguous():
+                raise ValueError(f"{n} must be contiguous")
+        row_stride = H * dk
+    dev = S.device
+    if o is None:
+        o = torch.empty((Bn, Tn, H, dv), dtype=torch.float32, device=dev)
+    la = torch.empty((Bn, Tn, H), dtype=torch.float32, device=dev)
+    ld = torch.empty((Bn, Tn, H, dv), dtype=torch.float32, device=dev)
+    lk = torch.empty((Bn, Tn, H, dk), dtype=torch.float32, device=dev)
+    _check("hgd_gdn_window_log", _lib.hgd_gdn_window_log(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), int(row_stride), _ptr(g), _ptr(b), _ptr(S), _ptr(o),
+        _ptr(o_bf16), _ptr(la), _ptr(ld), _ptr(lk), Bn, Tn, H, dk, dv, int(l2norm_qk), _stream(stream)))
+    return o, la, ld, lk
+
+
+def gdn_keep(S, log_alpha, log_delta, log_k, keep, status=None, stream=None):
+    """S [B,H,dv,dk] takes the first keep[b] logged rows of each stream (keep: int32 [B] device)."""
+    torch = _torch()
+    _need(S, torch.float32, "S")
+    _need(keep, torch.int32, "keep")
+    B, H, dv, dk = S.shape
+    T = log_alpha.shape[1]
+    _check("hgd_gdn_keep", _lib.hgd_gdn_keep(_ptr(S), _ptr(log_alpha), _ptr(log_delta), _ptr(log_k), _ptr(keep),
+                                             _ptr(status), B, T, H, dk, dv, _stream(stream)))
+
+
+def conv1d_keep(tail, x, keep, status=None, stream=None):
+    """tail [B,kc-1,C] takes the first keep[b] rows of x [B,T,C]."""
+    torch = _torch()
+    _need(tail, torch.float32, "tail")
+    _need(x, torch.float32, "x")
+    _need(keep, torch.int32, "keep")
+    B, nt, Cc = tail.shape
+    _check("hgd_conv1d_keep", _lib.hgd_conv1d_keep(_ptr(tail), _ptr(x), _ptr(keep), _ptr(status), B, x.shape[1],
+                                                   Cc, nt + 1, _stream(stream)))
+
+
 # ------------------------------------------------------------------ stack
 
 def make_config(cfg: dict) -> Config:
@@ -409,6 +464,41 @@ def decode_layer_stack_range(model: Model, state: State, tokens, T: int, layer_b
         C.byref(model.m), C.byref(state.st), _ptr(tokens), T, layer_begin, layer_end, int(run_head),
         _ptr(logits), _ptr(argmax), _ptr(S_rec), _ptr(tail_rec), _ptr(status), _stream(stream)))
     return argmax
+
+
+class VerifyLog:
+    """Device memory for the logs of one verify call of T rows per stream."""
+
+    def __init__(self, model: Model, B: int, T: int, device="cuda"):
+        torch = _torch()
+        n = C.c_size_t()
+        _check("hgd_verify_log_bytes", _lib.hgd_verify_log_bytes(C.byref(model.cfg), B, T, C.byref(n)))
+        self.B, self.T, self.nbytes = B, T, n.value
+        self.buf = torch.empty(n.value + 256, dtype=torch.uint8, device=device)
+        pad = (-self.buf.data_ptr()) % 256
+        self.ptr = self.buf.data_ptr() + pad
+
+
+def decode_layer_stack_verify(model: Model, state: State, tokens, T: int, log: VerifyLog, logits=None,
+                              argmax=None, status=None, stream=None):
+    """A verify window: logits/argmax as decode_layer_stack; the state is left as it
+    was and the rows are logged in `log`.  Returns argmax [B*T]."""
+    torch = _torch()
+    _need(tokens, torch.int32, "tokens")
+    if argmax is None:
+        argmax = torch.empty((state.B * T,), dtype=torch.int32, device=tokens.device)
+    _check("hgd_decode_layer_stack_verify", _lib.hgd_decode_layer_stack_verify(
+        C.byref(model.m), C.byref(state.st), _ptr(tokens), T, _ptr(logits), _ptr(argmax), log.ptr, log.nbytes,
+        _ptr(status), _stream(stream)))
+    return argmax
+
+
+def decode_layer_stack_keep(model: Model, state: State, T: int, log: VerifyLog, keep, status=None, stream=None):
+    """Stream b keeps the first keep[b] rows of the verify call logged in `log`."""
+    torch = _torch()
+    _need(keep, torch.int32, "keep")
+    _check("hgd_decode_layer_stack_keep", _lib.hgd_decode_layer_stack_keep(
+        C.byref(model.m), C.byref(state.st), T, log.ptr, log.nbytes, _ptr(keep), _ptr(status), _stream(stream)))
 
 
 def check_stack_timeout(model: Model, state: State, tokens, T: int, skip_cta: int, skip_phase: int,

@@ -424,6 +424,40 @@ constexpr int kBestG = 4096;  // max CTAs of the LM-head launch
 
 int max_chunks_of(int Lmax) { return (Lmax + ATTN_CHUNK - 1) / ATTN_CHUNK; }
 
+// A verify window's log (hgd_decode_layer_stack_verify): the copy of the conv
+// tails the window runs on, then per GDN layer the rows' decay [B][T][H], write
+// [B][T][H][dv], key [B][T][H][dk] and conv input [B][T][C] (fp32, each region
+// 256-byte aligned).
+struct VerifyLayout {
+    size_t conv, alpha, delta, k, x, per_layer, first, total;
+    size_t layer(int ig) const { return first + (size_t)ig * per_layer; }
+};
+VerifyLayout verify_layout(const Dims& d, int B, int T) {
+    VerifyLayout v{};
+    const size_t rows = (size_t)B * T;
+    v.conv = 0;
+    v.first = al256((size_t)d.n_gdn * B * (d.kc - 1) * d.C * 4);
+    v.alpha = 0;
+    v.delta = v.alpha + al256(rows * d.H * 4);
+    v.k = v.delta + al256(rows * d.H * d.dv * 4);
+    v.x = v.k + al256(rows * d.H * d.dk * 4);
+    v.per_layer = v.x + al256(rows * d.C * 4);
+    v.total = v.first + (size_t)d.n_gdn * v.per_layer;
+    return v;
+}
+
+// keep's position advance: pos[b] += keep[b] for every stream whose count is in
+// [0, T] (the others are reported and left).
+__global__ void k_pos_keep(int32_t* pos, const int32_t* keep, int32_t* status, int B, int T) {
+    pdl_launch();
+    pdl_wait();
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const int n = keep[b];
+        if (n < 0 || n > T) set_status(status, HGD_ERR_INVALID_ARG);
+        else pos[b] += n;
+    }
+}
+
 // Split-K workspace of the stack: the largest any of its GEMVs uses at M rows.
 size_t stack_ws_bytes(const Dims& d, int M) {
     size_t w = 0;
@@ -836,6 +870,77 @@ int hgd_gdn_decode_step(const float* q, const float* k, const float* v, int64_t 
     return launch_status(e);
 }
 
+// ------------------------------------------------- recurrence logs, keep
+
+int hgd_gdn_window_log(const float* q, const float* k, const float* v, int64_t row_stride, const float* g,
+                       const float* b, const float* S, float* o, uint16_t* o_bf16, float* log_alpha,
+                       float* log_delta, float* log_k, int B, int T, int H, int dk, int dv, int l2norm_qk,
+                       hgd_stream_t stream) {
+    if (!q || !k || !v || !g || !b || !S || !o || !log_alpha || !log_delta || !log_k || B < 1 || T < 1 ||
+        H < 1 || dk < 1 || dv < 1)
+        return HGD_ERR_INVALID_ARG;
+    if (!(dk == 32 || dk == 64 || dk == 128 || dk == 256) || dv % GDN_ROWS != 0 || dv > 1024)
+        return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (row_stride < (int64_t)H * dk || row_stride < (int64_t)H * dv) return HGD_ERR_INVALID_ARG;
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(g) || !al16(b) || !al16(S) || !al16(o) ||
+        (o_bf16 && !al16(o_bf16)) || !al16(log_alpha) || !al16(log_delta) || !al16(log_k))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    GdnLogParams p{q, k, v, row_stride, g, b, S, o, o_bf16, log_alpha, log_delta, log_k,
+                   B, T, H, dk, dv, l2norm_qk ? 1 : 0};
+    const dim3 grid(B * H, dv / GDN_ROWS), block(GDN_WARPS * 32);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    switch (dk) {
+        case 32: e = launch_pdl(k_gdn_window_log<1>, grid, block, 0, s, p); break;
+        case 64: e = launch_pdl(k_gdn_window_log<2>, grid, block, 0, s, p); break;
+        case 128: e = launch_pdl(k_gdn_window_log<4>, grid, block, 0, s, p); break;
+        default: e = launch_pdl(k_gdn_window_log<8>, grid, block, 0, s, p); break;
+    }
+    return launch_status(e);
+}
+
+int hgd_gdn_keep(float* S, const float* log_alpha, const float* log_delta, const float* log_k,
+                 const int32_t* keep, int32_t* status_dev, int B, int T, int H, int dk, int dv, hgd_stream_t stream) {
+    if (!S || !log_alpha || !log_delta || !log_k || !keep || B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1)
+        return HGD_ERR_INVALID_ARG;
+    if (!(dk == 32 || dk == 64 || dk == 128 || dk == 256) || dv % GDN_ROWS != 0 || dv > 1024)
+        return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(S) || !al16(log_alpha) || !al16(log_delta) || !al16(log_k) || !al16(keep) ||
+        (status_dev && !al16(status_dev)))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    GdnKeepParams p{S, log_alpha, log_delta, log_k, keep, status_dev, B, T, H, dv};
+    const dim3 grid(B * H, dv / GDN_ROWS), block(GDN_WARPS * 32);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    switch (dk) {
+        case 32: e = launch_pdl(k_gdn_keep<1>, grid, block, 0, s, p); break;
+        case 64: e = launch_pdl(k_gdn_keep<2>, grid, block, 0, s, p); break;
+        case 128: e = launch_pdl(k_gdn_keep<4>, grid, block, 0, s, p); break;
+        default: e = launch_pdl(k_gdn_keep<8>, grid, block, 0, s, p); break;
+    }
+    return launch_status(e);
+}
+
+int hgd_conv1d_keep(float* tail, const float* x, const int32_t* keep, int32_t* status_dev, int B, int T, int C,
+                    int kc, hgd_stream_t stream) {
+    if (!tail || !x || !keep || B < 1 || T < 1 || C < 1) return HGD_ERR_INVALID_ARG;
+    if (kc < 2 || kc > 8) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(tail) || !al16(x) || !al16(keep) || (status_dev && !al16(status_dev))) return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    ConvKeepParams p{tail, x, keep, status_dev, B, T, C, kc};
+    const int64_t n = (int64_t)B * C;
+    return launch_status(launch_pdl(k_conv_keep, dim3((unsigned)((n + 255) / 256)), dim3(256), 0,
+                                    (cudaStream_t)stream, p));
+}
+
 // ---------------------------------------------------------------- stack
 
 int hgd_model_arena_bytes(const hgd_config* cfg, size_t* bytes) {
@@ -1061,9 +1166,13 @@ int hgd_check_not_coresident(const hgd_model* m, const hgd_state* st, int T) {
     return sk_launch(d, prm, sk_smem_bytes(d, M, sk_ring_slots(d, M)), di.sms, nullptr, false, 0);
 }
 
-int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,
-                                 int layer_begin, int layer_end, int run_head, float* logits, int32_t* argmax,
-                                 float* S_rec, float* tail_rec, int32_t* status_dev, hgd_stream_t stream) {
+// The kernel chain of layers [layer_begin, layer_end) and, if run_head, the head.
+// With vl (a verify window): the conv runs on the log's copy of the tails and
+// logs each row's conv input, the GDN layers log (alpha, delta, k) instead of
+// writing the state, and the head leaves the positions as they are.
+static int chain_run(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T, int layer_begin,
+                     int layer_end, int run_head, float* logits, int32_t* argmax, float* S_rec, float* tail_rec,
+                     int32_t* status_dev, hgd_stream_t stream, uint8_t* vl) {
     if (!m || !st || !st->arena) return HGD_ERR_INVALID_ARG;
     if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
     Dims d;
@@ -1112,6 +1221,7 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
     const size_t kv_half = (size_t)B * d.nkv * Lmax * d.hd;
     const size_t srec_layer = (size_t)B * T * d.H * d.dv * d.dk;
     const size_t trec_layer = (size_t)B * T * (d.kc - 1) * d.C;
+    const VerifyLayout vlay = verify_layout(d, B, T);
     int ig = 0, ia = 0;
     for (int l = 0; l < layer_begin; ++l) (is_attn_layer(&m->cfg, l) ? ia : ig)++;
     for (int l = layer_begin; l < layer_end; ++l) {
@@ -1140,6 +1250,10 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             if (!att) {
                 p.conv_w = w[HGD_W_CONV]; p.conv_tail = conv + ig * c_layer;
                 p.conv_rec = tail_rec ? tail_rec + ig * trec_layer : nullptr;
+                if (vl) {
+                    p.conv_tail = reinterpret_cast<float*>(vl + vlay.conv) + ig * c_layer;
+                    p.conv_xlog = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.x);
+                }
                 p.conv_C = (int)d.C; p.conv_T = T;
                 rc = many     ? run_gemv<PRO_COPY, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s)
                      : (l == 0) ? run_gemv<PRO_EMBED_RMSNORM, EPI_QKV_CONV>(p, M, di.sms, ws, ws_bytes, s)
@@ -1159,6 +1273,11 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             g.o = obuf; g.o_ld = (int64_t)d.H * d.dv;
             g.S_rec = S_rec ? S_rec + ig * srec_layer : nullptr;
             g.B = B; g.T = T; g.H = d.H; g.dv = d.dv;
+            if (vl) {
+                g.log_alpha = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.alpha);
+                g.log_delta = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.delta);
+                g.log_k = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.k);
+            }
             const dim3 grid(B * d.H, d.dv / GDN_ROWS), block(GDN_WARPS * 32);
             cudaError_t e;
             switch (d.dk) {
@@ -1241,10 +1360,98 @@ int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const 
             return rc;
         }
         cudaError_t e = launch_pdl(k_argmax_finalize, dim3(M), dim3(128), 0, s, (const float*)bestv,
-                                   (const int32_t*)besti, G, M, argmax, status_dev, pos, B, T);
+                                   (const int32_t*)besti, G, M, argmax, status_dev, vl ? nullptr : pos, B, T);
         if ((rc = launch_status(e))) return rc;
     }
     return HGD_OK;
+}
+
+int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,
+                                 int layer_begin, int layer_end, int run_head, float* logits, int32_t* argmax,
+                                 float* S_rec, float* tail_rec, int32_t* status_dev, hgd_stream_t stream) {
+    return chain_run(m, st, tokens, T, layer_begin, layer_end, run_head, logits, argmax, S_rec, tail_rec, status_dev,
+                     stream, nullptr);
+}
+
+int hgd_verify_log_bytes(const hgd_config* cfg, int B, int T, size_t* bytes) {
+    if (!bytes) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if (B < 1 || T < 1) return HGD_ERR_INVALID_ARG;
+    if ((int64_t)B * T > 256) return HGD_ERR_UNSUPPORTED_SHAPE;
+    *bytes = verify_layout(d, B, T).total;
+    return HGD_OK;
+}
+
+int hgd_decode_layer_stack_verify(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,
+                                  float* logits, int32_t* argmax, void* log, size_t log_bytes, int32_t* status_dev,
+                                  hgd_stream_t stream) {
+    if (!m || !st || !st->arena || !tokens || !argmax || !log) return HGD_ERR_INVALID_ARG;
+    if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if (reinterpret_cast<uintptr_t>(log) & 255u) return HGD_ERR_MISALIGNED;
+    const VerifyLayout vlay = verify_layout(d, st->B, T);
+    if (log_bytes < vlay.total) return HGD_ERR_BUFFER_TOO_SMALL;
+    uint8_t* vl = static_cast<uint8_t*>(log);
+    const uint8_t* A = static_cast<const uint8_t*>(st->arena);
+    // the window's conv runs on a copy of the tails; the state's own stay as they are
+    if (d.n_gdn > 0 && cudaMemcpyAsync(vl + vlay.conv, A + st->off[SC_CONV],
+                                       (size_t)d.n_gdn * st->B * (d.kc - 1) * d.C * 4, cudaMemcpyDeviceToDevice,
+                                       (cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return HGD_ERR_CUDA;
+    }
+    return chain_run(m, st, tokens, T, 0, d.L, 1, logits, argmax, nullptr, nullptr, status_dev, stream, vl);
+}
+
+int hgd_decode_layer_stack_keep(const hgd_model* m, const hgd_state* st, int T, const void* log, size_t log_bytes,
+                                const int32_t* keep, int32_t* status_dev, hgd_stream_t stream) {
+    if (!m || !st || !st->arena || !log || !keep) return HGD_ERR_INVALID_ARG;
+    if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if ((reinterpret_cast<uintptr_t>(log) & 255u) || !al16(keep) || (status_dev && !al16(status_dev)))
+        return HGD_ERR_MISALIGNED;
+    const int B = st->B;
+    const VerifyLayout vlay = verify_layout(d, B, T);
+    if (log_bytes < vlay.total) return HGD_ERR_BUFFER_TOO_SMALL;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    const uint8_t* vl = static_cast<const uint8_t*>(log);
+    uint8_t* A = static_cast<uint8_t*>(st->arena);
+    float* Sall = reinterpret_cast<float*>(A + st->off[SC_S]);
+    float* conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
+    const size_t c_layer = (size_t)B * (d.kc - 1) * d.C;
+    for (int ig = 0; ig < d.n_gdn; ++ig) {
+        const uint8_t* ly = vl + vlay.layer(ig);
+        GdnKeepParams g{Sall + ig * s_layer, reinterpret_cast<const float*>(ly + vlay.alpha),
+                        reinterpret_cast<const float*>(ly + vlay.delta), reinterpret_cast<const float*>(ly + vlay.k),
+                        keep, status_dev, B, T, d.H, d.dv};
+        const dim3 grid(B * d.H, d.dv / GDN_ROWS), block(GDN_WARPS * 32);
+        cudaError_t e;
+        switch (d.dk) {
+            case 32: e = launch_pdl(k_gdn_keep<1>, grid, block, 0, s, g); break;
+            case 64: e = launch_pdl(k_gdn_keep<2>, grid, block, 0, s, g); break;
+            case 128: e = launch_pdl(k_gdn_keep<4>, grid, block, 0, s, g); break;
+            default: e = launch_pdl(k_gdn_keep<8>, grid, block, 0, s, g); break;
+        }
+        if ((rc = launch_status(e))) return rc;
+        ConvKeepParams c{conv + ig * c_layer, reinterpret_cast<const float*>(ly + vlay.x), keep, status_dev,
+                         B, T, (int)d.C, d.kc};
+        const int64_t n = (int64_t)B * d.C;
+        e = launch_pdl(k_conv_keep, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, c);
+        if ((rc = launch_status(e))) return rc;
+    }
+    int32_t* pos = reinterpret_cast<int32_t*>(A + st->off[SC_POS]);
+    return launch_status(launch_pdl(k_pos_keep, dim3(1), dim3(32), 0, s, pos, keep, status_dev, B, T));
 }
 
 }  // extern "C"

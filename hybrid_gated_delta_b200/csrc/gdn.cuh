@@ -58,13 +58,22 @@ __device__ __forceinline__ void st_vec(float* p, const float (&d)[KPL]) {
     }
 }
 
+// The rank-1 update of one state row by one logged row: S <- alpha S + delta k^T
+// (the one expression both the step and the replay of a log use).
+template <int KPL>
+__device__ __forceinline__ void gdn_row_update(float (&S)[KPL], float delta, const float (&kv)[KPL], float alpha) {
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) S[e] = fmaf(delta, kv[e], alpha * S[e]);
+}
+
 // One recurrent row for RPW state rows held by this warp.  kv/qv: this lane's
-// normalised key/query elements; vrow[r]: value of state row r; returns o in
-// every lane.
+// normalised key/query elements; vrow[r]: value of state row r; returns o and
+// the row's writes delta (every lane).
 template <int KPL>
 __device__ __forceinline__ void gdn_rows_step(float (&S)[GDN_RPW][KPL], const float (&kv)[KPL],
                                               const float (&qv)[KPL], float alpha, float beta,
-                                              const float (&vrow)[GDN_RPW], float (&o)[GDN_RPW]) {
+                                              const float (&vrow)[GDN_RPW], float (&o)[GDN_RPW],
+                                              float (&dl)[GDN_RPW]) {
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) {
         float w = 0.f;
@@ -72,12 +81,11 @@ __device__ __forceinline__ void gdn_rows_step(float (&S)[GDN_RPW][KPL], const fl
         for (int e = 0; e < KPL; ++e) w = fmaf(S[r][e], kv[e], w);
         w = warp_sum(w);
         const float delta = beta * (vrow[r] - alpha * w);
+        dl[r] = delta;
+        gdn_row_update<KPL>(S[r], delta, kv, alpha);
         float ov = 0.f;
 #pragma unroll
-        for (int e = 0; e < KPL; ++e) {
-            S[r][e] = fmaf(delta, kv[e], alpha * S[r][e]);
-            ov = fmaf(S[r][e], qv[e], ov);
-        }
+        for (int e = 0; e < KPL; ++e) ov = fmaf(S[r][e], qv[e], ov);
         o[r] = warp_sum(ov);
     }
 }
@@ -136,11 +144,11 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_step(const __grid_consta
         float kv[KPL], qv[KPL];
 #pragma unroll
         for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
-        float vrow[GDN_RPW], o[GDN_RPW];
+        float vrow[GDN_RPW], o[GDN_RPW], dl[GDN_RPW];
         const float* vp = p.v + row * p.stride + (int64_t)h * p.dv + row0;
 #pragma unroll
         for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
-        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o);
+        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o, dl);
         const int64_t orow = (row * p.H + h) * p.dv + row0;
         if (lane < GDN_RPW) {
             float ov = o[0];
@@ -157,6 +165,145 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_step(const __grid_consta
     }
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
+}
+
+// ------------------------------------------------- recurrence logs and keep
+// "qwen3_5 cuda ... #849", tree-window commit note: a verify window logs each
+// row's decay, write and key instead of snapshotting the state, and keep replays
+// the kept rows onto the recurrence in one pass.  The window kernel runs the
+// step's arithmetic on the state held in registers and never stores it; the
+// keep kernel applies the logged (alpha, delta, k) with the step's own update
+// expression, so keep(n) equals n one-row steps bit for bit.
+struct GdnLogParams {
+    const float* q; const float* k; const float* v; int64_t stride;
+    const float* g; const float* b;
+    const float* S; float* o; bf16_t* o_bf16;
+    float* log_alpha; float* log_delta; float* log_k;   // [B,T,H], [B,T,H,dv], [B,T,H,dk]
+    int B, T, H, dk, dv, l2norm;
+};
+
+// grid (B*H, dv/16), block 128, as k_gdn_step.
+template <int KPL>
+__global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_window_log(const __grid_constant__ GdnLogParams p) {
+    pdl_launch();
+    pdl_wait();
+    constexpr int DK = 32 * KPL;
+    __shared__ float qs[DK], ks[DK], coef[4];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int row0 = blockIdx.y * GDN_ROWS + warp * GDN_RPW;
+    float S[GDN_RPW][KPL];
+    const float* Sbase = p.S + ((int64_t)(b * p.H + h) * p.dv + row0) * DK + lane * KPL;
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
+
+    for (int t = 0; t < p.T; ++t) {
+        const int64_t row = (int64_t)b * p.T + t;
+        const float* qp = p.q + row * p.stride + (int64_t)h * DK;
+        const float* kp = p.k + row * p.stride + (int64_t)h * DK;
+        __syncthreads();
+        for (int i = tid; i < DK; i += GDN_WARPS * 32) { qs[i] = qp[i]; ks[i] = kp[i]; }
+        __syncthreads();
+        if (warp == 0) { const float s = p.l2norm ? l2_scale<KPL>(qs, lane) : 1.f; if (lane == 0) coef[0] = s; }
+        if (warp == 1) { const float s = p.l2norm ? l2_scale<KPL>(ks, lane) : 1.f; if (lane == 0) coef[1] = s; }
+        if (warp == 2 && lane == 0) {
+            coef[2] = expf(p.g[row * p.H + h]);
+            coef[3] = sigmoid_f(p.b[row * p.H + h]);
+        }
+        __syncthreads();
+        float kv[KPL], qv[KPL];
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
+        float vrow[GDN_RPW], o[GDN_RPW], dl[GDN_RPW];
+        const float* vp = p.v + row * p.stride + (int64_t)h * p.dv + row0;
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
+        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o, dl);
+        const int64_t orow = (row * p.H + h) * p.dv + row0;
+        if (lane < GDN_RPW) {
+            float ov = o[0], dv_ = dl[0];
+#pragma unroll
+            for (int r = 1; r < GDN_RPW; ++r) if (lane == r) { ov = o[r]; dv_ = dl[r]; }
+            p.o[orow + lane] = ov;
+            if (p.o_bf16) p.o_bf16[orow + lane] = f2bf(ov);
+            p.log_delta[orow + lane] = dv_;
+        }
+        if (blockIdx.y == 0 && warp == 0) {
+            st_vec<KPL>(p.log_k + (row * p.H + h) * DK + lane * KPL, kv);
+            if (lane == 0) p.log_alpha[row * p.H + h] = coef[2];
+        }
+    }
+}
+
+struct GdnKeepParams {
+    float* S; const float* log_alpha; const float* log_delta; const float* log_k;
+    const int32_t* keep; int32_t* status;
+    int B, T, H, dv;
+};
+
+// grid (B*H, dv/16), block 128: the CTA's 16 state rows of one (stream, head)
+// take the stream's first keep[b] logged rows.  A count outside [0, T] leaves
+// the stream's state as it is and reports HGD_ERR_INVALID_ARG.
+template <int KPL>
+__global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_keep(const __grid_constant__ GdnKeepParams p) {
+    pdl_launch();
+    pdl_wait();
+    constexpr int DK = 32 * KPL;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int row0 = blockIdx.y * GDN_ROWS + warp * GDN_RPW;
+    const int n = p.keep[b];
+    if (n < 0 || n > p.T) {
+        if (h == 0 && blockIdx.y == 0 && tid == 0) set_status(p.status, HGD_ERR_INVALID_ARG);
+        return;
+    }
+    if (n == 0) return;
+    float S[GDN_RPW][KPL];
+    float* Sbase = p.S + ((int64_t)(b * p.H + h) * p.dv + row0) * DK + lane * KPL;
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
+    for (int t = 0; t < n; ++t) {
+        const int64_t lr = ((int64_t)b * p.T + t) * p.H + h;
+        const float alpha = p.log_alpha[lr];
+        float kv[KPL], dl[GDN_RPW];
+        ld_vec<KPL>(kv, p.log_k + lr * DK + lane * KPL);
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) dl[r] = p.log_delta[lr * p.dv + row0 + r];
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) gdn_row_update<KPL>(S[r], dl[r], kv, alpha);
+    }
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
+}
+
+// The conv tail after the first keep[b] rows of a window: one thread per
+// (stream, channel) shifts in x rows 0..keep[b]-1 (the copies the stepped conv
+// makes).  A count outside [0, T] leaves the stream's tail and reports
+// HGD_ERR_INVALID_ARG.
+struct ConvKeepParams {
+    float* tail; const float* x; const int32_t* keep; int32_t* status;
+    int B, T, C, kc;
+};
+__global__ void k_conv_keep(const __grid_constant__ ConvKeepParams p) {
+    pdl_launch();
+    pdl_wait();
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)p.B * p.C) return;
+    const int b = (int)(idx / p.C), c = (int)(idx % p.C);
+    const int n = p.keep[b], nt = p.kc - 1;
+    if (n < 0 || n > p.T) {
+        if (c == 0) set_status(p.status, HGD_ERR_INVALID_ARG);
+        return;
+    }
+    float tl[8];
+    float* tb = p.tail + (int64_t)b * nt * p.C + c;
+    for (int j = 0; j < nt; ++j) tl[j] = tb[(int64_t)j * p.C];
+    for (int t = 0; t < n; ++t) {
+        const float xv = p.x[((int64_t)b * p.T + t) * p.C + c];
+        for (int j = 0; j + 1 < nt; ++j) tl[j] = tl[j + 1];
+        if (nt > 0) tl[nt - 1] = xv;
+    }
+    for (int j = 0; j < nt; ++j) tb[(int64_t)j * p.C] = tl[j];
 }
 
 // ---------------------------------------------------------- standalone conv
@@ -204,6 +351,9 @@ struct GdnLayerParams {
     float* S;                   // this layer: [B][H][dv][dk]
     float* o; int64_t o_ld;     // [M][o_ld]
     float* S_rec;               // this layer: [B][T][H][dv][dk] or null
+    // a verify window's logs ([B][T][H], [B][T][H][dv], [B][T][H][dk]) or null;
+    // when set, the rows run on the state in registers and S is not written back
+    float* log_alpha; float* log_delta; float* log_k;
     int B, T, H, dv;
 };
 
@@ -247,16 +397,21 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
         float kv[KPL], qv[KPL];
 #pragma unroll
         for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
-        float vrow[GDN_RPW], o[GDN_RPW];
+        float vrow[GDN_RPW], o[GDN_RPW], dl[GDN_RPW];
         const float* vp = pr + 2 * (int64_t)H * DK + (int64_t)h * dv + row0;
 #pragma unroll
         for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
-        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o);
+        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o, dl);
         if (lane < GDN_RPW) {
-            float ov = o[0];
+            float ov = o[0], dv_ = dl[0];
 #pragma unroll
-            for (int r = 1; r < GDN_RPW; ++r) if (lane == r) ov = o[r];
+            for (int r = 1; r < GDN_RPW; ++r) if (lane == r) { ov = o[r]; dv_ = dl[r]; }
             p.o[row * p.o_ld + (int64_t)h * dv + row0 + lane] = ov;
+            if (p.log_delta) p.log_delta[(row * H + h) * dv + row0 + lane] = dv_;
+        }
+        if (p.log_delta && blockIdx.y == 0 && warp == 0) {
+            st_vec<KPL>(p.log_k + (row * H + h) * DK + lane * KPL, kv);
+            if (lane == 0) p.log_alpha[row * H + h] = coef[2];
         }
         if (p.S_rec) {
             float* rp = p.S_rec + ((((int64_t)b * p.T + t) * H + h) * dv + row0) * DK + lane * KPL;
@@ -264,6 +419,7 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
             for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
         }
     }
+    if (p.log_delta) return;  // a verify window: the state stays as it was
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
 }

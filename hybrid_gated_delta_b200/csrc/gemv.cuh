@@ -76,6 +76,7 @@ struct GemvParams {
     // tail [B][3][conv_C] shifted in place, tail records [B][T][3][conv_C] (or null).
     // Token row m of this launch is stream (m0 + m) / conv_T, row (m0 + m) % conv_T.
     const bf16_t* conv_w; float* conv_tail; float* conv_rec; int conv_C, conv_T, m0;
+    float* conv_xlog;  // QKV_CONV: the conv input of each row [B][T][conv_C] (a verify window's log), or null
     // ROPE: the attention in-projection, packed with rope_src_row's row order:
     // q rows are rotated and stored fp32 in rope_q [M][nq*hd]; gate rows go to y
     // (fp32) at column nq*hd + g; k rows are rotated and v rows copied into the
@@ -381,6 +382,7 @@ __device__ __forceinline__ void gv_finish(const GemvParams& p, int rb, int s_ite
                             cur_b = b;
                         }
                         const float xv = cb[lane * MP + m];
+                        if (p.conv_xlog) p.conv_xlog[((int64_t)b * p.conv_T + t) * p.conv_C + ch] = xv;
                         float acc = 0.f;
 #pragma unroll
                         for (int j = 0; j < GV_CONV_K - 1; ++j) acc = fmaf(w[j], tl[j], acc);

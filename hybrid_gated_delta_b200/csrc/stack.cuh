@@ -720,7 +720,8 @@ __device__ void sk_gdn_item(const SkParams& s, int ig, int it, float (&S)[GDN_RP
         const float g = -A * softplus_f(a + dtb);
         const float alpha = expf(g);
         const float beta = sigmoid_f(braw);
-        gdn_rows_step<KPL>(S, kv, qv, alpha, beta, vrow, o);
+        float dl[GDN_RPW];
+        gdn_rows_step<KPL>(S, kv, qv, alpha, beta, vrow, o, dl);
         if (lane < GDN_RPW) {
             float ov = o[0];
 #pragma unroll

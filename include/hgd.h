@@ -209,6 +209,47 @@ HGD_API int hgd_gdn_decode_step(const float* q, const float* k, const float* v, 
                         float* S_rec, int B, int T, int H, int dk, int dv, int l2norm_qk,
                         hgd_stream_t stream);
 
+/* ------------------------------------------ recurrence logs and keep ---
+ * [TF] tree-window commit note: a verify window no longer snapshots every row's
+ * state; each stream logs its rows' decay, write and key, and keep replays the
+ * kept rows onto the recurrence in one pass.  Row t of a head updates
+ *   S_t = alpha_t S_{t-1} + delta_t k_t^T,   delta_t = beta_t (v_t - alpha_t S_{t-1} k_t)
+ * (the gated delta rule above, rewritten), so (alpha_t, delta_t, k_t) carry the
+ * row: 4 * (1 + dv + dk) bytes a head instead of the 4 * dv * dk of a snapshot.
+ *
+ * hgd_gdn_window_log: the rows of hgd_gdn_decode_step (same q, k, v, g, b,
+ * row_stride, o, o_bf16, shapes), but S is only read: every row runs on the
+ * state as the rows before it left it, and nothing is written back.  Per row
+ * (b,t) and head h it writes
+ *   log_alpha [B,T,H]     alpha = exp(g)
+ *   log_delta [B,T,H,dv]  the write delta
+ *   log_k     [B,T,H,dk]  k as the row used it (L2-normalised if l2norm_qk)
+ * (fp32 device arrays).  o equals the o of hgd_gdn_decode_step bit for bit. */
+HGD_API int hgd_gdn_window_log(const float* q, const float* k, const float* v, int64_t row_stride,
+                               const float* g, const float* b, const float* S, float* o,
+                               uint16_t* o_bf16, float* log_alpha, float* log_delta, float* log_k,
+                               int B, int T, int H, int dk, int dv, int l2norm_qk,
+                               hgd_stream_t stream);
+
+/* keep: S [B,H,dv,dk] (fp32 device, in place) takes the first keep[b] logged
+ * rows of stream b, S <- alpha_t S + delta_t k_t^T for t = 0..keep[b]-1, with
+ * the logs of a T-row hgd_gdn_window_log call.  keep [B] int32 is read on the
+ * device (so an accept decision made by a kernel needs no host round trip).
+ * S after keep(n) equals S after n one-row hgd_gdn_decode_step calls bit for
+ * bit.  A keep[b] outside [0, T] leaves stream b as it is and writes
+ * HGD_ERR_INVALID_ARG to *status_dev (device int32, or NULL). */
+HGD_API int hgd_gdn_keep(float* S, const float* log_alpha, const float* log_delta, const float* log_k,
+                         const int32_t* keep, int32_t* status_dev, int B, int T, int H, int dk, int dv,
+                         hgd_stream_t stream);
+
+/* The conv tail's keep: tail [B, kc-1, C] (fp32 device, in place) takes the
+ * first keep[b] rows of the window's conv inputs x [B, T, C] (each row shifts
+ * the tail by one and becomes its newest entry), which equals the tail
+ * hgd_conv1d_tail_update leaves after those rows, bit for bit.  keep and
+ * status_dev as hgd_gdn_keep.  Shapes: 2 <= kc <= 8. */
+HGD_API int hgd_conv1d_keep(float* tail, const float* x, const int32_t* keep, int32_t* status_dev,
+                            int B, int T, int C, int kc, hgd_stream_t stream);
+
 /* ------------------------------------------------------ decode stack ---- */
 
 /* Geometry of the hybrid stack ([LUCE] Model).  Layer l is a gated-attention
@@ -354,6 +395,39 @@ HGD_API int hgd_decode_layer_stack_range(const hgd_model* m, const hgd_state* st
                                          int T, int layer_begin, int layer_end, int run_head,
                                          float* logits, int32_t* argmax, float* S_rec, float* tail_rec,
                                          int32_t* status_dev, hgd_stream_t stream);
+
+/* ----------------------------------------------------- verify windows ---
+ * [TF] tree-window commit note: a verify window no longer snapshots every row's
+ * state; each stream logs its rows' decay, write and key, and keep replays the
+ * kept rows onto the recurrence in one pass; one-row steps update in place.
+ *
+ * hgd_decode_layer_stack_verify: one decode call over T rows of each stream,
+ * with the logits and argmax of hgd_decode_layer_stack (bit for bit: the same
+ * kernels), that leaves the recurrent state as it found it:
+ *  - the GDN layers log each row's (alpha, delta, k) instead of writing S;
+ *  - the causal conv runs on a copy of the tails kept in the log and logs each
+ *    row's conv input;
+ *  - the attention layers write K/V at positions pos[b]..pos[b]+T-1 as usual
+ *    (rows past what keep accepts are overwritten by later calls);
+ *  - positions do not advance.
+ * `log` is caller-owned device memory of hgd_verify_log_bytes(cfg, B, T) bytes,
+ * 256-byte aligned (HGD_ERR_BUFFER_TOO_SMALL if smaller); it needs no initial
+ * contents.  The call runs the kernel chain (never the persistent launch).
+ *
+ * hgd_decode_layer_stack_keep: stream b keeps the first keep[b] rows (int32 [B]
+ * device, read on the device) of the verify call whose log is given: every GDN
+ * layer's state takes those rows (hgd_gdn_keep), every conv tail takes their
+ * inputs (hgd_conv1d_keep), and pos[b] += keep[b].  The state then equals the
+ * state after keep[b] one-row decode calls on the same tokens, bit for bit.  A
+ * keep[b] outside [0, T] leaves stream b as it is and writes
+ * HGD_ERR_INVALID_ARG to *status_dev.  T must be the verify call's T. */
+HGD_API int hgd_verify_log_bytes(const hgd_config* cfg, int B, int T, size_t* bytes);
+HGD_API int hgd_decode_layer_stack_verify(const hgd_model* m, const hgd_state* st, const int32_t* tokens,
+                                          int T, float* logits, int32_t* argmax, void* log,
+                                          size_t log_bytes, int32_t* status_dev, hgd_stream_t stream);
+HGD_API int hgd_decode_layer_stack_keep(const hgd_model* m, const hgd_state* st, int T, const void* log,
+                                        size_t log_bytes, const int32_t* keep, int32_t* status_dev,
+                                        hgd_stream_t stream);
 
 /* Number of kernel launches one hgd_decode_layer_stack call over B streams and
  * T rows issues (-1 on bad arguments). */

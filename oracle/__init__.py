@@ -78,6 +78,11 @@ class Oracle:
         L.hgdo_swiglu.argtypes = [_p, _p, _p, _p, C.c_int, C.c_int, C.c_int]
         L.hgdo_conv1d_tail_update.argtypes = [_p, _p, _p, _p, _p] + [C.c_int] * 5
         L.hgdo_gdn_step.argtypes = [_p, _p, _p, C.c_int64, _p, _p, _p, _p, _p] + [C.c_int] * 6
+        L.hgdo_gdn_window_log.argtypes = [_p, _p, _p, C.c_int64, _p, _p, _p, _p, _p, _p, _p] + [C.c_int] * 6
+        L.hgdo_gdn_keep.restype = C.c_int
+        L.hgdo_gdn_keep.argtypes = [_p, _p, _p, _p, _p] + [C.c_int] * 5
+        L.hgdo_conv1d_keep.restype = C.c_int
+        L.hgdo_conv1d_keep.argtypes = [_p, _p, _p] + [C.c_int] * 4
         L.hgdo_softplus.restype = C.c_double if nb == 8 else C.c_float
         L.hgdo_softplus.argtypes = [C.c_double if nb == 8 else C.c_float]
         L.hgdo_gdn_gates.argtypes = [_p, _p, _p, _p, C.c_int]
@@ -159,6 +164,44 @@ class Oracle:
         self.lib.hgdo_gdn_step(_ptr(q), _ptr(k), _ptr(v), row_stride, _ptr(g), _ptr(b),
                                _ptr(S), _ptr(o), _ptr(rec), B, T, H, dk, dv, int(l2norm))
         return (o, rec) if record else o
+
+    def gdn_window_log(self, q, k, v, g, b, S, l2norm=True):
+        """As gdn_step (separate q,k,v [B,T,H,d]) but S is left unchanged; returns
+        (o [B,T,H,dv], log_alpha [B,T,H], log_delta [B,T,H,dv], log_k [B,T,H,dk])."""
+        assert S.dtype == self.real and S.flags["C_CONTIGUOUS"]
+        B, H, dv, dk = S.shape
+        g, b = self._r(g), self._r(b)
+        T = g.shape[1]
+        q, k, v = self._r(q), self._r(k), self._r(v)
+        assert q.shape == (B, T, H, dk) and k.shape == (B, T, H, dk) and v.shape == (B, T, H, dv) and dk == dv
+        o = np.empty((B, T, H, dv), self.real)
+        la = np.empty((B, T, H), self.real)
+        ld = np.empty((B, T, H, dv), self.real)
+        lk = np.empty((B, T, H, dk), self.real)
+        self.lib.hgdo_gdn_window_log(_ptr(q), _ptr(k), _ptr(v), H * dk, _ptr(g), _ptr(b), _ptr(S), _ptr(o),
+                                     _ptr(la), _ptr(ld), _ptr(lk), B, T, H, dk, dv, int(l2norm))
+        return o, la, ld, lk
+
+    def gdn_keep(self, S, log_alpha, log_delta, log_k, keep):
+        """S [B,H,dv,dk] updated in place by the first keep[b] logged rows of stream b."""
+        assert S.dtype == self.real and S.flags["C_CONTIGUOUS"]
+        B, H, dv, dk = S.shape
+        T = log_alpha.shape[1]
+        keep = np.ascontiguousarray(keep, np.int32)
+        la, ld, lk = self._r(log_alpha), self._r(log_delta), self._r(log_k)
+        rc = self.lib.hgdo_gdn_keep(_ptr(S), _ptr(la), _ptr(ld), _ptr(lk), _ptr(keep), B, T, H, dk, dv)
+        if rc:
+            raise ValueError("oracle gdn_keep: a keep count outside [0, T]")
+
+    def conv1d_keep(self, tail, x, keep):
+        """tail [B,kc-1,C] (in place) after the first keep[b] rows of x [B,T,C]."""
+        assert tail.dtype == self.real and tail.flags["C_CONTIGUOUS"]
+        B, nt, C_ = tail.shape
+        x = self._r(x)
+        keep = np.ascontiguousarray(keep, np.int32)
+        rc = self.lib.hgdo_conv1d_keep(_ptr(tail), _ptr(x), _ptr(keep), B, x.shape[1], C_, nt + 1)
+        if rc:
+            raise ValueError("oracle conv1d_keep: a keep count outside [0, T]")
 
     def gdn_step_packed(self, qkv, g, b, S, l2norm=True, record=False):
         """qkv [B,T,2*H*dk + H*dv] real with channels q|k|v."""

@@ -205,6 +205,92 @@ void hgdo_gdn_step(const real* q, const real* k, const real* v, int64_t row_stri
     free(qn); free(kn); free(A); free(Snew);
 }
 
+/* ------------------------------------------ recurrence logs and keep ---- */
+/* [TF] tree-window commit note: a verify window no longer snapshots every row's
+ * state; each stream logs its rows' decay, write and key, and keep replays the
+ * kept rows onto the recurrence in one pass.  Written out: the update of row t
+ *   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ * equals  alpha_t S_{t-1} + delta_t k_t^T  with the write
+ *   delta_t = beta_t (v_t - alpha_t S_{t-1} k_t),
+ * so (alpha_t, delta_t, k_t) determine S_t from S_{t-1} without v, beta or q. */
+
+void hgdo_gdn_window_log(const real* q, const real* k, const real* v, int64_t row_stride,
+                         const real* g, const real* braw, const real* S, real* o,
+                         real* log_alpha, real* log_delta, real* log_k,
+                         int B, int T, int H, int dk, int dv, int l2norm) {
+    real* qn = (real*)malloc(sizeof(real) * (size_t)dk);
+    real* kn = (real*)malloc(sizeof(real) * (size_t)dk);
+    real* A = (real*)malloc(sizeof(real) * (size_t)dk * dk);
+    real* Snew = (real*)malloc(sizeof(real) * (size_t)dv * dk);
+    real* Sw = (real*)malloc(sizeof(real) * (size_t)dv * dk);   /* the window's running state */
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            memcpy(Sw, S + ((int64_t)b * H + h) * dv * dk, sizeof(real) * (size_t)dv * dk);
+            for (int t = 0; t < T; ++t) {
+                const int64_t row = (int64_t)b * T + t;
+                const real* kr = k + row * row_stride + (int64_t)h * dk;
+                const real* vr = v + row * row_stride + (int64_t)h * dv;
+                const real alpha = R_EXP(g[row * H + h]);
+                const real beta = sigmoid(braw[row * H + h]);
+                /* the logged key: k, L2-normalised as the step normalises it */
+                real* lk = log_k + (row * H + h) * dk;
+                for (int i = 0; i < dk; ++i) lk[i] = kr[i];
+                if (l2norm) l2normalize(lk, dk);
+                /* the write, from the state before the row */
+                real* ld = log_delta + (row * H + h) * dv;
+                for (int i = 0; i < dv; ++i) {
+                    real w = 0;
+                    for (int j = 0; j < dk; ++j) w += Sw[(int64_t)i * dk + j] * lk[j];
+                    ld[i] = beta * (vr[i] - alpha * w);
+                }
+                log_alpha[row * H + h] = alpha;
+                /* the row itself, as hgdo_gdn_step computes it, on the running copy */
+                gdn_head_row(Sw, q + row * row_stride + (int64_t)h * dk, kr, vr, g[row * H + h],
+                             braw[row * H + h], o + (row * H + h) * dv, dk, dv, l2norm, qn, kn, A, Snew);
+            }
+        }
+    free(qn); free(kn); free(A); free(Snew); free(Sw);
+}
+
+int hgdo_gdn_keep(real* S, const real* log_alpha, const real* log_delta, const real* log_k,
+                  const int32_t* keep, int B, int T, int H, int dk, int dv) {
+    for (int b = 0; b < B; ++b)
+        if (keep[b] < 0 || keep[b] > T) return 2;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            real* Sh = S + ((int64_t)b * H + h) * dv * dk;
+            for (int t = 0; t < keep[b]; ++t) {
+                const int64_t lr = ((int64_t)b * T + t) * H + h;
+                const real alpha = log_alpha[lr];
+                const real* dl = log_delta + lr * dv;
+                const real* kk = log_k + lr * dk;
+                for (int i = 0; i < dv; ++i)
+                    for (int j = 0; j < dk; ++j)
+                        Sh[(int64_t)i * dk + j] = alpha * Sh[(int64_t)i * dk + j] + dl[i] * kk[j];
+            }
+        }
+    return 0;
+}
+
+/* The conv tail after the first keep[b] rows of a window whose inputs are x
+ * [B][T][C]: the newest kc-1 entries of (tail, x_0, ..., x_{keep-1}). */
+int hgdo_conv1d_keep(real* tail, const real* x, const int32_t* keep, int B, int T, int C, int kc) {
+    const int nt = kc - 1;
+    for (int b = 0; b < B; ++b)
+        if (keep[b] < 0 || keep[b] > T) return 2;
+    for (int b = 0; b < B; ++b) {
+        real* tb = tail + (int64_t)b * nt * C;
+        for (int t = 0; t < keep[b]; ++t) {
+            const real* xr = x + ((int64_t)b * T + t) * C;
+            for (int c = 0; c < C; ++c) {
+                for (int j = 0; j + 1 < nt; ++j) tb[(int64_t)j * C + c] = tb[(int64_t)(j + 1) * C + c];
+                if (nt > 0) tb[(int64_t)(nt - 1) * C + c] = xr[c];
+            }
+        }
+    }
+    return 0;
+}
+
 /* ----------------------------------------------------------- norms ----- */
 
 /* [FT] RMSNorm. */

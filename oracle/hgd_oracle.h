@@ -92,6 +92,30 @@ void hgdo_gdn_step(const hgdo_real* q, const hgdo_real* k, const hgdo_real* v, i
                    const hgdo_real* g, const hgdo_real* braw, hgdo_real* S, hgdo_real* o,
                    hgdo_real* S_rec, int B, int T, int H, int dk, int dv, int l2norm);
 
+/* Recurrence logs of a verify window ([TF] tree-window commit note: each stream
+ * logs its rows' decay, write and key; keep replays the kept rows onto the
+ * recurrence in one pass).  Same inputs and outputs o as hgdo_gdn_step, but S
+ * is left as it is; the rows run on a copy, and for row (b,t), head h:
+ *   log_alpha[b][t][h]    = alpha = exp(g)
+ *   log_k[b][t][h][dk]    = k (L2-normalised when l2norm, as the step uses it)
+ *   log_delta[b][t][h][dv] = beta (v - alpha S_{t-1} k)    (S_{t-1}: state before the row)
+ * so that S_t = alpha S_{t-1} + delta k^T. */
+void hgdo_gdn_window_log(const hgdo_real* q, const hgdo_real* k, const hgdo_real* v, int64_t row_stride,
+                         const hgdo_real* g, const hgdo_real* braw, const hgdo_real* S, hgdo_real* o,
+                         hgdo_real* log_alpha, hgdo_real* log_delta, hgdo_real* log_k,
+                         int B, int T, int H, int dk, int dv, int l2norm);
+
+/* keep: for each stream b, S[b] <- alpha_t S[b] + delta_t k_t^T for t = 0 ..
+ * keep[b]-1 from the logs above (T rows per stream).  Returns 2 (nothing
+ * changed) if some keep[b] is outside [0, T]. */
+int hgdo_gdn_keep(hgdo_real* S, const hgdo_real* log_alpha, const hgdo_real* log_delta,
+                  const hgdo_real* log_k, const int32_t* keep, int B, int T, int H, int dk, int dv);
+
+/* The conv tail [B][kc-1][C] after the first keep[b] rows of a window with inputs
+ * x [B][T][C]: each kept row shifts the tail by one and becomes its newest entry.
+ * Returns 2 (nothing changed) if some keep[b] is outside [0, T]. */
+int hgdo_conv1d_keep(hgdo_real* tail, const hgdo_real* x, const int32_t* keep, int B, int T, int C, int kc);
+
 /* softplus(t) = max(t,0) + log1p(exp(-|t|))  ([MOE] activation_topk's stable form). */
 hgdo_real hgdo_softplus(hgdo_real t);
 

@@ -277,3 +277,111 @@ def test_tiny_gdn_mixer(hgd, orc):
     for h in range(H):
         assert rel_l2(host(Sw)[0, h], oS[0, h]) <= STATE_REL_L2
     assert np.allclose(host(tw), ot, rtol=1e-5, atol=1e-5)
+
+
+# ------------------------------------------- recurrence logs and keep -------
+# "qwen3_5 cuda ... #849", tree-window commit note: a verify window logs each
+# row's decay, write and key; keep replays the kept rows in one pass.
+
+@pytest.mark.parametrize("B,H,dk,dv,T", [(3, 2, 64, 64, 7), (4, 16, 128, 128, 16), (2, 3, 32, 48, 5),
+                                         (1, 2, 256, 96, 4)])
+def test_gdn_window_log_and_keep(hgd, orc, B, H, dk, dv, T):
+    """A T-row logged window leaves S untouched and gives the o of T one-row steps
+    bit for bit; keep(n) per stream (0, some, all) gives the S of n one-row steps
+    bit for bit; the logs match the oracle's (decay and key to fp32 rounding, the
+    write within the state tolerance per head)."""
+    import torch
+    g = syn.rng(70 + dk + T)
+    S0 = syn.normal_f32(g, (B, H, dv, dk), 0.1)
+    q = syn.normal_f32(g, (B, T, H, dk))
+    k = syn.normal_f32(g, (B, T, H, dk))
+    v = syn.normal_f32(g, (B, T, H, dv))
+    gg = syn.neg_softplus_normal(g, (B, T, H))
+    bb = syn.normal_f32(g, (B, T, H))
+    # the GPU's q/k/v as one packed row per (b, t): q | k | v
+    stride = 2 * H * dk + H * dv
+    rows = np.concatenate([q.reshape(B * T, -1), k.reshape(B * T, -1), v.reshape(B * T, -1)], axis=1)
+    rd = dev_f32(rows)
+    qd, kd, vd = rd, rd[:, H * dk:], rd[:, 2 * H * dk:]
+    gd, bd = dev_f32(gg), dev_f32(bb)
+    S = dev_f32(S0)
+    o, la, ld, lk = hgd.gdn_window_log(qd, kd, vd, gd, bd, S, row_stride=stride, B=B, T=T)
+    torch.cuda.synchronize()
+    assert torch.equal(S, dev_f32(S0))
+    # one-row steps from the same state
+    Ss = dev_f32(S0)
+    steps_o, steps_S = [], []
+    for t in range(T):
+        rs = dev_f32(rows.reshape(B, T, -1)[:, t])
+        os_ = hgd.gdn_decode_step(rs, rs[:, H * dk:], rs[:, 2 * H * dk:], dev_f32(gg[:, t:t + 1]),
+                                  dev_f32(bb[:, t:t + 1]), Ss, row_stride=stride, B=B, T=1)
+        steps_o.append(os_)
+        steps_S.append(Ss.clone())
+    assert torch.equal(o, torch.cat(steps_o, dim=1))
+    keep = np.array({1: [T], 2: [0, T], 3: [0, T // 2, T], 4: [0, 1, T // 2, T]}[B], np.int32)
+    Sk = dev_f32(S0)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hgd.gdn_keep(Sk, la, ld, lk, torch.from_numpy(keep).cuda(), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for b in range(B):
+        n = int(keep[b])
+        ref = dev_f32(S0)[b] if n == 0 else steps_S[n - 1][b]
+        assert torch.equal(Sk[b], ref), f"stream {b}: keep({n}) differs from {n} steps"
+    # against the oracle's logs (dk == dv cases; the oracle's separate arrays share one stride)
+    if dk == dv:
+        oo, ola, old, olk = orc.gdn_window_log(q, k, v, gg, bb, S0.astype(np.float64))
+        assert np.allclose(host(la), ola, rtol=2e-6, atol=0)
+        assert np.allclose(host(lk), olk, rtol=0, atol=2e-6)
+        gdl = host(ld)
+        worst = max(rel_l2(gdl[b, t, h], old[b, t, h]) for b in range(B) for t in range(T) for h in range(H))
+        assert worst <= STATE_REL_L2, worst
+        assert rel_l2(host(o), oo) <= STATE_REL_L2
+
+
+def test_gdn_keep_rejects_out_of_range_counts(hgd):
+    """A keep count outside [0, T] leaves that stream's state as it is and reports
+    HGD_ERR_INVALID_ARG; the other streams are kept."""
+    import torch
+    B, H, d, T = 3, 2, 64, 4
+    g = syn.rng(77)
+    S0 = dev_f32(syn.normal_f32(g, (B, H, d, d), 0.1))
+    q = dev_f32(syn.normal_f32(g, (B, T, H, d)))
+    k = dev_f32(syn.normal_f32(g, (B, T, H, d)))
+    v = dev_f32(syn.normal_f32(g, (B, T, H, d)))
+    gd, bd = dev_f32(syn.neg_softplus_normal(g, (B, T, H))), dev_f32(syn.normal_f32(g, (B, T, H)))
+    _, la, ld, lk = hgd.gdn_window_log(q, k, v, gd, bd, S0)
+    S = S0.clone()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hgd.gdn_keep(S, la, ld, lk, torch.tensor([T + 1, 2, -1], dtype=torch.int32, device="cuda"), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+    assert torch.equal(S[0], S0[0]) and torch.equal(S[2], S0[2]) and not torch.equal(S[1], S0[1])
+
+
+def test_conv_keep_equals_stepped_tails(hgd):
+    """The conv tail after keep(n) rows of a window equals the tail left by n
+    one-row conv steps, bit for bit; out-of-range counts are refused per stream."""
+    import torch
+    B, T, C_, kc = 4, 6, 6144, 4
+    g = syn.rng(78)
+    x = dev_f32(syn.normal_f32(g, (B, T, C_)))
+    w = dev_bf16(syn.normal_bf16(g, (C_, kc), 0.5))
+    tail0 = dev_f32(syn.normal_f32(g, (B, kc - 1, C_)))
+    ts = tail0.clone()
+    stepped = []
+    for t in range(T):
+        hgd.conv1d_tail_update(x[:, t:t + 1].contiguous(), ts, w)
+        stepped.append(ts.clone())
+    keep = torch.tensor([0, 1, 5, T], dtype=torch.int32, device="cuda")
+    tk = tail0.clone()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hgd.conv1d_keep(tk, x, keep, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for b, n in enumerate(keep.tolist()):
+        assert torch.equal(tk[b], tail0[b] if n == 0 else stepped[n - 1][b])
+    bad = tail0.clone()
+    hgd.conv1d_keep(bad, x, torch.tensor([7, 0, 0, 0], dtype=torch.int32, device="cuda"), status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1 and torch.equal(bad, tail0)

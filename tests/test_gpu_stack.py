@@ -517,3 +517,81 @@ def test_not_coresident_is_refused_on_the_host(hgd):
     am = hgd.decode_layer_stack(model, st, torch.tensor([[3]], dtype=torch.int32, device="cuda"), 1)
     torch.cuda.synchronize()
     assert 0 <= int(am.item()) < cfg["vocab"]
+
+
+# ------------------------------------------------------- verify windows -----
+
+@pytest.mark.parametrize("which", ["small", "full_b2t4", "full_b8t16"])
+def test_verify_window_and_keep_equal_steps(hgd, orc, full, which):
+    """A verify window ("qwen3_5 cuda ... #849", tree-window commit note: rows log
+    their decay, write and key; keep replays the kept rows) gives the logits of
+    one-row steps bit for bit and leaves the state untouched; keep(n) per stream
+    (none, some, all) then leaves S, conv tails, positions and the cache rows
+    below each position equal to n one-row steps, bit for bit.  In the reduced
+    geometry the kept state is also compared with the oracle's after n rows."""
+    import torch
+    if which == "small":
+        cfg, w = syn.SMALL_CFG, weights("small", 5)
+        model = hgd.Model(cfg, w)
+        B, T, Lmax = 3, 5, 40
+    else:
+        cfg, (model, w) = syn.STACK_CFG, full
+        B, T, Lmax = (2, 4, 640) if which == "full_b2t4" else (8, 16, 768)
+    V = cfg["vocab"]
+    prefill = 16 if Lmax < 100 else 512
+    init = syn.stack_state(cfg, B, Lmax, prefill=prefill, seed=31)
+    toks = syn.stack_tokens(cfg, B, T, seed=31)
+    keep = {3: [0, 2, T], 2: [1, T], 8: [0, 1, 3, 7, 8, 15, 16, 5]}[B]
+    # one-row steps, with the state after every step
+    s1 = hgd.State(model, B, 1, Lmax, init)
+    step_logits, snaps = [], [s1.snapshot()]
+    for t in range(T):
+        lg = torch.empty((B, V), device="cuda")
+        hgd.decode_layer_stack(model, s1, torch.from_numpy(np.ascontiguousarray(toks[:, t:t + 1])).cuda(), 1,
+                               logits=lg)
+        step_logits.append(lg)
+        snaps.append(s1.snapshot())
+    # the verify window
+    s2 = hgd.State(model, B, T, Lmax, init)
+    before = s2.snapshot()
+    log = hgd.VerifyLog(model, B, T)
+    lv = torch.empty((B * T, V), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hgd.decode_layer_stack_verify(model, s2, torch.from_numpy(toks).cuda(), T, log, logits=lv, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for t in range(T):
+        assert torch.equal(lv[[b * T + t for b in range(B)]], step_logits[t]), f"row {t}: logits differ"
+    for k in ("S", "conv", "pos"):
+        assert torch.equal(getattr(s2, k), before[k]), f"verify changed {k}"
+    # keep
+    hgd.decode_layer_stack_keep(model, s2, T, log, torch.tensor(keep, dtype=torch.int32, device="cuda"),
+                                status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for b, n in enumerate(keep):
+        ref = snaps[n]
+        assert torch.equal(s2.S[:, b], ref["S"][:, b]), f"stream {b}: S after keep({n})"
+        assert torch.equal(s2.conv[:, b], ref["conv"][:, b]), f"stream {b}: conv tails after keep({n})"
+        assert int(s2.pos[b]) == prefill + n
+        P = prefill + n
+        assert torch.equal(s2.kv[:, :, b, :, :P], ref["kv"][:, :, b, :, :P])
+    if which == "small":
+        for b, n in enumerate(keep):
+            if n == 0:
+                continue
+            m = orc.make_model(cfg, w)
+            ost = oracle_state(orc, init, streams=slice(b, b + 1))
+            orc.decode_stack(m, ost, np.ascontiguousarray(toks[b:b + 1, :n]), logits=False)
+            compare_state_rel(host(s2.S[:, b:b + 1]), ost["S"], f"stream {b} S after keep({n}) vs oracle")
+            compare_state_rel(host(s2.conv[:, b:b + 1]), ost["tail"], f"stream {b} tails after keep({n})")
+    # a count outside [0, T] is refused for its stream only
+    s3 = hgd.State(model, B, T, Lmax, init)
+    hgd.decode_layer_stack_verify(model, s3, torch.from_numpy(toks).cuda(), T, log, status=status)
+    bad = [T + 1] + [T] * (B - 1)
+    hgd.decode_layer_stack_keep(model, s3, T, log, torch.tensor(bad, dtype=torch.int32, device="cuda"),
+                                status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+    assert torch.equal(s3.S[:, 0], before["S"][:, 0]) and int(s3.pos[0]) == prefill
+    assert torch.equal(s3.S[:, 1], snaps[T]["S"][:, 1])

@@ -290,6 +290,100 @@ def test_gdn_matches_rank1_and_unrolled_forms(orc):
             assert np.allclose(S[0, h], unrolled, rtol=1e-12, atol=1e-12)
 
 
+# ------------------------------------------- recurrence logs and keep -----
+# "qwen3_5 cuda ... #849", tree-window commit note: a verify window logs each
+# row's decay, write and key, and keep replays the kept rows in one pass.
+
+def test_gdn_log_exact_rational_tiny(orc):
+    """alpha = 1 (g = 0), beta = 1/2 (b = 0), no normalisation: every quantity is
+    rational.  The logged write delta_t = beta (v_t - alpha S_{t-1} k_t), the logged
+    key and decay, and the replay S_t = alpha S_{t-1} + delta_t k_t^T are compared
+    with exact Fraction arithmetic of the dense definition (which the replay must
+    reproduce exactly in rationals); S itself stays untouched by the window."""
+    d, T = 3, 3
+    g = syn.rng(61)
+    S0 = g.standard_normal((d, d))
+    ks, vs, qs = (g.standard_normal((T, d)) for _ in range(3))
+    S = S0[None, None].copy()
+    o, la, ld, lk = orc.gdn_window_log(qs[None, :, None], ks[None, :, None], vs[None, :, None],
+                                       np.zeros((1, T, 1)), np.zeros((1, T, 1)), S, l2norm=False)
+    assert np.array_equal(S[0, 0], S0)
+    Sx = [[Fr(float(S0[i, j])) for j in range(d)] for i in range(d)]
+    half = Fr(1, 2)
+    for t in range(T):
+        k = [Fr(float(a)) for a in ks[t]]
+        v = [Fr(float(a)) for a in vs[t]]
+        q = [Fr(float(a)) for a in qs[t]]
+        delta = [half * (v[i] - sum(Sx[i][j] * k[j] for j in range(d))) for i in range(d)]
+        A = [[(1 if i == j else 0) - half * k[i] * k[j] for j in range(d)] for i in range(d)]
+        dense = [[sum(Sx[i][l] * A[l][j] for l in range(d)) + half * v[i] * k[j] for j in range(d)]
+                 for i in range(d)]
+        replay = [[Sx[i][j] + delta[i] * k[j] for j in range(d)] for i in range(d)]
+        assert dense == replay  # the identity the logs rest on, exactly
+        Sx = dense
+        assert la[0, t, 0] == 1.0 and np.array_equal(lk[0, t, 0], ks[t])
+        for i in range(d):
+            assert abs(float(delta[i]) - ld[0, t, 0, i]) <= 1e-13 * (1 + abs(float(delta[i])))
+            ox = sum(Sx[i][j] * q[j] for j in range(d))
+            assert abs(float(ox) - o[0, t, 0, i]) <= 1e-13 * (1 + abs(float(ox)))
+    Sk = S0[None, None].copy()
+    orc.gdn_keep(Sk, la, ld, lk, np.array([T], np.int32))
+    for i in range(d):
+        for j in range(d):
+            assert abs(float(Sx[i][j]) - Sk[0, 0, i, j]) <= 1e-13 * (1 + abs(float(Sx[i][j])))
+
+
+def test_gdn_keep_equals_steps(orc):
+    """With gates and normalisation: o of the logged window equals the stepped o bit
+    for bit (same dense rows on a copy); keep(n) per stream equals n steps to
+    rounding (the replay is the rank-1 form, the steps the dense form); keep(0)
+    leaves S untouched; a keep count outside [0, T] is refused."""
+    B, T, H, d = 3, 6, 2, 8
+    g = syn.rng(62)
+    S0 = g.standard_normal((B, H, d, d))
+    inp = _gdn_inputs(g, B, T, H, d, d)
+    S = S0.copy()
+    o, la, ld, lk = orc.gdn_window_log(inp["q"], inp["k"], inp["v"], inp["g"], inp["b"], S)
+    assert np.array_equal(S, S0)
+    assert np.allclose(np.sum(lk ** 2, axis=-1), 1.0, rtol=1e-6)
+    assert np.allclose(la, np.exp(inp["g"]), rtol=1e-15, atol=0)
+    So = S0.copy()
+    ostep = orc.gdn_step(inp["q"], inp["k"], inp["v"], inp["g"], inp["b"], So)
+    assert np.array_equal(o, ostep)
+    keep = np.array([0, 4, T], np.int32)
+    Sk = S0.copy()
+    orc.gdn_keep(Sk, la, ld, lk, keep)
+    assert np.array_equal(Sk[0], S0[0])
+    for b in (1, 2):
+        n = int(keep[b])
+        Sn = S0[b:b + 1].copy()
+        orc.gdn_step(inp["q"][b:b + 1, :n], inp["k"][b:b + 1, :n], inp["v"][b:b + 1, :n],
+                     inp["g"][b:b + 1, :n], inp["b"][b:b + 1, :n], Sn)
+        assert np.allclose(Sk[b], Sn[0], rtol=1e-12, atol=1e-12)
+    with pytest.raises(ValueError):
+        orc.gdn_keep(S0.copy(), la, ld, lk, np.array([0, 1, T + 1], np.int32))
+
+
+def test_conv_keep_equals_recorded_tails(orc):
+    """The tail after keep(n) rows equals the tail the stepped conv records after
+    row n-1 (and the untouched tail for n = 0), bit for bit."""
+    B, T, C_, kc = 3, 5, 12, 4
+    g = syn.rng(63)
+    x = g.standard_normal((B, T, C_))
+    w = syn.normal_bf16(g, (C_, kc), 0.5)
+    tail0 = g.standard_normal((B, kc - 1, C_))
+    t1 = tail0.copy()
+    _, rec = orc.conv1d_tail_update(x, t1, w, record=True)
+    keep = np.array([0, 2, T], np.int32)
+    tk = tail0.copy()
+    orc.conv1d_keep(tk, x, keep)
+    assert np.array_equal(tk[0], tail0[0])
+    assert np.array_equal(tk[1], rec[1, 1])
+    assert np.array_equal(tk[2], rec[2, T - 1])
+    with pytest.raises(ValueError):
+        orc.conv1d_keep(tail0.copy(), x, np.array([-1, 0, 0], np.int32))
+
+
 def test_gdn_window_equals_steps(orc):
     """P5: a T-row call equals T one-row calls bit for bit (state carried row to row)."""
     B, T, H, d = 2, 8, 3, 16
