@@ -403,15 +403,25 @@ def run_kernels(args) -> None:
     stream = torch.cuda.current_stream()
 
     def timed(fn, ncopies, iters):
+        """us per call: `iters` calls (rotating over the copies) captured in one CUDA
+        graph and replayed between two events, so the time is the kernels' and not
+        the host binding's."""
         for i in range(3 * ncopies if ncopies < 8 else ncopies):
             fn(i % ncopies)
         torch.cuda.synchronize()
+        cap = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            for i in range(iters):
+                fn(i % ncopies)
+        graph.replay()
+        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for i in range(iters):
-            fn(i % ncopies)
+        graph.replay()
         b.record(stream)
         torch.cuda.synchronize()
+        graph.reset()
         return a.elapsed_time(b) * 1e3 / iters  # us per call
 
     def line(kernel, shape, us, nbytes):
@@ -489,7 +499,38 @@ def run_kernels(args) -> None:
         us = timed(lambda i: hgd.gdn_decode_step(q, k, v, g, bb, Ss[i], o=o), ncopies, 400)
         nbytes = 2 * sbytes + 4 * B * H * d * 4 + 2 * B * H * 4
         line("hgd_gdn_decode_step (k_gdn_step)", {"B": B, "H": H, "dk": d, "dv": d, "T": 1}, us, nbytes)
+        # a 16-row verify window that logs instead of writing the state, then keep(16)
+        T = 16
+        qw = torch.randn(B, T, H, d, device="cuda", generator=gen)
+        kw = torch.randn(B, T, H, d, device="cuda", generator=gen)
+        vw = torch.randn(B, T, H, d, device="cuda", generator=gen)
+        gw = -torch.nn.functional.softplus(torch.randn(B, T, H, device="cuda", generator=gen))
+        bw = torch.randn(B, T, H, device="cuda", generator=gen)
+        ow = torch.empty(B, T, H, d, device="cuda")
+        _, la, ld, lk = hgd.gdn_window_log(qw, kw, vw, gw, bw, Ss[0], o=ow)
+        us = timed(lambda i: hgd.gdn_window_log(qw, kw, vw, gw, bw, Ss[i], o=ow), ncopies, 200)
+        nbytes = sbytes + 4 * B * T * H * (3 * d + 2) + 4 * B * T * H * (d + 1 + d + d)
+        line("hgd_gdn_window_log (k_gdn_window_log)", {"B": B, "H": H, "dk": d, "dv": d, "T": T}, us, nbytes)
+        keep = torch.full((B,), T, dtype=torch.int32, device="cuda")
+        us = timed(lambda i: hgd.gdn_keep(Ss[i], la, ld, lk, keep), ncopies, 200)
+        nbytes = 2 * sbytes + 4 * B * T * H * (1 + 2 * d) + 4 * B
+        line("hgd_gdn_keep (k_gdn_keep)", {"B": B, "H": H, "dk": d, "dv": d, "T": T}, us, nbytes)
         del Ss
+        torch.cuda.empty_cache()
+
+    # the causal conv tail update of one GDN layer's q|k|v channels (6144), one row
+    Cc, kc = 6144, 4
+    for B in (1, 8, 64):
+        tbytes = B * (kc - 1) * Cc * 4
+        ncopies = max(4, min(256, rot_bytes // (2 * tbytes)))
+        xs = [torch.randn(B, 1, Cc, device="cuda", generator=gen) for _ in range(ncopies)]
+        tails = [torch.randn(B, kc - 1, Cc, device="cuda", generator=gen) for _ in range(ncopies)]
+        wc = torch.randn(Cc, kc, device="cuda", generator=gen).to(torch.bfloat16)
+        yc = torch.empty(B, 1, Cc, device="cuda")
+        us = timed(lambda i: hgd.conv1d_tail_update(xs[i], tails[i], wc, y=yc), ncopies, 400)
+        nbytes = 2 * tbytes + 2 * B * Cc * 4 + Cc * kc * 2
+        line("hgd_conv1d_tail_update (k_conv_tail)", {"B": B, "T": 1, "C": Cc, "kc": kc}, us, nbytes)
+        del xs, tails
         torch.cuda.empty_cache()
 
 

@@ -172,7 +172,9 @@ __device__ bool sk_wait(const SkParams& s, volatile int* cta_abort, volatile int
                 if ((++it & 31u) == 0u) {
                     if (ld_acquire_u32(&s.bar[0])) { *cta_abort = 1; break; }
                     if (globaltimer() - t0 > s.wait_ns) {
-                        if (warp == 0) sk_timeout(s, 1u, (unsigned)p, 0u);
+                        // whichever poller runs out first records it (the record is
+                        // first-wins); the others then leave through `seen`
+                        sk_timeout(s, 1u, (unsigned)p, 0u);
                         *cta_abort = 1;
                         break;
                     }

@@ -577,14 +577,25 @@ def test_verify_window_and_keep_equal_steps(hgd, orc, full, which):
         P = prefill + n
         assert torch.equal(s2.kv[:, :, b, :, :P], ref["kv"][:, :, b, :, :P])
     if which == "small":
+        # GDN layer 0 sees exact inputs (the embedding rows): the state tolerance.
+        # Deeper layers inherit last-bit flips of the bf16 residual stream, so they
+        # are held to the oracle's own fp32-vs-fp64 deviation (end to end).
+        from oracle import Oracle
+        orc32 = Oracle(fp32=True)
         for b, n in enumerate(keep):
             if n == 0:
                 continue
-            m = orc.make_model(cfg, w)
-            ost = oracle_state(orc, init, streams=slice(b, b + 1))
-            orc.decode_stack(m, ost, np.ascontiguousarray(toks[b:b + 1, :n]), logits=False)
-            compare_state_rel(host(s2.S[:, b:b + 1]), ost["S"], f"stream {b} S after keep({n}) vs oracle")
-            compare_state_rel(host(s2.conv[:, b:b + 1]), ost["tail"], f"stream {b} tails after keep({n})")
+            refs = {}
+            for o in (orc, orc32):
+                ost = oracle_state(o, init, streams=slice(b, b + 1))
+                o.decode_stack(o.make_model(cfg, w), ost, np.ascontiguousarray(toks[b:b + 1, :n]), logits=False)
+                refs[o.real] = (ost["S"].astype(np.float64), ost["tail"].astype(np.float64))
+            (S64, t64), (S32, t32) = refs[np.float64], refs[np.float32]
+            gS, gt = host(s2.S[:, b:b + 1]), host(s2.conv[:, b:b + 1])
+            compare_state_rel(gS[0], S64[0], f"stream {b} layer-0 S after keep({n}) vs oracle")
+            compare_state_rel(gt[0], t64[0], f"stream {b} layer-0 tails after keep({n}) vs oracle")
+            for got, r64, r32, what in ((gS, S64, S32, "S"), (gt, t64, t32, "tails")):
+                assert rel_l2(got, r64) <= 1.5 * rel_l2(r32, r64) + 1e-4, f"stream {b} {what} after keep({n})"
     # a count outside [0, T] is refused for its stream only
     s3 = hgd.State(model, B, T, Lmax, init)
     hgd.decode_layer_stack_verify(model, s3, torch.from_numpy(toks).cuda(), T, log, status=status)
