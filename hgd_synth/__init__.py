@@ -190,22 +190,34 @@ _NAMES = ("in_norm", "w_in", "conv_w", "A_log", "dt_bias", "gnorm_w", "w_out", "
           "w_up", "w_down")
 
 
+def gdn_heads(cfg: dict) -> tuple[int, int]:
+    """(key heads Hk, value heads H) of the GDN layers; gdn_v_heads 0 or absent: H = Hk."""
+    Hk = cfg["gdn_heads"]
+    return Hk, (cfg.get("gdn_v_heads") or Hk)
+
+
 def stack_weights(cfg: dict, seed: int = 4, std: float = 0.02) -> dict:
     """Random-init bf16 weights N(0, std) with gains 1 + N(0, std).
-    Returns {"embed", "final_norm", "layers": [dict per layer]}; the per-layer keys
-    match the oracle's layer struct (in_norm, w_in, conv_w, A_log, dt_bias, gnorm_w,
-    w_out, post_norm, w_gate, w_up, w_down).  Tensor (layer l, name) is drawn from
-    the key (seed, l, name index); the embedding and final norm use l = -1."""
-    D, V, H = cfg["hidden"], cfg["vocab"], cfg["gdn_heads"]
+    Returns {"embed", "final_norm", "layers": [dict per layer]} and, with
+    cfg["untied_head"], "lm_head" [V, D]; the per-layer keys match the oracle's
+    layer struct (in_norm, w_in, conv_w, A_log, dt_bias, gnorm_w, w_out,
+    post_norm, w_gate, w_up, w_down).  Tensor (layer l, name) is drawn from the
+    key (seed, l, name index); the model-level tensors use l = -1.  With Hk key
+    and H value heads the GDN in-projection has rows q (Hk*dk) | k (Hk*dk) |
+    v (H*dv) | z (H*dv) | a (H) | b (H)."""
+    D, V = cfg["hidden"], cfg["vocab"]
+    Hk, H = gdn_heads(cfg)
     dk, dv, kc = cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
     nq, nkv, hd, I = cfg["attn_q_heads"], cfg["attn_kv_heads"], cfg["attn_head_dim"], cfg["mlp_inter"]
-    Cc = 2 * H * dk + H * dv
+    Cc = 2 * Hk * dk + H * dv
 
     def w_(l, name, shape, mean=0.0):
         return keyed_normal_bf16((seed, l + 1, _NAMES.index(name) if name in _NAMES else 99 + len(name)),
                                  shape, std, mean)
 
     w = {"embed": w_(-1, "embed", (V, D)), "final_norm": w_(-1, "final_norm", (D,), 1.0), "layers": []}
+    if cfg.get("untied_head"):
+        w["lm_head"] = w_(-1, "lm_head", (V, D))
     for l in range(cfg["n_layers"]):
         lw = {"in_norm": w_(l, "in_norm", (D,), 1.0)}
         if not is_attn(cfg, l):
@@ -231,9 +243,10 @@ def stack_state(cfg: dict, B: int, Lmax: int, prefill: int = 512, seed: int = 4)
     rows 0..prefill-1 ~ N(0,1) bf16 (keys taken as already rotated), rows past it
     zero; every stream starts at position `prefill`."""
     n_gdn, n_attn = layer_counts(cfg)
-    H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+    Hk, H = gdn_heads(cfg)
+    dk, dv, kc = cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
     nkv, hd = cfg["attn_kv_heads"], cfg["attn_head_dim"]
-    Cc = 2 * H * dk + H * dv
+    Cc = 2 * Hk * dk + H * dv
     g = rng(seed * 31 + 17 + B)
     kv = np.zeros((n_attn, 2, B, nkv, Lmax, hd), np.uint16)
     if prefill > 0:

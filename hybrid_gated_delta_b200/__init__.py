@@ -29,7 +29,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned
 MAX_LAYERS = 64
 W_IN_NORM, W_IN, W_CONV, W_A_LOG, W_DT_BIAS, W_GNORM, W_OUT, W_POST_NORM, W_GATE, W_UP, W_DOWN = range(11)
 W_LAYER_COUNT = 11
-W_EMBED, W_FINAL_NORM = 100, 101
+W_EMBED, W_FINAL_NORM, W_LM_HEAD = 100, 101, 102
 LAYER_TENSORS = {"in_norm": W_IN_NORM, "w_in": W_IN, "conv_w": W_CONV, "A_log": W_A_LOG,
                  "dt_bias": W_DT_BIAS, "gnorm_w": W_GNORM, "w_out": W_OUT, "post_norm": W_POST_NORM,
                  "w_gate": W_GATE, "w_up": W_UP, "w_down": W_DOWN}
@@ -47,12 +47,14 @@ class Config(C.Structure):
                 ("gdn_heads", C.c_int32), ("gdn_dk", C.c_int32), ("gdn_dv", C.c_int32),
                 ("conv_k", C.c_int32), ("attn_q_heads", C.c_int32), ("attn_kv_heads", C.c_int32),
                 ("attn_head_dim", C.c_int32), ("mlp_inter", C.c_int32), ("attn_every", C.c_int32),
-                ("norm_eps", C.c_float), ("rope_base", C.c_float)]
+                ("norm_eps", C.c_float), ("rope_base", C.c_float), ("gdn_v_heads", C.c_int32),
+                ("untied_head", C.c_int32)]
 
 
 class _Model(C.Structure):
     _fields_ = [("cfg", Config), ("embed", C.c_void_p), ("final_norm", C.c_void_p),
-                ("w", (C.c_void_p * W_LAYER_COUNT) * MAX_LAYERS), ("arena_bytes", C.c_size_t)]
+                ("w", (C.c_void_p * W_LAYER_COUNT) * MAX_LAYERS), ("arena_bytes", C.c_size_t),
+                ("lm_head", C.c_void_p)]
 
 
 class _State(C.Structure):
@@ -75,6 +77,8 @@ _SIGS = {
     "hgd_gemm_tc_bf16": ([_p, _p, _p, _i, _i, _i, _p, _sz, _p, _p], _i),
     "hgd_conv1d_tail_update": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
+    "hgd_gdn_decode_step_grouped": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p],
+                                    _i),
     "hgd_gdn_window_log": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_keep": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_conv1d_keep": ([_p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
@@ -275,6 +279,22 @@ def gdn_decode_step(q, k, v, g, b, S, o=None, o_bf16=None, S_rec=None, l2norm_qk
     return o
 
 
+def gdn_decode_step_grouped(q, k, v, g, b, S, key_heads: int, row_stride: int, B: int, T: int, o=None,
+                            o_bf16=None, S_rec=None, l2norm_qk=True, stream=None):
+    """Gated delta rule rows with S's value heads over `key_heads` query/key heads
+    (value head h reads key head h // (H // key_heads)); q, k, v are views into one
+    packed [B*T, row_stride] buffer.  Returns o [B,T,H,dv]."""
+    torch = _torch()
+    _need(S, torch.float32, "S")
+    _, H, dv, dk = S.shape
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=S.device)
+    _check("hgd_gdn_decode_step_grouped", _lib.hgd_gdn_decode_step_grouped(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), int(row_stride), _ptr(g), _ptr(b), _ptr(S), _ptr(o), _ptr(o_bf16),
+        _ptr(S_rec), B, T, key_heads, H, dk, dv, int(l2norm_qk), _stream(stream)))
+    return o
+
+
 def gdn_window_log(q, k, v, g, b, S, o=None, o_bf16=None, l2norm_qk=True, row_stride=None, B=None, T=None,
                    stream=None):
     """The rows of gdn_decode_step with S only read; returns (o, log_alpha [B,T,H],
@@ -329,8 +349,13 @@ def conv1d_keep(tail, x, keep, status=None, stream=None):
 def make_config(cfg: dict) -> Config:
     c = Config()
     for name, _ in Config._fields_:
-        setattr(c, name, cfg[name])
+        setattr(c, name, cfg.get(name, 0) if name in ("gdn_v_heads", "untied_head") else cfg[name])
     return c
+
+
+def gdn_heads(cfg: dict) -> tuple:
+    """(query/key heads, value heads) of the GDN layers."""
+    return cfg["gdn_heads"], (cfg.get("gdn_v_heads") or cfg["gdn_heads"])
 
 
 class Model:
@@ -365,6 +390,8 @@ class Model:
     def _tensors(self, weights):
         yield "embed", W_EMBED, -1
         yield "final_norm", W_FINAL_NORM, -1
+        if self.cfg_dict.get("untied_head"):
+            yield "lm_head", W_LM_HEAD, -1
         for l, lw in enumerate(weights["layers"]):
             for name in lw:
                 yield name, LAYER_TENSORS[name], l
@@ -397,11 +424,12 @@ class State:
         _check("hgd_state_init", _lib.hgd_state_init(C.byref(self.st), C.byref(model.m), B, Tmax, Lmax,
                                                      self.arena_u8.data_ptr(), nbytes.value))
         cfg = model.cfg_dict
-        H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+        Hk, H = gdn_heads(cfg)
+        dk, dv, kc = cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
         nkv, hd = cfg["attn_kv_heads"], cfg["attn_head_dim"]
         n_attn = sum(1 for l in range(cfg["n_layers"]) if l % cfg["attn_every"] == cfg["attn_every"] - 1)
         n_gdn = cfg["n_layers"] - n_attn
-        Cc = 2 * H * dk + H * dv
+        Cc = 2 * Hk * dk + H * dv
         self.S = self._view(S_GDN, torch.float32, (n_gdn, B, H, dv, dk))
         self.conv = self._view(S_CONV, torch.float32, (n_gdn, B, kc - 1, Cc))
         self.kv = self._view(S_KV, torch.bfloat16, (n_attn, 2, B, nkv, Lmax, hd))

@@ -293,6 +293,8 @@ int gemv_chunks(int M, int K) {
 // ------------------------------------------------------------ stack layout
 struct Dims {
     int L, D, V, H, dk, dv, kc, nq, nkv, hd, I, every;
+    int Hk;       // GDN query/key heads; H is the value heads (a multiple of Hk)
+    int untied;   // 1: the LM head is its own tensor (HGD_W_LM_HEAD)
     int n_gdn, n_attn;
     int64_t C, gdn_out, attn_out;
 };
@@ -305,12 +307,17 @@ int dims_of(const hgd_config* c, Dims* d) {
     if (c->hidden < 32 || c->vocab < 1 || c->gdn_heads < 1 || c->mlp_inter < 1 || c->attn_q_heads < 1 ||
         c->attn_kv_heads < 1)
         return HGD_ERR_INVALID_ARG;
-    d->L = c->n_layers; d->D = c->hidden; d->V = c->vocab; d->H = c->gdn_heads;
+    if (c->gdn_v_heads < 0 || (c->gdn_v_heads > 0 && c->gdn_v_heads % c->gdn_heads != 0) ||
+        (c->untied_head != 0 && c->untied_head != 1))
+        return HGD_ERR_INVALID_ARG;
+    d->L = c->n_layers; d->D = c->hidden; d->V = c->vocab;
+    d->Hk = c->gdn_heads; d->H = c->gdn_v_heads > 0 ? c->gdn_v_heads : c->gdn_heads;
+    d->untied = c->untied_head;
     d->dk = c->gdn_dk; d->dv = c->gdn_dv; d->kc = c->conv_k; d->nq = c->attn_q_heads;
     d->nkv = c->attn_kv_heads; d->hd = c->attn_head_dim; d->I = c->mlp_inter; d->every = c->attn_every;
     d->n_gdn = d->n_attn = 0;
     for (int l = 0; l < d->L; ++l) (is_attn_layer(c, l) ? d->n_attn : d->n_gdn)++;
-    d->C = 2 * (int64_t)d->H * d->dk + (int64_t)d->H * d->dv;
+    d->C = 2 * (int64_t)d->Hk * d->dk + (int64_t)d->H * d->dv;
     d->gdn_out = d->C + (int64_t)d->H * d->dv + 2 * d->H;
     d->attn_out = 2 * (int64_t)d->nq * d->hd + 2 * (int64_t)d->nkv * d->hd;
     return HGD_OK;
@@ -336,6 +343,7 @@ size_t weight_numel(const Dims& d, const hgd_config* c, int layer, int t) {
     if (layer < 0) {
         if (t == HGD_W_EMBED) return (size_t)d.V * d.D;
         if (t == HGD_W_FINAL_NORM) return (size_t)d.D;
+        if (t == HGD_W_LM_HEAD) return d.untied ? (size_t)d.V * d.D : 0;
         return 0;
     }
     const bool att = is_attn_layer(c, layer);
@@ -361,6 +369,7 @@ struct WeightKind { int kind; int64_t rows, cols; };
 WeightKind weight_kind(const Dims& d, const hgd_config* c, int layer, int t) {
     if (layer < 0) {
         if (t == HGD_W_EMBED) return {1, d.V, d.D};
+        if (t == HGD_W_LM_HEAD && d.untied) return {1, d.V, d.D};
         return {0, 0, 0};
     }
     const bool att = is_attn_layer(c, layer);
@@ -388,8 +397,8 @@ size_t weight_bytes(const Dims& d, const hgd_config* c, int layer, int t) {
 // Walk the arena in order; returns the total and, if (layer, t) matches, its offset.
 size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_t, size_t* off) {
     size_t pos = 0;
-    const int glob[2] = {HGD_W_EMBED, HGD_W_FINAL_NORM};
-    for (int g = 0; g < 2; ++g) {
+    const int glob[3] = {HGD_W_EMBED, HGD_W_FINAL_NORM, HGD_W_LM_HEAD};
+    for (int g = 0; g < 3; ++g) {
         if (want_layer == -1 && want_t == glob[g] && off) *off = pos;
         pos += al256(weight_bytes(d, c, -1, glob[g]));
     }
@@ -679,6 +688,8 @@ int sk_run(const hgd_model* m, const hgd_state* st, const Dims& d, const int32_t
     prm.B = st->B; prm.T = T; prm.M = st->B * T; prm.Lmax = st->Lmax; prm.max_chunks = max_chunks_of(st->Lmax);
     prm.ns = sk_ring_slots(d, prm.M); prm.pb = kSkPartialSlabs;
     prm.embed = m->embed; prm.final_norm = m->final_norm;
+    prm.head = m->lm_head ? m->lm_head : m->embed;
+    prm.Hk = d.Hk;
     prm.S = reinterpret_cast<float*>(A + st->off[SC_S]);
     prm.conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
     prm.kv = reinterpret_cast<bf16_t*>(A + st->off[SC_KV]);
@@ -846,18 +857,27 @@ int hgd_conv1d_tail_update(const float* x, float* tail, const uint16_t* w, float
 int hgd_gdn_decode_step(const float* q, const float* k, const float* v, int64_t row_stride, const float* g,
                         const float* b, float* S, float* o, uint16_t* o_bf16, float* S_rec, int B, int T,
                         int H, int dk, int dv, int l2norm_qk, hgd_stream_t stream) {
-    if (!q || !k || !v || !g || !b || !S || !o || B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1)
+    return hgd_gdn_decode_step_grouped(q, k, v, row_stride, g, b, S, o, o_bf16, S_rec, B, T, H, H, dk, dv,
+                                       l2norm_qk, stream);
+}
+
+int hgd_gdn_decode_step_grouped(const float* q, const float* k, const float* v, int64_t row_stride,
+                                const float* g, const float* b, float* S, float* o, uint16_t* o_bf16,
+                                float* S_rec, int B, int T, int Hk, int H, int dk, int dv, int l2norm_qk,
+                                hgd_stream_t stream) {
+    if (!q || !k || !v || !g || !b || !S || !o || B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1 || Hk < 1 ||
+        H % Hk != 0)
         return HGD_ERR_INVALID_ARG;
     if (!(dk == 32 || dk == 64 || dk == 128 || dk == 256) || dv % GDN_ROWS != 0 || dv > 1024)
         return HGD_ERR_UNSUPPORTED_SHAPE;
-    if (row_stride < (int64_t)H * dk || row_stride < (int64_t)H * dv) return HGD_ERR_INVALID_ARG;
+    if (row_stride < (int64_t)Hk * dk || row_stride < (int64_t)H * dv) return HGD_ERR_INVALID_ARG;
     if (!al16(q) || !al16(k) || !al16(v) || !al16(g) || !al16(b) || !al16(S) || !al16(o) ||
         (o_bf16 && !al16(o_bf16)) || (S_rec && !al16(S_rec)))
         return HGD_ERR_MISALIGNED;
     DevInfo di;
     int rc = device_info(&di);
     if (rc) return rc;
-    GdnParams p{q, k, v, row_stride, g, b, S, o, o_bf16, S_rec, B, T, H, dk, dv, l2norm_qk ? 1 : 0};
+    GdnParams p{q, k, v, row_stride, g, b, S, o, o_bf16, S_rec, B, T, H, dk, dv, l2norm_qk ? 1 : 0, H / Hk};
     const dim3 grid(B * H, dv / GDN_ROWS), block(GDN_WARPS * 32);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
@@ -889,7 +909,7 @@ int hgd_gdn_window_log(const float* q, const float* k, const float* v, int64_t r
     int rc = device_info(&di);
     if (rc) return rc;
     GdnLogParams p{q, k, v, row_stride, g, b, S, o, o_bf16, log_alpha, log_delta, log_k,
-                   B, T, H, dk, dv, l2norm_qk ? 1 : 0};
+                   B, T, H, dk, dv, l2norm_qk ? 1 : 0, 1};
     const dim3 grid(B * H, dv / GDN_ROWS), block(GDN_WARPS * 32);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
@@ -958,7 +978,8 @@ int hgd_model_tensor(const hgd_config* cfg, int layer, int tensor, size_t* offse
     if (rc) return rc;
     if (!offset || !numel) return HGD_ERR_INVALID_ARG;
     if (layer < -1 || layer >= d.L) return HGD_ERR_INVALID_ARG;
-    if (layer == -1 && tensor != HGD_W_EMBED && tensor != HGD_W_FINAL_NORM) return HGD_ERR_INVALID_ARG;
+    if (layer == -1 && tensor != HGD_W_EMBED && tensor != HGD_W_FINAL_NORM && tensor != HGD_W_LM_HEAD)
+        return HGD_ERR_INVALID_ARG;
     if (layer >= 0 && (tensor < 0 || tensor >= HGD_W_LAYER_COUNT)) return HGD_ERR_INVALID_ARG;
     size_t off = 0;
     weight_walk(d, cfg, layer, tensor, &off);
@@ -975,7 +996,8 @@ int hgd_model_load_tensor(const hgd_config* cfg, void* arena, size_t arena_bytes
     if ((rc = check_supported(d))) return rc;
     if (!arena || !src) return HGD_ERR_INVALID_ARG;
     if (layer < -1 || layer >= d.L) return HGD_ERR_INVALID_ARG;
-    if (layer == -1 && tensor != HGD_W_EMBED && tensor != HGD_W_FINAL_NORM) return HGD_ERR_INVALID_ARG;
+    if (layer == -1 && tensor != HGD_W_EMBED && tensor != HGD_W_FINAL_NORM && tensor != HGD_W_LM_HEAD)
+        return HGD_ERR_INVALID_ARG;
     if (layer >= 0 && (tensor < 0 || tensor >= HGD_W_LAYER_COUNT)) return HGD_ERR_INVALID_ARG;
     const size_t n = weight_numel(d, cfg, layer, tensor);
     if (n == 0) return HGD_ERR_INVALID_ARG;
@@ -1021,6 +1043,10 @@ int hgd_model_init(hgd_model* m, const hgd_config* cfg, const void* arena, size_
     m->embed = reinterpret_cast<const uint16_t*>(base + off);
     weight_walk(d, cfg, -1, HGD_W_FINAL_NORM, &off);
     m->final_norm = reinterpret_cast<const uint16_t*>(base + off);
+    if (d.untied) {
+        weight_walk(d, cfg, -1, HGD_W_LM_HEAD, &off);
+        m->lm_head = reinterpret_cast<const uint16_t*>(base + off);
+    }
     for (int l = 0; l < d.L; ++l)
         for (int t = 0; t < HGD_W_LAYER_COUNT; ++t) {
             if (!weight_numel(d, cfg, l, t)) continue;
@@ -1272,7 +1298,7 @@ static int chain_run(const hgd_model* m, const hgd_state* st, const int32_t* tok
             g.S = Sall + ig * s_layer;
             g.o = obuf; g.o_ld = (int64_t)d.H * d.dv;
             g.S_rec = S_rec ? S_rec + ig * srec_layer : nullptr;
-            g.B = B; g.T = T; g.H = d.H; g.dv = d.dv;
+            g.B = B; g.T = T; g.H = d.H; g.dv = d.dv; g.Hk = d.Hk;
             if (vl) {
                 g.log_alpha = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.alpha);
                 g.log_delta = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.delta);
@@ -1348,7 +1374,7 @@ static int chain_run(const hgd_model* m, const hgd_state* st, const int32_t* tok
     // final norm + tied LM head + per-CTA argmax, then the row argmax
     if (run_head) {
         GemvParams p = {};
-        p.W = m->embed; p.packed = 1; p.N = d.V; p.K = d.D;
+        p.W = m->lm_head ? m->lm_head : m->embed; p.packed = 1; p.N = d.V; p.K = d.D;
         p.x = resid; p.x_ld = d.D; p.norm_w = m->final_norm; p.eps = eps;
         p.logits = logits; p.logits_ld = d.V; p.best_v = bestv; p.best_i = besti; p.status = status_dev;
         int G = 0;

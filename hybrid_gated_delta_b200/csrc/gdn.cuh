@@ -110,6 +110,7 @@ struct GdnParams {
     const float* g; const float* b;
     float* S; float* o; bf16_t* o_bf16; float* S_rec;
     int B, T, H, dk, dv, l2norm;
+    int grp;  // value heads per query/key head: value head h reads q, k of head h / grp
 };
 
 // grid (B*H, dv/16), block 128: a CTA owns 16 state rows of one (stream, head).
@@ -129,8 +130,8 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_step(const __grid_consta
 
     for (int t = 0; t < p.T; ++t) {
         const int64_t row = (int64_t)b * p.T + t;
-        const float* qp = p.q + row * p.stride + (int64_t)h * DK;
-        const float* kp = p.k + row * p.stride + (int64_t)h * DK;
+        const float* qp = p.q + row * p.stride + (int64_t)(h / p.grp) * DK;
+        const float* kp = p.k + row * p.stride + (int64_t)(h / p.grp) * DK;
         __syncthreads();
         for (int i = tid; i < DK; i += GDN_WARPS * 32) { qs[i] = qp[i]; ks[i] = kp[i]; }
         __syncthreads();
@@ -180,6 +181,7 @@ struct GdnLogParams {
     const float* S; float* o; bf16_t* o_bf16;
     float* log_alpha; float* log_delta; float* log_k;   // [B,T,H], [B,T,H,dv], [B,T,H,dk]
     int B, T, H, dk, dv, l2norm;
+    int grp;  // value heads per query/key head
 };
 
 // grid (B*H, dv/16), block 128, as k_gdn_step.
@@ -199,8 +201,8 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_window_log(const __grid_
 
     for (int t = 0; t < p.T; ++t) {
         const int64_t row = (int64_t)b * p.T + t;
-        const float* qp = p.q + row * p.stride + (int64_t)h * DK;
-        const float* kp = p.k + row * p.stride + (int64_t)h * DK;
+        const float* qp = p.q + row * p.stride + (int64_t)(h / p.grp) * DK;
+        const float* kp = p.k + row * p.stride + (int64_t)(h / p.grp) * DK;
         __syncthreads();
         for (int i = tid; i < DK; i += GDN_WARPS * 32) { qs[i] = qp[i]; ks[i] = kp[i]; }
         __syncthreads();
@@ -355,6 +357,7 @@ struct GdnLayerParams {
     // when set, the rows run on the state in registers and S is not written back
     float* log_alpha; float* log_delta; float* log_k;
     int B, T, H, dv;
+    int Hk;  // query/key heads (H, the value heads, is a multiple): value head h reads head h / (H / Hk)
 };
 
 template <int KPL>
@@ -367,7 +370,8 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
     const int H = p.H, dv = p.dv;
     const int b = blockIdx.x / H, h = blockIdx.x % H;
     const int row0 = blockIdx.y * GDN_ROWS + warp * GDN_RPW;
-    const int64_t C = 2 * (int64_t)H * DK + (int64_t)H * dv;
+    const int Hk = p.Hk, hk = h / (H / Hk);
+    const int64_t C = 2 * (int64_t)Hk * DK + (int64_t)H * dv;
     const float A = expf(bf2f(p.A_log[h])), dtb = bf2f(p.dt_bias[h]);
 
     float S[GDN_RPW][KPL];
@@ -380,8 +384,8 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
         const float* pr = p.proj + row * p.proj_ld;
         __syncthreads();
         for (int i = tid; i < DK; i += GDN_WARPS * 32) {
-            qs[i] = pr[(int64_t)h * DK + i];
-            ks[i] = pr[(int64_t)H * DK + (int64_t)h * DK + i];
+            qs[i] = pr[(int64_t)hk * DK + i];
+            ks[i] = pr[(int64_t)Hk * DK + (int64_t)hk * DK + i];
         }
         __syncthreads();
         if (warp == 0) { const float sc = l2_scale<KPL>(qs, lane); if (lane == 0) coef[0] = sc; }
@@ -398,7 +402,7 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
 #pragma unroll
         for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
         float vrow[GDN_RPW], o[GDN_RPW], dl[GDN_RPW];
-        const float* vp = pr + 2 * (int64_t)H * DK + (int64_t)h * dv + row0;
+        const float* vp = pr + 2 * (int64_t)Hk * DK + (int64_t)h * dv + row0;
 #pragma unroll
         for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
         gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o, dl);

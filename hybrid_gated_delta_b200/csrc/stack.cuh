@@ -67,6 +67,8 @@ struct SkLayer { const bf16_t* w[HGD_W_LAYER_COUNT]; };
 
 struct SkParams {
     int L, D, V, H, dk, dv, nq, nkv, hd, I, every;
+    int Hk;            // GDN query/key heads; H (the value heads) is a multiple
+    const bf16_t* head;  // the LM head [V][D] (packed): the embedding when tied
     int C, gdn_out, attn_out, proj_ld, kmax;
     float eps;
     double rope_inv1;  // base^(-2/hd)
@@ -233,7 +235,7 @@ __device__ __forceinline__ void sk_gemv_params(const SkParams& s, int kind, int 
             p.y = s.resid; p.y_ld = s.D; p.resid = s.resid; p.resid_ld = s.D;
             break;
         default:  // SK_HEAD
-            p.W = s.embed; p.N = s.V; p.K = s.D; p.norm_w = s.final_norm;
+            p.W = s.head; p.N = s.V; p.K = s.D; p.norm_w = s.final_norm;
             p.logits = s.logits; p.logits_ld = s.V; p.best_v = s.bestv; p.best_i = s.besti;
             break;
     }
@@ -705,12 +707,13 @@ __device__ void sk_gdn_item(const SkParams& s, int ig, int it, float (&S)[GDN_RP
         const int64_t row = (int64_t)b * s.T + t;
         const float* pr = s.proj + row * s.proj_ld;
         float qv[KPL], kv[KPL];
-        ld_vec<KPL>(qv, pr + (int64_t)h * DK + lane * KPL);
-        ld_vec<KPL>(kv, pr + (int64_t)H * DK + (int64_t)h * DK + lane * KPL);
+        const int hk = h / (H / s.Hk);
+        ld_vec<KPL>(qv, pr + (int64_t)hk * DK + lane * KPL);
+        ld_vec<KPL>(kv, pr + (int64_t)s.Hk * DK + (int64_t)hk * DK + lane * KPL);
         const float a = pr[s.C + (int64_t)H * dv + h];
         const float braw = pr[s.C + (int64_t)H * dv + H + h];
         float vrow[GDN_RPW], o[GDN_RPW];
-        const float* vp = pr + 2 * (int64_t)H * DK + (int64_t)h * dv + row0;
+        const float* vp = pr + 2 * (int64_t)s.Hk * DK + (int64_t)h * dv + row0;
 #pragma unroll
         for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
         float sq = 0.f, sk = 0.f;

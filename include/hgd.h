@@ -209,6 +209,17 @@ HGD_API int hgd_gdn_decode_step(const float* q, const float* k, const float* v, 
                         float* S_rec, int B, int T, int H, int dk, int dv, int l2norm_qk,
                         hgd_stream_t stream);
 
+/* The same rows with H value heads over Hk query/key heads ([TF] commit on the
+ * widths read from config.json: linear value heads over fewer key heads; H a
+ * multiple of Hk): value head h reads q and k of head h / (H / Hk), at
+ * q_ptr + (b*T+t)*row_stride + (h / (H/Hk))*dk; v, g, b, S, o, o_bf16 and S_rec
+ * are per value head exactly as above.  Hk = H is hgd_gdn_decode_step.
+ * row_stride >= Hk*dk and >= H*dv. */
+HGD_API int hgd_gdn_decode_step_grouped(const float* q, const float* k, const float* v,
+                                        int64_t row_stride, const float* g, const float* b, float* S,
+                                        float* o, uint16_t* o_bf16, float* S_rec, int B, int T, int Hk,
+                                        int H, int dk, int dv, int l2norm_qk, hgd_stream_t stream);
+
 /* ------------------------------------------ recurrence logs and keep ---
  * [TF] tree-window commit note: a verify window no longer snapshots every row's
  * state; each stream logs its rows' decay, write and key, and keep replays the
@@ -269,6 +280,13 @@ typedef struct hgd_config {
     int32_t attn_every;    /* 4 */
     float norm_eps;        /* 1e-6 */
     float rope_base;       /* 10000 */
+    /* [TF] commit on the widths read from config.json: linear value heads over
+     * fewer key heads, an untied head. */
+    int32_t gdn_v_heads;   /* GDN value heads Hv, a multiple of gdn_heads (the
+                              query/key heads); 0 = gdn_heads.  Value head h reads
+                              query/key head h / (Hv / gdn_heads). */
+    int32_t untied_head;   /* 0: the LM head is the embedding; 1: its own [V, D]
+                              tensor HGD_W_LM_HEAD */
 } hgd_config;
 
 #define HGD_MAX_LAYERS 64
@@ -276,9 +294,10 @@ typedef struct hgd_config {
 /* Tensors of the weight arena.  Per layer (layer >= 0):                 */
 enum hgd_weight_tensor {
     HGD_W_IN_NORM = 0,   /* [D] gain (bf16) */
-    HGD_W_IN = 1,        /* GDN: [2*H*dk + 2*H*dv + 2*H, D], rows q|k|v|z|a|b
+    /* (GDN: Hk = gdn_heads query/key heads, H = value heads, see hgd_config) */
+    HGD_W_IN = 1,        /* GDN: [2*Hk*dk + 2*H*dv + 2*H, D], rows q|k|v|z|a|b
                             attention: [2*nq*hd + 2*nkv*hd, D], rows q|gate|k|v */
-    HGD_W_CONV = 2,      /* GDN: [2*H*dk + H*dv, kc] over channels q|k|v */
+    HGD_W_CONV = 2,      /* GDN: [2*Hk*dk + H*dv, kc] over channels q|k|v */
     HGD_W_A_LOG = 3,     /* GDN: [H] */
     HGD_W_DT_BIAS = 4,   /* GDN: [H] */
     HGD_W_GNORM = 5,     /* GDN: [dv] gated-RMSNorm gain shared by heads */
@@ -289,8 +308,9 @@ enum hgd_weight_tensor {
     HGD_W_DOWN = 10,     /* [D, I] */
     HGD_W_LAYER_COUNT = 11,
     /* model-level tensors (layer = -1) */
-    HGD_W_EMBED = 100,      /* [V, D], also the LM head */
-    HGD_W_FINAL_NORM = 101  /* [D] */
+    HGD_W_EMBED = 100,      /* [V, D], also the LM head unless untied_head */
+    HGD_W_FINAL_NORM = 101, /* [D] */
+    HGD_W_LM_HEAD = 102     /* [V, D], present only with untied_head */
 };
 
 /* Model handle.  Filled by hgd_model_init from a caller-owned weight arena;
@@ -301,6 +321,7 @@ typedef struct hgd_model {
     const uint16_t* final_norm;
     const uint16_t* w[HGD_MAX_LAYERS][HGD_W_LAYER_COUNT];
     size_t arena_bytes;
+    const uint16_t* lm_head;  /* HGD_W_LM_HEAD with untied_head, else NULL (the embedding serves) */
 } hgd_model;
 
 /* Bytes of the weight arena for `cfg` (every tensor 256-byte aligned). */
@@ -331,8 +352,8 @@ HGD_API int hgd_model_init(hgd_model* m, const hgd_config* cfg, const void* weig
 /* Tensors of the state arena (per-stream recurrent state, KV cache, position,
  * and the activation scratch of one call). */
 enum hgd_state_tensor {
-    HGD_S_GDN = 0,    /* [n_gdn, B, H, dv, dk] fp32 recurrent state */
-    HGD_S_CONV = 1,   /* [n_gdn, B, kc-1, 2*H*dk + H*dv] fp32 conv tails, oldest first */
+    HGD_S_GDN = 0,    /* [n_gdn, B, H, dv, dk] fp32 recurrent state (H value heads) */
+    HGD_S_CONV = 1,   /* [n_gdn, B, kc-1, 2*Hk*dk + H*dv] fp32 conv tails, oldest first */
     HGD_S_KV = 2,     /* [n_attn, 2, B, nkv, Lmax, hd] bf16 (0 = keys, rotated) */
     HGD_S_POS = 3,    /* [B] int32 position of each stream's next row */
     HGD_S_RESID = 4,  /* [B*Tmax, D] bf16 residual stream of the current call */

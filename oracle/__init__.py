@@ -25,7 +25,7 @@ class Config(C.Structure):
                 ("conv_k", C.c_int32), ("attn_q_heads", C.c_int32),
                 ("attn_kv_heads", C.c_int32), ("attn_head_dim", C.c_int32),
                 ("mlp_inter", C.c_int32), ("attn_every", C.c_int32),
-                ("norm_eps", C.c_double), ("rope_base", C.c_double)]
+                ("norm_eps", C.c_double), ("rope_base", C.c_double), ("gdn_v_heads", C.c_int32)]
 
 
 class Layer(C.Structure):
@@ -35,7 +35,7 @@ class Layer(C.Structure):
 
 class Model(C.Structure):
     _fields_ = [("cfg", Config), ("embed", _p), ("final_norm", _p),
-                ("layers", Layer * MAX_LAYERS)]
+                ("layers", Layer * MAX_LAYERS), ("lm_head", _p)]
 
 
 class State(C.Structure):
@@ -78,6 +78,7 @@ class Oracle:
         L.hgdo_swiglu.argtypes = [_p, _p, _p, _p, C.c_int, C.c_int, C.c_int]
         L.hgdo_conv1d_tail_update.argtypes = [_p, _p, _p, _p, _p] + [C.c_int] * 5
         L.hgdo_gdn_step.argtypes = [_p, _p, _p, C.c_int64, _p, _p, _p, _p, _p] + [C.c_int] * 6
+        L.hgdo_gdn_step_grouped.argtypes = [_p, _p, _p, C.c_int64, _p, _p, _p, _p, _p] + [C.c_int] * 7
         L.hgdo_gdn_window_log.argtypes = [_p, _p, _p, C.c_int64, _p, _p, _p, _p, _p, _p, _p] + [C.c_int] * 6
         L.hgdo_gdn_keep.restype = C.c_int
         L.hgdo_gdn_keep.argtypes = [_p, _p, _p, _p, _p] + [C.c_int] * 5
@@ -203,6 +204,26 @@ class Oracle:
         if rc:
             raise ValueError("oracle conv1d_keep: a keep count outside [0, T]")
 
+    def gdn_step_grouped(self, q, k, v, g, b, S, l2norm=True):
+        """q,k [B,T,Hk,dk] (key heads), v [B,T,H,dv], g,b [B,T,H]; S [B,H,dv,dk] in place;
+        value head h reads key head h // (H // Hk).  Returns o [B,T,H,dv]."""
+        assert S.dtype == self.real and S.flags["C_CONTIGUOUS"]
+        B, H, dv, dk = S.shape
+        g, b = self._r(g), self._r(b)
+        T = g.shape[1]
+        Hk = q.shape[2]
+        # one packed row per (b, t): q | k | v, so that one stride serves all three
+        rows = np.concatenate([self._r(q).reshape(B * T, -1), self._r(k).reshape(B * T, -1),
+                               self._r(v).reshape(B * T, -1)], axis=1)
+        rows = np.ascontiguousarray(rows)
+        stride = rows.shape[1]
+        base = rows.reshape(-1)
+        o = np.empty((B, T, H, dv), self.real)
+        self.lib.hgdo_gdn_step_grouped(_ptr(base), base[Hk * dk:].ctypes.data_as(C.c_void_p),
+                                       base[2 * Hk * dk:].ctypes.data_as(C.c_void_p), stride, _ptr(g), _ptr(b),
+                                       _ptr(S), _ptr(o), None, B, T, Hk, H, dk, dv, int(l2norm))
+        return o
+
     def gdn_step_packed(self, qkv, g, b, S, l2norm=True, record=False):
         """qkv [B,T,2*H*dk + H*dv] real with channels q|k|v."""
         qkv = self._r(qkv)
@@ -281,6 +302,7 @@ class Oracle:
             return _ptr(a)
         m.embed = P(weights["embed"])
         m.final_norm = P(weights["final_norm"])
+        m.lm_head = P(weights["lm_head"]) if weights.get("lm_head") is not None else None
         for l, lw in enumerate(weights["layers"]):
             for name, arr in lw.items():
                 setattr(m.layers[l], name, P(arr))

@@ -181,9 +181,13 @@ static void gdn_head_row(real* S, const real* q_in, const real* k_in, const real
     }
 }
 
-void hgdo_gdn_step(const real* q, const real* k, const real* v, int64_t row_stride,
-                   const real* g, const real* braw, real* S, real* o, real* S_rec,
-                   int B, int T, int H, int dk, int dv, int l2norm) {
+/* [TF] commit on the widths read from config.json: linear (GDN) value heads over
+ * fewer key heads.  Value head h reads query/key head h / (Hv / Hk); the gates,
+ * the value, the state and the output are per value head. */
+void hgdo_gdn_step_grouped(const real* q, const real* k, const real* v, int64_t row_stride,
+                           const real* g, const real* braw, real* S, real* o, real* S_rec,
+                           int B, int T, int Hk, int H, int dk, int dv, int l2norm) {
+    const int grp = H / Hk;
     real* qn = (real*)malloc(sizeof(real) * (size_t)dk);
     real* kn = (real*)malloc(sizeof(real) * (size_t)dk);
     real* A = (real*)malloc(sizeof(real) * (size_t)dk * dk);
@@ -193,8 +197,8 @@ void hgdo_gdn_step(const real* q, const real* k, const real* v, int64_t row_stri
             const int64_t row = (int64_t)b * T + t;
             for (int h = 0; h < H; ++h) {
                 real* Sh = S + ((int64_t)b * H + h) * dv * dk;
-                gdn_head_row(Sh, q + row * row_stride + (int64_t)h * dk,
-                             k + row * row_stride + (int64_t)h * dk,
+                gdn_head_row(Sh, q + row * row_stride + (int64_t)(h / grp) * dk,
+                             k + row * row_stride + (int64_t)(h / grp) * dk,
                              v + row * row_stride + (int64_t)h * dv,
                              g[row * H + h], braw[row * H + h],
                              o + (row * H + h) * dv, dk, dv, l2norm, qn, kn, A, Snew);
@@ -203,6 +207,12 @@ void hgdo_gdn_step(const real* q, const real* k, const real* v, int64_t row_stri
             }
         }
     free(qn); free(kn); free(A); free(Snew);
+}
+
+void hgdo_gdn_step(const real* q, const real* k, const real* v, int64_t row_stride,
+                   const real* g, const real* braw, real* S, real* o, real* S_rec,
+                   int B, int T, int H, int dk, int dv, int l2norm) {
+    hgdo_gdn_step_grouped(q, k, v, row_stride, g, braw, S, o, S_rec, B, T, H, H, dk, dv, l2norm);
 }
 
 /* ------------------------------------------ recurrence logs and keep ---- */
@@ -371,14 +381,15 @@ static void add_residual(uint16_t* x, const real* delta, int D) {
 int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens, int T,
                       real* logits, int32_t* argmax, real* S_rec, real* tail_rec, uint16_t* x_rec) {
     const hgdo_config* c = &m->cfg;
-    const int L = c->n_layers, D = c->hidden, V = c->vocab, H = c->gdn_heads;
+    const int L = c->n_layers, D = c->hidden, V = c->vocab, Hk = c->gdn_heads;
+    const int H = c->gdn_v_heads > 0 ? c->gdn_v_heads : Hk;  /* value heads */
     const int dk = c->gdn_dk, dv = c->gdn_dv, kc = c->conv_k, nq = c->attn_q_heads;
     const int nkv = c->attn_kv_heads, hd = c->attn_head_dim, I = c->mlp_inter;
     const int B = st->B, Lmax = st->Lmax;
-    const int Cc = 2 * H * dk + H * dv;               /* conv channels q|k|v */
+    const int Cc = 2 * Hk * dk + H * dv;              /* conv channels q|k|v */
     const int n_gdn_out = Cc + H * dv + 2 * H;        /* q|k|v|z|a|b */
     const int n_att_out = 2 * nq * hd + 2 * nkv * hd; /* q|gate|k|v */
-    if (L > HGDO_MAX_LAYERS || L <= 0) return 2;
+    if (L > HGDO_MAX_LAYERS || L <= 0 || H % Hk != 0) return 2;
     int n_gdn = 0, n_attn = 0;
     for (int l = 0; l < L; ++l) { if (is_attn(c, l)) ++n_attn; else ++n_gdn; }
     for (int b = 0; b < B; ++b) {
@@ -421,8 +432,8 @@ int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens
                     hgdo_gdn_gates(p + Cc + H * dv, w->A_log, w->dt_bias, gg, H);
                     for (int hh = 0; hh < H; ++hh) bb[hh] = p[Cc + H * dv + H + hh];
                     real* srec = S_rec ? S_rec + (((int64_t)ig * B + b) * T + t) * H * dv * dk : NULL;
-                    hgdo_gdn_step(y, y + H * dk, y + 2 * H * dk, Cc, gg, bb, S, o, srec,
-                                  1, 1, H, dk, dv, 1);
+                    hgdo_gdn_step_grouped(y, y + Hk * dk, y + 2 * Hk * dk, Cc, gg, bb, S, o, srec,
+                                          1, 1, Hk, H, dk, dv, 1);
                     hgdo_gated_rmsnorm(o, z, w->gnorm_w, u, 1, H, dv, c->norm_eps);
                     hgdo_gemv(w->w_out, u, dlt, 1, D, H * dv);
                     add_residual(x, dlt, D);
@@ -454,7 +465,7 @@ int hgdo_decode_stack(const hgdo_model* m, hgdo_state* st, const int32_t* tokens
                 if (x_rec) memcpy(x_rec + (((int64_t)l * B + b) * T + t) * D, x, sizeof(uint16_t) * D);
             }
             hgdo_rmsnorm(x, m->final_norm, h, 1, D, c->norm_eps);
-            hgdo_gemv(m->embed, h, lg, 1, V, D);
+            hgdo_gemv(m->lm_head ? m->lm_head : m->embed, h, lg, 1, V, D);
             /* [MOE] top-k: on equal scores the lower index wins; the decision is
              * taken on the logits as binary32 values. */
             int best = -1;

@@ -92,6 +92,15 @@ void hgdo_gdn_step(const hgdo_real* q, const hgdo_real* k, const hgdo_real* v, i
                    const hgdo_real* g, const hgdo_real* braw, hgdo_real* S, hgdo_real* o,
                    hgdo_real* S_rec, int B, int T, int H, int dk, int dv, int l2norm);
 
+/* The same with H value heads over Hk query/key heads (H a multiple of Hk;
+ * [TF] commit on config.json widths: linear value heads over fewer key heads):
+ * value head h reads q and k of head h / (H / Hk) at q_ptr + row*row_stride +
+ * (h / (H/Hk))*dk; v, g, braw, S, o and S_rec are per value head as above. */
+void hgdo_gdn_step_grouped(const hgdo_real* q, const hgdo_real* k, const hgdo_real* v,
+                           int64_t row_stride, const hgdo_real* g, const hgdo_real* braw,
+                           hgdo_real* S, hgdo_real* o, hgdo_real* S_rec, int B, int T, int Hk,
+                           int H, int dk, int dv, int l2norm);
+
 /* Recurrence logs of a verify window ([TF] tree-window commit note: each stream
  * logs its rows' decay, write and key; keep replays the kept rows onto the
  * recurrence in one pass).  Same inputs and outputs o as hgdo_gdn_step, but S
@@ -153,8 +162,8 @@ void hgdo_attention_row(const hgdo_real* q, const hgdo_real* gate, const uint16_
 typedef struct hgdo_config {
     int32_t n_layers;       /* 24 */
     int32_t hidden;         /* D */
-    int32_t vocab;          /* V (the LM head is tied to the embedding) */
-    int32_t gdn_heads;      /* H */
+    int32_t vocab;          /* V */
+    int32_t gdn_heads;      /* Hk: GDN query/key heads */
     int32_t gdn_dk;
     int32_t gdn_dv;
     int32_t conv_k;         /* kc */
@@ -165,12 +174,13 @@ typedef struct hgdo_config {
     int32_t attn_every;     /* layer l is attention iff l % attn_every == attn_every-1 */
     double norm_eps;
     double rope_base;
+    int32_t gdn_v_heads;    /* value heads Hv (a multiple of gdn_heads); 0 = gdn_heads */
 } hgdo_config;
 
-/* One layer's weights, all bf16, row-major [out, in]:
- *  GDN layer: in_norm[D]; w_in [2*H*dk + 2*H*dv + 2*H, D] with output rows
- *    q (H*dk) | k (H*dk) | v (H*dv) | z (H*dv) | a (H) | b (H);
- *    conv_w [2*H*dk + H*dv, kc] over the channels q|k|v; A_log[H]; dt_bias[H];
+/* One layer's weights, all bf16, row-major [out, in] (Hk key heads, H value heads):
+ *  GDN layer: in_norm[D]; w_in [2*Hk*dk + 2*H*dv + 2*H, D] with output rows
+ *    q (Hk*dk) | k (Hk*dk) | v (H*dv) | z (H*dv) | a (H) | b (H);
+ *    conv_w [2*Hk*dk + H*dv, kc] over the channels q|k|v; A_log[H]; dt_bias[H];
  *    gnorm_w[dv]; w_out [D, H*dv].
  *  Attention layer: in_norm[D]; w_in [2*nq*hd + 2*nkv*hd, D] with output rows
  *    q (nq*hd) | gate (nq*hd) | k (nkv*hd) | v (nkv*hd); w_out [D, nq*hd].
@@ -196,12 +206,13 @@ typedef struct hgdo_model {
     const uint16_t* embed;      /* [V, D] */
     const uint16_t* final_norm; /* [D] */
     hgdo_layer layers[HGDO_MAX_LAYERS];
+    const uint16_t* lm_head;    /* [V, D], or NULL: the head is tied to the embedding */
 } hgdo_model;
 
 /* Per-stream decode state.  n_gdn / n_attn are the numbers of GDN / attention
  * layers in layer order.
- *   S    [n_gdn][B][H][dv][dk]        real
- *   tail [n_gdn][B][kc-1][C]          real, C = 2*H*dk + H*dv
+ *   S    [n_gdn][B][H][dv][dk]        real (H value heads)
+ *   tail [n_gdn][B][kc-1][C]          real, C = 2*Hk*dk + H*dv
  *   kv   [n_attn][2][B][nkv][Lmax][hd] bf16 (index 0 = keys, already rotated)
  *   pos  [B]  absolute position of the next row of each stream */
 typedef struct hgdo_state {
@@ -220,14 +231,16 @@ typedef struct hgdo_state {
  *   per layer:  h = bf16(RMSNorm(x) * in_norm)
  *     GDN:  p = W_in h;  conv(q|k|v) with SiLU;  z = bf16(p_z)
  *           g = hgdo_gdn_gates(a, A_log, dt_bias),  beta from b
- *           gated delta rule per head (dense form);  u = bf16(gatedRMSNorm(o, z))
+ *           gated delta rule per value head (dense form; value head h reads
+ *           key head h / (H/Hk));  u = bf16(gatedRMSNorm(o, z)) per value head
  *           x = bf16(x + W_out u)
  *     attn: p = W_in h;  RoPE(q), RoPE(k) at the row's position;
  *           K,V cache[pos] = bf16(k), bf16(v);  softmax attention over keys 0..pos
  *           times sigmoid(gate) -> bf16;  x = bf16(x + W_out attn)
  *     m = bf16(silu(W_gate hm) * (W_up hm)),  hm = bf16(RMSNorm(x) * post_norm)
  *     x = bf16(x + W_down m)
- *   logits = E * bf16(RMSNorm(x) * final_norm)   (real, tied head)
+ *   logits = W_head * bf16(RMSNorm(x) * final_norm)   (real; W_head = lm_head, or the
+ *            embedding E when lm_head is NULL: the tied head)
  *   argmax over the logits rounded to binary32, lowest index on ties ([MOE]).
  * logits [B*T][V] may be NULL.  argmax [B*T].  S_rec [n_gdn][B][T][H][dv][dk] and
  * tail_rec [n_gdn][B][T][kc-1][C] may be NULL.  x_rec [L][B][T][D] (bf16) may be

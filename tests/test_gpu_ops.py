@@ -385,3 +385,37 @@ def test_conv_keep_equals_stepped_tails(hgd):
     hgd.conv1d_keep(bad, x, torch.tensor([7, 0, 0, 0], dtype=torch.int32, device="cuda"), status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 1 and torch.equal(bad, tail0)
+
+
+# --------------------------------- value heads over fewer key heads ---------
+# "qwen3_5 cuda ... #849", commit on the widths read from config.json.
+
+@pytest.mark.parametrize("Hk,H,d,T", [(4, 16, 128, 3), (2, 6, 64, 2)])
+def test_gdn_grouped_step(hgd, orc, Hk, H, d, T):
+    """Value head h reads key head h // (H / Hk): the grouped step equals the
+    ungrouped step on q/k heads repeated per group, bit for bit, and the oracle's
+    grouped step within the state tolerance."""
+    import torch
+    B = 2
+    g = syn.rng(80 + H)
+    q, k = syn.normal_f32(g, (B, T, Hk, d)), syn.normal_f32(g, (B, T, Hk, d))
+    v = syn.normal_f32(g, (B, T, H, d))
+    gg, bb = syn.neg_softplus_normal(g, (B, T, H)), syn.normal_f32(g, (B, T, H))
+    S0 = syn.normal_f32(g, (B, H, d, d), 0.1)
+    stride = 2 * Hk * d + H * d
+    rows = dev_f32(np.concatenate([q.reshape(B * T, -1), k.reshape(B * T, -1), v.reshape(B * T, -1)], axis=1))
+    S = dev_f32(S0)
+    o = hgd.gdn_decode_step_grouped(rows, rows[:, Hk * d:], rows[:, 2 * Hk * d:], dev_f32(gg), dev_f32(bb), S,
+                                    key_heads=Hk, row_stride=stride, B=B, T=T)
+    G = H // Hk
+    Su = dev_f32(S0)
+    ou = hgd.gdn_decode_step(dev_f32(np.repeat(q, G, axis=2)), dev_f32(np.repeat(k, G, axis=2)), dev_f32(v),
+                             dev_f32(gg), dev_f32(bb), Su)
+    torch.cuda.synchronize()
+    assert torch.equal(o, ou) and torch.equal(S, Su)
+    oS = S0.astype(np.float64)
+    oo = orc.gdn_step_grouped(q, k, v, gg, bb, oS)
+    assert rel_l2(host(o), oo) <= STATE_REL_L2
+    for b in range(B):
+        for h in range(H):
+            assert rel_l2(host(S[b, h]), oS[b, h]) <= STATE_REL_L2

@@ -36,8 +36,9 @@ def _run(hgd, model, state, toks, T, record, V):
     B = state.B
     cfg = model.cfg_dict
     n_gdn, _ = syn.layer_counts(cfg)
-    H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
-    Cc = 2 * H * dk + H * dv
+    Hk, H = syn.gdn_heads(cfg)
+    dk, dv, kc = cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+    Cc = 2 * Hk * dk + H * dv
     logits = torch.full((B * T, V), float("nan"), device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     srec = trec = None
@@ -142,8 +143,9 @@ def _per_layer_check(hgd, model, state, m_orc_out, pre, toks, T, what):
     r = m_orc_out
     L, D, V = cfg["n_layers"], cfg["hidden"], cfg["vocab"]
     n_gdn, _ = syn.layer_counts(cfg)
-    H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
-    Cc = 2 * H * dk + H * dv
+    Hk, H = syn.gdn_heads(cfg)
+    dk, dv, kc = cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+    Cc = 2 * Hk * dk + H * dv
     _load_oracle_state(state, pre, B)
     srec = torch.full((n_gdn, B, T, H, dv, dk), float("nan"), device="cuda")
     trec = torch.full((n_gdn, B, T, kc - 1, Cc), float("nan"), device="cuda")
@@ -310,8 +312,9 @@ def _run_paths(hgd, model, cfg, B, T, Lmax, steps, seed, prefill=None, inputs=No
     `inputs` (a dict), the initial state and the tokens are left there."""
     import torch
     n_gdn, _ = syn.layer_counts(cfg)
-    H, dk, dv, kc = cfg["gdn_heads"], cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
-    Cc = 2 * H * dk + H * dv
+    Hk, H = syn.gdn_heads(cfg)
+    dk, dv, kc = cfg["gdn_dk"], cfg["gdn_dv"], cfg["conv_k"]
+    Cc = 2 * Hk * dk + H * dv
     V, L = cfg["vocab"], cfg["n_layers"]
     if prefill is None:
         prefill = 16 if Lmax < 100 else 512
@@ -606,3 +609,45 @@ def test_verify_window_and_keep_equal_steps(hgd, orc, full, which):
     assert int(status.item()) == 1
     assert torch.equal(s3.S[:, 0], before["S"][:, 0]) and int(s3.pos[0]) == prefill
     assert torch.equal(s3.S[:, 1], snaps[T]["S"][:, 1])
+
+
+# -------------------------------- value heads over key heads, untied head ---
+
+GROUPED_SMALL = dict(syn.SMALL_CFG, gdn_heads=2, gdn_v_heads=4, untied_head=1)
+GROUPED_WIDE = dict(syn.STACK_CFG, n_layers=4, vocab=8192, gdn_heads=8, gdn_v_heads=16, untied_head=1)
+
+
+@pytest.mark.parametrize("which", ["small", "wide"])
+def test_grouped_untied_stack(hgd, orc, orc32, which):
+    """GDN layers with value heads over fewer key heads and an untied LM head
+    ("qwen3_5 cuda ... #849", commit on config.json widths): the persistent launch
+    equals the kernel chain bit for bit (2 streams x 3-row windows; 8 one-row
+    streams at hidden 1024, 16 value over 8 key heads of 128), and the logits and
+    state follow the oracle: within the oracle's own fp32 deviation end to end
+    (GDN layer 0, which sees exact inputs, within the state tolerance), and in the
+    reduced geometry also within the bf16 tolerance."""
+    import torch
+    cfg = GROUPED_SMALL if which == "small" else GROUPED_WIDE
+    w = syn.stack_weights(cfg, seed=90)
+    model = hgd.Model(cfg, w)
+    B, T, Lmax = (2, 3, 40) if which == "small" else (8, 1, 640)
+    assert model.launches(B, T) == 1
+    inp = {}
+    (rp, sp), (rc, sc) = _run_paths(hgd, model, cfg, B, T, Lmax, 2, 91, inputs=inp)
+    _assert_paths_equal(rp, sp, rc, sc)
+    V = cfg["vocab"]
+    got = np.stack([host(lg).reshape(B, T, V) for (lg, _, _, _) in rp], axis=1).reshape(B, 2 * T, V)
+    refs = {}
+    for o in (orc, orc32):
+        ost = oracle_state(o, inp["init"])
+        r = o.decode_stack(o.make_model(cfg, w), ost, inp["toks"], logits=True)
+        refs[o.real] = (r["logits"].astype(np.float64), ost["S"].astype(np.float64))
+    l64, S64 = refs[np.float64]
+    l32, S32 = refs[np.float32]
+    gS = host(sp.S)
+    compare_state_rel(gS[0], S64[0], f"grouped {which}: GDN layer 0 state")  # exact inputs: the state tolerance
+    for b in range(B):
+        assert rel_l2(got[b], l64[b]) <= 1.5 * rel_l2(l32[b], l64[b]) + 1e-3, f"stream {b} logits"
+        assert rel_l2(gS[:, b], S64[:, b]) <= 1.5 * rel_l2(S32[:, b], S64[:, b]) + 1e-4, f"stream {b} state"
+    if which == "small":
+        compare_logits(got.reshape(-1, V), l64.reshape(-1, V), "grouped small")

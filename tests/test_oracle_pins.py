@@ -717,6 +717,102 @@ def test_stack_rejects_out_of_range(orc, small):
         orc.decode_stack(m, st, np.array([[1, 2]], np.int32))
 
 
+# ------------------------------------ value heads over key heads, untied head
+# "qwen3_5 cuda ... #849", commit on the widths read from config.json: linear
+# value heads over fewer key heads, an untied head.
+
+def test_gdn_grouped_equals_repeated_key_heads(orc):
+    """Value head h reads key head h // (H / Hk): a grouped step equals the
+    ungrouped step whose q and k heads are repeated per group, bit for bit, and
+    differs from it when the key heads are mapped any other way (interleaved)."""
+    B, T, Hk, H, d = 2, 3, 2, 6, 8
+    g = syn.rng(64)
+    q, k = g.standard_normal((B, T, Hk, d)), g.standard_normal((B, T, Hk, d))
+    v = g.standard_normal((B, T, H, d))
+    gg, bb = -np.log1p(np.exp(g.standard_normal((B, T, H)))), g.standard_normal((B, T, H))
+    S0 = g.standard_normal((B, H, d, d))
+    Sg = S0.copy()
+    og = orc.gdn_step_grouped(q, k, v, gg, bb, Sg)
+    Su = S0.copy()
+    ou = orc.gdn_step(np.repeat(q, H // Hk, axis=2), np.repeat(k, H // Hk, axis=2), v, gg, bb, Su)
+    assert np.array_equal(og, ou) and np.array_equal(Sg, Su)
+    Si = S0.copy()
+    oi = orc.gdn_step(np.tile(q, (1, 1, H // Hk, 1)), np.tile(k, (1, 1, H // Hk, 1)), v, gg, bb, Si)
+    assert not np.allclose(oi, og)
+
+
+def _expand_grouped(cfg_g, w_g, st_g):
+    """The ungrouped model (Hk = H) equivalent to a grouped one: the q and k rows of
+    the in-projection, the q and k channels of the conv weights and conv tails
+    repeated once per value head of each group."""
+    Hk, H = syn.gdn_heads(cfg_g)
+    dk, dv, D = cfg_g["gdn_dk"], cfg_g["gdn_dv"], cfg_g["hidden"]
+    G = H // Hk
+    rep = lambda a, axis: np.repeat(a.reshape(a.shape[:axis] + (Hk, dk) + a.shape[axis + 1:]), G,
+                                    axis=axis).reshape(a.shape[:axis] + (H * dk,) + a.shape[axis + 1:])
+    cfg_u = dict(cfg_g, gdn_heads=H, gdn_v_heads=H)
+    w_u = {kk: vv for kk, vv in w_g.items() if kk != "layers"}
+    w_u["layers"] = []
+    for lw in w_g["layers"]:
+        lu = dict(lw)
+        if "conv_w" in lw:
+            wi, cw = lw["w_in"], lw["conv_w"]
+            lu["w_in"] = np.concatenate([rep(wi[:Hk * dk], 0), rep(wi[Hk * dk:2 * Hk * dk], 0),
+                                         wi[2 * Hk * dk:]], axis=0)
+            lu["conv_w"] = np.concatenate([rep(cw[:Hk * dk], 0), rep(cw[Hk * dk:2 * Hk * dk], 0),
+                                           cw[2 * Hk * dk:]], axis=0)
+        w_u["layers"].append(lu)
+    tl = st_g["tail"]
+    st_u = dict(st_g, tail=np.ascontiguousarray(np.concatenate(
+        [rep(tl[..., :Hk * dk], tl.ndim - 1), rep(tl[..., Hk * dk:2 * Hk * dk], tl.ndim - 1),
+         tl[..., 2 * Hk * dk:]], axis=-1)))
+    return cfg_u, w_u, st_u
+
+
+def test_stack_grouped_heads_equal_expanded_model(orc):
+    """A stack with 4 GDN value heads over 2 key heads equals, bit for bit (logits,
+    argmax, recorded state), the 4-head stack whose q/k projection rows, conv
+    weights and conv tails are the grouped ones repeated per value head."""
+    cfg = dict(syn.SMALL_CFG, gdn_heads=2, gdn_v_heads=4)
+    w = syn.stack_weights(cfg, seed=65)
+    st = syn.stack_state(cfg, 2, 40, prefill=16, seed=66)
+    cfg_u, w_u, st_u = _expand_grouped(cfg, w, st)
+    toks = syn.stack_tokens(cfg, 2, 3, seed=67)
+    res = []
+    for c, ww, s0 in ((cfg, w, st), (cfg_u, w_u, st_u)):
+        s1 = {kk: (vv.astype(orc.real) if vv.dtype == np.float32 else vv).copy() for kk, vv in s0.items()}
+        r = orc.decode_stack(orc.make_model(c, ww), s1, toks, record=True)
+        res.append((r, s1))
+    (rg, sg), (ru, su) = res
+    assert np.array_equal(rg["logits"], ru["logits"]) and np.array_equal(rg["argmax"], ru["argmax"])
+    assert np.array_equal(rg["S_rec"], ru["S_rec"]) and np.array_equal(sg["S"], su["S"])
+    assert rg["S_rec"].shape[3] == 4 and rg["tail_rec"].shape[-1] == 2 * 2 * 64 + 4 * 64
+
+
+def test_stack_untied_head(orc):
+    """The untied head (its own [V, D] matrix): equal to the tied stack when it holds
+    the embedding, and with all mixers' and MLPs' output projections zero, the
+    logits are lm_head . bf16(RMSNorm(E[tok]) * final_norm) (numpy's product)."""
+    cfg = dict(syn.SMALL_CFG, untied_head=1)
+    w = syn.stack_weights(cfg, seed=68)
+    st = syn.stack_state(cfg, 1, 40, prefill=16, seed=69)
+    toks = syn.stack_tokens(cfg, 1, 2, seed=70)
+    fresh = lambda: {kk: (vv.astype(orc.real) if vv.dtype == np.float32 else vv).copy() for kk, vv in st.items()}
+    w_same = dict(w, lm_head=w["embed"])
+    r_same = orc.decode_stack(orc.make_model(cfg, w_same), fresh(), toks)
+    w_tied = {kk: vv for kk, vv in w.items() if kk != "lm_head"}
+    r_tied = orc.decode_stack(orc.make_model(syn.SMALL_CFG, w_tied), fresh(), toks)
+    assert np.array_equal(r_same["logits"], r_tied["logits"])
+    w0 = dict(w, layers=[{kk: (np.zeros_like(vv) if kk in ("w_out", "w_down") else vv) for kk, vv in lw.items()}
+                         for lw in w["layers"]])
+    r0 = orc.decode_stack(orc.make_model(cfg, w0), fresh(), toks)
+    for t in range(2):
+        h = orc.rmsnorm(w["embed"][toks[0, t]][None], w["final_norm"])
+        ref = bfv(w["lm_head"]) @ bfv(h)[0]
+        assert np.allclose(r0["logits"][0, t], ref, rtol=1e-12, atol=1e-12)
+        assert not np.allclose(ref, bfv(w["embed"]) @ bfv(h)[0], rtol=1e-3, atol=1e-3)
+
+
 def test_fp32_build_agrees_with_fp64(orc, orc32):
     """The float build (the pages' fp32 reference) stays within the fp32 state
     tolerance of the double build on the tiny GDN case."""
