@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import hgd_synth as syn
-from helpers import assert_bf16_close, dev_f32, host, rel_l2, STATE_REL_L2
+from helpers import assert_bf16_close, BF16_REL_L2, dev_f32, host, rel_l2, STATE_REL_L2
 from stack_common import (compare_argmax, compare_logits, compare_state_rel, oracle_state, weights)
 
 pytestmark = pytest.mark.gpu
@@ -597,8 +597,11 @@ def test_verify_window_and_keep_equal_steps(hgd, orc, full, which):
             gS, gt = host(s2.S[:, b:b + 1]), host(s2.conv[:, b:b + 1])
             compare_state_rel(gS[0], S64[0], f"stream {b} layer-0 S after keep({n}) vs oracle")
             compare_state_rel(gt[0], t64[0], f"stream {b} layer-0 tails after keep({n}) vs oracle")
+            # end to end: the fp32 oracle's own deviation, with one bf16 rounding
+            # quantum of the residual stream (relative 5e-3) as the floor, since a
+            # flip upstream need not happen in both fp32 evaluations
             for got, r64, r32, what in ((gS, S64, S32, "S"), (gt, t64, t32, "tails")):
-                assert rel_l2(got, r64) <= 1.5 * rel_l2(r32, r64) + 1e-4, f"stream {b} {what} after keep({n})"
+                assert rel_l2(got, r64) <= 1.5 * rel_l2(r32, r64) + BF16_REL_L2, f"stream {b} {what} after keep({n})"
     # a count outside [0, T] is refused for its stream only
     s3 = hgd.State(model, B, T, Lmax, init)
     hgd.decode_layer_stack_verify(model, s3, torch.from_numpy(toks).cuda(), T, log, status=status)
@@ -648,6 +651,8 @@ def test_grouped_untied_stack(hgd, orc, orc32, which):
     compare_state_rel(gS[0], S64[0], f"grouped {which}: GDN layer 0 state")  # exact inputs: the state tolerance
     for b in range(B):
         assert rel_l2(got[b], l64[b]) <= 1.5 * rel_l2(l32[b], l64[b]) + 1e-3, f"stream {b} logits"
-        assert rel_l2(gS[:, b], S64[:, b]) <= 1.5 * rel_l2(S32[:, b], S64[:, b]) + 1e-4, f"stream {b} state"
+        # end to end, floor one bf16 quantum of the residual (a flip upstream need
+        # not happen in both fp32 evaluations)
+        assert rel_l2(gS[:, b], S64[:, b]) <= 1.5 * rel_l2(S32[:, b], S64[:, b]) + BF16_REL_L2, f"stream {b} state"
     if which == "small":
         compare_logits(got.reshape(-1, V), l64.reshape(-1, V), "grouped small")
