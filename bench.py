@@ -221,9 +221,21 @@ def cpu_baseline_sample(tokens: int = 4) -> dict:
         for _ in range(tokens):
             tok = orc.decode_stack(m, st, tok, logits=False)["argmax"]
         dt = time.perf_counter() - t0
-    return {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{tokens} greedy tokens of the full stack, single-threaded C oracle (fp64), pinned to one core",
-            **host_info()}
+    out = {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{tokens} greedy tokens of the full stack, single-threaded C oracle (fp64), pinned to one core",
+           **host_info()}
+    # the same oracle loops with their output elements over every host core
+    # (OpenMP build; same results), on the next tokens of the same stream
+    omp = Oracle(all_cores=True)
+    mo = omp.make_model(cfg, syn.stack_weights(cfg, seed=4))
+    ncores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    for _ in range(tokens):
+        tok = omp.decode_stack(mo, st, tok, logits=False)["argmax"]
+    dt = time.perf_counter() - t0
+    out["all_cores"] = {"value": tokens / dt, "unit": UNIT, "cores": ncores, "kind": "oracle (OpenMP build)",
+                        "sample": f"{tokens} further greedy tokens of the same stream"}
+    return out
 
 
 # ---------------------------------------------------------------- replicas --
@@ -516,6 +528,28 @@ def run_kernels(args) -> None:
         nbytes = 2 * sbytes + 4 * B * T * H * (1 + 2 * d) + 4 * B
         line("hgd_gdn_keep (k_gdn_keep)", {"B": B, "H": H, "dk": d, "dv": d, "T": T}, us, nbytes)
         del Ss
+        torch.cuda.empty_cache()
+
+    # prefill: a 512-row prompt through one GDN layer's recurrence (16 heads of 128),
+    # the chunked form against the one-row-at-a-time kernel over the same rows
+    H, d, T = 16, 128, 512
+    for B in (1, 8):
+        qp = torch.randn(B, T, H, d, device="cuda", generator=gen)
+        kp = torch.randn(B, T, H, d, device="cuda", generator=gen)
+        vp = torch.randn(B, T, H, d, device="cuda", generator=gen)
+        gp = -torch.nn.functional.softplus(torch.randn(B, T, H, device="cuda", generator=gen))
+        bp = torch.randn(B, T, H, device="cuda", generator=gen)
+        Sp = [torch.randn(B, H, d, d, device="cuda", generator=gen).mul_(0.1) for _ in range(4)]
+        op = torch.empty(B, T, H, d, device="cuda")
+        for name, fn in (("hgd_gdn_prefill (k_gdn_chunked, 32-row chunks)",
+                          lambda i: hgd.gdn_prefill(qp, kp, vp, gp, bp, Sp[i], o=op)),
+                         ("hgd_gdn_decode_step over the prompt (k_gdn_step, row by row)",
+                          lambda i: hgd.gdn_decode_step(qp, kp, vp, gp, bp, Sp[i], o=op))):
+            us = timed(fn, 4, 20)
+            print(json.dumps({"kernel": name, "shape": {"B": B, "T": T, "H": H, "dk": d, "dv": d}, "us": us,
+                              "tokens_per_s": B * T / (us * 1e-6),
+                              "note": "prefill of one GDN layer's recurrence, not the benchmark line"}), flush=True)
+        del Sp
         torch.cuda.empty_cache()
 
     # the causal conv tail update of one GDN layer's q|k|v channels (6144), one row

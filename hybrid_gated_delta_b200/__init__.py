@@ -79,6 +79,7 @@ _SIGS = {
     "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_decode_step_grouped": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p],
                                     _i),
+    "hgd_gdn_prefill": ([_p, _p, _p, _i64, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_window_log": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_keep": ([_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_conv1d_keep": ([_p, _p, _p, _p, _i, _i, _i, _i, _p], _i),
@@ -292,6 +293,29 @@ def gdn_decode_step_grouped(q, k, v, g, b, S, key_heads: int, row_stride: int, B
     _check("hgd_gdn_decode_step_grouped", _lib.hgd_gdn_decode_step_grouped(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), int(row_stride), _ptr(g), _ptr(b), _ptr(S), _ptr(o), _ptr(o_bf16),
         _ptr(S_rec), B, T, key_heads, H, dk, dv, int(l2norm_qk), _stream(stream)))
+    return o
+
+
+def gdn_prefill(q, k, v, g, b, S, o=None, l2norm_qk=True, row_stride=None, B=None, T=None, stream=None):
+    """The T rows of a prompt through the gated delta rule, a chunk at a time
+    (same arguments and results as gdn_decode_step, to fp32 rounding).
+    Returns o [B,T,H,dv]."""
+    torch = _torch()
+    _need(S, torch.float32, "S")
+    Bs, H, dv, dk = S.shape
+    Tn = g.shape[1] if T is None else T
+    Bn = Bs if B is None else B
+    if row_stride is None:
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _need(t, torch.float32, n)
+            if not t.is_contiguous():
+                raise ValueError(f"{n} must be contiguous")
+        row_stride = H * dk
+    if o is None:
+        o = torch.empty((Bn, Tn, H, dv), dtype=torch.float32, device=S.device)
+    _check("hgd_gdn_prefill", _lib.hgd_gdn_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), int(row_stride),
+                                                   _ptr(g), _ptr(b), _ptr(S), _ptr(o), Bn, Tn, H, dk, dv,
+                                                   int(l2norm_qk), _stream(stream)))
     return o
 
 

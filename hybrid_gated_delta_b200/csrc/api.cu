@@ -15,6 +15,7 @@
 #include "attn.cuh"
 #include "common.cuh"
 #include "gdn.cuh"
+#include "gdn_chunk.cuh"
 #include "gemv.cuh"
 #include "gemm_tc.cuh"
 #include "stack.cuh"
@@ -886,6 +887,37 @@ int hgd_gdn_decode_step_grouped(const float* q, const float* k, const float* v, 
         case 64: e = launch_pdl(k_gdn_step<2>, grid, block, 0, s, p); break;
         case 128: e = launch_pdl(k_gdn_step<4>, grid, block, 0, s, p); break;
         default: e = launch_pdl(k_gdn_step<8>, grid, block, 0, s, p); break;
+    }
+    return launch_status(e);
+}
+
+int hgd_gdn_prefill(const float* q, const float* k, const float* v, int64_t row_stride, const float* g,
+                    const float* b, float* S, float* o, int B, int T, int H, int dk, int dv, int l2norm_qk,
+                    hgd_stream_t stream) {
+    if (!q || !k || !v || !g || !b || !S || !o || B < 1 || T < 1 || H < 1 || dk < 1 || dv < 1)
+        return HGD_ERR_INVALID_ARG;
+    if (!(dk == 64 || dk == 128) || dv % GCK_DVB != 0 || dv > 1024) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (row_stride < (int64_t)H * dk || row_stride < (int64_t)H * dv) return HGD_ERR_INVALID_ARG;
+    if (row_stride % 4 != 0) return HGD_ERR_MISALIGNED;
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(g) || !al16(b) || !al16(S) || !al16(o))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    GdnChunkParams p{q, k, v, row_stride, g, b, S, o, B, T, H, dv, l2norm_qk ? 1 : 0};
+    const dim3 grid(B * H, dv / GCK_DVB), block(GCK_THREADS);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (dk == 128) {
+        static CtxCache<int> attr;
+        const int smem = (int)sizeof(GckSmem<128>);
+        e = ensure_smem_attr(k_gdn_chunked<128>, attr);
+        if (e == cudaSuccess) e = launch_pdl(k_gdn_chunked<128>, grid, block, smem, s, p);
+    } else {
+        static CtxCache<int> attr;
+        const int smem = (int)sizeof(GckSmem<64>);
+        e = ensure_smem_attr(k_gdn_chunked<64>, attr);
+        if (e == cudaSuccess) e = launch_pdl(k_gdn_chunked<64>, grid, block, smem, s, p);
     }
     return launch_status(e);
 }

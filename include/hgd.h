@@ -220,6 +220,22 @@ HGD_API int hgd_gdn_decode_step_grouped(const float* q, const float* k, const fl
                                         float* o, uint16_t* o_bf16, float* S_rec, int B, int T, int Hk,
                                         int H, int dk, int dv, int l2norm_qk, hgd_stream_t stream);
 
+/* -------------------------------------------------------------- prefill ---
+ * The rows of a prompt ([LUCE] Architecture Summary: a prefill kernel beside the
+ * decode kernel; Expected Results: pp512): the same state and outputs as
+ * hgd_gdn_decode_step over the T rows (same q, k, v, row_stride, g, b, S, o and
+ * layouts), computed a chunk of 32 rows at a time: within a chunk the rows'
+ * writes solve the unit lower-triangular system (I + A) U = diag(beta) (V -
+ * diag(Gamma) K S_0^T) with A[t][s] = beta_t (Gamma_t / Gamma_s) (k_s . k_t),
+ * Gamma the running product of alpha, and the outputs and the next state follow
+ * from U in matrix products.  fp32 throughout; equal to the one-row steps to
+ * fp32 rounding (not bit for bit).  No per-row state records.
+ * Shapes: dk in {64, 128}; dv a multiple of 32 up to 1024; row_stride a
+ * multiple of 4 (q, k rows 16-byte aligned). */
+HGD_API int hgd_gdn_prefill(const float* q, const float* k, const float* v, int64_t row_stride,
+                            const float* g, const float* b, float* S, float* o, int B, int T, int H,
+                            int dk, int dv, int l2norm_qk, hgd_stream_t stream);
+
 /* ------------------------------------------ recurrence logs and keep ---
  * [TF] tree-window commit note: a verify window no longer snapshots every row's
  * state; each stream logs its rows' decay, write and key, and keep replays the

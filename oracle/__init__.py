@@ -59,8 +59,10 @@ def build_lib() -> None:
 class Oracle:
     """One loaded oracle library (double by default, float with fp32=True)."""
 
-    def __init__(self, fp32: bool = False):
-        name = "libhgd_oracle_f32.so" if fp32 else "libhgd_oracle.so"
+    def __init__(self, fp32: bool = False, all_cores: bool = False):
+        # all_cores: the double build whose GEMV and dense state product run over
+        # every host core (OpenMP); same results as the default build
+        name = "libhgd_oracle_f32.so" if fp32 else ("libhgd_oracle_omp.so" if all_cores else "libhgd_oracle.so")
         path = os.path.join(_HERE, name)
         if not os.path.exists(path):
             build_lib()

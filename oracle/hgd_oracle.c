@@ -89,9 +89,12 @@ void hgdo_gdn_gates(const real* a, const uint16_t* A_log, const uint16_t* dt_bia
 
 /* ------------------------------------------------------------ GEMV ----- */
 
-/* [AST] BF16 GEMV: y = x W^T with W in the [N,K] (Linear) layout. */
+/* [AST] BF16 GEMV: y = x W^T with W in the [N,K] (Linear) layout.  (In the
+ * all-cores build the output elements are shared out over threads; each one's
+ * sum runs in the same order, so the results do not change.) */
 void hgdo_gemv(const uint16_t* W, const uint16_t* x, real* y, int M, int N, int K) {
     for (int m = 0; m < M; ++m) {
+#pragma omp parallel for schedule(static)
         for (int n = 0; n < N; ++n) {
             real s = 0;
             for (int k = 0; k < K; ++k)
@@ -164,6 +167,7 @@ static void gdn_head_row(real* S, const real* q_in, const real* k_in, const real
     /* S A: element (i,j) is sum_l S[i][l] A[l][j], summed over ascending l
      * (the l-loop is outside the j-loop only so that A is read row by row). */
     for (int64_t n = 0; n < (int64_t)dv * dk; ++n) Snew[n] = 0;
+#pragma omp parallel for schedule(static)
     for (int i = 0; i < dv; ++i)
         for (int l = 0; l < dk; ++l) {
             const real s_il = S[(int64_t)i * dk + l];

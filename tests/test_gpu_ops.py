@@ -419,3 +419,41 @@ def test_gdn_grouped_step(hgd, orc, Hk, H, d, T):
     for b in range(B):
         for h in range(H):
             assert rel_l2(host(S[b, h]), oS[b, h]) <= STATE_REL_L2
+
+
+# ----------------------------------------------------- prefill (chunked) ----
+# "luce-megakernel HANDOFF.md", Architecture Summary (a prefill kernel) and
+# Expected Results (pp512): T rows at once, equal to T one-row steps to rounding.
+
+@pytest.mark.parametrize("B,H,dk,dv,T", [(2, 3, 128, 128, 100), (1, 4, 64, 64, 37), (2, 2, 128, 64, 512),
+                                         (1, 2, 128, 128, 1), (1, 16, 128, 128, 512)])
+def test_gdn_prefill_matches_steps_and_oracle(hgd, orc, B, H, dk, dv, T):
+    """The chunked form over T rows (whole chunks of 32 and a ragged tail) against
+    the oracle's row-by-row recurrence (fp64), output and final state per head
+    within the state tolerance, and against the GPU's own one-row-at-a-time
+    kernel over the same rows."""
+    import torch
+    g = syn.rng(90 + T + dk)
+    S0 = syn.normal_f32(g, (B, H, dv, dk), 0.1)
+    q = syn.normal_f32(g, (B, T, H, dk))
+    k = syn.normal_f32(g, (B, T, H, dk))
+    v = syn.normal_f32(g, (B, T, H, dv))
+    gg = syn.neg_softplus_normal(g, (B, T, H))
+    bb = syn.normal_f32(g, (B, T, H))
+    stride = 2 * H * dk + H * dv
+    rows = dev_f32(np.concatenate([q.reshape(B * T, -1), k.reshape(B * T, -1), v.reshape(B * T, -1)], axis=1))
+    qd, kd, vd = rows, rows[:, H * dk:], rows[:, 2 * H * dk:]
+    S = dev_f32(S0)
+    o = hgd.gdn_prefill(qd, kd, vd, dev_f32(gg), dev_f32(bb), S, row_stride=stride, B=B, T=T)
+    Ss = dev_f32(S0)
+    os_ = hgd.gdn_decode_step(qd, kd, vd, dev_f32(gg), dev_f32(bb), Ss, row_stride=stride, B=B, T=T)
+    torch.cuda.synchronize()
+    go, gS = host(o), host(S)
+    assert rel_l2(gS, host(Ss)) <= STATE_REL_L2 and rel_l2(go, host(os_)) <= STATE_REL_L2
+    if dk == dv:
+        oS = S0.astype(np.float64)
+        oo = orc.gdn_step(q, k, v, gg, bb, oS)
+        for b in range(B):
+            for h in range(H):
+                assert rel_l2(gS[b, h], oS[b, h]) <= STATE_REL_L2, (b, h)
+                assert rel_l2(go[b, :, h], oo[b, :, h]) <= STATE_REL_L2, (b, h)

@@ -813,6 +813,22 @@ def test_stack_untied_head(orc):
         assert not np.allclose(ref, bfv(w["embed"]) @ bfv(h)[0], rtol=1e-3, atol=1e-3)
 
 
+def test_all_cores_build_equals_default_build(orc):
+    """The OpenMP build (the all-cores CPU baseline) shares out output elements
+    only; every sum keeps its order, so a stack call gives the same bits."""
+    from oracle import Oracle
+    omp = Oracle(all_cores=True)
+    cfg = syn.SMALL_CFG
+    w = syn.stack_weights(cfg, seed=5)
+    out = []
+    for o in (orc, omp):
+        st = _state(o, cfg, 2)
+        r = o.decode_stack(o.make_model(cfg, w), st, syn.stack_tokens(cfg, 2, 3, seed=7), record=True)
+        out.append((r["logits"], r["S_rec"], st["S"], st["kv"]))
+    for a, b in zip(*out):
+        assert np.array_equal(a, b)
+
+
 def test_fp32_build_agrees_with_fp64(orc, orc32):
     """The float build (the pages' fp32 reference) stays within the fp32 state
     tolerance of the double build on the tiny GDN case."""
