@@ -580,18 +580,19 @@ def run_windows(args) -> None:
     cfg = syn.STACK_CFG
     B, T, n_win, warm = 8, 16, 16, 2
     Lmax = ((PREFILL + (n_win + warm + 1) * T + 63) // 64) * 64
-    model = hgd.Model(cfg, syn.stack_weights(cfg, seed=5))
+    model = hgd.Model(cfg, syn.stack_weights(cfg, seed=5), tc=args.tc)
     state = hgd.State(model, B, T, Lmax, syn.stack_state(cfg, B, Lmax, prefill=PREFILL, seed=5))
+    decode = hgd.decode_layer_stack_tc if args.tc else hgd.decode_layer_stack
     toks = torch.from_numpy(syn.stack_tokens(cfg, B, T, seed=5)).cuda()
     am = torch.zeros(B * T, dtype=torch.int32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
-        hgd.decode_layer_stack(model, state, toks, T, argmax=am, status=status, stream=stream)
+        decode(model, state, toks, T, argmax=am, status=status, stream=stream)
     stream.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
-        hgd.decode_layer_stack(model, state, toks, T, argmax=am, status=status)
+        decode(model, state, toks, T, argmax=am, status=status)
     for _ in range(warm):
         g.replay()
     torch.cuda.synchronize()
@@ -608,9 +609,10 @@ def run_windows(args) -> None:
     ab = algorithmic_bytes(cfg, PREFILL + (warm + 1 + n / 2.0) * T)
     nbytes = ab["weights"] + B * (ab["total"] - ab["weights"])  # weights once, state and cache per stream
     print(json.dumps({"workload": "8 streams x 16-row windows (128 token rows per call), 24-layer stack",
+                      "path": "tensor-core chain (tcgen05 GEMMs)" if args.tc else "mma.sync kernel chain",
                       "calls": n, "ms_per_call": ms, "tokens_per_s": B * T / (ms * 1e-3),
                       "algorithmic_bytes_per_call": nbytes, "gb_s": nbytes / (ms * 1e-3) / 1e9,
-                      "launches_per_call": model.launches(B, T),
+                      "launches_per_call": None if args.tc else model.launches(B, T),
                       "note": "window throughput, not the benchmark line"}), flush=True)
 
 
@@ -630,6 +632,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=12)  # about 13 s of oracle work at ~1 token/s
     ap.add_argument("--windows", action="store_true",
                     help="instead of the benchmark line: throughput of 8 streams x 16-row windows")
+    ap.add_argument("--tc", action="store_true",
+                    help="with --windows: the tensor-core decode chain (hgd_decode_layer_stack_tc)")
     ap.add_argument("--kernels", action="store_true",
                     help="instead of the benchmark line: per-kernel rooflines of the standalone GEMV and GDN "
                          "entry points at the sweep shapes")

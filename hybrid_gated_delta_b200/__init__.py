@@ -54,7 +54,7 @@ class Config(C.Structure):
 class _Model(C.Structure):
     _fields_ = [("cfg", Config), ("embed", C.c_void_p), ("final_norm", C.c_void_p),
                 ("w", (C.c_void_p * W_LAYER_COUNT) * MAX_LAYERS), ("arena_bytes", C.c_size_t),
-                ("lm_head", C.c_void_p)]
+                ("lm_head", C.c_void_p), ("tcw", (C.c_void_p * 4) * MAX_LAYERS), ("tc_head", C.c_void_p)]
 
 
 class _State(C.Structure):
@@ -97,6 +97,10 @@ _SIGS = {
     "hgd_verify_log_bytes": ([C.POINTER(Config), _i, _i, C.POINTER(_sz)], _i),
     "hgd_decode_layer_stack_verify": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _p, _p, _sz, _p, _p], _i),
     "hgd_decode_layer_stack_keep": ([C.POINTER(_Model), C.POINTER(_State), _i, _p, _sz, _p, _p, _p], _i),
+    "hgd_model_tc_bytes": ([C.POINTER(Config), C.POINTER(_sz)], _i),
+    "hgd_model_tc_load": ([C.POINTER(Config), _p, _sz, _i, _i, _p, _p], _i),
+    "hgd_model_attach_tc": ([C.POINTER(_Model), _p, _sz], _i),
+    "hgd_decode_layer_stack_tc": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _p, _p, _p, _p, _p], _i),
     "hgd_check_stack_timeout": ([C.POINTER(_Model), C.POINTER(_State), _p, _i, _p, _i, _i, _i, _p, _p, _p], _i),
     "hgd_check_not_coresident": ([C.POINTER(_Model), C.POINTER(_State), _i], _i),
 }
@@ -383,9 +387,11 @@ def gdn_heads(cfg: dict) -> tuple:
 
 
 class Model:
-    """Weights in one device arena laid out by libhgd (hgd_model_tensor offsets)."""
+    """Weights in one device arena laid out by libhgd (hgd_model_tensor offsets).
+    With tc=True the weights are also packed for the tensor-core decode chain
+    (hgd_decode_layer_stack_tc) into a second arena."""
 
-    def __init__(self, cfg: dict, weights: dict, device="cuda"):
+    def __init__(self, cfg: dict, weights: dict, device="cuda", tc: bool = False):
         torch = _torch()
         self.cfg_dict = dict(cfg)
         self.cfg = make_config(cfg)
@@ -410,6 +416,30 @@ class Model:
         self.m = _Model()
         _check("hgd_model_init", _lib.hgd_model_init(C.byref(self.m), C.byref(self.cfg),
                                                      self.arena_u8.data_ptr(), nbytes.value))
+        self.tc_arena = None
+        if tc:
+            self._load_tc(weights, device)
+
+    def _load_tc(self, weights, device):
+        torch = _torch()
+        nb = C.c_size_t()
+        _check("hgd_model_tc_bytes", _lib.hgd_model_tc_bytes(C.byref(self.cfg), C.byref(nb)))
+        self.tc_arena = torch.zeros(nb.value + 256, dtype=torch.uint8, device=device)
+        pad = (-self.tc_arena.data_ptr()) % 256
+        base = self.tc_arena.data_ptr() + pad
+        stream = torch.cuda.current_stream()
+        items = [(-1, W_LM_HEAD if self.cfg_dict.get("untied_head") else W_EMBED,
+                  weights["lm_head"] if self.cfg_dict.get("untied_head") else weights["embed"])]
+        for l, lw in enumerate(weights["layers"]):
+            for name, tid in (("w_in", W_IN), ("w_out", W_OUT), ("w_gate", W_GATE), ("w_up", W_UP),
+                              ("w_down", W_DOWN)):
+                items.append((l, tid, lw[name]))
+        for layer, tid, arr in items:
+            src = torch.from_numpy(np.ascontiguousarray(arr, dtype=np.uint16).view(np.int16)).to(device)
+            _check("hgd_model_tc_load", _lib.hgd_model_tc_load(C.byref(self.cfg), base, nb.value, layer, tid,
+                                                                src.data_ptr(), stream.cuda_stream))
+            stream.synchronize()
+        _check("hgd_model_attach_tc", _lib.hgd_model_attach_tc(C.byref(self.m), base, nb.value))
 
     def _tensors(self, weights):
         yield "embed", W_EMBED, -1
@@ -502,6 +532,20 @@ def decode_layer_stack(model: Model, state: State, tokens, T: int, logits=None, 
     if argmax is None:
         argmax = torch.empty((state.B * T,), dtype=torch.int32, device=tokens.device)
     _check("hgd_decode_layer_stack", _lib.hgd_decode_layer_stack(
+        C.byref(model.m), C.byref(state.st), _ptr(tokens), T, _ptr(logits), _ptr(argmax), _ptr(S_rec),
+        _ptr(tail_rec), _ptr(status), _stream(stream)))
+    return argmax
+
+
+def decode_layer_stack_tc(model: Model, state: State, tokens, T: int, logits=None, argmax=None, S_rec=None,
+                          tail_rec=None, status=None, stream=None):
+    """One decode call through the tensor-core chain (the model must be built with
+    tc=True).  Returns argmax [B*T] int32 (device)."""
+    torch = _torch()
+    _need(tokens, torch.int32, "tokens")
+    if argmax is None:
+        argmax = torch.empty((state.B * T,), dtype=torch.int32, device=tokens.device)
+    _check("hgd_decode_layer_stack_tc", _lib.hgd_decode_layer_stack_tc(
         C.byref(model.m), C.byref(state.st), _ptr(tokens), T, _ptr(logits), _ptr(argmax), _ptr(S_rec),
         _ptr(tail_rec), _ptr(status), _stream(stream)))
     return argmax

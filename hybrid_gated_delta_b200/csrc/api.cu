@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "gdn.cuh"
 #include "gdn_chunk.cuh"
+#include "tc_chain.cuh"
 #include "gemv.cuh"
 #include "gemm_tc.cuh"
 #include "stack.cuh"
@@ -416,7 +417,7 @@ size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_
 
 enum ScratchIdx {
     SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
-    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_GN, SC_XN, SC_END, SC_COUNT
+    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_GN, SC_XN, SC_TCY, SC_TCLOG, SC_TCWS, SC_END, SC_COUNT
 };
 // The persistent launch's control region: control words, one 128-byte line per
 // phase counter, then the phase timestamps.
@@ -469,6 +470,10 @@ __global__ void k_pos_keep(int32_t* pos, const int32_t* keep, int32_t* status, i
 }
 
 // Split-K workspace of the stack: the largest any of its GEMVs uses at M rows.
+struct TcPlan;
+size_t tc_chain_ws_bytes(const Dims& d, int M);
+int64_t tc_rows128(int64_t n) { return (n + 127) / 128 * 128; }
+
 size_t stack_ws_bytes(const Dims& d, int M) {
     size_t w = 0;
     w = std::max(w, gemv_ws_bytes(M, (int)d.gdn_out, d.D, false));
@@ -500,6 +505,10 @@ void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     sz[SC_BAR] = kBarBytes;
     sz[SC_GN] = (size_t)M * d.H * d.dv * 2;  // the chain's gated-norm rows for calls of many rows
     sz[SC_XN] = (size_t)M * d.D * 2;         // the chain's RMSNorm rows for calls of many rows
+    // the tensor-core chain: projection outputs, logits, and its GEMMs' workspace
+    sz[SC_TCY] = (size_t)M * std::max<int64_t>(d.D, 2 * tc_rows128(d.I)) * 4;
+    sz[SC_TCLOG] = (size_t)M * d.V * 4;
+    sz[SC_TCWS] = tc_chain_ws_bytes(d, (int)M);
     size_t pos = 0;
     for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
     off[SC_END] = pos;
@@ -622,6 +631,45 @@ TcPlan tc_plan(int M, int N, int K) {
     return q;
 }
 bool tc_shape_ok(int M, int N, int K) { return M >= 1 && M <= TC_MAXN && N >= 1 && K >= TC_BK && K % TC_BK == 0 && K <= 65536; }
+
+// Workspace of the tensor-core chain's GEMMs for M token rows: the largest over
+// its projections (packed rows and split partials).
+size_t tc_chain_ws_bytes(const Dims& d, int M) {
+    if (M < 1 || M > TC_MAXN) return 0;
+    const int64_t shapes[6][2] = {{d.gdn_out, d.D}, {d.attn_out, d.D}, {d.D, (int64_t)d.H * d.dv},
+                                  {d.D, (int64_t)d.nq * d.hd}, {2 * tc_rows128(d.I), d.D}, {d.D, d.I}};
+    size_t w = 0;
+    for (auto& sh : shapes) {
+        const TcPlan q = tc_plan(M, (int)sh[0], (int)sh[1]);
+        w = std::max(w, q.xp_bytes + q.part_bytes);
+    }
+    const TcPlan qh = tc_plan(M, d.V, d.D);
+    return std::max(w, qh.xp_bytes + qh.part_bytes);
+}
+
+// The tensor-core chain's packed weights, in one arena: the head, then per layer
+// the in-projection, the out-projection, gate and up (one matrix: the gate rows,
+// then the up rows from row tc_rows128(I)) and the down-projection; each in the
+// GEMM's 128 x 64 core-matrix tiles, 256-byte aligned.  which: 0 in, 1 out,
+// 2 gate+up, 3 down; layer -1: the head.
+size_t tc_weight_bytes_of(int64_t N, int64_t K) { return al256((size_t)tc_rows128(N) * K * 2); }
+size_t tc_walk(const Dims& d, const hgd_config* c, int want_layer, int want_which, size_t* off) {
+    size_t pos = 0;
+    if (want_layer == -1 && off) *off = pos;
+    pos += tc_weight_bytes_of(d.V, d.D);
+    for (int l = 0; l < d.L; ++l) {
+        const bool att = is_attn_layer(c, l);
+        const int64_t sh[4][2] = {{att ? d.attn_out : d.gdn_out, d.D},
+                                  {d.D, att ? (int64_t)d.nq * d.hd : (int64_t)d.H * d.dv},
+                                  {2 * tc_rows128(d.I), d.D},
+                                  {d.D, d.I}};
+        for (int w = 0; w < 4; ++w) {
+            if (l == want_layer && w == want_which && off) *off = pos;
+            pos += tc_weight_bytes_of(sh[w][0], sh[w][1]);
+        }
+    }
+    return pos;
+}
 
 int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int N, int K, void* ws,
            int32_t* status, cudaStream_t s) {
@@ -1510,6 +1558,202 @@ int hgd_decode_layer_stack_keep(const hgd_model* m, const hgd_state* st, int T, 
     }
     int32_t* pos = reinterpret_cast<int32_t*>(A + st->off[SC_POS]);
     return launch_status(launch_pdl(k_pos_keep, dim3(1), dim3(32), 0, s, pos, keep, status_dev, B, T));
+}
+
+// ------------------------------------------------- tensor-core decode chain
+
+int hgd_model_tc_bytes(const hgd_config* cfg, size_t* bytes) {
+    if (!bytes) return HGD_ERR_INVALID_ARG;
+    Dims d;
+    int rc = dims_of(cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    if (d.D % TC_BK || d.I % TC_BK || (d.H * d.dv) % TC_BK || (d.nq * d.hd) % TC_BK) return HGD_ERR_UNSUPPORTED_SHAPE;
+    *bytes = tc_walk(d, cfg, -2, -2, nullptr);
+    return HGD_OK;
+}
+
+int hgd_model_tc_load(const hgd_config* cfg, void* tc_arena, size_t bytes, int layer, int tensor,
+                      const uint16_t* src, hgd_stream_t stream) {
+    size_t need = 0;
+    int rc = hgd_model_tc_bytes(cfg, &need);
+    if (rc) return rc;
+    if (!tc_arena || !src) return HGD_ERR_INVALID_ARG;
+    if (bytes < need) return HGD_ERR_BUFFER_TOO_SMALL;
+    if ((reinterpret_cast<uintptr_t>(tc_arena) & 255u) || !al16(src)) return HGD_ERR_MISALIGNED;
+    Dims d;
+    dims_of(cfg, &d);
+    if (layer < -1 || layer >= d.L) return HGD_ERR_INVALID_ARG;
+    int which = -1;
+    int64_t N = 0, K = 0, row0 = 0;
+    if (layer == -1) {
+        if (tensor != (d.untied ? HGD_W_LM_HEAD : HGD_W_EMBED)) return HGD_ERR_INVALID_ARG;
+        N = d.V; K = d.D;
+    } else {
+        const bool att = is_attn_layer(cfg, layer);
+        switch (tensor) {
+            case HGD_W_IN: which = 0; N = att ? d.attn_out : d.gdn_out; K = d.D; break;
+            case HGD_W_OUT: which = 1; N = d.D; K = att ? (int64_t)d.nq * d.hd : (int64_t)d.H * d.dv; break;
+            case HGD_W_GATE: which = 2; N = d.I; K = d.D; break;
+            case HGD_W_UP: which = 2; N = d.I; K = d.D; row0 = tc_rows128(d.I); break;
+            case HGD_W_DOWN: which = 3; N = d.D; K = d.I; break;
+            default: return HGD_ERR_INVALID_ARG;
+        }
+    }
+    size_t off = 0;
+    tc_walk(d, cfg, layer, which, &off);
+    uint16_t* dst = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(tc_arena) + off) + row0 * K;
+    return hgd_gemm_tc_pack_weight(src, dst, (int)N, (int)K, stream);
+}
+
+int hgd_model_attach_tc(hgd_model* m, const void* tc_arena, size_t bytes) {
+    if (!m || !tc_arena) return HGD_ERR_INVALID_ARG;
+    size_t need = 0;
+    int rc = hgd_model_tc_bytes(&m->cfg, &need);
+    if (rc) return rc;
+    if (bytes < need) return HGD_ERR_BUFFER_TOO_SMALL;
+    if (reinterpret_cast<uintptr_t>(tc_arena) & 255u) return HGD_ERR_MISALIGNED;
+    Dims d;
+    dims_of(&m->cfg, &d);
+    const uint8_t* base = static_cast<const uint8_t*>(tc_arena);
+    size_t off = 0;
+    tc_walk(d, &m->cfg, -1, 0, &off);
+    m->tc_head = reinterpret_cast<const uint16_t*>(base + off);
+    for (int l = 0; l < d.L; ++l)
+        for (int w = 0; w < 4; ++w) {
+            tc_walk(d, &m->cfg, l, w, &off);
+            m->tcw[l][w] = reinterpret_cast<const uint16_t*>(base + off);
+        }
+    return HGD_OK;
+}
+
+int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T, float* logits,
+                              int32_t* argmax, float* S_rec, float* tail_rec, int32_t* status_dev,
+                              hgd_stream_t stream) {
+    if (!m || !st || !st->arena || !tokens || !argmax) return HGD_ERR_INVALID_ARG;
+    if (T < 1 || T > st->Tmax) return HGD_ERR_INVALID_ARG;
+    if (!m->tc_head) return HGD_ERR_INVALID_ARG;  // no tensor-core weights attached
+    Dims d;
+    int rc = dims_of(&m->cfg, &d);
+    if (rc) return rc;
+    if ((rc = check_supported(d))) return rc;
+    const int B = st->B, M = B * T, Lmax = st->Lmax;
+    if (M > TC_MAXN) return HGD_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(tokens) || !al16(argmax) || (logits && !al16(logits)) || (S_rec && !al16(S_rec)) ||
+        (tail_rec && !al16(tail_rec)))
+        return HGD_ERR_MISALIGNED;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* A = static_cast<uint8_t*>(st->arena);
+    float* Sall = reinterpret_cast<float*>(A + st->off[SC_S]);
+    float* conv = reinterpret_cast<float*>(A + st->off[SC_CONV]);
+    bf16_t* kv = reinterpret_cast<bf16_t*>(A + st->off[SC_KV]);
+    int32_t* pos = reinterpret_cast<int32_t*>(A + st->off[SC_POS]);
+    bf16_t* resid = reinterpret_cast<bf16_t*>(A + st->off[SC_RESID]);
+    float* proj = reinterpret_cast<float*>(A + st->off[SC_PROJ]);
+    float* obuf = reinterpret_cast<float*>(A + st->off[SC_O]);
+    float* qrot = reinterpret_cast<float*>(A + st->off[SC_QROT]);
+    bf16_t* attn = reinterpret_cast<bf16_t*>(A + st->off[SC_ATTN]);
+    float* part = reinterpret_cast<float*>(A + st->off[SC_PART]);
+    bf16_t* mlp = reinterpret_cast<bf16_t*>(A + st->off[SC_MLP]);
+    bf16_t* gn_rows = reinterpret_cast<bf16_t*>(A + st->off[SC_GN]);
+    bf16_t* xn_rows = reinterpret_cast<bf16_t*>(A + st->off[SC_XN]);
+    float* ty = reinterpret_cast<float*>(A + st->off[SC_TCY]);
+    float* lg = logits ? logits : reinterpret_cast<float*>(A + st->off[SC_TCLOG]);
+    void* tws = A + st->off[SC_TCWS];
+    const float eps = m->cfg.norm_eps;
+    const int Ip = (int)tc_rows128(d.I);
+    auto norm_rows = [&](const bf16_t* gains, bool embed) -> int {
+        NormRowsParams q{resid, d.D, tokens, m->embed, d.V, resid, d.D, gains, eps, xn_rows, d.D, M, d.D, status_dev};
+        cudaError_t e = embed ? launch_pdl(k_norm_rows<true>, dim3((M + 7) / 8), dim3(256), 0, s, q)
+                              : launch_pdl(k_norm_rows<false>, dim3((M + 7) / 8), dim3(256), 0, s, q);
+        return launch_status(e);
+    };
+    auto gemm = [&](const uint16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int N, int K) -> int {
+        return tc_run(reinterpret_cast<const bf16_t*>(Wp), x, x_ld, y, M, N, K, tws, status_dev, s);
+    };
+    auto resid_add = [&]() -> int {
+        const int64_t n = (int64_t)M * d.D;
+        return launch_status(launch_pdl(k_tc_resid, dim3((unsigned)std::min<int64_t>(592, (n + 255) / 256)),
+                                        dim3(256), 0, s, resid, (const float*)ty, n));
+    };
+    const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
+    const size_t c_layer = (size_t)B * (d.kc - 1) * d.C;
+    const size_t kv_half = (size_t)B * d.nkv * Lmax * d.hd;
+    const size_t srec_layer = (size_t)B * T * d.H * d.dv * d.dk;
+    const size_t trec_layer = (size_t)B * T * (d.kc - 1) * d.C;
+    int ig = 0, ia = 0;
+    for (int l = 0; l < d.L; ++l) {
+        const uint16_t* const* w = m->w[l];
+        const bool att = is_attn_layer(&m->cfg, l);
+        const int Nin = (int)(att ? d.attn_out : d.gdn_out);
+        // RMSNorm once per row (layer 0 gathers the embedding rows), the in-projection
+        if ((rc = norm_rows(w[HGD_W_IN_NORM], l == 0))) return rc;
+        if ((rc = gemm(m->tcw[l][0], xn_rows, d.D, proj, Nin, d.D))) return rc;
+        if (!att) {
+            TcConvParams cp{proj, Nin, conv + ig * c_layer, w[HGD_W_CONV],
+                            tail_rec ? tail_rec + ig * trec_layer : nullptr, B, T, (int)d.C};
+            const int64_t n = (int64_t)B * d.C;
+            if ((rc = launch_status(launch_pdl(k_tc_conv, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, cp))))
+                return rc;
+            GdnLayerParams g{};
+            g.proj = proj; g.proj_ld = Nin;
+            g.A_log = w[HGD_W_A_LOG]; g.dt_bias = w[HGD_W_DT_BIAS];
+            g.S = Sall + ig * s_layer;
+            g.o = obuf; g.o_ld = (int64_t)d.H * d.dv;
+            g.S_rec = S_rec ? S_rec + ig * srec_layer : nullptr;
+            g.B = B; g.T = T; g.H = d.H; g.dv = d.dv; g.Hk = d.Hk;
+            const dim3 grid(B * d.H, d.dv / GDN_ROWS), block(GDN_WARPS * 32);
+            cudaError_t e;
+            switch (d.dk) {
+                case 32: e = launch_pdl(k_gdn_layer<1>, grid, block, 0, s, g); break;
+                case 64: e = launch_pdl(k_gdn_layer<2>, grid, block, 0, s, g); break;
+                case 128: e = launch_pdl(k_gdn_layer<4>, grid, block, 0, s, g); break;
+                default: e = launch_pdl(k_gdn_layer<8>, grid, block, 0, s, g); break;
+            }
+            if ((rc = launch_status(e))) return rc;
+            GatedNormParams gq{obuf, (int64_t)d.H * d.dv, proj + d.C, Nin, w[HGD_W_GNORM], gn_rows,
+                               (int64_t)d.H * d.dv, M, d.H, d.dv, eps};
+            e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, gq);
+            if ((rc = launch_status(e))) return rc;
+            if ((rc = gemm(m->tcw[l][1], gn_rows, (int64_t)d.H * d.dv, ty, d.D, d.H * d.dv))) return rc;
+            ++ig;
+        } else {
+            TcRopeParams rp{proj, Nin, qrot, kv + (size_t)ia * 2 * kv_half, kv + (size_t)ia * 2 * kv_half + kv_half,
+                            pos, status_dev, T, d.nq, d.nkv, d.hd, Lmax, rope_inv1_of(d, m->cfg.rope_base)};
+            if ((rc = launch_status(launch_pdl(k_tc_rope, dim3(M), dim3(256), 0, s, rp)))) return rc;
+            AttnParams a{};
+            a.proj = proj; a.proj_ld = Nin; a.qrot = qrot;
+            a.kcache = kv + (size_t)ia * 2 * kv_half; a.vcache = a.kcache + kv_half;
+            a.pos = pos; a.part = part; a.out = attn; a.status = status_dev;
+            a.B = B; a.T = T; a.nq = d.nq; a.nkv = d.nkv; a.hd = d.hd; a.Lmax = Lmax;
+            a.max_chunks = max_chunks_of(Lmax);
+            cudaError_t e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(32 * (d.nq / d.nkv)), 0, s, a);
+            if ((rc = launch_status(e))) return rc;
+            e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
+            if ((rc = launch_status(e))) return rc;
+            if ((rc = gemm(m->tcw[l][1], attn, (int64_t)d.nq * d.hd, ty, d.D, d.nq * d.hd))) return rc;
+            ++ia;
+        }
+        if ((rc = resid_add())) return rc;
+        // MLP: RMSNorm once per row, gate and up in one GEMM, SwiGLU, down + residual
+        if ((rc = norm_rows(w[HGD_W_POST_NORM], false))) return rc;
+        if ((rc = gemm(m->tcw[l][2], xn_rows, d.D, ty, 2 * Ip, d.D))) return rc;
+        {
+            const int64_t n = (int64_t)M * d.I;
+            if ((rc = launch_status(launch_pdl(k_tc_swiglu, dim3((unsigned)std::min<int64_t>(1184, (n + 255) / 256)),
+                                               dim3(256), 0, s, (const float*)ty, (int64_t)2 * Ip, Ip, mlp, M, d.I))))
+                return rc;
+        }
+        if ((rc = gemm(m->tcw[l][3], mlp, d.I, ty, d.D, d.I))) return rc;
+        if ((rc = resid_add())) return rc;
+    }
+    // final RMSNorm, the head, the argmax of each row, the positions
+    if ((rc = norm_rows(m->final_norm, false))) return rc;
+    if ((rc = gemm(m->tc_head, xn_rows, d.D, lg, d.V, d.D))) return rc;
+    return launch_status(launch_pdl(k_tc_argmax, dim3(M), dim3(256), 0, s, (const float*)lg, (int64_t)d.V, d.V, argmax,
+                                    status_dev, pos, B, T));
 }
 
 }  // extern "C"

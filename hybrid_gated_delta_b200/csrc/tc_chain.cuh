@@ -1,0 +1,172 @@
+// tc_chain.cuh -- the per-row kernels of the tensor-core decode chain.
+//
+// "qwen3_5 cuda: mixed-width MLX checkpoints ... #849", PR body: windows of rows
+// (several streams of up to 16 rows each) whose rows equal one-row steps bit for
+// bit.  In the tensor-core chain every projection is one tcgen05 GEMM
+// (gemm_tc.cuh) over all of a call's token rows, and the tensor cores give each
+// token row the same result whatever the number of rows the call carries; the
+// kernels here are the work between the GEMMs, each computing every row from
+// that row's inputs alone.  So a window through this chain equals its one-row
+// steps through it, bit for bit, as the mma.sync chain's windows equal its
+// steps.  (The two chains sum their dot products in different orders: their
+// results agree to fp32 rounding, not bit for bit.)
+#pragma once
+
+#include "gemv.cuh"
+
+namespace hgd {
+
+// Causal conv over the first C columns of the in-projection rows, in place: one
+// thread per (stream, channel), rows in order, as k_conv_tail (tail records per
+// row when tail_rec is set).  Row (b, t) is x + (b*T + t) * x_ld.
+struct TcConvParams {
+    float* x; int64_t x_ld; float* tail; const bf16_t* w; float* tail_rec;
+    int B, T, C;
+};
+__global__ void k_tc_conv(const __grid_constant__ TcConvParams p) {
+    pdl_launch();
+    pdl_wait();
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)p.B * p.C) return;
+    const int b = (int)(idx / p.C), c = (int)(idx % p.C);
+    constexpr int NT = GV_CONV_K - 1;
+    float tl[NT], w[GV_CONV_K];
+#pragma unroll
+    for (int j = 0; j < GV_CONV_K; ++j) w[j] = bf2f(p.w[(int64_t)c * GV_CONV_K + j]);
+    float* tb = p.tail + (int64_t)b * NT * p.C + c;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) tl[j] = tb[(int64_t)j * p.C];
+    for (int t = 0; t < p.T; ++t) {
+        const int64_t row = (int64_t)b * p.T + t;
+        float* xr = p.x + row * p.x_ld + c;
+        const float xv = *xr;
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) acc = fmaf(w[j], tl[j], acc);
+        acc = fmaf(w[NT], xv, acc);
+        *xr = silu_f(acc);
+#pragma unroll
+        for (int j = 0; j + 1 < NT; ++j) tl[j] = tl[j + 1];
+        tl[NT - 1] = xv;
+        if (p.tail_rec)
+#pragma unroll
+            for (int j = 0; j < NT; ++j) p.tail_rec[(row * NT + j) * p.C + c] = tl[j];
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) tb[(int64_t)j * p.C] = tl[j];
+}
+
+// RoPE of the query and key heads of each row and the append of its key and
+// value rows to the cache at position pos[b] + t (rotate-half pairs (i, i +
+// hd/2), base^(-2i/hd) angles as the mma.sync chain's epilogue computes them).
+// In-projection rows, logical order: q (nq*hd) | gate (nq*hd) | k (nkv*hd) |
+// v (nkv*hd) at y + m * y_ld.  One CTA per token row.
+struct TcRopeParams {
+    const float* y; int64_t y_ld;
+    float* qrot;                     // [M][nq*hd]
+    bf16_t* kcache; bf16_t* vcache;  // this layer: [B][nkv][Lmax][hd]
+    const int32_t* pos; int32_t* status;
+    int T, nq, nkv, hd, Lmax;
+    double inv1;
+};
+__global__ void k_tc_rope(const __grid_constant__ TcRopeParams p) {
+    pdl_launch();
+    pdl_wait();
+    const int m = blockIdx.x, b = m / p.T, t = m % p.T;
+    const int P = p.pos[b] + t, hd = p.hd, half = hd / 2;
+    const float* yr = p.y + (int64_t)m * p.y_ld;
+    if (P < 0 || P >= p.Lmax) {
+        if (threadIdx.x == 0) set_status(p.status, HGD_ERR_INVALID_ARG);
+        return;
+    }
+    const int nqp = p.nq * half, nkp = p.nkv * half;
+    for (int e = threadIdx.x; e < nqp + nkp + p.nkv * hd; e += blockDim.x) {
+        if (e < nqp + nkp) {
+            const bool isk = e >= nqp;
+            const int ee = isk ? e - nqp : e, head = ee / half, i = ee % half;
+            const float* src = yr + (isk ? 2 * (int64_t)p.nq * hd : 0) + (int64_t)head * hd;
+            const float a = src[i], bb = src[i + half];
+            float sn, cs;
+            rope_sincos(P, i, p.inv1, &sn, &cs);
+            const float x0 = a * cs - bb * sn, x1 = bb * cs + a * sn;
+            if (!isk) {
+                float* qo = p.qrot + (int64_t)m * p.nq * hd + (int64_t)head * hd;
+                qo[i] = x0;
+                qo[i + half] = x1;
+            } else {
+                bf16_t* ko = p.kcache + (((int64_t)b * p.nkv + head) * p.Lmax + P) * hd;
+                ko[i] = f2bf(x0);
+                ko[i + half] = f2bf(x1);
+            }
+        } else {
+            const int ev = e - nqp - nkp, g = ev / hd, d = ev % hd;
+            p.vcache[(((int64_t)b * p.nkv + g) * p.Lmax + P) * hd + d] =
+                f2bf(yr[2 * (int64_t)p.nq * hd + (int64_t)p.nkv * hd + (int64_t)g * hd + d]);
+        }
+    }
+}
+
+// resid[m][n] = bf16(resid[m][n] + y[m][n]) (the residual add of a projection).
+__global__ void k_tc_resid(bf16_t* resid, const float* y, int64_t n_elem) {
+    pdl_launch();
+    pdl_wait();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_elem; i += (int64_t)gridDim.x * blockDim.x)
+        resid[i] = f2bf(bf2f(resid[i]) + y[i]);
+}
+
+// h[m][i] = bf16(silu(g) * u): g = y[m][i], u = y[m][up0 + i] (gate rows, then the
+// up rows from row up0 of the combined projection).
+__global__ void k_tc_swiglu(const float* y, int64_t y_ld, int up0, bf16_t* h, int M, int I) {
+    pdl_launch();
+    pdl_wait();
+    const int64_t n = (int64_t)M * I;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = e / I, i = e % I;
+        const float* yr = y + m * y_ld;
+        h[e] = f2bf(silu_f(yr[i]) * yr[up0 + i]);
+    }
+}
+
+// argmax[m] over the fp32 logits row m (first maximum: lowest index on ties; a
+// NaN gives -1 and HGD_ERR_NAN); then, if pos is set, every stream's position
+// advances by T (block 0, after its row).  One CTA of 256 threads per row.
+__global__ void k_tc_argmax(const float* logits, int64_t ld, int V, int32_t* argmax, int32_t* status, int32_t* pos,
+                            int B, int T) {
+    pdl_launch();
+    pdl_wait();
+    const int m = blockIdx.x;
+    const float* lr = logits + (int64_t)m * ld;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    bool nan = false;
+    for (int i = threadIdx.x; i < V; i += blockDim.x) {
+        const float v = lr[i];
+        if (v != v) nan = true;
+        else if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+    }
+    __shared__ float sv[8];
+    __shared__ int si[8], sn[8];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    nan = __any_sync(0xffffffffu, nan);
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) { sv[w] = bv; si[w] = bi; sn[w] = nan; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        bool anynan = sn[0];
+        for (int k = 1; k < (int)(blockDim.x >> 5); ++k) {
+            anynan = anynan || sn[k];
+            if (sv[k] > bv || (sv[k] == bv && si[k] < bi)) { bv = sv[k]; bi = si[k]; }
+        }
+        argmax[m] = anynan ? -1 : bi;
+        if (anynan) set_status(status, HGD_ERR_NAN);
+        if (pos && m == 0)
+            for (int s = 0; s < B; ++s) pos[s] += T;
+    }
+}
+
+}  // namespace hgd

@@ -338,6 +338,10 @@ typedef struct hgd_model {
     const uint16_t* w[HGD_MAX_LAYERS][HGD_W_LAYER_COUNT];
     size_t arena_bytes;
     const uint16_t* lm_head;  /* HGD_W_LM_HEAD with untied_head, else NULL (the embedding serves) */
+    /* the tensor-core chain's weights (hgd_model_attach_tc), else NULL: per layer
+     * in-projection, out-projection, gate+up, down; the head */
+    const uint16_t* tcw[HGD_MAX_LAYERS][4];
+    const uint16_t* tc_head;
 } hgd_model;
 
 /* Bytes of the weight arena for `cfg` (every tensor 256-byte aligned). */
@@ -469,6 +473,35 @@ HGD_API int hgd_decode_layer_stack_keep(const hgd_model* m, const hgd_state* st,
 /* Number of kernel launches one hgd_decode_layer_stack call over B streams and
  * T rows issues (-1 on bad arguments). */
 HGD_API int hgd_decode_layer_stack_launches(const hgd_model* m, int B, int T);
+
+/* ------------------------------------------------- tensor-core chain ---
+ * [TF] PR body: windows of up to 16 rows of several streams per call, a
+ * window's rows equal to one-row steps bit for bit.  A second decode path whose
+ * projections are tcgen05 GEMMs (hgd_gemm_tc_bf16's kernel) over all of the
+ * call's token rows: for windows of many rows the projections become dense
+ * contractions that stream each weight once per call.  The tensor cores give a
+ * token row the same bits whatever the number of rows in the call, and every
+ * kernel between the GEMMs computes a row from that row's inputs alone, so a
+ * window through this path equals its one-row steps through it bit for bit.
+ * Its sums are ordered as the tensor cores order them, so it agrees with
+ * hgd_decode_layer_stack (the mma.sync path) to fp32 rounding, not bit for bit:
+ * decode a stream through one path.
+ *
+ * The weights, packed for the tensor cores, live in a second caller-owned
+ * arena of hgd_model_tc_bytes bytes (256-byte aligned): fill it tensor by tensor
+ * with hgd_model_tc_load from row-major bf16 copies (HGD_W_IN, HGD_W_OUT,
+ * HGD_W_GATE, HGD_W_UP, HGD_W_DOWN per layer; layer -1: HGD_W_EMBED for the tied
+ * head, HGD_W_LM_HEAD for an untied one), then hgd_model_attach_tc.  Requires
+ * hidden, mlp_inter, the GDN and attention widths to be multiples of 64.
+ * hgd_decode_layer_stack_tc: the arguments of hgd_decode_layer_stack; B*T up to
+ * 256 rows; logits may be NULL (the state arena then holds them). */
+HGD_API int hgd_model_tc_bytes(const hgd_config* cfg, size_t* bytes);
+HGD_API int hgd_model_tc_load(const hgd_config* cfg, void* tc_arena, size_t bytes, int layer, int tensor,
+                              const uint16_t* src, hgd_stream_t stream);
+HGD_API int hgd_model_attach_tc(hgd_model* m, const void* tc_arena, size_t bytes);
+HGD_API int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int32_t* tokens, int T,
+                                      float* logits, int32_t* argmax, float* S_rec, float* tail_rec,
+                                      int32_t* status_dev, hgd_stream_t stream);
 
 /* ------------------------------------------------------ stack diagnostics --
  * The same check on the persistent decode launch itself ([LUCE] Known issues:
