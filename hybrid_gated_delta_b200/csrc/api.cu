@@ -671,8 +671,11 @@ size_t tc_walk(const Dims& d, const hgd_config* c, int want_layer, int want_whic
     return pos;
 }
 
+// With resid set, the product is added to the bf16 rows resid[M][N] instead of
+// written to y (which is then scratch): split partials are reduced and added in
+// one pass, an unsplit product goes through y and one add.
 int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int N, int K, void* ws,
-           int32_t* status, cudaStream_t s) {
+           int32_t* status, cudaStream_t s, bf16_t* resid = nullptr) {
     const TcPlan q = tc_plan(M, N, K);
     static CtxCache<int> attr_done;
     if (ensure_smem_attr(k_gemm_tc, attr_done) != cudaSuccess) {
@@ -690,10 +693,16 @@ int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int
     prm.M = M; prm.N = N; prm.K = K; prm.NTp = q.NTp; prm.ldo = N;
     prm.n_blocks = q.n_blocks; prm.kb_per_split = q.kb_per_split; prm.stages = q.stages; prm.tmem_cols = q.tmem_cols;
     e = launch_pdl(k_gemm_tc, dim3(q.n_blocks * q.splits), dim3(TC_THREADS), tc_smem_bytes(q.NTp, q.stages), s, prm);
-    if (e != cudaSuccess || q.splits == 1) return launch_status(e);
+    if (e != cudaSuccess) return launch_status(e);
     const int64_t n = (int64_t)M * N;
-    return launch_status(launch_pdl(k_tc_reduce, dim3((unsigned)std::min<int64_t>(1184, (n + 255) / 256)), dim3(256),
-                                    0, s, (const float*)part, y, q.splits, n));
+    const dim3 rg((unsigned)std::min<int64_t>(1184, (n + 255) / 256));
+    if (resid) {
+        if (q.splits == 1)
+            return launch_status(launch_pdl(k_tc_resid, rg, dim3(256), 0, s, resid, (const float*)y, n));
+        return launch_status(launch_pdl(k_tc_reduce_resid, rg, dim3(256), 0, s, (const float*)part, resid, q.splits, n));
+    }
+    if (q.splits == 1) return HGD_OK;
+    return launch_status(launch_pdl(k_tc_reduce, rg, dim3(256), 0, s, (const float*)part, y, q.splits, n));
 }
 
 // A wait that nothing completes: the bounded mbarrier wait of the slab rings and
@@ -1673,10 +1682,9 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
     auto gemm = [&](const uint16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int N, int K) -> int {
         return tc_run(reinterpret_cast<const bf16_t*>(Wp), x, x_ld, y, M, N, K, tws, status_dev, s);
     };
-    auto resid_add = [&]() -> int {
-        const int64_t n = (int64_t)M * d.D;
-        return launch_status(launch_pdl(k_tc_resid, dim3((unsigned)std::min<int64_t>(592, (n + 255) / 256)),
-                                        dim3(256), 0, s, resid, (const float*)ty, n));
+    // a projection added to the residual rows (ty is its scratch)
+    auto gemm_resid = [&](const uint16_t* Wp, const bf16_t* x, int64_t x_ld, int K) -> int {
+        return tc_run(reinterpret_cast<const bf16_t*>(Wp), x, x_ld, ty, M, d.D, K, tws, status_dev, s, resid);
     };
     const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
     const size_t c_layer = (size_t)B * (d.kc - 1) * d.C;
@@ -1717,7 +1725,7 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
                                (int64_t)d.H * d.dv, M, d.H, d.dv, eps};
             e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, gq);
             if ((rc = launch_status(e))) return rc;
-            if ((rc = gemm(m->tcw[l][1], gn_rows, (int64_t)d.H * d.dv, ty, d.D, d.H * d.dv))) return rc;
+            if ((rc = gemm_resid(m->tcw[l][1], gn_rows, (int64_t)d.H * d.dv, d.H * d.dv))) return rc;
             ++ig;
         } else {
             TcRopeParams rp{proj, Nin, qrot, kv + (size_t)ia * 2 * kv_half, kv + (size_t)ia * 2 * kv_half + kv_half,
@@ -1733,10 +1741,9 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
             if ((rc = launch_status(e))) return rc;
             e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
             if ((rc = launch_status(e))) return rc;
-            if ((rc = gemm(m->tcw[l][1], attn, (int64_t)d.nq * d.hd, ty, d.D, d.nq * d.hd))) return rc;
+            if ((rc = gemm_resid(m->tcw[l][1], attn, (int64_t)d.nq * d.hd, d.nq * d.hd))) return rc;
             ++ia;
         }
-        if ((rc = resid_add())) return rc;
         // MLP: RMSNorm once per row, gate and up in one GEMM, SwiGLU, down + residual
         if ((rc = norm_rows(w[HGD_W_POST_NORM], false))) return rc;
         if ((rc = gemm(m->tcw[l][2], xn_rows, d.D, ty, 2 * Ip, d.D))) return rc;
@@ -1746,8 +1753,7 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
                                                dim3(256), 0, s, (const float*)ty, (int64_t)2 * Ip, Ip, mlp, M, d.I))))
                 return rc;
         }
-        if ((rc = gemm(m->tcw[l][3], mlp, d.I, ty, d.D, d.I))) return rc;
-        if ((rc = resid_add())) return rc;
+        if ((rc = gemm_resid(m->tcw[l][3], mlp, d.I, d.I))) return rc;
     }
     // final RMSNorm, the head, the argmax of each row, the positions
     if ((rc = norm_rows(m->final_norm, false))) return rc;

@@ -75,6 +75,12 @@ __device__ void attn_partial_warp_t(const float* q, const bf16_t* K, const bf16_
                                     int lane) {
     constexpr int hd = 32 * DPL, KB = 16;
     const int d0 = lane * DPL;
+    // this lane's share of every key and value row of the chunk into L1 now, so
+    // the loads below (keys in two batches, then values after the softmax) hit it
+    for (int j = 0; j < nk; ++j) {
+        prefetch_l1(K + (int64_t)(key0 + j) * hd + d0);
+        prefetch_l1(V + (int64_t)(key0 + j) * hd + d0);
+    }
     float qv[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) qv[i] = q[d0 + i];

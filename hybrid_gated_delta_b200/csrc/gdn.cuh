@@ -379,20 +379,47 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
 
+    // Each row's inputs (this thread's q and k elements, the warp's value rows,
+    // a and b) are loaded one row ahead, so their latency overlaps the row before.
+    constexpr int NL = (DK + GDN_WARPS * 32 - 1) / (GDN_WARPS * 32);
+    float qn[NL], kn[NL], vn[GDN_RPW], an = 0.f, bn = 0.f;
+    auto load_row = [&](int t) {
+        const float* pr = p.proj + ((int64_t)b * p.T + t) * p.proj_ld;
+#pragma unroll
+        for (int u = 0; u < NL; ++u) {
+            const int i = tid + u * GDN_WARPS * 32;
+            if (i < DK) {
+                qn[u] = pr[(int64_t)hk * DK + i];
+                kn[u] = pr[(int64_t)Hk * DK + (int64_t)hk * DK + i];
+            }
+        }
+        const float* vp = pr + 2 * (int64_t)Hk * DK + (int64_t)h * dv + row0;
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) vn[r] = vp[r];
+        if (warp == 2 && lane == 0) {
+            an = pr[C + (int64_t)H * dv + h];
+            bn = pr[C + (int64_t)H * dv + H + h];
+        }
+    };
+    if (p.T > 0) load_row(0);
+
     for (int t = 0; t < p.T; ++t) {
         const int64_t row = (int64_t)b * p.T + t;
-        const float* pr = p.proj + row * p.proj_ld;
         __syncthreads();
-        for (int i = tid; i < DK; i += GDN_WARPS * 32) {
-            qs[i] = pr[(int64_t)hk * DK + i];
-            ks[i] = pr[(int64_t)Hk * DK + (int64_t)hk * DK + i];
+#pragma unroll
+        for (int u = 0; u < NL; ++u) {
+            const int i = tid + u * GDN_WARPS * 32;
+            if (i < DK) { qs[i] = qn[u]; ks[i] = kn[u]; }
         }
+        float vrow[GDN_RPW];
+#pragma unroll
+        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vn[r];
+        const float a = an, braw = bn;
+        if (t + 1 < p.T) load_row(t + 1);
         __syncthreads();
         if (warp == 0) { const float sc = l2_scale<KPL>(qs, lane); if (lane == 0) coef[0] = sc; }
         if (warp == 1) { const float sc = l2_scale<KPL>(ks, lane); if (lane == 0) coef[1] = sc; }
         if (warp == 2 && lane == 0) {
-            const float a = pr[C + (int64_t)H * dv + h];
-            const float braw = pr[C + (int64_t)H * dv + H + h];
             const float g = -A * softplus_f(a + dtb);
             coef[2] = expf(g);
             coef[3] = sigmoid_f(braw);
@@ -401,10 +428,7 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
         float kv[KPL], qv[KPL];
 #pragma unroll
         for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
-        float vrow[GDN_RPW], o[GDN_RPW], dl[GDN_RPW];
-        const float* vp = pr + 2 * (int64_t)Hk * DK + (int64_t)h * dv + row0;
-#pragma unroll
-        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vp[r];
+        float o[GDN_RPW], dl[GDN_RPW];
         gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o, dl);
         if (lane < GDN_RPW) {
             float ov = o[0], dv_ = dl[0];

@@ -36,21 +36,30 @@ __global__ void k_tc_conv(const __grid_constant__ TcConvParams p) {
     float* tb = p.tail + (int64_t)b * NT * p.C + c;
 #pragma unroll
     for (int j = 0; j < NT; ++j) tl[j] = tb[(int64_t)j * p.C];
-    for (int t = 0; t < p.T; ++t) {
-        const int64_t row = (int64_t)b * p.T + t;
-        float* xr = p.x + row * p.x_ld + c;
-        const float xv = *xr;
-        float acc = 0.f;
+    constexpr int RB = 8;  // rows whose inputs are loaded together
+    for (int t0 = 0; t0 < p.T; t0 += RB) {
+        float xin[RB];
 #pragma unroll
-        for (int j = 0; j < NT; ++j) acc = fmaf(w[j], tl[j], acc);
-        acc = fmaf(w[NT], xv, acc);
-        *xr = silu_f(acc);
+        for (int u = 0; u < RB; ++u)
+            if (t0 + u < p.T) xin[u] = p.x[((int64_t)b * p.T + t0 + u) * p.x_ld + c];
 #pragma unroll
-        for (int j = 0; j + 1 < NT; ++j) tl[j] = tl[j + 1];
-        tl[NT - 1] = xv;
-        if (p.tail_rec)
+        for (int u = 0; u < RB; ++u) {
+            const int t = t0 + u;
+            if (t >= p.T) break;
+            const int64_t row = (int64_t)b * p.T + t;
+            const float xv = xin[u];
+            float acc = 0.f;
 #pragma unroll
-            for (int j = 0; j < NT; ++j) p.tail_rec[(row * NT + j) * p.C + c] = tl[j];
+            for (int j = 0; j < NT; ++j) acc = fmaf(w[j], tl[j], acc);
+            acc = fmaf(w[NT], xv, acc);
+            p.x[row * p.x_ld + c] = silu_f(acc);
+#pragma unroll
+            for (int j = 0; j + 1 < NT; ++j) tl[j] = tl[j + 1];
+            tl[NT - 1] = xv;
+            if (p.tail_rec)
+#pragma unroll
+                for (int j = 0; j < NT; ++j) p.tail_rec[(row * NT + j) * p.C + c] = tl[j];
+        }
     }
 #pragma unroll
     for (int j = 0; j < NT; ++j) tb[(int64_t)j * p.C] = tl[j];
@@ -112,6 +121,19 @@ __global__ void k_tc_resid(bf16_t* resid, const float* y, int64_t n_elem) {
     pdl_wait();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_elem; i += (int64_t)gridDim.x * blockDim.x)
         resid[i] = f2bf(bf2f(resid[i]) + y[i]);
+}
+
+// resid[i] = bf16(resid[i] + sum_s part[s][i]): the split-K partials of a
+// projection added in split order (as k_tc_reduce adds them) and the residual
+// add, in one pass.
+__global__ void k_tc_reduce_resid(const float* __restrict__ part, bf16_t* resid, int splits, int64_t n_elem) {
+    pdl_launch();
+    pdl_wait();
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_elem; e += (int64_t)gridDim.x * blockDim.x) {
+        float acc = part[e];
+        for (int s = 1; s < splits; ++s) acc += part[(int64_t)s * n_elem + e];
+        resid[e] = f2bf(bf2f(resid[e]) + acc);
+    }
 }
 
 // h[m][i] = bf16(silu(g) * u): g = y[m][i], u = y[m][up0 + i] (gate rows, then the
