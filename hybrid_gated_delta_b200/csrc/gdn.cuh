@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
     pdl_launch();
     pdl_wait();
     constexpr int DK = 32 * KPL;
-    __shared__ float qs[DK], ks[DK], coef[4];
+    __shared__ float qs2[2][DK], ks2[2][DK];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, dv = p.dv;
     const int b = blockIdx.x / H, h = blockIdx.x % H;
@@ -381,6 +381,9 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
 
     // Each row's inputs (this thread's q and k elements, the warp's value rows,
     // a and b) are loaded one row ahead, so their latency overlaps the row before.
+    // q and k go through shared memory (double-buffered by row parity); every warp
+    // forms their L2 scales and every lane the gates itself (the functions the
+    // one-row kernels use, so the values are the same), one barrier per row.
     constexpr int NL = (DK + GDN_WARPS * 32 - 1) / (GDN_WARPS * 32);
     float qn[NL], kn[NL], vn[GDN_RPW], an = 0.f, bn = 0.f;
     auto load_row = [&](int t) {
@@ -396,20 +399,19 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
         const float* vp = pr + 2 * (int64_t)Hk * DK + (int64_t)h * dv + row0;
 #pragma unroll
         for (int r = 0; r < GDN_RPW; ++r) vn[r] = vp[r];
-        if (warp == 2 && lane == 0) {
-            an = pr[C + (int64_t)H * dv + h];
-            bn = pr[C + (int64_t)H * dv + H + h];
-        }
+        an = pr[C + (int64_t)H * dv + h];
+        bn = pr[C + (int64_t)H * dv + H + h];
     };
     if (p.T > 0) load_row(0);
 
     for (int t = 0; t < p.T; ++t) {
         const int64_t row = (int64_t)b * p.T + t;
-        __syncthreads();
+        float* qsb = qs2[t & 1];
+        float* ksb = ks2[t & 1];
 #pragma unroll
         for (int u = 0; u < NL; ++u) {
             const int i = tid + u * GDN_WARPS * 32;
-            if (i < DK) { qs[i] = qn[u]; ks[i] = kn[u]; }
+            if (i < DK) { qsb[i] = qn[u]; ksb[i] = kn[u]; }
         }
         float vrow[GDN_RPW];
 #pragma unroll
@@ -417,19 +419,14 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
         const float a = an, braw = bn;
         if (t + 1 < p.T) load_row(t + 1);
         __syncthreads();
-        if (warp == 0) { const float sc = l2_scale<KPL>(qs, lane); if (lane == 0) coef[0] = sc; }
-        if (warp == 1) { const float sc = l2_scale<KPL>(ks, lane); if (lane == 0) coef[1] = sc; }
-        if (warp == 2 && lane == 0) {
-            const float g = -A * softplus_f(a + dtb);
-            coef[2] = expf(g);
-            coef[3] = sigmoid_f(braw);
-        }
-        __syncthreads();
+        const float qsc = l2_scale<KPL>(qsb, lane), ksc = l2_scale<KPL>(ksb, lane);
+        const float alpha = expf(-A * softplus_f(a + dtb));
+        const float beta = sigmoid_f(braw);
         float kv[KPL], qv[KPL];
 #pragma unroll
-        for (int e = 0; e < KPL; ++e) { qv[e] = qs[lane * KPL + e] * coef[0]; kv[e] = ks[lane * KPL + e] * coef[1]; }
+        for (int e = 0; e < KPL; ++e) { qv[e] = qsb[lane * KPL + e] * qsc; kv[e] = ksb[lane * KPL + e] * ksc; }
         float o[GDN_RPW], dl[GDN_RPW];
-        gdn_rows_step<KPL>(S, kv, qv, coef[2], coef[3], vrow, o, dl);
+        gdn_rows_step<KPL>(S, kv, qv, alpha, beta, vrow, o, dl);
         if (lane < GDN_RPW) {
             float ov = o[0], dv_ = dl[0];
 #pragma unroll
@@ -439,7 +436,7 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
         }
         if (p.log_delta && blockIdx.y == 0 && warp == 0) {
             st_vec<KPL>(p.log_k + (row * H + h) * DK + lane * KPL, kv);
-            if (lane == 0) p.log_alpha[row * H + h] = coef[2];
+            if (lane == 0) p.log_alpha[row * H + h] = alpha;
         }
         if (p.S_rec) {
             float* rp = p.S_rec + ((((int64_t)b * p.T + t) * H + h) * dv + row0) * DK + lane * KPL;
