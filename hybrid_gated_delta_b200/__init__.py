@@ -74,6 +74,7 @@ _SIGS = {
     "hgd_gemm_tc_weight_bytes": ([_i, _i, C.POINTER(_sz)], _i),
     "hgd_gemm_tc_pack_weight": ([_p, _p, _i, _i, _p], _i),
     "hgd_gemm_tc_workspace_bytes": ([_i, _i, _i, C.POINTER(_sz)], _i),
+    "hgd_gemm_tc_plan": ([_i, _i, _i, C.POINTER(_i), C.POINTER(_i)], _i),
     "hgd_gemm_tc_bf16": ([_p, _p, _p, _i, _i, _i, _p, _sz, _p, _p], _i),
     "hgd_conv1d_tail_update": ([_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p], _i),
     "hgd_gdn_decode_step": ([_p, _p, _p, _i64, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p], _i),

@@ -154,6 +154,26 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
+// The same, with the grid in clusters of cluster_x consecutive CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                               int cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------- GEMV plans
 // Row blocks below this count use split slabs (partials through the workspace)
@@ -417,7 +437,7 @@ size_t weight_walk(const Dims& d, const hgd_config* c, int want_layer, int want_
 
 enum ScratchIdx {
     SC_S = 0, SC_CONV, SC_KV, SC_POS, SC_RESID, SC_PROJ, SC_O, SC_QROT, SC_ATTN, SC_PART, SC_MLP,
-    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_GN, SC_XN, SC_TCY, SC_TCLOG, SC_TCWS, SC_END, SC_COUNT
+    SC_BESTV, SC_BESTI, SC_WS, SC_BAR, SC_GN, SC_XN, SC_TCY, SC_TCLOG, SC_END, SC_COUNT
 };
 // The persistent launch's control region: control words, one 128-byte line per
 // phase counter, then the phase timestamps.
@@ -471,8 +491,8 @@ __global__ void k_pos_keep(int32_t* pos, const int32_t* keep, int32_t* status, i
 
 // Split-K workspace of the stack: the largest any of its GEMVs uses at M rows.
 struct TcPlan;
-size_t tc_chain_ws_bytes(const Dims& d, int M);
 int64_t tc_rows128(int64_t n) { return (n + 127) / 128 * 128; }
+int64_t tc_rows64(int64_t n) { return (n + 63) / 64 * 64; }
 
 size_t stack_ws_bytes(const Dims& d, int M) {
     size_t w = 0;
@@ -496,19 +516,20 @@ void state_layout(const Dims& d, int B, int Tmax, int Lmax, size_t* off) {
     sz[SC_PROJ] = (size_t)M * std::max(d.gdn_out, d.attn_out) * 4;
     sz[SC_O] = (size_t)M * d.H * d.dv * 4;
     sz[SC_QROT] = (size_t)M * d.nq * d.hd * 4;
-    sz[SC_ATTN] = (size_t)M * d.nq * d.hd * 2;
+    // (the tensor-core chain keeps these rows packed for its GEMMs: NTp rows)
+    const size_t Mt = (size_t)std::max<int64_t>(M, tc_ntp((int)std::min<int64_t>(M, TC_MAXN)));
+    sz[SC_ATTN] = Mt * d.nq * d.hd * 2;
     sz[SC_PART] = (size_t)M * d.nq * max_chunks_of(Lmax) * (d.hd + 2) * 4;
-    sz[SC_MLP] = (size_t)M * d.I * 2;
+    sz[SC_MLP] = Mt * d.I * 2;
     sz[SC_BESTV] = (size_t)M * kBestG * 4;
     sz[SC_BESTI] = (size_t)M * kBestG * 4;
     sz[SC_WS] = stack_ws_bytes(d, (int)M);
     sz[SC_BAR] = kBarBytes;
-    sz[SC_GN] = (size_t)M * d.H * d.dv * 2;  // the chain's gated-norm rows for calls of many rows
-    sz[SC_XN] = (size_t)M * d.D * 2;         // the chain's RMSNorm rows for calls of many rows
-    // the tensor-core chain: projection outputs, logits, and its GEMMs' workspace
-    sz[SC_TCY] = (size_t)M * std::max<int64_t>(d.D, 2 * tc_rows128(d.I)) * 4;
+    sz[SC_GN] = Mt * d.H * d.dv * 2;  // the chain's gated-norm rows for calls of many rows
+    sz[SC_XN] = Mt * d.D * 2;         // the chain's RMSNorm rows for calls of many rows
+    // the tensor-core chain: the head's argmax partials and its logits
+    sz[SC_TCY] = (size_t)M * TC_AM_SLICES * 2 * 4;  // the head's argmax partials
     sz[SC_TCLOG] = (size_t)M * d.V * 4;
-    sz[SC_TCWS] = tc_chain_ws_bytes(d, (int)M);
     size_t pos = 0;
     for (int i = 0; i < SC_END; ++i) { off[i] = pos; pos += al256(sz[i]); }
     off[SC_END] = pos;
@@ -606,16 +627,20 @@ int sk_launch(const Dims& d, const SkParams& prm, size_t smem, int sms, cudaStre
 struct TcPlan {
     int NTp, n_blocks, kb_per_split, splits, stages;
     uint32_t tmem_cols;
-    size_t xp_bytes, part_bytes;
+    size_t xp_bytes;
 };
-TcPlan tc_plan(int M, int N, int K) {
+// swiglu: the epilogue pairs gate and up rows through shared memory.
+TcPlan tc_plan(int M, int N, int K, bool swiglu = false) {
     TcPlan q{};
     q.NTp = tc_ntp(M);
     q.n_blocks = tc_nblocks(N);
     const int nkb = K / TC_BK;
-    const int want = std::max(1, std::min(nkb, TC_TARGET_CTAS / q.n_blocks));
-    q.kb_per_split = (nkb + want - 1) / want;
-    q.splits = (nkb + q.kb_per_split - 1) / q.kb_per_split;
+    // splits: a power of two up to a portable cluster, so the grid fills about
+    // one wave of SMs; the last splits may get fewer K blocks (or none)
+    const int want = std::max(1, std::min(std::min(nkb, TC_TARGET_CTAS / q.n_blocks), TC_MAX_SPLITS));
+    q.splits = 1;
+    while (q.splits * 2 <= want) q.splits *= 2;
+    q.kb_per_split = (nkb + q.splits - 1) / q.splits;
     // more than one wave of CTAs: stages for two CTAs per SM, so one's epilogue
     // overlaps the other's stream; otherwise every stage that fits
     const int per_sm = q.n_blocks * q.splits > TC_TARGET_CTAS ? 2 : 1;
@@ -623,29 +648,19 @@ TcPlan tc_plan(int M, int N, int K) {
     q.stages = (int)std::min<size_t>(TC_MAX_STAGES, avail / tc_stage_bytes(q.NTp));
     if (q.stages < 2) q.stages = (int)std::min<size_t>(TC_MAX_STAGES, ((size_t)GV_SMEM_LIMIT - tc_smem_bytes(q.NTp, 0)) /
                                                                       tc_stage_bytes(q.NTp));
+    // with splits (or the SwiGLU pairing) the stages also hold the accumulator
+    if (q.splits > 1 || swiglu) {
+        const size_t bytes = q.splits > 1 ? tc_red_bytes(q.NTp, q.splits) : (size_t)q.NTp * TC_BM * 4;
+        const int need = (int)((bytes + tc_stage_bytes(q.NTp) - 1) / tc_stage_bytes(q.NTp));
+        q.stages = std::max(q.stages, need);
+    }
     uint32_t c = 32;
     while ((int)c < q.NTp) c <<= 1;
     q.tmem_cols = c;
     q.xp_bytes = ((size_t)q.NTp * K * 2 + 255) / 256 * 256;
-    q.part_bytes = q.splits > 1 ? (size_t)q.splits * M * N * 4 : 0;
     return q;
 }
 bool tc_shape_ok(int M, int N, int K) { return M >= 1 && M <= TC_MAXN && N >= 1 && K >= TC_BK && K % TC_BK == 0 && K <= 65536; }
-
-// Workspace of the tensor-core chain's GEMMs for M token rows: the largest over
-// its projections (packed rows and split partials).
-size_t tc_chain_ws_bytes(const Dims& d, int M) {
-    if (M < 1 || M > TC_MAXN) return 0;
-    const int64_t shapes[6][2] = {{d.gdn_out, d.D}, {d.attn_out, d.D}, {d.D, (int64_t)d.H * d.dv},
-                                  {d.D, (int64_t)d.nq * d.hd}, {2 * tc_rows128(d.I), d.D}, {d.D, d.I}};
-    size_t w = 0;
-    for (auto& sh : shapes) {
-        const TcPlan q = tc_plan(M, (int)sh[0], (int)sh[1]);
-        w = std::max(w, q.xp_bytes + q.part_bytes);
-    }
-    const TcPlan qh = tc_plan(M, d.V, d.D);
-    return std::max(w, qh.xp_bytes + qh.part_bytes);
-}
 
 // The tensor-core chain's packed weights, in one arena: the head, then per layer
 // the in-projection, the out-projection, gate and up (one matrix: the gate rows,
@@ -661,7 +676,7 @@ size_t tc_walk(const Dims& d, const hgd_config* c, int want_layer, int want_whic
         const bool att = is_attn_layer(c, l);
         const int64_t sh[4][2] = {{att ? d.attn_out : d.gdn_out, d.D},
                                   {d.D, att ? (int64_t)d.nq * d.hd : (int64_t)d.H * d.dv},
-                                  {2 * tc_rows128(d.I), d.D},
+                                  {2 * tc_rows64(d.I), d.D},  // gate and up, interleaved by 64 rows
                                   {d.D, d.I}};
         for (int w = 0; w < 4; ++w) {
             if (l == want_layer && w == want_which && off) *off = pos;
@@ -671,38 +686,41 @@ size_t tc_walk(const Dims& d, const hgd_config* c, int want_layer, int want_whic
     return pos;
 }
 
-// With resid set, the product is added to the bf16 rows resid[M][N] instead of
-// written to y (which is then scratch): split partials are reduced and added in
-// one pass, an unsplit product goes through y and one add.
+// With resid set, the product is added to the bf16 rows resid[M][N] by the
+// GEMM's epilogue instead of written to y.
+// x_packed: x already holds the token rows in the GEMM's layout (tc_x_elem, NTp
+// rows), and ws is not used.
+// h (with I): the SwiGLU epilogue (W packed by k_tc_pack_w_swiglu, N = 2 *
+// tc_rows64(I)); h receives bf16(silu(gate) * up) packed for the next GEMM.
 int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int N, int K, void* ws,
-           int32_t* status, cudaStream_t s, bf16_t* resid = nullptr) {
-    const TcPlan q = tc_plan(M, N, K);
+           int32_t* status, cudaStream_t s, bf16_t* resid = nullptr, bool x_packed = false, bf16_t* h = nullptr,
+           int I = 0) {
+    const TcPlan q = tc_plan(M, N, K, h != nullptr);
     static CtxCache<int> attr_done;
     if (ensure_smem_attr(k_gemm_tc, attr_done) != cudaSuccess) {
         cudaGetLastError();
         return HGD_ERR_CUDA;
     }
-    bf16_t* Xp = static_cast<bf16_t*>(ws);
-    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + q.xp_bytes);
-    const int chunks = q.NTp * (K / 8);
-    cudaError_t e = launch_pdl(k_tc_pack_x, dim3(std::min(1184, (chunks + 255) / 256)), dim3(256), 0, s, x, x_ld, Xp,
-                               M, K, q.NTp);
-    if (e != cudaSuccess) return launch_status(e);
-    TcParams prm{};
-    prm.Wp = Wp; prm.Xp = Xp; prm.out = q.splits > 1 ? part : y; prm.status = status;
-    prm.M = M; prm.N = N; prm.K = K; prm.NTp = q.NTp; prm.ldo = N;
-    prm.n_blocks = q.n_blocks; prm.kb_per_split = q.kb_per_split; prm.stages = q.stages; prm.tmem_cols = q.tmem_cols;
-    e = launch_pdl(k_gemm_tc, dim3(q.n_blocks * q.splits), dim3(TC_THREADS), tc_smem_bytes(q.NTp, q.stages), s, prm);
-    if (e != cudaSuccess) return launch_status(e);
-    const int64_t n = (int64_t)M * N;
-    const dim3 rg((unsigned)std::min<int64_t>(1184, (n + 255) / 256));
-    if (resid) {
-        if (q.splits == 1)
-            return launch_status(launch_pdl(k_tc_resid, rg, dim3(256), 0, s, resid, (const float*)y, n));
-        return launch_status(launch_pdl(k_tc_reduce_resid, rg, dim3(256), 0, s, (const float*)part, resid, q.splits, n));
+    const bf16_t* Xp = x;
+    cudaError_t e;
+    if (!x_packed) {
+        bf16_t* xp = static_cast<bf16_t*>(ws);
+        const int chunks = q.NTp * (K / 8);
+        e = launch_pdl(k_tc_pack_x, dim3(std::min(1184, (chunks + 255) / 256)), dim3(256), 0, s, x, x_ld, xp, M, K,
+                       q.NTp);
+        if (e != cudaSuccess) return launch_status(e);
+        Xp = xp;
     }
-    if (q.splits == 1) return HGD_OK;
-    return launch_status(launch_pdl(k_tc_reduce, rg, dim3(256), 0, s, (const float*)part, y, q.splits, n));
+    TcParams prm{};
+    prm.Wp = Wp; prm.Xp = Xp; prm.out = y; prm.resid = resid; prm.h = h; prm.I = I; prm.status = status;
+    prm.M = M; prm.N = N; prm.K = K; prm.NTp = q.NTp; prm.ldo = N;
+    prm.n_blocks = q.n_blocks; prm.kb_per_split = q.kb_per_split; prm.splits = q.splits; prm.stages = q.stages;
+    prm.tmem_cols = q.tmem_cols;
+    const dim3 grid(q.n_blocks * q.splits), block(TC_THREADS);
+    const size_t smem = tc_smem_bytes(q.NTp, q.stages);
+    e = q.splits > 1 ? launch_pdl_cluster(k_gemm_tc, grid, block, smem, s, q.splits, prm)
+                     : launch_pdl(k_gemm_tc, grid, block, smem, s, prm);
+    return launch_status(e);
 }
 
 // A wait that nothing completes: the bounded mbarrier wait of the slab rings and
@@ -879,7 +897,16 @@ int hgd_gemm_tc_workspace_bytes(int M, int N, int K, size_t* bytes) {
     if (!bytes || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
     if (!tc_shape_ok(M, N, K)) return HGD_ERR_UNSUPPORTED_SHAPE;
     const TcPlan q = tc_plan(M, N, K);
-    *bytes = q.xp_bytes + q.part_bytes;
+    *bytes = q.xp_bytes;
+    return HGD_OK;
+}
+
+int hgd_gemm_tc_plan(int M, int N, int K, int* splits, int* stages) {
+    if (!splits || !stages || M < 1 || N < 1 || K < 1) return HGD_ERR_INVALID_ARG;
+    if (!tc_shape_ok(M, N, K)) return HGD_ERR_UNSUPPORTED_SHAPE;
+    const TcPlan q = tc_plan(M, N, K);
+    *splits = q.splits;
+    *stages = q.stages;
     return HGD_OK;
 }
 
@@ -889,7 +916,7 @@ int hgd_gemm_tc_bf16(const uint16_t* Wp, const uint16_t* x, float* y, int M, int
     if (!tc_shape_ok(M, N, K)) return HGD_ERR_UNSUPPORTED_SHAPE;
     if (!al16(Wp) || !al16(x) || !al16(y) || !al16(workspace)) return HGD_ERR_MISALIGNED;
     const TcPlan q = tc_plan(M, N, K);
-    if (workspace_bytes < q.xp_bytes + q.part_bytes) return HGD_ERR_BUFFER_TOO_SMALL;
+    if (workspace_bytes < q.xp_bytes) return HGD_ERR_BUFFER_TOO_SMALL;
     DevInfo di;
     int rc = device_info(&di);
     if (rc) return rc;
@@ -1427,7 +1454,8 @@ static int chain_run(const hgd_model* m, const hgd_state* st, const int32_t* tok
             a.pos = pos; a.part = part; a.out = attn; a.status = status_dev;
             a.B = B; a.T = T; a.nq = d.nq; a.nkv = d.nkv; a.hd = d.hd; a.Lmax = Lmax;
             a.max_chunks = max_chunks_of(Lmax);
-            cudaError_t e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(32 * (d.nq / d.nkv)), 0, s, a);
+            cudaError_t e = launch_pdl(k_attn_partial, dim3(B, d.nkv, a.max_chunks), dim3(32 * ATTN_PART_WARPS),
+                                       attn_part_smem_bytes(d.hd), s, a);
             if ((rc = launch_status(e))) return rc;
             e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
             if ((rc = launch_status(e))) return rc;
@@ -1594,7 +1622,8 @@ int hgd_model_tc_load(const hgd_config* cfg, void* tc_arena, size_t bytes, int l
     dims_of(cfg, &d);
     if (layer < -1 || layer >= d.L) return HGD_ERR_INVALID_ARG;
     int which = -1;
-    int64_t N = 0, K = 0, row0 = 0;
+    int64_t N = 0, K = 0;
+    int half = -1;
     if (layer == -1) {
         if (tensor != (d.untied ? HGD_W_LM_HEAD : HGD_W_EMBED)) return HGD_ERR_INVALID_ARG;
         N = d.V; K = d.D;
@@ -1603,16 +1632,20 @@ int hgd_model_tc_load(const hgd_config* cfg, void* tc_arena, size_t bytes, int l
         switch (tensor) {
             case HGD_W_IN: which = 0; N = att ? d.attn_out : d.gdn_out; K = d.D; break;
             case HGD_W_OUT: which = 1; N = d.D; K = att ? (int64_t)d.nq * d.hd : (int64_t)d.H * d.dv; break;
-            case HGD_W_GATE: which = 2; N = d.I; K = d.D; break;
-            case HGD_W_UP: which = 2; N = d.I; K = d.D; row0 = tc_rows128(d.I); break;
+            case HGD_W_GATE: which = 2; N = d.I; K = d.D; half = 0; break;
+            case HGD_W_UP: which = 2; N = d.I; K = d.D; half = 1; break;
             case HGD_W_DOWN: which = 3; N = d.D; K = d.I; break;
             default: return HGD_ERR_INVALID_ARG;
         }
     }
     size_t off = 0;
     tc_walk(d, cfg, layer, which, &off);
-    uint16_t* dst = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(tc_arena) + off) + row0 * K;
-    return hgd_gemm_tc_pack_weight(src, dst, (int)N, (int)K, stream);
+    uint16_t* dst = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(tc_arena) + off);
+    if (half < 0) return hgd_gemm_tc_pack_weight(src, dst, (int)N, (int)K, stream);
+    const int64_t chunks = tc_rows64(N) * (K / 8);
+    k_tc_pack_w_swiglu<<<(unsigned)std::min<int64_t>(4736, (chunks + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const bf16_t*>(src), reinterpret_cast<bf16_t*>(dst), (int)N, (int)K, half);
+    return launch_status(cudaGetLastError());
 }
 
 int hgd_model_attach_tc(hgd_model* m, const void* tc_arena, size_t bytes) {
@@ -1670,21 +1703,24 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
     bf16_t* xn_rows = reinterpret_cast<bf16_t*>(A + st->off[SC_XN]);
     float* ty = reinterpret_cast<float*>(A + st->off[SC_TCY]);
     float* lg = logits ? logits : reinterpret_cast<float*>(A + st->off[SC_TCLOG]);
-    void* tws = A + st->off[SC_TCWS];
     const float eps = m->cfg.norm_eps;
-    const int Ip = (int)tc_rows128(d.I);
+    const int64_t Ih = tc_rows64(d.I);
+    // every GEMM input is written straight into the GEMM's packed layout (NTp
+    // rows; the rows past M are never read back into a result)
+    const int NTp = tc_ntp(M);
     auto norm_rows = [&](const bf16_t* gains, bool embed) -> int {
-        NormRowsParams q{resid, d.D, tokens, m->embed, d.V, resid, d.D, gains, eps, xn_rows, d.D, M, d.D, status_dev};
+        NormRowsParams q{resid, d.D, tokens, m->embed, d.V, resid, d.D, gains, eps, xn_rows, d.D, M, d.D, status_dev,
+                         NTp};
         cudaError_t e = embed ? launch_pdl(k_norm_rows<true>, dim3((M + 7) / 8), dim3(256), 0, s, q)
                               : launch_pdl(k_norm_rows<false>, dim3((M + 7) / 8), dim3(256), 0, s, q);
         return launch_status(e);
     };
     auto gemm = [&](const uint16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int N, int K) -> int {
-        return tc_run(reinterpret_cast<const bf16_t*>(Wp), x, x_ld, y, M, N, K, tws, status_dev, s);
+        return tc_run(reinterpret_cast<const bf16_t*>(Wp), x, x_ld, y, M, N, K, nullptr, status_dev, s, nullptr, true);
     };
     // a projection added to the residual rows (ty is its scratch)
     auto gemm_resid = [&](const uint16_t* Wp, const bf16_t* x, int64_t x_ld, int K) -> int {
-        return tc_run(reinterpret_cast<const bf16_t*>(Wp), x, x_ld, ty, M, d.D, K, tws, status_dev, s, resid);
+        return tc_run(reinterpret_cast<const bf16_t*>(Wp), x, x_ld, ty, M, d.D, K, nullptr, status_dev, s, resid, true);
     };
     const size_t s_layer = (size_t)B * d.H * d.dv * d.dk;
     const size_t c_layer = (size_t)B * (d.kc - 1) * d.C;
@@ -1722,7 +1758,7 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
             }
             if ((rc = launch_status(e))) return rc;
             GatedNormParams gq{obuf, (int64_t)d.H * d.dv, proj + d.C, Nin, w[HGD_W_GNORM], gn_rows,
-                               (int64_t)d.H * d.dv, M, d.H, d.dv, eps};
+                               (int64_t)d.H * d.dv, M, d.H, d.dv, eps, NTp};
             e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, gq);
             if ((rc = launch_status(e))) return rc;
             if ((rc = gemm_resid(m->tcw[l][1], gn_rows, (int64_t)d.H * d.dv, d.H * d.dv))) return rc;
@@ -1737,29 +1773,34 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
             a.pos = pos; a.part = part; a.out = attn; a.status = status_dev;
             a.B = B; a.T = T; a.nq = d.nq; a.nkv = d.nkv; a.hd = d.hd; a.Lmax = Lmax;
             a.max_chunks = max_chunks_of(Lmax);
-            cudaError_t e = launch_pdl(k_attn_partial, dim3(M, d.nkv, a.max_chunks), dim3(32 * (d.nq / d.nkv)), 0, s, a);
+            a.pack_ntp = NTp;
+            cudaError_t e = launch_pdl(k_attn_partial, dim3(B, d.nkv, a.max_chunks), dim3(32 * ATTN_PART_WARPS),
+                                       attn_part_smem_bytes(d.hd), s, a);
             if ((rc = launch_status(e))) return rc;
             e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
             if ((rc = launch_status(e))) return rc;
             if ((rc = gemm_resid(m->tcw[l][1], attn, (int64_t)d.nq * d.hd, d.nq * d.hd))) return rc;
             ++ia;
         }
-        // MLP: RMSNorm once per row, gate and up in one GEMM, SwiGLU, down + residual
+        // MLP: RMSNorm once per row, gate and up in one GEMM whose epilogue forms the
+        // SwiGLU rows (packed for the down GEMM), down + residual
         if ((rc = norm_rows(w[HGD_W_POST_NORM], false))) return rc;
-        if ((rc = gemm(m->tcw[l][2], xn_rows, d.D, ty, 2 * Ip, d.D))) return rc;
-        {
-            const int64_t n = (int64_t)M * d.I;
-            if ((rc = launch_status(launch_pdl(k_tc_swiglu, dim3((unsigned)std::min<int64_t>(1184, (n + 255) / 256)),
-                                               dim3(256), 0, s, (const float*)ty, (int64_t)2 * Ip, Ip, mlp, M, d.I))))
-                return rc;
-        }
+        if ((rc = tc_run(reinterpret_cast<const bf16_t*>(m->tcw[l][2]), xn_rows, d.D, nullptr, M, (int)(2 * Ih),
+                         d.D, nullptr, status_dev, s, nullptr, true, mlp, d.I)))
+            return rc;
         if ((rc = gemm_resid(m->tcw[l][3], mlp, d.I, d.I))) return rc;
     }
     // final RMSNorm, the head, the argmax of each row, the positions
     if ((rc = norm_rows(m->final_norm, false))) return rc;
     if ((rc = gemm(m->tc_head, xn_rows, d.D, lg, d.V, d.D))) return rc;
-    return launch_status(launch_pdl(k_tc_argmax, dim3(M), dim3(256), 0, s, (const float*)lg, (int64_t)d.V, d.V, argmax,
-                                    status_dev, pos, B, T));
+    // the argmax partials in the projection scratch (free after the last layer)
+    float* am_v = ty;
+    int* am_i = reinterpret_cast<int*>(ty + (size_t)M * TC_AM_SLICES);
+    if ((rc = launch_status(launch_pdl(k_tc_argmax_part, dim3(M, TC_AM_SLICES), dim3(256), 0, s, (const float*)lg,
+                                       (int64_t)d.V, d.V, am_v, am_i))))
+        return rc;
+    return launch_status(launch_pdl(k_tc_argmax_final, dim3(M), dim3(32), 0, s, (const float*)am_v, (const int*)am_i,
+                                    argmax, status_dev, pos, B, T));
 }
 
 }  // extern "C"

@@ -36,6 +36,7 @@ struct AttnParams {
     bf16_t* out;                         // [M][nq*hd]
     int32_t* status;
     int B, T, nq, nkv, hd, Lmax, max_chunks;
+    int pack_ntp;  // > 0: out holds the rows packed for the tensor-core GEMM (tc_x_elem, NTp rows)
 };
 
 // One attention partial, computed by one warp: query q (fp32, rotated) over
@@ -70,24 +71,29 @@ __device__ __forceinline__ float attn_elem(const AttnRow<DPL>& r, int i) {
     return (i & 1) ? bf_hi(r.w[i >> 1]) : bf_lo(r.w[i >> 1]);
 }
 
-template <int DPL>
+// PF: K and V are in global memory and this lane's share of the chunk is
+// prefetched into L1 first; without it they may be shared-memory rows.
+template <int DPL, bool PF = true>
 __device__ void attn_partial_warp_t(const float* q, const bf16_t* K, const bf16_t* V, int key0, int nk, float* dst,
                                     int lane) {
     constexpr int hd = 32 * DPL, KB = 16;
     const int d0 = lane * DPL;
     // this lane's share of every key and value row of the chunk into L1 now, so
     // the loads below (keys in two batches, then values after the softmax) hit it
-    for (int j = 0; j < nk; ++j) {
-        prefetch_l1(K + (int64_t)(key0 + j) * hd + d0);
-        prefetch_l1(V + (int64_t)(key0 + j) * hd + d0);
-    }
+    if (PF)
+        for (int j = 0; j < nk; ++j) {
+            prefetch_l1(K + (int64_t)(key0 + j) * hd + d0);
+            prefetch_l1(V + (int64_t)(key0 + j) * hd + d0);
+        }
     float qv[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) qv[i] = q[d0 + i];
-    float sc = -INFINITY;  // lane j: key j's scaled score
+    // this lane's share of every key's dot product, then all 32 summed over the
+    // lanes at once (warp_sum_transposed: warp_sum's pairings, so each score is
+    // bitwise warp_sum's), which leaves key j's in lane j
+    float dd[32];
 #pragma unroll
     for (int b = 0; b < 32; b += KB) {
-        if (b >= nk) break;
         AttnRow<DPL> kr[KB];
 #pragma unroll
         for (int j = 0; j < KB; ++j) {
@@ -99,13 +105,13 @@ __device__ void attn_partial_warp_t(const float* q, const bf16_t* K, const bf16_
         }
 #pragma unroll
         for (int j = 0; j < KB; ++j) {
-            float dd = 0.f;
+            dd[b + j] = 0.f;
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) dd = fmaf(qv[i], attn_elem<DPL>(kr[j], i), dd);
-            dd = warp_sum(dd);
-            if (lane == b + j && b + j < nk) sc = dd * (1.0f / sqrtf((float)hd));
+            for (int i = 0; i < DPL; ++i) dd[b + j] = fmaf(qv[i], attn_elem<DPL>(kr[j], i), dd[b + j]);
         }
     }
+    const float tot = warp_sum_transposed<32>(dd, lane);
+    const float sc = lane < nk ? tot * (1.0f / sqrtf((float)hd)) : -INFINITY;  // lane j: key j's scaled score
     float m = sc;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -172,47 +178,114 @@ __device__ __forceinline__ bf16_t attn_merge_dim(const float* base, int nch, int
     return f2bf(acc / L * sigmoid_f(gate));
 }
 
-// grid (M, nkv, max_chunks), block 32 * group (one warp per query head of the
-// group; group <= 8).  Chunk of ATTN_CHUNK (= 32) keys, one key per lane.
-__global__ void __launch_bounds__(32 * ATTN_MAX_GROUP) k_attn_partial(const __grid_constant__ AttnParams p) {
+// grid (B, nkv, max_chunks), block 256: one CTA per (stream, kv head, chunk of
+// ATTN_CHUNK keys) stages the chunk's key and value rows in shared memory once,
+// then its eight warps take the (row, query head) pairs of the stream's T rows
+// whose position reaches the chunk, each with attn_partial_warp_t's arithmetic
+// (the same partial, bit for bit, as one warp per pair reading the cache).
+constexpr int ATTN_PART_WARPS = 8;
+__host__ __device__ inline size_t attn_part_smem_bytes(int hd) { return (size_t)2 * ATTN_CHUNK * hd * 2; }
+__global__ void __launch_bounds__(32 * ATTN_PART_WARPS) k_attn_partial(const __grid_constant__ AttnParams p) {
+    extern __shared__ __align__(16) uint8_t attn_smem[];
     pdl_launch();
     pdl_wait();
-    const int row = blockIdx.x, g = blockIdx.y, ch = blockIdx.z;
-    const int b = row / p.T, t = row % p.T;
-    const int P = p.pos[b] + t;
-    if (P < 0 || P >= p.Lmax) return;
-    const int key0 = ch * ATTN_CHUNK;
-    if (key0 > P) return;
-    const int nk = min(ATTN_CHUNK, P + 1 - key0);
-    const int group = p.nq / p.nkv, hd = p.hd;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = g * group + warp;  // this warp's query head
-    const bf16_t* K = p.kcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd;
-    const bf16_t* V = p.vcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd;
-    const float* q = p.qrot + (int64_t)row * p.nq * hd + (int64_t)h * hd;
-    float* dst = p.part + (((int64_t)row * p.nq + h) * p.max_chunks + ch) * (hd + 2);
-    attn_partial_warp(q, K, V, key0, nk, hd, dst, lane);
+    const int b = blockIdx.x, g = blockIdx.y, ch = blockIdx.z, hd = p.hd;
+    const int key0 = ch * ATTN_CHUNK, pos = p.pos[b];
+    // the rows of this stream with a valid position that reaches the chunk
+    int tlo = max(0, key0 - pos), thi = min(p.T, p.Lmax - pos);
+    if (pos < 0) tlo = max(tlo, -pos);
+    if (tlo >= thi) return;
+    const int nkc = min(ATTN_CHUNK, pos + thi - key0);  // keys the chunk's last row sees
+    const bf16_t* K = p.kcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd + (int64_t)key0 * hd;
+    const bf16_t* V = p.vcache + ((int64_t)b * p.nkv + g) * p.Lmax * hd + (int64_t)key0 * hd;
+    bf16_t* Ks = reinterpret_cast<bf16_t*>(attn_smem);
+    bf16_t* Vs = Ks + ATTN_CHUNK * hd;
+    const int n16 = nkc * hd / 8;
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) {
+        reinterpret_cast<uint4*>(Ks)[i] = reinterpret_cast<const uint4*>(K)[i];
+        reinterpret_cast<uint4*>(Vs)[i] = reinterpret_cast<const uint4*>(V)[i];
+    }
+    __syncthreads();
+    const int group = p.nq / p.nkv, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int pi = tlo * group + warp; pi < thi * group; pi += ATTN_PART_WARPS) {
+        const int t = pi / group, h = g * group + pi % group, row = b * p.T + t;
+        const int nk = min(ATTN_CHUNK, pos + t + 1 - key0);
+        const float* q = p.qrot + (int64_t)row * p.nq * hd + (int64_t)h * hd;
+        float* dst = p.part + (((int64_t)row * p.nq + h) * p.max_chunks + ch) * (hd + 2);
+        switch (hd) {
+            case 256: attn_partial_warp_t<8, false>(q, Ks, Vs, 0, nk, dst, lane); break;
+            case 128: attn_partial_warp_t<4, false>(q, Ks, Vs, 0, nk, dst, lane); break;
+            case 64: attn_partial_warp_t<2, false>(q, Ks, Vs, 0, nk, dst, lane); break;
+            default: attn_partial_warp_t<1, false>(q, Ks, Vs, 0, nk, dst, lane); break;
+        }
+    }
 }
 
-// grid (M, nq), block hd.
+// grid (M, nq), block hd: the merge of attn_merge_max / attn_merge_dim, with
+// every load issued up front (thread c: chunk c's m and l; thread d: its gate
+// and the first ATTN_MERGE_Q chunks' values of dim d) and w_c = exp(m_c - M)
+// formed once per chunk into shared memory; max is exact and w_c the same
+// expression, so the result is theirs bit for bit.
+constexpr int ATTN_MERGE_Q = 24;
+constexpr int ATTN_MAX_CHUNKS = 512;  // positions up to 16384
 __global__ void __launch_bounds__(256) k_attn_merge(const __grid_constant__ AttnParams p) {
+    __shared__ float wv[ATTN_MAX_CHUNKS], lv[ATTN_MAX_CHUNKS], wm[8];
     pdl_launch();
     pdl_wait();
     const int row = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
     const int b = row / p.T, t = row % p.T;
     const int P = p.pos[b] + t;
     const int hd = p.hd;
-    bf16_t* out = p.out + (int64_t)row * p.nq * hd + (int64_t)h * hd;
+    bf16_t* out = p.pack_ntp ? p.out + tc_x_elem(row, h * hd + d, p.pack_ntp)
+                             : p.out + (int64_t)row * p.nq * hd + (int64_t)h * hd + d;
     if (P < 0 || P >= p.Lmax) {
-        if (d < hd) out[d] = 0;
+        if (d < hd) *out = 0;
         return;
     }
-    if (d >= hd) return;
     const int nch = P / ATTN_CHUNK + 1;
     const float* base = p.part + ((int64_t)row * p.nq + h) * p.max_chunks * (hd + 2);
-    const float M = attn_merge_max(base, nch, hd);
-    const float gate = p.proj[(int64_t)row * p.proj_ld + p.nq * hd + (int64_t)h * hd + d];
-    out[d] = attn_merge_dim(base, nch, hd, M, d, gate);
+    float a[ATTN_MERGE_Q];
+    float gate = 0.f;
+    if (d < hd) {
+        gate = p.proj[(int64_t)row * p.proj_ld + p.nq * hd + (int64_t)h * hd + d];
+#pragma unroll
+        for (int c = 0; c < ATTN_MERGE_Q; ++c) a[c] = c < nch ? base[c * (hd + 2) + 2 + d] : 0.f;
+    }
+    float mx = -INFINITY;
+    for (int c = d; c < nch; c += blockDim.x) {
+        const float2 ml = *reinterpret_cast<const float2*>(base + c * (hd + 2));
+        wv[c] = ml.x;
+        lv[c] = ml.y;
+        mx = fmaxf(mx, ml.x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((d & 31) == 0) wm[d >> 5] = mx;
+    __syncthreads();
+    float M = wm[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) M = fmaxf(M, wm[w]);
+    for (int c = d; c < nch; c += blockDim.x) wv[c] = expf(wv[c] - M);
+    __syncthreads();
+    if (d >= hd) return;
+    float L = 0.f, acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < ATTN_MERGE_Q; ++c)
+        if (c < nch) {
+            L = fmaf(wv[c], lv[c], L);
+            acc = fmaf(wv[c], a[c], acc);
+        }
+    for (int c0 = ATTN_MERGE_Q; c0 < nch; c0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = c0 + u < nch ? base[(c0 + u) * (hd + 2) + 2 + d] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (c0 + u < nch) {
+                L = fmaf(wv[c0 + u], lv[c0 + u], L);
+                acc = fmaf(wv[c0 + u], v[u], acc);
+            }
+    }
+    *out = f2bf(acc / L * sigmoid_f(gate));
 }
 
 }  // namespace hgd

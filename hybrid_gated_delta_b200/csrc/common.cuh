@@ -40,6 +40,33 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Sums over the warp of N = 2, 4, 8, 16 or 32 values per lane (x[i] the lane's
+// share of sum i), with warp_sum's pairings: level m pairs lane l with l ^ m
+// (m = 16, 8, 4, 2, 1), so every total is bitwise warp_sum(x[i]).  At each level
+// a lane keeps half of its running sums (the lower half where bit m of the lane
+// is clear) and sends the other half, so the whole reduction takes about N - 1
+// shuffles instead of 5 N.  Afterwards sum i sits in the lanes whose bits
+// 4..(5 - log2 N) spell i from the top; returned is this lane's sum.
+template <int N>
+__device__ __forceinline__ float warp_sum_transposed(float (&x)[N], int lane) {
+    static_assert(N == 2 || N == 4 || N == 8 || N == 16 || N == 32, "N");
+#pragma unroll
+    for (int m = 16, c = N; m >= 1 && c > 1; m >>= 1, c >>= 1) {
+        const bool up = lane & m;
+#pragma unroll
+        for (int i = 0; i < c / 2; ++i) {
+            const float keep = up ? x[i + c / 2] : x[i], send = up ? x[i] : x[i + c / 2];
+            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    float v = x[0];
+    // the levels below the last split: plain butterfly on the one sum left
+#pragma unroll
+    for (int m = 16 >> (N == 32 ? 5 : N == 16 ? 4 : N == 8 ? 3 : N == 4 ? 2 : 1); m >= 1; m >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, m);
+    return v;
+}
+
 __device__ __forceinline__ unsigned long long globaltimer() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -173,6 +200,17 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------- tensor-core operand layout
+// Token rows as the tensor-core GEMM (gemm_tc.cuh) reads them: per 64-wide k
+// block a tile of NTp rows in 8 x 8 core matrices (8 rows of 16 bytes, 128
+// contiguous bytes), core (row group g, k group j) at element (g * 8 + j) * 64.
+// Element offset of X[t][k]; the 8 elements of an aligned k octet are contiguous.
+constexpr int TC_BK = 64;  // k per block (and per GEMM pipeline stage)
+__host__ __device__ inline size_t tc_x_elem(int t, int k, int NTp) {
+    const int kk = k & (TC_BK - 1);
+    return (size_t)(k >> 6) * NTp * TC_BK + (size_t)(((t >> 3) * 8 + (kk >> 3)) * 64 + (t & 7) * 8 + (kk & 7));
 }
 
 // Named barrier over the first `nthreads` threads of the CTA (id 1..15).

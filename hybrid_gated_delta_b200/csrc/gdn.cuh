@@ -68,26 +68,40 @@ __device__ __forceinline__ void gdn_row_update(float (&S)[KPL], float delta, con
 
 // One recurrent row for RPW state rows held by this warp.  kv/qv: this lane's
 // normalised key/query elements; vrow[r]: value of state row r; returns o and
-// the row's writes delta (every lane).
+// the row's writes delta (every lane).  The RPW dot products of a kind are
+// summed over the lanes together (warp_sum_transposed: warp_sum's pairings, so
+// each sum is bitwise warp_sum's) and then broadcast.
 template <int KPL>
 __device__ __forceinline__ void gdn_rows_step(float (&S)[GDN_RPW][KPL], const float (&kv)[KPL],
                                               const float (&qv)[KPL], float alpha, float beta,
                                               const float (&vrow)[GDN_RPW], float (&o)[GDN_RPW],
                                               float (&dl)[GDN_RPW]) {
+    constexpr int LPR = 32 / GDN_RPW;  // lanes holding each sum after the transposed reduction
+    const int lane = threadIdx.x & 31;
+    float w[GDN_RPW];
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) {
-        float w = 0.f;
+        w[r] = 0.f;
 #pragma unroll
-        for (int e = 0; e < KPL; ++e) w = fmaf(S[r][e], kv[e], w);
-        w = warp_sum(w);
-        const float delta = beta * (vrow[r] - alpha * w);
+        for (int e = 0; e < KPL; ++e) w[r] = fmaf(S[r][e], kv[e], w[r]);
+    }
+    const float ws = warp_sum_transposed<GDN_RPW>(w, lane);
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) {
+        const float delta = beta * (vrow[r] - alpha * __shfl_sync(0xffffffffu, ws, r * LPR));
         dl[r] = delta;
         gdn_row_update<KPL>(S[r], delta, kv, alpha);
-        float ov = 0.f;
-#pragma unroll
-        for (int e = 0; e < KPL; ++e) ov = fmaf(S[r][e], qv[e], ov);
-        o[r] = warp_sum(ov);
     }
+    float ov[GDN_RPW];
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) {
+        ov[r] = 0.f;
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) ov[r] = fmaf(S[r][e], qv[e], ov[r]);
+    }
+    const float os = warp_sum_transposed<GDN_RPW>(ov, lane);
+#pragma unroll
+    for (int r = 0; r < GDN_RPW; ++r) o[r] = __shfl_sync(0xffffffffu, os, r * LPR);
 }
 
 // L2 normalisation scale 1/sqrt(sum x^2 + 1e-6) of a dk-vector held in shared
@@ -360,12 +374,22 @@ struct GdnLayerParams {
     int Hk;  // query/key heads (H, the value heads, is a multiple): value head h reads head h / (H / Hk)
 };
 
+// Rows whose inputs k_gdn_layer stages in shared memory at once.
+constexpr int GDN_TB = 16;
+
 template <int KPL>
 __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_constant__ GdnLayerParams p) {
     pdl_launch();
     pdl_wait();
-    constexpr int DK = 32 * KPL;
-    __shared__ float qs2[2][DK], ks2[2][DK];
+    constexpr int DK = 32 * KPL, NT = GDN_WARPS * 32;
+    // A block of up to GDN_TB rows at a time: every input of the block (q and k
+    // of the key head, this CTA's value rows, a and b) is loaded in one batch,
+    // the rows' L2 scales and gates are formed in parallel, and then only the
+    // recurrence runs row after row, from shared memory, with no barrier.  Each
+    // value comes from the function the one-row kernels use (l2_scale, the gate
+    // expressions, gdn_rows_step), so the results are theirs bit for bit.
+    __shared__ float qs[GDN_TB][DK], ks[GDN_TB][DK], vs[GDN_TB][GDN_ROWS];
+    __shared__ float qsc[GDN_TB], ksc[GDN_TB], al[GDN_TB], be[GDN_TB];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, dv = p.dv;
     const int b = blockIdx.x / H, h = blockIdx.x % H;
@@ -379,70 +403,83 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
 
-    // Each row's inputs (this thread's q and k elements, the warp's value rows,
-    // a and b) are loaded one row ahead, so their latency overlaps the row before.
-    // q and k go through shared memory (double-buffered by row parity); every warp
-    // forms their L2 scales and every lane the gates itself (the functions the
-    // one-row kernels use, so the values are the same), one barrier per row.
-    constexpr int NL = (DK + GDN_WARPS * 32 - 1) / (GDN_WARPS * 32);
-    float qn[NL], kn[NL], vn[GDN_RPW], an = 0.f, bn = 0.f;
-    auto load_row = [&](int t) {
-        const float* pr = p.proj + ((int64_t)b * p.T + t) * p.proj_ld;
+    constexpr int QN = GDN_TB * DK / NT;  // q (and k) elements of a block per thread
+    static_assert(GDN_TB * DK % NT == 0 && GDN_TB * GDN_ROWS <= 2 * NT, "block staging");
+    for (int t0 = 0; t0 < p.T; t0 += GDN_TB) {
+        const int n = min(GDN_TB, p.T - t0);
+        const float* pr0 = p.proj + ((int64_t)b * p.T + t0) * p.proj_ld;
+        {
+            float qr[QN], kr[QN], vr[2];
 #pragma unroll
-        for (int u = 0; u < NL; ++u) {
-            const int i = tid + u * GDN_WARPS * 32;
-            if (i < DK) {
-                qn[u] = pr[(int64_t)hk * DK + i];
-                kn[u] = pr[(int64_t)Hk * DK + (int64_t)hk * DK + i];
+            for (int u = 0; u < QN; ++u) {
+                const int i = tid + u * NT, t = i / DK, e = i % DK;
+                const float* pr = pr0 + (int64_t)t * p.proj_ld;
+                qr[u] = t < n ? pr[(int64_t)hk * DK + e] : 0.f;
+                kr[u] = t < n ? pr[(int64_t)Hk * DK + (int64_t)hk * DK + e] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = tid + u * NT, t = i / GDN_ROWS, r = i % GDN_ROWS;
+                vr[u] = (i < GDN_TB * GDN_ROWS && t < n)
+                            ? pr0[(int64_t)t * p.proj_ld + 2 * (int64_t)Hk * DK + (int64_t)h * dv +
+                                  blockIdx.y * GDN_ROWS + r]
+                            : 0.f;
+            }
+            float ar = 0.f, br = 0.f;
+            if (tid < n) {
+                ar = pr0[(int64_t)tid * p.proj_ld + C + (int64_t)H * dv + h];
+                br = pr0[(int64_t)tid * p.proj_ld + C + (int64_t)H * dv + H + h];
+            }
+#pragma unroll
+            for (int u = 0; u < QN; ++u) {
+                const int i = tid + u * NT;
+                qs[i / DK][i % DK] = qr[u];
+                ks[i / DK][i % DK] = kr[u];
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = tid + u * NT;
+                if (i < GDN_TB * GDN_ROWS) vs[i / GDN_ROWS][i % GDN_ROWS] = vr[u];
+            }
+            if (tid < n) {
+                al[tid] = expf(-A * softplus_f(ar + dtb));
+                be[tid] = sigmoid_f(br);
             }
         }
-        const float* vp = pr + 2 * (int64_t)Hk * DK + (int64_t)h * dv + row0;
-#pragma unroll
-        for (int r = 0; r < GDN_RPW; ++r) vn[r] = vp[r];
-        an = pr[C + (int64_t)H * dv + h];
-        bn = pr[C + (int64_t)H * dv + H + h];
-    };
-    if (p.T > 0) load_row(0);
-
-    for (int t = 0; t < p.T; ++t) {
-        const int64_t row = (int64_t)b * p.T + t;
-        float* qsb = qs2[t & 1];
-        float* ksb = ks2[t & 1];
-#pragma unroll
-        for (int u = 0; u < NL; ++u) {
-            const int i = tid + u * GDN_WARPS * 32;
-            if (i < DK) { qsb[i] = qn[u]; ksb[i] = kn[u]; }
-        }
-        float vrow[GDN_RPW];
-#pragma unroll
-        for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vn[r];
-        const float a = an, braw = bn;
-        if (t + 1 < p.T) load_row(t + 1);
         __syncthreads();
-        const float qsc = l2_scale<KPL>(qsb, lane), ksc = l2_scale<KPL>(ksb, lane);
-        const float alpha = expf(-A * softplus_f(a + dtb));
-        const float beta = sigmoid_f(braw);
-        float kv[KPL], qv[KPL];
-#pragma unroll
-        for (int e = 0; e < KPL; ++e) { qv[e] = qsb[lane * KPL + e] * qsc; kv[e] = ksb[lane * KPL + e] * ksc; }
-        float o[GDN_RPW], dl[GDN_RPW];
-        gdn_rows_step<KPL>(S, kv, qv, alpha, beta, vrow, o, dl);
-        if (lane < GDN_RPW) {
-            float ov = o[0], dv_ = dl[0];
-#pragma unroll
-            for (int r = 1; r < GDN_RPW; ++r) if (lane == r) { ov = o[r]; dv_ = dl[r]; }
-            p.o[row * p.o_ld + (int64_t)h * dv + row0 + lane] = ov;
-            if (p.log_delta) p.log_delta[(row * H + h) * dv + row0 + lane] = dv_;
+        for (int t = warp; t < n; t += GDN_WARPS) {
+            const float a = l2_scale<KPL>(qs[t], lane), c = l2_scale<KPL>(ks[t], lane);
+            if (lane == 0) { qsc[t] = a; ksc[t] = c; }
         }
-        if (p.log_delta && blockIdx.y == 0 && warp == 0) {
-            st_vec<KPL>(p.log_k + (row * H + h) * DK + lane * KPL, kv);
-            if (lane == 0) p.log_alpha[row * H + h] = alpha;
-        }
-        if (p.S_rec) {
-            float* rp = p.S_rec + ((((int64_t)b * p.T + t) * H + h) * dv + row0) * DK + lane * KPL;
+        __syncthreads();
+        for (int t = 0; t < n; ++t) {
+            const int64_t row = (int64_t)b * p.T + t0 + t;
+            const float qa = qsc[t], ka = ksc[t], alpha = al[t], beta = be[t];
+            float kv[KPL], qv[KPL], vrow[GDN_RPW];
 #pragma unroll
-            for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
+            for (int e = 0; e < KPL; ++e) { qv[e] = qs[t][lane * KPL + e] * qa; kv[e] = ks[t][lane * KPL + e] * ka; }
+#pragma unroll
+            for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vs[t][warp * GDN_RPW + r];
+            float o[GDN_RPW], dl[GDN_RPW];
+            gdn_rows_step<KPL>(S, kv, qv, alpha, beta, vrow, o, dl);
+            if (lane < GDN_RPW) {
+                float ov = o[0], dv_ = dl[0];
+#pragma unroll
+                for (int r = 1; r < GDN_RPW; ++r) if (lane == r) { ov = o[r]; dv_ = dl[r]; }
+                p.o[row * p.o_ld + (int64_t)h * dv + row0 + lane] = ov;
+                if (p.log_delta) p.log_delta[(row * H + h) * dv + row0 + lane] = dv_;
+            }
+            if (p.log_delta && blockIdx.y == 0 && warp == 0) {
+                st_vec<KPL>(p.log_k + (row * H + h) * DK + lane * KPL, kv);
+                if (lane == 0) p.log_alpha[row * H + h] = alpha;
+            }
+            if (p.S_rec) {
+                float* rp = p.S_rec + ((row * H + h) * dv + row0) * DK + lane * KPL;
+#pragma unroll
+                for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
+            }
         }
+        __syncthreads();  // the next block's inputs overwrite these
     }
     if (p.log_delta) return;  // a verify window: the state stays as it was
 #pragma unroll

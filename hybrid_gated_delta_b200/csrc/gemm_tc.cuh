@@ -22,8 +22,12 @@
 // 128 contiguous bytes), core (row group g, k group j) of a tile at byte
 // (g * 8 + j) * 128, so the leading-dimension (k) stride is 128 bytes and the
 // stride-dimension (8-row group) stride is 1024 bytes.  A fixed split of K over
-// CTAs (a function of N and K only) fills the SMs for short-N projections; its
-// partials are added in split order by a second kernel.
+// CTAs (a function of N and K only, at most 8) fills the SMs for short-N
+// projections.  The splits of a 128-row block run as one thread-block cluster:
+// each CTA parks its accumulator in its own shared memory, and after a cluster
+// barrier CTA r sums the r-th share of the token rows over the cluster's
+// shared memories in split order and writes it, so the partials never leave
+// the SMs.  The epilogue writes fp32 rows or adds them to bf16 residual rows.
 //
 // Every wait is bounded (HGD_ERR_TIMEOUT in *status), the producer waits for
 // its copies before the CTA leaves, the issuer's final commit covers every MMA
@@ -34,12 +38,12 @@
 namespace hgd {
 
 constexpr int TC_BM = 128;                    // W rows per tile (the MMA's M)
-constexpr int TC_BK = 64;                     // K per stage (four MMAs of K = 16)
 constexpr int TC_MAXN = 256;                  // token rows per call (the MMA's N)
 constexpr int TC_THREADS = 128;
 constexpr int TC_WTILE = TC_BM * TC_BK;       // elements of a weight tile (16 KB)
 constexpr int TC_MAX_STAGES = 8;
 constexpr int TC_TARGET_CTAS = 148;           // split-K target: one wave of B200 SMs
+constexpr int TC_MAX_SPLITS = 8;              // a portable cluster
 
 __host__ __device__ inline int tc_ntp(int M) { return M <= 16 ? 16 : (M + 15) / 16 * 16; }
 __host__ __device__ inline int tc_nblocks(int N) { return (N + TC_BM - 1) / TC_BM; }
@@ -51,11 +55,7 @@ __host__ __device__ inline size_t tc_w_elem(int n, int k, int K) {
     const size_t tile = (size_t)(n >> 7) * (K / TC_BK) + (k >> 6);
     return tile * TC_WTILE + (size_t)(((r >> 3) * 8 + (kk >> 3)) * 64 + (r & 7) * 8 + (kk & 7));
 }
-// Packed token rows: for each k block a tile of NTp rows x 64 in the same core order.
-__host__ __device__ inline size_t tc_x_elem(int t, int k, int NTp) {
-    const int kk = k & (TC_BK - 1);
-    return (size_t)(k >> 6) * NTp * TC_BK + (size_t)(((t >> 3) * 8 + (kk >> 3)) * 64 + (t & 7) * 8 + (kk & 7));
-}
+// Packed token rows: tc_x_elem (common.cuh), the same core order per k block.
 
 // One 16-byte chunk (8 consecutive k) per thread: rows n >= N are zero.
 __global__ void k_tc_pack_w(const bf16_t* __restrict__ W, bf16_t* __restrict__ Wp, int N, int K) {
@@ -65,6 +65,18 @@ __global__ void k_tc_pack_w(const bf16_t* __restrict__ W, bf16_t* __restrict__ W
         const int n = (int)(e / cpr), k = (int)(e % cpr) * 8;
         const uint4 v = n < N ? *reinterpret_cast<const uint4*>(W + (int64_t)n * K + k) : make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(Wp + tc_w_elem(n, k, K)) = v;
+    }
+}
+// The gate (half 0) or up (half 1) rows [N, K] of a SwiGLU projection into the
+// interleaved packed matrix: source row n goes to row (n / 64) * 128 + half * 64
+// + n % 64; rows past N are zero.
+__global__ void k_tc_pack_w_swiglu(const bf16_t* __restrict__ W, bf16_t* __restrict__ Wp, int N, int K, int half) {
+    const int cpr = K / 8;
+    const int64_t total = (int64_t)((N + 63) / 64) * 64 * cpr;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int n = (int)(e / cpr), k = (int)(e % cpr) * 8;
+        const uint4 v = n < N ? *reinterpret_cast<const uint4*>(W + (int64_t)n * K + k) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(Wp + tc_w_elem((n >> 6) * 128 + half * 64 + (n & 63), k, K)) = v;
     }
 }
 __global__ void k_tc_pack_x(const bf16_t* __restrict__ X, int64_t x_ld, bf16_t* __restrict__ Xp, int M, int K,
@@ -120,16 +132,64 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 struct TcParams {
     const bf16_t* Wp;   // packed weight (tc_w_elem), N padded to 128-row tiles
     const bf16_t* Xp;   // packed token rows (tc_x_elem), NTp rows
-    float* out;         // splits == 1: Y [M][ldo]; else partials [splits][M][ldo]
+    float* out;         // Y [M][ldo] (fp32), when resid and h are null
+    bf16_t* resid;      // or: resid[t][n] = bf16(resid[t][n] + Y[t][n]), [M][ldo]
+    bf16_t* h;          // or (SwiGLU): W holds gate and up rows interleaved by 64 (k_tc_pack_w_swiglu);
+    int I;              //   h[t][i] = bf16(silu(gate_i) * up_i), i < I, packed (tc_x_elem, NTp rows)
     int32_t* status;    // optional: HGD_ERR_TIMEOUT if a wait ran out
     int M, N, K, NTp, ldo;
-    int n_blocks, kb_per_split, stages;
+    int n_blocks, kb_per_split, splits, stages;  // splits: the cluster size (1: no cluster)
     uint32_t tmem_cols;
 };
 
+// ------------------------------------------------ cluster shared memory
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+// (no memory clobber: these loads follow a cluster barrier, whose clobber orders
+// them, and a batch of them must issue back to back)
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ int ld_dsmem_s32(uint32_t a) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+// SwiGLU of token rows t_lo.. t_hi - 1 of row block nb from st (row t at
+// st[(t - t_lo) * 128 ..]: 64 gate rows, then the 64 matching up rows).
+__device__ __forceinline__ void tc_swiglu_rows(const TcParams& p, const float* st, int t_lo, int t_hi, int nb,
+                                               int tid) {
+    for (int e = tid; e < (t_hi - t_lo) * 64; e += TC_THREADS) {
+        const int tt = e >> 6, il = e & 63, i = nb * 64 + il, t = t_lo + tt;
+        if (i < p.I && t < p.M)
+            p.h[tc_x_elem(t, i, p.NTp)] = f2bf(silu_f(st[tt * TC_BM + il]) * st[tt * TC_BM + 64 + il]);
+    }
+}
+__device__ __forceinline__ void tc_store(const TcParams& p, int t, int n, float v) {
+    const size_t e = (size_t)t * p.ldo + n;
+    if (p.resid) p.resid[e] = f2bf(bf2f(p.resid[e]) + v);
+    else p.out[e] = v;
+}
+
 // Shared memory: stages x (weight tile 16 KB, token tile NTp x 128 B), then the
-// full / empty / done mbarriers, the TMEM address and the abort flag.
+// full / empty / done mbarriers, the TMEM address and the abort flag.  With
+// splits, the stages then hold the accumulator (NTp x 128 fp32, tc_red_bytes):
+// the plan gives enough stages for it.
 __host__ __device__ inline size_t tc_stage_bytes(int NTp) { return (size_t)TC_WTILE * 2 + (size_t)NTp * TC_BK * 2; }
+// Shared memory the split epilogue needs in the stages: every split's
+// accumulator, then (SwiGLU) this CTA's share of the summed token rows.
+__host__ __device__ inline size_t tc_red_bytes(int NTp, int splits) {
+    return (size_t)NTp * TC_BM * 4 + (size_t)(NTp / splits) * TC_BM * 4;
+}
 __host__ __device__ inline size_t tc_smem_bytes(int NTp, int stages) {
     return (size_t)stages * tc_stage_bytes(NTp) + (2 * TC_MAX_STAGES + 1) * 8 + 16;
 }
@@ -144,9 +204,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     uint64_t* done = empty + TC_MAX_STAGES;
     volatile uint32_t* tslot = reinterpret_cast<volatile uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1) + 1;
-    const int nb = blockIdx.x % p.n_blocks, sp = blockIdx.x / p.n_blocks;
+    // the splits of a row block are consecutive CTAs, one cluster: sp is the rank
+    const int nb = blockIdx.x / p.splits, sp = blockIdx.x % p.splits;
     const int nkb_all = p.K / TC_BK;
-    const int kb0 = sp * p.kb_per_split, nkb = min(nkb_all, kb0 + p.kb_per_split) - kb0;
+    const int kb0 = sp * p.kb_per_split, nkb = max(0, min(nkb_all, kb0 + p.kb_per_split) - kb0);
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -231,37 +292,89 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     const bool got = mbar_wait_bounded(done, 0u, nullptr);
     tc_fence_after();
     if (!got && lane == 0 && p.status) set_status(p.status, HGD_ERR_TIMEOUT);
-    const bool live = __all_sync(0xffffffffu, got) && !*abort_flag && nkb > 0;
-    if (live) {
-        const int n = nb * TC_BM + warp * 32 + lane;
-        float* out = p.out + (size_t)sp * p.M * p.ldo;
+    const bool good = __syncthreads_and(got && !*abort_flag);  // no wait of this CTA ran out
+    const bool live = good && nkb > 0;
+    const int n = nb * TC_BM + warp * 32 + lane;
+    if (p.splits == 1 && p.h) {
+        // SwiGLU: the accumulator through shared memory (the stages are free), so
+        // a thread sees both rows of a gate / up pair
+        float* st = reinterpret_cast<float*>(smem);
+        if (live)
+            for (int c0 = 0; c0 < p.NTp; c0 += 16) {
+                uint32_t v[16];
+                tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) st[(c0 + j) * TC_BM + warp * 32 + lane] = __uint_as_float(v[j]);
+            }
+        __syncthreads();
+        if (live) tc_swiglu_rows(p, st, 0, p.NTp, nb, tid);
+    } else if (p.splits == 1) {
+        if (live)
+            for (int c0 = 0; c0 < p.NTp; c0 += 16) {
+                uint32_t v[16];
+                tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (c0 + j < p.M && n < p.N) tc_store(p, c0 + j, n, __uint_as_float(v[j]));
+            }
+    } else {
+        // every MMA has completed and every stage has been read: the stages take
+        // this split's accumulator, red[t][row] (a split with no K blocks, or one
+        // whose waits ran out, parks zeros; the status word says which)
+        float* red = reinterpret_cast<float*>(smem);
+        volatile int* good_w = reinterpret_cast<volatile int*>(done + 1) + 2;
+        if (tid == 0) *good_w = good ? 1 : 0;
         for (int c0 = 0; c0 < p.NTp; c0 += 16) {
             uint32_t v[16];
-            tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            if (live) tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int t = c0 + j;
-                if (t < p.M && n < p.N) out[(size_t)t * p.ldo + n] = __uint_as_float(v[j]);
+            for (int j = 0; j < 16; ++j) red[(c0 + j) * TC_BM + warp * 32 + lane] = live ? __uint_as_float(v[j]) : 0.f;
+        }
+        cluster_sync_all();
+        // this CTA's share of the token rows, summed over the splits in split
+        // order; nothing is written unless every split's waits completed
+        bool all_good = true;
+        for (int r = 0; r < p.splits; ++r) all_good = all_good && ld_dsmem_s32(dsmem_addr((const void*)good_w, (uint32_t)r)) != 0;
+        const int per = all_good ? p.NTp / p.splits : 0;
+        const int nn = nb * TC_BM + tid;
+        float* own = red + (size_t)p.NTp * TC_BM;  // SwiGLU: this CTA's summed rows, nobody else reads them
+        uint32_t rb[TC_MAX_SPLITS];  // red in each rank's shared memory
+#pragma unroll
+        for (int r = 0; r < TC_MAX_SPLITS; ++r) rb[r] = r < p.splits ? dsmem_addr(red, (uint32_t)r) : 0u;
+        constexpr int TG = 4;  // token rows whose loads are in flight together
+        const int t_end = min((sp + 1) * per, p.M);
+        for (int t0 = sp * per; t0 < t_end; t0 += TG) {
+            float v[TG][TC_MAX_SPLITS];
+#pragma unroll
+            for (int u = 0; u < TG; ++u)
+#pragma unroll
+                for (int r = 0; r < TC_MAX_SPLITS; ++r)
+                    v[u][r] = (r < p.splits && t0 + u < t_end)
+                                  ? ld_dsmem_f32(rb[r] + (uint32_t)(((t0 + u) * TC_BM + tid) * 4))
+                                  : 0.f;
+#pragma unroll
+            for (int u = 0; u < TG; ++u) {
+                float acc = v[u][0];
+#pragma unroll
+                for (int r = 1; r < TC_MAX_SPLITS; ++r)
+                    if (r < p.splits) acc += v[u][r];
+                if (t0 + u < t_end) {
+                    if (p.h) own[(t0 + u - sp * per) * TC_BM + tid] = acc;
+                    else if (nn < p.N) tc_store(p, t0 + u, nn, acc);
+                }
             }
         }
+        if (p.h) {
+            __syncthreads();
+            tc_swiglu_rows(p, own, sp * per, t_end, nb, tid);
+        }
+        cluster_sync_all();  // no CTA leaves while another still reads its shared memory
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols) : "memory");
-    }
-}
-
-// Y[t][n] = sum over splits, in split order, of the partials.
-__global__ void k_tc_reduce(const float* __restrict__ part, float* __restrict__ y, int splits, int64_t n_elem) {
-    pdl_launch();
-    pdl_wait();
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n_elem;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        float acc = part[e];
-        for (int s = 1; s < splits; ++s) acc += part[(int64_t)s * n_elem + e];
-        y[e] = acc;
     }
 }
 

@@ -505,6 +505,7 @@ struct NormRowsParams {
     bf16_t* out; int64_t out_ld;
     int M, K;
     int32_t* status;
+    int pack_ntp;  // > 0: out holds the rows packed for the tensor-core GEMM (tc_x_elem, NTp rows)
 };
 template <bool EMBED>
 __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormRowsParams p) {
@@ -513,14 +514,16 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
     const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (m >= p.M) return;
     const int K = p.K;
-    bf16_t* dst = p.out + m * p.out_ld;
+    auto dst = [&](int c) -> bf16_t* {
+        return p.pack_ntp ? p.out + tc_x_elem(m, c * 8, p.pack_ntp) : p.out + m * p.out_ld + c * 8;
+    };
     int tok = 0;
     if (EMBED) {
         tok = p.tokens[m];
         if (tok < 0 || tok >= p.vocab) {
             if (lane == 0) set_status(p.status, HGD_ERR_INVALID_ARG);
             for (int c = lane; c < K / 8; c += 32) {
-                *reinterpret_cast<uint4*>(dst + c * 8) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(dst(c)) = make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4*>(p.resid_out + m * p.resid_out_ld + c * 8) = make_uint4(0, 0, 0, 0);
             }
             return;
@@ -552,7 +555,7 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             o4[q] = pack_bf2(bf_lo(w4[q]) * r * bf_lo(g4[q]), bf_hi(w4[q]) * r * bf_hi(g4[q]));
-        *reinterpret_cast<uint4*>(dst + c * 8) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        *reinterpret_cast<uint4*>(dst(c)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         if (EMBED) *reinterpret_cast<uint4*>(p.resid_out + m * p.resid_out_ld + c * 8) = v;
     }
 }
@@ -567,6 +570,7 @@ struct GatedNormParams {
     bf16_t* u; int64_t u_ld;
     int M, nh, d;
     float eps;
+    int pack_ntp;  // > 0: u holds the rows packed for the tensor-core GEMM (tc_x_elem, NTp rows)
 };
 __global__ void __launch_bounds__(256) k_gated_norm(const __grid_constant__ GatedNormParams p) {
     pdl_launch();
@@ -576,14 +580,15 @@ __global__ void __launch_bounds__(256) k_gated_norm(const __grid_constant__ Gate
     const int m = e / p.nh, h = e % p.nh, d = p.d;
     const float* orow = p.o + m * p.o_ld + h * d;
     const float* zrow = p.z + m * p.z_ld + h * d;
-    bf16_t* dst = p.u + m * p.u_ld + h * d;
     float ss = 0.f;
     for (int i = lane; i < d; i += 32) ss = fmaf(orow[i], orow[i], ss);
     ss = warp_sum(ss);
     const float r = rsqrtf(ss / (float)d + p.eps);
     for (int i = lane; i < d; i += 32) {
         const float zb = bf2f(f2bf(zrow[i]));
-        dst[i] = f2bf(orow[i] * r * bf2f(p.w[i]) * silu_f(zb));
+        const bf16_t v = f2bf(orow[i] * r * bf2f(p.w[i]) * silu_f(zb));
+        if (p.pack_ntp) p.u[tc_x_elem(m, h * d + i, p.pack_ntp)] = v;
+        else p.u[m * p.u_ld + h * d + i] = v;
     }
 }
 

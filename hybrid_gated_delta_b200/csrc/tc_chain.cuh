@@ -115,56 +115,36 @@ __global__ void k_tc_rope(const __grid_constant__ TcRopeParams p) {
     }
 }
 
-// resid[m][n] = bf16(resid[m][n] + y[m][n]) (the residual add of a projection).
-__global__ void k_tc_resid(bf16_t* resid, const float* y, int64_t n_elem) {
-    pdl_launch();
-    pdl_wait();
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_elem; i += (int64_t)gridDim.x * blockDim.x)
-        resid[i] = f2bf(bf2f(resid[i]) + y[i]);
-}
-
-// resid[i] = bf16(resid[i] + sum_s part[s][i]): the split-K partials of a
-// projection added in split order (as k_tc_reduce adds them) and the residual
-// add, in one pass.
-__global__ void k_tc_reduce_resid(const float* __restrict__ part, bf16_t* resid, int splits, int64_t n_elem) {
-    pdl_launch();
-    pdl_wait();
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_elem; e += (int64_t)gridDim.x * blockDim.x) {
-        float acc = part[e];
-        for (int s = 1; s < splits; ++s) acc += part[(int64_t)s * n_elem + e];
-        resid[e] = f2bf(bf2f(resid[e]) + acc);
-    }
-}
-
-// h[m][i] = bf16(silu(g) * u): g = y[m][i], u = y[m][up0 + i] (gate rows, then the
-// up rows from row up0 of the combined projection).
-__global__ void k_tc_swiglu(const float* y, int64_t y_ld, int up0, bf16_t* h, int M, int I) {
-    pdl_launch();
-    pdl_wait();
-    const int64_t n = (int64_t)M * I;
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = e / I, i = e % I;
-        const float* yr = y + m * y_ld;
-        h[e] = f2bf(silu_f(yr[i]) * yr[up0 + i]);
-    }
-}
-
 // argmax[m] over the fp32 logits row m (first maximum: lowest index on ties; a
-// NaN gives -1 and HGD_ERR_NAN); then, if pos is set, every stream's position
-// advances by T (block 0, after its row).  One CTA of 256 threads per row.
-__global__ void k_tc_argmax(const float* logits, int64_t ld, int V, int32_t* argmax, int32_t* status, int32_t* pos,
-                            int B, int T) {
+// NaN gives -1 and HGD_ERR_NAN), in two passes.  k_tc_argmax_part: grid (M,
+// TC_AM_SLICES), block 256; CTA (m, s) scans slice s of the row (contiguous
+// index ranges, four loads in flight per thread) into the partial pv/pi[m][s]
+// (pi = -2: the slice holds a NaN).  k_tc_argmax_final: grid M, one warp; the
+// slices merge in index order; then, if pos is set, every stream's position
+// advances by T (block 0).
+constexpr int TC_AM_SLICES = 32;
+__global__ void __launch_bounds__(256) k_tc_argmax_part(const float* logits, int64_t ld, int V, float* pv, int* pi) {
     pdl_launch();
     pdl_wait();
-    const int m = blockIdx.x;
+    const int m = blockIdx.x, sl = blockIdx.y;
+    const int span = (V + TC_AM_SLICES - 1) / TC_AM_SLICES;
+    const int lo = sl * span, hi = min(V, lo + span);
     const float* lr = logits + (int64_t)m * ld;
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     bool nan = false;
-    for (int i = threadIdx.x; i < V; i += blockDim.x) {
-        const float v = lr[i];
-        if (v != v) nan = true;
-        else if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+    constexpr int U = 4;
+    for (int i0 = lo + (int)threadIdx.x; i0 < hi; i0 += U * 256) {
+        float v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) v[u] = i0 + u * 256 < hi ? lr[i0 + u * 256] : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * 256;
+            if (i >= hi) break;
+            if (v[u] != v[u]) nan = true;
+            else if (v[u] > bv || (v[u] == bv && i < bi)) { bv = v[u]; bi = i; }
+        }
     }
     __shared__ float sv[8];
     __shared__ int si[8], sn[8];
@@ -184,8 +164,34 @@ __global__ void k_tc_argmax(const float* logits, int64_t ld, int V, int32_t* arg
             anynan = anynan || sn[k];
             if (sv[k] > bv || (sv[k] == bv && si[k] < bi)) { bv = sv[k]; bi = si[k]; }
         }
-        argmax[m] = anynan ? -1 : bi;
-        if (anynan) set_status(status, HGD_ERR_NAN);
+        pv[m * TC_AM_SLICES + sl] = bv;
+        pi[m * TC_AM_SLICES + sl] = anynan ? -2 : bi;
+    }
+}
+__global__ void k_tc_argmax_final(const float* pv, const int* pi, int32_t* argmax, int32_t* status, int32_t* pos,
+                                  int B, int T) {
+    pdl_launch();
+    pdl_wait();
+    const int m = blockIdx.x, lane = threadIdx.x;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    bool nan = false;
+    if (lane < TC_AM_SLICES) {
+        bv = pv[m * TC_AM_SLICES + lane];
+        bi = pi[m * TC_AM_SLICES + lane];
+        nan = bi == -2;
+        if (nan) { bv = -INFINITY; bi = 0x7fffffff; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    nan = __any_sync(0xffffffffu, nan);
+    if (lane == 0) {
+        argmax[m] = nan ? -1 : bi;
+        if (nan) set_status(status, HGD_ERR_NAN);
         if (pos && m == 0)
             for (int s = 0; s < B; ++s) pos[s] += T;
     }

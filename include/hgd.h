@@ -117,9 +117,10 @@ HGD_API int hgd_check_bounded_wait(int32_t* status, hgd_stream_t stream);
  *   y[m][n] = sum_k x[m][k] * W[n][k],  fp32 out [M, N] (row-major).
  * The weight is packed once (hgd_gemm_tc_pack_weight) into 128 x 64 tiles in the
  * tensor core's core-matrix order; the call packs x into its workspace, streams
- * each tile once, and splits K over CTAs by a fixed function of N and K (the
- * partials are added in split order), so results do not depend on the device
- * or the call's neighbours.  The sums follow the tensor core's order, not the
+ * each tile once, and splits K over at most 8 CTAs by a fixed function of N
+ * and K (the splits of a 128-row block run as one thread-block cluster and add
+ * their partials in split order through shared memory), so results do not
+ * depend on the device or the call's neighbours.  The sums follow the tensor core's order, not the
  * GEMV's: results agree with hgd_gemv_bf16 to fp32 rounding, not bit for bit.
  * Shapes: 1 <= M <= 256, 1 <= N, 64 <= K <= 65536 with K % 64 == 0
  * (HGD_ERR_UNSUPPORTED_SHAPE otherwise). */
@@ -130,8 +131,13 @@ HGD_API int hgd_gemm_tc_weight_bytes(int N, int K, size_t* bytes);
  * starts streaming it before it waits for the kernel that precedes it on the
  * stream, so that kernel must not be the one writing Wp. */
 HGD_API int hgd_gemm_tc_pack_weight(const uint16_t* W, uint16_t* Wp, int N, int K, hgd_stream_t stream);
-/* Bytes of the workspace of a GEMM of this shape (packed x and split partials). */
+/* Bytes of the workspace of a GEMM of this shape (the packed token rows). */
 HGD_API int hgd_gemm_tc_workspace_bytes(int M, int N, int K, size_t* bytes);
+/* The plan of a GEMM of this shape, for inspection: *splits, the CTAs (one
+ * cluster) that share each 128-row block's K range (a power of two, 1..8, a
+ * function of N and K only), and *stages, its shared-memory pipeline depth.
+ * Same shape rules as hgd_gemm_tc_bf16; no device work. */
+HGD_API int hgd_gemm_tc_plan(int M, int N, int K, int* splits, int* stages);
 /* Wp: packed weight; x [M, K] bf16; y [M, N] fp32; workspace of at least
  * hgd_gemm_tc_workspace_bytes bytes (HGD_ERR_BUFFER_TOO_SMALL otherwise; no
  * initial contents needed; calls sharing one must not overlap on the device);

@@ -140,26 +140,37 @@ def test_model_init_rejects_unsupported(hgd):
 
 
 def test_tensor_core_split_depends_on_n_and_k_only(hgd):
-    """The tensor-core GEMM splits K over CTAs by a fixed function of N and K (a
-    split never depends on M or on the device): its workspace is the packed x
-    plus splits x M x N fp32 partials, with the same split count at every M, and
-    no partials once the row tiles alone fill the device (N = 248320)."""
+    """The tensor-core GEMM splits K over the CTAs of one cluster by a fixed
+    function of N and K (a split never depends on M or on the device): a power
+    of two up to 8, the same at every M, one split once the row tiles alone fill
+    the device (N = 248320); its workspace is the packed token rows only, and
+    with splits its pipeline holds the NTp x 128 fp32 accumulator."""
     L = hgd._lib
     n = C.c_size_t()
+    sp, st = C.c_int(), C.c_int()
 
     def ws(M, N, K):
         assert L.hgd_gemm_tc_workspace_bytes(M, N, K, C.byref(n)) == 0
         return n.value
 
-    def xp(M, K):
-        ntp = 16 if M <= 16 else (M + 15) // 16 * 16
-        return (ntp * K * 2 + 255) // 256 * 256
+    def plan(M, N, K):
+        assert L.hgd_gemm_tc_plan(M, N, K, C.byref(sp), C.byref(st)) == 0
+        return sp.value, st.value
 
-    for N, K in ((1024, 3584), (1024, 2048), (8224, 1024), (300, 640)):
-        splits = {(ws(M, N, K) - xp(M, K)) // (M * N * 4) for M in (1, 16, 33, 128, 256)}
+    def ntp(M):
+        return 16 if M <= 16 else (M + 15) // 16 * 16
+
+    for N, K in ((1024, 3584), (1024, 2048), (8224, 1024), (7168, 1024), (300, 640), (128, 64)):
+        splits = {plan(M, N, K)[0] for M in (1, 16, 33, 128, 256)}
         assert len(splits) == 1, (N, K, splits)
         s = splits.pop()
-        assert 1 <= s <= K // 64
+        assert s in (1, 2, 4, 8) and s <= max(1, K // 64)
         for M in (1, 16, 33, 128, 256):
-            assert ws(M, N, K) == xp(M, K) + (s * M * N * 4 if s > 1 else 0)
-    assert ws(128, 248320, 1024) == xp(128, 1024)
+            assert ws(M, N, K) == (ntp(M) * K * 2 + 255) // 256 * 256
+            if s > 1:
+                stages = plan(M, N, K)[1]
+                assert stages * (128 * 64 * 2 + ntp(M) * 64 * 2) >= ntp(M) * 128 * 4
+    assert plan(128, 1024, 2048)[0] == 8 and plan(128, 1024, 3584)[0] == 8 and plan(128, 8224, 1024)[0] == 2
+    assert plan(128, 248320, 1024)[0] == 1
+    assert L.hgd_gemm_tc_plan(0, 1024, 1024, C.byref(sp), C.byref(st)) != 0
+    assert L.hgd_gemm_tc_plan(16, 1024, 100, C.byref(sp), C.byref(st)) != 0
