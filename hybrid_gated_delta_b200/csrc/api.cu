@@ -625,7 +625,7 @@ int sk_launch(const Dims& d, const SkParams& prm, size_t smem, int sms, cudaStre
 // weight tiles, a split of the K blocks that brings the CTA count near one wave
 // (it depends on N and K only), as many shared-memory stages as fit.
 struct TcPlan {
-    int NTp, n_blocks, kb_per_split, splits, stages;
+    int NTp, n_blocks, kb_per_split, splits, stages, wpb;
     uint32_t tmem_cols;
     size_t xp_bytes;
 };
@@ -641,13 +641,19 @@ TcPlan tc_plan(int M, int N, int K, bool swiglu = false) {
     q.splits = 1;
     while (q.splits * 2 <= want) q.splits *= 2;
     q.kb_per_split = (nkb + q.splits - 1) / q.splits;
+    // many row blocks (the LM head): two weight blocks per CTA share each token
+    // tile, so more of the bytes in flight are weights and the token rows are
+    // re-read half as often (two CTAs of 2 x NTp TMEM columns fit an SM's 512)
+    q.wpb = (q.splits == 1 && !swiglu && q.n_blocks >= 2 * TC_TARGET_CTAS && q.NTp <= 128) ? 2 : 1;
+    const int ctas = (q.n_blocks + q.wpb - 1) / q.wpb * q.splits;
     // more than one wave of CTAs: stages for two CTAs per SM, so one's epilogue
     // overlaps the other's stream; otherwise every stage that fits
-    const int per_sm = q.n_blocks * q.splits > TC_TARGET_CTAS ? 2 : 1;
-    const size_t avail = (size_t)GV_SMEM_LIMIT / per_sm - tc_smem_bytes(q.NTp, 0);
-    q.stages = (int)std::min<size_t>(TC_MAX_STAGES, avail / tc_stage_bytes(q.NTp));
-    if (q.stages < 2) q.stages = (int)std::min<size_t>(TC_MAX_STAGES, ((size_t)GV_SMEM_LIMIT - tc_smem_bytes(q.NTp, 0)) /
-                                                                      tc_stage_bytes(q.NTp));
+    const int per_sm = ctas > TC_TARGET_CTAS ? 2 : 1;
+    const size_t avail = (size_t)GV_SMEM_LIMIT / per_sm - tc_smem_bytes(q.NTp, 0, q.wpb);
+    q.stages = (int)std::min<size_t>(TC_MAX_STAGES, avail / tc_stage_bytes(q.NTp, q.wpb));
+    if (q.stages < 2)
+        q.stages = (int)std::min<size_t>(TC_MAX_STAGES, ((size_t)GV_SMEM_LIMIT - tc_smem_bytes(q.NTp, 0, q.wpb)) /
+                                                            tc_stage_bytes(q.NTp, q.wpb));
     // with splits (or the SwiGLU pairing) the stages also hold the accumulator
     if (q.splits > 1 || swiglu) {
         const size_t bytes = q.splits > 1 ? tc_red_bytes(q.NTp, q.splits) : (size_t)q.NTp * TC_BM * 4;
@@ -655,7 +661,7 @@ TcPlan tc_plan(int M, int N, int K, bool swiglu = false) {
         q.stages = std::max(q.stages, need);
     }
     uint32_t c = 32;
-    while ((int)c < q.NTp) c <<= 1;
+    while ((int)c < (q.wpb - 1) * 128 + q.NTp) c <<= 1;  // weight block j at column j * 128
     q.tmem_cols = c;
     q.xp_bytes = ((size_t)q.NTp * K * 2 + 255) / 256 * 256;
     return q;
@@ -715,9 +721,10 @@ int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int
     prm.Wp = Wp; prm.Xp = Xp; prm.out = y; prm.resid = resid; prm.h = h; prm.I = I; prm.status = status;
     prm.M = M; prm.N = N; prm.K = K; prm.NTp = q.NTp; prm.ldo = N;
     prm.n_blocks = q.n_blocks; prm.kb_per_split = q.kb_per_split; prm.splits = q.splits; prm.stages = q.stages;
+    prm.wpb = q.wpb;
     prm.tmem_cols = q.tmem_cols;
-    const dim3 grid(q.n_blocks * q.splits), block(TC_THREADS);
-    const size_t smem = tc_smem_bytes(q.NTp, q.stages);
+    const dim3 grid((q.n_blocks + q.wpb - 1) / q.wpb * q.splits), block(TC_THREADS);
+    const size_t smem = tc_smem_bytes(q.NTp, q.stages, q.wpb);
     e = q.splits > 1 ? launch_pdl_cluster(k_gemm_tc, grid, block, smem, s, q.splits, prm)
                      : launch_pdl(k_gemm_tc, grid, block, smem, s, prm);
     return launch_status(e);
@@ -1739,7 +1746,9 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
             TcConvParams cp{proj, Nin, conv + ig * c_layer, w[HGD_W_CONV],
                             tail_rec ? tail_rec + ig * trec_layer : nullptr, B, T, (int)d.C};
             const int64_t n = (int64_t)B * d.C;
-            if ((rc = launch_status(launch_pdl(k_tc_conv, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, cp))))
+            const dim3 cg((unsigned)((n + 255) / 256)), cb(256);
+            if ((rc = launch_status(tail_rec ? launch_pdl(k_tc_conv<true>, cg, cb, 0, s, cp)
+                                             : launch_pdl(k_tc_conv<false>, cg, cb, 0, s, cp))))
                 return rc;
             GdnLayerParams g{};
             g.proj = proj; g.proj_ld = Nin;

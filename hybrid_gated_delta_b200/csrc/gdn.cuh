@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
     // recurrence runs row after row, from shared memory, with no barrier.  Each
     // value comes from the function the one-row kernels use (l2_scale, the gate
     // expressions, gdn_rows_step), so the results are theirs bit for bit.
-    __shared__ float qs[GDN_TB][DK], ks[GDN_TB][DK], vs[GDN_TB][GDN_ROWS];
+    __shared__ __align__(16) float qs[GDN_TB][DK], ks[GDN_TB][DK], vs[GDN_TB][GDN_ROWS];
     __shared__ float qsc[GDN_TB], ksc[GDN_TB], al[GDN_TB], be[GDN_TB];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, dv = p.dv;
@@ -403,50 +403,45 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
 #pragma unroll
     for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
 
-    constexpr int QN = GDN_TB * DK / NT;  // q (and k) elements of a block per thread
-    static_assert(GDN_TB * DK % NT == 0 && GDN_TB * GDN_ROWS <= 2 * NT, "block staging");
+    __shared__ float abr[2][GDN_TB];  // raw a and b of the block's rows
+    // rows start on 16-byte boundaries (q and k heads are multiples of 32 floats)
+    const bool v16 = (p.proj_ld & 3) == 0 && (reinterpret_cast<uintptr_t>(p.proj) & 15) == 0;
     for (int t0 = 0; t0 < p.T; t0 += GDN_TB) {
         const int n = min(GDN_TB, p.T - t0);
         const float* pr0 = p.proj + ((int64_t)b * p.T + t0) * p.proj_ld;
-        {
-            float qr[QN], kr[QN], vr[2];
-#pragma unroll
-            for (int u = 0; u < QN; ++u) {
-                const int i = tid + u * NT, t = i / DK, e = i % DK;
+        // the block's inputs straight into shared memory (cp.async): q and k in
+        // 16-byte pieces, this CTA's value rows, a and b
+        if (v16) {
+            for (int i = tid; i < n * (DK / 4); i += NT) {
+                const int t = i / (DK / 4), e = (i % (DK / 4)) * 4;
                 const float* pr = pr0 + (int64_t)t * p.proj_ld;
-                qr[u] = t < n ? pr[(int64_t)hk * DK + e] : 0.f;
-                kr[u] = t < n ? pr[(int64_t)Hk * DK + (int64_t)hk * DK + e] : 0.f;
+                cp_async16(&qs[t][e], pr + (int64_t)hk * DK + e);
+                cp_async16(&ks[t][e], pr + (int64_t)Hk * DK + (int64_t)hk * DK + e);
             }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int i = tid + u * NT, t = i / GDN_ROWS, r = i % GDN_ROWS;
-                vr[u] = (i < GDN_TB * GDN_ROWS && t < n)
-                            ? pr0[(int64_t)t * p.proj_ld + 2 * (int64_t)Hk * DK + (int64_t)h * dv +
-                                  blockIdx.y * GDN_ROWS + r]
-                            : 0.f;
-            }
-            float ar = 0.f, br = 0.f;
-            if (tid < n) {
-                ar = pr0[(int64_t)tid * p.proj_ld + C + (int64_t)H * dv + h];
-                br = pr0[(int64_t)tid * p.proj_ld + C + (int64_t)H * dv + H + h];
-            }
-#pragma unroll
-            for (int u = 0; u < QN; ++u) {
-                const int i = tid + u * NT;
-                qs[i / DK][i % DK] = qr[u];
-                ks[i / DK][i % DK] = kr[u];
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int i = tid + u * NT;
-                if (i < GDN_TB * GDN_ROWS) vs[i / GDN_ROWS][i % GDN_ROWS] = vr[u];
-            }
-            if (tid < n) {
-                al[tid] = expf(-A * softplus_f(ar + dtb));
-                be[tid] = sigmoid_f(br);
+        } else {
+            for (int i = tid; i < n * DK; i += NT) {
+                const int t = i / DK, e = i % DK;
+                const float* pr = pr0 + (int64_t)t * p.proj_ld;
+                cp_async4(&qs[t][e], pr + (int64_t)hk * DK + e);
+                cp_async4(&ks[t][e], pr + (int64_t)Hk * DK + (int64_t)hk * DK + e);
             }
         }
+        for (int i = tid; i < n * GDN_ROWS; i += NT) {
+            const int t = i / GDN_ROWS, r = i % GDN_ROWS;
+            cp_async4(&vs[t][r], pr0 + (int64_t)t * p.proj_ld + 2 * (int64_t)Hk * DK + (int64_t)h * dv +
+                                     blockIdx.y * GDN_ROWS + r);
+        }
+        if (tid < n) {
+            cp_async4(&abr[0][tid], pr0 + (int64_t)tid * p.proj_ld + C + (int64_t)H * dv + h);
+            cp_async4(&abr[1][tid], pr0 + (int64_t)tid * p.proj_ld + C + (int64_t)H * dv + H + h);
+        }
+        cp_async_commit();
+        cp_async_wait_all();
         __syncthreads();
+        if (tid < n) {
+            al[tid] = expf(-A * softplus_f(abr[0][tid] + dtb));
+            be[tid] = sigmoid_f(abr[1][tid]);
+        }
         for (int t = warp; t < n; t += GDN_WARPS) {
             const float a = l2_scale<KPL>(qs[t], lane), c = l2_scale<KPL>(ks[t], lane);
             if (lane == 0) { qsc[t] = a; ksc[t] = c; }

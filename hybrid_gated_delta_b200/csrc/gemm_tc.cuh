@@ -39,7 +39,7 @@ namespace hgd {
 
 constexpr int TC_BM = 128;                    // W rows per tile (the MMA's M)
 constexpr int TC_MAXN = 256;                  // token rows per call (the MMA's N)
-constexpr int TC_THREADS = 128;
+constexpr int TC_THREADS = 256;  // warp 0 lane 0: copies, warp 1 lane 0: MMAs; all eight: the epilogue
 constexpr int TC_WTILE = TC_BM * TC_BK;       // elements of a weight tile (16 KB)
 constexpr int TC_MAX_STAGES = 8;
 constexpr int TC_TARGET_CTAS = 148;           // split-K target: one wave of B200 SMs
@@ -139,6 +139,7 @@ struct TcParams {
     int32_t* status;    // optional: HGD_ERR_TIMEOUT if a wait ran out
     int M, N, K, NTp, ldo;
     int n_blocks, kb_per_split, splits, stages;  // splits: the cluster size (1: no cluster)
+    int wpb;            // 128-row weight blocks per CTA (2: two accumulators share each token tile; splits 1)
     uint32_t tmem_cols;
 };
 
@@ -152,13 +153,16 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
     return r;
 }
-// (no memory clobber: these loads follow a cluster barrier, whose clobber orders
-// them, and a batch of them must issue back to back)
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t a) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a));
-    return v;
+// Bulk copy (the async proxy) of `bytes` from this CTA's shared memory to shared
+// memory of a CTA of the cluster, completing `bytes` of transaction count on that
+// CTA's mbarrier (dst and mbar: cluster addresses, dsmem_addr).  No multicast.
+__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "r"(smem_addr(src)), "r"(bytes), "r"(mbar)
+                 : "memory");
 }
+// Generic-proxy writes to shared memory made visible to the async proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ int ld_dsmem_s32(uint32_t a) {
     int v;
     asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
@@ -168,10 +172,56 @@ __device__ __forceinline__ int ld_dsmem_s32(uint32_t a) {
 // st[(t - t_lo) * 128 ..]: 64 gate rows, then the 64 matching up rows).
 __device__ __forceinline__ void tc_swiglu_rows(const TcParams& p, const float* st, int t_lo, int t_hi, int nb,
                                                int tid) {
+#pragma unroll 4
     for (int e = tid; e < (t_hi - t_lo) * 64; e += TC_THREADS) {
         const int tt = e >> 6, il = e & 63, i = nb * 64 + il, t = t_lo + tt;
         if (i < p.I && t < p.M)
             p.h[tc_x_elem(t, i, p.NTp)] = f2bf(silu_f(st[tt * TC_BM + il]) * st[tt * TC_BM + 64 + il]);
+    }
+}
+// The split sum of this CTA's token rows t_lo .. t_hi - 1 of one pass: red holds
+// split sp's own partials ([t][row]), rcv the others' (slot per sender), summed
+// in split order, four rows per thread (float4), eight token lanes.  The sums go
+// back into red (SwiGLU), onto the bf16 residual, or out as fp32.
+template <int SPLITS>
+__device__ __forceinline__ void tc_split_sum(const TcParams& p, float* red, const float* rcv, int per, int sp,
+                                             int t_lo, int t_hi, int tq, int nb, int tid, bool vec) {
+    const int q4 = tid & 31, tl = tid >> 5, nn = nb * TC_BM + 4 * q4;
+#pragma unroll 2
+    for (int t = t_lo + tl; t < t_hi; t += TC_THREADS / 32) {
+        float4 v[SPLITS];
+#pragma unroll
+        for (int r = 0; r < SPLITS; ++r) {
+            const float* src = r == sp ? red + (size_t)t * TC_BM
+                                       : rcv + ((size_t)(r < sp ? r : r - 1) * per + (t - t_lo)) * TC_BM;
+            v[r] = *reinterpret_cast<const float4*>(src + 4 * q4);
+        }
+        float4 a = v[0];
+#pragma unroll
+        for (int r = 1; r < SPLITS; ++r) { a.x += v[r].x; a.y += v[r].y; a.z += v[r].z; a.w += v[r].w; }
+        if (p.h) {
+            *reinterpret_cast<float4*>(red + (size_t)t * TC_BM + 4 * q4) = a;  // this CTA's own rows
+            continue;
+        }
+        const size_t e = (size_t)(tq + t) * p.ldo + nn;
+        const float av[4] = {a.x, a.y, a.z, a.w};
+        if (vec && nn + 3 < p.N) {
+            if (p.resid) {
+                const uint2 r2 = *reinterpret_cast<const uint2*>(p.resid + e);
+                *reinterpret_cast<uint2*>(p.resid + e) =
+                    make_uint2(pack_bf2(bf_lo(r2.x) + av[0], bf_hi(r2.x) + av[1]),
+                               pack_bf2(bf_lo(r2.y) + av[2], bf_hi(r2.y) + av[3]));
+            } else {
+                *reinterpret_cast<float4*>(p.out + e) = a;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (nn + j < p.N) {
+                    if (p.resid) p.resid[e + j] = f2bf(bf2f(p.resid[e + j]) + av[j]);
+                    else p.out[e + j] = av[j];
+                }
+        }
     }
 }
 __device__ __forceinline__ void tc_store(const TcParams& p, int t, int n, float v) {
@@ -184,34 +234,43 @@ __device__ __forceinline__ void tc_store(const TcParams& p, int t, int n, float 
 // full / empty / done mbarriers, the TMEM address and the abort flag.  With
 // splits, the stages then hold the accumulator (NTp x 128 fp32, tc_red_bytes):
 // the plan gives enough stages for it.
-__host__ __device__ inline size_t tc_stage_bytes(int NTp) { return (size_t)TC_WTILE * 2 + (size_t)NTp * TC_BK * 2; }
-// Shared memory the split epilogue needs in the stages: every split's
-// accumulator, then (SwiGLU) this CTA's share of the summed token rows.
-__host__ __device__ inline size_t tc_red_bytes(int NTp, int splits) {
-    return (size_t)NTp * TC_BM * 4 + (size_t)(NTp / splits) * TC_BM * 4;
+__host__ __device__ inline size_t tc_stage_bytes(int NTp, int wpb = 1) {
+    return (size_t)wpb * TC_WTILE * 2 + (size_t)NTp * TC_BK * 2;
 }
-__host__ __device__ inline size_t tc_smem_bytes(int NTp, int stages) {
-    return (size_t)stages * tc_stage_bytes(NTp) + (2 * TC_MAX_STAGES + 1) * 8 + 16;
+// The split epilogue works on up to TC_RED_T token rows at a time.  Shared
+// memory it needs in the stages: the pass's accumulator rows, then the other
+// splits' partials of this CTA's share of them.
+constexpr int TC_RED_T = 128;
+__host__ __device__ inline size_t tc_red_bytes(int NTp, int splits) {
+    const int rows = NTp < TC_RED_T ? NTp : TC_RED_T;
+    return (size_t)rows * TC_BM * 4 + (size_t)(splits - 1) * (rows / splits) * TC_BM * 4;
+}
+__host__ __device__ inline size_t tc_smem_bytes(int NTp, int stages, int wpb = 1) {
+    return (size_t)stages * tc_stage_bytes(NTp, wpb) + (2 * TC_MAX_STAGES + 1) * 8 + 32;
 }
 
 __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int S = p.stages;
-    const size_t sb = tc_stage_bytes(p.NTp);
+    const size_t sb = tc_stage_bytes(p.NTp, p.wpb);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * sb);
     uint64_t* empty = full + TC_MAX_STAGES;
     uint64_t* done = empty + TC_MAX_STAGES;
     volatile uint32_t* tslot = reinterpret_cast<volatile uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1) + 1;
-    // the splits of a row block are consecutive CTAs, one cluster: sp is the rank
-    const int nb = blockIdx.x / p.splits, sp = blockIdx.x % p.splits;
+    uint64_t* rbar = done + 3;  // the split epilogue: the other splits' partials have landed
+    // the splits of a row block are consecutive CTAs, one cluster: sp is the rank;
+    // with wpb = 2 a CTA owns blocks nb and nb + 1 (only nb if that is the last)
+    const int nb = (blockIdx.x / p.splits) * p.wpb, sp = blockIdx.x % p.splits;
+    const int wn = min(p.wpb, p.n_blocks - nb);  // weight blocks this CTA computes
     const int nkb_all = p.K / TC_BK;
     const int kb0 = sp * p.kb_per_split, nkb = max(0, min(nkb_all, kb0 + p.kb_per_split) - kb0);
 
     if (tid == 0) {
         for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
         mbar_init(done, 1);
+        mbar_init(rbar, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -233,16 +292,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
         // previous kernel on the stream (weights are never written by it), their
         // token tiles after it; then stage by stage as the MMAs free them
         const uint32_t xbytes = (uint32_t)p.NTp * TC_BK * 2, wbytes = (uint32_t)TC_WTILE * 2;
+        const uint32_t xoff = (uint32_t)p.wpb * wbytes;  // the token tile follows the weight tiles
         const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
         const int pre = min(S, nkb);
         for (int i = 0; i < pre; ++i) {
-            mbar_arrive_expect_tx(&full[i], wbytes + xbytes);
-            bulk_g2s(smem + (size_t)i * sb, p.Wp + ((size_t)nb * nkb_all + kb0 + i) * TC_WTILE, wbytes, &full[i],
-                     pol_w);
+            mbar_arrive_expect_tx(&full[i], (uint32_t)wn * wbytes + xbytes);
+            for (int j = 0; j < wn; ++j)
+                bulk_g2s(smem + (size_t)i * sb + j * wbytes, p.Wp + ((size_t)(nb + j) * nkb_all + kb0 + i) * TC_WTILE,
+                         wbytes, &full[i], pol_w);
         }
         pdl_wait();
         for (int i = 0; i < pre; ++i)
-            bulk_g2s(smem + (size_t)i * sb + wbytes, p.Xp + (size_t)(kb0 + i) * p.NTp * TC_BK, xbytes, &full[i],
+            bulk_g2s(smem + (size_t)i * sb + xoff, p.Xp + (size_t)(kb0 + i) * p.NTp * TC_BK, xbytes, &full[i],
                      pol_x);
         int issued = pre;
         bool ok = true;
@@ -252,10 +313,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
                 ok = false;
                 break;
             }
-            mbar_arrive_expect_tx(&full[st], wbytes + xbytes);
+            mbar_arrive_expect_tx(&full[st], (uint32_t)wn * wbytes + xbytes);
             uint8_t* dst = smem + (size_t)st * sb;
-            bulk_g2s(dst, p.Wp + ((size_t)nb * nkb_all + kb0 + i) * TC_WTILE, wbytes, &full[st], pol_w);
-            bulk_g2s(dst + wbytes, p.Xp + (size_t)(kb0 + i) * p.NTp * TC_BK, xbytes, &full[st], pol_x);
+            for (int j = 0; j < wn; ++j)
+                bulk_g2s(dst + j * wbytes, p.Wp + ((size_t)(nb + j) * nkb_all + kb0 + i) * TC_WTILE, wbytes, &full[st],
+                         pol_w);
+            bulk_g2s(dst + xoff, p.Xp + (size_t)(kb0 + i) * p.NTp * TC_BK, xbytes, &full[st], pol_x);
             issued = i + 1;
         }
         if (!ok) {
@@ -277,11 +340,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
             }
             tc_fence_after();
             const uint8_t* a = smem + (size_t)st * sb;
-            const uint8_t* b = a + (size_t)TC_WTILE * 2;
+            const uint8_t* b = a + (size_t)p.wpb * TC_WTILE * 2;
+            // weight block j accumulates in TMEM columns j * 128 .. (NTp <= 128 with wpb = 2)
+            for (int j = 0; j < wn; ++j)
 #pragma unroll
-            for (int s = 0; s < TC_BK / 16; ++s)
-                tc_mma(tmem, tc_desc(a + s * 256, 128, 1024), tc_desc(b + s * 256, 128, 1024), idesc,
-                       (i > 0 || s > 0) ? 1u : 0u);
+                for (int s = 0; s < TC_BK / 16; ++s)
+                    tc_mma(tmem + (uint32_t)(j * 128), tc_desc(a + (size_t)j * TC_WTILE * 2 + s * 256, 128, 1024),
+                           tc_desc(b + s * 256, 128, 1024), idesc, (i > 0 || s > 0) ? 1u : 0u);
             tc_commit(&empty[st]);
         }
         tc_commit(done);  // covers every MMA issued above
@@ -294,81 +359,102 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     if (!got && lane == 0 && p.status) set_status(p.status, HGD_ERR_TIMEOUT);
     const bool good = __syncthreads_and(got && !*abort_flag);  // no wait of this CTA ran out
     const bool live = good && nkb > 0;
-    const int n = nb * TC_BM + warp * 32 + lane;
+    // warp w reads TMEM lane quarter w & 3 (W rows 32 (w & 3) + lane of a block) and
+    // half w >> 2 of the accumulator's columns (token rows)
+    const int lq = warp & 3, ch = warp >> 2;
+    const int n = nb * TC_BM + lq * 32 + lane;
+    auto col_range = [&](int c_lo, int c_n, int& b, int& e) {  // this warp's columns of [c_lo, c_lo + c_n)
+        const int half = ((c_n / 2 + 15) / 16) * 16;
+        b = c_lo + (ch ? min(half, c_n) : 0);
+        e = c_lo + (ch ? c_n : min(half, c_n));
+    };
+    auto park = [&](float* dst, int c_lo, int c_n, uint32_t col0) {  // dst[(c - c_lo)][row] = accumulator
+        int cb, ce;
+        col_range(c_lo, c_n, cb, ce);
+        for (int c0 = cb; c0 < ce; c0 += 16) {
+            uint32_t v[16];
+            if (live) tc_ld16(tmem + ((uint32_t)(lq * 32) << 16) + col0 + (uint32_t)c0, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                dst[(c0 - c_lo + j) * TC_BM + lq * 32 + lane] = live ? __uint_as_float(v[j]) : 0.f;
+        }
+    };
     if (p.splits == 1 && p.h) {
         // SwiGLU: the accumulator through shared memory (the stages are free), so
         // a thread sees both rows of a gate / up pair
         float* st = reinterpret_cast<float*>(smem);
-        if (live)
-            for (int c0 = 0; c0 < p.NTp; c0 += 16) {
-                uint32_t v[16];
-                tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) st[(c0 + j) * TC_BM + warp * 32 + lane] = __uint_as_float(v[j]);
-            }
+        park(st, 0, p.NTp, 0u);
         __syncthreads();
         if (live) tc_swiglu_rows(p, st, 0, p.NTp, nb, tid);
     } else if (p.splits == 1) {
         if (live)
-            for (int c0 = 0; c0 < p.NTp; c0 += 16) {
-                uint32_t v[16];
-                tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            for (int wj = 0; wj < wn; ++wj) {
+                const int nw = n + wj * TC_BM;
+                int cb, ce;
+                col_range(0, p.NTp, cb, ce);
+                for (int c0 = cb; c0 < ce; c0 += 16) {
+                    uint32_t v[16];
+                    tc_ld16(tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(wj * 128 + c0), v);
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (c0 + j < p.M && n < p.N) tc_store(p, c0 + j, n, __uint_as_float(v[j]));
-            }
-    } else {
-        // every MMA has completed and every stage has been read: the stages take
-        // this split's accumulator, red[t][row] (a split with no K blocks, or one
-        // whose waits ran out, parks zeros; the status word says which)
-        float* red = reinterpret_cast<float*>(smem);
-        volatile int* good_w = reinterpret_cast<volatile int*>(done + 1) + 2;
-        if (tid == 0) *good_w = good ? 1 : 0;
-        for (int c0 = 0; c0 < p.NTp; c0 += 16) {
-            uint32_t v[16];
-            if (live) tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) red[(c0 + j) * TC_BM + warp * 32 + lane] = live ? __uint_as_float(v[j]) : 0.f;
-        }
-        cluster_sync_all();
-        // this CTA's share of the token rows, summed over the splits in split
-        // order; nothing is written unless every split's waits completed
-        bool all_good = true;
-        for (int r = 0; r < p.splits; ++r) all_good = all_good && ld_dsmem_s32(dsmem_addr((const void*)good_w, (uint32_t)r)) != 0;
-        const int per = all_good ? p.NTp / p.splits : 0;
-        const int nn = nb * TC_BM + tid;
-        float* own = red + (size_t)p.NTp * TC_BM;  // SwiGLU: this CTA's summed rows, nobody else reads them
-        uint32_t rb[TC_MAX_SPLITS];  // red in each rank's shared memory
-#pragma unroll
-        for (int r = 0; r < TC_MAX_SPLITS; ++r) rb[r] = r < p.splits ? dsmem_addr(red, (uint32_t)r) : 0u;
-        constexpr int TG = 4;  // token rows whose loads are in flight together
-        const int t_end = min((sp + 1) * per, p.M);
-        for (int t0 = sp * per; t0 < t_end; t0 += TG) {
-            float v[TG][TC_MAX_SPLITS];
-#pragma unroll
-            for (int u = 0; u < TG; ++u)
-#pragma unroll
-                for (int r = 0; r < TC_MAX_SPLITS; ++r)
-                    v[u][r] = (r < p.splits && t0 + u < t_end)
-                                  ? ld_dsmem_f32(rb[r] + (uint32_t)(((t0 + u) * TC_BM + tid) * 4))
-                                  : 0.f;
-#pragma unroll
-            for (int u = 0; u < TG; ++u) {
-                float acc = v[u][0];
-#pragma unroll
-                for (int r = 1; r < TC_MAX_SPLITS; ++r)
-                    if (r < p.splits) acc += v[u][r];
-                if (t0 + u < t_end) {
-                    if (p.h) own[(t0 + u - sp * per) * TC_BM + tid] = acc;
-                    else if (nn < p.N) tc_store(p, t0 + u, nn, acc);
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < p.M && nw < p.N) tc_store(p, c0 + j, nw, __uint_as_float(v[j]));
                 }
             }
+    } else {
+        // every MMA has completed and every stage has been read: the stages take the
+        // accumulator, TC_RED_T token rows per pass.  Each CTA parks the pass's rows
+        // (red[t][row]; zeros if this split has no K blocks or a wait ran out: the
+        // status word says which), then hands every other split the rows that split
+        // sums by one bulk copy into its receive buffer (rcv, one slot per sender),
+        // and sums its own rows from its shared memory in split order.
+        float* red = reinterpret_cast<float*>(smem);
+        const int rows = min(p.NTp, TC_RED_T), per = rows / p.splits;
+        float* rcv = red + (size_t)rows * TC_BM;
+        volatile int* good_w = reinterpret_cast<volatile int*>(done + 1) + 2;
+        if (tid == 0) *good_w = good ? 1 : 0;
+        const uint32_t bytes_in = (uint32_t)((p.splits - 1) * per * TC_BM * 4);
+        const bool vec = (p.ldo & 3) == 0 &&
+                         ((reinterpret_cast<uintptr_t>(p.resid ? (const void*)p.resid : (const void*)p.out) & 15) == 0);
+        bool all_good = true;
+        for (int q = 0; q * TC_RED_T < p.NTp; ++q) {
+            const int tq = q * TC_RED_T;
+            park(red, 0, rows, (uint32_t)tq);
+            fence_proxy_async_smem();
+            if (tid == 0) mbar_arrive_expect_tx(rbar, bytes_in);
+            cluster_sync_all();
+            if (q == 0)  // thread r reads rank r's word: one remote round trip
+                all_good = __syncthreads_and(tid >= p.splits ||
+                                             ld_dsmem_s32(dsmem_addr((const void*)good_w, (uint32_t)tid)) != 0);
+            if (!all_good) {  // every CTA of the cluster sees the same words and leaves here
+                cluster_sync_all();  // (after every CTA has read them)
+                break;
+            }
+            if (tid < p.splits && tid != sp) {
+                const int slot = sp < tid ? sp : sp - 1;  // this CTA's slot in the receiver's buffer
+                bulk_s2cluster(dsmem_addr(rcv + (size_t)slot * per * TC_BM, (uint32_t)tid),
+                               red + (size_t)tid * per * TC_BM, (uint32_t)(per * TC_BM * 4),
+                               dsmem_addr(rbar, (uint32_t)tid));
+            }
+            bool got = mbar_wait_bounded(rbar, (uint32_t)(q & 1), nullptr);
+            if (!got && p.status) set_status(p.status, HGD_ERR_TIMEOUT);
+            got = __syncthreads_and(got);
+            if (got) {
+                const int t_lo = sp * per, t_hi = min(t_lo + per, p.M - tq);
+                switch (p.splits) {
+                    case 2: tc_split_sum<2>(p, red, rcv, per, sp, t_lo, t_hi, tq, nb, tid, vec); break;
+                    case 4: tc_split_sum<4>(p, red, rcv, per, sp, t_lo, t_hi, tq, nb, tid, vec); break;
+                    default: tc_split_sum<8>(p, red, rcv, per, sp, t_lo, t_hi, tq, nb, tid, vec); break;
+                }
+                if (p.h) {
+                    __syncthreads();
+                    tc_swiglu_rows(p, red + (size_t)t_lo * TC_BM, tq + t_lo, tq + t_lo + per, nb, tid);
+                }
+            }
+            // every copy of the pass has landed (each CTA waited for its own) before
+            // red and rcv are written again, and before any CTA leaves; every CTA of
+            // the cluster runs every pass, so the cluster barriers always match
+            cluster_sync_all();
         }
-        if (p.h) {
-            __syncthreads();
-            tc_swiglu_rows(p, own, sp * per, t_end, nb, tid);
-        }
-        cluster_sync_all();  // no CTA leaves while another still reads its shared memory
     }
     tc_fence_before();
     __syncthreads();

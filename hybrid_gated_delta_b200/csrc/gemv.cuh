@@ -533,9 +533,8 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
         if (EMBED) return *reinterpret_cast<const uint4*>(p.embed + gv_packed_chunk(tok, c, K >> 5));
         return *reinterpret_cast<const uint4*>(p.x + m * p.x_ld + c * 8);
     };
-    float ss = 0.f;
-    for (int c = lane; c < K / 8; c += 32) {
-        const uint4 v = chunk(c);
+    // one row chunk c (8 elements) into the sum of squares, in the row's order
+    auto sumsq = [](const uint4& v, float ss) {
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -543,11 +542,9 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
             ss = fmaf(a, a, ss);
             ss = fmaf(b, b, ss);
         }
-    }
-    ss = warp_sum(ss);
-    const float r = rsqrtf(ss / (float)K + p.eps);
-    for (int c = lane; c < K / 8; c += 32) {
-        const uint4 v = chunk(c);
+        return ss;
+    };
+    auto emit = [&](int c, const uint4& v, float r) {
         const uint4 g = *reinterpret_cast<const uint4*>(p.norm_w + c * 8);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
         const uint32_t g4[4] = {g.x, g.y, g.z, g.w};
@@ -557,7 +554,30 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
             o4[q] = pack_bf2(bf_lo(w4[q]) * r * bf_lo(g4[q]), bf_hi(w4[q]) * r * bf_hi(g4[q]));
         *reinterpret_cast<uint4*>(dst(c)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         if (EMBED) *reinterpret_cast<uint4*>(p.resid_out + m * p.resid_out_ld + c * 8) = v;
+    };
+    // rows of up to NR * 256 elements are read once, into registers; longer rows twice
+    constexpr int NR = 8;
+    if (K / 8 <= NR * 32) {
+        uint4 xr[NR];
+#pragma unroll
+        for (int u = 0; u < NR; ++u)
+            if (lane + 32 * u < K / 8) xr[u] = chunk(lane + 32 * u);
+        float ss = 0.f;
+#pragma unroll
+        for (int u = 0; u < NR; ++u)
+            if (lane + 32 * u < K / 8) ss = sumsq(xr[u], ss);
+        ss = warp_sum(ss);
+        const float r = rsqrtf(ss / (float)K + p.eps);
+#pragma unroll
+        for (int u = 0; u < NR; ++u)
+            if (lane + 32 * u < K / 8) emit(lane + 32 * u, xr[u], r);
+        return;
     }
+    float ss = 0.f;
+    for (int c = lane; c < K / 8; c += 32) ss = sumsq(chunk(c), ss);
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)K + p.eps);
+    for (int c = lane; c < K / 8; c += 32) emit(c, chunk(c), r);
 }
 
 // The GDN out-projection's input for calls of many token rows, computed once per
@@ -580,16 +600,35 @@ __global__ void __launch_bounds__(256) k_gated_norm(const __grid_constant__ Gate
     const int m = e / p.nh, h = e % p.nh, d = p.d;
     const float* orow = p.o + m * p.o_ld + h * d;
     const float* zrow = p.z + m * p.z_ld + h * d;
+    auto put = [&](int i, float ov, float zv, float r) {
+        const float zb = bf2f(f2bf(zv));
+        const bf16_t v = f2bf(ov * r * bf2f(p.w[i]) * silu_f(zb));
+        if (p.pack_ntp) p.u[tc_x_elem(m, h * d + i, p.pack_ntp)] = v;
+        else p.u[m * p.u_ld + h * d + i] = v;
+    };
+    // heads of up to GR * 32 values are read once, into registers
+    constexpr int GR = 8;
+    if (d <= GR * 32) {
+        float ov[GR], zv[GR];
+#pragma unroll
+        for (int u = 0; u < GR; ++u)
+            if (lane + 32 * u < d) { ov[u] = orow[lane + 32 * u]; zv[u] = zrow[lane + 32 * u]; }
+        float ss = 0.f;
+#pragma unroll
+        for (int u = 0; u < GR; ++u)
+            if (lane + 32 * u < d) ss = fmaf(ov[u], ov[u], ss);
+        ss = warp_sum(ss);
+        const float r = rsqrtf(ss / (float)d + p.eps);
+#pragma unroll
+        for (int u = 0; u < GR; ++u)
+            if (lane + 32 * u < d) put(lane + 32 * u, ov[u], zv[u], r);
+        return;
+    }
     float ss = 0.f;
     for (int i = lane; i < d; i += 32) ss = fmaf(orow[i], orow[i], ss);
     ss = warp_sum(ss);
     const float r = rsqrtf(ss / (float)d + p.eps);
-    for (int i = lane; i < d; i += 32) {
-        const float zb = bf2f(f2bf(zrow[i]));
-        const bf16_t v = f2bf(orow[i] * r * bf2f(p.w[i]) * silu_f(zb));
-        if (p.pack_ntp) p.u[tc_x_elem(m, h * d + i, p.pack_ntp)] = v;
-        else p.u[m * p.u_ld + h * d + i] = v;
-    }
+    for (int i = lane; i < d; i += 32) put(i, orow[i], zrow[i], r);
 }
 
 // Per-CTA argmax partials: reduce each token over the row lanes of every warp,

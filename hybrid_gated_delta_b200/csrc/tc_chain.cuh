@@ -23,12 +23,18 @@ struct TcConvParams {
     float* x; int64_t x_ld; float* tail; const bf16_t* w; float* tail_rec;
     int B, T, C;
 };
-__global__ void k_tc_conv(const __grid_constant__ TcConvParams p) {
+// REC: tail records on (tail_rec set).  Each thread stages its channel's inputs
+// of up to 16 rows in shared memory at once (cp.async; every thread reads back
+// only its own column, so no barrier), then runs the rows in order.
+template <bool REC>
+__global__ void __launch_bounds__(256) k_tc_conv(const __grid_constant__ TcConvParams p) {
+    constexpr int RB = 16;
+    __shared__ float xs[RB][256];
     pdl_launch();
     pdl_wait();
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (int64_t)p.B * p.C) return;
-    const int b = (int)(idx / p.C), c = (int)(idx % p.C);
+    const int b = (int)(idx / p.C), c = (int)(idx % p.C), tid = threadIdx.x;
     constexpr int NT = GV_CONV_K - 1;
     float tl[NT], w[GV_CONV_K];
 #pragma unroll
@@ -36,29 +42,29 @@ __global__ void k_tc_conv(const __grid_constant__ TcConvParams p) {
     float* tb = p.tail + (int64_t)b * NT * p.C + c;
 #pragma unroll
     for (int j = 0; j < NT; ++j) tl[j] = tb[(int64_t)j * p.C];
-    constexpr int RB = 8;  // rows whose inputs are loaded together
+    const int64_t ld = p.x_ld;
+    float* xb = p.x + (int64_t)b * p.T * ld + c;  // row t of this stream at xb + t * ld
     for (int t0 = 0; t0 < p.T; t0 += RB) {
-        float xin[RB];
-#pragma unroll
-        for (int u = 0; u < RB; ++u)
-            if (t0 + u < p.T) xin[u] = p.x[((int64_t)b * p.T + t0 + u) * p.x_ld + c];
-#pragma unroll
-        for (int u = 0; u < RB; ++u) {
+        const int n = min(RB, p.T - t0);
+        for (int u = 0; u < n; ++u) cp_async4(&xs[u][tid], xb + (int64_t)(t0 + u) * ld);
+        cp_async_commit();
+        cp_async_wait_all();
+        for (int u = 0; u < n; ++u) {
             const int t = t0 + u;
-            if (t >= p.T) break;
-            const int64_t row = (int64_t)b * p.T + t;
-            const float xv = xin[u];
+            const float xv = xs[u][tid];
             float acc = 0.f;
 #pragma unroll
             for (int j = 0; j < NT; ++j) acc = fmaf(w[j], tl[j], acc);
             acc = fmaf(w[NT], xv, acc);
-            p.x[row * p.x_ld + c] = silu_f(acc);
+            xb[(int64_t)t * ld] = silu_f(acc);
 #pragma unroll
             for (int j = 0; j + 1 < NT; ++j) tl[j] = tl[j + 1];
             tl[NT - 1] = xv;
-            if (p.tail_rec)
+            if (REC) {
+                float* rp = p.tail_rec + ((int64_t)b * p.T + t) * NT * p.C + c;
 #pragma unroll
-                for (int j = 0; j < NT; ++j) p.tail_rec[(row * NT + j) * p.C + c] = tl[j];
+                for (int j = 0; j < NT; ++j) rp[(int64_t)j * p.C] = tl[j];
+            }
         }
     }
 #pragma unroll
