@@ -1315,6 +1315,28 @@ int hgd_check_not_coresident(const hgd_model* m, const hgd_state* st, int T) {
     return sk_launch(d, prm, sk_smem_bytes(d, M, sk_ring_slots(d, M)), di.sms, nullptr, false, 0);
 }
 
+// The GDN layer kernel over B streams: 8 state rows per warp where dv allows
+// (32 rows per CTA), else 4; either way each row's arithmetic is the same.
+cudaError_t launch_gdn_layer(const Dims& d, int B, const GdnLayerParams& g, cudaStream_t s) {
+    const dim3 block(GDN_WARPS * 32);
+    if (d.dv % (GDN_WARPS * 8) == 0) {
+        const dim3 grid(B * d.H, d.dv / (GDN_WARPS * 8));
+        switch (d.dk) {
+            case 32: return launch_pdl(k_gdn_layer<1, 8>, grid, block, 0, s, g);
+            case 64: return launch_pdl(k_gdn_layer<2, 8>, grid, block, 0, s, g);
+            case 128: return launch_pdl(k_gdn_layer<4, 8>, grid, block, 0, s, g);
+            default: return launch_pdl(k_gdn_layer<8, 8>, grid, block, 0, s, g);
+        }
+    }
+    const dim3 grid(B * d.H, d.dv / GDN_ROWS);
+    switch (d.dk) {
+        case 32: return launch_pdl(k_gdn_layer<1, GDN_RPW>, grid, block, 0, s, g);
+        case 64: return launch_pdl(k_gdn_layer<2, GDN_RPW>, grid, block, 0, s, g);
+        case 128: return launch_pdl(k_gdn_layer<4, GDN_RPW>, grid, block, 0, s, g);
+        default: return launch_pdl(k_gdn_layer<8, GDN_RPW>, grid, block, 0, s, g);
+    }
+}
+
 // The kernel chain of layers [layer_begin, layer_end) and, if run_head, the head.
 // With vl (a verify window): the conv runs on the log's copy of the tails and
 // logs each row's conv input, the GDN layers log (alpha, delta, k) instead of
@@ -1427,15 +1449,7 @@ static int chain_run(const hgd_model* m, const hgd_state* st, const int32_t* tok
                 g.log_delta = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.delta);
                 g.log_k = reinterpret_cast<float*>(vl + vlay.layer(ig) + vlay.k);
             }
-            const dim3 grid(B * d.H, d.dv / GDN_ROWS), block(GDN_WARPS * 32);
-            cudaError_t e;
-            switch (d.dk) {
-                case 32: e = launch_pdl(k_gdn_layer<1>, grid, block, 0, s, g); break;
-                case 64: e = launch_pdl(k_gdn_layer<2>, grid, block, 0, s, g); break;
-                case 128: e = launch_pdl(k_gdn_layer<4>, grid, block, 0, s, g); break;
-                default: e = launch_pdl(k_gdn_layer<8>, grid, block, 0, s, g); break;
-            }
-            if ((rc = launch_status(e))) return rc;
+            if ((rc = launch_status(launch_gdn_layer(d, B, g, s)))) return rc;
             GemvParams p = {};
             p.W = w[HGD_W_OUT]; p.packed = 1; p.N = d.D; p.K = d.H * d.dv;
             p.y = resid; p.y_ld = d.D; p.resid = resid; p.resid_ld = d.D; p.status = status_dev;
@@ -1757,18 +1771,10 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
             g.o = obuf; g.o_ld = (int64_t)d.H * d.dv;
             g.S_rec = S_rec ? S_rec + ig * srec_layer : nullptr;
             g.B = B; g.T = T; g.H = d.H; g.dv = d.dv; g.Hk = d.Hk;
-            const dim3 grid(B * d.H, d.dv / GDN_ROWS), block(GDN_WARPS * 32);
-            cudaError_t e;
-            switch (d.dk) {
-                case 32: e = launch_pdl(k_gdn_layer<1>, grid, block, 0, s, g); break;
-                case 64: e = launch_pdl(k_gdn_layer<2>, grid, block, 0, s, g); break;
-                case 128: e = launch_pdl(k_gdn_layer<4>, grid, block, 0, s, g); break;
-                default: e = launch_pdl(k_gdn_layer<8>, grid, block, 0, s, g); break;
-            }
-            if ((rc = launch_status(e))) return rc;
+            if ((rc = launch_status(launch_gdn_layer(d, B, g, s)))) return rc;
             GatedNormParams gq{obuf, (int64_t)d.H * d.dv, proj + d.C, Nin, w[HGD_W_GNORM], gn_rows,
                                (int64_t)d.H * d.dv, M, d.H, d.dv, eps, NTp};
-            e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, gq);
+            cudaError_t e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, gq);
             if ((rc = launch_status(e))) return rc;
             if ((rc = gemm_resid(m->tcw[l][1], gn_rows, (int64_t)d.H * d.dv, d.H * d.dv))) return rc;
             ++ig;

@@ -71,37 +71,37 @@ __device__ __forceinline__ void gdn_row_update(float (&S)[KPL], float delta, con
 // the row's writes delta (every lane).  The RPW dot products of a kind are
 // summed over the lanes together (warp_sum_transposed: warp_sum's pairings, so
 // each sum is bitwise warp_sum's) and then broadcast.
-template <int KPL>
-__device__ __forceinline__ void gdn_rows_step(float (&S)[GDN_RPW][KPL], const float (&kv)[KPL],
+template <int KPL, int RPW>
+__device__ __forceinline__ void gdn_rows_step(float (&S)[RPW][KPL], const float (&kv)[KPL],
                                               const float (&qv)[KPL], float alpha, float beta,
-                                              const float (&vrow)[GDN_RPW], float (&o)[GDN_RPW],
-                                              float (&dl)[GDN_RPW]) {
-    constexpr int LPR = 32 / GDN_RPW;  // lanes holding each sum after the transposed reduction
+                                              const float (&vrow)[RPW], float (&o)[RPW],
+                                              float (&dl)[RPW]) {
+    constexpr int LPR = 32 / RPW;  // lanes holding each sum after the transposed reduction
     const int lane = threadIdx.x & 31;
-    float w[GDN_RPW];
+    float w[RPW];
 #pragma unroll
-    for (int r = 0; r < GDN_RPW; ++r) {
+    for (int r = 0; r < RPW; ++r) {
         w[r] = 0.f;
 #pragma unroll
         for (int e = 0; e < KPL; ++e) w[r] = fmaf(S[r][e], kv[e], w[r]);
     }
-    const float ws = warp_sum_transposed<GDN_RPW>(w, lane);
+    const float ws = warp_sum_transposed<RPW>(w, lane);
 #pragma unroll
-    for (int r = 0; r < GDN_RPW; ++r) {
+    for (int r = 0; r < RPW; ++r) {
         const float delta = beta * (vrow[r] - alpha * __shfl_sync(0xffffffffu, ws, r * LPR));
         dl[r] = delta;
         gdn_row_update<KPL>(S[r], delta, kv, alpha);
     }
-    float ov[GDN_RPW];
+    float ov[RPW];
 #pragma unroll
-    for (int r = 0; r < GDN_RPW; ++r) {
+    for (int r = 0; r < RPW; ++r) {
         ov[r] = 0.f;
 #pragma unroll
         for (int e = 0; e < KPL; ++e) ov[r] = fmaf(S[r][e], qv[e], ov[r]);
     }
-    const float os = warp_sum_transposed<GDN_RPW>(ov, lane);
+    const float os = warp_sum_transposed<RPW>(ov, lane);
 #pragma unroll
-    for (int r = 0; r < GDN_RPW; ++r) o[r] = __shfl_sync(0xffffffffu, os, r * LPR);
+    for (int r = 0; r < RPW; ++r) o[r] = __shfl_sync(0xffffffffu, os, r * LPR);
 }
 
 // L2 normalisation scale 1/sqrt(sum x^2 + 1e-6) of a dk-vector held in shared
@@ -377,31 +377,32 @@ struct GdnLayerParams {
 // Rows whose inputs k_gdn_layer stages in shared memory at once.
 constexpr int GDN_TB = 16;
 
-template <int KPL>
+// RPW: state rows per warp (4 or 8; the per-row arithmetic does not depend on it).
+template <int KPL, int RPW>
 __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_constant__ GdnLayerParams p) {
     pdl_launch();
     pdl_wait();
-    constexpr int DK = 32 * KPL, NT = GDN_WARPS * 32;
+    constexpr int DK = 32 * KPL, NT = GDN_WARPS * 32, ROWS = GDN_WARPS * RPW;
     // A block of up to GDN_TB rows at a time: every input of the block (q and k
     // of the key head, this CTA's value rows, a and b) is loaded in one batch,
     // the rows' L2 scales and gates are formed in parallel, and then only the
     // recurrence runs row after row, from shared memory, with no barrier.  Each
     // value comes from the function the one-row kernels use (l2_scale, the gate
     // expressions, gdn_rows_step), so the results are theirs bit for bit.
-    __shared__ __align__(16) float qs[GDN_TB][DK], ks[GDN_TB][DK], vs[GDN_TB][GDN_ROWS];
+    __shared__ __align__(16) float qs[GDN_TB][DK], ks[GDN_TB][DK], vs[GDN_TB][ROWS];
     __shared__ float qsc[GDN_TB], ksc[GDN_TB], al[GDN_TB], be[GDN_TB];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H, dv = p.dv;
     const int b = blockIdx.x / H, h = blockIdx.x % H;
-    const int row0 = blockIdx.y * GDN_ROWS + warp * GDN_RPW;
+    const int row0 = blockIdx.y * ROWS + warp * RPW;
     const int Hk = p.Hk, hk = h / (H / Hk);
     const int64_t C = 2 * (int64_t)Hk * DK + (int64_t)H * dv;
     const float A = expf(bf2f(p.A_log[h])), dtb = bf2f(p.dt_bias[h]);
 
-    float S[GDN_RPW][KPL];
+    float S[RPW][KPL];
     float* Sbase = p.S + ((int64_t)(b * H + h) * dv + row0) * DK + lane * KPL;
 #pragma unroll
-    for (int r = 0; r < GDN_RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
+    for (int r = 0; r < RPW; ++r) ld_vec<KPL>(S[r], Sbase + (int64_t)r * DK);
 
     __shared__ float abr[2][GDN_TB];  // raw a and b of the block's rows
     // rows start on 16-byte boundaries (q and k heads are multiples of 32 floats)
@@ -426,10 +427,10 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
                 cp_async4(&ks[t][e], pr + (int64_t)Hk * DK + (int64_t)hk * DK + e);
             }
         }
-        for (int i = tid; i < n * GDN_ROWS; i += NT) {
-            const int t = i / GDN_ROWS, r = i % GDN_ROWS;
+        for (int i = tid; i < n * ROWS; i += NT) {
+            const int t = i / ROWS, r = i % ROWS;
             cp_async4(&vs[t][r], pr0 + (int64_t)t * p.proj_ld + 2 * (int64_t)Hk * DK + (int64_t)h * dv +
-                                     blockIdx.y * GDN_ROWS + r);
+                                     blockIdx.y * ROWS + r);
         }
         if (tid < n) {
             cp_async4(&abr[0][tid], pr0 + (int64_t)tid * p.proj_ld + C + (int64_t)H * dv + h);
@@ -450,17 +451,17 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
         for (int t = 0; t < n; ++t) {
             const int64_t row = (int64_t)b * p.T + t0 + t;
             const float qa = qsc[t], ka = ksc[t], alpha = al[t], beta = be[t];
-            float kv[KPL], qv[KPL], vrow[GDN_RPW];
+            float kv[KPL], qv[KPL], vrow[RPW];
 #pragma unroll
             for (int e = 0; e < KPL; ++e) { qv[e] = qs[t][lane * KPL + e] * qa; kv[e] = ks[t][lane * KPL + e] * ka; }
 #pragma unroll
-            for (int r = 0; r < GDN_RPW; ++r) vrow[r] = vs[t][warp * GDN_RPW + r];
-            float o[GDN_RPW], dl[GDN_RPW];
-            gdn_rows_step<KPL>(S, kv, qv, alpha, beta, vrow, o, dl);
-            if (lane < GDN_RPW) {
+            for (int r = 0; r < RPW; ++r) vrow[r] = vs[t][warp * RPW + r];
+            float o[RPW], dl[RPW];
+            gdn_rows_step<KPL, RPW>(S, kv, qv, alpha, beta, vrow, o, dl);
+            if (lane < RPW) {
                 float ov = o[0], dv_ = dl[0];
 #pragma unroll
-                for (int r = 1; r < GDN_RPW; ++r) if (lane == r) { ov = o[r]; dv_ = dl[r]; }
+                for (int r = 1; r < RPW; ++r) if (lane == r) { ov = o[r]; dv_ = dl[r]; }
                 p.o[row * p.o_ld + (int64_t)h * dv + row0 + lane] = ov;
                 if (p.log_delta) p.log_delta[(row * H + h) * dv + row0 + lane] = dv_;
             }
@@ -471,14 +472,14 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
             if (p.S_rec) {
                 float* rp = p.S_rec + ((row * H + h) * dv + row0) * DK + lane * KPL;
 #pragma unroll
-                for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
+                for (int r = 0; r < RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
             }
         }
         __syncthreads();  // the next block's inputs overwrite these
     }
     if (p.log_delta) return;  // a verify window: the state stays as it was
 #pragma unroll
-    for (int r = 0; r < GDN_RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
+    for (int r = 0; r < RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
 }
 
 }  // namespace hgd

@@ -544,8 +544,7 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
         }
         return ss;
     };
-    auto emit = [&](int c, const uint4& v, float r) {
-        const uint4 g = *reinterpret_cast<const uint4*>(p.norm_w + c * 8);
+    auto emit = [&](int c, const uint4& v, const uint4& g, float r) {
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
         const uint32_t g4[4] = {g.x, g.y, g.z, g.w};
         uint32_t o4[4];
@@ -557,11 +556,12 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
     };
     // rows of up to NR * 256 elements are read once, into registers; longer rows twice
     constexpr int NR = 8;
+    auto gain = [&](int c) { return *reinterpret_cast<const uint4*>(p.norm_w + c * 8); };
     if (K / 8 <= NR * 32) {
-        uint4 xr[NR];
+        uint4 xr[NR], gr[NR];  // the row and its gains, loaded together
 #pragma unroll
         for (int u = 0; u < NR; ++u)
-            if (lane + 32 * u < K / 8) xr[u] = chunk(lane + 32 * u);
+            if (lane + 32 * u < K / 8) { xr[u] = chunk(lane + 32 * u); gr[u] = gain(lane + 32 * u); }
         float ss = 0.f;
 #pragma unroll
         for (int u = 0; u < NR; ++u)
@@ -570,14 +570,14 @@ __global__ void __launch_bounds__(256) k_norm_rows(const __grid_constant__ NormR
         const float r = rsqrtf(ss / (float)K + p.eps);
 #pragma unroll
         for (int u = 0; u < NR; ++u)
-            if (lane + 32 * u < K / 8) emit(lane + 32 * u, xr[u], r);
+            if (lane + 32 * u < K / 8) emit(lane + 32 * u, xr[u], gr[u], r);
         return;
     }
     float ss = 0.f;
     for (int c = lane; c < K / 8; c += 32) ss = sumsq(chunk(c), ss);
     ss = warp_sum(ss);
     const float r = rsqrtf(ss / (float)K + p.eps);
-    for (int c = lane; c < K / 8; c += 32) emit(c, chunk(c), r);
+    for (int c = lane; c < K / 8; c += 32) emit(c, chunk(c), gain(c), r);
 }
 
 // The GDN out-projection's input for calls of many token rows, computed once per
@@ -600,19 +600,23 @@ __global__ void __launch_bounds__(256) k_gated_norm(const __grid_constant__ Gate
     const int m = e / p.nh, h = e % p.nh, d = p.d;
     const float* orow = p.o + m * p.o_ld + h * d;
     const float* zrow = p.z + m * p.z_ld + h * d;
-    auto put = [&](int i, float ov, float zv, float r) {
+    auto put = [&](int i, float ov, float zv, float wv, float r) {
         const float zb = bf2f(f2bf(zv));
-        const bf16_t v = f2bf(ov * r * bf2f(p.w[i]) * silu_f(zb));
+        const bf16_t v = f2bf(ov * r * wv * silu_f(zb));
         if (p.pack_ntp) p.u[tc_x_elem(m, h * d + i, p.pack_ntp)] = v;
         else p.u[m * p.u_ld + h * d + i] = v;
     };
     // heads of up to GR * 32 values are read once, into registers
     constexpr int GR = 8;
     if (d <= GR * 32) {
-        float ov[GR], zv[GR];
+        float ov[GR], zv[GR], wv[GR];  // o, z and the gains, loaded together
 #pragma unroll
         for (int u = 0; u < GR; ++u)
-            if (lane + 32 * u < d) { ov[u] = orow[lane + 32 * u]; zv[u] = zrow[lane + 32 * u]; }
+            if (lane + 32 * u < d) {
+                ov[u] = orow[lane + 32 * u];
+                zv[u] = zrow[lane + 32 * u];
+                wv[u] = bf2f(p.w[lane + 32 * u]);
+            }
         float ss = 0.f;
 #pragma unroll
         for (int u = 0; u < GR; ++u)
@@ -621,14 +625,14 @@ __global__ void __launch_bounds__(256) k_gated_norm(const __grid_constant__ Gate
         const float r = rsqrtf(ss / (float)d + p.eps);
 #pragma unroll
         for (int u = 0; u < GR; ++u)
-            if (lane + 32 * u < d) put(lane + 32 * u, ov[u], zv[u], r);
+            if (lane + 32 * u < d) put(lane + 32 * u, ov[u], zv[u], wv[u], r);
         return;
     }
     float ss = 0.f;
     for (int i = lane; i < d; i += 32) ss = fmaf(orow[i], orow[i], ss);
     ss = warp_sum(ss);
     const float r = rsqrtf(ss / (float)d + p.eps);
-    for (int i = lane; i < d; i += 32) put(i, orow[i], zrow[i], r);
+    for (int i = lane; i < d; i += 32) put(i, orow[i], zrow[i], bf2f(p.w[i]), r);
 }
 
 // Per-CTA argmax partials: reduce each token over the row lanes of every warp,
