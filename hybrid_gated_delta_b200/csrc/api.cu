@@ -1315,6 +1315,9 @@ int hgd_check_not_coresident(const hgd_model* m, const hgd_state* st, int T) {
     return sk_launch(d, prm, sk_smem_bytes(d, M, sk_ring_slots(d, M)), di.sms, nullptr, false, 0);
 }
 
+// dv of the GDN layer kernel's fused gated-norm form (16 warps x 8 rows: a head per CTA).
+constexpr int GDN_FUSED_DV = 128;
+
 // The GDN layer kernel over B streams: 8 state rows per warp where dv allows
 // (32 rows per CTA), else 4; either way each row's arithmetic is the same.
 cudaError_t launch_gdn_layer(const Dims& d, int B, const GdnLayerParams& g, cudaStream_t s) {
@@ -1771,11 +1774,24 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
             g.o = obuf; g.o_ld = (int64_t)d.H * d.dv;
             g.S_rec = S_rec ? S_rec + ig * srec_layer : nullptr;
             g.B = B; g.T = T; g.H = d.H; g.dv = d.dv; g.Hk = d.Hk;
-            if ((rc = launch_status(launch_gdn_layer(d, B, g, s)))) return rc;
-            GatedNormParams gq{obuf, (int64_t)d.H * d.dv, proj + d.C, Nin, w[HGD_W_GNORM], gn_rows,
-                               (int64_t)d.H * d.dv, M, d.H, d.dv, eps, NTp};
-            cudaError_t e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, gq);
-            if ((rc = launch_status(e))) return rc;
+            if (d.dv == GDN_FUSED_DV && d.dk <= 128) {
+                // one CTA per (stream, head) forms the gated norm too, packed for the GEMM
+                g.z = proj + d.C; g.z_ld = Nin; g.gn_w = w[HGD_W_GNORM]; g.u = gn_rows; g.u_ntp = NTp; g.eps = eps;
+                const dim3 grid(B * d.H), block(GDN_FUSED_DV / 8 * 32);
+                cudaError_t e;
+                switch (d.dk) {
+                    case 32: e = launch_pdl(k_gdn_layer<1, 8, GDN_FUSED_DV / 8, true>, grid, block, 0, s, g); break;
+                    case 64: e = launch_pdl(k_gdn_layer<2, 8, GDN_FUSED_DV / 8, true>, grid, block, 0, s, g); break;
+                    default: e = launch_pdl(k_gdn_layer<4, 8, GDN_FUSED_DV / 8, true>, grid, block, 0, s, g); break;
+                }
+                if ((rc = launch_status(e))) return rc;
+            } else {
+                if ((rc = launch_status(launch_gdn_layer(d, B, g, s)))) return rc;
+                GatedNormParams gq{obuf, (int64_t)d.H * d.dv, proj + d.C, Nin, w[HGD_W_GNORM], gn_rows,
+                                   (int64_t)d.H * d.dv, M, d.H, d.dv, eps, NTp};
+                cudaError_t e = launch_pdl(k_gated_norm, dim3((M * d.H + 7) / 8), dim3(256), 0, s, gq);
+                if ((rc = launch_status(e))) return rc;
+            }
             if ((rc = gemm_resid(m->tcw[l][1], gn_rows, (int64_t)d.H * d.dv, d.H * d.dv))) return rc;
             ++ig;
         } else {

@@ -207,6 +207,46 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// One (row, head) of the gated RMSNorm by one warp: o row orow[d], z row
+// zrow[d], gains w[d]; put(i, value) receives bf16(o r w silu(bf16(z))) with
+// r = rsqrt(mean(o^2) + eps).  Shared by k_gated_norm and the GDN layer kernel's
+// fused form, so both give the same bits.
+template <class Put>
+__device__ __forceinline__ void gated_norm_warp(const float* orow, const float* zrow, const bf16_t* w, int d,
+                                                float eps, int lane, Put put) {
+    auto emit = [&](int i, float ov, float zv, float wv, float r) {
+        const float zb = bf2f(f2bf(zv));
+        put(i, f2bf(ov * r * wv * silu_f(zb)));
+    };
+    // heads of up to GR * 32 values are read once, into registers
+    constexpr int GR = 8;
+    if (d <= GR * 32) {
+        float ov[GR], zv[GR], wv[GR];  // o, z and the gains, loaded together
+#pragma unroll
+        for (int u = 0; u < GR; ++u)
+            if (lane + 32 * u < d) {
+                ov[u] = orow[lane + 32 * u];
+                zv[u] = zrow[lane + 32 * u];
+                wv[u] = bf2f(w[lane + 32 * u]);
+            }
+        float ss = 0.f;
+#pragma unroll
+        for (int u = 0; u < GR; ++u)
+            if (lane + 32 * u < d) ss = fmaf(ov[u], ov[u], ss);
+        ss = warp_sum(ss);
+        const float r = rsqrtf(ss / (float)d + eps);
+#pragma unroll
+        for (int u = 0; u < GR; ++u)
+            if (lane + 32 * u < d) emit(lane + 32 * u, ov[u], zv[u], wv[u], r);
+        return;
+    }
+    float ss = 0.f;
+    for (int i = lane; i < d; i += 32) ss = fmaf(orow[i], orow[i], ss);
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)d + eps);
+    for (int i = lane; i < d; i += 32) emit(i, orow[i], zrow[i], bf2f(w[i]), r);
+}
+
 // ------------------------------------------- tensor-core operand layout
 // Token rows as the tensor-core GEMM (gemm_tc.cuh) reads them: per 64-wide k
 // block a tile of NTp rows in 8 x 8 core matrices (8 rows of 16 bytes, 128

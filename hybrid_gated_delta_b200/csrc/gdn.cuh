@@ -372,17 +372,25 @@ struct GdnLayerParams {
     float* log_alpha; float* log_delta; float* log_k;
     int B, T, H, dv;
     int Hk;  // query/key heads (H, the value heads, is a multiple): value head h reads head h / (H / Hk)
+    // the fused gated RMSNorm (k_gdn_layer<.., GN = true>, one CTA per (stream, head)):
+    // z rows, the norm gains and the output rows packed for the tensor-core GEMM
+    const float* z; int64_t z_ld; const bf16_t* gn_w; bf16_t* u; int u_ntp; float eps;
 };
 
 // Rows whose inputs k_gdn_layer stages in shared memory at once.
 constexpr int GDN_TB = 16;
 
-// RPW: state rows per warp (4 or 8; the per-row arithmetic does not depend on it).
-template <int KPL, int RPW>
-__global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_constant__ GdnLayerParams p) {
+// RPW: state rows per warp (4 or 8; the per-row arithmetic does not depend on it);
+// NW warps per CTA.  GN: the CTA holds all dv rows of its head (NW * RPW = dv,
+// one CTA per (stream, head)) and forms the gated RMSNorm of the rows' outputs
+// itself (gated_norm_warp, the arithmetic of k_gated_norm) into p.u, instead of
+// writing o.
+template <int KPL, int RPW, int NW = GDN_WARPS, bool GN = false>
+__global__ void __launch_bounds__(NW * 32) k_gdn_layer(const __grid_constant__ GdnLayerParams p) {
     pdl_launch();
     pdl_wait();
-    constexpr int DK = 32 * KPL, NT = GDN_WARPS * 32, ROWS = GDN_WARPS * RPW;
+    constexpr int DK = 32 * KPL, NT = NW * 32, ROWS = NW * RPW;
+    __shared__ float os[GN ? GDN_TB : 1][GN ? ROWS : 1];  // GN: the block's output rows
     // A block of up to GDN_TB rows at a time: every input of the block (q and k
     // of the key head, this CTA's value rows, a and b) is loaded in one batch,
     // the rows' L2 scales and gates are formed in parallel, and then only the
@@ -443,7 +451,7 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
             al[tid] = expf(-A * softplus_f(abr[0][tid] + dtb));
             be[tid] = sigmoid_f(abr[1][tid]);
         }
-        for (int t = warp; t < n; t += GDN_WARPS) {
+        for (int t = warp; t < n; t += NW) {
             const float a = l2_scale<KPL>(qs[t], lane), c = l2_scale<KPL>(ks[t], lane);
             if (lane == 0) { qsc[t] = a; ksc[t] = c; }
         }
@@ -462,7 +470,8 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
                 float ov = o[0], dv_ = dl[0];
 #pragma unroll
                 for (int r = 1; r < RPW; ++r) if (lane == r) { ov = o[r]; dv_ = dl[r]; }
-                p.o[row * p.o_ld + (int64_t)h * dv + row0 + lane] = ov;
+                if (GN) os[t][warp * RPW + lane] = ov;
+                else p.o[row * p.o_ld + (int64_t)h * dv + row0 + lane] = ov;
                 if (p.log_delta) p.log_delta[(row * H + h) * dv + row0 + lane] = dv_;
             }
             if (p.log_delta && blockIdx.y == 0 && warp == 0) {
@@ -473,6 +482,14 @@ __global__ void __launch_bounds__(GDN_WARPS * 32) k_gdn_layer(const __grid_const
                 float* rp = p.S_rec + ((row * H + h) * dv + row0) * DK + lane * KPL;
 #pragma unroll
                 for (int r = 0; r < RPW; ++r) st_vec<KPL>(rp + (int64_t)r * DK, S[r]);
+            }
+        }
+        if (GN) {
+            __syncthreads();
+            for (int t = warp; t < n; t += NW) {
+                const int64_t row = (int64_t)b * p.T + t0 + t;
+                gated_norm_warp(os[t], p.z + row * p.z_ld + (int64_t)h * dv, p.gn_w, dv, p.eps, lane,
+                                [&](int i, bf16_t v) { p.u[tc_x_elem((int)row, h * dv + i, p.u_ntp)] = v; });
             }
         }
         __syncthreads();  // the next block's inputs overwrite these

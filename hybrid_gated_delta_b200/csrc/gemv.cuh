@@ -598,41 +598,10 @@ __global__ void __launch_bounds__(256) k_gated_norm(const __grid_constant__ Gate
     const int e = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (e >= p.M * p.nh) return;
     const int m = e / p.nh, h = e % p.nh, d = p.d;
-    const float* orow = p.o + m * p.o_ld + h * d;
-    const float* zrow = p.z + m * p.z_ld + h * d;
-    auto put = [&](int i, float ov, float zv, float wv, float r) {
-        const float zb = bf2f(f2bf(zv));
-        const bf16_t v = f2bf(ov * r * wv * silu_f(zb));
+    gated_norm_warp(p.o + m * p.o_ld + h * d, p.z + m * p.z_ld + h * d, p.w, d, p.eps, lane, [&](int i, bf16_t v) {
         if (p.pack_ntp) p.u[tc_x_elem(m, h * d + i, p.pack_ntp)] = v;
         else p.u[m * p.u_ld + h * d + i] = v;
-    };
-    // heads of up to GR * 32 values are read once, into registers
-    constexpr int GR = 8;
-    if (d <= GR * 32) {
-        float ov[GR], zv[GR], wv[GR];  // o, z and the gains, loaded together
-#pragma unroll
-        for (int u = 0; u < GR; ++u)
-            if (lane + 32 * u < d) {
-                ov[u] = orow[lane + 32 * u];
-                zv[u] = zrow[lane + 32 * u];
-                wv[u] = bf2f(p.w[lane + 32 * u]);
-            }
-        float ss = 0.f;
-#pragma unroll
-        for (int u = 0; u < GR; ++u)
-            if (lane + 32 * u < d) ss = fmaf(ov[u], ov[u], ss);
-        ss = warp_sum(ss);
-        const float r = rsqrtf(ss / (float)d + p.eps);
-#pragma unroll
-        for (int u = 0; u < GR; ++u)
-            if (lane + 32 * u < d) put(lane + 32 * u, ov[u], zv[u], wv[u], r);
-        return;
-    }
-    float ss = 0.f;
-    for (int i = lane; i < d; i += 32) ss = fmaf(orow[i], orow[i], ss);
-    ss = warp_sum(ss);
-    const float r = rsqrtf(ss / (float)d + p.eps);
-    for (int i = lane; i < d; i += 32) put(i, orow[i], zrow[i], bf2f(p.w[i]), r);
+    });
 }
 
 // Per-CTA argmax partials: reduce each token over the row lanes of every warp,
