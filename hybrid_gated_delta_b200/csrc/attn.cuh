@@ -147,6 +147,96 @@ __device__ void attn_partial_warp_t(const float* q, const bf16_t* K, const bf16_
     __syncwarp();
 }
 
+// Two query heads of one row over one chunk whose key and value rows sit in
+// shared memory (K, V at the chunk's first key), by one warp: every key and
+// value row is read and unpacked once for both heads.  Per head the arithmetic
+// of attn_partial_warp_t: the same fmaf order per key, and every sum over the
+// lanes with warp_sum's pairings (the scores summed 16 keys at a time by
+// warp_sum_transposed, then moved to lane j), so each partial is bitwise its.
+template <int DPL>
+__device__ void attn_partial_pair(const float* q0, const float* q1, const bf16_t* K, const bf16_t* V, int nk,
+                                  float* dst0, float* dst1, int lane) {
+    constexpr int hd = 32 * DPL, KB = 16;
+    const int d0 = lane * DPL;
+    float qa[DPL], qb[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) { qa[i] = q0[d0 + i]; qb[i] = q1[d0 + i]; }
+    float ta[2], tb[2];  // batch bi: key (lane >> 1) of the batch, summed over the lanes
+#pragma unroll
+    for (int bi = 0; bi < 2; ++bi) {
+        const int b = bi * KB;
+        AttnRow<DPL> kr[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            if (b + j < nk) kr[j] = attn_rowload<DPL>(K + (int64_t)(b + j) * hd + d0);
+            else {
+#pragma unroll
+                for (int i = 0; i < (DPL + 1) / 2; ++i) kr[j].w[i] = 0u;
+            }
+        }
+        float da[KB], db[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            da[j] = 0.f;
+            db[j] = 0.f;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) {
+                const float kv = attn_elem<DPL>(kr[j], i);
+                da[j] = fmaf(qa[i], kv, da[j]);
+                db[j] = fmaf(qb[i], kv, db[j]);
+            }
+        }
+        ta[bi] = warp_sum_transposed<KB>(da, lane);
+        tb[bi] = warp_sum_transposed<KB>(db, lane);
+    }
+    // key L's sum to lane L: batch L >> 4 holds it in lanes 2 (L & 15), 2 (L & 15) + 1
+    const int src = 2 * (lane & 15);
+    const float xa0 = __shfl_sync(0xffffffffu, ta[0], src), xa1 = __shfl_sync(0xffffffffu, ta[1], src);
+    const float xb0 = __shfl_sync(0xffffffffu, tb[0], src), xb1 = __shfl_sync(0xffffffffu, tb[1], src);
+    const float sa = lane < nk ? (lane < KB ? xa0 : xa1) * (1.0f / sqrtf((float)hd)) : -INFINITY;
+    const float sb = lane < nk ? (lane < KB ? xb0 : xb1) * (1.0f / sqrtf((float)hd)) : -INFINITY;
+    float ma = sa, mb = sb;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, o));
+        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    }
+    const float ea = (lane < nk) ? expf(sa - ma) : 0.f, eb = (lane < nk) ? expf(sb - mb) : 0.f;
+    const float la = warp_sum(ea), lb = warp_sum(eb);
+    float acca[DPL], accb[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) { acca[i] = 0.f; accb[i] = 0.f; }
+#pragma unroll
+    for (int b = 0; b < 32; b += KB) {
+        if (b >= nk) break;
+        AttnRow<DPL> vr[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            if (b + j < nk) vr[j] = attn_rowload<DPL>(V + (int64_t)(b + j) * hd + d0);
+            else {
+#pragma unroll
+                for (int i = 0; i < (DPL + 1) / 2; ++i) vr[j].w[i] = 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            const float wa = __shfl_sync(0xffffffffu, ea, b + j), wb = __shfl_sync(0xffffffffu, eb, b + j);
+            if (b + j < nk) {
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) {
+                    const float vv = attn_elem<DPL>(vr[j], i);
+                    acca[i] = fmaf(wa, vv, acca[i]);
+                    accb[i] = fmaf(wb, vv, accb[i]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) { dst0[2 + d0 + i] = acca[i]; dst1[2 + d0 + i] = accb[i]; }
+    if (lane == 0) { dst0[0] = ma; dst0[1] = la; dst1[0] = mb; dst1[1] = lb; }
+    __syncwarp();
+}
+
 // hd = 32 * DPL with DPL one of 1, 2, 4, 8 (the shapes check_supported admits).
 __device__ __forceinline__ void attn_partial_warp(const float* q, const bf16_t* K, const bf16_t* V, int key0,
                                                   int nk, int hd, float* dst, int lane) {
@@ -207,6 +297,23 @@ __global__ void __launch_bounds__(32 * ATTN_PART_WARPS) k_attn_partial(const __g
     }
     __syncthreads();
     const int group = p.nq / p.nkv, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if ((group & 1) == 0) {  // head pairs: the chunk's rows read once for two heads
+        const int hp = group / 2;
+        for (int pi = tlo * hp + warp; pi < thi * hp; pi += ATTN_PART_WARPS) {
+            const int t = pi / hp, h = g * group + 2 * (pi % hp), row = b * p.T + t;
+            const int nk = min(ATTN_CHUNK, pos + t + 1 - key0);
+            const float* q = p.qrot + (int64_t)row * p.nq * hd + (int64_t)h * hd;
+            float* dst = p.part + (((int64_t)row * p.nq + h) * p.max_chunks + ch) * (hd + 2);
+            float* dst1 = dst + (int64_t)p.max_chunks * (hd + 2);  // head h + 1
+            switch (hd) {
+                case 256: attn_partial_pair<8>(q, q + hd, Ks, Vs, nk, dst, dst1, lane); break;
+                case 128: attn_partial_pair<4>(q, q + hd, Ks, Vs, nk, dst, dst1, lane); break;
+                case 64: attn_partial_pair<2>(q, q + hd, Ks, Vs, nk, dst, dst1, lane); break;
+                default: attn_partial_pair<1>(q, q + hd, Ks, Vs, nk, dst, dst1, lane); break;
+            }
+        }
+        return;
+    }
     for (int pi = tlo * group + warp; pi < thi * group; pi += ATTN_PART_WARPS) {
         const int t = pi / group, h = g * group + pi % group, row = b * p.T + t;
         const int nk = min(ATTN_CHUNK, pos + t + 1 - key0);
