@@ -1317,6 +1317,7 @@ int hgd_check_not_coresident(const hgd_model* m, const hgd_state* st, int T) {
 
 // dv of the GDN layer kernel's fused gated-norm form (16 warps x 8 rows: a head per CTA).
 constexpr int GDN_FUSED_DV = 128;
+static_assert(GDN_CONV_K == GV_CONV_K, "one conv width");
 
 // The GDN layer kernel over B streams: 8 state rows per warp where dv allows
 // (32 rows per CTA), else 4; either way each row's arithmetic is the same.
@@ -1760,13 +1761,18 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
         if ((rc = norm_rows(w[HGD_W_IN_NORM], l == 0))) return rc;
         if ((rc = gemm(m->tcw[l][0], xn_rows, d.D, proj, Nin, d.D))) return rc;
         if (!att) {
-            TcConvParams cp{proj, Nin, conv + ig * c_layer, w[HGD_W_CONV],
-                            tail_rec ? tail_rec + ig * trec_layer : nullptr, B, T, (int)d.C};
-            const int64_t n = (int64_t)B * d.C;
-            const dim3 cg((unsigned)((n + 255) / 256)), cb(256);
-            if ((rc = launch_status(tail_rec ? launch_pdl(k_tc_conv<true>, cg, cb, 0, s, cp)
-                                             : launch_pdl(k_tc_conv<false>, cg, cb, 0, s, cp))))
-                return rc;
+            // the conv runs inside the GDN kernel where one CTA holds a head's q, k and
+            // v channels alone (dk = dv = 128, a key head per value head)
+            const bool fused_conv = d.dv == GDN_FUSED_DV && d.dk == 128 && d.Hk == d.H;
+            if (!fused_conv) {
+                TcConvParams cp{proj, Nin, conv + ig * c_layer, w[HGD_W_CONV],
+                                tail_rec ? tail_rec + ig * trec_layer : nullptr, B, T, (int)d.C};
+                const int64_t n = (int64_t)B * d.C;
+                const dim3 cg((unsigned)((n + 255) / 256)), cb(256);
+                if ((rc = launch_status(tail_rec ? launch_pdl(k_tc_conv<true>, cg, cb, 0, s, cp)
+                                                 : launch_pdl(k_tc_conv<false>, cg, cb, 0, s, cp))))
+                    return rc;
+            }
             GdnLayerParams g{};
             g.proj = proj; g.proj_ld = Nin;
             g.A_log = w[HGD_W_A_LOG]; g.dt_bias = w[HGD_W_DT_BIAS];
@@ -1779,7 +1785,11 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
                 g.z = proj + d.C; g.z_ld = Nin; g.gn_w = w[HGD_W_GNORM]; g.u = gn_rows; g.u_ntp = NTp; g.eps = eps;
                 const dim3 grid(B * d.H), block(GDN_FUSED_DV / 8 * 32);
                 cudaError_t e;
-                switch (d.dk) {
+                if (fused_conv) {
+                    g.conv_tail = conv + ig * c_layer; g.conv_w = w[HGD_W_CONV];
+                    g.conv_tail_rec = tail_rec ? tail_rec + ig * trec_layer : nullptr; g.C = (int)d.C;
+                    e = launch_pdl(k_gdn_layer<4, 8, GDN_FUSED_DV / 8, true, true>, grid, block, 0, s, g);
+                } else switch (d.dk) {
                     case 32: e = launch_pdl(k_gdn_layer<1, 8, GDN_FUSED_DV / 8, true>, grid, block, 0, s, g); break;
                     case 64: e = launch_pdl(k_gdn_layer<2, 8, GDN_FUSED_DV / 8, true>, grid, block, 0, s, g); break;
                     default: e = launch_pdl(k_gdn_layer<4, 8, GDN_FUSED_DV / 8, true>, grid, block, 0, s, g); break;

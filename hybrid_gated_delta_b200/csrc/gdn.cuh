@@ -375,7 +375,12 @@ struct GdnLayerParams {
     // the fused gated RMSNorm (k_gdn_layer<.., GN = true>, one CTA per (stream, head)):
     // z rows, the norm gains and the output rows packed for the tensor-core GEMM
     const float* z; int64_t z_ld; const bf16_t* gn_w; bf16_t* u; int u_ntp; float eps;
+    // the fused causal conv (CONV = true, with GN and H = Hk): this layer's tails
+    // [B][kc-1][C], the conv weights [C][kc], tail records [B][T][kc-1][C] or null,
+    // and the conv channel count C; proj then holds the raw in-projection rows
+    float* conv_tail; const bf16_t* conv_w; float* conv_tail_rec; int C;
 };
+constexpr int GDN_CONV_K = 4;  // the causal conv's width
 
 // Rows whose inputs k_gdn_layer stages in shared memory at once.
 constexpr int GDN_TB = 16;
@@ -385,7 +390,10 @@ constexpr int GDN_TB = 16;
 // one CTA per (stream, head)) and forms the gated RMSNorm of the rows' outputs
 // itself (gated_norm_warp, the arithmetic of k_gated_norm) into p.u, instead of
 // writing o.
-template <int KPL, int RPW, int NW = GDN_WARPS, bool GN = false>
+// CONV (with GN, H = Hk): the CTA also runs the causal conv of its head's q, k and
+// v channels (one thread per channel, rows in order, the arithmetic of k_tc_conv)
+// on the staged raw rows, so no separate conv pass runs.
+template <int KPL, int RPW, int NW = GDN_WARPS, bool GN = false, bool CONV = false>
 __global__ void __launch_bounds__(NW * 32) k_gdn_layer(const __grid_constant__ GdnLayerParams p) {
     pdl_launch();
     pdl_wait();
@@ -406,6 +414,21 @@ __global__ void __launch_bounds__(NW * 32) k_gdn_layer(const __grid_constant__ G
     const int Hk = p.Hk, hk = h / (H / Hk);
     const int64_t C = 2 * (int64_t)Hk * DK + (int64_t)H * dv;
     const float A = expf(bf2f(p.A_log[h])), dtb = bf2f(p.dt_bias[h]);
+
+    // CONV: this thread's channel (q, k, then v channels of the head), its weights
+    // and tail, in registers for the whole call
+    constexpr int NT3 = GDN_CONV_K - 1;
+    static_assert(!CONV || (GN && 2 * DK + ROWS <= NT), "one thread per conv channel");
+    int cch = -1;
+    float cw[GDN_CONV_K], ctl[NT3];
+    if (CONV && tid < 2 * DK + ROWS) {
+        cch = tid < DK ? hk * DK + tid
+                       : tid < 2 * DK ? Hk * DK + hk * DK + (tid - DK) : 2 * Hk * DK + h * dv + (tid - 2 * DK);
+#pragma unroll
+        for (int j = 0; j < GDN_CONV_K; ++j) cw[j] = bf2f(p.conv_w[(int64_t)cch * GDN_CONV_K + j]);
+#pragma unroll
+        for (int j = 0; j < NT3; ++j) ctl[j] = p.conv_tail[((int64_t)b * NT3 + j) * p.C + cch];
+    }
 
     float S[RPW][KPL];
     float* Sbase = p.S + ((int64_t)(b * H + h) * dv + row0) * DK + lane * KPL;
@@ -447,6 +470,29 @@ __global__ void __launch_bounds__(NW * 32) k_gdn_layer(const __grid_constant__ G
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
+        if (CONV) {
+            if (cch >= 0) {
+                float* col = tid < DK ? &qs[0][tid] : tid < 2 * DK ? &ks[0][tid - DK] : &vs[0][tid - 2 * DK];
+                const int stride = tid < 2 * DK ? DK : ROWS;
+                for (int t = 0; t < n; ++t) {
+                    const float xv = col[t * stride];
+                    float acc = 0.f;
+#pragma unroll
+                    for (int j = 0; j < NT3; ++j) acc = fmaf(cw[j], ctl[j], acc);
+                    acc = fmaf(cw[NT3], xv, acc);
+                    col[t * stride] = silu_f(acc);
+#pragma unroll
+                    for (int j = 0; j + 1 < NT3; ++j) ctl[j] = ctl[j + 1];
+                    ctl[NT3 - 1] = xv;
+                    if (p.conv_tail_rec) {
+                        float* rp = p.conv_tail_rec + ((int64_t)b * p.T + t0 + t) * NT3 * p.C + cch;
+#pragma unroll
+                        for (int j = 0; j < NT3; ++j) rp[(int64_t)j * p.C] = ctl[j];
+                    }
+                }
+            }
+            __syncthreads();
+        }
         if (tid < n) {
             al[tid] = expf(-A * softplus_f(abr[0][tid] + dtb));
             be[tid] = sigmoid_f(abr[1][tid]);
@@ -497,6 +543,9 @@ __global__ void __launch_bounds__(NW * 32) k_gdn_layer(const __grid_constant__ G
     if (p.log_delta) return;  // a verify window: the state stays as it was
 #pragma unroll
     for (int r = 0; r < RPW; ++r) st_vec<KPL>(Sbase + (int64_t)r * DK, S[r]);
+    if (CONV && cch >= 0)
+#pragma unroll
+        for (int j = 0; j < NT3; ++j) p.conv_tail[((int64_t)b * NT3 + j) * p.C + cch] = ctl[j];
 }
 
 }  // namespace hgd
