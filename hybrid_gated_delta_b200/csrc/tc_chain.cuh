@@ -12,6 +12,7 @@
 // results agree to fp32 rounding, not bit for bit.)
 #pragma once
 
+#include "attn.cuh"
 #include "gemv.cuh"
 
 namespace hgd {
@@ -94,6 +95,10 @@ __global__ void k_tc_rope(const __grid_constant__ TcRopeParams p) {
         if (threadIdx.x == 0) set_status(p.status, HGD_ERR_INVALID_ARG);
         return;
     }
+    // the row's angles, one per rotated pair, shared by every head (rope_sincos at P)
+    __shared__ float rsn[ATTN_MAX_HD / 2], rcs[ATTN_MAX_HD / 2];
+    for (int i = threadIdx.x; i < half; i += blockDim.x) rope_sincos(P, i, p.inv1, &rsn[i], &rcs[i]);
+    __syncthreads();
     const int nqp = p.nq * half, nkp = p.nkv * half;
     for (int e = threadIdx.x; e < nqp + nkp + p.nkv * hd; e += blockDim.x) {
         if (e < nqp + nkp) {
@@ -101,8 +106,7 @@ __global__ void k_tc_rope(const __grid_constant__ TcRopeParams p) {
             const int ee = isk ? e - nqp : e, head = ee / half, i = ee % half;
             const float* src = yr + (isk ? 2 * (int64_t)p.nq * hd : 0) + (int64_t)head * hd;
             const float a = src[i], bb = src[i + half];
-            float sn, cs;
-            rope_sincos(P, i, p.inv1, &sn, &cs);
+            const float sn = rsn[i], cs = rcs[i];
             const float x0 = a * cs - bb * sn, x1 = bb * cs + a * sn;
             if (!isk) {
                 float* qo = p.qrot + (int64_t)m * p.nq * hd + (int64_t)head * hd;
@@ -139,8 +143,29 @@ __global__ void __launch_bounds__(256) k_tc_argmax_part(const float* logits, int
     float bv = -INFINITY;
     int bi = 0x7fffffff;
     bool nan = false;
+    auto take = [&](float v, int i) {
+        if (v != v) nan = true;
+        else if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+    };
+    int lo4 = lo;  // the 16-byte aligned part of the slice runs as float4 loads
+    if ((ld & 3) == 0 && (lo & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0) {
+        const int n4 = (hi - lo) / 4;
+        const float4* l4 = reinterpret_cast<const float4*>(lr + lo);
+        for (int q0 = (int)threadIdx.x; q0 < n4; q0 += 2 * 256) {
+            float4 v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) v[u] = q0 + u * 256 < n4 ? l4[q0 + u * 256] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (q0 + u * 256 < n4) {
+                    const int i = lo + 4 * (q0 + u * 256);
+                    take(v[u].x, i); take(v[u].y, i + 1); take(v[u].z, i + 2); take(v[u].w, i + 3);
+                }
+        }
+        lo4 = lo + 4 * n4;
+    }
     constexpr int U = 4;
-    for (int i0 = lo + (int)threadIdx.x; i0 < hi; i0 += U * 256) {
+    for (int i0 = lo4 + (int)threadIdx.x; i0 < hi; i0 += U * 256) {
         float v[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) v[u] = i0 + u * 256 < hi ? lr[i0 + u * 256] : -INFINITY;
