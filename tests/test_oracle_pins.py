@@ -416,9 +416,11 @@ def test_gdn_packed_rows_match_separate(orc):
 # --------------------------------------------------------------- norms -----
 
 # --------------------------------------------------------- GDN gates -----
-# North_star: alpha_t = exp(g_t).  The stack's log-decay is
-# g = -exp(A_log) * softplus(a + dt_bias) with the stable softplus
-# max(x,0) + log1p(exp(-|x|)) ("nvfp4-megamoe-kernel commit log", activation_topk).
+# The gated delta rule decays the state by alpha_t = exp(g_t).  The stack's
+# log-decay is g = -exp(A_log) * softplus(a + dt_bias) (A_log per head, stored as
+# bf16: "qwen3_5 cuda: mixed-width MLX checkpoints ... #849", the commit on widths
+# read from config.json) with the stable softplus max(x,0) + log1p(exp(-|x|))
+# ("nvfp4-megamoe-kernel commit log", activation_topk).
 # The references below are evaluated with mpmath at 50 digits from the closed
 # form log(1 + e^x), not from the oracle's formula.
 
