@@ -625,7 +625,7 @@ int sk_launch(const Dims& d, const SkParams& prm, size_t smem, int sms, cudaStre
 // weight tiles, a split of the K blocks that brings the CTA count near one wave
 // (it depends on N and K only), as many shared-memory stages as fit.
 struct TcPlan {
-    int NTp, n_blocks, kb_per_split, splits, stages, wpb;
+    int NTp, n_blocks, kb_per_split, splits, stages, wpb, npair, ctas;
     uint32_t tmem_cols;
     size_t xp_bytes;
 };
@@ -645,7 +645,12 @@ TcPlan tc_plan(int M, int N, int K, bool swiglu = false) {
     // tile, so more of the bytes in flight are weights and the token rows are
     // re-read half as often (two CTAs of 2 x NTp TMEM columns fit an SM's 512)
     q.wpb = (q.splits == 1 && !swiglu && q.n_blocks >= 2 * TC_TARGET_CTAS && q.NTp <= 128) ? 2 : 1;
-    const int ctas = (q.n_blocks + q.wpb - 1) / q.wpb * q.splits;
+    // block pairs fill whole waves of two CTAs per SM; the remaining blocks run one
+    // per CTA, so the last wave is made of half-length CTAs
+    q.npair = q.wpb == 2 ? (q.n_blocks / 2) / (2 * TC_TARGET_CTAS) * (2 * TC_TARGET_CTAS) : 0;
+    if (q.wpb == 2 && q.npair == 0) q.wpb = 1;
+    q.ctas = q.wpb == 2 ? q.npair + (q.n_blocks - 2 * q.npair) : q.n_blocks * q.splits;
+    const int ctas = q.ctas;
     // more than one wave of CTAs: stages for two CTAs per SM, so one's epilogue
     // overlaps the other's stream; otherwise every stage that fits
     const int per_sm = ctas > TC_TARGET_CTAS ? 2 : 1;
@@ -722,8 +727,9 @@ int tc_run(const bf16_t* Wp, const bf16_t* x, int64_t x_ld, float* y, int M, int
     prm.M = M; prm.N = N; prm.K = K; prm.NTp = q.NTp; prm.ldo = N;
     prm.n_blocks = q.n_blocks; prm.kb_per_split = q.kb_per_split; prm.splits = q.splits; prm.stages = q.stages;
     prm.wpb = q.wpb;
+    prm.npair = q.npair;
     prm.tmem_cols = q.tmem_cols;
-    const dim3 grid((q.n_blocks + q.wpb - 1) / q.wpb * q.splits), block(TC_THREADS);
+    const dim3 grid(q.ctas), block(TC_THREADS);
     const size_t smem = tc_smem_bytes(q.NTp, q.stages, q.wpb);
     e = q.splits > 1 ? launch_pdl_cluster(k_gemm_tc, grid, block, smem, s, q.splits, prm)
                      : launch_pdl(k_gemm_tc, grid, block, smem, s, prm);

@@ -140,6 +140,7 @@ struct TcParams {
     int M, N, K, NTp, ldo;
     int n_blocks, kb_per_split, splits, stages;  // splits: the cluster size (1: no cluster)
     int wpb;            // 128-row weight blocks per CTA (2: two accumulators share each token tile; splits 1)
+    int npair;          // wpb 2: CTAs [0, npair) own block pairs, the later CTAs one block each
     uint32_t tmem_cols;
 };
 
@@ -261,9 +262,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     volatile int* abort_flag = reinterpret_cast<volatile int*>(done + 1) + 1;
     uint64_t* rbar = done + 3;  // the split epilogue: the other splits' partials have landed
     // the splits of a row block are consecutive CTAs, one cluster: sp is the rank;
-    // with wpb = 2 a CTA owns blocks nb and nb + 1 (only nb if that is the last)
-    const int nb = (blockIdx.x / p.splits) * p.wpb, sp = blockIdx.x % p.splits;
-    const int wn = min(p.wpb, p.n_blocks - nb);  // weight blocks this CTA computes
+    // with wpb = 2 the first npair CTAs own blocks nb and nb + 1 and the rest one
+    // block each, so the last wave of CTAs is made of short ones
+    const int cta = blockIdx.x / p.splits, sp = blockIdx.x % p.splits;
+    const int nb = p.wpb == 2 ? (cta < p.npair ? 2 * cta : 2 * p.npair + (cta - p.npair)) : cta;
+    const int wn = p.wpb == 2 ? min(cta < p.npair ? 2 : 1, p.n_blocks - nb) : 1;  // weight blocks of this CTA
     const int nkb_all = p.K / TC_BK;
     const int kb0 = sp * p.kb_per_split, nkb = max(0, min(nkb_all, kb0 + p.kb_per_split) - kb0);
 
