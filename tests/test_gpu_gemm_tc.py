@@ -110,6 +110,28 @@ def test_gemm_tc_window_shapes(hgd, orc, name):
     assert np.all(err <= 2 * bound + 1e-30), (name, err.max(), (err / (bound + 1e-30)).max())
 
 
+@pytest.mark.parametrize("name", ["lm_head", "down", "gdn_in"])
+def test_gemm_tc_rows_independent_of_m(hgd, name):
+    """Each token row's result does not depend on how many rows the call carries
+    (the property a window equal to its one-row steps rests on): the first M rows
+    of a 200-row call, bit for bit, at M = 1 .. 128.  At 200 rows the LM-head
+    shape runs one weight block per CTA, at 128 rows or fewer two blocks per CTA
+    for its first waves and one for the rest: the same bits either way.  The split
+    shapes (down: 8 splits in a cluster, gdn_in: 2) keep their split at every M."""
+    import torch
+    N, K = WINDOW[name]
+    c = syn.gemv_case(N, K, 200, seed=17)
+    W, x = dev_bf16(c["W"]), dev_bf16(c["x"])
+    y_all, guard_ok, Wp, status = _run(hgd, W, x, N)
+    assert guard_ok
+    for M in (1, 8, 16, 100, 128):
+        y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        hgd.gemm_tc_bf16(Wp, x[:M].contiguous(), N, y=y, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(y, y_all[:M]), (name, M)
+
+
 def test_stuck_wait_reports_timeout_and_context_survives(hgd, orc):
     """A bounded in-kernel wait that nothing completes ends after its limit with
     HGD_ERR_TIMEOUT in the status word; the next calls still compute correctly."""
