@@ -127,3 +127,47 @@ def test_tc_chain_config5_window_equals_steps_and_oracle(hgd):
     gs = host(srw[:, 0:1])
     compare_state_rel(gs[0], sr64[0], "tensor-core chain, GDN layer 0 records")
     assert rel_l2(gs, sr64) <= 1.5 * rel_l2(sr32, sr64) + BF16_REL_L2
+
+
+# value heads over fewer key heads and an untied head ("qwen3_5 cuda ... #849",
+# the commit on widths read from config.json): the reduced geometry, and hidden
+# 1024 with 16 value heads over 8 key heads of 128 (the head-per-CTA GDN kernel
+# with the gated norm fused and the conv separate), both through the tensor cores
+GROUPED_SMALL = dict(syn.SMALL_CFG, gdn_heads=2, gdn_v_heads=4, untied_head=1)
+GROUPED_WIDE = dict(syn.STACK_CFG, n_layers=4, vocab=8192, gdn_heads=8, gdn_v_heads=16, untied_head=1)
+
+
+@pytest.mark.parametrize("which", ["small", "wide"])
+def test_tc_chain_grouped_untied(hgd, orc, orc32, which):
+    """A window equals its one-row steps bit for bit; the window's logits follow the
+    oracle within its own fp32 deviation (the end-to-end reading: at most 1.5x the
+    fp32 oracle's deviation from fp64, over the window; a single row within 3x, since
+    a bf16 rounding flip upstream in one evaluation and not the other moves one row
+    by about that much), and in the reduced geometry within the bf16 tolerance.  The
+    mma.sync chain on the same inputs agrees to the same fp32 noise (a wrong head or
+    row mapping would not)."""
+    import torch
+    cfg = GROUPED_SMALL if which == "small" else GROUPED_WIDE
+    w = syn.stack_weights(cfg, seed=92)
+    model = hgd.Model(cfg, w, tc=True)
+    B, T, Lmax, pre = (2, 5, 40, 16) if which == "small" else (4, 8, 640, 512)
+    init, toks, amw, lw, srw, trw, sw = _window_vs_steps(hgd, model, cfg, B, T, Lmax, pre, 93)
+    V = cfg["vocab"]
+    refs = {}
+    for o in (orc, orc32):
+        ost = oracle_state(o, init)
+        r = o.decode_stack(o.make_model(cfg, w), ost, toks, logits=True)
+        refs[o.real] = r["logits"].reshape(B * T, V).astype(np.float64)
+    l64, l32 = refs[np.float64], refs[np.float32]
+    g = host(lw)
+    assert rel_l2(g, l64) <= 1.5 * rel_l2(l32, l64) + 1e-3, which
+    for row in range(B * T):
+        assert rel_l2(g[row], l64[row]) <= 3 * rel_l2(l32[row], l64[row]) + 2e-3, f"{which}: row {row} logits"
+    model_m = hgd.Model(cfg, w)
+    sm = hgd.State(model_m, B, T, Lmax, init)
+    lg_m = torch.empty((B * T, V), device="cuda")
+    hgd.decode_layer_stack(model_m, sm, torch.from_numpy(toks).cuda(), T, logits=lg_m)
+    torch.cuda.synchronize()
+    assert rel_l2(g, host(lg_m)) <= 2 * rel_l2(l32, l64) + 1e-3, f"{which}: tensor-core vs mma.sync chain"
+    if which == "small":
+        compare_logits(g, l64, "tensor-core chain, grouped small")
