@@ -818,6 +818,24 @@ int sk_run(const hgd_model* m, const hgd_state* st, const Dims& d, const int32_t
     return sk_launch(d, prm, smem, di.sms, s, true);
 }
 
+// The tensor-core chain's attention partials (k_attn_partial_tc), by head dim
+// (one of 32, 64, 128, 256: check_supported admits no other).
+template <int HD>
+cudaError_t launch_attn_partial_tc_t(dim3 grid, cudaStream_t s, const AttnParams& a) {
+    static CtxCache<int> attr_done;
+    const cudaError_t e = ensure_smem_attr(k_attn_partial_tc<HD>, attr_done);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_attn_partial_tc<HD>, grid, dim3(256), attn_tc_smem_bytes(HD), s, a);
+}
+cudaError_t launch_attn_partial_tc(int hd, dim3 grid, cudaStream_t s, const AttnParams& a) {
+    switch (hd) {
+        case 256: return launch_attn_partial_tc_t<256>(grid, s, a);
+        case 128: return launch_attn_partial_tc_t<128>(grid, s, a);
+        case 64: return launch_attn_partial_tc_t<64>(grid, s, a);
+        default: return launch_attn_partial_tc_t<32>(grid, s, a);
+    }
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -1821,10 +1839,8 @@ int hgd_decode_layer_stack_tc(const hgd_model* m, const hgd_state* st, const int
             a.B = B; a.T = T; a.nq = d.nq; a.nkv = d.nkv; a.hd = d.hd; a.Lmax = Lmax;
             a.max_chunks = max_chunks_of(Lmax);
             a.pack_ntp = NTp;
-            cudaError_t e = launch_pdl(k_attn_partial, dim3(B, d.nkv, a.max_chunks), dim3(32 * ATTN_PART_WARPS),
-                                       attn_part_smem_bytes(d.hd), s, a);
-            if ((rc = launch_status(e))) return rc;
-            e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
+            if ((rc = launch_status(launch_attn_partial_tc(d.hd, dim3(B, d.nkv, a.max_chunks), s, a)))) return rc;
+            cudaError_t e = launch_pdl(k_attn_merge, dim3(M, d.nq), dim3(d.hd), 0, s, a);
             if ((rc = launch_status(e))) return rc;
             if ((rc = gemm_resid(m->tcw[l][1], attn, (int64_t)d.nq * d.hd, d.nq * d.hd))) return rc;
             ++ia;

@@ -171,3 +171,27 @@ def test_tc_chain_grouped_untied(hgd, orc, orc32, which):
     assert rel_l2(g, host(lg_m)) <= 2 * rel_l2(l32, l64) + 1e-3, f"{which}: tensor-core vs mma.sync chain"
     if which == "small":
         compare_logits(g, l64, "tensor-core chain, grouped small")
+
+
+# attention geometries of the tensor-core partials: head dims 128 and 32, eight
+# query heads over one kv head with 12-row windows (96 query vectors of a stream
+# per chunk: two passes of the 64-vector tiles), and a window that starts 7 keys
+# before a chunk boundary (its first rows see only the chunk before it)
+ATTN_GEOMS = {
+    "hd128_group8": (dict(syn.SMALL_CFG, attn_q_heads=8, attn_kv_heads=1, attn_head_dim=128), 2, 12, 64, 25),
+    "hd32": (dict(syn.SMALL_CFG, attn_head_dim=32), 3, 5, 48, 30),
+}
+
+
+@pytest.mark.parametrize("which", list(ATTN_GEOMS))
+def test_tc_chain_attention_geometries(hgd, orc, which):
+    """A window equals its one-row steps bit for bit and follows the oracle within
+    the bf16 tolerance, at attention geometries the stack's own shape does not reach."""
+    cfg, B, T, Lmax, pre = ATTN_GEOMS[which]
+    w = syn.stack_weights(cfg, seed=94)
+    model = hgd.Model(cfg, w, tc=True)
+    init, toks, amw, lw, srw, trw, sw = _window_vs_steps(hgd, model, cfg, B, T, Lmax, pre, 95)
+    V = cfg["vocab"]
+    r = orc.decode_stack(orc.make_model(cfg, w), oracle_state(orc, init), toks, logits=True)
+    compare_logits(host(lw), r["logits"].reshape(B * T, V), f"tensor-core chain, {which}")
+    compare_argmax(host(amw), r["logits"].reshape(B * T, V), f"tensor-core chain, {which}")
