@@ -270,12 +270,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     const int nkb_all = p.K / TC_BK;
     const int kb0 = sp * p.kb_per_split, nkb = max(0, min(nkb_all, kb0 + p.kb_per_split) - kb0);
 
+    const uint32_t xbytes = (uint32_t)p.NTp * TC_BK * 2, wbytes = (uint32_t)TC_WTILE * 2;
+    const int pre = min(S, nkb);
     if (tid == 0) {
         for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
         mbar_init(done, 1);
         mbar_init(rbar, 1);
         *abort_flag = 0;
         mbar_fence_init();
+        // the first stages' weight tiles go out at once, by the thread that set up
+        // their barriers, before the TMEM allocation and the CTA barrier (weights
+        // are never written by the previous kernel on the stream); their token
+        // tiles follow the wait for that kernel
+        const uint64_t pol_w = policy_evict_first();
+        for (int i = 0; i < pre; ++i) {
+            mbar_arrive_expect_tx(&full[i], (uint32_t)wn * wbytes + xbytes);
+            for (int j = 0; j < wn; ++j)
+                bulk_g2s(smem + (size_t)i * sb + j * wbytes, p.Wp + ((size_t)(nb + j) * nkb_all + kb0 + i) * TC_WTILE,
+                         wbytes, &full[i], pol_w);
+        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -291,19 +304,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_gemm_tc(const __grid_constant
     pdl_launch();
 
     if (warp == 0 && lane == 0) {
-        // producer: the first stages' weight tiles go out before the wait for the
-        // previous kernel on the stream (weights are never written by it), their
-        // token tiles after it; then stage by stage as the MMAs free them
-        const uint32_t xbytes = (uint32_t)p.NTp * TC_BK * 2, wbytes = (uint32_t)TC_WTILE * 2;
+        // producer (the same thread): the first stages' token tiles after the wait
+        // for the previous kernel; then stage by stage as the MMAs free them
         const uint32_t xoff = (uint32_t)p.wpb * wbytes;  // the token tile follows the weight tiles
         const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
-        const int pre = min(S, nkb);
-        for (int i = 0; i < pre; ++i) {
-            mbar_arrive_expect_tx(&full[i], (uint32_t)wn * wbytes + xbytes);
-            for (int j = 0; j < wn; ++j)
-                bulk_g2s(smem + (size_t)i * sb + j * wbytes, p.Wp + ((size_t)(nb + j) * nkb_all + kb0 + i) * TC_WTILE,
-                         wbytes, &full[i], pol_w);
-        }
         pdl_wait();
         for (int i = 0; i < pre; ++i)
             bulk_g2s(smem + (size_t)i * sb + xoff, p.Xp + (size_t)(kb0 + i) * p.NTp * TC_BK, xbytes, &full[i],
