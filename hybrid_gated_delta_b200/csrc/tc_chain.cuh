@@ -138,9 +138,9 @@ __global__ void k_tc_rope(const __grid_constant__ TcRopeParams p) {
 //   S = Q K^T (vectors x the chunk's keys, over the head's dims: two partial
 //             products over its two halves, summed first half first),
 //   O = P V   (vectors x dims, over the chunk's keys).
-// An fp32 operand enters as two bf16 terms (x = hi + lo, hi = bf16(x), lo =
-// bf16(x - hi), exact: about 16 significant bits of x) against the bf16 cache
-// rows, summed in fp32.  Per vector: s_j = S_j / sqrt(hd), m = max over the keys
+// An fp32 operand enters as two bf16 terms, hi = bf16(x) and lo = bf16(x - hi)
+// (the difference exact in fp32; hi + lo carries about 16 significant bits of x),
+// against the bf16 cache rows, summed in fp32.  Per vector: s_j = S_j / sqrt(hd), m = max over the keys
 // it sees, p_j = exp(s_j - m) for those and 0 for the rest, l = sum_j p_j
 // (warp_sum), acc = O: the partial row (m, l, acc) k_attn_merge reads.
 // A tensor-core output element depends on its own row and column only, the keys
